@@ -1,0 +1,181 @@
+"""Plain fp64 CPU oracle for StiefAttention latent-KV decode (test infrastructure).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline / reference arm
+of ``bench.py`` may import this package.  The product path (the CUDA library and
+its Python binding) never imports it and has no CPU fallback.
+
+The arithmetic lives in ``stief_oracle.c`` (plain C, IEEE double, sequential sums
+in the order of the definition).  This module only converts numpy arrays to
+contiguous float64 / int32 buffers and calls it through ctypes.  The C source is
+compiled with gcc on first use if the shared object is missing or stale; no
+flags that reorder floating point (no -ffast-math) are used.
+
+Definitions followed (StiefAttention technical summary, "Mecanismo Central" /
+"Kernmechanismus", items 2 and 5): stored latent ``K_down = K . P_K`` and
+``V_down = V . P_V``; on-the-fly reconstruction ``K~ = K_down . P_K^T`` and
+``V~ = V_down . P_V^T`` before softmax attention.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "stief_oracle.c")
+_LIB = os.path.join(_HERE, "libstief_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+_D = ctypes.POINTER(ctypes.c_double)
+_I32 = ctypes.POINTER(ctypes.c_int32)
+
+
+def build(src: str = _SRC, out: str = _LIB, force: bool = False) -> str:
+    """Compile the oracle C source into a shared object (gcc -O2, OpenMP, no fast-math)."""
+    stale = (not os.path.exists(out)) or os.path.getmtime(out) < os.path.getmtime(src)
+    if force or stale:
+        tmp = out + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
+               "-fno-fast-math", "-ffp-contract=off", src, "-o", tmp, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, out)
+    return out
+
+
+def _f64(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a: np.ndarray, typ=_D):
+    return a.ctypes.data_as(typ)
+
+
+class Oracle:
+    """ctypes view of one compiled oracle shared object."""
+
+    def __init__(self, path: str):
+        lib = ctypes.CDLL(path)
+        lib.stief_oracle_round_bf16.restype = ctypes.c_double
+        lib.stief_oracle_round_bf16.argtypes = [ctypes.c_double]
+        lib.stief_oracle_round_bf16_array.restype = None
+        lib.stief_oracle_round_bf16_array.argtypes = [_D, _D, ctypes.c_long]
+        lib.stief_oracle_project.restype = None
+        lib.stief_oracle_project.argtypes = [_D, _D, _D, ctypes.c_long, ctypes.c_int,
+                                             ctypes.c_int, ctypes.c_int]
+        lib.stief_oracle_compress_append.restype = ctypes.c_int
+        lib.stief_oracle_compress_append.argtypes = (
+            [_D, _D, _D, _D, _D, _D, _I32] + [ctypes.c_int] * 8)
+        lib.stief_oracle_decode.restype = ctypes.c_int
+        lib.stief_oracle_decode.argtypes = (
+            [_D, _D, _D, _D, _D, _I32, _D] + [ctypes.c_int] * 8)
+        lib.stief_oracle_max_threads.restype = ctypes.c_int
+        lib.stief_oracle_max_threads.argtypes = []
+        self.lib = lib
+        self.path = path
+
+    def max_threads(self) -> int:
+        """OpenMP threads a decode call uses by default."""
+        return int(self.lib.stief_oracle_max_threads())
+
+    def round_bf16(self, x) -> np.ndarray:
+        """Round every element to the nearest bfloat16 value, ties to even (fp64 result)."""
+        x = _f64(x)
+        y = np.empty_like(x)
+        self.lib.stief_oracle_round_bf16_array(_ptr(x), _ptr(y), x.size)
+        return y
+
+    def project(self, x, P, round_to_bf16: bool = True) -> np.ndarray:
+        """Compressed storage of rows: y = x . P (x [T][d], P [d][r]), optionally bf16-rounded."""
+        x = _f64(x)
+        P = _f64(P)
+        T, d = x.shape
+        d2, r = P.shape
+        if d2 != d:
+            raise ValueError("project: inner dimensions differ")
+        y = np.empty((T, r), dtype=np.float64)
+        self.lib.stief_oracle_project(_ptr(x), _ptr(P), _ptr(y), T, d, r, int(round_to_bf16))
+        return y
+
+    def compress_append(self, k_new, v_new, P_K, P_V, k_lat, v_lat, seq_lens,
+                        round_to_bf16: bool = True):
+        """Append T projected rows per (sequence, KV head).
+
+        Shapes: k_new/v_new [B][Hkv][T][d], P_K [Hkv][d][rK], P_V [Hkv][d][rV],
+        k_lat [B][Hkv][L_max][rK], v_lat [B][Hkv][L_max][rV], seq_lens [B].
+        The inputs are not modified; returns (k_lat, v_lat, seq_lens, n_overflow)
+        as updated copies.
+        """
+        k_new, v_new, P_K, P_V = map(_f64, (k_new, v_new, P_K, P_V))
+        k_lat = _f64(k_lat).copy()
+        v_lat = _f64(v_lat).copy()
+        lens = np.ascontiguousarray(np.asarray(seq_lens, dtype=np.int32)).copy()
+        B, Hkv, T, d = k_new.shape
+        rK = P_K.shape[2]
+        rV = P_V.shape[2]
+        L_max = k_lat.shape[2]
+        if v_new.shape != k_new.shape or P_K.shape[:2] != (Hkv, d) or P_V.shape[:2] != (Hkv, d):
+            raise ValueError("compress_append: inconsistent shapes")
+        if k_lat.shape != (B, Hkv, L_max, rK) or v_lat.shape != (B, Hkv, L_max, rV):
+            raise ValueError("compress_append: inconsistent cache shapes")
+        n_bad = self.lib.stief_oracle_compress_append(
+            _ptr(k_new), _ptr(v_new), _ptr(P_K), _ptr(P_V), _ptr(k_lat), _ptr(v_lat),
+            _ptr(lens, _I32), B, Hkv, T, d, rK, rV, L_max, int(round_to_bf16))
+        return k_lat, v_lat, lens, int(n_bad)
+
+    def decode(self, q, P_K, P_V, k_lat, v_lat, seq_lens, num_threads: int = 0) -> np.ndarray:
+        """One decode step over the reconstructed latent cache; returns out [B][Hq][d] (fp64).
+
+        Shapes: q [B][Hq][d], P_K [Hkv][d][rK], P_V [Hkv][d][rV],
+        k_lat [B][Hkv][L_max][rK], v_lat [B][Hkv][L_max][rV], seq_lens [B].
+        """
+        q, P_K, P_V, k_lat, v_lat = map(_f64, (q, P_K, P_V, k_lat, v_lat))
+        lens = np.ascontiguousarray(np.asarray(seq_lens, dtype=np.int32))
+        B, Hq, d = q.shape
+        Hkv, d2, rK = P_K.shape
+        rV = P_V.shape[2]
+        L_max = k_lat.shape[2]
+        if d2 != d or Hq % Hkv != 0 or P_V.shape[:2] != (Hkv, d):
+            raise ValueError("decode: inconsistent shapes")
+        if k_lat.shape != (B, Hkv, L_max, rK) or v_lat.shape != (B, Hkv, L_max, rV):
+            raise ValueError("decode: inconsistent cache shapes")
+        out = np.empty((B, Hq, d), dtype=np.float64)
+        rc = self.lib.stief_oracle_decode(_ptr(q), _ptr(P_K), _ptr(P_V), _ptr(k_lat),
+                                          _ptr(v_lat), _ptr(lens, _I32), _ptr(out),
+                                          B, Hq, Hkv, d, rK, rV, L_max, int(num_threads))
+        if rc != 0:
+            raise ValueError("decode: a sequence length is outside [0, L_max]")
+        return out
+
+
+def default() -> Oracle:
+    """The oracle built from stief_oracle.c (compiled on first use)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            _lib = Oracle(build())
+    return _lib
+
+
+def max_threads() -> int:
+    return default().max_threads()
+
+
+def round_bf16(x) -> np.ndarray:
+    return default().round_bf16(x)
+
+
+def project(x, P, round_to_bf16: bool = True) -> np.ndarray:
+    return default().project(x, P, round_to_bf16)
+
+
+def compress_append(k_new, v_new, P_K, P_V, k_lat, v_lat, seq_lens, round_to_bf16: bool = True):
+    return default().compress_append(k_new, v_new, P_K, P_V, k_lat, v_lat, seq_lens,
+                                     round_to_bf16)
+
+
+def decode(q, P_K, P_V, k_lat, v_lat, seq_lens, num_threads: int = 0) -> np.ndarray:
+    return default().decode(q, P_K, P_V, k_lat, v_lat, seq_lens, num_threads)

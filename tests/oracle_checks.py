@@ -1,0 +1,297 @@
+"""Pins for the fp64 oracle, written as functions of an ``oracle.Oracle`` object.
+
+Each check ties the oracle to something other than itself: a library routine
+(torch's float32->bfloat16 conversion, torch's scaled_dot_product_attention in
+float64), a closed form, an invariance the pages state, or exact arithmetic.
+``test_oracle_pins.py`` runs them on the oracle; ``test_oracle_mutants.py`` runs
+them on copies of the oracle with a planted mistake and expects a failure.
+
+Pages: "Don't be so Stief! Learning KV Cache low-rank approximation over the
+Stiefel manifold", StiefAttention technical summary, "Mecanismo Central" /
+"Kernmechanismus": item 2 (orthonormal bases on the Stiefel manifold), item 3
+(QR orthonormalisation; R is only a change of coordinates inside the subspace),
+item 5 (stored K_down = K P_K, reconstruction K~ = K_down P_K^T before
+attention); "Resultados Experimentais" (the uncompressed FP16 baseline, i.e.
+plain attention, which the r = d case must reproduce).
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+import torch.nn.functional as F
+
+import stief_inputs as si
+
+
+def _rel_err(a: np.ndarray, b: np.ndarray) -> float:
+    scale = max(float(np.max(np.abs(b))), 1e-300)
+    return float(np.max(np.abs(a - b))) / scale
+
+
+def _identity_basis(d: int, r: int) -> np.ndarray:
+    """P = [I_r; 0]: the first r columns of the d x d identity (exactly representable)."""
+    P = np.zeros((d, r))
+    P[np.arange(r), np.arange(r)] = 1.0
+    return P
+
+
+# ----------------------------------------------------------------------------- bf16 rounding
+
+def check_round_bf16_matches_torch(o, n: int = 200_000, seed: int = 0) -> None:
+    """RNE to bf16 equals torch's float32 -> bfloat16 conversion on float32 inputs."""
+    rng = np.random.default_rng(seed)
+    mant = rng.uniform(1.0, 2.0, n)
+    expo = rng.integers(-140, 128, n)
+    sign = np.where(rng.random(n) < 0.5, -1.0, 1.0)
+    x32 = (sign * mant * np.exp2(expo.astype(np.float64))).astype(np.float32)
+    # also every tie pattern: low 16 bits exactly 0x8000 around random high halves
+    hi = rng.integers(0, 0x7F7F, 4096, dtype=np.uint32)
+    ties = ((hi << 16) | 0x8000).astype(np.uint32).view(np.float32)
+    x32 = np.concatenate([x32, ties, -ties])
+    ref = torch.from_numpy(x32).to(torch.bfloat16).to(torch.float64).numpy()
+    got = o.round_bf16(x32.astype(np.float64))
+    assert np.array_equal(got, ref), "bf16 rounding differs from torch's float32->bf16"
+
+
+def check_round_bf16_edges(o) -> None:
+    """Hand-derived cases: ties to even, subnormal grid, overflow to infinity."""
+    cases = [
+        (1.0 + 2.0 ** -8, 1.0),                       # tie, 1.0 has an even last bit
+        (1.0 + 3 * 2.0 ** -8, 1.0 + 2.0 ** -6),       # tie, rounds up to the even neighbour
+        (1.0 + 2.0 ** -8 + 2.0 ** -30, 1.0 + 2.0 ** -7),  # just above the tie
+        (-(1.0 + 2.0 ** -8), -1.0),
+        (2.0 ** -133, 2.0 ** -133),                   # smallest subnormal
+        (2.0 ** -134, 0.0),                           # tie between 0 and 2^-133 -> 0
+        (3 * 2.0 ** -134, 2.0 ** -132),               # tie between 1 and 2 ulps -> 2
+        ((2 - 2.0 ** -7) * 2.0 ** 127, (2 - 2.0 ** -7) * 2.0 ** 127),  # largest finite
+        ((2 - 2.0 ** -8) * 2.0 ** 127, math.inf),     # tie above the largest -> overflow
+        (0.0, 0.0),
+    ]
+    x = np.array([c[0] for c in cases])
+    want = np.array([c[1] for c in cases])
+    got = o.round_bf16(x)
+    assert np.array_equal(got, want), f"bf16 edge cases: got {got}, want {want}"
+
+
+# ----------------------------------------------------------------------------- bases
+
+def check_qr_bases_orthonormal(d: int = 128, ranks=(16, 32, 48, 64, 96, 128)) -> None:
+    """P^T P = I to 1e-6 for the QR-generated bases (before bf16 rounding)."""
+    for r in ranks:
+        P = si.bases(1234, 2, d, r)
+        for h in range(P.shape[0]):
+            err = np.max(np.abs(P[h].T @ P[h] - np.eye(r)))
+            assert err <= 1e-6, f"P^T P - I = {err} for r={r}"
+
+
+# ----------------------------------------------------------------------------- attention
+
+def _sdpa_reference(q, K, V, lens) -> np.ndarray:
+    """Textbook softmax attention (torch SDPA, float64, GQA by contiguous groups)."""
+    B, Hq, d = q.shape
+    out = np.zeros_like(q)
+    for b in range(B):
+        L = int(lens[b])
+        if L == 0:
+            continue
+        qt = torch.from_numpy(q[b][None, :, None, :])          # [1, Hq, 1, d]
+        kt = torch.from_numpy(np.ascontiguousarray(K[b][None, :, :L, :]))
+        vt = torch.from_numpy(np.ascontiguousarray(V[b][None, :, :L, :]))
+        o = F.scaled_dot_product_attention(qt, kt, vt, enable_gqa=True)
+        out[b] = o[0, :, 0, :].numpy()
+    return out
+
+
+def check_full_rank_is_plain_attention(o, q_scale: float = 1.0, d: int = 128,
+                                       tol: float = 1e-12) -> None:
+    """r = d: P is square orthogonal, so the method is exactly uncompressed attention."""
+    B, Hq, Hkv, L_max = 2, 8, 2, 40
+    lens = np.array([37, 5], dtype=np.int32)
+    rng = np.random.default_rng(11)
+    K = np.stack([si.low_rank_rows(rng, L_max, d) for _ in range(B * Hkv)]).reshape(B, Hkv, L_max, d)
+    V = np.stack([si.low_rank_rows(rng, L_max, d) for _ in range(B * Hkv)]).reshape(B, Hkv, L_max, d)
+    q = q_scale * rng.standard_normal((B, Hq, d))
+    P_K = si.bases(21, Hkv, d, d)
+    P_V = si.bases(22, Hkv, d, d)
+    zk = np.zeros((B, Hkv, L_max, d))
+    k_lat, v_lat, _, nbad = o.compress_append(K, V, P_K, P_V, zk, zk.copy(),
+                                              np.zeros(B, np.int32), round_to_bf16=False)
+    assert nbad == 0
+    got = o.decode(q, P_K, P_V, k_lat, v_lat, lens)
+    want = _sdpa_reference(q, K, V, lens)
+    assert np.all(np.isfinite(got)), "non-finite output"
+    err = _rel_err(got, want)
+    assert err <= tol, f"r=d differs from plain attention: rel err {err}"
+
+
+def check_gauge_invariance(o, r: int = 48, d: int = 128) -> None:
+    """P -> P.O (O orthogonal r x r) leaves the output unchanged (QR: R is a change of coordinates)."""
+    B, Hq, Hkv, L = 2, 4, 2, 29
+    rng = np.random.default_rng(12)
+    K = np.stack([si.low_rank_rows(rng, L, d) for _ in range(B * Hkv)]).reshape(B, Hkv, L, d)
+    V = np.stack([si.low_rank_rows(rng, L, d) for _ in range(B * Hkv)]).reshape(B, Hkv, L, d)
+    q = rng.standard_normal((B, Hq, d))
+    lens = np.array([L, 17], dtype=np.int32)
+    P_K = si.bases(31, Hkv, d, r)
+    P_V = si.bases(32, Hkv, d, r)
+    O = np.stack([si.stiefel_basis(rng, r, r) for _ in range(Hkv)])
+    outs = []
+    for PK, PV in ((P_K, P_V), (P_K @ O, P_V @ O)):
+        z = np.zeros((B, Hkv, L, r))
+        kl, vl, _, _ = o.compress_append(K, V, PK, PV, z, z.copy(), np.zeros(B, np.int32),
+                                         round_to_bf16=False)
+        outs.append(o.decode(q, PK, PV, kl, vl, lens))
+    err = _rel_err(outs[1], outs[0])
+    assert err <= 1e-12, f"basis change moved the output: rel err {err}"
+
+
+def check_single_token(o, r: int = 64, d: int = 128) -> None:
+    """L = 1: softmax of one score is 1, so o = V~_0 whatever q and K are."""
+    rng = np.random.default_rng(13)
+    B, Hq, Hkv = 1, 4, 1
+    P_K = si.bases(41, Hkv, d, r)
+    P_V = _identity_basis(d, r)[None]
+    k_lat = rng.standard_normal((B, Hkv, 3, r))
+    v_lat = rng.standard_normal((B, Hkv, 3, r))
+    q = 5.0 * rng.standard_normal((B, Hq, d))
+    got = o.decode(q, P_K, P_V, k_lat, v_lat, np.array([1], np.int32))
+    want = np.zeros((B, Hq, d))
+    want[:, :, :r] = v_lat[0, 0, 0]
+    assert np.array_equal(got, want), "one-token output is not the reconstructed value row"
+
+
+def check_two_tokens(o, r: int = 64, d: int = 128) -> None:
+    """Two tokens with scores a/sqrt(d) and 0: weights sigma(a/sqrt(d)) and 1 - sigma."""
+    Hq = 4
+    a = np.array([0.5, 3.0, -7.0, 20.0])
+    P = _identity_basis(d, r)[None]
+    q = np.zeros((1, Hq, d))
+    q[0, :, 0] = a
+    k_lat = np.zeros((1, 1, 2, r))
+    k_lat[0, 0, 0, 0] = 1.0
+    v_lat = np.zeros((1, 1, 2, r))
+    v_lat[0, 0, 0, 1] = 1.0
+    v_lat[0, 0, 1, 2] = 1.0
+    got = o.decode(q, P, P, k_lat, v_lat, np.array([2], np.int32))
+    p0 = 1.0 / (1.0 + np.exp(-a / math.sqrt(d)))
+    assert np.allclose(got[0, :, 1], p0, rtol=0, atol=1e-15), f"{got[0, :, 1]} vs {p0}"
+    assert np.allclose(got[0, :, 2], 1.0 - p0, rtol=0, atol=1e-15)
+    mask = np.ones(d, bool)
+    mask[[1, 2]] = False
+    assert np.all(got[0][:, mask] == 0.0)
+
+
+def check_uniform_keys(o, r: int = 32, d: int = 128) -> None:
+    """Identical keys give uniform weights: o is the mean of the reconstructed values."""
+    rng = np.random.default_rng(14)
+    L = 23
+    P_K = si.bases(51, 1, d, r)
+    P_V = _identity_basis(d, r)[None]
+    k_lat = np.repeat(rng.standard_normal((1, 1, 1, r)), L, axis=2)
+    v_lat = rng.standard_normal((1, 1, L, r))
+    q = rng.standard_normal((1, 2, d))
+    got = o.decode(q, P_K, P_V, k_lat, v_lat, np.array([L], np.int32))
+    want = np.zeros((1, 2, d))
+    want[0, :, :r] = v_lat[0, 0].mean(axis=0)
+    assert _rel_err(got, want) <= 1e-13
+
+
+def check_token_order_invariance(o, r: int = 48, d: int = 128) -> None:
+    """Permuting the cache rows (keys and values together) does not change the output."""
+    rng = np.random.default_rng(15)
+    L = 31
+    P_K = si.bases(61, 2, d, r)
+    P_V = si.bases(62, 2, d, r)
+    k_lat = rng.standard_normal((1, 2, L, r))
+    v_lat = rng.standard_normal((1, 2, L, r))
+    q = 3.0 * rng.standard_normal((1, 4, d))
+    lens = np.array([L], np.int32)
+    perm = rng.permutation(L)
+    a = o.decode(q, P_K, P_V, k_lat, v_lat, lens)
+    b = o.decode(q, P_K, P_V, k_lat[:, :, perm], v_lat[:, :, perm], lens)
+    assert _rel_err(b, a) <= 1e-12
+
+
+def check_empty_sequence(o, r: int = 64, d: int = 128) -> None:
+    """Length 0 attends to nothing: output exactly zero (and finite)."""
+    rng = np.random.default_rng(16)
+    P = si.bases(71, 1, d, r)
+    got = o.decode(rng.standard_normal((2, 4, d)), P, P, rng.standard_normal((2, 1, 8, r)),
+                   rng.standard_normal((2, 1, 8, r)), np.array([0, 3], np.int32))
+    assert np.all(got[0] == 0.0)
+    assert np.all(np.isfinite(got[1])) and np.any(got[1] != 0.0)
+
+
+# ----------------------------------------------------------------------------- compression
+
+def check_compress_identity_basis(o, r: int = 48, d: int = 128) -> None:
+    """P = [I_r; 0]: the stored latent is exactly the first r coordinates of each bf16 row."""
+    rng = np.random.default_rng(17)
+    x = si.bf16_to_f64(si.to_bf16(rng.standard_normal((19, d))))
+    y = o.project(x, _identity_basis(d, r), round_to_bf16=True)
+    assert np.array_equal(y, x[:, :r])
+
+
+def check_compress_matches_exact_product(o, r: int = 64, d: int = 128) -> None:
+    """Unrounded compression equals x.P to fp64 round-off; rounded is its RNE bf16 value."""
+    rng = np.random.default_rng(18)
+    x = si.bf16_to_f64(si.to_bf16(rng.standard_normal((33, d))))
+    P = si.bf16_to_f64(si.to_bf16(si.bases(81, 1, d, r)[0]))
+    exact = o.project(x, P, round_to_bf16=False)
+    lib = x @ P
+    assert _rel_err(exact, lib) <= 1e-14
+    rounded = o.project(x, P, round_to_bf16=True)
+    ref = torch.from_numpy(exact.astype(np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
+    # double rounding fp64 -> fp32 -> bf16 can differ from direct RNE only at near-ties
+    ulp = np.exp2(np.floor(np.log2(np.abs(ref) + 1e-300)) - 7)
+    assert np.all(np.abs(rounded - ref) <= ulp)
+    assert np.mean(rounded == ref) > 0.999
+
+
+def check_compress_append_bookkeeping(o, r: int = 32, d: int = 128) -> None:
+    """Rows land exactly at [len, len+T); other slots are untouched; overflow writes nothing."""
+    rng = np.random.default_rng(19)
+    B, Hkv, T, L_max = 3, 2, 3, 10
+    lens = np.array([0, 7, 8], np.int32)   # the second fills the cache exactly, the last overflows
+    k_new = si.bf16_to_f64(si.to_bf16(rng.standard_normal((B, Hkv, T, d))))
+    v_new = si.bf16_to_f64(si.to_bf16(rng.standard_normal((B, Hkv, T, d))))
+    P = _identity_basis(d, r)[None].repeat(Hkv, axis=0)
+    canary = 12345.0
+    k_lat = np.full((B, Hkv, L_max, r), canary)
+    v_lat = np.full((B, Hkv, L_max, r), -canary)
+    kl, vl, new_lens, nbad = o.compress_append(k_new, v_new, P, P, k_lat, v_lat, lens)
+    assert nbad == 1
+    assert new_lens.tolist() == [3, 10, 8]
+    for b in range(B):
+        for h in range(Hkv):
+            if b < 2:
+                s = int(lens[b])
+                assert np.array_equal(kl[b, h, s:s + T], k_new[b, h, :, :r])
+                assert np.array_equal(vl[b, h, s:s + T], v_new[b, h, :, :r])
+                keep = np.ones(L_max, bool)
+                keep[s:s + T] = False
+            else:
+                keep = np.ones(L_max, bool)
+            assert np.all(kl[b, h, keep] == canary)
+            assert np.all(vl[b, h, keep] == -canary)
+
+
+ALL_ORACLE_CHECKS = {
+    "round_bf16_matches_torch": check_round_bf16_matches_torch,
+    "round_bf16_edges": check_round_bf16_edges,
+    "full_rank_is_plain_attention": check_full_rank_is_plain_attention,
+    # scores in the hundreds: exp() overflows unless the maximum is subtracted first
+    "full_rank_large_scores": lambda o: check_full_rank_is_plain_attention(o, q_scale=400.0,
+                                                                           tol=1e-10),
+    "gauge_invariance": check_gauge_invariance,
+    "single_token": check_single_token,
+    "two_tokens": check_two_tokens,
+    "uniform_keys": check_uniform_keys,
+    "token_order_invariance": check_token_order_invariance,
+    "empty_sequence": check_empty_sequence,
+    "compress_identity_basis": check_compress_identity_basis,
+    "compress_matches_exact_product": check_compress_matches_exact_product,
+    "compress_append_bookkeeping": check_compress_append_bookkeeping,
+}

@@ -1,0 +1,79 @@
+"""Plant a mistake in a copy of the oracle's C source; some pin must catch it.
+
+Each mutant is a plausible slip (wrong scale, wrong GQA mapping, transposed
+basis, missing normalisation, off-by-one in the append offset, ...).  The copy is
+compiled with gcc into a temporary directory and exercised in a child process
+(an off-by-one may write outside an array, so the child may also die: that
+counts as caught).  The oracle source itself is never changed.
+"""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+import oracle
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "stief_oracle.c")
+TESTS = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(TESTS)
+
+# (name, original text, replacement, checks expected to fail)
+MUTANTS = [
+    ("scale_uses_rank", "1.0 / sqrt((double)d)", "1.0 / sqrt((double)rK)", ["two_tokens"]),
+    ("gqa_interleaved", "(long)g * G + j", "(long)j * Hkv + g", ["full_rank_is_plain_attention"]),
+    ("reconstruct_transposed", "acc += lat[c] * P[(long)i * r + c];",
+     "acc += lat[c] * P[(long)c * d + i];", ["single_token", "gauge_invariance"]),
+    ("compress_transposed", "acc += x[t * d + i] * P[(long)i * r + c];",
+     "acc += x[t * d + i] * P[(long)c * d + i];",
+     ["compress_identity_basis", "full_rank_is_plain_attention"]),
+    ("no_max_subtraction", "sj[t] = exp(sj[t] - mx);", "sj[t] = exp(sj[t]);",
+     ["full_rank_large_scores"]),
+    ("unnormalised_weights", "double p = s[(long)j * L + t] / denom[j];",
+     "double p = s[(long)j * L + t];", ["two_tokens", "uniform_keys"]),
+    ("values_use_key_basis", "reconstruct_row(Vd + t * rV, PV, d, rV, row);",
+     "reconstruct_row(Vd + t * rV, PK, d, rV, row);", ["full_rank_is_plain_attention"]),
+    ("first_value_dropped",
+     "for (long t = 0; t < L; ++t) {\n            reconstruct_row(Vd",
+     "for (long t = 1; t < L; ++t) {\n            reconstruct_row(Vd",
+     ["single_token", "two_tokens"]),
+    ("round_ties_away", "nearbyint(x / q)", "round(x / q)",
+     ["round_bf16_edges", "round_bf16_matches_torch"]),
+    ("append_off_by_one", "long dst = ((long)b * Hkv + h) * L_max + L;",
+     "long dst = ((long)b * Hkv + h) * L_max + L + 1;", ["compress_append_bookkeeping"]),
+    ("capacity_rejects_exact_fit", "if (L < 0 || L + T > L_max) {",
+     "if (L < 0 || L + T >= L_max) {", ["compress_append_bookkeeping"]),
+]
+
+_CHILD = r"""
+import json, sys
+sys.path[:0] = [{root!r}, {tests!r}]
+import oracle, oracle_checks as oc
+m = oracle.Oracle({lib!r})
+caught = {{}}
+for name in {checks!r}:
+    try:
+        oc.ALL_ORACLE_CHECKS[name](m)
+        caught[name] = False
+    except (AssertionError, ValueError):
+        caught[name] = True
+print(json.dumps(caught))
+"""
+
+
+@pytest.mark.parametrize("name,orig,repl,checks", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_mutant_is_caught(tmp_path, name, orig, repl, checks):
+    src = open(SRC).read()
+    assert src.count(orig) >= 1, f"mutation site for {name} not found"
+    mutated = tmp_path / f"{name}.c"
+    mutated.write_text(src.replace(orig, repl))
+    lib = oracle.build(str(mutated), str(tmp_path / f"{name}.so"), force=True)
+    code = _CHILD.format(root=ROOT, tests=TESTS, lib=lib, checks=checks)
+    proc = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True,
+                          timeout=300)
+    if proc.returncode != 0:
+        return  # the planted mistake crashed the child (e.g. an out-of-bounds write): caught
+    caught = json.loads(proc.stdout.strip().splitlines()[-1])
+    missed = [c for c, ok in caught.items() if not ok]
+    assert not missed, f"mutant {name} passed pins {missed}"
