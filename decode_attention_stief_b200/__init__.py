@@ -1,0 +1,24 @@
+"""B200 (sm_100a) StiefAttention latent-KV decode: Python binding of libstief.so.
+
+The compute path is the CUDA library ``libstief.so`` (C ABI in include/stief.h).
+This package only marshals torch tensors (device pointers, sizes, the current
+stream) into those calls.  There is no CPU fallback: if the library cannot be
+loaded, every call raises.
+"""
+from ._binding import (  # noqa: F401
+    StiefError,
+    STATUS,
+    DEV_CAPACITY_OVERFLOW,
+    DEV_WAIT_TIMEOUT,
+    DEV_BAD_LENGTH,
+    library,
+    library_path,
+    stief_compress_append,
+    stief_decode_attention,
+    stief_decode_auto_splits,
+    stief_decode_max_splits,
+    stief_decode_workspace_bytes,
+    stief_read_device_status,
+    stief_status_string,
+    workspace_for,
+)

@@ -1,0 +1,219 @@
+"""ctypes binding of libstief.so: argument marshalling only.
+
+Every function here takes torch tensors, checks dtype / device / contiguity /
+shape agreement, and passes raw device pointers, sizes and the current CUDA
+stream to the C entry point of the same name.  All arithmetic runs in the
+library's CUDA kernels.  There is no fallback path: a missing or unloadable
+library raises ``StiefError``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.environ.get("STIEF_LIBRARY", os.path.join(_PKG, "libstief.so"))
+
+STATUS = {
+    0: "STIEF_OK",
+    1: "STIEF_ERR_INVALID_ARG",
+    2: "STIEF_ERR_ALIGNMENT",
+    3: "STIEF_ERR_CAPACITY",
+    4: "STIEF_ERR_WORKSPACE",
+    5: "STIEF_ERR_CUDA",
+    6: "STIEF_ERR_DEVICE_STATUS",
+    7: "STIEF_ERR_UNSUPPORTED_DEVICE",
+}
+DEV_CAPACITY_OVERFLOW = 0x1
+DEV_WAIT_TIMEOUT = 0x2
+DEV_BAD_LENGTH = 0x4
+
+
+class StiefError(RuntimeError):
+    """A libstief call returned a non-OK status (or the library is missing)."""
+
+    def __init__(self, func: str, code: int):
+        self.code = code
+        super().__init__(f"{func}: {STATUS.get(code, code)}")
+
+
+_lock = threading.Lock()
+_lib = None
+
+_u16p = ctypes.c_void_p
+_i = ctypes.c_int
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def library() -> ctypes.CDLL:
+    """Load libstief.so (once).  Raises StiefError if it is missing."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(_LIB_PATH):
+                raise StiefError(f"libstief.so not found at {_LIB_PATH}; build it with "
+                                 "python -m decode_attention_stief_b200.build", -1)
+            lib = ctypes.CDLL(_LIB_PATH)
+            vp = ctypes.c_void_p
+            lib.stief_compress_append.restype = _i
+            lib.stief_compress_append.argtypes = [vp] * 7 + [_i] * 7 + [vp, vp]
+            lib.stief_decode_attention.restype = _i
+            lib.stief_decode_attention.argtypes = ([vp] * 8 + [ctypes.c_size_t] + [_i] * 9
+                                                   + [vp, vp])
+            lib.stief_decode_workspace_bytes.restype = ctypes.c_size_t
+            lib.stief_decode_workspace_bytes.argtypes = [_i] * 5
+            lib.stief_decode_max_splits.restype = _i
+            lib.stief_decode_max_splits.argtypes = [_i]
+            lib.stief_decode_auto_splits.restype = _i
+            lib.stief_decode_auto_splits.argtypes = [_i] * 5
+            lib.stief_read_device_status.restype = _i
+            lib.stief_read_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32), vp]
+            lib.stief_status_string.restype = ctypes.c_char_p
+            lib.stief_status_string.argtypes = [_i]
+            _lib = lib
+    return _lib
+
+
+def _check(func: str, code: int) -> None:
+    if code != 0:
+        raise StiefError(func, code)
+
+
+def _stream_ptr(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _dev(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int) -> int:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be on a CUDA device")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _opt_status(dev_status: Optional[torch.Tensor]) -> Optional[int]:
+    if dev_status is None:
+        return None
+    if dev_status.dtype not in (torch.int32, torch.uint32) or dev_status.numel() < 1 or not dev_status.is_cuda:
+        raise ValueError("dev_status must be a CUDA int32/uint32 tensor with at least one element")
+    return dev_status.data_ptr()
+
+
+def stief_status_string(code: int) -> str:
+    return library().stief_status_string(int(code)).decode()
+
+
+def stief_decode_max_splits(max_seq_len: int) -> int:
+    return int(library().stief_decode_max_splits(int(max_seq_len)))
+
+
+def stief_decode_auto_splits(B: int, Hq: int, Hkv: int, max_seq_len: int, num_sms: int) -> int:
+    return int(library().stief_decode_auto_splits(B, Hq, Hkv, max_seq_len, num_sms))
+
+
+def stief_decode_workspace_bytes(B: int, Hq: int, Hkv: int, rV: int, max_seq_len: int) -> int:
+    return int(library().stief_decode_workspace_bytes(B, Hq, Hkv, rV, max_seq_len))
+
+
+def workspace_for(B: int, Hq: int, Hkv: int, rV: int, max_seq_len: int,
+                  device="cuda") -> torch.Tensor:
+    """A uint8 device tensor of stief_decode_workspace_bytes(...) bytes."""
+    n = stief_decode_workspace_bytes(B, Hq, Hkv, rV, max_seq_len)
+    if n == 0:
+        raise ValueError("invalid sizes for the decode workspace")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def stief_compress_append(k_new: torch.Tensor, v_new: torch.Tensor, P_K: torch.Tensor,
+                          P_V: torch.Tensor, k_lat: torch.Tensor, v_lat: torch.Tensor,
+                          seq_lens: torch.Tensor, dev_status: Optional[torch.Tensor] = None,
+                          stream=None) -> None:
+    """Project T new rows per (sequence, KV head) into the latent cache and advance seq_lens.
+
+    k_new, v_new [B][Hkv][T][d] bf16; P_K [Hkv][d][rK], P_V [Hkv][d][rV] bf16;
+    k_lat [B][Hkv][L_max][rK], v_lat [B][Hkv][L_max][rV] bf16; seq_lens [B] int32.
+    """
+    pk = _dev(k_new, "k_new", torch.bfloat16, 4)
+    pv = _dev(v_new, "v_new", torch.bfloat16, 4)
+    ppk = _dev(P_K, "P_K", torch.bfloat16, 3)
+    ppv = _dev(P_V, "P_V", torch.bfloat16, 3)
+    pkl = _dev(k_lat, "k_lat", torch.bfloat16, 4)
+    pvl = _dev(v_lat, "v_lat", torch.bfloat16, 4)
+    psl = _dev(seq_lens, "seq_lens", torch.int32, 1)
+    B, Hkv, T, d = k_new.shape
+    rK, rV = P_K.shape[2], P_V.shape[2]
+    L_max = k_lat.shape[2]
+    if tuple(v_new.shape) != (B, Hkv, T, d) or tuple(P_K.shape) != (Hkv, d, rK) \
+            or tuple(P_V.shape) != (Hkv, d, rV) or tuple(k_lat.shape) != (B, Hkv, L_max, rK) \
+            or tuple(v_lat.shape) != (B, Hkv, L_max, rV) or seq_lens.shape[0] != B:
+        raise ValueError("stief_compress_append: inconsistent shapes")
+    code = library().stief_compress_append(pk, pv, ppk, ppv, pkl, pvl, psl, B, Hkv, T, d, rK,
+                                           rV, L_max, _opt_status(dev_status),
+                                           _stream_ptr(stream))
+    _check("stief_compress_append", code)
+
+
+def stief_decode_attention(q: torch.Tensor, P_K: torch.Tensor, P_V: torch.Tensor,
+                           k_lat: torch.Tensor, v_lat: torch.Tensor, seq_lens: torch.Tensor,
+                           out: torch.Tensor, workspace: torch.Tensor, max_seq_len: int,
+                           num_splits: int = 0, dev_status: Optional[torch.Tensor] = None,
+                           stream=None) -> torch.Tensor:
+    """One decode step: out [B][Hq][d] = softmax(q K~^T / sqrt(d)) V~ over the latent cache.
+
+    q [B][Hq][d] bf16; P_K [Hkv][d][rK], P_V [Hkv][d][rV] bf16;
+    k_lat [B][Hkv][L_max][rK], v_lat [B][Hkv][L_max][rV] bf16; seq_lens [B] int32;
+    out [B][Hq][d] bf16 (written); workspace: uint8 device tensor of at least
+    stief_decode_workspace_bytes(...) bytes.
+    """
+    pq = _dev(q, "q", torch.bfloat16, 3)
+    ppk = _dev(P_K, "P_K", torch.bfloat16, 3)
+    ppv = _dev(P_V, "P_V", torch.bfloat16, 3)
+    pkl = _dev(k_lat, "k_lat", torch.bfloat16, 4)
+    pvl = _dev(v_lat, "v_lat", torch.bfloat16, 4)
+    psl = _dev(seq_lens, "seq_lens", torch.int32, 1)
+    po = _dev(out, "out", torch.bfloat16, 3)
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    B, Hq, d = q.shape
+    Hkv, _, rK = P_K.shape
+    rV = P_V.shape[2]
+    L_max = k_lat.shape[2]
+    if tuple(P_K.shape) != (Hkv, d, rK) or tuple(P_V.shape) != (Hkv, d, rV) \
+            or tuple(k_lat.shape) != (B, Hkv, L_max, rK) \
+            or tuple(v_lat.shape) != (B, Hkv, L_max, rV) or seq_lens.shape[0] != B \
+            or tuple(out.shape) != (B, Hq, d):
+        raise ValueError("stief_decode_attention: inconsistent shapes")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    code = library().stief_decode_attention(pq, ppk, ppv, pkl, pvl, psl, po,
+                                            workspace.data_ptr(), ws_bytes, B, Hq, Hkv, d, rK,
+                                            rV, L_max, int(max_seq_len), int(num_splits),
+                                            _opt_status(dev_status), _stream_ptr(stream))
+    _check("stief_decode_attention", code)
+    return out
+
+
+def stief_read_device_status(dev_status: torch.Tensor, stream=None) -> int:
+    """Synchronise the stream and return the device status word (0 = no condition seen)."""
+    v = ctypes.c_uint32(0)
+    code = library().stief_read_device_status(_opt_status(dev_status), ctypes.byref(v),
+                                              _stream_ptr(stream))
+    if code not in (0, 6):
+        raise StiefError("stief_read_device_status", code)
+    return int(v.value)

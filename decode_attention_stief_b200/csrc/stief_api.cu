@@ -1,0 +1,209 @@
+// stief_api.cu -- the C ABI declared in include/stief.h: argument checking,
+// split planning, workspace sizing and kernel launches.  Host code only.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include <cuda_runtime.h>
+
+#include "../../include/stief.h"
+#include "stief_internal.h"
+
+namespace {
+
+constexpr int kHeadDim = 128;          // the only supported d
+constexpr int kMinTokensPerSplit = 128;
+constexpr int kMaxSplits = 512;
+constexpr int kMaxGroup = 64;          // largest Hq / Hkv
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool rank_ok(int r) { return r >= 16 && r <= kHeadDim && (r % 16) == 0; }
+
+int group_tile(int G) { return G <= 1 ? 1 : G <= 2 ? 2 : G <= 4 ? 4 : 8; }
+
+stief_status device_check() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return STIEF_ERR_CUDA;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return STIEF_ERR_CUDA;
+  if (major != 10 || minor != 0) return STIEF_ERR_UNSUPPORTED_DEVICE;
+  return STIEF_OK;
+}
+
+// Common decode shape checks (host only, no CUDA call).
+stief_status check_decode_shape(int B, int Hq, int Hkv, int d, int rK, int rV, int L_max,
+                                int max_seq_len) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || Hq / Hkv > kMaxGroup) return STIEF_ERR_INVALID_ARG;
+  if (d != kHeadDim || !rank_ok(rK) || !rank_ok(rV)) return STIEF_ERR_INVALID_ARG;
+  if (L_max < 1 || max_seq_len < 0) return STIEF_ERR_INVALID_ARG;
+  if (max_seq_len > L_max) return STIEF_ERR_CAPACITY;
+  return STIEF_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* stief_status_string(stief_status s) {
+  switch (s) {
+    case STIEF_OK: return "STIEF_OK";
+    case STIEF_ERR_INVALID_ARG: return "STIEF_ERR_INVALID_ARG";
+    case STIEF_ERR_ALIGNMENT: return "STIEF_ERR_ALIGNMENT";
+    case STIEF_ERR_CAPACITY: return "STIEF_ERR_CAPACITY";
+    case STIEF_ERR_WORKSPACE: return "STIEF_ERR_WORKSPACE";
+    case STIEF_ERR_CUDA: return "STIEF_ERR_CUDA";
+    case STIEF_ERR_DEVICE_STATUS: return "STIEF_ERR_DEVICE_STATUS";
+    case STIEF_ERR_UNSUPPORTED_DEVICE: return "STIEF_ERR_UNSUPPORTED_DEVICE";
+  }
+  return "STIEF_ERR_UNKNOWN";
+}
+
+int stief_decode_max_splits(int max_seq_len) {
+  if (max_seq_len < 0) return 0;
+  int s = (max_seq_len + kMinTokensPerSplit - 1) / kMinTokensPerSplit;
+  if (s < 1) s = 1;
+  if (s > kMaxSplits) s = kMaxSplits;
+  return s;
+}
+
+int stief_decode_auto_splits(int B, int Hq, int Hkv, int max_seq_len, int num_sms) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || max_seq_len < 0 || num_sms < 1) return 0;
+  const int G = Hq / Hkv;
+  const int qsub = (G + group_tile(G) - 1) / group_tile(G);
+  const long long units = (long long)B * Hkv * qsub;
+  // one split CTA per SM: split only while there are fewer units than SMs
+  long long s = units >= num_sms ? 1 : num_sms / units;
+  const int smax = stief_decode_max_splits(max_seq_len);
+  if (s > smax) s = smax;
+  if (s < 1) s = 1;
+  return (int)s;
+}
+
+size_t stief_decode_workspace_bytes(int B, int Hq, int Hkv, int rV, int max_seq_len) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || !rank_ok(rV) || max_seq_len < 0) return 0;
+  const int G = Hq / Hkv;
+  const int G_T = group_tile(G);
+  const int qsub = (G + G_T - 1) / G_T;
+  const size_t parts = (size_t)B * Hkv * qsub * G_T * stief_decode_max_splits(max_seq_len);
+  return parts * (size_t)(rV + 2) * sizeof(float);
+}
+
+stief_status stief_compress_append(const uint16_t* k_new, const uint16_t* v_new,
+                                   const uint16_t* P_K, const uint16_t* P_V, uint16_t* k_lat,
+                                   uint16_t* v_lat, int32_t* seq_lens, int B, int Hkv, int T,
+                                   int d, int rK, int rV, int L_max, uint32_t* dev_status,
+                                   stief_stream_t stream) {
+  if (!k_new || !v_new || !P_K || !P_V || !k_lat || !v_lat || !seq_lens) return STIEF_ERR_INVALID_ARG;
+  if (B < 1 || Hkv < 1 || T < 0 || d != kHeadDim || !rank_ok(rK) || !rank_ok(rV) || L_max < 1)
+    return STIEF_ERR_INVALID_ARG;
+  if (T > L_max) return STIEF_ERR_CAPACITY;
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(P_K) || !aligned16(P_V) ||
+      !aligned16(k_lat) || !aligned16(v_lat))
+    return STIEF_ERR_ALIGNMENT;
+  if (T == 0) return STIEF_OK;
+  stief_status st = device_check();
+  if (st != STIEF_OK) return st;
+  stief::CompressArgs a{};
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.P_K = P_K;
+  a.P_V = P_V;
+  a.k_lat = k_lat;
+  a.v_lat = v_lat;
+  a.seq_lens = seq_lens;
+  a.dev_status = dev_status;
+  a.B = B;
+  a.Hkv = Hkv;
+  a.T = T;
+  a.d = d;
+  a.rK = rK;
+  a.rV = rV;
+  a.L_max = L_max;
+  if (stief::launch_compress(a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return STIEF_ERR_CUDA;
+  return STIEF_OK;
+}
+
+stief_status stief_decode_attention(const uint16_t* q, const uint16_t* P_K, const uint16_t* P_V,
+                                    const uint16_t* k_lat, const uint16_t* v_lat,
+                                    const int32_t* seq_lens, uint16_t* out, void* workspace,
+                                    size_t workspace_bytes, int B, int Hq, int Hkv, int d, int rK,
+                                    int rV, int L_max, int max_seq_len, int num_splits,
+                                    uint32_t* dev_status, stief_stream_t stream) {
+  if (!q || !P_K || !P_V || !k_lat || !v_lat || !seq_lens || !out) return STIEF_ERR_INVALID_ARG;
+  stief_status st = check_decode_shape(B, Hq, Hkv, d, rK, rV, L_max, max_seq_len);
+  if (st != STIEF_OK) return st;
+  const int smax = stief_decode_max_splits(max_seq_len);
+  if (num_splits < 0 || num_splits > smax) return STIEF_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(P_K) || !aligned16(P_V) || !aligned16(k_lat) ||
+      !aligned16(v_lat) || !aligned16(out) || !aligned16(workspace))
+    return STIEF_ERR_ALIGNMENT;
+  const size_t need = stief_decode_workspace_bytes(B, Hq, Hkv, rV, max_seq_len);
+  if (!workspace || workspace_bytes < need) return STIEF_ERR_WORKSPACE;
+  st = device_check();
+  if (st != STIEF_OK) return st;
+
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return STIEF_ERR_CUDA;
+
+  stief::DecodeArgs a{};
+  a.q = q;
+  a.P_K = P_K;
+  a.P_V = P_V;
+  a.k_lat = k_lat;
+  a.v_lat = v_lat;
+  a.seq_lens = seq_lens;
+  a.out = out;
+  a.dev_status = dev_status;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.G = Hq / Hkv;
+  a.G_T = group_tile(a.G);
+  a.qsub = (a.G + a.G_T - 1) / a.G_T;
+  a.d = d;
+  a.rK = rK;
+  a.rV = rV;
+  a.L_max = L_max;
+  a.S = num_splits > 0 ? num_splits : stief_decode_auto_splits(B, Hq, Hkv, max_seq_len, sms);
+  a.qscale = (float)(1.4426950408889634 / std::sqrt((double)d));
+  a.pdl_first = false;
+  // the workspace is laid out for the split count actually used
+  const size_t parts = (size_t)B * Hkv * a.qsub * a.G_T * a.S;
+  a.ws_o = static_cast<float*>(workspace);
+  a.ws_ml = a.ws_o + parts * rV;
+
+  // widest configuration that fits: 8 warps with as many stages as fit, else 4 warps
+  a.nwarps = 0;
+  for (int nw : {8, 4}) {
+    for (int ns = 4; ns >= 2; --ns) {
+      if (stief::decode_split_smem_bytes(nw, ns, a.G_T, d, rK, rV) <= (uint32_t)stief::kMaxSmemPerBlock) {
+        a.nwarps = nw;
+        a.nstage = ns;
+        break;
+      }
+    }
+    if (a.nwarps) break;
+  }
+  if (!a.nwarps) return STIEF_ERR_INVALID_ARG;
+  if (stief::launch_decode(a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return STIEF_ERR_CUDA;
+  return STIEF_OK;
+}
+
+stief_status stief_read_device_status(const uint32_t* dev_status, uint32_t* value,
+                                      stief_stream_t stream) {
+  if (!dev_status || !value) return STIEF_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(value, dev_status, sizeof(uint32_t), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return STIEF_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return STIEF_ERR_CUDA;
+  return *value == 0 ? STIEF_OK : STIEF_ERR_DEVICE_STATUS;
+}
+
+}  // extern "C"

@@ -1,0 +1,188 @@
+/*
+ * stief.h -- C ABI of the B200 (sm_100a) StiefAttention latent-KV decode library.
+ *
+ * The operation comes from "Don't be so Stief! Learning KV Cache low-rank
+ * approximation over the Stiefel manifold" (StiefAttention technical summary,
+ * "Mecanismo Central" / "Kernmechanismus"):
+ *   item 2 -- the projection bases P_K (d x r_K) and P_V (d x r_V) have
+ *             orthonormal columns (points on the Stiefel manifold);
+ *   item 5 -- keys and values are stored compressed, K_down = K . P_K and
+ *             V_down = V . P_V, and the full dimensions are reconstructed on the
+ *             fly, K~ = K_down . P_K^T, V~ = V_down . P_V^T, before attention.
+ * The pages give no interface, precision, scale, head mapping or layout.  This
+ * library fixes them as follows:
+ *   - one basis pair per KV head, bf16, row-major [Hkv][d][r];
+ *   - scores are scaled by 1/sqrt(d), d the full head dimension;
+ *   - grouped-query attention with contiguous groups: query head h reads KV
+ *     head h / (Hq / Hkv);
+ *   - the latent cache is bf16, row-major [B][Hkv][L_max][r] (one row per
+ *     token); all arithmetic accumulates in fp32; outputs are bf16 (RNE).
+ *
+ * Conventions for every call:
+ *   - "bf16" arguments are arrays of IEEE bfloat16 bit patterns (uint16_t).
+ *   - Every pointer is caller-owned DEVICE memory on the current CUDA device,
+ *     dense (no strides), and 16-byte aligned.  The library never allocates,
+ *     frees or retains memory and keeps no state between calls.
+ *   - Calls are asynchronous on `stream` (NULL = the legacy default stream).
+ *     A call that returns an error from argument checking launches nothing.
+ *   - Supported: d == 128; 16 <= r_K, r_V <= 128 with r % 16 == 0; Hq % Hkv == 0;
+ *     1 <= Hq / Hkv <= 64; B, Hkv >= 1.
+ *   - `dev_status` (may be NULL) is a device uint32 word.  Kernels OR the
+ *     STIEF_DEV_* bits below into it when they meet a condition that host-side
+ *     checks cannot see.  The library never clears it: the caller zeroes it
+ *     and reads it back with stief_read_device_status().
+ *   - Calls on one stream are ordered; concurrent calls on different streams
+ *     must not share output or workspace buffers.
+ */
+#ifndef STIEF_H
+#define STIEF_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define STIEF_API __attribute__((visibility("default")))
+#else
+#define STIEF_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* The same type as cudaStream_t (a pointer to the runtime's opaque stream). */
+typedef struct CUstream_st* stief_stream_t;
+
+typedef enum stief_status {
+    STIEF_OK = 0,
+    STIEF_ERR_INVALID_ARG = 1,      /* null pointer, bad size or unsupported shape */
+    STIEF_ERR_ALIGNMENT = 2,        /* a pointer is not 16-byte aligned */
+    STIEF_ERR_CAPACITY = 3,         /* max_seq_len > L_max, or T > L_max */
+    STIEF_ERR_WORKSPACE = 4,        /* workspace missing or smaller than required */
+    STIEF_ERR_CUDA = 5,             /* a CUDA runtime call failed (launch, attribute) */
+    STIEF_ERR_DEVICE_STATUS = 6,    /* stief_read_device_status found a non-zero word */
+    STIEF_ERR_UNSUPPORTED_DEVICE = 7 /* current device is not compute capability 10.0 */
+} stief_status;
+
+/* Bits kernels OR into *dev_status. */
+#define STIEF_DEV_CAPACITY_OVERFLOW 0x1u /* compress: seq_lens[b] + T > L_max; that
+                                            sequence was left untouched */
+#define STIEF_DEV_WAIT_TIMEOUT 0x2u      /* a bounded wait on an asynchronous copy or
+                                            tensor-core completion gave up */
+#define STIEF_DEV_BAD_LENGTH 0x4u        /* a seq_lens entry was negative or > L_max
+                                            (decode: that sequence's output is zero;
+                                            compress: it is left untouched) */
+
+/*
+ * stief_compress_append -- compressed storage of new keys and values
+ * (StiefAttention technical summary, "Mecanismo Central" item 5: K_down = K P_K).
+ *
+ * For every sequence b and KV head h, projects the T new rows
+ *     k_lat[b][h][seq_lens[b] + t][:] = bf16_RNE( k_new[b][h][t][:] . P_K[h] )
+ *     v_lat[b][h][seq_lens[b] + t][:] = bf16_RNE( v_new[b][h][t][:] . P_V[h] )
+ * for t < T (fp32 accumulation), then sets seq_lens[b] += T.  Rows outside
+ * [seq_lens[b], seq_lens[b] + T) are not touched.
+ *
+ *   k_new, v_new : bf16 [B][Hkv][T][d]              (read)
+ *   P_K, P_V     : bf16 [Hkv][d][rK], [Hkv][d][rV]  (read)
+ *   k_lat, v_lat : bf16 [B][Hkv][L_max][rK], [B][Hkv][L_max][rV]  (written)
+ *   seq_lens     : int32 [B] on the device          (read, then advanced by T)
+ *   T            : rows per (sequence, head); T == 0 is a no-op returning OK
+ *
+ * A sequence whose seq_lens[b] + T exceeds L_max (or whose length is negative)
+ * is skipped entirely -- no row written, length unchanged -- and
+ * STIEF_DEV_CAPACITY_OVERFLOW (or STIEF_DEV_BAD_LENGTH) is set in *dev_status.
+ * Small T runs on CUDA cores; prefill-sized T runs as a tcgen05 tensor-core
+ * GEMM with the accumulator in tensor memory.
+ * Returns STIEF_OK or an argument error (nothing launched).
+ */
+STIEF_API stief_status stief_compress_append(const uint16_t* k_new, const uint16_t* v_new,
+                                   const uint16_t* P_K, const uint16_t* P_V,
+                                   uint16_t* k_lat, uint16_t* v_lat, int32_t* seq_lens,
+                                   int B, int Hkv, int T, int d, int rK, int rV, int L_max,
+                                   uint32_t* dev_status, stief_stream_t stream);
+
+/*
+ * stief_decode_max_splits -- the largest split count a decode over sequences of
+ * at most max_seq_len tokens may use (explicit or automatic).  Pure host
+ * function.  Returns 0 for invalid arguments.
+ */
+STIEF_API int stief_decode_max_splits(int max_seq_len);
+
+/*
+ * stief_decode_auto_splits -- the split count stief_decode_attention picks when
+ * num_splits == 0, for a device with num_sms streaming multiprocessors.  Pure
+ * host function (no CUDA call).  Returns 0 for invalid arguments.
+ */
+STIEF_API int stief_decode_auto_splits(int B, int Hq, int Hkv, int max_seq_len, int num_sms);
+
+/*
+ * stief_decode_workspace_bytes -- bytes of device workspace stief_decode_attention
+ * needs for these sizes, for any split count it may use (at most
+ * stief_decode_max_splits(max_seq_len)).  The workspace holds the per-split
+ * partial softmax states (running maximum, sum and unnormalised latent output).
+ * Pure host function.  Returns 0 for invalid arguments.
+ */
+STIEF_API size_t stief_decode_workspace_bytes(int B, int Hq, int Hkv, int rV, int max_seq_len);
+
+/*
+ * stief_decode_attention -- one autoregressive decode step over the latent cache
+ * (StiefAttention technical summary, "Mecanismo Central" item 5: attention over
+ * K~ = K_down P_K^T and V~ = V_down P_V^T).
+ *
+ * For every sequence b and query head h (KV head g = h / (Hq/Hkv), L = seq_lens[b]):
+ *     s_t = q[b][h] . K~_t / sqrt(d)                       t < L
+ *     out[b][h] = bf16_RNE( sum_t softmax(s)_t V~_t )
+ * computed without materialising K~ or V~:
+ *     q~ = q[b][h] . P_K[g]                  (fp32, per CTA)
+ *     s_t = q~ . K_down[b][g][t] / sqrt(d)
+ *     o~ = sum_t softmax(s)_t V_down[b][g][t] (split-KV, online softmax, fp32)
+ *     out[b][h] = o~ . P_V[g]^T
+ * which equals the definition up to rounding by associativity of the products,
+ * (q . P_K) . K_down[t] = q . (K_down[t] . P_K^T) and
+ * (sum_t p_t V_down[t]) . P_V^T = sum_t p_t (V_down[t] . P_V^T);
+ * orthonormality of the bases is not needed for this.
+ * L == 0 gives out = 0.  Rows at or beyond seq_lens[b] are never read.
+ *
+ *   q            : bf16 [B][Hq][d]
+ *   P_K, P_V     : bf16 [Hkv][d][rK], [Hkv][d][rV]
+ *   k_lat, v_lat : bf16 [B][Hkv][L_max][rK], [B][Hkv][L_max][rV]
+ *   seq_lens     : int32 [B] on the device, each in [0, max_seq_len]
+ *   out          : bf16 [B][Hq][d] (written)
+ *   workspace    : device scratch of at least workspace_bytes >=
+ *                  stief_decode_workspace_bytes(B, Hq, Hkv, rV, max_seq_len)
+ *                  bytes; its contents on entry do not matter
+ *   max_seq_len  : host-side upper bound of seq_lens (<= L_max); sizes the grid
+ *   num_splits   : 0 = automatic, otherwise the number of KV splits per sequence
+ *                  (1 .. stief_decode_max_splits(max_seq_len))
+ *
+ * Two kernels run on `stream`: the split kernel (query projection, scores,
+ * online softmax, latent value mix) and the combine kernel (log-sum-exp merge of
+ * the splits and up-projection with P_V^T), the second launched as a
+ * programmatic dependent of the first.
+ * Returns STIEF_OK or an argument error (nothing launched).
+ */
+STIEF_API stief_status stief_decode_attention(const uint16_t* q, const uint16_t* P_K,
+                                    const uint16_t* P_V, const uint16_t* k_lat,
+                                    const uint16_t* v_lat, const int32_t* seq_lens,
+                                    uint16_t* out, void* workspace, size_t workspace_bytes,
+                                    int B, int Hq, int Hkv, int d, int rK, int rV, int L_max,
+                                    int max_seq_len, int num_splits,
+                                    uint32_t* dev_status, stief_stream_t stream);
+
+/*
+ * stief_read_device_status -- synchronises `stream`, copies the device status
+ * word to *value, and returns STIEF_OK if it is zero, STIEF_ERR_DEVICE_STATUS
+ * if not, STIEF_ERR_CUDA if the copy failed, STIEF_ERR_INVALID_ARG for NULLs.
+ */
+STIEF_API stief_status stief_read_device_status(const uint32_t* dev_status, uint32_t* value,
+                                      stief_stream_t stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+STIEF_API const char* stief_status_string(stief_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* STIEF_H */

@@ -1,0 +1,128 @@
+"""The C-ABI library on the host: it loads, exports every declared symbol, and its
+argument checks and planning functions behave (no CUDA call is made here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import decode_attention_stief_b200 as stief
+from decode_attention_stief_b200 import build as stief_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "stief.h")
+
+OK, INVALID, ALIGN, CAPACITY, WORKSPACE = 0, 1, 2, 3, 4
+
+
+@pytest.fixture(scope="module")
+def lib():
+    stief_build.build_library()
+    return stief.library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(stief_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for required in ("stief_compress_append", "stief_decode_attention",
+                     "stief_decode_workspace_bytes", "stief_read_device_status",
+                     "stief_status_string"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, f"not exported: {missing}"
+
+
+def test_only_declared_symbols_are_exported():
+    out = os.popen(f"nm -D --defined-only {stief.library_path()}").read()
+    exported = set(re.findall(r"\b(stief_[a-z_0-9]+)\b", out))
+    assert exported <= set(declared_functions()), exported - set(declared_functions())
+
+
+def test_status_strings(lib):
+    for code, name in stief.STATUS.items():
+        assert stief.stief_status_string(code) == name
+    assert stief.stief_status_string(99) == "STIEF_ERR_UNKNOWN"
+
+
+FAKE = 0x10000  # an aligned non-null address; never dereferenced by argument checking
+
+
+def _decode(lib, **kw):
+    a = dict(q=FAKE, P_K=FAKE, P_V=FAKE, k_lat=FAKE, v_lat=FAKE, seq_lens=FAKE, out=FAKE,
+             ws=FAKE, ws_bytes=1 << 40, B=1, Hq=32, Hkv=8, d=128, rK=64, rV=64, L_max=1024,
+             max_seq_len=1024, num_splits=0)
+    a.update(kw)
+    return lib.stief_decode_attention(a["q"], a["P_K"], a["P_V"], a["k_lat"], a["v_lat"],
+                                      a["seq_lens"], a["out"], a["ws"], a["ws_bytes"], a["B"],
+                                      a["Hq"], a["Hkv"], a["d"], a["rK"], a["rV"], a["L_max"],
+                                      a["max_seq_len"], a["num_splits"], None, None)
+
+
+def _compress(lib, **kw):
+    a = dict(k=FAKE, v=FAKE, P_K=FAKE, P_V=FAKE, kl=FAKE, vl=FAKE, sl=FAKE, B=1, Hkv=8, T=1,
+             d=128, rK=64, rV=64, L_max=1024)
+    a.update(kw)
+    return lib.stief_compress_append(a["k"], a["v"], a["P_K"], a["P_V"], a["kl"], a["vl"],
+                                     a["sl"], a["B"], a["Hkv"], a["T"], a["d"], a["rK"],
+                                     a["rV"], a["L_max"], None, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), INVALID), (dict(out=None), INVALID), (dict(seq_lens=None), INVALID),
+    (dict(d=64), INVALID), (dict(rK=8), INVALID), (dict(rV=72), INVALID), (dict(rK=144), INVALID),
+    (dict(Hq=30), INVALID), (dict(B=0), INVALID), (dict(Hkv=0), INVALID),
+    (dict(Hq=8 * 65, Hkv=8), INVALID), (dict(num_splits=-1), INVALID),
+    (dict(num_splits=9), INVALID),  # max for 1024 tokens is 8
+    (dict(max_seq_len=2048), CAPACITY), (dict(max_seq_len=-1), INVALID),
+    (dict(q=FAKE + 8), ALIGN), (dict(k_lat=FAKE + 2), ALIGN), (dict(out=FAKE + 4), ALIGN),
+    (dict(ws=None), WORKSPACE), (dict(ws_bytes=16), WORKSPACE),
+])
+def test_decode_argument_errors(lib, kw, code):
+    assert _decode(lib, **kw) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(k=None), INVALID), (dict(sl=None), INVALID), (dict(d=96), INVALID),
+    (dict(rK=24), INVALID), (dict(T=-1), INVALID), (dict(B=0), INVALID),
+    (dict(T=2048), CAPACITY), (dict(kl=FAKE + 4), ALIGN), (dict(P_V=FAKE + 8), ALIGN),
+    (dict(T=0), OK),  # nothing to do: returns before any CUDA call
+])
+def test_compress_argument_errors(lib, kw, code):
+    assert _compress(lib, **kw) == code
+
+
+def test_split_planning():
+    assert stief.stief_decode_max_splits(0) == 1
+    assert stief.stief_decode_max_splits(128) == 1
+    assert stief.stief_decode_max_splits(129) == 2
+    assert stief.stief_decode_max_splits(10 ** 9) == 512
+    assert stief.stief_decode_max_splits(-1) == 0
+    # one split CTA per SM: 8 KV heads at batch 1 on 148 SMs -> 18 splits
+    assert stief.stief_decode_auto_splits(1, 32, 8, 32768, 148) == 18
+    assert stief.stief_decode_auto_splits(1, 32, 8, 131072, 148) == 18
+    assert stief.stief_decode_auto_splits(1, 4, 1, 1024, 148) == 8     # capped by the length
+    assert stief.stief_decode_auto_splits(16, 32, 8, 8192, 148) == 1
+    assert stief.stief_decode_auto_splits(64, 32, 8, 4096, 148) == 1
+    assert stief.stief_decode_auto_splits(1, 64, 2, 32768, 148) == 18   # G=32 -> 4 sub-groups
+    assert stief.stief_decode_auto_splits(1, 16, 1, 32768, 148) == 74   # G=16 -> 2 sub-groups
+    for B in (1, 2, 5, 64):
+        for L in (1, 100, 5000, 200000):
+            s = stief.stief_decode_auto_splits(B, 32, 8, L, 148)
+            assert 1 <= s <= stief.stief_decode_max_splits(L)
+            assert s == 1 or B * 8 * s <= 148
+
+
+def test_workspace_bytes():
+    # [B * Hkv * qsub * G_T * splits] partial states of (rV + 2) floats
+    assert stief.stief_decode_workspace_bytes(1, 32, 8, 64, 32768) == 32 * 256 * 66 * 4
+    assert stief.stief_decode_workspace_bytes(2, 24, 8, 48, 100) == 2 * 8 * 4 * 1 * 50 * 4
+    assert stief.stief_decode_workspace_bytes(1, 32, 8, 72, 100) == 0
+    assert stief.stief_decode_workspace_bytes(1, 30, 8, 64, 100) == 0

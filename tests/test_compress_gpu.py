@@ -1,0 +1,139 @@
+"""Compress/append parity: stief_compress_append (CUDA, through the C ABI) against the oracle.
+
+The latent must equal the oracle's round-to-nearest-even bf16 value of the exact
+product, up to one bf16 ulp (fp32 accumulation can sit on the other side of a
+rounding boundary); cache indexing and lengths must be bit-exact.
+"""
+import numpy as np
+import pytest
+import torch
+
+import decode_attention_stief_b200 as stief
+import oracle
+import stief_inputs as si
+from gpu_util import (assert_decode_close, bf16_ulp, f64, gpu_decode, oracle_decode)
+
+pytestmark = pytest.mark.gpu
+
+CANARY_K = 0x7FC1  # a quiet-NaN bf16 pattern: any stray write changes it
+CANARY_V = 0xFFC3
+
+
+def _s16(pattern: int) -> int:
+    """A 16-bit pattern as the signed int16 value with the same bits."""
+    return int(np.uint16(pattern).view(np.int16))
+
+
+def _cache(B, Hkv, L_max, r, pattern):
+    return torch.full((B, Hkv, L_max, r), _s16(pattern), dtype=torch.int16).view(torch.bfloat16)
+
+
+def _run_append(k_new, v_new, P_K, P_V, k_lat, v_lat, lens, expect_status=0):
+    dev = torch.device("cuda")
+    args = [x.to(dev).contiguous() for x in (k_new, v_new, P_K, P_V, k_lat, v_lat)]
+    lens_t = torch.as_tensor(np.asarray(lens, np.int32)).to(dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stief.stief_compress_append(*args, lens_t, dev_status=status)
+    st = stief.stief_read_device_status(status)
+    assert st == expect_status, f"device status {st:#x}"
+    return args[4].cpu(), args[5].cpu(), lens_t.cpu().numpy()
+
+
+def _check_latent(got_bits: torch.Tensor, want: np.ndarray):
+    g = f64(got_bits)
+    diff = np.abs(g - want)
+    assert np.all(diff <= bf16_ulp(want)), f"max diff {diff.max()}"
+    return float(np.mean(g == want))
+
+
+@pytest.mark.parametrize("T", [1, 3, 8, 9, 40, 200])
+@pytest.mark.parametrize("rK,rV", [(64, 64), (32, 48), (16, 128), (96, 112)])
+def test_append_matches_oracle(T, rK, rV):
+    B, Hkv, d, L_max = 2, 3, 128, 260
+    seed = 10 * T + rK
+    k_new, v_new = si.full_kv(seed, B, Hkv, T, d)
+    P_K, P_V = si.bases_bf16(seed, Hkv, d, rK, rV)
+    lens = [5, 60]
+    k_lat = _cache(B, Hkv, L_max, rK, CANARY_K)
+    v_lat = _cache(B, Hkv, L_max, rV, CANARY_V)
+    gk, gv, glens = _run_append(k_new, v_new, P_K, P_V, k_lat, v_lat, lens)
+    assert glens.tolist() == [L + T for L in lens]
+    for b, L in enumerate(lens):
+        for h in range(Hkv):
+            wk = oracle.project(f64(k_new[b, h]), f64(P_K[h]))
+            wv = oracle.project(f64(v_new[b, h]), f64(P_V[h]))
+            exact_k = _check_latent(gk[b, h, L:L + T], wk)
+            exact_v = _check_latent(gv[b, h, L:L + T], wv)
+            assert exact_k > 0.98 and exact_v > 0.98
+            keep = np.ones(L_max, bool)
+            keep[L:L + T] = False
+            assert torch.all(gk[b, h, keep].view(torch.int16) == _s16(CANARY_K))
+            assert torch.all(gv[b, h, keep].view(torch.int16) == _s16(CANARY_V))
+
+
+def test_identity_basis_is_bit_exact():
+    B, Hkv, T, d, r, L_max = 1, 2, 37, 128, 48, 64
+    k_new, v_new = si.full_kv(3, B, Hkv, T, d)
+    P = torch.zeros((Hkv, d, r))
+    P[:, torch.arange(r), torch.arange(r)] = 1.0
+    P = P.to(torch.bfloat16)
+    gk, gv, _ = _run_append(k_new, v_new, P, P, _cache(B, Hkv, L_max, r, 0),
+                            _cache(B, Hkv, L_max, r, 0), [0])
+    assert torch.equal(gk[:, :, :T], k_new[..., :r])
+    assert torch.equal(gv[:, :, :T], v_new[..., :r])
+
+
+def test_capacity_overflow_leaves_sequence_untouched():
+    B, Hkv, T, d, r, L_max = 3, 2, 3, 128, 32, 10
+    k_new, v_new = si.full_kv(4, B, Hkv, T, d)
+    P_K, P_V = si.bases_bf16(4, Hkv, d, r, r)
+    lens = [0, 7, 8]                 # the second fits exactly, the third overflows
+    k_lat = _cache(B, Hkv, L_max, r, CANARY_K)
+    v_lat = _cache(B, Hkv, L_max, r, CANARY_K)
+    gk, gv, glens = _run_append(k_new, v_new, P_K, P_V, k_lat, v_lat, lens,
+                                expect_status=stief.DEV_CAPACITY_OVERFLOW)
+    assert glens.tolist() == [3, 10, 8]
+    assert torch.all(gk[2].view(torch.int16) == _s16(CANARY_K))
+    assert torch.all(gv[2].view(torch.int16) == _s16(CANARY_K))
+    _, _, olens, nbad = oracle.compress_append(f64(k_new), f64(v_new), f64(P_K), f64(P_V),
+                                               f64(k_lat), f64(v_lat), lens)
+    assert nbad == 1 and olens.tolist() == glens.tolist()
+
+
+def test_negative_length_is_reported():
+    B, Hkv, T, d, r, L_max = 2, 1, 2, 128, 16, 8
+    k_new, v_new = si.full_kv(5, B, Hkv, T, d)
+    P_K, P_V = si.bases_bf16(5, Hkv, d, r, r)
+    gk, gv, glens = _run_append(k_new, v_new, P_K, P_V, _cache(B, Hkv, L_max, r, CANARY_K),
+                                _cache(B, Hkv, L_max, r, CANARY_K), [-1, 0],
+                                expect_status=stief.DEV_BAD_LENGTH)
+    assert glens.tolist() == [-1, 2]
+    assert torch.all(gk[0].view(torch.int16) == _s16(CANARY_K))
+
+
+def test_append_then_decode_end_to_end():
+    """Prefill chunk + single-token appends, then decode; each side compresses itself."""
+    B, Hq, Hkv, d, rK, rV, L_max = 2, 8, 2, 128, 64, 48, 600
+    seed = 77
+    P_K, P_V = si.bases_bf16(seed, Hkv, d, rK, rV)
+    k_lat = torch.zeros((B, Hkv, L_max, rK), dtype=torch.bfloat16)
+    v_lat = torch.zeros((B, Hkv, L_max, rV), dtype=torch.bfloat16)
+    ok_lat, ov_lat = f64(k_lat), f64(v_lat)
+    lens = np.zeros(B, np.int32)
+    olens = lens.copy()
+    dev = torch.device("cuda")
+    gk, gv = k_lat.to(dev), v_lat.to(dev)
+    glens = torch.as_tensor(lens).to(dev)
+    for step, T in enumerate([500, 1, 1, 1, 7]):
+        k_new, v_new = si.full_kv(seed + step, B, Hkv, T, d)
+        stief.stief_compress_append(k_new.to(dev), v_new.to(dev), P_K.to(dev), P_V.to(dev),
+                                    gk, gv, glens)
+        ok_lat, ov_lat, olens, nbad = oracle.compress_append(
+            f64(k_new), f64(v_new), f64(P_K), f64(P_V), ok_lat, ov_lat, olens)
+        assert nbad == 0
+    torch.cuda.synchronize()
+    assert glens.cpu().numpy().tolist() == olens.tolist() == [510, 510]
+    q = si.queries(seed, B, Hq, d)
+    got = gpu_decode(q, P_K, P_V, gk, gv, olens)
+    want = oracle.decode(f64(q), f64(P_K), f64(P_V), ok_lat, ov_lat, olens)
+    assert_decode_close(got, want)
