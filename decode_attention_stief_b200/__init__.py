@@ -15,6 +15,7 @@ from ._binding import (  # noqa: F401
     library_path,
     stief_compress_append,
     stief_decode_attention,
+    stief_decode_attention_noalloc,
     stief_decode_auto_splits,
     stief_decode_max_splits,
     stief_decode_workspace_bytes,

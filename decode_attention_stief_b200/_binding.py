@@ -73,6 +73,8 @@ def library() -> ctypes.CDLL:
             lib.stief_decode_max_splits.argtypes = [_i]
             lib.stief_decode_auto_splits.restype = _i
             lib.stief_decode_auto_splits.argtypes = [_i] * 5
+            lib.stief_decode_attention_noalloc.restype = _i
+            lib.stief_decode_attention_noalloc.argtypes = [vp] * 7 + [_i] * 9 + [vp, vp]
             lib.stief_read_device_status.restype = _i
             lib.stief_read_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32), vp]
             lib.stief_status_string.restype = ctypes.c_char_p
@@ -206,6 +208,41 @@ def stief_decode_attention(q: torch.Tensor, P_K: torch.Tensor, P_V: torch.Tensor
                                             rV, L_max, int(max_seq_len), int(num_splits),
                                             _opt_status(dev_status), _stream_ptr(stream))
     _check("stief_decode_attention", code)
+    return out
+
+
+def stief_decode_attention_noalloc(q: torch.Tensor, P_K: torch.Tensor, P_V: torch.Tensor,
+                                   k_lat: torch.Tensor, v_lat: torch.Tensor,
+                                   seq_lens: torch.Tensor, out: torch.Tensor, max_seq_len: int,
+                                   num_splits: int = 0, dev_status: Optional[torch.Tensor] = None,
+                                   stream=None) -> torch.Tensor:
+    """stief_decode_attention for callers that cannot allocate: no workspace argument.
+
+    The library keeps the split partial states in its own fixed 8 MiB device array
+    (one per GPU); calls that overlap on the GPU race on it.  Raises StiefError
+    (STIEF_ERR_WORKSPACE) when the sizes need more than that.
+    """
+    pq = _dev(q, "q", torch.bfloat16, 3)
+    ppk = _dev(P_K, "P_K", torch.bfloat16, 3)
+    ppv = _dev(P_V, "P_V", torch.bfloat16, 3)
+    pkl = _dev(k_lat, "k_lat", torch.bfloat16, 4)
+    pvl = _dev(v_lat, "v_lat", torch.bfloat16, 4)
+    psl = _dev(seq_lens, "seq_lens", torch.int32, 1)
+    po = _dev(out, "out", torch.bfloat16, 3)
+    B, Hq, d = q.shape
+    Hkv, _, rK = P_K.shape
+    rV = P_V.shape[2]
+    L_max = k_lat.shape[2]
+    if tuple(P_K.shape) != (Hkv, d, rK) or tuple(P_V.shape) != (Hkv, d, rV) \
+            or tuple(k_lat.shape) != (B, Hkv, L_max, rK) \
+            or tuple(v_lat.shape) != (B, Hkv, L_max, rV) or seq_lens.shape[0] != B \
+            or tuple(out.shape) != (B, Hq, d):
+        raise ValueError("stief_decode_attention_noalloc: inconsistent shapes")
+    code = library().stief_decode_attention_noalloc(pq, ppk, ppv, pkl, pvl, psl, po, B, Hq, Hkv,
+                                                    d, rK, rV, L_max, int(max_seq_len),
+                                                    int(num_splits), _opt_status(dev_status),
+                                                    _stream_ptr(stream))
+    _check("stief_decode_attention_noalloc", code)
     return out
 
 

@@ -171,6 +171,34 @@ STIEF_API stief_status stief_decode_attention(const uint16_t* q, const uint16_t*
                                     uint32_t* dev_status, stief_stream_t stream);
 
 /*
+ * stief_decode_attention_noalloc -- stief_decode_attention without a workspace
+ * argument and without any device allocation.  The paper has no counterpart: this
+ * is a deployment variant for callers that cannot obtain device memory when they
+ * decode (a serving engine whose KV-cache pool already holds nearly all of HBM, a
+ * host framework whose operator interface passes only inputs and outputs, a
+ * latency-critical loop that must not call cudaMalloc).
+ *
+ * Same arguments, meaning and result as stief_decode_attention, minus
+ * workspace / workspace_bytes.  The per-split partial states live in a fixed 8 MiB
+ * array of device memory owned by the library (one per GPU that loads it, held
+ * until the process exits).  Sizes whose partial states, for the split count
+ * actually used, exceed 8 MiB -- B*Hkv*ceil(G/G_T)*G_T*splits*(rV+2)*4 bytes with
+ * G = Hq/Hkv and G_T the smallest of 1, 2, 4, 8 that is >= min(G, 8) -- return
+ * STIEF_ERR_WORKSPACE and launch nothing.  The first call on each device looks up
+ * the array's device address (cudaGetSymbolAddress) with that device current; make
+ * that first call before any stream capture.  All calls on a device share the
+ * array: calls whose kernels overlap on the GPU race on it, so the caller must
+ * order them (e.g. one stream).  The array keeps the last call's contents; no part
+ * of it needs clearing between calls.  Calls no cudaMalloc, cudaFree or
+ * allocating library routine.
+ */
+STIEF_API stief_status stief_decode_attention_noalloc(
+    const uint16_t* q, const uint16_t* P_K, const uint16_t* P_V, const uint16_t* k_lat,
+    const uint16_t* v_lat, const int32_t* seq_lens, uint16_t* out, int B, int Hq, int Hkv, int d,
+    int rK, int rV, int L_max, int max_seq_len, int num_splits, uint32_t* dev_status,
+    stief_stream_t stream);
+
+/*
  * stief_read_device_status -- synchronises `stream`, copies the device status
  * word to *value, and returns STIEF_OK if it is zero, STIEF_ERR_DEVICE_STATUS
  * if not, STIEF_ERR_CUDA if the copy failed, STIEF_ERR_INVALID_ARG for NULLs.
