@@ -205,7 +205,7 @@ def run_gpu(args, w: si.Workload):
                                         lay.seq_lens, dev_status=status)
             stief.stief_decode_attention(q_i, lay.P_K, lay.P_V, lay.k_lat, lay.v_lat,
                                          lay.seq_lens, out[li], lay.ws, max_seq_len=L_max,
-                                         dev_status=status)
+                                         num_splits=args.splits, dev_status=status)
 
     def barrier():
         if ws_n > 1:
@@ -263,7 +263,7 @@ def run_gpu(args, w: si.Workload):
         dec_evs[j][0].record(stream)
         stief.stief_decode_attention(q[0], lay0.P_K, lay0.P_V, lay0.k_lat, lay0.v_lat,
                                      lay0.seq_lens, out[0], lay0.ws, max_seq_len=L_max,
-                                     dev_status=status)
+                                     num_splits=args.splits, dev_status=status)
         dec_evs[j][1].record(stream)
     torch.cuda.synchronize()
     dec_ms = sorted(a.elapsed_time(b) for a, b in dec_evs)
@@ -338,7 +338,7 @@ def run_gpu(args, w: si.Workload):
         },
         "hbm_gbs_step": round(step_bytes / (ms_per_step / 1e3) / 1e9, 1),
         "roofline": {
-            "kernel": "stief_decode_attention (split + combine kernels)",
+            "kernel": "stief_decode_kernel (stief_decode_attention)",
             "bound": "hbm",
             "achieved": round(achieved, 1),
             "peak": peak,
@@ -352,7 +352,7 @@ def run_gpu(args, w: si.Workload):
         },
         "e2e": {"value": round(tokens_per_step / (e2e_ms / 1e3), 2), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 4 * len(layers) * K,
+        "gpu_launches": 3 * len(layers) * K,  # compress rows, length update, decode
         "clocks": clocks,
         "wall_s_timed_region": round(t_wall, 3),
     }
@@ -469,12 +469,20 @@ def main():
     ap.add_argument("--decode-iters", type=int, default=50)
     ap.add_argument("--cpu-seconds", type=float, default=30.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="diagnostics: run only the first N layers of the workload")
+    ap.add_argument("--splits", type=int, default=0,
+                    help="diagnostics: force the decode split count (0 = automatic)")
     ap.add_argument("--clock-window", type=float, default=0.6,
                     help="seconds of untimed decode load before the timed region")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     w = si.WORKLOADS[args.workload]
+    if args.layers > 0:
+        import dataclasses
+        w = dataclasses.replace(w, layers=min(args.layers, w.layers),
+                                ranks=w.ranks[:args.layers] if w.ranks else None)
     if args.impl == "reference":
         run_reference(args, w)
     else:

@@ -136,11 +136,15 @@ def stief_decode_workspace_bytes(B: int, Hq: int, Hkv: int, rV: int, max_seq_len
 
 def workspace_for(B: int, Hq: int, Hkv: int, rV: int, max_seq_len: int,
                   device="cuda") -> torch.Tensor:
-    """A uint8 device tensor of stief_decode_workspace_bytes(...) bytes."""
+    """A zero-filled uint8 device tensor of stief_decode_workspace_bytes(...) bytes.
+
+    Zero-filled once here; every completed decode call leaves its ticket counters at
+    zero, so the tensor can be reused for any later call on the same stream.
+    """
     n = stief_decode_workspace_bytes(B, Hq, Hkv, rV, max_seq_len)
     if n == 0:
         raise ValueError("invalid sizes for the decode workspace")
-    return torch.empty(n, dtype=torch.uint8, device=device)
+    return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
 def stief_compress_append(k_new: torch.Tensor, v_new: torch.Tensor, P_K: torch.Tensor,

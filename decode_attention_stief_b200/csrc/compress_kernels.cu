@@ -7,7 +7,7 @@
 // [seq_lens[b], seq_lens[b] + T) of the latent cache; then seq_lens[b] += T.
 //
 // Kernels:
-//   stief_compress_rows_kernel  -- CUDA-core projection, grid (ceil(T/TT), Hkv, B);
+//   stief_compress_rows_kernel  -- CUDA-core projection, grid (ceil(T/TT), 2 Hkv, B);
 //                                  used for decode-sized appends (small T)
 //   stief_seq_lens_kernel       -- the length update, launched as a programmatic
 //                                  dependent of the projection so that it runs
@@ -20,67 +20,91 @@
 
 namespace stief {
 
-constexpr int kRowsPerCta = 8;  // TT: new rows handled by one CTA of the CUDA-core path
+constexpr int kRowsPerCta = 8;  // new rows per CTA of the CUDA-core path (T > 1)
+constexpr int kSmallThreads = 256;
 
-// Shared memory: P_K[h] (d x rK), P_V[h] (d x rV), then TT rows of k and of v.
-__global__ void __launch_bounds__(256) stief_compress_rows_kernel(const CompressArgs a) {
+__device__ __forceinline__ float2 fma2c(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+
+// CUDA-core projection of up to TT new rows of one (sequence, KV head, K or V).
+// grid (ceil(T/TT), Hkv * 2, B); blockIdx.y = 2 * head + (0: keys, 1: values).
+// The basis and the rows arrive by bulk copy; thread = (column pair, slice of d);
+// slices are summed through shared memory.
+template <int TT>
+__global__ void __launch_bounds__(kSmallThreads) stief_compress_rows_kernel(const CompressArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x;
-  const int h = blockIdx.y, b = blockIdx.z;
-  const int d = a.d, rK = a.rK, rV = a.rV, T = a.T;
-  const int r0 = blockIdx.x * kRowsPerCta;
-  const int nrows = min(kRowsPerCta, T - r0);
+  const int h = blockIdx.y >> 1;
+  const bool is_v = blockIdx.y & 1;
+  const int b = blockIdx.z;
+  const int d = a.d, T = a.T;
+  const int r = is_v ? a.rV : a.rK;
+  const int r0 = blockIdx.x * TT;
+  const int nrows = min(TT, T - r0);
+  const uint16_t* P = (is_v ? a.P_V : a.P_K) + (size_t)h * d * r;
+  const uint16_t* X = (is_v ? a.v_new : a.k_new) + (((size_t)b * a.Hkv + h) * T + r0) * d;
 
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem);
+  uint16_t* ps = reinterpret_cast<uint16_t*>(smem + 128);
+  uint16_t* xs = ps + d * r;
+  float2* red = reinterpret_cast<float2*>(xs + TT * d);
+
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_barrier_init();
+    const uint32_t pb = 2u * d * r, xb = 2u * nrows * d;
+    mbar_arrive_expect_tx(bar, pb + xb);
+    bulk_g2s(ps, P, pb, bar);
+    bulk_g2s(xs, X, xb, bar);
+  }
   pdl_launch_dependents();
 
   const int Lb = a.seq_lens[b];
-  if (Lb < 0 || Lb > a.L_max) {
-    if (tid == 0 && blockIdx.x == 0 && h == 0) report(a.dev_status, STIEF_DEV_BAD_LENGTH);
-    return;
+  const bool bad = Lb < 0 || Lb > a.L_max;
+  const bool full = !bad && (long long)Lb + T > a.L_max;
+  if (tid == 0 && blockIdx.x == 0 && blockIdx.y == 0) {
+    if (bad) report(a.dev_status, STIEF_DEV_BAD_LENGTH);
+    if (full) report(a.dev_status, STIEF_DEV_CAPACITY_OVERFLOW);
   }
-  if ((long long)Lb + T > a.L_max) {
-    if (tid == 0 && blockIdx.x == 0 && h == 0) report(a.dev_status, STIEF_DEV_CAPACITY_OVERFLOW);
-    return;
-  }
+  __syncthreads();  // barrier initialised before anyone waits on it
+  const bool ok = mbar_wait_bounded(bar, 0, a.dev_status);
+  if (bad || full || !ok) return;  // the copies have landed (or the wait gave up)
 
-  uint16_t* pk = reinterpret_cast<uint16_t*>(smem);
-  uint16_t* pv = pk + d * rK;
-  uint16_t* xk = pv + d * rV;
-  uint16_t* xv = xk + kRowsPerCta * d;
-  {
-    const uint4* src = reinterpret_cast<const uint4*>(a.P_K + (size_t)h * d * rK);
-    uint4* dst = reinterpret_cast<uint4*>(pk);
-    for (int i = tid; i < d * rK / 8; i += blockDim.x) dst[i] = src[i];
-    src = reinterpret_cast<const uint4*>(a.P_V + (size_t)h * d * rV);
-    dst = reinterpret_cast<uint4*>(pv);
-    for (int i = tid; i < d * rV / 8; i += blockDim.x) dst[i] = src[i];
-    const size_t row0 = (((size_t)b * a.Hkv + h) * T + r0) * d;
-    src = reinterpret_cast<const uint4*>(a.k_new + row0);
-    dst = reinterpret_cast<uint4*>(xk);
-    for (int i = tid; i < nrows * d / 8; i += blockDim.x) dst[i] = src[i];
-    src = reinterpret_cast<const uint4*>(a.v_new + row0);
-    dst = reinterpret_cast<uint4*>(xv);
-    for (int i = tid; i < nrows * d / 8; i += blockDim.x) dst[i] = src[i];
+  const int pairs = r / 2;  // 8 .. 64
+  int slices = 1;           // a power of two with pairs * slices <= 256 (so it divides d)
+  while (pairs * slices * 2 <= kSmallThreads) slices *= 2;
+  const int rows_per_slice = d / slices;
+  const int cp = tid % pairs, sl = tid / pairs;
+  const bool active = sl < slices;
+  const uint32_t* P2 = reinterpret_cast<const uint32_t*>(ps);
+  float2 acc[TT];
+#pragma unroll
+  for (int t = 0; t < TT; ++t) acc[t] = make_float2(0.f, 0.f);
+  for (int i = sl * rows_per_slice; active && i < (sl + 1) * rows_per_slice; ++i) {
+    const uint32_t pw = P2[i * pairs + cp];
+    const float2 pf = make_float2(bf16lo(pw), bf16hi(pw));
+#pragma unroll
+    for (int t = 0; t < TT; ++t) {
+      const float xv = bf16_to_f32(xs[t * d + i]);
+      acc[t] = fma2c(make_float2(xv, xv), pf, acc[t]);
+    }
+  }
+  if (active) {
+#pragma unroll
+    for (int t = 0; t < TT; ++t) red[(sl * TT + t) * pairs + cp] = acc[t];
   }
   __syncthreads();
-
-  // threads [0, 128): key column tid; threads [128, 256): value column tid - 128
-  const bool is_v = tid >= 128;
-  const int c = is_v ? tid - 128 : tid;
-  const int r = is_v ? rV : rK;
-  if (c >= r) return;
-  const uint16_t* P = is_v ? pv : pk;
-  const uint16_t* X = is_v ? xv : xk;
-  float acc[kRowsPerCta];
-#pragma unroll
-  for (int t = 0; t < kRowsPerCta; ++t) acc[t] = 0.f;
-  for (int i = 0; i < d; ++i) {
-    const float p = bf16_to_f32(P[i * r + c]);
-#pragma unroll
-    for (int t = 0; t < kRowsPerCta; ++t) acc[t] = fmaf(bf16_to_f32(X[t * d + i]), p, acc[t]);
+  uint32_t* dst = reinterpret_cast<uint32_t*>((is_v ? a.v_lat : a.k_lat) +
+                                              (((size_t)b * a.Hkv + h) * a.L_max + Lb + r0) * r);
+  for (int o = tid; o < nrows * pairs; o += kSmallThreads) {
+    const int t = o / pairs, c2 = o - t * pairs;
+    float2 sum = make_float2(0.f, 0.f);
+    for (int s2 = 0; s2 < slices; ++s2) {
+      const float2 v = red[(s2 * TT + t) * pairs + c2];
+      sum.x += v.x;
+      sum.y += v.y;
+    }
+    dst[(size_t)t * pairs + c2] = pack_bf16x2_rn(sum.x, sum.y);
   }
-  uint16_t* dst = (is_v ? a.v_lat : a.k_lat) + (((size_t)b * a.Hkv + h) * a.L_max + Lb + r0) * r;
-  for (int t = 0; t < nrows; ++t) dst[(size_t)t * r + c] = f32_to_bf16_rn(acc[t]);
 }
 
 __global__ void __launch_bounds__(256) stief_seq_lens_kernel(int32_t* seq_lens, int B, int T,
@@ -105,14 +129,20 @@ static cudaError_t launch_seq_lens(const CompressArgs& a, cudaStream_t stream) {
   return cudaLaunchKernelEx(&cfg, stief_seq_lens_kernel, a.seq_lens, a.B, a.T, a.L_max);
 }
 
-cudaError_t launch_compress(const CompressArgs& a, cudaStream_t stream) {
-  const uint32_t smem = 2u * (a.d * (a.rK + a.rV) + 2 * kRowsPerCta * a.d);
-  cudaError_t e = cudaFuncSetAttribute(stief_compress_rows_kernel,
+template <int TT>
+static cudaError_t launch_rows(const CompressArgs& a, cudaStream_t stream) {
+  const int rmax = a.rK > a.rV ? a.rK : a.rV;
+  const uint32_t smem = 128u + 2u * a.d * rmax + 2u * TT * a.d + 8u * TT * kSmallThreads;
+  cudaError_t e = cudaFuncSetAttribute(stief_compress_rows_kernel<TT>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((a.T + kRowsPerCta - 1) / kRowsPerCta, a.Hkv, a.B);
-  stief_compress_rows_kernel<<<grid, 256, smem, stream>>>(a);
-  e = cudaGetLastError();
+  dim3 grid((a.T + TT - 1) / TT, a.Hkv * 2, a.B);
+  stief_compress_rows_kernel<TT><<<grid, kSmallThreads, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_compress(const CompressArgs& a, cudaStream_t stream) {
+  cudaError_t e = (a.T == 1) ? launch_rows<1>(a, stream) : launch_rows<kRowsPerCta>(a, stream);
   if (e != cudaSuccess) return e;
   return launch_seq_lens(a, stream);
 }

@@ -3,29 +3,41 @@
 //
 // Operation (StiefAttention technical summary, "Mecanismo Central" item 5): keys
 // and values are stored as K_down = K P_K, V_down = V P_V and attention runs over
-// the reconstructions K~ = K_down P_K^T, V~ = V_down P_V^T.  The kernels never
-// form K~ or V~; they use the equal products
+// the reconstructions K~ = K_down P_K^T, V~ = V_down P_V^T.  The kernel never forms
+// K~ or V~; it uses the equal products
 //     s_t = (q P_K) . K_down[t] / sqrt(d)          (query projected once per CTA)
 //     o   = (sum_t softmax(s)_t V_down[t]) P_V^T   (up-projection after the mix)
 // so the HBM stream is the bf16 latent cache, read once per KV head.
 //
-// Kernel 1 (stief_decode_split_kernel), grid (splits, Hkv * qsub, B):
-//   one CTA serves up to G_T query heads of one KV head over one token range.
-//   - q~ = q . P_K * log2(e)/sqrt(d) in fp32 (shared memory, padded chunk-major)
-//   - every warp streams its own 32-token tiles of K_down and V_down through a
-//     private ring of shared-memory stages filled by 1-D bulk copies (TMA engine)
-//     that complete on per-stage mbarriers; no CTA-wide barrier in the loop
-//   - scores: one lane per token; each lane walks the 16-byte chunks of its row
-//     in a lane-rotated order so the 8 lanes of a shared-memory phase hit 8
-//     different bank groups, while q~ is read with broadcasts
-//   - online softmax in the log2 domain with lazy rescaling: accumulators are
-//     rescaled only when a score exceeds the running reference by more than 8
-//     (so every weight stays <= 2^8 in fp32)
-//   - latent value mix: r_V/8 lanes per token, 8 values per lane, fp32 FMA
-//   - partial (m, l, o~[r_V]) per (query head, split) written to the workspace
-// Kernel 2 (stief_decode_combine_kernel), grid (Hkv * qsub, B), launched as a
-// programmatic dependent: log-sum-exp merge of the splits, division by the sum,
-// up-projection o~ . P_V^T, bf16 store.
+// One kernel, stief_decode_kernel<G_T, NP>, grid (splits, Hkv * qsub, B).  A CTA
+// serves up to G_T query heads of one KV head ("unit") over one token range, with
+// NP warp pairs (2*NP warps):
+//   - prologue: q and P_K[h] arrive by bulk copy; q~ = q . P_K * log2(e)/sqrt(d)
+//     in fp32, stored padded chunk-major
+//   - streaming: pair i owns two rings of shared-memory stages holding the keys
+//     and the values of 32-token tiles, each slot filled by a 1-D bulk copy (TMA
+//     engine, L2 evict-first) that completes on the slot's mbarrier, and works
+//     through tiles i, i + NP, ...  Its K-warp computes the scores -- one lane
+//     per token; key tiles land by 2-D TMA tensor copies in 64/32/16-column pieces
+//     with the matching 128/64/32-byte swizzle, so all lanes read the same logical
+//     chunk at once without bank conflicts and q~ is read as warp-wide broadcasts;
+//     packed fp32x2 FMAs -- and the online
+//     softmax in the log2
+//     domain with lazy rescaling (accumulators rescaled only when a score passes
+//     the running reference by more than 8, so every weight stays <= 2^8).  It
+//     hands the weights (as duplicated pairs) and any rescale factors to its
+//     V-warp through a double buffer guarded by two mbarriers.  The V-warp mixes
+//     the latent values (r_V/8 lanes per token, packed FMAs).  Key and value halves
+//     of a tile live in separate rings, each refilled by its own consumer as soon
+//     as it is done, which keeps more bytes in flight.  Splitting the roles halves the registers each warp needs, so twice
+//     as many warps hide shared-memory and FMA latency.  No CTA-wide barrier in
+//     the loop.
+//   - epilogue: merge the pairs; with one split the CTA finishes the unit itself;
+//     otherwise it stores its partial state (o~[r_V], m, l) and takes a ticket,
+//     and the last CTA of the unit merges all splits (log-sum-exp) -- that CTA
+//     resets the ticket counter, so the workspace counters stay zero between
+//     calls.  P_V arrives by bulk copy into the freed stage region while the
+//     merge runs; then o = o~ . P_V^T, bf16 out.
 #include <cfloat>
 #include <cmath>
 #include <cstdint>
@@ -35,7 +47,7 @@
 
 namespace stief {
 
-constexpr int kTile = 32;            // tokens per warp tile
+constexpr int kTile = 32;            // tokens per pair tile
 constexpr float kRescaleTau = 8.0f;  // lazy-rescale threshold (log2 units)
 
 __device__ __forceinline__ float ex2(float x) {
@@ -55,82 +67,132 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// Shared-memory carve-up of the split kernel (byte offsets from the dynamic base).
-struct SplitSmem {
-  uint32_t bars;    // (NW * nstage + 1) mbarriers
-  uint32_t q;       // G_T x d bf16 query rows
-  uint32_t pk;      // d x rK bf16 basis
-  uint32_t qt;      // (rK/8) chunks x (G_T*8 + 4) fp32 projected, scaled queries
-  uint32_t p;       // NW x 32 x G_T fp32 softmax weights of the current tile
-  uint32_t ml;      // NW x G_T x 2 fp32 per-warp (m, l)
-  uint32_t region;  // stage buffers, reused for the cross-warp reduction
-  uint32_t total;
-};
+__device__ __forceinline__ float2 f2(float x, float y) { return make_float2(x, y); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+// the 4 bf16 pairs of a 16-byte chunk, widened exactly to fp32 pairs
+__device__ __forceinline__ void unpack8(const uint4 w, float2 (&v)[4]) {
+  v[0] = f2(bf16lo(w.x), bf16hi(w.x));
+  v[1] = f2(bf16lo(w.y), bf16hi(w.y));
+  v[2] = f2(bf16lo(w.z), bf16hi(w.z));
+  v[3] = f2(bf16lo(w.w), bf16hi(w.w));
+}
+
+__device__ __forceinline__ float4 ldcg4(const float* p) {
+  return __ldcg(reinterpret_cast<const float4*>(p));
+}
 
 __host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
-__host__ __device__ inline SplitSmem split_smem_layout(int NW, int nstage, int G_T, int d, int rK,
-                                                       int rV) {
-  SplitSmem s;
+// Shared-memory carve-up (byte offsets from the dynamic base).
+struct DecodeSmem {
+  uint32_t bars;     // NP*ns K-stage, NP*ns V-stage, NP*2 weights-full, NP*2 weights-empty, 1 setup
+  uint32_t q;        // G_T x d bf16 query rows
+  uint32_t qt;       // (rK/8) chunks x G_T x 8 fp32 projected, scaled queries
+  uint32_t fbuf;     // NP x 2 x (G_T factors + flag): rescale handed from K- to V-warp
+  uint32_t ml;       // NP x G_T x (m, l); then G_T x (M, L, rescale); then a flag
+  uint32_t scratch;  // P_K (prologue); NP x 2 x 32 x G_T x 2 fp32 weights; o~ (epilogue)
+  uint32_t region;   // per pair a K ring then a V ring of stages; later reduction /
+                     // split-merge staging + P_V at its end
+  uint32_t region_bytes;
+  uint32_t pv;       // offset of P_V inside the region (epilogue)
+  uint32_t total;
+};
+
+__host__ __device__ inline DecodeSmem decode_smem_layout(int NP, int nstage, int G_T, int d, int rK,
+                                                         int rV) {
+  DecodeSmem s;
   uint32_t off = 0;
   s.bars = off;
-  off = align_up(off + 8u * (NW * nstage + 1), 128);
+  off = align_up(off + 8u * (2 * NP * nstage + 4 * NP + 1), 128);
   s.q = off;
   off = align_up(off + 2u * G_T * d, 128);
-  s.pk = off;
-  off = align_up(off + 2u * d * rK, 128);
   s.qt = off;
-  off = align_up(off + 4u * (rK / 8) * (G_T * 8 + 4), 128);
-  s.p = off;
-  off = align_up(off + 4u * NW * kTile * G_T, 128);
+  off = align_up(off + 4u * rK * G_T, 128);
+  s.fbuf = off;
+  off = align_up(off + 4u * NP * 2 * (G_T + 1), 128);
   s.ml = off;
-  off = align_up(off + 8u * NW * G_T, 128);
+  off = align_up(off + 4u * (2 * NP * G_T + 3 * G_T + 4), 128);
+  s.scratch = off;
+  const uint32_t pbuf = 8u * NP * 2 * kTile * G_T;
+  const uint32_t pk = 2u * d * rK;
+  const uint32_t ob = 4u * G_T * rV;
+  uint32_t sb = pbuf > pk ? pbuf : pk;
+  sb = sb > ob ? sb : ob;
+  off = align_up(off + sb, 128);
+  off = align_up(off, 1024);  // swizzled key slots need 1 KiB alignment
   s.region = off;
-  const uint32_t stage = (uint32_t)NW * nstage * kTile * (rK + rV) * 2u;
-  const uint32_t red = (uint32_t)NW * 32u * G_T * 8u * 4u;
-  off = align_up(off + (stage > red ? stage : red), 128);
+  const uint32_t stage = (uint32_t)NP * nstage * kTile * (rK + rV) * 2u;
+  const uint32_t red = (uint32_t)NP * 32u * G_T * 8u * 4u;
+  const uint32_t pvb = align_up(2u * d * rV, 128);
+  const uint32_t need = align_up(red, 128) + pvb;
+  s.region_bytes = align_up(stage > need ? stage : need, 128);
+  s.pv = s.region_bytes - pvb;
+  off += s.region_bytes;
   s.total = off;
   return s;
 }
 
-template <int G_T, int NW>
-__global__ void __launch_bounds__(NW * 32, 1) stief_decode_split_kernel(const DecodeArgs a) {
-  extern __shared__ __align__(128) uint8_t smem[];
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Warp-specialised: warps [0, NP) are K-warps (scores, softmax), warps [NP, 2NP) are
+// V-warps (value mix, stage refills).  K-warp i and V-warp i form pair i, which owns a
+// ring of `nstage` stages and processes the CTA's tiles i, i + NP, i + 2NP, ...
+template <int G_T, int NP>
+__global__ void __launch_bounds__(NP * 64, 1) stief_decode_kernel(const __grid_constant__ DecodeArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  constexpr int NT = NP * 64;
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
+  const bool is_k = warp < NP;
+  const int pair = is_k ? warp : warp - NP;
   const int s_idx = blockIdx.x;                 // split
   const int kvh = blockIdx.y / a.qsub;          // KV head
   const int qs = blockIdx.y - kvh * a.qsub;     // query sub-group of that head
   const int b = blockIdx.z;
   const int d = a.d, rK = a.rK, rV = a.rV, S = a.S;
-  const int nstage = a.nstage;
+  const int ns = a.nstage;
   const int h0 = kvh * a.G + qs * G_T;          // first query head of this CTA
   const int gcount = min(G_T, a.G - qs * G_T);  // valid query heads here
+  const size_t unit = ((size_t)b * a.Hkv + kvh) * a.qsub + qs;
 
-  const SplitSmem L = split_smem_layout(NW, nstage, G_T, d, rK, rV);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
-  uint64_t* setup_bar = bars + NW * nstage;
-  const uint32_t tile_bytes = (uint32_t)kTile * (rK + rV) * 2u;
-  uint8_t* my_stages = smem + L.region + (size_t)warp * nstage * tile_bytes;
+  const DecodeSmem L = decode_smem_layout(NP, ns, G_T, d, rK, rV);
+  uint64_t* kfull = reinterpret_cast<uint64_t*>(smem + L.bars);  // [NP][ns]
+  uint64_t* vfull = kfull + NP * ns;                              // [NP][ns]
+  uint64_t* pfull = vfull + NP * ns;                              // [NP][2]
+  uint64_t* pempty = pfull + NP * 2;                             // [NP][2]
+  uint64_t* setup_bar = pempty + NP * 2;  // phase 0: q + P_K, phase 1: P_V
+  // a key slot holds the tile's column pieces (64/32/16 wide) as the TMA engine writes
+  // them, each with its shared-memory swizzle; a value slot holds the rows unchanged
+  const uint32_t kt_bytes = (uint32_t)kTile * rK * 2u, vt_bytes = (uint32_t)kTile * rV * 2u;
+  uint8_t* my_kring = smem + L.region + (size_t)pair * ns * (kt_bytes + vt_bytes);
+  uint8_t* my_vring = my_kring + (size_t)ns * kt_bytes;
+  float* ml = reinterpret_cast<float*>(smem + L.ml);
+  float* fin = ml + 2 * NP * G_T;                    // [G_T] M, [G_T] L, [G_T] rescale
+  int* flag = reinterpret_cast<int*>(fin + 3 * G_T);
+  float* fbuf = reinterpret_cast<float*>(smem + L.fbuf) + pair * 2 * (G_T + 1);
 
+  if ((smem_u32(smem + L.region) & 1023u) != 0) {  // swizzle patterns assume 1 KiB alignment
+    if (tid == 0) report(a.dev_status, STIEF_DEV_SMEM_ALIGN);
+    return;
+  }
   if (tid == 0) {
-    for (int i = 0; i < NW * nstage + 1; ++i) mbar_init(&bars[i], 1);
+    for (int i = 0; i < 2 * NP * ns + 4 * NP + 1; ++i) mbar_init(&kfull[i], 1);
     fence_barrier_init();
   }
   __syncthreads();
 
-  // Query rows and the key basis: independent of any earlier kernel in this call.
+  // q and the bases were written before this kernel started (it is not launched
+  // as a programmatic dependent), so they may be fetched before the wait below.
   if (tid == 0) {
     const uint32_t qbytes = 2u * gcount * d;
     const uint32_t pbytes = 2u * d * rK;
     mbar_arrive_expect_tx(setup_bar, qbytes + pbytes);
     bulk_g2s(smem + L.q, a.q + ((size_t)b * a.Hq + h0) * d, qbytes, setup_bar);
-    bulk_g2s(smem + L.pk, a.P_K + (size_t)kvh * d * rK, pbytes, setup_bar);
+    bulk_g2s(smem + L.scratch, a.P_K + (size_t)kvh * d * rK, pbytes, setup_bar);
   }
-  pdl_launch_dependents();
-
-  // Everything below may read what the preceding kernel in the stream wrote.
   pdl_wait();
 
   int Lb = a.seq_lens[b];
@@ -142,214 +204,321 @@ __global__ void __launch_bounds__(NW * 32, 1) stief_decode_split_kernel(const De
   const int t0 = min(Lb, s_idx * chunk);
   const int t1 = min(Lb, t0 + chunk);
   const int n_tiles = (t1 - t0 + kTile - 1) / kTile;
-  const int my_tiles = warp < n_tiles ? (n_tiles - warp + NW - 1) / NW : 0;
+  const int my_tiles = pair < n_tiles ? (n_tiles - pair + NP - 1) / NP : 0;
 
   const size_t head_row0 = ((size_t)b * a.Hkv + kvh) * a.L_max;
-  const uint16_t* kbase_g = a.k_lat + head_row0 * rK;
   const uint16_t* vbase_g = a.v_lat + head_row0 * rV;
-  const uint64_t policy = l2_policy_evict_first();
 
-  auto issue = [&](int k) {  // tile k of this warp into stage k % nstage (lane 0 only)
-    const int j = warp + k * NW;
-    const int tok0 = t0 + j * kTile;
-    const int n = min(kTile, t1 - tok0);
-    uint8_t* st = my_stages + (size_t)(k % nstage) * tile_bytes;
-    uint64_t* bar = &bars[warp * nstage + (k % nstage)];
-    const uint32_t kb = (uint32_t)n * rK * 2u, vb = (uint32_t)n * rV * 2u;
-    mbar_arrive_expect_tx(bar, kb + vb);
-    bulk_g2s_hint(st, kbase_g + (size_t)tok0 * rK, kb, bar, policy);
-    bulk_g2s_hint(st + (size_t)kTile * rK * 2, vbase_g + (size_t)tok0 * rV, vb, bar, policy);
+  // K and V halves of a tile travel separately, so each ring slot is refilled as soon
+  // as its own consumer is done with it (the K-warp after its scores, the V-warp
+  // after its mix): more bytes stay in flight per SM.
+  // K and V halves of a tile travel separately, so each ring slot is refilled as soon
+  // as its own consumer is done with it (the K-warp after its scores, the V-warp
+  // after its mix).  Keys arrive by 2-D TMA tensor copies (swizzled), values by
+  // one 1-D bulk copy.
+  auto issue_k = [&](int k, uint64_t policy) {  // lane 0 of the K-warp
+    const int tok0 = t0 + (pair + k * NP) * kTile;
+    uint8_t* dst = my_kring + (size_t)(k % ns) * kt_bytes;
+    uint64_t* bar = &kfull[pair * ns + (k % ns)];
+    // whole 32-row boxes land (rows past the tile are masked out of the softmax)
+    mbar_arrive_expect_tx(bar, kt_bytes);
+    const int y = (int)(head_row0 + tok0);
+    for (int p = 0; p < a.npieces; ++p)
+      tma_load_2d(dst + a.kp[p].smem_off, &a.tmk[a.kp[p].map], a.kp[p].x, y, bar, policy);
   };
-  if (lane == 0) {
-    const int pre = min(nstage, my_tiles);
-    for (int k = 0; k < pre; ++k) issue(k);
+  auto issue_v = [&](int k, uint64_t policy) {  // lane 0 of the V-warp
+    const int tok0 = t0 + (pair + k * NP) * kTile;
+    const int n = min(kTile, t1 - tok0);
+    uint64_t* bar = &vfull[pair * ns + (k % ns)];
+    const uint32_t bytes = (uint32_t)n * rV * 2u;
+    mbar_arrive_expect_tx(bar, bytes);
+    bulk_g2s_hint(my_vring + (size_t)(k % ns) * vt_bytes, vbase_g + (size_t)tok0 * rV, bytes, bar,
+                  policy);
+  };
+  int issued = min(ns, my_tiles);  // tiles this warp has requested
+  {
+    const uint64_t policy = l2_policy_evict_first();
+    if (lane == 0)
+      for (int k = 0; k < issued; ++k) {
+        if (is_k) issue_k(k, policy);
+        else issue_v(k, policy);
+      }
   }
 
-  // ---- q~ = q . P_K, scaled into the log2 domain ---------------------------------
+  // ---- q~ = q . P_K, scaled into the log2 domain -----------------------------------
+  // thread = (query head g, column pair cp, half of d); the two halves of a pair sit in
+  // adjacent lanes and are added with one shuffle.
   bool ok = mbar_wait_bounded(setup_bar, 0, a.dev_status);
-  const float qscale = a.qscale;
   {
-    const int RK = rK / 8;
-    const int qstride = G_T * 8 + 4;  // floats per chunk row (odd multiple of 16 bytes)
-    const uint16_t* qs_ = reinterpret_cast<const uint16_t*>(smem + L.q);
-    const uint16_t* pk = reinterpret_cast<const uint16_t*>(smem + L.pk);
+    const int qstride = G_T * 8;  // floats per chunk row
+    const uint32_t* q2 = reinterpret_cast<const uint32_t*>(smem + L.q);
+    const uint32_t* pk2 = reinterpret_cast<const uint32_t*>(smem + L.scratch);
     float* qt = reinterpret_cast<float*>(smem + L.qt);
-    for (int idx = tid; idx < G_T * rK; idx += NW * 32) {
-      const int g = idx / rK, c = idx - g * rK;
-      float acc = 0.f;
-      if (ok && g < gcount) {
-        const uint16_t* qrow = qs_ + g * d;
-#pragma unroll 8
-        for (int i = 0; i < d; ++i) acc = fmaf(bf16_to_f32(qrow[i]), bf16_to_f32(pk[i * rK + c]), acc);
+    const int half = rK / 2;  // column pairs
+    const int outs = G_T * half;
+    const int parts = NT >= 2 * outs ? 2 : 1;
+    const int total = outs * parts;
+    const int total_r = (total + 31) & ~31;  // whole warps take part in the shuffle
+    const int span = (d / 2) / parts;
+    for (int idx = tid; idx < total_r; idx += NT) {
+      const bool act = idx < total;
+      const int o = idx / parts, part = idx - o * parts;
+      const int g = o / half, cp = o - g * half;
+      float2 acc = f2(0.f, 0.f);
+      if (act && ok && g < gcount) {
+        const uint32_t* qrow = q2 + g * (d / 2);
+#pragma unroll 4
+        for (int i2 = part * span; i2 < (part + 1) * span; ++i2) {
+          const uint32_t qq = qrow[i2];  // q[2*i2], q[2*i2+1]
+          const uint32_t pa = pk2[(2 * i2) * half + cp];
+          const uint32_t pb = pk2[(2 * i2 + 1) * half + cp];
+          const float q0 = bf16lo(qq), q1 = bf16hi(qq);
+          acc = fma2(f2(q0, q0), f2(bf16lo(pa), bf16hi(pa)), acc);
+          acc = fma2(f2(q1, q1), f2(bf16lo(pb), bf16hi(pb)), acc);
+        }
       }
-      qt[(c >> 3) * qstride + g * 8 + (c & 7)] = acc * qscale;
+      if (parts == 2) {
+        acc.x += __shfl_xor_sync(0xffffffffu, acc.x, 1);
+        acc.y += __shfl_xor_sync(0xffffffffu, acc.y, 1);
+      }
+      if (act && part == 0) {
+        const int c = 2 * cp;
+        float* dst = qt + (c >> 3) * qstride + g * 8 + (c & 7);
+        dst[0] = acc.x * a.qscale;
+        dst[1] = acc.y * a.qscale;
+      }
     }
-    (void)RK;
   }
   __syncthreads();
 
-  // ---- streaming loop (per warp) ----------------------------------------------------
-  const int RK = rK >> 3;
+  // ---- streaming ------------------------------------------------------------------------
   const int RV = rV >> 3;
-  const int sh = (RK & 7) == 0 ? 0 : ((RK & 3) == 0 ? 1 : 2);
-  const int delta = (lane & 7) >> sh;
-  const uint32_t qstride_b = (uint32_t)(G_T * 8 + 4) * 4u;
-  const uint32_t qt_addr = smem_u32(smem + L.qt);
-  float* p_tile = reinterpret_cast<float*>(smem + L.p) + warp * kTile * G_T;
-  const uint32_t p_addr = smem_u32(p_tile);
   const int TPW = 32 / RV;            // tokens per value step
   const int vslot = lane / RV;
   const int vchunk = lane - vslot * RV;
   const bool vactive = vslot < TPW;
+  float* pbuf = reinterpret_cast<float*>(smem + L.scratch) + pair * 2 * kTile * G_T * 2;
 
-  float m_ref[G_T], l_lane[G_T], acc[G_T][8];
+  float m_ref[G_T], l_lane[G_T];
+  float2 acc[G_T][4];
 #pragma unroll
   for (int g = 0; g < G_T; ++g) {
     m_ref[g] = -INFINITY;
     l_lane[g] = 0.f;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[g][e] = 0.f;
+    for (int e = 0; e < 4; ++e) acc[g][e] = f2(0.f, 0.f);
   }
+  int consumed = 0;
 
-  int k_done = 0;
-  for (int k = 0; k < my_tiles && ok; ++k) {
-    const int stg = k % nstage;
-    if (!mbar_wait_bounded(&bars[warp * nstage + stg], (uint32_t)((k / nstage) & 1), a.dev_status)) {
-      ok = false;
-      break;
-    }
-    k_done = k + 1;
-    const int tok0 = t0 + (warp + k * NW) * kTile;
-    const int n = min(kTile, t1 - tok0);
-    uint8_t* st = my_stages + (size_t)stg * tile_bytes;
-    const uint32_t kst = smem_u32(st);
-    const uint32_t vst = kst + (uint32_t)kTile * rK * 2u;
+  if (is_k) {
+    const uint32_t qstride_b = (uint32_t)G_T * 32u;
+    const uint32_t qt_addr = smem_u32(smem + L.qt);
+    const uint64_t policy = l2_policy_evict_first();
+    for (int k = 0; k < my_tiles && ok; ++k) {
+      const int stg = k % ns;
+      if (!mbar_wait_bounded(&kfull[pair * ns + stg], (uint32_t)((k / ns) & 1), a.dev_status)) {
+        ok = false;
+        break;
+      }
+      const int tok0 = t0 + (pair + k * NP) * kTile;
+      const int n = min(kTile, t1 - tok0);
+      const uint32_t kst = smem_u32(my_kring + (size_t)stg * kt_bytes);
 
-    // scores: lane = token
-    float s[G_T];
-#pragma unroll
-    for (int g = 0; g < G_T; ++g) s[g] = 0.f;
-    {
-      const uint32_t krow = kst + (uint32_t)lane * rK * 2u;
-      int c = delta;
-      for (int jj = 0; jj < RK; ++jj) {
-        const uint4 kv = lds128(krow + c * 16u);
-        const float k0 = bf16lo(kv.x), k1 = bf16hi(kv.x), k2 = bf16lo(kv.y), k3 = bf16hi(kv.y);
-        const float k4 = bf16lo(kv.z), k5 = bf16hi(kv.z), k6 = bf16lo(kv.w), k7 = bf16hi(kv.w);
-        const uint32_t qa = qt_addr + (uint32_t)c * qstride_b;
+      // scores: lane = token; two chunks per iteration (RK is even); q~ chunk reads are
+      // warp-wide broadcasts
+      float s[G_T];
+      {
+        float2 sa[G_T], sb[G_T];
 #pragma unroll
         for (int g = 0; g < G_T; ++g) {
-          const float4 x = lds128f(qa + g * 32u);
-          const float4 y = lds128f(qa + g * 32u + 16u);
-          float t = s[g];
-          t = fmaf(x.x, k0, t);
-          t = fmaf(x.y, k1, t);
-          t = fmaf(x.z, k2, t);
-          t = fmaf(x.w, k3, t);
-          t = fmaf(y.x, k4, t);
-          t = fmaf(y.y, k5, t);
-          t = fmaf(y.z, k6, t);
-          t = fmaf(y.w, k7, t);
-          s[g] = t;
+          sa[g] = f2(0.f, 0.f);
+          sb[g] = f2(0.f, 0.f);
         }
-        c = (c + 1 == RK) ? 0 : c + 1;
+        for (int p = 0; p < a.npieces; ++p) {
+          const int w = a.kp[p].width;
+          // row `lane` of this piece; its 16-byte chunk c sits at position c ^ sw
+          const uint32_t prow = kst + (uint32_t)a.kp[p].smem_off + (uint32_t)lane * w * 2u;
+          const int sw = w == 64 ? (lane & 7) : (w == 32 ? ((lane >> 1) & 3) : ((lane >> 2) & 1));
+          const uint32_t q0 = qt_addr + (uint32_t)(a.kp[p].x >> 3) * qstride_b;
+          for (int cc = 0; cc < (w >> 3); cc += 2) {
+            float2 ka[4], kb[4];
+            unpack8(lds128(prow + (uint32_t)((cc ^ sw) << 4)), ka);
+            unpack8(lds128(prow + (uint32_t)(((cc + 1) ^ sw) << 4)), kb);
+            const uint32_t qa = q0 + (uint32_t)cc * qstride_b;
+            const uint32_t qb = qa + qstride_b;
+#pragma unroll
+            for (int g = 0; g < G_T; ++g) {
+              const float4 xa = lds128f(qa + g * 32u), ya = lds128f(qa + g * 32u + 16u);
+              const float4 xb = lds128f(qb + g * 32u), yb = lds128f(qb + g * 32u + 16u);
+              sa[g] = fma2(f2(xa.x, xa.y), ka[0], sa[g]);
+              sb[g] = fma2(f2(xb.x, xb.y), kb[0], sb[g]);
+              sa[g] = fma2(f2(xa.z, xa.w), ka[1], sa[g]);
+              sb[g] = fma2(f2(xb.z, xb.w), kb[1], sb[g]);
+              sa[g] = fma2(f2(ya.x, ya.y), ka[2], sa[g]);
+              sb[g] = fma2(f2(yb.x, yb.y), kb[2], sb[g]);
+              sa[g] = fma2(f2(ya.z, ya.w), ka[3], sa[g]);
+              sb[g] = fma2(f2(yb.z, yb.w), kb[3], sb[g]);
+            }
+          }
+        }
+#pragma unroll
+        for (int g = 0; g < G_T; ++g) s[g] = (sa[g].x + sa[g].y) + (sb[g].x + sb[g].y);
+      }
+      // the key slot is free: request the keys of tile k + ns
+      __syncwarp();
+      consumed = k + 1;
+      if (k + ns < my_tiles) {
+        if (lane == 0) issue_k(k + ns, policy);
+        issued = k + ns + 1;
+      }
+
+      // online softmax (log2 domain), lazy rescale; factors go to the V-warp
+      const bool valid = lane < n;
+      float pw[G_T], fac[G_T];
+      bool rescaled = false;
+#pragma unroll
+      for (int g = 0; g < G_T; ++g) {
+        const float sg = valid ? s[g] : -INFINITY;
+        fac[g] = 1.f;
+        if (__any_sync(0xffffffffu, sg > m_ref[g] + kRescaleTau)) {
+          const float m_new = fmaxf(m_ref[g], warp_max(sg));
+          fac[g] = ex2(m_ref[g] - m_new);  // 0 when m_ref was -inf
+          l_lane[g] *= fac[g];
+          m_ref[g] = m_new;
+          rescaled = true;
+        }
+        pw[g] = valid ? ex2(sg - m_ref[g]) : 0.f;
+        l_lane[g] += pw[g];
+      }
+      const int pb = k & 1;
+      if (k >= 2 && !mbar_wait_bounded(&pempty[pair * 2 + pb], (uint32_t)(((k >> 1) - 1) & 1),
+                                       a.dev_status)) {
+        ok = false;
+        break;
+      }
+      float* pt = pbuf + pb * kTile * G_T * 2;
+      if constexpr (G_T >= 2) {
+#pragma unroll
+        for (int g2 = 0; g2 < G_T; g2 += 2)
+          *reinterpret_cast<float4*>(pt + (lane * G_T + g2) * 2) =
+              make_float4(pw[g2], pw[g2], pw[g2 + 1], pw[g2 + 1]);
+      } else {
+        *reinterpret_cast<float2*>(pt + lane * 2) = f2(pw[0], pw[0]);
+      }
+      if (lane == 0) {
+        float* fb = fbuf + pb * (G_T + 1);
+#pragma unroll
+        for (int g = 0; g < G_T; ++g) fb[g] = fac[g];
+        fb[G_T] = rescaled ? 1.f : 0.f;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&pfull[pair * 2 + pb]);
+    }
+  } else {
+    const uint64_t policy = l2_policy_evict_first();
+    for (int k = 0; k < my_tiles && ok; ++k) {
+      const int pb = k & 1;
+      if (!mbar_wait_bounded(&pfull[pair * 2 + pb], (uint32_t)((k >> 1) & 1), a.dev_status) ||
+          !mbar_wait_bounded(&vfull[pair * ns + (k % ns)], (uint32_t)((k / ns) & 1), a.dev_status)) {
+        ok = false;
+        break;
+      }
+      const int tok0 = t0 + (pair + k * NP) * kTile;
+      const int n = min(kTile, t1 - tok0);
+      const uint32_t vst = smem_u32(my_vring + (size_t)(k % ns) * vt_bytes);
+      const float* fb = fbuf + pb * (G_T + 1);
+      if (fb[G_T] != 0.f) {
+#pragma unroll
+        for (int g = 0; g < G_T; ++g) {
+          const float f = fb[g];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[g][e] = f2(acc[g][e].x * f, acc[g][e].y * f);
+        }
+      }
+      const uint32_t p_addr = smem_u32(pbuf + pb * kTile * G_T * 2);
+      if (vactive) {
+#pragma unroll 2
+        for (int t = vslot; t < n; t += TPW) {
+          float2 v[4];
+          unpack8(lds128(vst + (uint32_t)t * rV * 2u + vchunk * 16u), v);
+          float2 pp[G_T];
+          if constexpr (G_T >= 2) {
+#pragma unroll
+            for (int g2 = 0; g2 < G_T; g2 += 2) {
+              const float4 x = lds128f(p_addr + (uint32_t)(t * G_T + g2) * 8u);
+              pp[g2] = f2(x.x, x.y);
+              pp[g2 + 1] = f2(x.z, x.w);
+            }
+          } else {
+            const float4 x = lds128f(p_addr + (uint32_t)(t & ~1) * 8u);
+            pp[0] = (t & 1) ? f2(x.z, x.w) : f2(x.x, x.y);
+          }
+#pragma unroll
+          for (int g = 0; g < G_T; ++g)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[g][e] = fma2(pp[g], v[e], acc[g][e]);
+        }
+      }
+      __syncwarp();
+      consumed = k + 1;
+      if (lane == 0) {
+        mbar_arrive(&pempty[pair * 2 + pb]);
+        if (k + ns < my_tiles) {
+          issue_v(k + ns, policy);
+          issued = k + ns + 1;
+        }
       }
     }
-    // online softmax (log2 domain), lazy rescale
-    const bool valid = lane < n;
-    float pw_own[G_T];
+  }
+  // copies that were requested but not consumed (only after a timed-out wait) must land
+  // before the region is reused or the CTA exits
+  if (lane == 0)
+    for (int k = consumed; k < issued; ++k)
+      mbar_wait_bounded(&(is_k ? kfull : vfull)[pair * ns + (k % ns)], (uint32_t)((k / ns) & 1),
+                        nullptr);
+
+  // ---- merge the pairs ---------------------------------------------------------------
+  if (is_k) {
 #pragma unroll
     for (int g = 0; g < G_T; ++g) {
-      const float sg = valid ? s[g] : -INFINITY;
-      if (__any_sync(0xffffffffu, sg > m_ref[g] + kRescaleTau)) {
-        const float m_new = fmaxf(m_ref[g], warp_max(sg));
-        const float f = ex2(m_ref[g] - m_new);  // 0 when m_ref was -inf
-        l_lane[g] *= f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[g][e] *= f;
-        m_ref[g] = m_new;
-      }
-      pw_own[g] = valid ? ex2(sg - m_ref[g]) : 0.f;
-      l_lane[g] += pw_own[g];
-    }
-    if constexpr (G_T >= 4) {
-#pragma unroll
-      for (int g4 = 0; g4 < G_T; g4 += 4)
-        *reinterpret_cast<float4*>(p_tile + lane * G_T + g4) =
-            make_float4(pw_own[g4], pw_own[g4 + 1], pw_own[g4 + 2], pw_own[g4 + 3]);
-    } else {
-#pragma unroll
-      for (int g = 0; g < G_T; ++g) p_tile[lane * G_T + g] = pw_own[g];
-    }
-    __syncwarp();
-
-    // latent value mix: RV lanes per token
-    if (vactive) {
-      for (int t = vslot; t < n; t += TPW) {
-        const uint4 vv = lds128(vst + (uint32_t)t * rV * 2u + vchunk * 16u);
-        float v[8] = {bf16lo(vv.x), bf16hi(vv.x), bf16lo(vv.y), bf16hi(vv.y),
-                      bf16lo(vv.z), bf16hi(vv.z), bf16lo(vv.w), bf16hi(vv.w)};
-        float pw[G_T];
-        if constexpr (G_T >= 4) {
-#pragma unroll
-          for (int g4 = 0; g4 < G_T; g4 += 4) {
-            const float4 pp = lds128f(p_addr + (uint32_t)(t * G_T + g4) * 4u);
-            pw[g4] = pp.x;
-            pw[g4 + 1] = pp.y;
-            pw[g4 + 2] = pp.z;
-            pw[g4 + 3] = pp.w;
-          }
-        } else {
-#pragma unroll
-          for (int g = 0; g < G_T; ++g) pw[g] = p_tile[t * G_T + g];
-        }
-#pragma unroll
-        for (int g = 0; g < G_T; ++g)
-#pragma unroll
-          for (int e = 0; e < 8; ++e) acc[g][e] = fmaf(pw[g], v[e], acc[g][e]);
+      const float lw = warp_sum(l_lane[g]);
+      if (lane == 0) {
+        ml[(pair * G_T + g) * 2 + 0] = m_ref[g];
+        ml[(pair * G_T + g) * 2 + 1] = lw;
       }
     }
-    __syncwarp();
-    if (lane == 0 && k + nstage < my_tiles) issue(k + nstage);
   }
-
-  // After a timed-out wait: give the copies still in flight a bounded chance to land
-  // before this CTA's shared memory is released.
-  if (!ok && lane == 0) {
-    for (int k = k_done; k < min(my_tiles, k_done + nstage); ++k)
-      mbar_wait_bounded(&bars[warp * nstage + (k % nstage)], (uint32_t)((k / nstage) & 1), nullptr);
-    if (warp == 0) mbar_wait_bounded(setup_bar, 0, nullptr);
+  __syncthreads();  // every pair is done with its stages: the region becomes the reduction buffer
+  // P_V for the up-projection: needed here when this CTA finishes the unit itself
+  if (tid == 0 && S == 1) {
+    fence_proxy_async_smem();
+    const uint32_t vbytes = 2u * d * rV;
+    mbar_arrive_expect_tx(setup_bar, vbytes);
+    bulk_g2s(smem + L.region + L.pv, a.P_V + (size_t)kvh * d * rV, vbytes, setup_bar);
   }
-
-  // ---- cross-warp merge --------------------------------------------------------------
-  float* ml = reinterpret_cast<float*>(smem + L.ml);
-#pragma unroll
-  for (int g = 0; g < G_T; ++g) {
-    const float lw = warp_sum(l_lane[g]);
-    if (lane == 0) {
-      ml[(warp * G_T + g) * 2 + 0] = m_ref[g];
-      ml[(warp * G_T + g) * 2 + 1] = lw;
-    }
-  }
-  __syncthreads();  // every warp is done with its stages: the region becomes the reduction buffer
   float* red = reinterpret_cast<float*>(smem + L.region);
-  {
-    float* mine = red + ((size_t)warp * 32 + lane) * G_T * 8;
+  if (!is_k) {
+    float* mine = red + ((size_t)pair * 32 + lane) * G_T * 8;
 #pragma unroll
     for (int g = 0; g < G_T; ++g)
 #pragma unroll
-      for (int e = 0; e < 8; ++e) mine[g * 8 + e] = vactive ? acc[g][e] : 0.f;
+      for (int e = 0; e < 4; ++e) {
+        mine[g * 8 + 2 * e] = vactive ? acc[g][e].x : 0.f;
+        mine[g * 8 + 2 * e + 1] = vactive ? acc[g][e].y : 0.f;
+      }
   }
   __syncthreads();
 
-  const size_t unit = ((size_t)b * a.Hkv + kvh) * a.qsub + qs;
-  for (int idx = tid; idx < G_T * rV; idx += NW * 32) {
+  float* ot = reinterpret_cast<float*>(smem + L.scratch);  // o~ [G_T][rV] for the up-projection
+  const int part_stride = rV + 4;
+  float* parts = a.ws_part + unit * (size_t)S * G_T * part_stride;  // this unit's S x G_T states
+  for (int idx = tid; idx < G_T * rV; idx += NT) {
     const int g = idx / rV, jj = idx - g * rV;
     const int c = jj >> 3, e = jj & 7;
     float M = -INFINITY;
-    for (int w = 0; w < NW; ++w) M = fmaxf(M, ml[(w * G_T + g) * 2]);
+    for (int w = 0; w < NP; ++w) M = fmaxf(M, ml[(w * G_T + g) * 2]);
     float o = 0.f, lsum = 0.f;
-    for (int w = 0; w < NW; ++w) {
+    for (int w = 0; w < NP; ++w) {
       const float mw = ml[(w * G_T + g) * 2];
       const float sc = (mw == -INFINITY) ? 0.f : ex2(mw - M);
       float part = 0.f;
@@ -358,125 +527,152 @@ __global__ void __launch_bounds__(NW * 32, 1) stief_decode_split_kernel(const De
       o = fmaf(sc, part, o);
       lsum = fmaf(sc, ml[(w * G_T + g) * 2 + 1], lsum);
     }
-    const size_t pi = (unit * S + s_idx) * G_T + g;
-    a.ws_o[pi * rV + jj] = o;
-    if (jj == 0) {
-      a.ws_ml[pi * 2 + 0] = M;
-      a.ws_ml[pi * 2 + 1] = lsum;
-    }
-  }
-}
-
-// Combine the splits and up-project: out[b][h] = bf16( (sum_s w_s o~_s / sum_s w_s l_s) . P_V^T ).
-template <int G_T>
-__global__ void __launch_bounds__(128) stief_decode_combine_kernel(const DecodeArgs a) {
-  __shared__ float ot[G_T][128];
-  const int tid = threadIdx.x;
-  const int kvh = blockIdx.x / a.qsub;
-  const int qs = blockIdx.x - kvh * a.qsub;
-  const int b = blockIdx.y;
-  const int rV = a.rV, S = a.S, d = a.d;
-  const int h0 = kvh * a.G + qs * G_T;
-  const int gcount = min(G_T, a.G - qs * G_T);
-  const size_t unit = ((size_t)b * a.Hkv + kvh) * a.qsub + qs;
-
-  pdl_wait();
-
-  for (int idx = tid; idx < gcount * rV; idx += blockDim.x) {
-    const int g = idx / rV, jj = idx - g * rV;
-    float M = -INFINITY;
-    for (int s = 0; s < S; ++s) M = fmaxf(M, a.ws_ml[((unit * S + s) * G_T + g) * 2]);
-    float o = 0.f, lsum = 0.f;
-    if (M != -INFINITY) {
-      for (int s = 0; s < S; ++s) {
-        const size_t pi = (unit * S + s) * G_T + g;
-        const float ms = a.ws_ml[pi * 2];
-        if (ms == -INFINITY) continue;
-        const float w = ex2(ms - M);
-        lsum = fmaf(w, a.ws_ml[pi * 2 + 1], lsum);
-        o = fmaf(w, a.ws_o[pi * rV + jj], o);
+    if (S == 1) {
+      ot[g * rV + jj] = lsum > 0.f ? o / lsum : 0.f;
+    } else {
+      float* pdst = parts + ((size_t)s_idx * G_T + g) * part_stride;
+      pdst[jj] = o;
+      if (jj == 0) {
+        pdst[rV] = M;
+        pdst[rV + 1] = lsum;
       }
     }
-    ot[g][jj] = lsum > 0.f ? o / lsum : 0.f;
+  }
+
+  if (S > 1) {
+    // publish this split and take a ticket; the last CTA of the unit merges every split
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+      const uint32_t ticket = atomicAdd(a.ws_cnt + unit, 1u);
+      const int last = ticket == (uint32_t)(S - 1);
+      if (last) {
+        a.ws_cnt[unit] = 0u;  // ready for the next call
+        fence_proxy_async_smem();
+        const uint32_t vbytes = 2u * d * rV;
+        mbar_arrive_expect_tx(setup_bar, vbytes);
+        bulk_g2s(smem + L.region + L.pv, a.P_V + (size_t)kvh * d * rV, vbytes, setup_bar);
+      }
+      *flag = last;
+    }
+    __syncthreads();
+    if (!*flag) return;
+    __threadfence();
+    // stage the unit's split states through shared memory (below P_V), a chunk of splits
+    // at a time, accumulating against a running maximum
+    float* stage_p = reinterpret_cast<float*>(smem + L.region);
+    const int per_split = G_T * part_stride;  // floats
+    const int s_chunk = max(1, (int)(L.pv / 4u) / per_split);
+    for (int s0 = 0; s0 < S; s0 += s_chunk) {
+      const int nsp = min(s_chunk, S - s0);
+      const int n4 = nsp * per_split / 4;
+      const float* src = parts + (size_t)s0 * per_split;
+      for (int i = tid; i < n4; i += NT * 4) {
+        float4 x[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (i + u * NT < n4) x[u] = ldcg4(src + 4 * (i + u * NT));
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (i + u * NT < n4) reinterpret_cast<float4*>(stage_p)[i + u * NT] = x[u];
+      }
+      __syncthreads();
+      if (tid < G_T) {
+        const float M_old = (s0 == 0) ? -INFINITY : fin[tid];
+        float M = M_old;
+        for (int s = 0; s < nsp; ++s) M = fmaxf(M, stage_p[(s * G_T + tid) * part_stride + rV]);
+        const float f = (M_old == -INFINITY) ? 0.f : ex2(M_old - M);
+        float lsum = (s0 == 0) ? 0.f : fin[G_T + tid] * f;
+        for (int s = 0; s < nsp; ++s) {
+          const float ms = stage_p[(s * G_T + tid) * part_stride + rV];
+          if (ms != -INFINITY) lsum = fmaf(ex2(ms - M), stage_p[(s * G_T + tid) * part_stride + rV + 1], lsum);
+        }
+        fin[tid] = M;
+        fin[G_T + tid] = lsum;
+        fin[2 * G_T + tid] = f;  // rescale of what was accumulated before this chunk
+      }
+      __syncthreads();
+      const bool final_chunk = s0 + nsp >= S;
+      for (int idx = tid; idx < G_T * rV; idx += NT) {
+        const int g = idx / rV, jj = idx - g * rV;
+        const float M = fin[g];
+        float o = (s0 == 0) ? 0.f : ot[idx] * fin[2 * G_T + g];
+        if (M != -INFINITY)
+          for (int s = 0; s < nsp; ++s) {
+            const float ms = stage_p[(s * G_T + g) * part_stride + rV];
+            if (ms != -INFINITY) o = fmaf(ex2(ms - M), stage_p[(s * G_T + g) * part_stride + jj], o);
+          }
+        if (final_chunk) {
+          const float lsum = fin[G_T + g];
+          o = lsum > 0.f ? o / lsum : 0.f;
+        }
+        ot[idx] = o;
+      }
+      __syncthreads();
+    }
   }
   __syncthreads();
 
-  for (int i = tid; i < d; i += blockDim.x) {
-    const uint4* prow = reinterpret_cast<const uint4*>(a.P_V + ((size_t)kvh * d + i) * rV);
-    float accs[G_T];
-#pragma unroll
-    for (int g = 0; g < G_T; ++g) accs[g] = 0.f;
-    for (int c = 0; c < rV / 8; ++c) {
-      const uint4 pv = prow[c];
-      const float p8[8] = {bf16lo(pv.x), bf16hi(pv.x), bf16lo(pv.y), bf16hi(pv.y),
-                           bf16lo(pv.z), bf16hi(pv.z), bf16lo(pv.w), bf16hi(pv.w)};
-#pragma unroll
-      for (int g = 0; g < G_T; ++g)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) accs[g] = fmaf(ot[g][c * 8 + e], p8[e], accs[g]);
+  // ---- up-projection o = o~ . P_V^T from shared memory, bf16 out --------------------------
+  if (!mbar_wait_bounded(setup_bar, 1, a.dev_status)) return;
+  {
+    const uint32_t pv_addr = smem_u32(smem + L.region + L.pv);
+    const int shv = (RV & 7) == 0 ? 0 : ((RV & 3) == 0 ? 1 : 2);
+    for (int idx = tid; idx < gcount * d; idx += NT) {
+      const int g = idx / d, i = idx - g * d;
+      const uint32_t prow = pv_addr + (uint32_t)i * rV * 2u;
+      const float* og = ot + g * rV;
+      int c = ((i & 7) >> shv) % RV;
+      float2 accv = f2(0.f, 0.f);
+      for (int jj = 0; jj < RV; ++jj) {
+        float2 pv[4];
+        unpack8(lds128(prow + c * 16u), pv);
+        const float4 x = *reinterpret_cast<const float4*>(og + c * 8);
+        const float4 y = *reinterpret_cast<const float4*>(og + c * 8 + 4);
+        accv = fma2(f2(x.x, x.y), pv[0], accv);
+        accv = fma2(f2(x.z, x.w), pv[1], accv);
+        accv = fma2(f2(y.x, y.y), pv[2], accv);
+        accv = fma2(f2(y.z, y.w), pv[3], accv);
+        c = (c + 1 == RV) ? 0 : c + 1;
+      }
+      a.out[((size_t)b * a.Hq + h0 + g) * d + i] = f32_to_bf16_rn(accv.x + accv.y);
     }
-    for (int g = 0; g < gcount; ++g)
-      a.out[((size_t)b * a.Hq + h0 + g) * d + i] = f32_to_bf16_rn(accs[g]);
   }
 }
 
 // ------------------------------------------------------------------------------ launch
 
-template <int G_T, int NW>
-static cudaError_t launch_split(const DecodeArgs& a, cudaStream_t stream, bool pdl) {
-  const SplitSmem L = split_smem_layout(NW, a.nstage, G_T, a.d, a.rK, a.rV);
-  auto kern = stief_decode_split_kernel<G_T, NW>;
+template <int G_T, int NP>
+static cudaError_t launch_t(const DecodeArgs& a, cudaStream_t stream) {
+  const DecodeSmem L = decode_smem_layout(NP, a.nstage, G_T, a.d, a.rK, a.rV);
+  auto kern = stief_decode_kernel<G_T, NP>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.S, a.Hkv * a.qsub, a.B);
-  cfg.blockDim = dim3(NW * 32);
+  cfg.blockDim = dim3(NP * 64);
   cfg.dynamicSmemBytes = L.total;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  attr[0].val.programmaticStreamSerializationAllowed = a.pdl_first ? 1 : 0;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
-template <int G_T>
-static cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t stream) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(a.Hkv * a.qsub, a.B);
-  cfg.blockDim = dim3(128);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, stief_decode_combine_kernel<G_T>, a);
-}
-
-uint32_t decode_split_smem_bytes(int NW, int nstage, int G_T, int d, int rK, int rV) {
-  return split_smem_layout(NW, nstage, G_T, d, rK, rV).total;
+uint32_t decode_smem_bytes(int NP, int nstage, int G_T, int d, int rK, int rV) {
+  return decode_smem_layout(NP, nstage, G_T, d, rK, rV).total;
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
-  cudaError_t e;
-#define STIEF_SPLIT(GT)                                                        \
-  case GT:                                                                     \
-    e = (a.nwarps == 8) ? launch_split<GT, 8>(a, stream, a.pdl_first)          \
-                        : launch_split<GT, 4>(a, stream, a.pdl_first);         \
-    if (e != cudaSuccess) return e;                                            \
-    return launch_combine<GT>(a, stream);
   switch (a.G_T) {
-    STIEF_SPLIT(1)
-    STIEF_SPLIT(2)
-    STIEF_SPLIT(4)
-    STIEF_SPLIT(8)
-    default:
-      return cudaErrorInvalidValue;
+    case 1: return a.npairs == 8 ? launch_t<1, 8>(a, stream) : launch_t<1, 4>(a, stream);
+    case 2: return a.npairs == 8 ? launch_t<2, 8>(a, stream) : launch_t<2, 4>(a, stream);
+    case 4: return a.npairs == 8 ? launch_t<4, 8>(a, stream) : launch_t<4, 4>(a, stream);
+    case 8: return a.npairs == 8 ? launch_t<8, 8>(a, stream) : launch_t<8, 4>(a, stream);
+    default: return cudaErrorInvalidValue;
   }
-#undef STIEF_SPLIT
 }
 
 }  // namespace stief

@@ -6,7 +6,7 @@
 
 #include <cuda_runtime.h>
 
-#include "../../include/stief.h"
+#include "stief.h"
 #include "stief_internal.h"
 
 namespace {
@@ -36,7 +36,8 @@ stief_status device_check() {
 // Common decode shape checks (host only, no CUDA call).
 stief_status check_decode_shape(int B, int Hq, int Hkv, int d, int rK, int rV, int L_max,
                                 int max_seq_len) {
-  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || Hq / Hkv > kMaxGroup) return STIEF_ERR_INVALID_ARG;
+  if (B < 1 || B > 65535 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || Hq / Hkv > kMaxGroup)
+    return STIEF_ERR_INVALID_ARG;
   if (d != kHeadDim || !rank_ok(rK) || !rank_ok(rV)) return STIEF_ERR_INVALID_ARG;
   if (L_max < 1 || max_seq_len < 0) return STIEF_ERR_INVALID_ARG;
   if (max_seq_len > L_max) return STIEF_ERR_CAPACITY;
@@ -87,8 +88,8 @@ size_t stief_decode_workspace_bytes(int B, int Hq, int Hkv, int rV, int max_seq_
   const int G = Hq / Hkv;
   const int G_T = group_tile(G);
   const int qsub = (G + G_T - 1) / G_T;
-  const size_t parts = (size_t)B * Hkv * qsub * G_T * stief_decode_max_splits(max_seq_len);
-  return parts * (size_t)(rV + 2) * sizeof(float);
+  const size_t units = (size_t)B * Hkv * qsub;
+  return stief::decode_ws_bytes(units, G_T, stief_decode_max_splits(max_seq_len), rV);
 }
 
 stief_status stief_compress_append(const uint16_t* k_new, const uint16_t* v_new,
@@ -133,6 +134,7 @@ stief_status stief_decode_attention(const uint16_t* q, const uint16_t* P_K, cons
                                     size_t workspace_bytes, int B, int Hq, int Hkv, int d, int rK,
                                     int rV, int L_max, int max_seq_len, int num_splits,
                                     uint32_t* dev_status, stief_stream_t stream) {
+  // cheap host checks first, so argument errors never touch CUDA
   if (!q || !P_K || !P_V || !k_lat || !v_lat || !seq_lens || !out) return STIEF_ERR_INVALID_ARG;
   stief_status st = check_decode_shape(B, Hq, Hkv, d, rK, rV, L_max, max_seq_len);
   if (st != STIEF_OK) return st;
@@ -143,54 +145,16 @@ stief_status stief_decode_attention(const uint16_t* q, const uint16_t* P_K, cons
     return STIEF_ERR_ALIGNMENT;
   const size_t need = stief_decode_workspace_bytes(B, Hq, Hkv, rV, max_seq_len);
   if (!workspace || workspace_bytes < need) return STIEF_ERR_WORKSPACE;
-  st = device_check();
-  if (st != STIEF_OK) return st;
-
-  int dev = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return STIEF_ERR_CUDA;
 
   stief::DecodeArgs a{};
-  a.q = q;
-  a.P_K = P_K;
-  a.P_V = P_V;
-  a.k_lat = k_lat;
-  a.v_lat = v_lat;
-  a.seq_lens = seq_lens;
-  a.out = out;
-  a.dev_status = dev_status;
-  a.B = B;
-  a.Hq = Hq;
-  a.Hkv = Hkv;
-  a.G = Hq / Hkv;
-  a.G_T = group_tile(a.G);
-  a.qsub = (a.G + a.G_T - 1) / a.G_T;
-  a.d = d;
-  a.rK = rK;
-  a.rV = rV;
-  a.L_max = L_max;
-  a.S = num_splits > 0 ? num_splits : stief_decode_auto_splits(B, Hq, Hkv, max_seq_len, sms);
-  a.qscale = (float)(1.4426950408889634 / std::sqrt((double)d));
-  a.pdl_first = false;
-  // the workspace is laid out for the split count actually used
-  const size_t parts = (size_t)B * Hkv * a.qsub * a.G_T * a.S;
-  a.ws_o = static_cast<float*>(workspace);
-  a.ws_ml = a.ws_o + parts * rV;
-
-  // widest configuration that fits: 8 warps with as many stages as fit, else 4 warps
-  a.nwarps = 0;
-  for (int nw : {8, 4}) {
-    for (int ns = 4; ns >= 2; --ns) {
-      if (stief::decode_split_smem_bytes(nw, ns, a.G_T, d, rK, rV) <= (uint32_t)stief::kMaxSmemPerBlock) {
-        a.nwarps = nw;
-        a.nstage = ns;
-        break;
-      }
-    }
-    if (a.nwarps) break;
-  }
-  if (!a.nwarps) return STIEF_ERR_INVALID_ARG;
+  st = stief::plan_decode(a, q, P_K, P_V, k_lat, v_lat, seq_lens, out, B, Hq, Hkv, d, rK, rV,
+                          L_max, max_seq_len, num_splits, dev_status);
+  if (st != STIEF_OK) return st;
+  // counters at the start, then the partial states laid out for the split count used
+  const size_t units = (size_t)B * Hkv * a.qsub;
+  a.ws_cnt = static_cast<uint32_t*>(workspace);
+  a.ws_part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                       stief::decode_ws_counter_bytes(units));
   if (stief::launch_decode(a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return STIEF_ERR_CUDA;
   return STIEF_OK;

@@ -72,6 +72,9 @@ typedef enum stief_status {
 #define STIEF_DEV_BAD_LENGTH 0x4u        /* a seq_lens entry was negative or > L_max
                                             (decode: that sequence's output is zero;
                                             compress: it is left untouched) */
+#define STIEF_DEV_SMEM_ALIGN 0x8u        /* decode: dynamic shared memory was not 1 KiB
+                                            aligned as the swizzled key tiles need;
+                                            nothing was computed */
 
 /*
  * stief_compress_append -- compressed storage of new keys and values
@@ -119,9 +122,10 @@ STIEF_API int stief_decode_auto_splits(int B, int Hq, int Hkv, int max_seq_len, 
 /*
  * stief_decode_workspace_bytes -- bytes of device workspace stief_decode_attention
  * needs for these sizes, for any split count it may use (at most
- * stief_decode_max_splits(max_seq_len)).  The workspace holds the per-split
- * partial softmax states (running maximum, sum and unnormalised latent output).
- * Pure host function.  Returns 0 for invalid arguments.
+ * stief_decode_max_splits(max_seq_len)).  The workspace holds one ticket counter
+ * per (sequence, KV head, query sub-group) followed by the per-split partial
+ * softmax states (running maximum, sum and unnormalised latent output).  Pure host
+ * function.  Returns 0 for invalid arguments.
  */
 STIEF_API size_t stief_decode_workspace_bytes(int B, int Hq, int Hkv, int rV, int max_seq_len);
 
@@ -151,15 +155,19 @@ STIEF_API size_t stief_decode_workspace_bytes(int B, int Hq, int Hkv, int rV, in
  *   out          : bf16 [B][Hq][d] (written)
  *   workspace    : device scratch of at least workspace_bytes >=
  *                  stief_decode_workspace_bytes(B, Hq, Hkv, rV, max_seq_len)
- *                  bytes; its contents on entry do not matter
+ *                  bytes.  Zero-fill it once before its first use: its ticket
+ *                  counters must be zero when a call starts, and every call that
+ *                  runs to completion leaves them at zero again, so the same
+ *                  workspace serves any later call (any sizes) on the same
+ *                  stream without clearing
  *   max_seq_len  : host-side upper bound of seq_lens (<= L_max); sizes the grid
  *   num_splits   : 0 = automatic, otherwise the number of KV splits per sequence
  *                  (1 .. stief_decode_max_splits(max_seq_len))
  *
- * Two kernels run on `stream`: the split kernel (query projection, scores,
- * online softmax, latent value mix) and the combine kernel (log-sum-exp merge of
- * the splits and up-projection with P_V^T), the second launched as a
- * programmatic dependent of the first.
+ * One kernel runs on `stream`, a CTA per (split, KV head, query sub-group,
+ * sequence): query projection, scores, online softmax and latent value mix over
+ * its token range; the last CTA of each (sequence, KV head, sub-group) to finish
+ * merges the splits (log-sum-exp) and up-projects with P_V^T.
  * Returns STIEF_OK or an argument error (nothing launched).
  */
 STIEF_API stief_status stief_decode_attention(const uint16_t* q, const uint16_t* P_K,
@@ -182,15 +190,17 @@ STIEF_API stief_status stief_decode_attention(const uint16_t* q, const uint16_t*
  * workspace / workspace_bytes.  The per-split partial states live in a fixed 8 MiB
  * array of device memory owned by the library (one per GPU that loads it, held
  * until the process exits).  Sizes whose partial states, for the split count
- * actually used, exceed 8 MiB -- B*Hkv*ceil(G/G_T)*G_T*splits*(rV+2)*4 bytes with
- * G = Hq/Hkv and G_T the smallest of 1, 2, 4, 8 that is >= min(G, 8) -- return
+ * actually used, exceed 8 MiB -- B*Hkv*ceil(G/G_T)*G_T*splits*(rV+4)*4 bytes with
+ * G = Hq/Hkv and G_T the smallest of 1, 2, 4, 8 that is >= min(G, 8) -- plus the
+ * ticket counters, return
  * STIEF_ERR_WORKSPACE and launch nothing.  The first call on each device looks up
  * the array's device address (cudaGetSymbolAddress) with that device current; make
  * that first call before any stream capture.  All calls on a device share the
  * array: calls whose kernels overlap on the GPU race on it, so the caller must
- * order them (e.g. one stream).  The array keeps the last call's contents; no part
- * of it needs clearing between calls.  Calls no cudaMalloc, cudaFree or
- * allocating library routine.
+ * order them (e.g. one stream).  The array keeps the last call's contents; its
+ * ticket counters are zero at load and every call that runs to completion leaves
+ * them at zero, so nothing needs clearing between calls.  Calls no cudaMalloc,
+ * cudaFree or allocating library routine.
  */
 STIEF_API stief_status stief_decode_attention_noalloc(
     const uint16_t* q, const uint16_t* P_K, const uint16_t* P_V, const uint16_t* k_lat,

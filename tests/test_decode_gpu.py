@@ -131,3 +131,24 @@ def test_bad_length_is_reported_and_gives_zero():
 def test_status_word_stays_clear_on_success():
     case = make_decode_case(1, 4, 1, 64, 64, 128, 901)
     gpu_decode(*case, [128], expect_status=0)
+
+
+def test_workspace_counters_return_to_zero_and_partials_may_hold_garbage():
+    """The ticket counters are the only workspace state that must be zero on entry; every
+    completed call leaves them at zero, whatever the partial-state area holds."""
+    import decode_attention_stief_b200 as stief
+    case = make_decode_case(2, 32, 8, 64, 48, 4096, 950)
+    dev = torch.device("cuda")
+    q, P_K, P_V, k_lat, v_lat = (x.to(dev) for x in case)
+    lens = torch.tensor([4096, 2500], dtype=torch.int32, device=dev)
+    ws = stief.workspace_for(2, 32, 8, 48, 4096)
+    counter_bytes = 256  # 16 units x 4 bytes, padded to 256
+    ws[counter_bytes:].fill_(0xFF)
+    want = oracle_decode(*case, [4096, 2500])
+    for splits in (9, 9, 32, 1, 5):
+        out = torch.empty((2, 32, 128), dtype=torch.bfloat16, device=dev)
+        stief.stief_decode_attention(q, P_K, P_V, k_lat, v_lat, lens, out, ws, 4096,
+                                     num_splits=splits)
+        torch.cuda.synchronize()
+        assert int(ws[:counter_bytes].count_nonzero()) == 0
+        assert_decode_close(out.cpu(), want)
