@@ -136,6 +136,73 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// Scores of one key piece for the lane's token: WC 16-byte chunks per row, stored
+// swizzled (chunk c of the lane's row at byte (c << 4) ^ sw4 of the row); q~ chunks are
+// warp-wide broadcasts.  prow_sw = row address ^ sw4 (rows are at least 32-byte aligned
+// and the swizzle only touches bits below the row size, so XOR equals addition).
+template <int G_T, int WC>
+__device__ __forceinline__ void score_piece(uint32_t prow_sw, uint32_t q0, float2 (&sa)[G_T],
+                                            float2 (&sb)[G_T]) {
+  constexpr uint32_t QS = (uint32_t)G_T * 32u;  // bytes per q~ chunk row
+#pragma unroll
+  for (int cc = 0; cc < WC; cc += 2) {
+    float2 ka[4], kb[4];
+    unpack8(lds128(prow_sw ^ (uint32_t)(cc << 4)), ka);
+    unpack8(lds128(prow_sw ^ (uint32_t)((cc + 1) << 4)), kb);
+    const uint32_t qa = q0 + (uint32_t)cc * QS;
+#pragma unroll
+    for (int g = 0; g < G_T; ++g) {
+      const float4 xa = lds128f(qa + g * 32u), ya = lds128f(qa + g * 32u + 16u);
+      const float4 xb = lds128f(qa + QS + g * 32u), yb = lds128f(qa + QS + g * 32u + 16u);
+      sa[g] = fma2(f2(xa.x, xa.y), ka[0], sa[g]);
+      sb[g] = fma2(f2(xb.x, xb.y), kb[0], sb[g]);
+      sa[g] = fma2(f2(xa.z, xa.w), ka[1], sa[g]);
+      sb[g] = fma2(f2(xb.z, xb.w), kb[1], sb[g]);
+      sa[g] = fma2(f2(ya.x, ya.y), ka[2], sa[g]);
+      sb[g] = fma2(f2(yb.x, yb.y), kb[2], sb[g]);
+      sa[g] = fma2(f2(ya.z, ya.w), ka[3], sa[g]);
+      sb[g] = fma2(f2(yb.z, yb.w), kb[3], sb[g]);
+    }
+  }
+}
+
+// Latent value mix of one tile: RVC = rV/8 lanes per token, TPW tokens per step; the
+// lane's token slot and chunk are fixed, so every address is a constant offset.
+template <int G_T, int RVC>
+__device__ __forceinline__ void mix_tile(uint32_t vst, uint32_t p_addr, int n, int lane,
+                                         float2 (&acc)[G_T][4]) {
+  constexpr int TPW = 32 / RVC;
+  constexpr int STEPS = (32 + TPW - 1) / TPW;
+  const int vslot = lane / RVC;
+  if (vslot >= TPW) return;
+  const int vchunk = lane - vslot * RVC;
+  const uint32_t vb = vst + (uint32_t)(vslot * RVC + vchunk) * 16u;
+  const uint32_t pb = p_addr + (uint32_t)vslot * G_T * 8u;
+#pragma unroll
+  for (int st = 0; st < STEPS; ++st) {
+    if (st * TPW + vslot < n) {
+      float2 v[4];
+      unpack8(lds128(vb + (uint32_t)(st * TPW * RVC * 16)), v);
+      float2 pp[G_T];
+      if constexpr (G_T >= 2) {
+#pragma unroll
+        for (int g2 = 0; g2 < G_T; g2 += 2) {
+          const float4 x = lds128f(pb + (uint32_t)(st * TPW * G_T * 8 + g2 * 8));
+          pp[g2] = f2(x.x, x.y);
+          pp[g2 + 1] = f2(x.z, x.w);
+        }
+      } else {
+        pp[0] = *reinterpret_cast<const float2*>(
+            __cvta_shared_to_generic(pb + (uint32_t)(st * TPW * 8)));
+      }
+#pragma unroll
+      for (int g = 0; g < G_T; ++g)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[g][e] = fma2(pp[g], v[e], acc[g][e]);
+    }
+  }
+}
+
 // Warp-specialised: warps [0, NP) are K-warps (scores, softmax), warps [NP, 2NP) are
 // V-warps (value mix, stage refills).  K-warp i and V-warp i form pair i, which owns a
 // ring of `nstage` stages and processes the CTA's tiles i, i + NP, i + 2NP, ...
@@ -295,7 +362,6 @@ __global__ void __launch_bounds__(NP * 64, 1) stief_decode_kernel(const __grid_c
   const int RV = rV >> 3;
   const int TPW = 32 / RV;            // tokens per value step
   const int vslot = lane / RV;
-  const int vchunk = lane - vslot * RV;
   const bool vactive = vslot < TPW;
   float* pbuf = reinterpret_cast<float*>(smem + L.scratch) + pair * 2 * kTile * G_T * 2;
 
@@ -336,30 +402,11 @@ __global__ void __launch_bounds__(NP * 64, 1) stief_decode_kernel(const __grid_c
         }
         for (int p = 0; p < a.npieces; ++p) {
           const int w = a.kp[p].width;
-          // row `lane` of this piece; its 16-byte chunk c sits at position c ^ sw
           const uint32_t prow = kst + (uint32_t)a.kp[p].smem_off + (uint32_t)lane * w * 2u;
-          const int sw = w == 64 ? (lane & 7) : (w == 32 ? ((lane >> 1) & 3) : ((lane >> 2) & 1));
           const uint32_t q0 = qt_addr + (uint32_t)(a.kp[p].x >> 3) * qstride_b;
-          for (int cc = 0; cc < (w >> 3); cc += 2) {
-            float2 ka[4], kb[4];
-            unpack8(lds128(prow + (uint32_t)((cc ^ sw) << 4)), ka);
-            unpack8(lds128(prow + (uint32_t)(((cc + 1) ^ sw) << 4)), kb);
-            const uint32_t qa = q0 + (uint32_t)cc * qstride_b;
-            const uint32_t qb = qa + qstride_b;
-#pragma unroll
-            for (int g = 0; g < G_T; ++g) {
-              const float4 xa = lds128f(qa + g * 32u), ya = lds128f(qa + g * 32u + 16u);
-              const float4 xb = lds128f(qb + g * 32u), yb = lds128f(qb + g * 32u + 16u);
-              sa[g] = fma2(f2(xa.x, xa.y), ka[0], sa[g]);
-              sb[g] = fma2(f2(xb.x, xb.y), kb[0], sb[g]);
-              sa[g] = fma2(f2(xa.z, xa.w), ka[1], sa[g]);
-              sb[g] = fma2(f2(xb.z, xb.w), kb[1], sb[g]);
-              sa[g] = fma2(f2(ya.x, ya.y), ka[2], sa[g]);
-              sb[g] = fma2(f2(yb.x, yb.y), kb[2], sb[g]);
-              sa[g] = fma2(f2(ya.z, ya.w), ka[3], sa[g]);
-              sb[g] = fma2(f2(yb.z, yb.w), kb[3], sb[g]);
-            }
-          }
+          if (w == 64) score_piece<G_T, 8>(prow ^ ((uint32_t)(lane & 7) << 4), q0, sa, sb);
+          else if (w == 32) score_piece<G_T, 4>(prow ^ ((uint32_t)((lane >> 1) & 3) << 4), q0, sa, sb);
+          else score_piece<G_T, 2>(prow ^ ((uint32_t)((lane >> 2) & 1) << 4), q0, sa, sb);
         }
 #pragma unroll
         for (int g = 0; g < G_T; ++g) s[g] = (sa[g].x + sa[g].y) + (sb[g].x + sb[g].y);
@@ -436,28 +483,15 @@ __global__ void __launch_bounds__(NP * 64, 1) stief_decode_kernel(const __grid_c
         }
       }
       const uint32_t p_addr = smem_u32(pbuf + pb * kTile * G_T * 2);
-      if (vactive) {
-#pragma unroll 2
-        for (int t = vslot; t < n; t += TPW) {
-          float2 v[4];
-          unpack8(lds128(vst + (uint32_t)t * rV * 2u + vchunk * 16u), v);
-          float2 pp[G_T];
-          if constexpr (G_T >= 2) {
-#pragma unroll
-            for (int g2 = 0; g2 < G_T; g2 += 2) {
-              const float4 x = lds128f(p_addr + (uint32_t)(t * G_T + g2) * 8u);
-              pp[g2] = f2(x.x, x.y);
-              pp[g2 + 1] = f2(x.z, x.w);
-            }
-          } else {
-            const float4 x = lds128f(p_addr + (uint32_t)(t & ~1) * 8u);
-            pp[0] = (t & 1) ? f2(x.z, x.w) : f2(x.x, x.y);
-          }
-#pragma unroll
-          for (int g = 0; g < G_T; ++g)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) acc[g][e] = fma2(pp[g], v[e], acc[g][e]);
-        }
+      switch (RV) {
+        case 2: mix_tile<G_T, 2>(vst, p_addr, n, lane, acc); break;
+        case 4: mix_tile<G_T, 4>(vst, p_addr, n, lane, acc); break;
+        case 6: mix_tile<G_T, 6>(vst, p_addr, n, lane, acc); break;
+        case 8: mix_tile<G_T, 8>(vst, p_addr, n, lane, acc); break;
+        case 10: mix_tile<G_T, 10>(vst, p_addr, n, lane, acc); break;
+        case 12: mix_tile<G_T, 12>(vst, p_addr, n, lane, acc); break;
+        case 14: mix_tile<G_T, 14>(vst, p_addr, n, lane, acc); break;
+        default: mix_tile<G_T, 16>(vst, p_addr, n, lane, acc); break;
       }
       __syncwarp();
       consumed = k + 1;
