@@ -9,6 +9,8 @@
 // Kernels:
 //   stief_compress_rows_kernel  -- CUDA-core projection, grid (ceil(T/TT), 2 Hkv, B);
 //                                  used for decode-sized appends (small T)
+//   stief_compress_tc_kernel    -- tcgen05 tensor-core projection of prefill-sized
+//                                  chunks (T >= 128), compress_tc.cu
 //   stief_seq_lens_kernel       -- the length update, launched as a programmatic
 //                                  dependent of the projection so that it runs
 //                                  only after every projection CTA has read the
@@ -21,6 +23,7 @@
 namespace stief {
 
 constexpr int kRowsPerCta = 8;  // new rows per CTA of the CUDA-core path (T > 1)
+constexpr int kTensorCoreMinRows = 128;  // T from which the tcgen05 path is used
 constexpr int kSmallThreads = 256;
 
 __device__ __forceinline__ float2 fma2c(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
@@ -141,8 +144,14 @@ static cudaError_t launch_rows(const CompressArgs& a, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+cudaError_t launch_compress_tc(const CompressArgs& a, cudaStream_t stream);
+
 cudaError_t launch_compress(const CompressArgs& a, cudaStream_t stream) {
-  cudaError_t e = (a.T == 1) ? launch_rows<1>(a, stream) : launch_rows<kRowsPerCta>(a, stream);
+  cudaError_t e;
+  if (a.T >= kTensorCoreMinRows)
+    e = launch_compress_tc(a, stream);
+  else
+    e = (a.T == 1) ? launch_rows<1>(a, stream) : launch_rows<kRowsPerCta>(a, stream);
   if (e != cudaSuccess) return e;
   return launch_seq_lens(a, stream);
 }

@@ -34,21 +34,28 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // 2-D view of the key cache: [B*Hkv*L_max rows][rK columns] bf16, boxes of 32 rows x width.
 bool encode_key_map(CUtensorMap* map, const uint16_t* k_lat, int rK, uint64_t rows, int width) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {(cuuint64_t)rK, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)rK * 2u};
-  const cuuint32_t box[2] = {(cuuint32_t)width, 32u};
-  const cuuint32_t estr[2] = {1u, 1u};
   const CUtensorMapSwizzle sw = width == 64   ? CU_TENSOR_MAP_SWIZZLE_128B
                                 : width == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
                                               : CU_TENSOR_MAP_SWIZZLE_32B;
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(k_lat), dims, strides,
-            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return encode_tiled_bf16_2d(map, k_lat, (uint64_t)rK, rows, (uint64_t)rK * 2u, (uint32_t)width,
+                              32u, sw);
 }
 
 }  // namespace
+
+bool encode_tiled_bf16_2d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
+                          uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows,
+                          CUtensorMapSwizzle swizzle) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)row_stride_bytes};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1u, 1u};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 stief_status plan_decode(DecodeArgs& a, const uint16_t* q, const uint16_t* P_K,
                          const uint16_t* P_V, const uint16_t* k_lat, const uint16_t* v_lat,

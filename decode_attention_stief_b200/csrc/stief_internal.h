@@ -60,6 +60,15 @@ constexpr int kMaxSmemPerBlock = 232448;  // 227 KB opt-in dynamic shared memory
 
 uint32_t decode_smem_bytes(int NW, int nstage, int G_T, int d, int rK, int rV);
 
+// 2-D tiled TMA tensor map over a row-major bf16 matrix [rows][cols] (row stride in
+// bytes), boxes of box_cols x box_rows with the given swizzle.  Host only.
+bool encode_tiled_bf16_2d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
+                          uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows,
+                          CUtensorMapSwizzle swizzle);
+
+struct CompressTcArgs;
+uint32_t compress_tc_smem_bytes(int rK, int rV);
+
 // Validates a decode call and fills everything in `a` except the workspace pointers
 // (split count, group tiling, CTA configuration, key tensor maps).  Host only.
 stief_status plan_decode(DecodeArgs& a, const uint16_t* q, const uint16_t* P_K,

@@ -150,3 +150,41 @@ def test_append_then_decode_end_to_end():
     got = gpu_decode(q, P_K, P_V, gk, gv, olens)
     want = oracle.decode(f64(q), f64(P_K), f64(P_V), ok_lat, ov_lat, olens)
     assert_decode_close(got, want)
+
+
+@pytest.mark.parametrize("T,rK,rV", [(128, 64, 64), (300, 32, 48), (257, 96, 112), (640, 16, 128)])
+def test_tensor_core_chunks(T, rK, rV):
+    """Prefill-sized appends (T >= 128) run on the tcgen05 path: full tiles and ragged tails."""
+    B, Hkv, d, L_max = 2, 2, 128, T + 40
+    seed = 1000 + T + rK
+    k_new, v_new = si.full_kv(seed, B, Hkv, T, d)
+    P_K, P_V = si.bases_bf16(seed, Hkv, d, rK, rV)
+    lens = [0, 33]
+    gk, gv, glens = _run_append(k_new, v_new, P_K, P_V, _cache(B, Hkv, L_max, rK, CANARY_K),
+                                _cache(B, Hkv, L_max, rV, CANARY_V), lens)
+    assert glens.tolist() == [L + T for L in lens]
+    for b, L in enumerate(lens):
+        for h in range(Hkv):
+            assert _check_latent(gk[b, h, L:L + T], f64(k_new[b, h]), f64(P_K[h])) > 0.98
+            assert _check_latent(gv[b, h, L:L + T], f64(v_new[b, h]), f64(P_V[h])) > 0.98
+            keep = np.ones(L_max, bool)
+            keep[L:L + T] = False
+            assert torch.all(gk[b, h, keep].view(torch.int16) == _s16(CANARY_K))
+            assert torch.all(gv[b, h, keep].view(torch.int16) == _s16(CANARY_V))
+
+
+def test_prefill_chunk_full_size():
+    """One layer of the prefill workload: a 4096-token chunk for 8 KV heads, ranks 64/64."""
+    w = si.PREFILL_CHUNK
+    B, Hkv, T, d, rK, rV = w["B"], w["Hkv"], w["T"], w["d"], w["rK"], w["rV"]
+    dev = torch.device("cuda")
+    k_new = si.low_rank_rows_torch(si.sub_seed(w["seed"], 1), B * Hkv, T, d, dev).view(B, Hkv, T, d)
+    v_new = si.low_rank_rows_torch(si.sub_seed(w["seed"], 2), B * Hkv, T, d, dev).view(B, Hkv, T, d)
+    P_K, P_V = si.bases_bf16(w["seed"], Hkv, d, rK, rV)
+    gk, gv, glens = _run_append(k_new, v_new, P_K, P_V,
+                                torch.zeros((B, Hkv, T, rK), dtype=torch.bfloat16),
+                                torch.zeros((B, Hkv, T, rV), dtype=torch.bfloat16), [0])
+    assert glens.tolist() == [T]
+    for h in range(Hkv):
+        assert _check_latent(gk[0, h], f64(k_new[0, h]), f64(P_K[h])) > 0.98
+        assert _check_latent(gv[0, h], f64(v_new[0, h]), f64(P_V[h])) > 0.98
