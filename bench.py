@@ -306,6 +306,12 @@ def run_gpu(args, w: si.Workload):
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         ms_per_step, e2e_ms, dec_ms_mean = (float(x) for x in t.tolist())
 
+    # ---- prefill compress (the prefill + batched decode workload): one 4096-token chunk
+    # per layer through stief_compress_append (tcgen05 path), timed separately
+    compress = None
+    if w.name == "prefill_b64" and not args.no_prefill:
+        compress = time_prefill_compress(args, len(layers), dev, flush, stream)
+
     # ---- numbers
     tokens_per_step = w.B * ws_n
     value = tokens_per_step / (ms_per_step / 1e3)
@@ -356,12 +362,62 @@ def run_gpu(args, w: si.Workload):
         "clocks": clocks,
         "wall_s_timed_region": round(t_wall, 3),
     }
+    if compress is not None:
+        result["compress"] = compress
     if rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     if ws_n > 1:
         torch.distributed.destroy_process_group()
     if rank == 0:
         print(json.dumps(result), flush=True)
+
+
+def time_prefill_compress(args, n_layers: int, dev, flush, stream):
+    """Time stief_compress_append of one prefill chunk (B=1, Hkv=8, T=4096, ranks 64/64)
+    for every layer; L2 flushed before each repetition.  Returns a summary dict."""
+    import decode_attention_stief_b200 as stief
+    c = si.PREFILL_CHUNK
+    B, Hkv, T, d, rK, rV = c["B"], c["Hkv"], c["T"], c["d"], c["rK"], c["rV"]
+    ks = [si.low_rank_rows_torch(si.sub_seed(c["seed"], 21, li), B * Hkv, T, d, dev).view(B, Hkv, T, d)
+          for li in range(n_layers)]
+    vs = [si.low_rank_rows_torch(si.sub_seed(c["seed"], 22, li), B * Hkv, T, d, dev).view(B, Hkv, T, d)
+          for li in range(n_layers)]
+    P_K, P_V = si.bases_bf16(c["seed"], Hkv, d, rK, rV)
+    P_K, P_V = P_K.to(dev), P_V.to(dev)
+    kl = [torch.empty((B, Hkv, T, rK), dtype=torch.bfloat16, device=dev) for _ in range(n_layers)]
+    vl = [torch.empty((B, Hkv, T, rV), dtype=torch.bfloat16, device=dev) for _ in range(n_layers)]
+    lens = torch.zeros((n_layers, B), dtype=torch.int32, device=dev)
+
+    def chunk():
+        for li in range(n_layers):
+            stief.stief_compress_append(ks[li], vs[li], P_K, P_V, kl[li], vl[li], lens[li])
+
+    for _ in range(args.warmup):
+        lens.zero_()
+        chunk()
+    reps = max(3, min(args.steps, 20))
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(reps)]
+    for r in range(reps):
+        lens.zero_()
+        flush.zero_()
+        evs[r][0].record(stream)
+        chunk()
+        evs[r][1].record(stream)
+    torch.cuda.synchronize()
+    ms = sorted(a.elapsed_time(b) for a, b in evs)
+    ms_med = ms[len(ms) // 2]
+    bytes_moved = n_layers * B * Hkv * T * (2 * d * 2 + 2 * (rK + rV))
+    flops = n_layers * B * Hkv * T * 2 * d * (rK + rV)
+    peak, kind = _hbm_peak()
+    return {"what": f"stief_compress_append of a {T}-token chunk, {Hkv} KV heads, ranks {rK}/{rV}, "
+                    f"x{n_layers} layers (tcgen05 path), L2 flushed",
+            "us_total": round(ms_med * 1e3, 2), "us_per_layer": round(ms_med * 1e3 / n_layers, 3),
+            "algorithmic_bytes": bytes_moved,
+            "GBs": round(bytes_moved / (ms_med / 1e3) / 1e9, 1),
+            "frac_of_hbm_peak": round(bytes_moved / (ms_med / 1e3) / 1e9 / peak, 4),
+            "TFLOPs": round(flops / (ms_med / 1e3) / 1e12, 2),
+            "kernel_launches_per_layer": 2}
 
 
 # ----------------------------------------------------------------------------- CPU oracle
@@ -469,6 +525,8 @@ def main():
     ap.add_argument("--decode-iters", type=int, default=50)
     ap.add_argument("--cpu-seconds", type=float, default=30.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="skip the prefill-compress measurement of the prefill_b64 workload")
     ap.add_argument("--layers", type=int, default=0,
                     help="diagnostics: run only the first N layers of the workload")
     ap.add_argument("--splits", type=int, default=0,
