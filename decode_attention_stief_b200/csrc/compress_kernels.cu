@@ -136,8 +136,9 @@ template <int TT>
 static cudaError_t launch_rows(const CompressArgs& a, cudaStream_t stream) {
   const int rmax = a.rK > a.rV ? a.rK : a.rV;
   const uint32_t smem = 128u + 2u * a.d * rmax + 2u * TT * a.d + 8u * TT * kSmallThreads;
-  cudaError_t e = cudaFuncSetAttribute(stief_compress_rows_kernel<TT>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  static SmemLimit limit;
+  cudaError_t e = limit.ensure(reinterpret_cast<const void*>(stief_compress_rows_kernel<TT>),
+                               a.device, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((a.T + TT - 1) / TT, a.Hkv * 2, a.B);
   stief_compress_rows_kernel<TT><<<grid, kSmallThreads, smem, stream>>>(a);

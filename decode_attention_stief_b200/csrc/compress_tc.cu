@@ -283,17 +283,17 @@ cudaError_t launch_compress_tc(const CompressArgs& a, cudaStream_t stream) {
   if (!encode_tiled_bf16_2d(&ta.mk, a.k_new, 128, rows, 256, 64, kTcRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_tiled_bf16_2d(&ta.mv, a.v_new, 128, rows, 256, 64, kTcRows, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int dev = 0, sms = 0;
+  bool sm100 = false;
+  if (!query_device(&dev, &sms, &sm100)) return cudaErrorInvalidDevice;
   const int heads = a.B * a.Hkv;
   int gx = heads >= sms ? 1 : sms / heads;
   if (gx > ta.tiles) gx = ta.tiles;
   // at least 80 KiB so no more than two CTAs (2 x 256 TMEM columns) share an SM
   uint32_t smem = tc_smem_layout(a.rK, a.rV).total;
   if (smem < 80u * 1024u) smem = 80u * 1024u;
-  cudaError_t e = cudaFuncSetAttribute(stief_compress_tc_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  static SmemLimit limit;
+  cudaError_t e = limit.ensure(reinterpret_cast<const void*>(stief_compress_tc_kernel), dev, (int)smem);
   if (e != cudaSuccess) return e;
   stief_compress_tc_kernel<<<dim3(gx, a.Hkv, a.B), kTcThreads, smem, stream>>>(ta);
   return cudaGetLastError();

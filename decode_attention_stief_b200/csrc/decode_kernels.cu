@@ -9,35 +9,30 @@
 //     o   = (sum_t softmax(s)_t V_down[t]) P_V^T   (up-projection after the mix)
 // so the HBM stream is the bf16 latent cache, read once per KV head.
 //
-// One kernel, stief_decode_kernel<G_T, NP>, grid (splits, Hkv * qsub, B).  A CTA
-// serves up to G_T query heads of one KV head ("unit") over one token range, with
-// NP warp pairs (2*NP warps):
-//   - prologue: q and P_K[h] arrive by bulk copy; q~ = q . P_K * log2(e)/sqrt(d)
-//     in fp32, stored padded chunk-major
-//   - streaming: pair i owns two rings of shared-memory stages holding the keys
-//     and the values of 32-token tiles, each slot filled by a 1-D bulk copy (TMA
-//     engine, L2 evict-first) that completes on the slot's mbarrier, and works
-//     through tiles i, i + NP, ...  Its K-warp computes the scores -- one lane
-//     per token; key tiles land by 2-D TMA tensor copies in 64/32/16-column pieces
-//     with the matching 128/64/32-byte swizzle, so all lanes read the same logical
-//     chunk at once without bank conflicts and q~ is read as warp-wide broadcasts;
-//     packed fp32x2 FMAs -- and the online
-//     softmax in the log2
-//     domain with lazy rescaling (accumulators rescaled only when a score passes
-//     the running reference by more than 8, so every weight stays <= 2^8).  It
-//     hands the weights (as duplicated pairs) and any rescale factors to its
-//     V-warp through a double buffer guarded by two mbarriers.  The V-warp mixes
-//     the latent values (r_V/8 lanes per token, packed FMAs).  Key and value halves
-//     of a tile live in separate rings, each refilled by its own consumer as soon
-//     as it is done, which keeps more bytes in flight.  Splitting the roles halves the registers each warp needs, so twice
-//     as many warps hide shared-memory and FMA latency.  No CTA-wide barrier in
-//     the loop.
-//   - epilogue: merge the pairs; with one split the CTA finishes the unit itself;
-//     otherwise it stores its partial state (o~[r_V], m, l) and takes a ticket,
-//     and the last CTA of the unit merges all splits (log-sum-exp) -- that CTA
-//     resets the ticket counter, so the workspace counters stay zero between
-//     calls.  P_V arrives by bulk copy into the freed stage region while the
-//     merge runs; then o = o~ . P_V^T, bf16 out.
+// One kernel, grid (splits, Hkv * qsub, B).  A CTA serves up to G_T <= 8 query heads
+// of one KV head (a "unit") over one token range, with nwarps warps that each stream
+// their own 32-token tiles (warp w takes tiles w, w + nwarps, ...) through a private
+// ring of shared-memory stages.  Every stage holds the keys and the values of one tile,
+// fetched by 2-D TMA tensor copies in 64/32/16-column pieces with the matching swizzle
+// and completing on the stage's mbarrier.
+//
+// The contractions run on the warp-level tensor-core MMA (m16n8k16, bf16 operands,
+// fp32 accumulators), with the query heads as the N = 8 dimension: column n of the
+// MMA is head n & 3 for groups of up to 4 heads (part n >> 2), or head n with the part
+// given by the n-tile for groups of 8.  Part 0 carries the bf16 rounding hi(x) of an
+// fp32 operand x and part 1 its residual lo(x) = bf16(x - hi(x)); the two products are
+// added in fp32, which keeps q~, the softmax weights and o~ at about 16 significant
+// bits although the MMA takes bf16.  Per tile and warp:
+//   scores  S[token][n]  = K_down[token][:] . Q^T[:][n]     (M = tokens, K = r_K)
+//   online softmax over the tile (log2 domain, lazy rescale: accumulators are only
+//   rescaled when a head's maximum passes its running reference by more than 8)
+//   mix     O^T[dim][n] += V_down^T[dim][token] . P^T[token][n]  (M = r_V dims, K = tokens)
+// where P^T comes from the score accumulators through an in-register 8x8 transpose
+// (movmatrix).  The epilogue merges the warps (log-sum-exp), up-projects with P_V^T
+// on the same MMA (M = d, K = r_V), and either writes the output (one split) or
+// stores an up-projected partial state and takes a ticket; the last CTA of the unit
+// merges the splits and resets the ticket counter, so the workspace counters stay
+// zero between calls.
 #include <cfloat>
 #include <cmath>
 #include <cstdint>
@@ -47,8 +42,9 @@
 
 namespace stief {
 
-constexpr int kTile = 32;            // tokens per pair tile
+constexpr int kPreIssue = 1;         // stages per warp requested before q~ is ready
 constexpr float kRescaleTau = 8.0f;  // lazy-rescale threshold (log2 units)
+constexpr uint32_t kFull = 0xffffffffu;
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -56,657 +52,798 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
+// A bounded mbarrier wait whose outcome is the same in every lane of the warp (the
+// warp-wide MMA and ldmatrix instructions that follow need all 32 lanes).
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint32_t* dev_status) {
+  return __all_sync(kFull, mbar_wait_bounded(bar, parity, dev_status));
 }
 
-__device__ __forceinline__ float2 f2(float x, float y) { return make_float2(x, y); }
-__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
-// the 4 bf16 pairs of a 16-byte chunk, widened exactly to fp32 pairs
-__device__ __forceinline__ void unpack8(const uint4 w, float2 (&v)[4]) {
-  v[0] = f2(bf16lo(w.x), bf16hi(w.x));
-  v[1] = f2(bf16lo(w.y), bf16hi(w.y));
-  v[2] = f2(bf16lo(w.z), bf16hi(w.z));
-  v[3] = f2(bf16lo(w.w), bf16hi(w.w));
+// ---------------------------------------------------------------------------- warp MMA
+
+// Four 8x8 b16 matrices; lanes 8i..8i+7 give the row addresses of matrix i.
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+// Same, each matrix transposed on the way.
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+// Transpose of an 8x8 b16 matrix held in the warp's registers (one pair per lane).
+__device__ __forceinline__ uint32_t movm_t(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+// c += A(16x16, row) . B(16x8, col), bf16 in, fp32 accumulate.
+__device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ float4 ldcg4(const float* p) {
-  return __ldcg(reinterpret_cast<const float4*>(p));
+// c = A . B (accumulators start at zero).
+__device__ __forceinline__ void mma_bf16_z(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                           uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%10,%10,%10,%10};"
+      : "=f"(c[0]), "=f"(c[1]), "=f"(c[2]), "=f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.f));
+}
+
+// hi / lo bf16 parts of an fp32 pair, packed (first element in the low half)
+__device__ __forceinline__ uint32_t hi_pair(float x0, float x1) { return pack_bf16x2_rn(x0, x1); }
+__device__ __forceinline__ uint32_t lo_pair(float x0, float x1, uint32_t hi) {
+  return pack_bf16x2_rn(x0 - bf16lo(hi), x1 - bf16hi(hi));
+}
+
+// ---------------------------------------------------------------------------- tile addressing
+
+// Where 16-byte column chunk `chunk` of a row lives inside a tile of `rows` rows stacked
+// from the pieces of a rank-r matrix: r / 64 pieces 64 columns wide, then one 32 wide if
+// r % 64 >= 32, then one 16 wide if r % 32 == 16 (the order the host plans them in).
+struct PieceLoc {
+  uint32_t off;  // piece offset in the tile
+  uint32_t w;    // piece width (columns)
+  uint32_t lc;   // chunk index inside the piece
+};
+__device__ __forceinline__ PieceLoc locate(int r, int rows, int chunk) {
+  const int col = chunk * 8;
+  const int x64 = r & ~63;
+  const bool has32 = r - x64 >= 32;
+  PieceLoc pl;
+  if (col < x64) {
+    pl.w = 64u;
+    pl.off = (uint32_t)((col >> 6) * rows * 128);
+    pl.lc = (uint32_t)((col & 63) >> 3);
+  } else if (has32 && col < x64 + 32) {
+    pl.w = 32u;
+    pl.off = (uint32_t)(x64 * rows * 2);
+    pl.lc = (uint32_t)((col - x64) >> 3);
+  } else {
+    const int x16 = x64 + (has32 ? 32 : 0);
+    pl.w = 16u;
+    pl.off = (uint32_t)(x16 * rows * 2);
+    pl.lc = (uint32_t)((col - x16) >> 3);
+  }
+  return pl;
+}
+// Byte offset of (row, chunk) under the piece's TMA swizzle: 128-byte rows XOR the chunk
+// with row & 7, 64-byte rows with (row >> 1) & 3, 32-byte rows with (row >> 2) & 1.
+__device__ __forceinline__ uint32_t swz(const PieceLoc& pl, int row) {
+  const uint32_t sw = pl.w == 64u ? (uint32_t)(row & 7)
+                      : pl.w == 32u ? (uint32_t)((row >> 1) & 3)
+                                    : (uint32_t)((row >> 2) & 1);
+  return pl.off + (uint32_t)row * pl.w * 2u + ((pl.lc ^ sw) << 4);
+}
+// Lane row / chunk for an x4 ldmatrix of a 16x16 block read as an A operand:
+//  - row-major (no transpose; the block's rows are the MMA's M): matrices
+//    (rows 0-7, chunk 0), (rows 8-15, chunk 0), (rows 0-7, chunk 1), (rows 8-15, chunk 1)
+//  - transposed (the block's rows are the MMA's K): matrices
+//    (rows 0-7, chunk 0), (rows 0-7, chunk 1), (rows 8-15, chunk 0), (rows 8-15, chunk 1)
+__device__ __forceinline__ int a_row(int lane) { return (lane & 7) + ((lane >> 3) & 1) * 8; }
+__device__ __forceinline__ int a_chunk(int lane) { return lane >> 4; }
+__device__ __forceinline__ int at_row(int lane) { return (lane & 7) + (lane >> 4) * 8; }
+__device__ __forceinline__ int at_chunk(int lane) { return (lane >> 3) & 1; }
+
+// B fragments (k-step ks) of X^T for an fp32 matrix X[head][col] in shared memory (row
+// stride xs floats): column n = lane >> 2 of n-tile j is (head, part) as described at the
+// top; k = cols 16 ks + 2 (lane & 3) + {0, 1} (first register) and + 8 (second).
+template <int NB>
+__device__ __forceinline__ void bfrag_hilo(const float* X, int xs, int ks, int lane,
+                                           uint32_t (&bf)[NB][2]) {
+  const int n = lane >> 2;
+  const int c = 16 * ks + 2 * (lane & 3);
+  const int head = NB == 1 ? (n & 3) : n;
+  const float2 x = *reinterpret_cast<const float2*>(X + head * xs + c);
+  const float2 y = *reinterpret_cast<const float2*>(X + head * xs + c + 8);
+  const uint32_t hx = hi_pair(x.x, x.y), hy = hi_pair(y.x, y.y);
+  const uint32_t lx = lo_pair(x.x, x.y, hx), ly = lo_pair(y.x, y.y, hy);
+  if constexpr (NB == 1) {
+    const bool lo = (n >> 2) != 0;
+    bf[0][0] = lo ? lx : hx;
+    bf[0][1] = lo ? ly : hy;
+  } else {
+    bf[0][0] = hx;
+    bf[0][1] = hy;
+    bf[NB - 1][0] = lx;
+    bf[NB - 1][1] = ly;
+  }
 }
 
 __host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
 // Shared-memory carve-up (byte offsets from the dynamic base).
 struct DecodeSmem {
-  uint32_t bars;     // NP*ns K-stage, NP*ns V-stage, NP*2 weights-full, NP*2 weights-empty, 1 setup
-  uint32_t q;        // G_T x d bf16 query rows
-  uint32_t qt;       // (rK/8) chunks x G_T x 8 fp32 projected, scaled queries
-  uint32_t fbuf;     // NP x 2 x (G_T factors + flag): rescale handed from K- to V-warp
-  uint32_t ml;       // NP x G_T x (m, l); then G_T x (M, L, rescale); then a flag
-  uint32_t scratch;  // P_K (prologue); NP x 2 x 32 x G_T x 2 fp32 weights; o~ (epilogue)
-  uint32_t region;   // per pair a K ring then a V ring of stages; later reduction /
-                     // split-merge staging + P_V at its end
+  uint32_t bars;    // nwarps*nstage "full" and nwarps*nstage "empty" stage barriers, then
+                    // 1 setup barrier (q and P_K, then P_V)
+  uint32_t ml;      // [nwarps][8] (m, l); then [8] M, [8] L; then a flag
+  uint32_t qraw;    // [G_T][d] bf16 query rows
+  uint32_t qt;      // [8][xs] fp32: q~ (prologue), o~ (epilogue)
+  uint32_t pmat;    // P_K (prologue), then P_V: d rows, pieces, swizzled
+  uint32_t region;  // per warp a ring of stages (keys then values of a tile); later the
+                    // cross-warp reduction and the split-merge staging
   uint32_t region_bytes;
-  uint32_t pv;       // offset of P_V inside the region (epilogue)
   uint32_t total;
+  int xs;  // row stride of qt in floats
 };
 
-__host__ __device__ inline DecodeSmem decode_smem_layout(int NP, int nstage, int G_T, int d, int rK,
-                                                         int rV) {
+__host__ __device__ inline DecodeSmem decode_smem_layout(int NW, int ns, int rK, int rV, int tile) {
   DecodeSmem s;
+  const int rmax = rK > rV ? rK : rV;
   uint32_t off = 0;
   s.bars = off;
-  off = align_up(off + 8u * (2 * NP * nstage + 4 * NP + 1), 128);
-  s.q = off;
-  off = align_up(off + 2u * G_T * d, 128);
-  s.qt = off;
-  off = align_up(off + 4u * rK * G_T, 128);
-  s.fbuf = off;
-  off = align_up(off + 4u * NP * 2 * (G_T + 1), 128);
+  off = align_up(off + 8u * (2 * NW * ns + 1), 16);
   s.ml = off;
-  off = align_up(off + 4u * (2 * NP * G_T + 3 * G_T + 4), 128);
-  s.scratch = off;
-  const uint32_t pbuf = 8u * NP * 2 * kTile * G_T;
-  const uint32_t pk = 2u * d * rK;
-  const uint32_t ob = 4u * G_T * rV;
-  uint32_t sb = pbuf > pk ? pbuf : pk;
-  sb = sb > ob ? sb : ob;
-  off = align_up(off + sb, 128);
-  off = align_up(off, 1024);  // swizzled key slots need 1 KiB alignment
+  off = align_up(off + 4u * (NW * 16 + 16 + 4), 16);
+  s.qraw = off;
+  off = align_up(off + 2u * 8u * 128u, 16);  // up to 8 heads of d = 128
+  s.xs = rmax + 4;
+  s.qt = off;
+  off = align_up(off + 4u * 8u * s.xs, 1024);
+  s.pmat = off;
+  off += 256u * rmax;  // d = 128 rows x r bf16
   s.region = off;
-  const uint32_t stage = (uint32_t)NP * nstage * kTile * (rK + rV) * 2u;
-  const uint32_t red = (uint32_t)NP * 32u * G_T * 8u * 4u;
-  const uint32_t pvb = align_up(2u * d * rV, 128);
-  const uint32_t need = align_up(red, 128) + pvb;
-  s.region_bytes = align_up(stage > need ? stage : need, 128);
-  s.pv = s.region_bytes - pvb;
+  s.region_bytes = (uint32_t)NW * ns * tile * (rK + rV) * 2u;
   off += s.region_bytes;
   s.total = off;
   return s;
 }
 
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
+// One CTA = nwarps consumer warps + 1 producer warp.  Lane w of the producer requests the
+// tiles (TMA) of consumer warp w and refills its stages as the warp releases them; the
+// consumer warps only compute.  NB: B n-tiles (1: up to 4 heads, 2: up to 8);
+// NKS >= rK/16; NMV >= rV/16.
+constexpr int kMaxConsumerWarps = 8;
 
-// Scores of one key piece for the lane's token: WC 16-byte chunks per row, stored
-// swizzled (chunk c of the lane's row at byte (c << 4) ^ sw4 of the row); q~ chunks are
-// warp-wide broadcasts.  prow_sw = row address ^ sw4 (rows are at least 32-byte aligned
-// and the swizzle only touches bits below the row size, so XOR equals addition).
-template <int G_T, int WC>
-__device__ __forceinline__ void score_piece(uint32_t prow_sw, uint32_t q0, float2 (&sa)[G_T],
-                                            float2 (&sb)[G_T]) {
-  constexpr uint32_t QS = (uint32_t)G_T * 32u;  // bytes per q~ chunk row
-#pragma unroll
-  for (int cc = 0; cc < WC; cc += 2) {
-    float2 ka[4], kb[4];
-    unpack8(lds128(prow_sw ^ (uint32_t)(cc << 4)), ka);
-    unpack8(lds128(prow_sw ^ (uint32_t)((cc + 1) << 4)), kb);
-    const uint32_t qa = q0 + (uint32_t)cc * QS;
-#pragma unroll
-    for (int g = 0; g < G_T; ++g) {
-      const float4 xa = lds128f(qa + g * 32u), ya = lds128f(qa + g * 32u + 16u);
-      const float4 xb = lds128f(qa + QS + g * 32u), yb = lds128f(qa + QS + g * 32u + 16u);
-      sa[g] = fma2(f2(xa.x, xa.y), ka[0], sa[g]);
-      sb[g] = fma2(f2(xb.x, xb.y), kb[0], sb[g]);
-      sa[g] = fma2(f2(xa.z, xa.w), ka[1], sa[g]);
-      sb[g] = fma2(f2(xb.z, xb.w), kb[1], sb[g]);
-      sa[g] = fma2(f2(ya.x, ya.y), ka[2], sa[g]);
-      sb[g] = fma2(f2(yb.x, yb.y), kb[2], sb[g]);
-      sa[g] = fma2(f2(ya.z, ya.w), ka[3], sa[g]);
-      sb[g] = fma2(f2(yb.z, yb.w), kb[3], sb[g]);
-    }
-  }
-}
-
-// Latent value mix of one tile: RVC = rV/8 lanes per token, TPW tokens per step; the
-// lane's token slot and chunk are fixed, so every address is a constant offset.
-template <int G_T, int RVC>
-__device__ __forceinline__ void mix_tile(uint32_t vst, uint32_t p_addr, int n, int lane,
-                                         float2 (&acc)[G_T][4]) {
-  constexpr int TPW = 32 / RVC;
-  constexpr int STEPS = (32 + TPW - 1) / TPW;
-  const int vslot = lane / RVC;
-  if (vslot >= TPW) return;
-  const int vchunk = lane - vslot * RVC;
-  const uint32_t vb = vst + (uint32_t)(vslot * RVC + vchunk) * 16u;
-  const uint32_t pb = p_addr + (uint32_t)vslot * G_T * 8u;
-#pragma unroll
-  for (int st = 0; st < STEPS; ++st) {
-    if (st * TPW + vslot < n) {
-      float2 v[4];
-      unpack8(lds128(vb + (uint32_t)(st * TPW * RVC * 16)), v);
-      float2 pp[G_T];
-      if constexpr (G_T >= 2) {
-#pragma unroll
-        for (int g2 = 0; g2 < G_T; g2 += 2) {
-          const float4 x = lds128f(pb + (uint32_t)(st * TPW * G_T * 8 + g2 * 8));
-          pp[g2] = f2(x.x, x.y);
-          pp[g2 + 1] = f2(x.z, x.w);
-        }
-      } else {
-        pp[0] = *reinterpret_cast<const float2*>(
-            __cvta_shared_to_generic(pb + (uint32_t)(st * TPW * 8)));
-      }
-#pragma unroll
-      for (int g = 0; g < G_T; ++g)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[g][e] = fma2(pp[g], v[e], acc[g][e]);
-    }
-  }
-}
-
-// Warp-specialised: warps [0, NP) are K-warps (scores, softmax), warps [NP, 2NP) are
-// V-warps (value mix, stage refills).  K-warp i and V-warp i form pair i, which owns a
-// ring of `nstage` stages and processes the CTA's tiles i, i + NP, i + 2NP, ...
-template <int G_T, int NP>
-__global__ void __launch_bounds__(NP * 64, 1) stief_decode_kernel(const __grid_constant__ DecodeArgs a) {
+template <int NB, int NKS, int NMV, int TT>
+__global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
+    stief_decode_kernel(const __grid_constant__ DecodeArgs a) {
+  constexpr int kTile = TT;
+  constexpr int MT = TT / 16;              // 16-token m-tiles (scores) / k-steps (mix) per tile
+  // score k-steps / value m-tiles whose fragments are loaded together (fewer where the
+  // accumulators already take many registers)
+  constexpr bool kLean = TT == 32 && NB == 1 && NKS == 4 && NMV == 4;
+  constexpr int KG = kLean ? 4 : (NB == 1 ? 2 : 1);
+  constexpr int VG = kLean ? 4 : (NB == 1 ? 2 : 1);
   extern __shared__ __align__(1024) uint8_t smem[];
-  constexpr int NT = NP * 64;
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
-  const bool is_k = warp < NP;
-  const int pair = is_k ? warp : warp - NP;
-  const int s_idx = blockIdx.x;                 // split
-  const int kvh = blockIdx.y / a.qsub;          // KV head
-  const int qs = blockIdx.y - kvh * a.qsub;     // query sub-group of that head
+  const int NW = a.nwarps, ns = a.nstage;
+  const int NT = (NW + 1) * 32;  // all threads, the producer warp included
+  const bool producer = warp == NW;
+  const int s_idx = blockIdx.x;              // split
+  const int kvh = blockIdx.y / a.qsub;       // KV head
+  const int qs = blockIdx.y - kvh * a.qsub;  // query sub-group of that head
   const int b = blockIdx.z;
-  const int d = a.d, rK = a.rK, rV = a.rV, S = a.S;
-  const int ns = a.nstage;
+  const int d = a.d, rK = a.rK, rV = a.rV, S = a.S, G_T = a.G_T;
+  const int nks = rK >> 4, nmv = rV >> 4;
   const int h0 = kvh * a.G + qs * G_T;          // first query head of this CTA
   const int gcount = min(G_T, a.G - qs * G_T);  // valid query heads here
   const size_t unit = ((size_t)b * a.Hkv + kvh) * a.qsub + qs;
 
-  const DecodeSmem L = decode_smem_layout(NP, ns, G_T, d, rK, rV);
-  uint64_t* kfull = reinterpret_cast<uint64_t*>(smem + L.bars);  // [NP][ns]
-  uint64_t* vfull = kfull + NP * ns;                              // [NP][ns]
-  uint64_t* pfull = vfull + NP * ns;                              // [NP][2]
-  uint64_t* pempty = pfull + NP * 2;                             // [NP][2]
-  uint64_t* setup_bar = pempty + NP * 2;  // phase 0: q + P_K, phase 1: P_V
-  // a key slot holds the tile's column pieces (64/32/16 wide) as the TMA engine writes
-  // them, each with its shared-memory swizzle; a value slot holds the rows unchanged
-  const uint32_t kt_bytes = (uint32_t)kTile * rK * 2u, vt_bytes = (uint32_t)kTile * rV * 2u;
-  uint8_t* my_kring = smem + L.region + (size_t)pair * ns * (kt_bytes + vt_bytes);
-  uint8_t* my_vring = my_kring + (size_t)ns * kt_bytes;
+  const DecodeSmem L = decode_smem_layout(NW, ns, rK, rV, TT);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);  // [NW][ns]: tile landed
+  uint64_t* empty = full + NW * ns;                             // [NW][ns]: tile consumed
+  uint64_t* setup_bar = empty + NW * ns;  // phase 0: q and P_K, phase 1: P_V
   float* ml = reinterpret_cast<float*>(smem + L.ml);
-  float* fin = ml + 2 * NP * G_T;                    // [G_T] M, [G_T] L, [G_T] rescale
-  int* flag = reinterpret_cast<int*>(fin + 3 * G_T);
-  float* fbuf = reinterpret_cast<float*>(smem + L.fbuf) + pair * 2 * (G_T + 1);
+  float* fin = ml + NW * 16;  // [8] M, [8] L
+  int* flag = reinterpret_cast<int*>(fin + 16);
+  float* qt = reinterpret_cast<float*>(smem + L.qt);
+  const int xs = L.xs;
+  uint8_t* pmat = smem + L.pmat;
+  const uint32_t kt_bytes = (uint32_t)kTile * rK * 2u;
+  const uint32_t st_bytes = kt_bytes + (uint32_t)kTile * rV * 2u;
 
-  if ((smem_u32(smem + L.region) & 1023u) != 0) {  // swizzle patterns assume 1 KiB alignment
+  // the swizzle patterns assume 1 KiB-aligned tiles
+  if (((smem_u32(smem + L.pmat) | smem_u32(smem + L.region)) & 1023u) != 0) {
     if (tid == 0) report(a.dev_status, STIEF_DEV_SMEM_ALIGN);
     return;
   }
   if (tid == 0) {
-    for (int i = 0; i < 2 * NP * ns + 4 * NP + 1; ++i) mbar_init(&kfull[i], 1);
+    for (int i = 0; i < 2 * NW * ns + 1; ++i) mbar_init(&full[i], 1);
     fence_barrier_init();
   }
   __syncthreads();
-
-  // q and the bases were written before this kernel started (it is not launched
-  // as a programmatic dependent), so they may be fetched before the wait below.
-  if (tid == 0) {
-    const uint32_t qbytes = 2u * gcount * d;
-    const uint32_t pbytes = 2u * d * rK;
-    mbar_arrive_expect_tx(setup_bar, qbytes + pbytes);
-    bulk_g2s(smem + L.q, a.q + ((size_t)b * a.Hq + h0) * d, qbytes, setup_bar);
-    bulk_g2s(smem + L.scratch, a.P_K + (size_t)kvh * d * rK, pbytes, setup_bar);
-  }
+  // inputs may come from the preceding kernel in the stream: read nothing before this
   pdl_wait();
 
-  int Lb = a.seq_lens[b];
-  if (Lb < 0 || Lb > a.L_max) {
+  // ---- split range and tiles --------------------------------------------------------------
+  // Splits partition [0, S * chunk) by the host bound max_seq_len (the grid was sized by it),
+  // so the first tiles can be requested before seq_lens has been read.  Consumer warp w takes
+  // the split's tiles w, w + NW, ...
+  const int t0 = s_idx * a.chunk;
+  const int t_spec = min(t0 + a.chunk, a.max_seq_len);
+  const int spec_tiles = t_spec > t0 ? (t_spec - t0 + kTile - 1) / kTile : 0;
+  int Lb = __ldcg(a.seq_lens + b);
+  if (Lb < 0 || Lb > a.max_seq_len) {
     if (tid == 0 && s_idx == 0 && blockIdx.y == 0) report(a.dev_status, STIEF_DEV_BAD_LENGTH);
     Lb = 0;
   }
-  const int chunk = (Lb + S - 1) / S;
-  const int t0 = min(Lb, s_idx * chunk);
-  const int t1 = min(Lb, t0 + chunk);
-  const int n_tiles = (t1 - t0 + kTile - 1) / kTile;
-  const int my_tiles = pair < n_tiles ? (n_tiles - pair + NP - 1) / NP : 0;
-
+  const int t1 = min(t0 + a.chunk, Lb);
+  const int n_tiles = t1 > t0 ? (t1 - t0 + kTile - 1) / kTile : 0;
+  auto warp_tiles = [NW](int w, int tiles) { return w < tiles ? (tiles - w + NW - 1) / NW : 0; };
   const size_t head_row0 = ((size_t)b * a.Hkv + kvh) * a.L_max;
-  const uint16_t* vbase_g = a.v_lat + head_row0 * rV;
-
-  // K and V halves of a tile travel separately, so each ring slot is refilled as soon
-  // as its own consumer is done with it (the K-warp after its scores, the V-warp
-  // after its mix): more bytes stay in flight per SM.
-  // K and V halves of a tile travel separately, so each ring slot is refilled as soon
-  // as its own consumer is done with it (the K-warp after its scores, the V-warp
-  // after its mix).  Keys arrive by 2-D TMA tensor copies (swizzled), values by
-  // one 1-D bulk copy.
-  auto issue_k = [&](int k, uint64_t policy) {  // lane 0 of the K-warp
-    const int tok0 = t0 + (pair + k * NP) * kTile;
-    uint8_t* dst = my_kring + (size_t)(k % ns) * kt_bytes;
-    uint64_t* bar = &kfull[pair * ns + (k % ns)];
-    // whole 32-row boxes land (rows past the tile are masked out of the softmax)
-    mbar_arrive_expect_tx(bar, kt_bytes);
-    const int y = (int)(head_row0 + tok0);
-    for (int p = 0; p < a.npieces; ++p)
-      tma_load_2d(dst + a.kp[p].smem_off, &a.tmk[a.kp[p].map], a.kp[p].x, y, bar, policy);
+  // TMA parameters of the cache pieces (at most three per matrix), kept in registers
+  const void* kmap[3];
+  const void* vmap[3];
+  int kx[3], vx[3];
+  uint32_t ko[3], vo[3];
+#pragma unroll
+  for (int p = 0; p < 3; ++p) {
+    const int pk = p < a.pk.n ? p : 0, pv = p < a.pv.n ? p : 0;
+    kmap[p] = &a.maps[a.pk.p[pk].map];
+    kx[p] = a.pk.p[pk].x;
+    ko[p] = (uint32_t)a.pk.p[pk].smem_off;
+    vmap[p] = &a.maps[a.pv.p[pv].map];
+    vx[p] = a.pv.p[pv].x;
+    vo[p] = kt_bytes + (uint32_t)a.pv.p[pv].smem_off;
+  }
+  const int npk = a.pk.n, npv = a.pv.n;
+  auto issue = [&](int w, int k, uint64_t policy) {  // producer: tile k of consumer warp w
+    uint8_t* dst = smem + L.region + ((size_t)w * ns + (k % ns)) * st_bytes;
+    uint64_t* bar = &full[w * ns + (k % ns)];
+    // whole 32-row boxes land (rows past the sequence are masked on chip)
+    mbar_arrive_expect_tx(bar, st_bytes);
+    const int y = (int)(head_row0 + t0 + (w + k * NW) * kTile);
+#pragma unroll
+    for (int p = 0; p < 3; ++p)
+      if (p < npk) tma_load_2d(dst + ko[p], kmap[p], kx[p], y, bar, policy);
+#pragma unroll
+    for (int p = 0; p < 3; ++p)
+      if (p < npv) tma_load_2d(dst + vo[p], vmap[p], vx[p], y, bar, policy);
   };
-  auto issue_v = [&](int k, uint64_t policy) {  // lane 0 of the V-warp
-    const int tok0 = t0 + (pair + k * NP) * kTile;
-    const int n = min(kTile, t1 - tok0);
-    uint64_t* bar = &vfull[pair * ns + (k % ns)];
-    const uint32_t bytes = (uint32_t)n * rV * 2u;
-    mbar_arrive_expect_tx(bar, bytes);
-    bulk_g2s_hint(my_vring + (size_t)(k % ns) * vt_bytes, vbase_g + (size_t)tok0 * rV, bytes, bar,
-                  policy);
-  };
-  int issued = min(ns, my_tiles);  // tiles this warp has requested
-  {
-    const uint64_t policy = l2_policy_evict_first();
-    if (lane == 0)
-      for (int k = 0; k < issued; ++k) {
-        if (is_k) issue_k(k, policy);
-        else issue_v(k, policy);
-      }
-  }
 
-  // ---- q~ = q . P_K, scaled into the log2 domain -----------------------------------
-  // thread = (query head g, column pair cp, half of d); the two halves of a pair sit in
-  // adjacent lanes and are added with one shuffle.
-  bool ok = mbar_wait_bounded(setup_bar, 0, a.dev_status);
-  {
-    const int qstride = G_T * 8;  // floats per chunk row
-    const uint32_t* q2 = reinterpret_cast<const uint32_t*>(smem + L.q);
-    const uint32_t* pk2 = reinterpret_cast<const uint32_t*>(smem + L.scratch);
-    float* qt = reinterpret_cast<float*>(smem + L.qt);
-    const int half = rK / 2;  // column pairs
-    const int outs = G_T * half;
-    const int parts = NT >= 2 * outs ? 2 : 1;
-    const int total = outs * parts;
-    const int total_r = (total + 31) & ~31;  // whole warps take part in the shuffle
-    const int span = (d / 2) / parts;
-    for (int idx = tid; idx < total_r; idx += NT) {
-      const bool act = idx < total;
-      const int o = idx / parts, part = idx - o * parts;
-      const int g = o / half, cp = o - g * half;
-      float2 acc = f2(0.f, 0.f);
-      if (act && ok && g < gcount) {
-        const uint32_t* qrow = q2 + g * (d / 2);
-#pragma unroll 4
-        for (int i2 = part * span; i2 < (part + 1) * span; ++i2) {
-          const uint32_t qq = qrow[i2];  // q[2*i2], q[2*i2+1]
-          const uint32_t pa = pk2[(2 * i2) * half + cp];
-          const uint32_t pb = pk2[(2 * i2 + 1) * half + cp];
-          const float q0 = bf16lo(qq), q1 = bf16hi(qq);
-          acc = fma2(f2(q0, q0), f2(bf16lo(pa), bf16hi(pa)), acc);
-          acc = fma2(f2(q1, q1), f2(bf16lo(pb), bf16hi(pb)), acc);
-        }
-      }
-      if (parts == 2) {
-        acc.x += __shfl_xor_sync(0xffffffffu, acc.x, 1);
-        acc.y += __shfl_xor_sync(0xffffffffu, acc.y, 1);
-      }
-      if (act && part == 0) {
-        const int c = 2 * cp;
-        float* dst = qt + (c >> 3) * qstride + g * 8 + (c & 7);
-        dst[0] = acc.x * a.qscale;
-        dst[1] = acc.y * a.qscale;
-      }
+  // ---- prologue ------------------------------------------------------------------------------
+  bool ok = true;
+  if (producer) {
+    if (lane < 12 && lane < a.nmaps) prefetch_tensormap(&a.maps[lane]);
+    if (lane == 0) {
+      // q and P_K first (they gate q~), then every warp's ring
+      const uint64_t keep = l2_policy_evict_last();  // bases are shared by many CTAs
+      mbar_arrive_expect_tx(setup_bar, 2u * d * rK + 2u * gcount * d);
+      bulk_g2s(smem + L.qraw, a.q + ((size_t)b * a.Hq + h0) * d, 2u * gcount * d, setup_bar);
+      for (int p = 0; p < a.ppk.n; ++p)
+        tma_load_2d(pmat + a.ppk.p[p].smem_off, &a.maps[a.ppk.p[p].map], a.ppk.p[p].x, kvh * d,
+                    setup_bar, keep);
     }
-  }
-  __syncthreads();
-
-  // ---- streaming ------------------------------------------------------------------------
-  const int RV = rV >> 3;
-  const int TPW = 32 / RV;            // tokens per value step
-  const int vslot = lane / RV;
-  const bool vactive = vslot < TPW;
-  float* pbuf = reinterpret_cast<float*>(smem + L.scratch) + pair * 2 * kTile * G_T * 2;
-
-  float m_ref[G_T], l_lane[G_T];
-  float2 acc[G_T][4];
-#pragma unroll
-  for (int g = 0; g < G_T; ++g) {
-    m_ref[g] = -INFINITY;
-    l_lane[g] = 0.f;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) acc[g][e] = f2(0.f, 0.f);
-  }
-  int consumed = 0;
-
-  if (is_k) {
-    const uint32_t qstride_b = (uint32_t)G_T * 32u;
-    const uint32_t qt_addr = smem_u32(smem + L.qt);
-    const uint64_t policy = l2_policy_evict_first();
-    for (int k = 0; k < my_tiles && ok; ++k) {
-      const int stg = k % ns;
-      if (!mbar_wait_bounded(&kfull[pair * ns + stg], (uint32_t)((k / ns) & 1), a.dev_status)) {
-        ok = false;
-        break;
-      }
-      const int tok0 = t0 + (pair + k * NP) * kTile;
-      const int n = min(kTile, t1 - tok0);
-      const uint32_t kst = smem_u32(my_kring + (size_t)stg * kt_bytes);
-
-      // scores: lane = token; two chunks per iteration (RK is even); q~ chunk reads are
-      // warp-wide broadcasts
-      float s[G_T];
-      {
-        float2 sa[G_T], sb[G_T];
-#pragma unroll
-        for (int g = 0; g < G_T; ++g) {
-          sa[g] = f2(0.f, 0.f);
-          sb[g] = f2(0.f, 0.f);
-        }
-        for (int p = 0; p < a.npieces; ++p) {
-          const int w = a.kp[p].width;
-          const uint32_t prow = kst + (uint32_t)a.kp[p].smem_off + (uint32_t)lane * w * 2u;
-          const uint32_t q0 = qt_addr + (uint32_t)(a.kp[p].x >> 3) * qstride_b;
-          if (w == 64) score_piece<G_T, 8>(prow ^ ((uint32_t)(lane & 7) << 4), q0, sa, sb);
-          else if (w == 32) score_piece<G_T, 4>(prow ^ ((uint32_t)((lane >> 1) & 3) << 4), q0, sa, sb);
-          else score_piece<G_T, 2>(prow ^ ((uint32_t)((lane >> 2) & 1) << 4), q0, sa, sb);
-        }
-#pragma unroll
-        for (int g = 0; g < G_T; ++g) s[g] = (sa[g].x + sa[g].y) + (sb[g].x + sb[g].y);
-      }
-      // the key slot is free: request the keys of tile k + ns
-      __syncwarp();
-      consumed = k + 1;
-      if (k + ns < my_tiles) {
-        if (lane == 0) issue_k(k + ns, policy);
-        issued = k + ns + 1;
-      }
-
-      // online softmax (log2 domain), lazy rescale; factors go to the V-warp
-      const bool valid = lane < n;
-      float pw[G_T], fac[G_T];
-      bool rescaled = false;
-#pragma unroll
-      for (int g = 0; g < G_T; ++g) {
-        const float sg = valid ? s[g] : -INFINITY;
-        fac[g] = 1.f;
-        if (__any_sync(0xffffffffu, sg > m_ref[g] + kRescaleTau)) {
-          const float m_new = fmaxf(m_ref[g], warp_max(sg));
-          fac[g] = ex2(m_ref[g] - m_new);  // 0 when m_ref was -inf
-          l_lane[g] *= fac[g];
-          m_ref[g] = m_new;
-          rescaled = true;
-        }
-        pw[g] = valid ? ex2(sg - m_ref[g]) : 0.f;
-        l_lane[g] += pw[g];
-      }
-      const int pb = k & 1;
-      if (k >= 2 && !mbar_wait_bounded(&pempty[pair * 2 + pb], (uint32_t)(((k >> 1) - 1) & 1),
-                                       a.dev_status)) {
-        ok = false;
-        break;
-      }
-      float* pt = pbuf + pb * kTile * G_T * 2;
-      if constexpr (G_T >= 2) {
-#pragma unroll
-        for (int g2 = 0; g2 < G_T; g2 += 2)
-          *reinterpret_cast<float4*>(pt + (lane * G_T + g2) * 2) =
-              make_float4(pw[g2], pw[g2], pw[g2 + 1], pw[g2 + 1]);
-      } else {
-        *reinterpret_cast<float2*>(pt + lane * 2) = f2(pw[0], pw[0]);
-      }
-      if (lane == 0) {
-        float* fb = fbuf + pb * (G_T + 1);
-#pragma unroll
-        for (int g = 0; g < G_T; ++g) fb[g] = fac[g];
-        fb[G_T] = rescaled ? 1.f : 0.f;
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&pfull[pair * 2 + pb]);
+    __syncwarp();
+    if (lane < NW) {  // lane w requests consumer warp w's tiles
+      const uint64_t stream = l2_policy_evict_first();
+      for (int k = 0; k < min(min(kPreIssue, ns), warp_tiles(lane, spec_tiles)); ++k)
+        issue(lane, k, stream);
     }
+    __syncwarp();
   } else {
-    const uint64_t policy = l2_policy_evict_first();
+    // q~ = q P_K on the MMA: q~^T[j][head] = sum_i P_K[i][j] q[head][i]
+    // (M = the r_K columns of P_K, N = 8 heads, K = d), scaled into log2 units
+    const int n = lane >> 2;  // B column = head
+    ok = warp_wait(setup_bar, 0, a.dev_status);
+    uint32_t qb[8][2];  // d / 16 k-steps
+    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(smem + L.qraw) + min(n, gcount - 1) * (d / 2);
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      qb[ks][0] = n < gcount ? qrow[8 * ks + (lane & 3)] : 0u;
+      qb[ks][1] = n < gcount ? qrow[8 * ks + 4 + (lane & 3)] : 0u;
+    }
+    for (int mt = warp; mt < nks && ok; mt += NW) {
+      float c[4];
+      const PieceLoc pl = locate(rK, d, 2 * mt + at_chunk(lane));
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        uint32_t af[4];
+        ldsm_x4_t(smem_u32(pmat) + swz(pl, 16 * ks + at_row(lane)), af);
+        if (ks == 0) mma_bf16_z(c, af, qb[ks][0], qb[ks][1]);
+        else mma_bf16(c, af, qb[ks][0], qb[ks][1]);
+      }
+      const int j = 16 * mt + (lane >> 2), hh = 2 * (lane & 3);
+      qt[hh * xs + j] = c[0] * a.qscale;
+      qt[(hh + 1) * xs + j] = c[1] * a.qscale;
+      qt[hh * xs + j + 8] = c[2] * a.qscale;
+      qt[(hh + 1) * xs + j + 8] = c[3] * a.qscale;
+    }
+  }
+  __syncthreads();  // q~ is in shared memory and every read of P_K is done
+
+  // this lane's two heads (hA, hB = hA + 1) and, for NB == 1, its part of the MMA columns
+  const int hA = NB == 1 ? 2 * (lane & 1) : 2 * (lane & 3);
+  const bool lo_lane = NB == 1 && (lane & 2) != 0;
+  float mA = -INFINITY, mB = -INFINITY, lA = 0.f, lB = 0.f;
+  float oacc[NMV][NB][4];
+#pragma unroll
+  for (int mt = 0; mt < NMV; ++mt)
+#pragma unroll
+    for (int j = 0; j < NB; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) oacc[mt][j][e] = 0.f;
+
+  if (producer) {
+    // ---- producer: P_V, the rest of every ring, then refills as stages are released ----
+    if (lane == 0) {
+      fence_proxy_async_smem();  // P_V replaces P_K, read through the generic proxy above
+      const uint64_t keep = l2_policy_evict_last();
+      mbar_arrive_expect_tx(setup_bar, 2u * d * rV);
+      for (int p = 0; p < a.ppv.n; ++p)
+        tma_load_2d(pmat + a.ppv.p[p].smem_off, &a.maps[a.ppv.p[p].map], a.ppv.p[p].x, kvh * d,
+                    setup_bar, keep);
+    }
+    __syncwarp();
+    {
+      // Lane w serves consumer warp w: tile k goes into the stage the warp released after
+      // tile k - ns.  The lanes stay converged: every pass tests all their stages at once
+      // (non-blocking) and issues whatever is free, so one slow warp holds up no other.
+      const int w = lane;
+      const uint64_t stream = l2_policy_evict_first();
+      const int pre = min(kPreIssue, ns);
+      const int tiles_w = lane < NW ? warp_tiles(w, n_tiles) : 0;
+      for (int k = pre; k < min(ns, tiles_w); ++k) issue(w, k, stream);
+      int k = ns;
+      uint64_t last_progress = global_timer_ns();
+      while (__any_sync(kFull, k < tiles_w)) {
+        const bool ready = k < tiles_w && mbar_test(&empty[w * ns + (k % ns)], (uint32_t)((k / ns - 1) & 1));
+        if (ready) {
+          issue(w, k, stream);
+          ++k;
+        }
+        if (__any_sync(kFull, ready)) {
+          last_progress = global_timer_ns();
+        } else {
+          __nanosleep(64);
+          if (global_timer_ns() - last_progress > kWaitLimitNs) {  // the consumers gave up
+            if (lane == 0) report(a.dev_status, STIEF_DEV_WAIT_TIMEOUT);
+            break;
+          }
+        }
+      }
+      // tiles requested before seq_lens was known but past the sequence are never consumed:
+      // they must land before the region is reused
+      if (lane < NW) {
+        const int requested = min(pre, warp_tiles(w, spec_tiles));
+        for (int kk = tiles_w; kk < requested; ++kk) mbar_wait_bounded(&full[w * ns + kk], 0u, nullptr);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---- consumers: stream the warp's tiles ------------------------------------------------
+    const int my_tiles = warp_tiles(warp, n_tiles);
+    uint8_t* ring = smem + L.region + (size_t)warp * ns * st_bytes;
+    uint32_t qf[NKS][NB][2];  // B fragments of Q^T (hi / lo parts)
+#pragma unroll
+    for (int ks = 0; ks < NKS; ++ks)
+      if (ks < nks) bfrag_hilo<NB>(qt, xs, ks, lane, qf[ks]);
+    uint32_t koff[NKS], kstep[NKS], voff[NMV], vstep[NMV];
+#pragma unroll
+    for (int ks = 0; ks < NKS; ++ks) {
+      const PieceLoc pl = locate(rK, kTile, 2 * ks + a_chunk(lane));
+      koff[ks] = swz(pl, a_row(lane));
+      kstep[ks] = 32u * pl.w;  // 16 rows further (the swizzle repeats every 8 rows)
+    }
+#pragma unroll
+    for (int mt = 0; mt < NMV; ++mt) {
+      const PieceLoc pl = locate(rV, kTile, 2 * mt + at_chunk(lane));
+      voff[mt] = kt_bytes + swz(pl, at_row(lane));
+      vstep[mt] = 32u * pl.w;
+    }
+
     for (int k = 0; k < my_tiles && ok; ++k) {
-      const int pb = k & 1;
-      if (!mbar_wait_bounded(&pfull[pair * 2 + pb], (uint32_t)((k >> 1) & 1), a.dev_status) ||
-          !mbar_wait_bounded(&vfull[pair * ns + (k % ns)], (uint32_t)((k / ns) & 1), a.dev_status)) {
+      const int st = k % ns;
+      if (!warp_wait(&full[warp * ns + st], (uint32_t)((k / ns) & 1), a.dev_status)) {
         ok = false;
         break;
       }
-      const int tok0 = t0 + (pair + k * NP) * kTile;
+      const uint32_t sbase = smem_u32(ring + (size_t)st * st_bytes);
+      const int tok0 = t0 + (warp + k * NW) * kTile;
       const int n = min(kTile, t1 - tok0);
-      const uint32_t vst = smem_u32(my_vring + (size_t)(k % ns) * vt_bytes);
-      const float* fb = fbuf + pb * (G_T + 1);
-      if (fb[G_T] != 0.f) {
-#pragma unroll
-        for (int g = 0; g < G_T; ++g) {
-          const float f = fb[g];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) acc[g][e] = f2(acc[g][e].x * f, acc[g][e].y * f);
-        }
-      }
-      const uint32_t p_addr = smem_u32(pbuf + pb * kTile * G_T * 2);
-      switch (RV) {
-        case 2: mix_tile<G_T, 2>(vst, p_addr, n, lane, acc); break;
-        case 4: mix_tile<G_T, 4>(vst, p_addr, n, lane, acc); break;
-        case 6: mix_tile<G_T, 6>(vst, p_addr, n, lane, acc); break;
-        case 8: mix_tile<G_T, 8>(vst, p_addr, n, lane, acc); break;
-        case 10: mix_tile<G_T, 10>(vst, p_addr, n, lane, acc); break;
-        case 12: mix_tile<G_T, 12>(vst, p_addr, n, lane, acc); break;
-        case 14: mix_tile<G_T, 14>(vst, p_addr, n, lane, acc); break;
-        default: mix_tile<G_T, 16>(vst, p_addr, n, lane, acc); break;
-      }
-      __syncwarp();
-      consumed = k + 1;
-      if (lane == 0) {
-        mbar_arrive(&pempty[pair * 2 + pb]);
-        if (k + ns < my_tiles) {
-          issue_v(k + ns, policy);
-          issued = k + ns + 1;
-        }
-      }
-    }
-  }
-  // copies that were requested but not consumed (only after a timed-out wait) must land
-  // before the region is reused or the CTA exits
-  if (lane == 0)
-    for (int k = consumed; k < issued; ++k)
-      mbar_wait_bounded(&(is_k ? kfull : vfull)[pair * ns + (k % ns)], (uint32_t)((k / ns) & 1),
-                        nullptr);
 
-  // ---- merge the pairs ---------------------------------------------------------------
-  if (is_k) {
+      // Fragments are requested a group of k-steps (m-tiles) at a time, so their latencies
+      // overlap; asm volatile keeps the order written here.
+      // scores: c[mt][j][e] is token 16 mt + (lane >> 2) + 8 (e >> 1), column
+      // 2 (lane & 3) + (e & 1)
+      float c[MT][NB][4];
 #pragma unroll
-    for (int g = 0; g < G_T; ++g) {
-      const float lw = warp_sum(l_lane[g]);
-      if (lane == 0) {
-        ml[(pair * G_T + g) * 2 + 0] = m_ref[g];
-        ml[(pair * G_T + g) * 2 + 1] = lw;
-      }
-    }
-  }
-  __syncthreads();  // every pair is done with its stages: the region becomes the reduction buffer
-  // P_V for the up-projection: needed here when this CTA finishes the unit itself
-  if (tid == 0 && S == 1) {
-    fence_proxy_async_smem();
-    const uint32_t vbytes = 2u * d * rV;
-    mbar_arrive_expect_tx(setup_bar, vbytes);
-    bulk_g2s(smem + L.region + L.pv, a.P_V + (size_t)kvh * d * rV, vbytes, setup_bar);
-  }
-  float* red = reinterpret_cast<float*>(smem + L.region);
-  if (!is_k) {
-    float* mine = red + ((size_t)pair * 32 + lane) * G_T * 8;
+      for (int g0 = 0; g0 < NKS; g0 += KG)
+        if (g0 < nks) {
+          uint32_t kf[KG][MT][4];
 #pragma unroll
-    for (int g = 0; g < G_T; ++g)
+          for (int u = 0; u < KG; ++u)
+            if (g0 + u < nks) {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        mine[g * 8 + 2 * e] = vactive ? acc[g][e].x : 0.f;
-        mine[g * 8 + 2 * e + 1] = vactive ? acc[g][e].y : 0.f;
-      }
-  }
-  __syncthreads();
-
-  float* ot = reinterpret_cast<float*>(smem + L.scratch);  // o~ [G_T][rV] for the up-projection
-  const int part_stride = rV + 4;
-  float* parts = a.ws_part + unit * (size_t)S * G_T * part_stride;  // this unit's S x G_T states
-  for (int idx = tid; idx < G_T * rV; idx += NT) {
-    const int g = idx / rV, jj = idx - g * rV;
-    const int c = jj >> 3, e = jj & 7;
-    float M = -INFINITY;
-    for (int w = 0; w < NP; ++w) M = fmaxf(M, ml[(w * G_T + g) * 2]);
-    float o = 0.f, lsum = 0.f;
-    for (int w = 0; w < NP; ++w) {
-      const float mw = ml[(w * G_T + g) * 2];
-      const float sc = (mw == -INFINITY) ? 0.f : ex2(mw - M);
-      float part = 0.f;
-      for (int slot = 0; slot < TPW; ++slot)
-        part += red[((size_t)w * 32 + slot * RV + c) * G_T * 8 + g * 8 + e];
-      o = fmaf(sc, part, o);
-      lsum = fmaf(sc, ml[(w * G_T + g) * 2 + 1], lsum);
-    }
-    if (S == 1) {
-      ot[g * rV + jj] = lsum > 0.f ? o / lsum : 0.f;
-    } else {
-      float* pdst = parts + ((size_t)s_idx * G_T + g) * part_stride;
-      pdst[jj] = o;
-      if (jj == 0) {
-        pdst[rV] = M;
-        pdst[rV + 1] = lsum;
-      }
-    }
-  }
-
-  if (S > 1) {
-    // publish this split and take a ticket; the last CTA of the unit merges every split
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) {
-      const uint32_t ticket = atomicAdd(a.ws_cnt + unit, 1u);
-      const int last = ticket == (uint32_t)(S - 1);
-      if (last) {
-        a.ws_cnt[unit] = 0u;  // ready for the next call
-        fence_proxy_async_smem();
-        const uint32_t vbytes = 2u * d * rV;
-        mbar_arrive_expect_tx(setup_bar, vbytes);
-        bulk_g2s(smem + L.region + L.pv, a.P_V + (size_t)kvh * d * rV, vbytes, setup_bar);
-      }
-      *flag = last;
-    }
-    __syncthreads();
-    if (!*flag) return;
-    __threadfence();
-    // stage the unit's split states through shared memory (below P_V), a chunk of splits
-    // at a time, accumulating against a running maximum
-    float* stage_p = reinterpret_cast<float*>(smem + L.region);
-    const int per_split = G_T * part_stride;  // floats
-    const int s_chunk = max(1, (int)(L.pv / 4u) / per_split);
-    for (int s0 = 0; s0 < S; s0 += s_chunk) {
-      const int nsp = min(s_chunk, S - s0);
-      const int n4 = nsp * per_split / 4;
-      const float* src = parts + (size_t)s0 * per_split;
-      for (int i = tid; i < n4; i += NT * 4) {
-        float4 x[4];
+              for (int mt = 0; mt < MT; ++mt)
+                ldsm_x4(sbase + koff[g0 + u] + mt * kstep[g0 + u], kf[u][mt]);
+            }
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-          if (i + u * NT < n4) x[u] = ldcg4(src + 4 * (i + u * NT));
+          for (int u = 0; u < KG; ++u)
+            if (g0 + u < nks) {
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-          if (i + u * NT < n4) reinterpret_cast<float4*>(stage_p)[i + u * NT] = x[u];
-      }
-      __syncthreads();
-      if (tid < G_T) {
-        const float M_old = (s0 == 0) ? -INFINITY : fin[tid];
-        float M = M_old;
-        for (int s = 0; s < nsp; ++s) M = fmaxf(M, stage_p[(s * G_T + tid) * part_stride + rV]);
-        const float f = (M_old == -INFINITY) ? 0.f : ex2(M_old - M);
-        float lsum = (s0 == 0) ? 0.f : fin[G_T + tid] * f;
-        for (int s = 0; s < nsp; ++s) {
-          const float ms = stage_p[(s * G_T + tid) * part_stride + rV];
-          if (ms != -INFINITY) lsum = fmaf(ex2(ms - M), stage_p[(s * G_T + tid) * part_stride + rV + 1], lsum);
+              for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                for (int j = 0; j < NB; ++j) {
+                  if (g0 + u == 0) mma_bf16_z(c[mt][j], kf[u][mt], qf[0][j][0], qf[0][j][1]);
+                  else mma_bf16(c[mt][j], kf[u][mt], qf[g0 + u][j][0], qf[g0 + u][j][1]);
+                }
+            }
         }
-        fin[tid] = M;
-        fin[G_T + tid] = lsum;
-        fin[2 * G_T + tid] = f;  // rescale of what was accumulated before this chunk
-      }
-      __syncthreads();
-      const bool final_chunk = s0 + nsp >= S;
-      for (int idx = tid; idx < G_T * rV; idx += NT) {
-        const int g = idx / rV, jj = idx - g * rV;
-        const float M = fin[g];
-        float o = (s0 == 0) ? 0.f : ot[idx] * fin[2 * G_T + g];
-        if (M != -INFINITY)
-          for (int s = 0; s < nsp; ++s) {
-            const float ms = stage_p[(s * G_T + g) * part_stride + rV];
-            if (ms != -INFINITY) o = fmaf(ex2(ms - M), stage_p[(s * G_T + g) * part_stride + jj], o);
+      // value fragments do not depend on the scores: request the first group now
+      uint32_t vf[VG][MT][4];
+      auto load_v = [&](int g0) {
+#pragma unroll
+        for (int u = 0; u < VG; ++u)
+          if (g0 + u < nmv) {
+#pragma unroll
+            for (int kk = 0; kk < MT; ++kk)
+              ldsm_x4_t(sbase + voff[g0 + u] + kk * vstep[g0 + u], vf[u][kk]);
           }
-        if (final_chunk) {
-          const float lsum = fin[G_T + g];
-          o = lsum > 0.f ? o / lsum : 0.f;
+        if (n < kTile) {
+          // the sequence ends inside this tile: the value rows past it may hold anything
+          // (0 * NaN would reach the accumulators), so their fragment halves become zero.
+          // Register r of a fragment holds tokens 16 kk + 8 (r >> 1) + 2 (lane & 3) + {0, 1}.
+#pragma unroll
+          for (int u = 0; u < VG; ++u)
+#pragma unroll
+            for (int kk = 0; kk < MT; ++kk)
+#pragma unroll
+              for (int r = 0; r < 4; ++r) {
+                const int tok = 16 * kk + 8 * (r >> 1) + 2 * (lane & 3);
+                vf[u][kk][r] = tok + 1 < n ? vf[u][kk][r] : (tok < n ? (vf[u][kk][r] & 0xffffu) : 0u);
+              }
         }
-        ot[idx] = o;
+      };
+      load_v(0);
+      // add the hi and lo parts: s[mt][e] is the score of head hA + (e & 1)
+      float s[MT][4];
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          s[mt][e] = NB == 1 ? c[mt][0][e] + __shfl_xor_sync(kFull, c[mt][0][e], 2)
+                             : c[mt][0][e] + c[mt][NB - 1][e];
+      if (n < kTile) {  // missing tokens take no weight
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (16 * mt + (lane >> 2) + 8 * (e >> 1) >= n) s[mt][e] = -INFINITY;
       }
-      __syncthreads();
+
+      // online softmax, log2 domain.  The lane maxima are voted on first: only when some
+      // head passes its reference by more than the threshold are the maxima over the 8
+      // lanes sharing the heads formed and the accumulators rescaled.
+      float tA = fmaxf(s[0][0], s[0][2]), tB = fmaxf(s[0][1], s[0][3]);
+#pragma unroll
+      for (int mt = 1; mt < MT; ++mt) {
+        tA = fmaxf(tA, fmaxf(s[mt][0], s[mt][2]));
+        tB = fmaxf(tB, fmaxf(s[mt][1], s[mt][3]));
+      }
+      if (__any_sync(kFull, tA > mA + kRescaleTau || tB > mB + kRescaleTau)) {
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+          tA = fmaxf(tA, __shfl_xor_sync(kFull, tA, o));
+          tB = fmaxf(tB, __shfl_xor_sync(kFull, tB, o));
+        }
+        if (tA > mA + kRescaleTau) {
+          const float mn = fmaxf(mA, tA);
+          const float f = ex2(mA - mn);  // 0 while mA is -inf
+          lA *= f;
+          mA = mn;
+#pragma unroll
+          for (int mt = 0; mt < NMV; ++mt)
+#pragma unroll
+            for (int j = 0; j < NB; ++j) {
+              oacc[mt][j][0] *= f;
+              oacc[mt][j][2] *= f;
+            }
+        }
+        if (tB > mB + kRescaleTau) {
+          const float mn = fmaxf(mB, tB);
+          const float f = ex2(mB - mn);
+          lB *= f;
+          mB = mn;
+#pragma unroll
+          for (int mt = 0; mt < NMV; ++mt)
+#pragma unroll
+            for (int j = 0; j < NB; ++j) {
+              oacc[mt][j][1] *= f;
+              oacc[mt][j][3] *= f;
+            }
+        }
+      }
+      const float uA = mA == -INFINITY ? 0.f : mA, uB = mB == -INFINITY ? 0.f : mB;
+      // weights of the tile as B fragments of P^T: block r = tokens 8r..8r+7 in the score
+      // layout (row = token, columns = this lane's two heads), transposed to (token pairs, head)
+      uint32_t pb[NB][2 * MT];
+      float pa_sum = 0.f, pb_sum = 0.f;
+#pragma unroll
+      for (int r = 0; r < 2 * MT; ++r) {
+        const int mt = r >> 1, e0 = (r & 1) * 2;
+        const float pA = ex2(s[mt][e0] - uA), pB = ex2(s[mt][e0 + 1] - uB);
+        pa_sum += pA;
+        pb_sum += pB;
+        const uint32_t hw = hi_pair(pA, pB);
+        const uint32_t lw = lo_pair(pA, pB, hw);
+        if constexpr (NB == 1) {
+          pb[0][r] = movm_t(lo_lane ? lw : hw);
+        } else {
+          pb[0][r] = movm_t(hw);
+          pb[NB - 1][r] = movm_t(lw);
+        }
+      }
+      lA += pa_sum;
+      lB += pb_sum;
+
+      // value mix: O^T[dim][n] += V^T[dim][token] P^T[token][n]
+#pragma unroll
+      for (int g0 = 0; g0 < NMV; g0 += VG)
+        if (g0 < nmv) {
+          if (g0 > 0) load_v(g0);
+#pragma unroll
+          for (int u = 0; u < VG; ++u)
+            if (g0 + u < nmv) {
+#pragma unroll
+              for (int kk = 0; kk < MT; ++kk)
+#pragma unroll
+                for (int j = 0; j < NB; ++j)
+                  mma_bf16(oacc[g0 + u][j], vf[u][kk], pb[j][2 * kk], pb[j][2 * kk + 1]);
+            }
+        }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[warp * ns + st]);  // the stage may be refilled
+    }
+  }
+  pdl_launch_dependents();
+
+  // ---- merge the warps ------------------------------------------------------------------
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    lA += __shfl_xor_sync(kFull, lA, o);
+    lB += __shfl_xor_sync(kFull, lB, o);
+  }
+  float ov[NMV][4];  // o~ of (dim 16 mt + (lane >> 2) + 8 (e >> 1), head hA + (e & 1))
+#pragma unroll
+  for (int mt = 0; mt < NMV; ++mt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      ov[mt][e] = NB == 1 ? oacc[mt][0][e] + __shfl_xor_sync(kFull, oacc[mt][0][e], 2)
+                          : oacc[mt][0][e] + oacc[mt][NB - 1][e];
+  __syncthreads();  // every warp is done with its ring: the region becomes the reduction buffer
+  float* red = reinterpret_cast<float*>(smem + L.region);  // [NW][8][rV]
+  const int HR = NB == 1 ? 4 : 8;                          // heads the MMA columns carry
+  if (!producer && !lo_lane) {
+#pragma unroll
+    for (int mt = 0; mt < NMV; ++mt)
+      if (mt < nmv)
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          red[(warp * 8 + hA + (e & 1)) * rV + 16 * mt + (lane >> 2) + 8 * (e >> 1)] = ov[mt][e];
+    if ((lane >> 2) == 0) {
+      ml[(warp * 8 + hA) * 2] = mA;
+      ml[(warp * 8 + hA) * 2 + 1] = lA;
+      ml[(warp * 8 + hA + 1) * 2] = mB;
+      ml[(warp * 8 + hA + 1) * 2 + 1] = lB;
+    }
+  }
+  __syncthreads();
+  // o~ of the CTA (normalised when this CTA finishes the unit alone) becomes the B operand
+  // of the up-projection
+  for (int idx = tid; idx < HR * rV; idx += NT) {
+    const int h = idx / rV, jj = idx - h * rV;
+    float M = -INFINITY;
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, ml[(w * 8 + h) * 2]);
+    float o = 0.f, lsum = 0.f;
+    if (M != -INFINITY)
+      for (int w = 0; w < NW; ++w) {
+        const float mw = ml[(w * 8 + h) * 2];
+        if (mw != -INFINITY) {
+          const float f = ex2(mw - M);
+          o = fmaf(f, red[(w * 8 + h) * rV + jj], o);
+          lsum = fmaf(f, ml[(w * 8 + h) * 2 + 1], lsum);
+        }
+      }
+    if (S == 1) o = lsum > 0.f ? o / lsum : 0.f;
+    qt[h * xs + jj] = o;
+    if (jj == 0) {
+      fin[h] = M;
+      fin[8 + h] = lsum;
     }
   }
   __syncthreads();
 
-  // ---- up-projection o = o~ . P_V^T from shared memory, bf16 out --------------------------
-  if (!mbar_wait_bounded(setup_bar, 1, a.dev_status)) return;
-  {
-    const uint32_t pv_addr = smem_u32(smem + L.region + L.pv);
-    const int shv = (RV & 7) == 0 ? 0 : ((RV & 3) == 0 ? 1 : 2);
-    for (int idx = tid; idx < gcount * d; idx += NT) {
-      const int g = idx / d, i = idx - g * d;
-      const uint32_t prow = pv_addr + (uint32_t)i * rV * 2u;
-      const float* og = ot + g * rV;
-      int c = ((i & 7) >> shv) % RV;
-      float2 accv = f2(0.f, 0.f);
-      for (int jj = 0; jj < RV; ++jj) {
-        float2 pv[4];
-        unpack8(lds128(prow + c * 16u), pv);
-        const float4 x = *reinterpret_cast<const float4*>(og + c * 8);
-        const float4 y = *reinterpret_cast<const float4*>(og + c * 8 + 4);
-        accv = fma2(f2(x.x, x.y), pv[0], accv);
-        accv = fma2(f2(x.z, x.w), pv[1], accv);
-        accv = fma2(f2(y.x, y.y), pv[2], accv);
-        accv = fma2(f2(y.z, y.w), pv[3], accv);
-        c = (c + 1 == RV) ? 0 : c + 1;
+  // ---- up-projection o = o~ P_V^T on the MMA: o^T[i][n] = sum_j P_V[i][j] o~^T[j][n] ----
+  // (M = d, N = heads, K = r_V); warp w takes rows 16 w, 16 (w + NW + 1), ...
+  const int rec = d + 4;  // floats per partial state
+  float* parts = a.ws_part + unit * (size_t)S * G_T * rec;
+  if (!warp_wait(setup_bar, 1, a.dev_status)) ok = false;
+  for (int mt = warp; mt < d / 16 && ok; mt += NW + 1) {
+    float c[NB][4];
+#pragma unroll
+    for (int ks = 0; ks < NMV; ++ks)
+      if (ks < nmv) {
+        uint32_t af[4];
+        const PieceLoc pl = locate(rV, d, 2 * ks + a_chunk(lane));
+        ldsm_x4(smem_u32(pmat) + swz(pl, 16 * mt + a_row(lane)), af);
+        uint32_t bf[NB][2];
+        bfrag_hilo<NB>(qt, xs, ks, lane, bf);
+#pragma unroll
+        for (int j = 0; j < NB; ++j) {
+          if (ks == 0) mma_bf16_z(c[j], af, bf[j][0], bf[j][1]);
+          else mma_bf16(c[j], af, bf[j][0], bf[j][1]);
+        }
       }
-      a.out[((size_t)b * a.Hq + h0 + g) * d + i] = f32_to_bf16_rn(accv.x + accv.y);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float o = NB == 1 ? c[0][e] + __shfl_xor_sync(kFull, c[0][e], 2) : c[0][e] + c[NB - 1][e];
+      const int head = hA + (e & 1), i = 16 * mt + (lane >> 2) + 8 * (e >> 1);
+      if (!lo_lane && head < gcount) {
+        if (S == 1) a.out[((size_t)b * a.Hq + h0 + head) * d + i] = f32_to_bf16_rn(o);
+        else parts[((size_t)s_idx * G_T + head) * rec + i] = o;
+      }
+    }
+  }
+  if (S == 1) return;
+
+  // ---- split merge: publish this split, take a ticket; the last CTA merges them all ---------
+  if (tid < gcount) {
+    parts[((size_t)s_idx * G_T + tid) * rec + d] = fin[tid];
+    parts[((size_t)s_idx * G_T + tid) * rec + d + 1] = fin[8 + tid];
+  }
+  __syncthreads();  // every state of this CTA is written (block scope) ...
+  if (tid == 0) {
+    // ... and the acquire-release ticket makes them, by cumulativity, visible device-wide
+    // before the count moves; the last CTA's acquire orders its reads of the others' states
+    uint32_t ticket;
+    asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], 1;"
+                 : "=r"(ticket)
+                 : "l"(a.ws_cnt + unit)
+                 : "memory");
+    const int last = ticket == (uint32_t)(S - 1);
+    if (last) a.ws_cnt[unit] = 0u;  // ready for the next call
+    *flag = last;
+  }
+  __syncthreads();
+  if (!*flag) return;
+  // Thread groups of tpi consecutive lanes take one item = (head, 4 output columns); lane
+  // `sub` of a group merges splits sub, sub + tpi, ... (sixteen loads in flight at a time),
+  // then the group combines its tpi running states with shuffles.
+  const int nitems = gcount * (d / 4);
+  int tpi = 1;
+  while (tpi < 8 && tpi * 2 * nitems <= NT) tpi *= 2;
+  const int sub = tid & (tpi - 1);
+  const int iters = (nitems * tpi + NT - 1) / NT;
+  auto merge = [](float& M, float& Ls, float4& o, float m2, float l2, const float4& o2) {
+    if (m2 == -INFINITY) return;
+    if (m2 > M) {
+      const float f = ex2(M - m2);  // 0 while M is -inf
+      Ls *= f;
+      o.x *= f;
+      o.y *= f;
+      o.z *= f;
+      o.w *= f;
+      M = m2;
+    }
+    const float w = ex2(m2 - M);
+    Ls = fmaf(w, l2, Ls);
+    o.x = fmaf(w, o2.x, o.x);
+    o.y = fmaf(w, o2.y, o.y);
+    o.z = fmaf(w, o2.z, o.z);
+    o.w = fmaf(w, o2.w, o.w);
+  };
+  constexpr int kBatch = 16;
+  for (int it = 0; it < iters; ++it) {
+    const int item = (it * NT + tid) / tpi;
+    const bool valid = item < nitems;
+    const int g = valid ? item / (d / 4) : 0, c4 = valid ? item - g * (d / 4) : 0;
+    float M = -INFINITY, Ls = 0.f;
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s0 = sub; s0 < S; s0 += kBatch * tpi) {
+      float ms[kBatch], ls[kBatch];
+      float4 os[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int s = s0 + u * tpi;
+        if (valid && s < S) {
+          const float* r = parts + ((size_t)s * G_T + g) * rec;
+          const float2 m2 = __ldcg(reinterpret_cast<const float2*>(r + d));
+          ms[u] = m2.x;
+          ls[u] = m2.y;
+          os[u] = __ldcg(reinterpret_cast<const float4*>(r) + c4);
+        } else {
+          ms[u] = -INFINITY;
+          ls[u] = 0.f;
+          os[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) merge(M, Ls, o, ms[u], ls[u], os[u]);
+    }
+    for (int off = 1; off < tpi; off <<= 1) {
+      const float M2 = __shfl_xor_sync(kFull, M, off), L2 = __shfl_xor_sync(kFull, Ls, off);
+      float4 o2;
+      o2.x = __shfl_xor_sync(kFull, o.x, off);
+      o2.y = __shfl_xor_sync(kFull, o.y, off);
+      o2.z = __shfl_xor_sync(kFull, o.z, off);
+      o2.w = __shfl_xor_sync(kFull, o.w, off);
+      merge(M, Ls, o, M2, L2, o2);
+    }
+    if (valid && sub == 0) {
+      const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+      uint2 packed;
+      packed.x = pack_bf16x2_rn(o.x * inv, o.y * inv);
+      packed.y = pack_bf16x2_rn(o.z * inv, o.w * inv);
+      *reinterpret_cast<uint2*>(a.out + ((size_t)b * a.Hq + h0 + g) * d + 4 * c4) = packed;
     }
   }
 }
 
 // ------------------------------------------------------------------------------ launch
 
-template <int G_T, int NP>
+template <int NB, int NKS, int NMV, int TT>
 static cudaError_t launch_t(const DecodeArgs& a, cudaStream_t stream) {
-  const DecodeSmem L = decode_smem_layout(NP, a.nstage, G_T, a.d, a.rK, a.rV);
-  auto kern = stief_decode_kernel<G_T, NP>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
+  const DecodeSmem L = decode_smem_layout(a.nwarps, a.nstage, a.rK, a.rV, TT);
+  auto kern = stief_decode_kernel<NB, NKS, NMV, TT>;
+  static SmemLimit limit;
+  cudaError_t e = limit.ensure(reinterpret_cast<const void*>(kern), a.device, (int)L.total);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.S, a.Hkv * a.qsub, a.B);
-  cfg.blockDim = dim3(NP * 64);
+  cfg.blockDim = dim3((a.nwarps + 1) * 32);  // consumer warps + the producer warp
   cfg.dynamicSmemBytes = L.total;
   cfg.stream = stream;
+  // programmatic dependent launch: the CTAs may be scheduled while the previous kernel in
+  // the stream drains; they wait for it (griddepcontrol.wait) before reading any input
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = a.pdl_first ? 1 : 0;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
-uint32_t decode_smem_bytes(int NP, int nstage, int G_T, int d, int rK, int rV) {
-  return decode_smem_layout(NP, nstage, G_T, d, rK, rV).total;
+uint32_t decode_smem_bytes(int nwarps, int nstage, int rK, int rV, int tile) {
+  return decode_smem_layout(nwarps, nstage, rK, rV, tile).total;
+}
+
+template <int NB>
+static cudaError_t launch_nb(const DecodeArgs& a, cudaStream_t stream) {
+  const bool wk = a.rK > 64, wv = a.rV > 64;
+  if (a.tile == 64) {  // only small ranks (both <= 64, rK + rV <= 96) take 64-token tiles
+    if (wk || wv) return cudaErrorInvalidValue;
+    return launch_t<NB, 4, 4, 64>(a, stream);
+  }
+  if (!wk && !wv) return launch_t<NB, 4, 4, 32>(a, stream);
+  if (!wk) return launch_t<NB, 4, 8, 32>(a, stream);
+  if (!wv) return launch_t<NB, 8, 4, 32>(a, stream);
+  return launch_t<NB, 8, 8, 32>(a, stream);
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
-  switch (a.G_T) {
-    case 1: return a.npairs == 8 ? launch_t<1, 8>(a, stream) : launch_t<1, 4>(a, stream);
-    case 2: return a.npairs == 8 ? launch_t<2, 8>(a, stream) : launch_t<2, 4>(a, stream);
-    case 4: return a.npairs == 8 ? launch_t<4, 8>(a, stream) : launch_t<4, 4>(a, stream);
-    case 8: return a.npairs == 8 ? launch_t<8, 8>(a, stream) : launch_t<8, 4>(a, stream);
-    default: return cudaErrorInvalidValue;
-  }
+  return a.G_T <= 4 ? launch_nb<1>(a, stream) : launch_nb<2>(a, stream);
 }
 
 }  // namespace stief

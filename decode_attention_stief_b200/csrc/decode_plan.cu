@@ -32,16 +32,107 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D view of the key cache: [B*Hkv*L_max rows][rK columns] bf16, boxes of 32 rows x width.
-bool encode_key_map(CUtensorMap* map, const uint16_t* k_lat, int rK, uint64_t rows, int width) {
+// Tensor maps are pure functions of (base, r, rows, box rows, width); decoding the same
+// layer's cache over and over re-uses them from this table instead of re-encoding (an
+// encode costs on the order of a microsecond of host time per map).
+struct MapKey {
+  const void* base;
+  uint64_t rows;
+  int r, box_rows, width;
+  bool operator==(const MapKey& o) const {
+    return base == o.base && rows == o.rows && r == o.r && box_rows == o.box_rows && width == o.width;
+  }
+};
+constexpr int kMapCacheSlots = 1024;
+struct MapSlot {
+  MapKey key;
+  CUtensorMap map;
+  bool used;
+};
+std::mutex g_map_mu;
+MapSlot g_map_cache[kMapCacheSlots];
+
+bool cached_map(CUtensorMap* out, const void* base, int r, uint64_t rows, int box_rows, int width) {
+  const MapKey key{base, rows, r, box_rows, width};
+  uint64_t h = reinterpret_cast<uintptr_t>(base) * 0x9E3779B97F4A7C15ull;
+  h ^= rows * 0xC2B2AE3D27D4EB4Full + (uint64_t)r * 131 + (uint64_t)box_rows * 7 + (uint64_t)width;
+  h ^= h >> 29;
+  MapSlot& slot = g_map_cache[h % kMapCacheSlots];
+  {
+    std::lock_guard<std::mutex> lock(g_map_mu);
+    if (slot.used && slot.key == key) {
+      *out = slot.map;
+      return true;
+    }
+  }
   const CUtensorMapSwizzle sw = width == 64   ? CU_TENSOR_MAP_SWIZZLE_128B
                                 : width == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
                                               : CU_TENSOR_MAP_SWIZZLE_32B;
-  return encode_tiled_bf16_2d(map, k_lat, (uint64_t)rK, rows, (uint64_t)rK * 2u, (uint32_t)width,
-                              32u, sw);
+  if (!encode_tiled_bf16_2d(out, base, (uint64_t)r, rows, (uint64_t)r * 2u, (uint32_t)width,
+                            (uint32_t)box_rows, sw))
+    return false;
+  std::lock_guard<std::mutex> lock(g_map_mu);
+  slot.key = key;
+  slot.map = *out;
+  slot.used = true;
+  return true;
 }
 
+// Column pieces of a rank-r matrix (r a multiple of 16): widths 64, 64, 32, 16 taken in
+// that order while they fit, each with its own tensor map (one per width, shared by
+// the pieces of that width) over `base` viewed as [rows][r] bf16, boxes of
+// width x box_rows.  Pieces are stacked in shared memory in the same order.
+bool plan_pieces(DecodeArgs& a, int* nmaps, PieceSet& ps, const void* base, int r, uint64_t rows,
+                 int box_rows) {
+  int map_of_width[3] = {-1, -1, -1};  // for 64, 32, 16
+  int x = 0, off = 0;
+  ps.n = 0;
+  for (int w : {64, 64, 32, 16}) {
+    if (r - x < w) continue;
+    const int wi = w == 64 ? 0 : w == 32 ? 1 : 2;
+    if (map_of_width[wi] < 0) {
+      if (*nmaps >= 12) return false;
+      if (!cached_map(&a.maps[*nmaps], base, r, rows, box_rows, w)) return false;
+      map_of_width[wi] = (*nmaps)++;
+    }
+    Piece& p = ps.p[ps.n++];
+    p.x = x;
+    p.width = w;
+    p.smem_off = off;
+    p.map = map_of_width[wi];
+    x += w;
+    off += box_rows * w * 2;
+  }
+  return x == r;
+}
+
+struct DevInfo {
+  int sms;
+  bool sm100;
+  bool ok;
+};
+DevInfo g_dev_info[kMaxDevices];
+std::once_flag g_dev_once[kMaxDevices];
+
 }  // namespace
+
+bool query_device(int* dev_out, int* sms, bool* sm100) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  std::call_once(g_dev_once[dev], [dev] {
+    int major = 0, minor = 0, n = 0;
+    DevInfo di{0, false, false};
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
+      di = DevInfo{n, major == 10 && minor == 0, true};
+    g_dev_info[dev] = di;
+  });
+  *dev_out = dev;
+  *sms = g_dev_info[dev].sms;
+  *sm100 = g_dev_info[dev].sm100;
+  return g_dev_info[dev].ok;
+}
 
 bool encode_tiled_bf16_2d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
                           uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows,
@@ -76,19 +167,13 @@ stief_status plan_decode(DecodeArgs& a, const uint16_t* q, const uint16_t* P_K,
   const uint64_t rows = (uint64_t)B * Hkv * L_max;
   if (rows >= (1ull << 31)) return STIEF_ERR_INVALID_ARG;  // TMA row coordinates are int32
 
-  int dev = 0, major = 0, minor = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return STIEF_ERR_CUDA;
-  if (major != 10 || minor != 0) return STIEF_ERR_UNSUPPORTED_DEVICE;
+  int dev = 0, sms = 0;
+  bool sm100 = false;
+  if (!query_device(&dev, &sms, &sm100)) return STIEF_ERR_CUDA;
+  if (!sm100) return STIEF_ERR_UNSUPPORTED_DEVICE;
+  a.device = dev;
 
   a.q = q;
-  a.P_K = P_K;
-  a.P_V = P_V;
-  a.k_lat = k_lat;
-  a.v_lat = v_lat;
   a.seq_lens = seq_lens;
   a.out = out;
   a.dev_status = dev_status;
@@ -103,30 +188,22 @@ stief_status plan_decode(DecodeArgs& a, const uint16_t* q, const uint16_t* P_K,
   a.rV = rV;
   a.L_max = L_max;
   a.S = num_splits > 0 ? num_splits : stief_decode_auto_splits(B, Hq, Hkv, max_seq_len, sms);
+  a.max_seq_len = max_seq_len;
+  // tokens per split: the split's share rounded up to whole 32-token tiles, so that only
+  // the last tile of a sequence can be partial
+  a.tile = choose_decode_tile(rK, rV);
+  a.chunk = ((max_seq_len + a.S - 1) / a.S + a.tile - 1) / a.tile * a.tile;
   a.qscale = (float)(1.4426950408889634 / std::sqrt((double)d));
-  a.pdl_first = false;
-  if (!choose_decode_config(a.G_T, d, rK, rV, &a.npairs, &a.nstage)) return STIEF_ERR_INVALID_ARG;
+  if (!choose_decode_config(rK, rV, a.tile, &a.nwarps, &a.nstage)) return STIEF_ERR_INVALID_ARG;
 
-  // key pieces: widths 64, 32, 16 in decreasing order (rK is a multiple of 16)
-  int map_of_width[3] = {-1, -1, -1};  // for 64, 32, 16
-  int nmaps = 0, x = 0, off = 0;
-  a.npieces = 0;
-  for (int w : {64, 64, 32, 16}) {
-    if (rK - x < w) continue;
-    const int wi = w == 64 ? 0 : w == 32 ? 1 : 2;
-    if (map_of_width[wi] < 0) {
-      if (!encode_key_map(&a.tmk[nmaps], k_lat, rK, rows, w)) return STIEF_ERR_CUDA;
-      map_of_width[wi] = nmaps++;
-    }
-    KeyPiece& kp = a.kp[a.npieces++];
-    kp.x = x;
-    kp.width = w;
-    kp.smem_off = off;
-    kp.map = map_of_width[wi];
-    x += w;
-    off += 32 * w * 2;
-  }
-  if (x != rK) return STIEF_ERR_INVALID_ARG;
+  int nmaps = 0;
+  const uint64_t prow = (uint64_t)Hkv * d;
+  if (!plan_pieces(a, &nmaps, a.pk, k_lat, rK, rows, a.tile) ||
+      !plan_pieces(a, &nmaps, a.pv, v_lat, rV, rows, a.tile) ||
+      !plan_pieces(a, &nmaps, a.ppk, P_K, rK, prow, d) ||
+      !plan_pieces(a, &nmaps, a.ppv, P_V, rV, prow, d))
+    return STIEF_ERR_CUDA;
+  a.nmaps = nmaps;
   return STIEF_OK;
 }
 

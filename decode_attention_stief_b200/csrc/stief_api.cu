@@ -22,14 +22,11 @@ bool rank_ok(int r) { return r >= 16 && r <= kHeadDim && (r % 16) == 0; }
 
 int group_tile(int G) { return G <= 1 ? 1 : G <= 2 ? 2 : G <= 4 ? 4 : 8; }
 
-stief_status device_check() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return STIEF_ERR_CUDA;
-  int major = 0, minor = 0;
-  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
-    return STIEF_ERR_CUDA;
-  if (major != 10 || minor != 0) return STIEF_ERR_UNSUPPORTED_DEVICE;
+stief_status device_check(int* dev) {
+  int sms = 0;
+  bool sm100 = false;
+  if (!stief::query_device(dev, &sms, &sm100)) return STIEF_ERR_CUDA;
+  if (!sm100) return STIEF_ERR_UNSUPPORTED_DEVICE;
   return STIEF_OK;
 }
 
@@ -89,7 +86,7 @@ size_t stief_decode_workspace_bytes(int B, int Hq, int Hkv, int rV, int max_seq_
   const int G_T = group_tile(G);
   const int qsub = (G + G_T - 1) / G_T;
   const size_t units = (size_t)B * Hkv * qsub;
-  return stief::decode_ws_bytes(units, G_T, stief_decode_max_splits(max_seq_len), rV);
+  return stief::decode_ws_bytes(units, G_T, stief_decode_max_splits(max_seq_len), kHeadDim);
 }
 
 stief_status stief_compress_append(const uint16_t* k_new, const uint16_t* v_new,
@@ -105,9 +102,11 @@ stief_status stief_compress_append(const uint16_t* k_new, const uint16_t* v_new,
       !aligned16(k_lat) || !aligned16(v_lat))
     return STIEF_ERR_ALIGNMENT;
   if (T == 0) return STIEF_OK;
-  stief_status st = device_check();
+  int dev = 0;
+  stief_status st = device_check(&dev);
   if (st != STIEF_OK) return st;
   stief::CompressArgs a{};
+  a.device = dev;
   a.k_new = k_new;
   a.v_new = v_new;
   a.P_K = P_K;

@@ -2,6 +2,7 @@
 // C-ABI host code (stief_api.cu) and the kernel files.  Not a public header.
 #pragma once
 
+#include <atomic>
 #include <cstddef>
 #include <cstdint>
 #include <cuda.h>
@@ -11,37 +12,42 @@
 
 namespace stief {
 
-// One column piece of the key cache: keys are fetched by 2-D TMA tensor copies in
-// pieces 64, 32 or 16 columns wide, each with the matching 128-, 64- or 32-byte
-// shared-memory swizzle (widths decrease along the row).
-struct KeyPiece {
+// One column piece of a bf16 matrix fetched by 2-D TMA tensor copies: matrices of
+// rank r are read in pieces 64, 32 or 16 columns wide (widths decreasing along the
+// row), each landing with the matching 128-, 64- or 32-byte shared-memory swizzle,
+// so that eight rows of one 16-byte column chunk sit in eight different bank groups.
+struct Piece {
   int x;         // first column (a multiple of 16)
   int width;     // 64, 32 or 16 columns
-  int smem_off;  // byte offset inside a key slot
-  int map;       // index into DecodeArgs::tmk
+  int smem_off;  // byte offset of the piece inside the tile
+  int map;       // index into DecodeArgs::maps
+};
+struct PieceSet {
+  Piece p[4];
+  int n;
 };
 
 // Everything the decode kernel needs, validated by the host code.  Passed as a
 // __grid_constant__ parameter so the tensor maps can be addressed in place.
 struct DecodeArgs {
-  CUtensorMap tmk[3];  // key-cache maps for piece widths 64, 32, 16 (those in use)
-  KeyPiece kp[4];
-  int npieces;
+  CUtensorMap maps[12];  // per (matrix, piece width) in use
+  int nmaps;
+  PieceSet pk, pv;       // key / value cache tiles of 32 rows
+  PieceSet ppk, ppv;     // P_K / P_V of d rows
   const uint16_t* q;
-  const uint16_t* P_K;
-  const uint16_t* P_V;
-  const uint16_t* k_lat;
-  const uint16_t* v_lat;
   const int32_t* seq_lens;
   uint16_t* out;
   uint32_t* ws_cnt;  // [units] split tickets; zero between calls
-  float* ws_part;    // [units * S * G_T][rV + 4] partial states: o~[rV], m, l, 0, 0
+  float* ws_part;    // [units * S * G_T][d + 4] partial states: o[d] (up-projected), m, l, 0, 0
   uint32_t* dev_status;
   int B, Hq, Hkv, G, G_T, qsub, d, rK, rV, L_max, S;
-  int npairs;     // K-warp / V-warp pairs per CTA (4 or 8)
-  int nstage;     // shared-memory stages per pair
-  float qscale;   // log2(e) / sqrt(d), applied to q . P_K
-  bool pdl_first; // launch the split kernel as a programmatic dependent
+  int max_seq_len;  // host bound of seq_lens; the splits partition [0, S * chunk)
+  int chunk;        // tokens per split, a multiple of the 32-token tile
+  int tile;         // tokens per tile: 32, or 64 when rK + rV <= 96
+  int nwarps;       // consumer warps per CTA, each streaming its own tiles
+  int nstage;       // shared-memory stages per warp
+  float qscale;     // log2(e) / sqrt(d), applied to q . P_K
+  int device;       // current device at planning time (host bookkeeping only)
 };
 
 struct CompressArgs {
@@ -54,11 +60,33 @@ struct CompressArgs {
   int32_t* seq_lens;
   uint32_t* dev_status;
   int B, Hkv, T, d, rK, rV, L_max;
+  int device;  // current device (host bookkeeping only)
 };
 
 constexpr int kMaxSmemPerBlock = 232448;  // 227 KB opt-in dynamic shared memory (sm_100)
+constexpr int kMaxDevices = 64;
 
-uint32_t decode_smem_bytes(int NW, int nstage, int G_T, int d, int rK, int rV);
+// The current device, its SM count and whether it is sm_100 (queried once per device).
+// Returns false if the CUDA runtime cannot answer.  Host only.
+bool query_device(int* dev, int* sms, bool* sm100);
+
+// A kernel's dynamic shared-memory limit, raised once per device to the largest size
+// requested so far (cudaFuncSetAttribute is not repeated on every launch).
+struct SmemLimit {
+  std::atomic<int> set[kMaxDevices] = {};
+  cudaError_t ensure(const void* kern, int dev, int bytes) {
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    int cur = set[dev].load(std::memory_order_relaxed);
+    if (bytes <= cur) return cudaSuccess;
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    while (bytes > cur && !set[dev].compare_exchange_weak(cur, bytes)) {
+    }
+    return cudaSuccess;
+  }
+};
+
+uint32_t decode_smem_bytes(int nwarps, int nstage, int rK, int rV, int tile);
 
 // 2-D tiled TMA tensor map over a row-major bf16 matrix [rows][cols] (row stride in
 // bytes), boxes of box_cols x box_rows with the given swizzle.  Host only.
@@ -78,26 +106,27 @@ stief_status plan_decode(DecodeArgs& a, const uint16_t* q, const uint16_t* P_K,
                          uint32_t* dev_status);
 
 // Decode workspace layout: `units` = B * Hkv * qsub ticket counters (uint32, padded to
-// 256 bytes), then units * G_T * splits partial states of (rV + 4) floats.
+// 256 bytes), then units * G_T * splits partial states of (d + 4) floats.
 inline size_t decode_ws_counter_bytes(size_t units) { return (units * 4u + 255u) / 256u * 256u; }
-inline size_t decode_ws_bytes(size_t units, int G_T, int splits, int rV) {
-  return decode_ws_counter_bytes(units) + units * (size_t)G_T * splits * (size_t)(rV + 4) * 4u;
+inline size_t decode_ws_bytes(size_t units, int G_T, int splits, int d) {
+  return decode_ws_counter_bytes(units) + units * (size_t)G_T * splits * (size_t)(d + 4) * 4u;
 }
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
 
-// Pairs per CTA and stages per pair for the decode kernel: at least 3 stages per pair
-// (one tile in the K-warp, one in the V-warp, one in flight) where shared memory allows,
-// 8 pairs unless G_T == 8 (whose 8-pair build would spill), else the widest that fits.
-inline bool choose_decode_config(int G_T, int d, int rK, int rV, int* npairs, int* nstage) {
-  const int first = G_T == 8 ? 4 : 8;
-  for (int min_ns : {3, 2})
-    for (int np : {first, 4})
-      for (int ns = 4; ns >= min_ns; --ns)
-        if (decode_smem_bytes(np, ns, G_T, d, rK, rV) <= (uint32_t)kMaxSmemPerBlock) {
-          *npairs = np;
-          *nstage = ns;
-          return true;
-        }
+// Tokens per tile: 64 for small ranks (an SM sustains a roughly fixed number of tiles per
+// microsecond, so small tiles would leave the memory system idle), 32 otherwise.
+inline int choose_decode_tile(int rK, int rV) { return rK <= 64 && rV <= 64 && rK + rV <= 96 ? 64 : 32; }
+
+// Consumer warps per CTA and stages per warp for the decode kernel: 8 warps with as many
+// stages (up to 8) as shared memory allows, fewer warps only when 8 cannot have two each.
+inline bool choose_decode_config(int rK, int rV, int tile, int* nwarps, int* nstage) {
+  for (int nw = 8; nw >= 2; --nw)
+    for (int ns = 8; ns >= 2; --ns)
+      if (decode_smem_bytes(nw, ns, rK, rV, tile) <= (uint32_t)kMaxSmemPerBlock) {
+        *nwarps = nw;
+        *nstage = ns;
+        return true;
+      }
   return false;
 }
 cudaError_t launch_compress(const CompressArgs& a, cudaStream_t stream);

@@ -38,7 +38,7 @@
 namespace {
 
 constexpr size_t kScratchBytes = size_t(8) << 20;
-constexpr int kMaxDevices = 64;
+using stief::kMaxDevices;
 
 __device__ __align__(256) float g_decode_scratch[kScratchBytes / sizeof(float)];
 
@@ -74,7 +74,7 @@ extern "C" STIEF_API stief_status stief_decode_attention_noalloc(
 
   // ticket counters and the partial states of the split count actually used must fit
   const size_t units = (size_t)B * Hkv * a.qsub;
-  if (stief::decode_ws_bytes(units, a.G_T, a.S, rV) > kScratchBytes) return STIEF_ERR_WORKSPACE;
+  if (stief::decode_ws_bytes(units, a.G_T, a.S, a.d) > kScratchBytes) return STIEF_ERR_WORKSPACE;
 
   void* scratch = nullptr;
   st = scratch_address(&scratch);

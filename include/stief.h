@@ -124,8 +124,10 @@ STIEF_API int stief_decode_auto_splits(int B, int Hq, int Hkv, int max_seq_len, 
  * needs for these sizes, for any split count it may use (at most
  * stief_decode_max_splits(max_seq_len)).  The workspace holds one ticket counter
  * per (sequence, KV head, query sub-group) followed by the per-split partial
- * softmax states (running maximum, sum and unnormalised latent output).  Pure host
- * function.  Returns 0 for invalid arguments.
+ * states: for each query head, the split's up-projected unnormalised output
+ * (d floats), its running maximum and sum, and two pad words.  rV is validated
+ * but does not change the size.  Pure host function.  Returns 0 for invalid
+ * arguments.
  */
 STIEF_API size_t stief_decode_workspace_bytes(int B, int Hq, int Hkv, int rV, int max_seq_len);
 
@@ -138,20 +140,25 @@ STIEF_API size_t stief_decode_workspace_bytes(int B, int Hq, int Hkv, int rV, in
  *     s_t = q[b][h] . K~_t / sqrt(d)                       t < L
  *     out[b][h] = bf16_RNE( sum_t softmax(s)_t V~_t )
  * computed without materialising K~ or V~:
- *     q~ = q[b][h] . P_K[g]                  (fp32, per CTA)
+ *     q~ = q[b][h] . P_K[g]                  (per CTA)
  *     s_t = q~ . K_down[b][g][t] / sqrt(d)
- *     o~ = sum_t softmax(s)_t V_down[b][g][t] (split-KV, online softmax, fp32)
+ *     o~ = sum_t softmax(s)_t V_down[b][g][t] (split-KV, online softmax)
  *     out[b][h] = o~ . P_V[g]^T
  * which equals the definition up to rounding by associativity of the products,
  * (q . P_K) . K_down[t] = q . (K_down[t] . P_K^T) and
  * (sum_t p_t V_down[t]) . P_V^T = sum_t p_t (V_down[t] . P_V^T);
- * orthonormality of the bases is not needed for this.
- * L == 0 gives out = 0.  Rows at or beyond seq_lens[b] are never read.
+ * orthonormality of the bases is not needed for this.  The products run on the
+ * tensor cores with fp32 accumulation; q~, the softmax weights and o~ enter them
+ * as a bf16 pair (rounding plus rounded residual), about 16 significant bits.
+ * L == 0 gives out = 0.  Rows at or beyond seq_lens[b] do not affect the result
+ * (they may be fetched with a 32-row tile, and are masked and zeroed on chip).
  *
  *   q            : bf16 [B][Hq][d]
  *   P_K, P_V     : bf16 [Hkv][d][rK], [Hkv][d][rV]
  *   k_lat, v_lat : bf16 [B][Hkv][L_max][rK], [B][Hkv][L_max][rV]
- *   seq_lens     : int32 [B] on the device, each in [0, max_seq_len]
+ *   seq_lens     : int32 [B] on the device, each in [0, max_seq_len]; a length
+ *                  outside that range sets STIEF_DEV_BAD_LENGTH in *dev_status
+ *                  and gives out = 0 for that sequence
  *   out          : bf16 [B][Hq][d] (written)
  *   workspace    : device scratch of at least workspace_bytes >=
  *                  stief_decode_workspace_bytes(B, Hq, Hkv, rV, max_seq_len)
@@ -165,9 +172,11 @@ STIEF_API size_t stief_decode_workspace_bytes(int B, int Hq, int Hkv, int rV, in
  *                  (1 .. stief_decode_max_splits(max_seq_len))
  *
  * One kernel runs on `stream`, a CTA per (split, KV head, query sub-group,
- * sequence): query projection, scores, online softmax and latent value mix over
- * its token range; the last CTA of each (sequence, KV head, sub-group) to finish
- * merges the splits (log-sum-exp) and up-projects with P_V^T.
+ * sequence): query projection, scores, online softmax, latent value mix and
+ * up-projection over its token range; the last CTA of each (sequence, KV head,
+ * sub-group) to finish merges the splits (log-sum-exp).  The kernel is launched
+ * as a programmatic dependent of the preceding work in the stream: it may be
+ * scheduled while that work drains but reads no input before it has completed.
  * Returns STIEF_OK or an argument error (nothing launched).
  */
 STIEF_API stief_status stief_decode_attention(const uint16_t* q, const uint16_t* P_K,
@@ -190,7 +199,7 @@ STIEF_API stief_status stief_decode_attention(const uint16_t* q, const uint16_t*
  * workspace / workspace_bytes.  The per-split partial states live in a fixed 8 MiB
  * array of device memory owned by the library (one per GPU that loads it, held
  * until the process exits).  Sizes whose partial states, for the split count
- * actually used, exceed 8 MiB -- B*Hkv*ceil(G/G_T)*G_T*splits*(rV+4)*4 bytes with
+ * actually used, exceed 8 MiB -- B*Hkv*ceil(G/G_T)*G_T*splits*(d+4)*4 bytes with
  * G = Hq/Hkv and G_T the smallest of 1, 2, 4, 8 that is >= min(G, 8) -- plus the
  * ticket counters, return
  * STIEF_ERR_WORKSPACE and launch nothing.  The first call on each device looks up
