@@ -198,7 +198,8 @@ def run_gpu(args, w: si.Workload):
     R = replica_count(w)
     reps = []
     for r in range(R):
-        layers, L_max = build_state(w, W + K + 8, seed + 104729 * r, dev)
+        # room for every append of the warm-up, timed and kernel-timing runs of a replica
+        layers, L_max = build_state(w, W + K + 2 * args.decode_iters + 64, seed + 104729 * r, dev)
         reps.append(layers)
     layers = reps[0]
     g = torch.Generator(device=dev)
@@ -210,19 +211,31 @@ def run_gpu(args, w: si.Workload):
     out = torch.empty((len(layers), w.B, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
 
-    def step(lays):
-        for li, lay in enumerate(lays):
+    def layer_step(li, lay):
+        if args.unfused:  # the two separate calls (three kernels)
             stief.stief_compress_append(k_s, v_s, lay.P_K, lay.P_V, lay.k_lat, lay.v_lat,
                                         lay.seq_lens, dev_status=status)
             stief.stief_decode_attention(q_s, lay.P_K, lay.P_V, lay.k_lat, lay.v_lat,
                                          lay.seq_lens, out[li], lay.ws, max_seq_len=L_max,
                                          num_splits=args.splits, dev_status=status)
+        else:  # append + decode in one kernel
+            stief.stief_append_decode(q_s, k_s, v_s, lay.P_K, lay.P_V, lay.k_lat, lay.v_lat,
+                                      lay.seq_lens, out[li], lay.ws, max_seq_len=L_max,
+                                      num_splits=args.splits, dev_status=status)
+
+    def step(lays):
+        for li, lay in enumerate(lays):
+            layer_step(li, lay)
 
     def decode_only(lays):
+        """One launch of the step's attention kernel on layer 0 (for the kernel's own timing)."""
         lay = lays[0]
-        stief.stief_decode_attention(q_s, lay.P_K, lay.P_V, lay.k_lat, lay.v_lat, lay.seq_lens,
-                                     out[0], lay.ws, max_seq_len=L_max, num_splits=args.splits,
-                                     dev_status=status)
+        if args.unfused:
+            stief.stief_decode_attention(q_s, lay.P_K, lay.P_V, lay.k_lat, lay.v_lat,
+                                         lay.seq_lens, out[0], lay.ws, max_seq_len=L_max,
+                                         num_splits=args.splits, dev_status=status)
+        else:
+            layer_step(0, lay)
 
     def reset_lengths(L0):
         for lays in reps:
@@ -247,7 +260,11 @@ def run_gpu(args, w: si.Workload):
     cap = torch.cuda.Stream(device=dev)
     cap.wait_stream(torch.cuda.current_stream())
     step_graphs, e2e_graphs = [], []
+    cycle_graph = torch.cuda.CUDAGraph()  # one step on every replica in turn
     with torch.cuda.stream(cap):
+        with torch.cuda.graph(cycle_graph, stream=cap):
+            for r in range(R):
+                step(reps[r])
         for r in range(R):
             gr = torch.cuda.CUDAGraph()
             with torch.cuda.graph(gr, stream=cap):
@@ -265,6 +282,14 @@ def run_gpu(args, w: si.Workload):
         with torch.cuda.graph(dec_graph, stream=cap):
             for i in range(n_dec):
                 decode_only(reps[i % R])
+        # load for the clock samples: attention without appends (lengths stay put)
+        warm_graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(warm_graph, stream=cap):
+            for i in range(n_dec):
+                lay = reps[i % R][0]
+                stief.stief_decode_attention(q_s, lay.P_K, lay.P_V, lay.k_lat, lay.v_lat,
+                                             lay.seq_lens, out[0], lay.ws, max_seq_len=L_max,
+                                             dev_status=status)
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
 
@@ -275,8 +300,7 @@ def run_gpu(args, w: si.Workload):
         step_graphs[i % R].replay()
     reset_lengths(w.L - 1)
     torch.cuda.synchronize()
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(K)]
+    t0_ev, t1_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     cvd = os.environ.get("CUDA_VISIBLE_DEVICES")
     smi_id = cvd.split(",")[local].strip() if cvd else str(local)
     with ClockSampler(smi_id) as clk:
@@ -285,22 +309,24 @@ def run_gpu(args, w: si.Workload):
         t_keep = time.perf_counter()
         while time.perf_counter() - t_keep < args.clock_window:
             for _ in range(10):
-                dec_graph.replay()
+                warm_graph.replay()
             torch.cuda.synchronize()
         barrier()
         torch.cuda.synchronize()
         t_wall0 = time.perf_counter()
         _backlog()
-        for j in range(K):
-            evs[j][0].record(stream)
-            step_graphs[j % R].replay()
-            evs[j][1].record(stream)
+        # exactly K steps: K // R replays of the R-step cycle, then single steps
+        t0_ev.record(stream)
+        for _ in range(K // R):
+            cycle_graph.replay()
+        for j in range(K % R):
+            step_graphs[j].replay()
+        t1_ev.record(stream)
         torch.cuda.synchronize()
         barrier()
         t_wall = time.perf_counter() - t_wall0
         time.sleep(0.25)  # one more sample after the timed region
-    step_ms = [a.elapsed_time(b) for a, b in evs]
-    ms_per_step = sum(step_ms) / K
+    ms_per_step = t0_ev.elapsed_time(t1_ev) / K
     clocks = clk.summary()
     st = stief.stief_read_device_status(status)
     if st != 0:
@@ -309,8 +335,10 @@ def run_gpu(args, w: si.Workload):
     ctx_first, ctx_last = w.L, int(max(int(lays[0].seq_lens[0].item()) for lays in reps))
 
     # ---- decode kernel timing for the roofline: runs of n_dec back-to-back launches
-    # (replicas rotating), averaged over the timed region; plus single launches
-    reset_lengths(L_dec)
+    # (replicas rotating), averaged over the timed region; plus single launches.  The fused
+    # kernel appends a token per launch: lengths restart at L_dec - 1 for each run.
+    L_run0 = L_dec - (0 if args.unfused else 1)
+    reset_lengths(L_run0)
     dec_reps = max(3, args.decode_iters // n_dec)
     torch.cuda.synchronize()
     _backlog()
@@ -321,6 +349,8 @@ def run_gpu(args, w: si.Workload):
     d1.record(stream)
     torch.cuda.synchronize()
     dec_us = d0.elapsed_time(d1) * 1e3 / (dec_reps * n_dec)
+    L_dec_mean = L_dec + (0 if args.unfused else (dec_reps * n_dec // R) / 2)
+    reset_lengths(L_run0)
     iso = []
     for j in range(max(5, min(args.decode_iters, 30))):
         _backlog()
@@ -339,18 +369,17 @@ def run_gpu(args, w: si.Workload):
     for i in range(W):
         e2e_graphs[i % R].replay()
     reset_lengths(w.L - 1)
-    e2e_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(K)]
+    e0_ev, e1_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     _backlog()
+    e0_ev.record(stream)
     for j in range(K):
-        e2e_evs[j][0].record(stream)
         e2e_graphs[j % R].replay()
-        e2e_evs[j][1].record(stream)
+    e1_ev.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_evs) / K
+    e2e_ms = e0_ev.elapsed_time(e1_ev) / K
     h2d = (q_s.numel() + k_s.numel() + v_s.numel()) * 2
     d2h = out.numel() * 2
     st = stief.stief_read_device_status(status)
@@ -361,7 +390,7 @@ def run_gpu(args, w: si.Workload):
         t = torch.tensor([ms_per_step, e2e_ms, dec_us], device=dev, dtype=torch.float64)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         ms_per_step, e2e_ms, dec_us = (float(x) for x in t.tolist())
-    del step_graphs, e2e_graphs, dec_graph
+    del step_graphs, e2e_graphs, dec_graph, warm_graph, cycle_graph
 
     # ---- prefill compress (the prefill + batched decode workload): one 4096-token chunk
     # per layer through stief_compress_append (tcgen05 path), timed separately
@@ -373,7 +402,7 @@ def run_gpu(args, w: si.Workload):
     tokens_per_step = w.B * ws_n
     value = tokens_per_step / (ms_per_step / 1e3)
     lay0 = layers[0]
-    bytes_per_dec = 2 * (lay0.rK + lay0.rV) * w.B * w.Hkv * L_dec
+    bytes_per_dec = int(2 * (lay0.rK + lay0.rV) * w.B * w.Hkv * L_dec_mean)
     achieved = bytes_per_dec / (dec_us / 1e6) / 1e9
     peak, peak_kind = _hbm_peak()
     step_bytes = sum(2 * (lay.rK + lay.rV) * w.B * w.Hkv for lay in layers) * (
@@ -396,8 +425,11 @@ def run_gpu(args, w: si.Workload):
             "workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "context": w.L,
             "layers": len(layers), "ranks": [list(r) for r in w.layer_ranks()][:4]
             + (["..."] if len(layers) > 4 else []),
-            "step": "append 1 token per (sequence, KV head) + decode, every layer; one CUDA "
-                    "graph replay of the API calls",
+            "step": ("append 1 token per (sequence, KV head) + decode, every layer; the API "
+                     "calls captured in CUDA graphs (one step per replica, the timed region "
+                     "replays the replica cycle back to back); " +
+                     ("stief_compress_append + stief_decode_attention (3 kernels per layer)"
+                      if args.unfused else "stief_append_decode (1 kernel per layer)")),
             "context_growth": f"+1 token per step of a replica (contexts {ctx_first}..{ctx_last})",
             "l2": (f"no flush: steps rotate over {R} copies of the layer caches "
                    f"({rot_mb:.0f} MiB in all, > 3x the 126 MB L2)" if R > 1 else
@@ -408,7 +440,8 @@ def run_gpu(args, w: si.Workload):
         },
         "hbm_gbs_step": round(step_bytes / (ms_per_step / 1e3) / 1e9, 1),
         "roofline": {
-            "kernel": "stief_decode_kernel (stief_decode_attention)",
+            "kernel": "stief_decode_kernel (" + ("stief_decode_attention" if args.unfused
+                                                 else "stief_append_decode") + ")",
             "bound": "hbm",
             "achieved": round(achieved, 1),
             "peak": peak,
@@ -427,7 +460,7 @@ def run_gpu(args, w: si.Workload):
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "how": "per step one CUDA-graph replay of the public API calls with the "
                        "pinned host copies (inputs H2D, outputs D2H) inside"},
-        "gpu_launches": 3 * len(layers) * K,  # compress rows, length update, decode
+        "gpu_launches": (3 if args.unfused else 1) * len(layers) * K,
         "clocks": clocks,
         "wall_s_timed_region": round(t_wall, 3),
     }
@@ -602,6 +635,9 @@ def main():
                     help="diagnostics: run only the first N layers of the workload")
     ap.add_argument("--splits", type=int, default=0,
                     help="diagnostics: force the decode split count (0 = automatic)")
+    ap.add_argument("--unfused", action="store_true",
+                    help="time the step as the two separate calls (append kernel, length "
+                         "update, decode) instead of stief_append_decode")
     ap.add_argument("--clock-window", type=float, default=0.6,
                     help="seconds of untimed decode load before the timed region")
     args = ap.parse_args()

@@ -13,6 +13,7 @@ from ._binding import (  # noqa: F401
     DEV_BAD_LENGTH,
     library,
     library_path,
+    stief_append_decode,
     stief_compress_append,
     stief_decode_attention,
     stief_decode_attention_noalloc,

@@ -73,6 +73,9 @@ def library() -> ctypes.CDLL:
             lib.stief_decode_max_splits.argtypes = [_i]
             lib.stief_decode_auto_splits.restype = _i
             lib.stief_decode_auto_splits.argtypes = [_i] * 5
+            lib.stief_append_decode.restype = _i
+            lib.stief_append_decode.argtypes = ([vp] * 10 + [ctypes.c_size_t] + [_i] * 9
+                                                + [vp, vp])
             lib.stief_decode_attention_noalloc.restype = _i
             lib.stief_decode_attention_noalloc.argtypes = [vp] * 7 + [_i] * 9 + [vp, vp]
             lib.stief_read_device_status.restype = _i
@@ -212,6 +215,50 @@ def stief_decode_attention(q: torch.Tensor, P_K: torch.Tensor, P_V: torch.Tensor
                                             rV, L_max, int(max_seq_len), int(num_splits),
                                             _opt_status(dev_status), _stream_ptr(stream))
     _check("stief_decode_attention", code)
+    return out
+
+
+def stief_append_decode(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                        P_K: torch.Tensor, P_V: torch.Tensor, k_lat: torch.Tensor,
+                        v_lat: torch.Tensor, seq_lens: torch.Tensor, out: torch.Tensor,
+                        workspace: torch.Tensor, max_seq_len: int, num_splits: int = 0,
+                        dev_status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """One whole decode step in one kernel: append the new token's compressed key and value
+    rows (k_new P_K, v_new P_V at row seq_lens[b]), attend over the grown cache, and
+    increment seq_lens.
+
+    q [B][Hq][d] bf16; k_new, v_new [B][Hkv][d] (or [B][Hkv][1][d]) bf16; the other
+    arguments as for stief_decode_attention; max_seq_len bounds the lengths after the append.
+    """
+    pq = _dev(q, "q", torch.bfloat16, 3)
+    kn = k_new.reshape(k_new.shape[0], k_new.shape[1], -1) if k_new.dim() == 4 else k_new
+    vn = v_new.reshape(v_new.shape[0], v_new.shape[1], -1) if v_new.dim() == 4 else v_new
+    pkn = _dev(kn, "k_new", torch.bfloat16, 3)
+    pvn = _dev(vn, "v_new", torch.bfloat16, 3)
+    ppk = _dev(P_K, "P_K", torch.bfloat16, 3)
+    ppv = _dev(P_V, "P_V", torch.bfloat16, 3)
+    pkl = _dev(k_lat, "k_lat", torch.bfloat16, 4)
+    pvl = _dev(v_lat, "v_lat", torch.bfloat16, 4)
+    psl = _dev(seq_lens, "seq_lens", torch.int32, 1)
+    po = _dev(out, "out", torch.bfloat16, 3)
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    B, Hq, d = q.shape
+    Hkv, _, rK = P_K.shape
+    rV = P_V.shape[2]
+    L_max = k_lat.shape[2]
+    if tuple(P_K.shape) != (Hkv, d, rK) or tuple(P_V.shape) != (Hkv, d, rV) \
+            or tuple(kn.shape) != (B, Hkv, d) or tuple(vn.shape) != (B, Hkv, d) \
+            or tuple(k_lat.shape) != (B, Hkv, L_max, rK) \
+            or tuple(v_lat.shape) != (B, Hkv, L_max, rV) or seq_lens.shape[0] != B \
+            or tuple(out.shape) != (B, Hq, d):
+        raise ValueError("stief_append_decode: inconsistent shapes")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    code = library().stief_append_decode(pq, pkn, pvn, ppk, ppv, pkl, pvl, psl, po,
+                                         workspace.data_ptr(), ws_bytes, B, Hq, Hkv, d, rK, rV,
+                                         L_max, int(max_seq_len), int(num_splits),
+                                         _opt_status(dev_status), _stream_ptr(stream))
+    _check("stief_append_decode", code)
     return out
 
 

@@ -183,9 +183,11 @@ __host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) { return (x
 // Shared-memory carve-up (byte offsets from the dynamic base).
 struct DecodeSmem {
   uint32_t bars;    // nwarps*nstage "full" and nwarps*nstage "empty" stage barriers, then
-                    // 1 setup barrier (q and P_K, then P_V)
+                    // the setup barrier (q and P_K, then P_V) and the new-row barrier
   uint32_t ml;      // [nwarps][8] (m, l); then [8] M, [8] L; then a flag
   uint32_t qraw;    // [G_T][d] bf16 query rows
+  uint32_t newraw;  // append: the new token's k and v rows, bf16 [2][d]
+  uint32_t newlat;  // append: its projected key and value rows, bf16 [rK] then [rV]
   uint32_t qt;      // [8][xs] fp32: q~ (prologue), o~ (epilogue)
   uint32_t pmat;    // P_K (prologue), then P_V: d rows, pieces, swizzled
   uint32_t region;  // per warp a ring of stages (keys then values of a tile); later the
@@ -200,11 +202,15 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int NW, int ns, int rK,
   const int rmax = rK > rV ? rK : rV;
   uint32_t off = 0;
   s.bars = off;
-  off = align_up(off + 8u * (2 * NW * ns + 1), 16);
+  off = align_up(off + 8u * (2 * NW * ns + 2), 16);
   s.ml = off;
   off = align_up(off + 4u * (NW * 16 + 16 + 4), 16);
   s.qraw = off;
   off = align_up(off + 2u * 8u * 128u, 16);  // up to 8 heads of d = 128
+  s.newraw = off;
+  off = align_up(off + 2u * 2u * 128u, 16);
+  s.newlat = off;
+  off = align_up(off + 2u * (uint32_t)(rK + rV), 16);
   s.xs = rmax + 4;
   s.qt = off;
   off = align_up(off + 4u * 8u * s.xs, 1024);
@@ -230,9 +236,8 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
   constexpr int MT = TT / 16;              // 16-token m-tiles (scores) / k-steps (mix) per tile
   // score k-steps / value m-tiles whose fragments are loaded together (fewer where the
   // accumulators already take many registers)
-  constexpr bool kLean = TT == 32 && NB == 1 && NKS == 4 && NMV == 4;
-  constexpr int KG = kLean ? 4 : (NB == 1 ? 2 : 1);
-  constexpr int VG = kLean ? 4 : (NB == 1 ? 2 : 1);
+  constexpr int KG = NB == 1 && TT == 32 ? 2 : 1;
+  constexpr int VG = NB == 1 && TT == 32 ? 2 : 1;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -254,6 +259,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);  // [NW][ns]: tile landed
   uint64_t* empty = full + NW * ns;                             // [NW][ns]: tile consumed
   uint64_t* setup_bar = empty + NW * ns;  // phase 0: q and P_K, phase 1: P_V
+  uint64_t* newrow_bar = setup_bar + 1;   // append: the new value row is in shared memory
   float* ml = reinterpret_cast<float*>(smem + L.ml);
   float* fin = ml + NW * 16;  // [8] M, [8] L
   int* flag = reinterpret_cast<int*>(fin + 16);
@@ -269,7 +275,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
     return;
   }
   if (tid == 0) {
-    for (int i = 0; i < 2 * NW * ns + 1; ++i) mbar_init(&full[i], 1);
+    for (int i = 0; i < 2 * NW * ns + 2; ++i) mbar_init(&full[i], 1);
     fence_barrier_init();
   }
   __syncthreads();
@@ -288,7 +294,34 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
     if (tid == 0 && s_idx == 0 && blockIdx.y == 0) report(a.dev_status, STIEF_DEV_BAD_LENGTH);
     Lb = 0;
   }
-  const int t1 = min(t0 + a.chunk, Lb);
+  // append path: the new token becomes row Lb and is attended to, when the cache has room
+  // (Lb + 1 <= L_max; the host bound max_seq_len must cover the grown length too)
+  bool appended = false;
+  if (a.append) {
+    if (Lb + 1 > a.L_max) {
+      if (tid == 0 && s_idx == 0 && blockIdx.y == 0) report(a.dev_status, STIEF_DEV_CAPACITY_OVERFLOW);
+    } else if (Lb + 1 > a.max_seq_len) {
+      if (tid == 0 && s_idx == 0 && blockIdx.y == 0) report(a.dev_status, STIEF_DEV_BAD_LENGTH);
+    } else {
+      appended = true;
+    }
+  }
+  const int L_att = Lb + (appended ? 1 : 0);  // tokens attended to
+  const bool owns_new = appended && Lb >= t0 && Lb < t0 + a.chunk;  // the new token is in range
+  const int t1 = min(t0 + a.chunk, L_att);
+  // append path: each CTA of a sequence takes a ticket once it has read the old length;
+  // the CTA holding the last ticket (every CTA of the sequence has read it by then) stores
+  // the grown length.  The ticket is requested here by an idle producer lane and only looked
+  // at when the producer is done, so its round trip is off every critical path.
+  const bool seq_lane = a.append && warp == NW && lane == 31;
+  uint32_t seq_ticket = 0u;
+  if (seq_lane) seq_ticket = atomicAdd(a.ws_seq + b, 1u);
+  auto finish_sequence = [&]() {
+    if (seq_lane && seq_ticket == (uint32_t)gridDim.x * gridDim.y - 1u) {
+      a.ws_seq[b] = 0u;
+      if (appended) a.seq_lens_w[b] = Lb + 1;
+    }
+  };
   const int n_tiles = t1 > t0 ? (t1 - t0 + kTile - 1) / kTile : 0;
   auto warp_tiles = [NW](int w, int tiles) { return w < tiles ? (tiles - w + NW - 1) / NW : 0; };
   const size_t head_row0 = ((size_t)b * a.Hkv + kvh) * a.L_max;
@@ -329,8 +362,13 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
     if (lane == 0) {
       // q and P_K first (they gate q~), then every warp's ring
       const uint64_t keep = l2_policy_evict_last();  // bases are shared by many CTAs
-      mbar_arrive_expect_tx(setup_bar, 2u * d * rK + 2u * gcount * d);
+      mbar_arrive_expect_tx(setup_bar, 2u * d * rK + 2u * gcount * d + (owns_new ? 4u * d : 0u));
       bulk_g2s(smem + L.qraw, a.q + ((size_t)b * a.Hq + h0) * d, 2u * gcount * d, setup_bar);
+      if (owns_new) {
+        const size_t row = ((size_t)b * a.Hkv + kvh) * d;
+        bulk_g2s(smem + L.newraw, a.k_new + row, 2u * d, setup_bar);
+        bulk_g2s(smem + L.newraw + 2u * d, a.v_new + row, 2u * d, setup_bar);
+      }
       for (int p = 0; p < a.ppk.n; ++p)
         tma_load_2d(pmat + a.ppk.p[p].smem_off, &a.maps[a.ppk.p[p].map], a.ppk.p[p].x, kvh * d,
                     setup_bar, keep);
@@ -354,8 +392,12 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
       qb[ks][0] = n < gcount ? qrow[8 * ks + (lane & 3)] : 0u;
       qb[ks][1] = n < gcount ? qrow[8 * ks + 4 + (lane & 3)] : 0u;
     }
+    // append: the new key row k_down = k_new P_K takes B column 0 of a second MMA on the
+    // same P_K fragments (fp32 accumulation, one rounding to bf16)
+    const uint32_t* krow = reinterpret_cast<const uint32_t*>(smem + L.newraw);
+    const bool kcol = owns_new && n == 0;  // lanes holding B column 0
     for (int mt = warp; mt < nks && ok; mt += NW) {
-      float c[4];
+      float c[4], ck[4];
       const PieceLoc pl = locate(rK, d, 2 * mt + at_chunk(lane));
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
@@ -363,12 +405,28 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
         ldsm_x4_t(smem_u32(pmat) + swz(pl, 16 * ks + at_row(lane)), af);
         if (ks == 0) mma_bf16_z(c, af, qb[ks][0], qb[ks][1]);
         else mma_bf16(c, af, qb[ks][0], qb[ks][1]);
+        if (owns_new) {
+          const uint32_t k0 = kcol ? krow[8 * ks + (lane & 3)] : 0u;
+          const uint32_t k1 = kcol ? krow[8 * ks + 4 + (lane & 3)] : 0u;
+          if (ks == 0) mma_bf16_z(ck, af, k0, k1);
+          else mma_bf16(ck, af, k0, k1);
+        }
       }
       const int j = 16 * mt + (lane >> 2), hh = 2 * (lane & 3);
       qt[hh * xs + j] = c[0] * a.qscale;
       qt[(hh + 1) * xs + j] = c[1] * a.qscale;
       qt[hh * xs + j + 8] = c[2] * a.qscale;
       qt[(hh + 1) * xs + j + 8] = c[3] * a.qscale;
+      if (owns_new && (lane & 3) == 0) {  // column 0: k_down[j], k_down[j + 8]
+        uint16_t* kl = reinterpret_cast<uint16_t*>(smem + L.newlat);
+        kl[j] = f32_to_bf16_rn(ck[0]);
+        kl[j + 8] = f32_to_bf16_rn(ck[2]);
+        if (qs == 0) {  // the cache row itself (every sub-group computes the same values)
+          uint16_t* dst = a.k_lat_w + (head_row0 + Lb) * rK;
+          dst[j] = kl[j];
+          dst[j + 8] = kl[j + 8];
+        }
+      }
     }
   }
   __syncthreads();  // q~ is in shared memory and every read of P_K is done
@@ -407,7 +465,41 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
       for (int k = pre; k < min(ns, tiles_w); ++k) issue(w, k, stream);
       int k = ns;
       uint64_t last_progress = global_timer_ns();
+      // append: once P_V has landed, the new value row v_down = v_new P_V is projected on
+      // the MMA (B column 0) into shared memory (and the cache) for the tile that holds it
+      bool vrow_done = !owns_new;
+      auto project_vrow = [&]() {
+        const uint32_t* vrow = reinterpret_cast<const uint32_t*>(smem + L.newraw + 2u * d);
+        const bool vcol = (lane >> 2) == 0;  // lanes holding B column 0
+        uint16_t* vl = reinterpret_cast<uint16_t*>(smem + L.newlat) + rK;
+        for (int mv = 0; mv < nmv; ++mv) {
+          float cv[4];
+          const PieceLoc pl = locate(rV, d, 2 * mv + at_chunk(lane));
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {
+            uint32_t af[4];
+            ldsm_x4_t(smem_u32(pmat) + swz(pl, 16 * ks + at_row(lane)), af);
+            const uint32_t v0 = vcol ? vrow[8 * ks + (lane & 3)] : 0u;
+            const uint32_t v1 = vcol ? vrow[8 * ks + 4 + (lane & 3)] : 0u;
+            if (ks == 0) mma_bf16_z(cv, af, v0, v1);
+            else mma_bf16(cv, af, v0, v1);
+          }
+          if ((lane & 3) == 0) {  // column 0: v_down[j], v_down[j + 8]
+            const int j = 16 * mv + (lane >> 2);
+            vl[j] = f32_to_bf16_rn(cv[0]);
+            vl[j + 8] = f32_to_bf16_rn(cv[2]);
+            if (qs == 0) {
+              a.v_lat_w[(head_row0 + Lb) * rV + j] = vl[j];
+              a.v_lat_w[(head_row0 + Lb) * rV + j + 8] = vl[j + 8];
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(newrow_bar);  // release: the row is visible to the consumers
+        vrow_done = true;
+      };
       while (__any_sync(kFull, k < tiles_w)) {
+        if (!vrow_done && mbar_test(setup_bar, 1u)) project_vrow();
         const bool ready = k < tiles_w && mbar_test(&empty[w * ns + (k % ns)], (uint32_t)((k / ns - 1) & 1));
         if (ready) {
           issue(w, k, stream);
@@ -423,6 +515,8 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
           }
         }
       }
+      if (!vrow_done && mbar_wait_bounded(setup_bar, 1u, a.dev_status)) project_vrow();
+      finish_sequence();
       // tiles requested before seq_lens was known but past the sequence are never consumed:
       // they must land before the region is reused
       if (lane < NW) {
@@ -462,6 +556,25 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
       const uint32_t sbase = smem_u32(ring + (size_t)st * st_bytes);
       const int tok0 = t0 + (warp + k * NW) * kTile;
       const int n = min(kTile, t1 - tok0);
+      if (owns_new && tok0 <= Lb && Lb < tok0 + kTile) {
+        // This tile holds the new token, whose cache rows were not written yet when the tile
+        // was fetched: put the projected rows (key row from the prologue, value row from
+        // the producer) into the tile.
+        if (!warp_wait(newrow_bar, 0, a.dev_status)) {
+          ok = false;
+          break;
+        }
+        const int r_new = Lb - tok0;
+        const uint16_t* kl = reinterpret_cast<const uint16_t*>(smem + L.newlat);
+        for (int cch = lane; cch < (rK + rV) / 8; cch += 32) {
+          const bool key = cch < rK / 8;
+          const PieceLoc pt = key ? locate(rK, kTile, cch) : locate(rV, kTile, cch - rK / 8);
+          *reinterpret_cast<uint4*>(ring + (size_t)st * st_bytes + (key ? 0u : kt_bytes) +
+                                    swz(pt, r_new)) = *reinterpret_cast<const uint4*>(kl + 8 * cch);
+        }
+        fence_proxy_async_smem();  // generic writes into a stage the TMA engine fills
+        __syncwarp();
+      }
 
       // Fragments are requested a group of k-steps (m-tiles) at a time, so their latencies
       // overlap; asm volatile keeps the order written here.

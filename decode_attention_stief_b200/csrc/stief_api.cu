@@ -86,7 +86,7 @@ size_t stief_decode_workspace_bytes(int B, int Hq, int Hkv, int rV, int max_seq_
   const int G_T = group_tile(G);
   const int qsub = (G + G_T - 1) / G_T;
   const size_t units = (size_t)B * Hkv * qsub;
-  return stief::decode_ws_bytes(units, G_T, stief_decode_max_splits(max_seq_len), kHeadDim);
+  return stief::decode_ws_bytes(units, (size_t)B, G_T, stief_decode_max_splits(max_seq_len), kHeadDim);
 }
 
 stief_status stief_compress_append(const uint16_t* k_new, const uint16_t* v_new,
@@ -127,14 +127,18 @@ stief_status stief_compress_append(const uint16_t* k_new, const uint16_t* v_new,
   return STIEF_OK;
 }
 
-stief_status stief_decode_attention(const uint16_t* q, const uint16_t* P_K, const uint16_t* P_V,
-                                    const uint16_t* k_lat, const uint16_t* v_lat,
-                                    const int32_t* seq_lens, uint16_t* out, void* workspace,
-                                    size_t workspace_bytes, int B, int Hq, int Hkv, int d, int rK,
-                                    int rV, int L_max, int max_seq_len, int num_splits,
-                                    uint32_t* dev_status, stief_stream_t stream) {
+namespace {
+
+// Shared body of stief_decode_attention and stief_append_decode.
+stief_status decode_common(const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new,
+                           const uint16_t* P_K, const uint16_t* P_V, uint16_t* k_lat,
+                           uint16_t* v_lat, int32_t* seq_lens, uint16_t* out, void* workspace,
+                           size_t workspace_bytes, int B, int Hq, int Hkv, int d, int rK, int rV,
+                           int L_max, int max_seq_len, int num_splits, uint32_t* dev_status,
+                           stief_stream_t stream, bool append) {
   // cheap host checks first, so argument errors never touch CUDA
   if (!q || !P_K || !P_V || !k_lat || !v_lat || !seq_lens || !out) return STIEF_ERR_INVALID_ARG;
+  if (append && (!k_new || !v_new)) return STIEF_ERR_INVALID_ARG;
   stief_status st = check_decode_shape(B, Hq, Hkv, d, rK, rV, L_max, max_seq_len);
   if (st != STIEF_OK) return st;
   const int smax = stief_decode_max_splits(max_seq_len);
@@ -142,6 +146,7 @@ stief_status stief_decode_attention(const uint16_t* q, const uint16_t* P_K, cons
   if (!aligned16(q) || !aligned16(P_K) || !aligned16(P_V) || !aligned16(k_lat) ||
       !aligned16(v_lat) || !aligned16(out) || !aligned16(workspace))
     return STIEF_ERR_ALIGNMENT;
+  if (append && (!aligned16(k_new) || !aligned16(v_new))) return STIEF_ERR_ALIGNMENT;
   const size_t need = stief_decode_workspace_bytes(B, Hq, Hkv, rV, max_seq_len);
   if (!workspace || workspace_bytes < need) return STIEF_ERR_WORKSPACE;
 
@@ -149,14 +154,48 @@ stief_status stief_decode_attention(const uint16_t* q, const uint16_t* P_K, cons
   st = stief::plan_decode(a, q, P_K, P_V, k_lat, v_lat, seq_lens, out, B, Hq, Hkv, d, rK, rV,
                           L_max, max_seq_len, num_splits, dev_status);
   if (st != STIEF_OK) return st;
-  // counters at the start, then the partial states laid out for the split count used
+  a.append = append ? 1 : 0;
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.k_lat_w = k_lat;
+  a.v_lat_w = v_lat;
+  a.seq_lens_w = seq_lens;
+  // counters at the start (split tickets, then sequence tickets), then the partial states
+  // laid out for the split count used
   const size_t units = (size_t)B * Hkv * a.qsub;
   a.ws_cnt = static_cast<uint32_t*>(workspace);
+  a.ws_seq = a.ws_cnt + units;
   a.ws_part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
-                                       stief::decode_ws_counter_bytes(units));
+                                       stief::decode_ws_counter_bytes(units, (size_t)B));
   if (stief::launch_decode(a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return STIEF_ERR_CUDA;
   return STIEF_OK;
+}
+
+}  // namespace
+
+stief_status stief_decode_attention(const uint16_t* q, const uint16_t* P_K, const uint16_t* P_V,
+                                    const uint16_t* k_lat, const uint16_t* v_lat,
+                                    const int32_t* seq_lens, uint16_t* out, void* workspace,
+                                    size_t workspace_bytes, int B, int Hq, int Hkv, int d, int rK,
+                                    int rV, int L_max, int max_seq_len, int num_splits,
+                                    uint32_t* dev_status, stief_stream_t stream) {
+  // the caches and lengths are only read on this path
+  return decode_common(q, nullptr, nullptr, P_K, P_V, const_cast<uint16_t*>(k_lat),
+                       const_cast<uint16_t*>(v_lat), const_cast<int32_t*>(seq_lens), out,
+                       workspace, workspace_bytes, B, Hq, Hkv, d, rK, rV, L_max, max_seq_len,
+                       num_splits, dev_status, stream, false);
+}
+
+stief_status stief_append_decode(const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new,
+                                 const uint16_t* P_K, const uint16_t* P_V, uint16_t* k_lat,
+                                 uint16_t* v_lat, int32_t* seq_lens, uint16_t* out,
+                                 void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv,
+                                 int d, int rK, int rV, int L_max, int max_seq_len,
+                                 int num_splits, uint32_t* dev_status, stief_stream_t stream) {
+  return decode_common(q, k_new, v_new, P_K, P_V, k_lat, v_lat, seq_lens, out, workspace,
+                       workspace_bytes, B, Hq, Hkv, d, rK, rV, L_max, max_seq_len, num_splits,
+                       dev_status, stream, true);
 }
 
 stief_status stief_read_device_status(const uint32_t* dev_status, uint32_t* value,

@@ -37,6 +37,14 @@ struct DecodeArgs {
   const uint16_t* q;
   const int32_t* seq_lens;
   uint16_t* out;
+  // append path (stief_append_decode): the new token's rows, the caches and lengths it writes
+  int append;
+  const uint16_t* k_new;  // [B][Hkv][d]
+  const uint16_t* v_new;  // [B][Hkv][d]
+  uint16_t* k_lat_w;
+  uint16_t* v_lat_w;
+  int32_t* seq_lens_w;
+  uint32_t* ws_seq;  // [B] per-sequence finish tickets; zero between calls
   uint32_t* ws_cnt;  // [units] split tickets; zero between calls
   float* ws_part;    // [units * S * G_T][d + 4] partial states: o[d] (up-projected), m, l, 0, 0
   uint32_t* dev_status;
@@ -105,11 +113,14 @@ stief_status plan_decode(DecodeArgs& a, const uint16_t* q, const uint16_t* P_K,
                          int rK, int rV, int L_max, int max_seq_len, int num_splits,
                          uint32_t* dev_status);
 
-// Decode workspace layout: `units` = B * Hkv * qsub ticket counters (uint32, padded to
-// 256 bytes), then units * G_T * splits partial states of (d + 4) floats.
-inline size_t decode_ws_counter_bytes(size_t units) { return (units * 4u + 255u) / 256u * 256u; }
-inline size_t decode_ws_bytes(size_t units, int G_T, int splits, int d) {
-  return decode_ws_counter_bytes(units) + units * (size_t)G_T * splits * (size_t)(d + 4) * 4u;
+// Decode workspace layout: `units` = B * Hkv * qsub split-ticket counters, then B sequence
+// tickets (uint32, padded together to 256 bytes), then units * G_T * splits partial states
+// of (d + 4) floats.
+inline size_t decode_ws_counter_bytes(size_t units, size_t B) {
+  return ((units + B) * 4u + 255u) / 256u * 256u;
+}
+inline size_t decode_ws_bytes(size_t units, size_t B, int G_T, int splits, int d) {
+  return decode_ws_counter_bytes(units, B) + units * (size_t)G_T * splits * (size_t)(d + 4) * 4u;
 }
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
 

@@ -74,14 +74,16 @@ extern "C" STIEF_API stief_status stief_decode_attention_noalloc(
 
   // ticket counters and the partial states of the split count actually used must fit
   const size_t units = (size_t)B * Hkv * a.qsub;
-  if (stief::decode_ws_bytes(units, a.G_T, a.S, a.d) > kScratchBytes) return STIEF_ERR_WORKSPACE;
+  if (stief::decode_ws_bytes(units, (size_t)B, a.G_T, a.S, a.d) > kScratchBytes)
+    return STIEF_ERR_WORKSPACE;
 
   void* scratch = nullptr;
   st = scratch_address(&scratch);
   if (st != STIEF_OK) return st;
   a.ws_cnt = static_cast<uint32_t*>(scratch);
+  a.ws_seq = a.ws_cnt + units;
   a.ws_part = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) +
-                                       stief::decode_ws_counter_bytes(units));
+                                       stief::decode_ws_counter_bytes(units, (size_t)B));
   if (stief::launch_decode(a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return STIEF_ERR_CUDA;
   return STIEF_OK;

@@ -123,11 +123,11 @@ STIEF_API int stief_decode_auto_splits(int B, int Hq, int Hkv, int max_seq_len, 
  * stief_decode_workspace_bytes -- bytes of device workspace stief_decode_attention
  * needs for these sizes, for any split count it may use (at most
  * stief_decode_max_splits(max_seq_len)).  The workspace holds one ticket counter
- * per (sequence, KV head, query sub-group) followed by the per-split partial
- * states: for each query head, the split's up-projected unnormalised output
- * (d floats), its running maximum and sum, and two pad words.  rV is validated
- * but does not change the size.  Pure host function.  Returns 0 for invalid
- * arguments.
+ * per (sequence, KV head, query sub-group) and one per sequence, followed by the
+ * per-split partial states: for each query head, the split's up-projected
+ * unnormalised output (d floats), its running maximum and sum, and two pad words.
+ * rV is validated but does not change the size.  The same workspace serves
+ * stief_append_decode.  Pure host function.  Returns 0 for invalid arguments.
  */
 STIEF_API size_t stief_decode_workspace_bytes(int B, int Hq, int Hkv, int rV, int max_seq_len);
 
@@ -166,7 +166,8 @@ STIEF_API size_t stief_decode_workspace_bytes(int B, int Hq, int Hkv, int rV, in
  *                  counters must be zero when a call starts, and every call that
  *                  runs to completion leaves them at zero again, so the same
  *                  workspace serves any later call (any sizes) on the same
- *                  stream without clearing
+ *                  stream without clearing.  After a call whose dev_status reports
+ *                  a timeout, zero it again
  *   max_seq_len  : host-side upper bound of seq_lens (<= L_max); sizes the grid
  *   num_splits   : 0 = automatic, otherwise the number of KV splits per sequence
  *                  (1 .. stief_decode_max_splits(max_seq_len))
@@ -186,6 +187,40 @@ STIEF_API stief_status stief_decode_attention(const uint16_t* q, const uint16_t*
                                     int B, int Hq, int Hkv, int d, int rK, int rV, int L_max,
                                     int max_seq_len, int num_splits,
                                     uint32_t* dev_status, stief_stream_t stream);
+
+/*
+ * stief_append_decode -- one whole decode step of the hot path in one kernel: the
+ * append of stief_compress_append with T = 1 followed by stief_decode_attention over
+ * the grown cache (StiefAttention technical summary, "Mecanismo Central" item 5:
+ * keys and values are stored compressed, K_down = K P_K, V_down = V P_V, and
+ * attention runs over their reconstructions).
+ *
+ * For every sequence b (L = seq_lens[b] on entry) and KV head g:
+ *     k_lat[b][g][L] = bf16_RNE(k_new[b][g] . P_K[g])      (fp32 accumulation)
+ *     v_lat[b][g][L] = bf16_RNE(v_new[b][g] . P_V[g])
+ * then, for every query head h of g, out[b][h] is stief_decode_attention's result
+ * over the L + 1 tokens [0, L], and seq_lens[b] = L + 1 once the kernel completes.
+ * Rows other than L are not written.  If L + 1 > L_max the sequence is not appended
+ * to (STIEF_DEV_CAPACITY_OVERFLOW is set, seq_lens[b] stays L) and out[b] attends over
+ * the L tokens present; if L + 1 > max_seq_len, STIEF_DEV_BAD_LENGTH is set likewise.
+ *
+ *   k_new, v_new : bf16 [B][Hkv][d] (the new token's key and value rows)
+ *   seq_lens     : int32 [B] on the device, read and then incremented
+ *   max_seq_len  : host-side upper bound of the lengths after the append (<= L_max)
+ *   other arguments as for stief_decode_attention (same workspace size and rules)
+ *
+ * The stored rows equal stief_compress_append's up to the order of the fp32 sums
+ * (both round once to bf16).  The paper has no fused call: this one removes the two
+ * extra kernel launches of the separate append from every step.
+ * Returns STIEF_OK or an argument error (nothing launched).
+ */
+STIEF_API stief_status stief_append_decode(const uint16_t* q, const uint16_t* k_new,
+                                 const uint16_t* v_new, const uint16_t* P_K,
+                                 const uint16_t* P_V, uint16_t* k_lat, uint16_t* v_lat,
+                                 int32_t* seq_lens, uint16_t* out, void* workspace,
+                                 size_t workspace_bytes, int B, int Hq, int Hkv, int d, int rK,
+                                 int rV, int L_max, int max_seq_len, int num_splits,
+                                 uint32_t* dev_status, stief_stream_t stream);
 
 /*
  * stief_decode_attention_noalloc -- stief_decode_attention without a workspace
