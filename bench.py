@@ -589,6 +589,40 @@ def cpu_baseline(w: si.Workload, budget_s: float = 20.0):
                       f"x{w.L / L_s:.2f} to the context and x{len(w.layer_ranks())} layers"}
 
 
+def run_profile_launches(args, w: si.Workload):
+    """Diagnostics for profilers: N launches of the step's attention kernel (layer 0 of the
+    workload, lengths reset before each so every launch sees the same context), then exit."""
+    import decode_attention_stief_b200 as stief
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    layers, L_max = build_state(w, 16, w.seed, dev)
+    lay = layers[0]
+    g = torch.Generator(device=dev)
+    g.manual_seed(w.seed + 1)
+    q = torch.randn((w.B, w.Hq, w.d), generator=g, device=dev).to(torch.bfloat16)
+    kn = torch.randn((w.B, w.Hkv, w.d), generator=g, device=dev).to(torch.bfloat16)
+    vn = torch.randn((w.B, w.Hkv, w.d), generator=g, device=dev).to(torch.bfloat16)
+    out = torch.empty_like(q)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    for _ in range(args.profile_launches):
+        lay.seq_lens.fill_(w.L - 1)
+        if args.unfused:
+            lay.seq_lens.fill_(w.L)
+            stief.stief_decode_attention(q, lay.P_K, lay.P_V, lay.k_lat, lay.v_lat, lay.seq_lens,
+                                         out, lay.ws, max_seq_len=L_max, num_splits=args.splits,
+                                         dev_status=status)
+        else:
+            stief.stief_append_decode(q, kn, vn, lay.P_K, lay.P_V, lay.k_lat, lay.v_lat,
+                                      lay.seq_lens, out, lay.ws, max_seq_len=L_max,
+                                      num_splits=args.splits, dev_status=status)
+    torch.cuda.synchronize()
+    st = stief.stief_read_device_status(status)
+    if st != 0:
+        raise RuntimeError(f"device status {st:#x}")
+    print(f"{args.profile_launches} launches of the attention kernel, workload {w.name}, "
+          f"context {w.L}", flush=True)
+
+
 def run_reference(args, w: si.Workload):
     """The reference arm: the fp64 oracle on host cores, W warm-up + K timed steps, each a
     bounded sample (layer 0 at a shortened context) of the GPU arm's step."""
@@ -638,6 +672,9 @@ def main():
     ap.add_argument("--unfused", action="store_true",
                     help="time the step as the two separate calls (append kernel, length "
                          "update, decode) instead of stief_append_decode")
+    ap.add_argument("--profile-launches", type=int, default=0,
+                    help="diagnostics for profilers: make N launches of the step's attention "
+                         "kernel on layer 0 and exit (no timing, no JSON line)")
     ap.add_argument("--clock-window", type=float, default=0.6,
                     help="seconds of untimed decode load before the timed region")
     args = ap.parse_args()
@@ -648,7 +685,9 @@ def main():
         import dataclasses
         w = dataclasses.replace(w, layers=min(args.layers, w.layers),
                                 ranks=w.ranks[:args.layers] if w.ranks else None)
-    if args.impl == "reference":
+    if args.profile_launches > 0:
+        run_profile_launches(args, w)
+    elif args.impl == "reference":
         run_reference(args, w)
     else:
         run_gpu(args, w)
