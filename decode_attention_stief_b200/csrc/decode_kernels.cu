@@ -392,35 +392,38 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
       qb[ks][0] = n < gcount ? qrow[8 * ks + (lane & 3)] : 0u;
       qb[ks][1] = n < gcount ? qrow[8 * ks + 4 + (lane & 3)] : 0u;
     }
-    // append: the new key row k_down = k_new P_K takes B column 0 of a second MMA on the
-    // same P_K fragments (fp32 accumulation, one rounding to bf16)
+    // append: the new key row k_down = k_new P_K is the same contraction with B column 0 =
+    // k_new (fp32 accumulation, one rounding to bf16).  Tasks 0..nks-1 are the q~ m-tiles,
+    // nks..2 nks-1 the k_down m-tiles; the warps share them out.
     const uint32_t* krow = reinterpret_cast<const uint32_t*>(smem + L.newraw);
-    const bool kcol = owns_new && n == 0;  // lanes holding B column 0
-    for (int mt = warp; mt < nks && ok; mt += NW) {
-      float c[4], ck[4];
+    const int ntasks = owns_new ? 2 * nks : nks;
+    for (int task = warp; task < ntasks && ok; task += NW) {
+      const bool key = task >= nks;
+      const int mt = key ? task - nks : task;
+      float c[4];
       const PieceLoc pl = locate(rK, d, 2 * mt + at_chunk(lane));
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
         uint32_t af[4];
         ldsm_x4_t(smem_u32(pmat) + swz(pl, 16 * ks + at_row(lane)), af);
-        if (ks == 0) mma_bf16_z(c, af, qb[ks][0], qb[ks][1]);
-        else mma_bf16(c, af, qb[ks][0], qb[ks][1]);
-        if (owns_new) {
-          const uint32_t k0 = kcol ? krow[8 * ks + (lane & 3)] : 0u;
-          const uint32_t k1 = kcol ? krow[8 * ks + 4 + (lane & 3)] : 0u;
-          if (ks == 0) mma_bf16_z(ck, af, k0, k1);
-          else mma_bf16(ck, af, k0, k1);
+        uint32_t b0 = qb[ks][0], b1 = qb[ks][1];
+        if (key) {
+          b0 = n == 0 ? krow[8 * ks + (lane & 3)] : 0u;
+          b1 = n == 0 ? krow[8 * ks + 4 + (lane & 3)] : 0u;
         }
+        if (ks == 0) mma_bf16_z(c, af, b0, b1);
+        else mma_bf16(c, af, b0, b1);
       }
       const int j = 16 * mt + (lane >> 2), hh = 2 * (lane & 3);
-      qt[hh * xs + j] = c[0] * a.qscale;
-      qt[(hh + 1) * xs + j] = c[1] * a.qscale;
-      qt[hh * xs + j + 8] = c[2] * a.qscale;
-      qt[(hh + 1) * xs + j + 8] = c[3] * a.qscale;
-      if (owns_new && (lane & 3) == 0) {  // column 0: k_down[j], k_down[j + 8]
+      if (!key) {
+        qt[hh * xs + j] = c[0] * a.qscale;
+        qt[(hh + 1) * xs + j] = c[1] * a.qscale;
+        qt[hh * xs + j + 8] = c[2] * a.qscale;
+        qt[(hh + 1) * xs + j + 8] = c[3] * a.qscale;
+      } else if ((lane & 3) == 0) {  // column 0: k_down[j], k_down[j + 8]
         uint16_t* kl = reinterpret_cast<uint16_t*>(smem + L.newlat);
-        kl[j] = f32_to_bf16_rn(ck[0]);
-        kl[j + 8] = f32_to_bf16_rn(ck[2]);
+        kl[j] = f32_to_bf16_rn(c[0]);
+        kl[j + 8] = f32_to_bf16_rn(c[2]);
         if (qs == 0) {  // the cache row itself (every sub-group computes the same values)
           uint16_t* dst = a.k_lat_w + (head_row0 + Lb) * rK;
           dst[j] = kl[j];
@@ -467,12 +470,14 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
       uint64_t last_progress = global_timer_ns();
       // append: once P_V has landed, the new value row v_down = v_new P_V is projected on
       // the MMA (B column 0) into shared memory (and the cache) for the tile that holds it
-      bool vrow_done = !owns_new;
+      // (one 16-row m-tile per call, so the refills in between are not held up)
+      int vrow_next = owns_new ? 0 : nmv;  // next m-tile of the new value row to project
       auto project_vrow = [&]() {
         const uint32_t* vrow = reinterpret_cast<const uint32_t*>(smem + L.newraw + 2u * d);
         const bool vcol = (lane >> 2) == 0;  // lanes holding B column 0
         uint16_t* vl = reinterpret_cast<uint16_t*>(smem + L.newlat) + rK;
-        for (int mv = 0; mv < nmv; ++mv) {
+        {
+          const int mv = vrow_next;
           float cv[4];
           const PieceLoc pl = locate(rV, d, 2 * mv + at_chunk(lane));
 #pragma unroll
@@ -494,12 +499,13 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
             }
           }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(newrow_bar);  // release: the row is visible to the consumers
-        vrow_done = true;
+        if (++vrow_next == nmv) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(newrow_bar);  // release: the row is visible to the consumers
+        }
       };
       while (__any_sync(kFull, k < tiles_w)) {
-        if (!vrow_done && mbar_test(setup_bar, 1u)) project_vrow();
+        if (vrow_next < nmv && mbar_test(setup_bar, 1u)) project_vrow();
         const bool ready = k < tiles_w && mbar_test(&empty[w * ns + (k % ns)], (uint32_t)((k / ns - 1) & 1));
         if (ready) {
           issue(w, k, stream);
@@ -515,7 +521,8 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
           }
         }
       }
-      if (!vrow_done && mbar_wait_bounded(setup_bar, 1u, a.dev_status)) project_vrow();
+      if (vrow_next < nmv && mbar_wait_bounded(setup_bar, 1u, a.dev_status))
+        while (vrow_next < nmv) project_vrow();
       finish_sequence();
       // tiles requested before seq_lens was known but past the sequence are never consumed:
       // they must land before the region is reused
