@@ -775,10 +775,13 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
   for (int idx = tid; idx < HR * rV; idx += NT) {
     const int h = idx / rV, jj = idx - h * rV;
     float M = -INFINITY;
-    for (int w = 0; w < NW; ++w) M = fmaxf(M, ml[(w * 8 + h) * 2]);
+#pragma unroll
+    for (int w = 0; w < kMaxConsumerWarps; ++w)
+      if (w < NW) M = fmaxf(M, ml[(w * 8 + h) * 2]);
     float o = 0.f, lsum = 0.f;
-    if (M != -INFINITY)
-      for (int w = 0; w < NW; ++w) {
+#pragma unroll
+    for (int w = 0; w < kMaxConsumerWarps; ++w)
+      if (w < NW) {
         const float mw = ml[(w * 8 + h) * 2];
         if (mw != -INFINITY) {
           const float f = ex2(mw - M);
