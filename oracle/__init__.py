@@ -72,6 +72,9 @@ class Oracle:
         lib.stief_oracle_decode.restype = ctypes.c_int
         lib.stief_oracle_decode.argtypes = (
             [_D, _D, _D, _D, _D, _I32, _D] + [ctypes.c_int] * 8)
+        lib.stief_oracle_decode_latent.restype = ctypes.c_int
+        lib.stief_oracle_decode_latent.argtypes = (
+            [_D, _D, _D, _I32, _D] + [ctypes.c_int] * 8)
         lib.stief_oracle_max_threads.restype = ctypes.c_int
         lib.stief_oracle_max_threads.argtypes = []
         self.lib = lib
@@ -151,6 +154,30 @@ class Oracle:
         return out
 
 
+    def decode_latent(self, q_lat, k_lat, v_lat, seq_lens, d: int = 128,
+                      num_threads: int = 0) -> np.ndarray:
+        """Decode in the latent space (bases folded into the attention weights); returns
+        o~ [B][Hq][rV] (fp64).  Scores are scaled by 1/sqrt(d), d the full head dimension.
+
+        Shapes: q_lat [B][Hq][rK], k_lat [B][Hkv][L_max][rK], v_lat [B][Hkv][L_max][rV],
+        seq_lens [B].
+        """
+        q_lat, k_lat, v_lat = map(_f64, (q_lat, k_lat, v_lat))
+        lens = np.ascontiguousarray(np.asarray(seq_lens, dtype=np.int32))
+        B, Hq, rK = q_lat.shape
+        Hkv, L_max = k_lat.shape[1], k_lat.shape[2]
+        rV = v_lat.shape[3]
+        if Hq % Hkv != 0 or k_lat.shape != (B, Hkv, L_max, rK) \
+                or v_lat.shape != (B, Hkv, L_max, rV):
+            raise ValueError("decode_latent: inconsistent shapes")
+        out = np.empty((B, Hq, rV), dtype=np.float64)
+        rc = self.lib.stief_oracle_decode_latent(_ptr(q_lat), _ptr(k_lat), _ptr(v_lat),
+                                                 _ptr(lens, _I32), _ptr(out), B, Hq, Hkv, int(d),
+                                                 rK, rV, L_max, int(num_threads))
+        if rc != 0:
+            raise ValueError("decode_latent: a sequence length is outside [0, L_max]")
+        return out
+
 def default() -> Oracle:
     """The oracle built from stief_oracle.c (compiled on first use)."""
     global _lib
@@ -179,3 +206,7 @@ def compress_append(k_new, v_new, P_K, P_V, k_lat, v_lat, seq_lens, round_to_bf1
 
 def decode(q, P_K, P_V, k_lat, v_lat, seq_lens, num_threads: int = 0) -> np.ndarray:
     return default().decode(q, P_K, P_V, k_lat, v_lat, seq_lens, num_threads)
+
+
+def decode_latent(q_lat, k_lat, v_lat, seq_lens, d: int = 128, num_threads: int = 0) -> np.ndarray:
+    return default().decode_latent(q_lat, k_lat, v_lat, seq_lens, d, num_threads)

@@ -259,6 +259,83 @@ int stief_oracle_decode(const double* q, const double* P_K, const double* P_V,
     return bad ? -1 : 0;
 }
 
+/*
+ * Decode in the latent space, for models whose attention weights absorb the bases
+ * (StiefAttention technical summary, "Mecanismo Central" item 5, last sentence:
+ * the projection bases can be folded into the attention's linear weights).
+ *
+ *   q_lat        : [B][Hq][rK]   (the query already projected, q~ = q . P_K)
+ *   k_lat, v_lat : [B][Hkv][L_max][rK], [B][Hkv][L_max][rV]
+ *   seq_lens     : [B]
+ *   out_lat      : [B][Hq][rV]   (o~; the model's folded output weight applies P_V^T)
+ *
+ * For each (b, KV head g) and each of its query heads h (h / G == g):
+ *   s_t = (q~_h . K_down[t]) / sqrt(d)        t < L, d the full head dimension
+ *   p   = softmax(s)   (maximum subtracted, then normalised)
+ *   o~_h = sum_t p_t V_down[t]
+ * L == 0 gives o~_h = 0.  Returns 0, or -1 if a length is outside [0, L_max].
+ */
+int stief_oracle_decode_latent(const double* q_lat, const double* k_lat, const double* v_lat,
+                               const int32_t* seq_lens, double* out_lat,
+                               int B, int Hq, int Hkv, int d, int rK, int rV, int L_max,
+                               int num_threads)
+{
+    const int G = Hq / Hkv;
+    const double inv_sqrt_d = 1.0 / sqrt((double)d);
+    int bad = 0;
+    memset(out_lat, 0, sizeof(double) * (size_t)B * Hq * rV);
+
+#ifdef _OPENMP
+    if (num_threads > 0)
+        omp_set_num_threads(num_threads);
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+#endif
+    for (long unit = 0; unit < (long)B * Hkv; ++unit) {
+        const int b = (int)(unit / Hkv);
+        const int g = (int)(unit % Hkv);
+        const long L = seq_lens[b];
+        if (L < 0 || L > L_max) {
+            bad |= 1;
+            continue;
+        }
+        if (L == 0)
+            continue;
+        const double* Kd = k_lat + ((long)b * Hkv + g) * L_max * rK;
+        const double* Vd = v_lat + ((long)b * Hkv + g) * L_max * rV;
+        double* w_lat = (double*)malloc(sizeof(double) * (size_t)L);
+        for (int j = 0; j < G; ++j) {
+            const long head = (long)b * Hq + (long)g * G + j;  /* query head of group g */
+            const double* qh = q_lat + head * rK;
+            /* scores */
+            for (long t = 0; t < L; ++t) {
+                double acc = 0.0;
+                for (int c = 0; c < rK; ++c)
+                    acc += qh[c] * Kd[t * rK + c];
+                w_lat[t] = acc * inv_sqrt_d;
+            }
+            /* softmax: subtract the maximum, exponentiate, sum */
+            double mx = w_lat[0];
+            for (long t = 1; t < L; ++t)
+                if (w_lat[t] > mx)
+                    mx = w_lat[t];
+            double sum_lat = 0.0;
+            for (long t = 0; t < L; ++t) {
+                w_lat[t] = exp(w_lat[t] - mx);
+                sum_lat += w_lat[t];
+            }
+            /* value mix in the latent space */
+            double* oh = out_lat + head * rV;
+            for (long t = 0; t < L; ++t) {
+                const double p_lat = w_lat[t] / sum_lat;
+                for (int c = 0; c < rV; ++c)
+                    oh[c] += p_lat * Vd[t * rV + c];
+            }
+        }
+        free(w_lat);
+    }
+    return bad ? -1 : 0;
+}
+
 /* Number of OpenMP threads a parallel region would use (1 without OpenMP). */
 int stief_oracle_max_threads(void)
 {

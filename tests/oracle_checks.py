@@ -11,7 +11,7 @@ Stiefel manifold", StiefAttention technical summary, "Mecanismo Central" /
 "Kernmechanismus": item 2 (orthonormal bases on the Stiefel manifold), item 3
 (QR orthonormalisation; R is only a change of coordinates inside the subspace),
 item 5 (stored K_down = K P_K, reconstruction K~ = K_down P_K^T before
-attention); "Resultados Experimentais" (the uncompressed FP16 baseline, i.e.
+attention; the bases may be folded into the attention weights); "Resultados Experimentais" (the uncompressed FP16 baseline, i.e.
 plain attention, which the r = d case must reproduce).
 """
 from __future__ import annotations
@@ -224,6 +224,62 @@ def check_empty_sequence(o, r: int = 64, d: int = 128) -> None:
     assert np.all(np.isfinite(got[1])) and np.any(got[1] != 0.0)
 
 
+# ----------------------------------------------------------------------------- latent decode
+
+def check_latent_is_sdpa_on_latent_rows(o, q_scale: float = 1.0, tol: float = 1e-12) -> None:
+    """The latent decode is softmax attention over the latent rows themselves, with the
+    score scale 1/sqrt(d) of the full head dimension (torch SDPA, float64, explicit scale)."""
+    d = 128
+    B, Hq, Hkv, L_max, rK, rV = 2, 8, 2, 40, 48, 32
+    lens = np.array([37, 5], dtype=np.int32)
+    rng = np.random.default_rng(17)
+    q = q_scale * rng.standard_normal((B, Hq, rK))
+    k = rng.standard_normal((B, Hkv, L_max, rK))
+    v = rng.standard_normal((B, Hkv, L_max, rV))
+    got = o.decode_latent(q, k, v, lens, d=d)
+    want = np.zeros((B, Hq, rV))
+    for b in range(B):
+        L = int(lens[b])
+        oq = F.scaled_dot_product_attention(
+            torch.from_numpy(q[b][None, :, None, :]),
+            torch.from_numpy(np.ascontiguousarray(k[b][None, :, :L])),
+            torch.from_numpy(np.ascontiguousarray(v[b][None, :, :L])),
+            scale=1.0 / math.sqrt(d), enable_gqa=True)
+        want[b] = oq[0, :, 0, :].numpy()
+    assert np.all(np.isfinite(got)), "non-finite output"
+    err = _rel_err(got, want)
+    assert err <= tol, f"latent decode differs from attention over the latent rows: {err}"
+
+
+def check_latent_folding_identity(o, d: int = 128) -> None:
+    """Folding the bases into the weights changes nothing: decode_latent(q P_K) P_V^T equals
+    decode(q) over the same cache (associativity of the products)."""
+    rng = np.random.default_rng(18)
+    B, Hq, Hkv, L, rK, rV = 2, 8, 4, 33, 64, 48
+    q = rng.standard_normal((B, Hq, d))
+    P_K = si.bases(81, Hkv, d, rK)
+    P_V = si.bases(82, Hkv, d, rV)
+    k = rng.standard_normal((B, Hkv, L, rK))
+    v = rng.standard_normal((B, Hkv, L, rV))
+    lens = np.array([L, 12], np.int32)
+    G = Hq // Hkv
+    q_lat = np.stack([np.stack([q[b, h] @ P_K[h // G] for h in range(Hq)]) for b in range(B)])
+    o_lat = o.decode_latent(q_lat, k, v, lens, d=d)
+    got = np.stack([np.stack([o_lat[b, h] @ P_V[h // G].T for h in range(Hq)]) for b in range(B)])
+    want = o.decode(q, P_K, P_V, k, v, lens)
+    assert _rel_err(got, want) <= 1e-12
+
+
+def check_latent_edges(o, r: int = 32) -> None:
+    """Length 0 gives exactly 0; length 1 gives exactly the one value row."""
+    rng = np.random.default_rng(19)
+    k = rng.standard_normal((2, 1, 6, r))
+    v = rng.standard_normal((2, 1, 6, 2 * r))
+    got = o.decode_latent(7.0 * rng.standard_normal((2, 3, r)), k, v, np.array([0, 1], np.int32))
+    assert np.all(got[0] == 0.0)
+    assert np.array_equal(got[1], np.repeat(v[1, 0, :1], 3, axis=0))
+
+
 # ----------------------------------------------------------------------------- compression
 
 def check_compress_identity_basis(o, r: int = 48, d: int = 128) -> None:
@@ -291,6 +347,12 @@ ALL_ORACLE_CHECKS = {
     "uniform_keys": check_uniform_keys,
     "token_order_invariance": check_token_order_invariance,
     "empty_sequence": check_empty_sequence,
+    "latent_is_sdpa_on_latent_rows": check_latent_is_sdpa_on_latent_rows,
+    # scores past 709, where exp() overflows: the latent path must subtract the maximum too
+    "latent_large_scores": lambda o: check_latent_is_sdpa_on_latent_rows(o, q_scale=2000.0,
+                                                                         tol=1e-10),
+    "latent_folding_identity": check_latent_folding_identity,
+    "latent_edges": check_latent_edges,
     "compress_identity_basis": check_compress_identity_basis,
     "compress_matches_exact_product": check_compress_matches_exact_product,
     "compress_append_bookkeeping": check_compress_append_bookkeeping,

@@ -38,6 +38,17 @@ MUTANTS = [
      "for (long t = 0; t < L; ++t) {\n            reconstruct_row(Vd",
      "for (long t = 1; t < L; ++t) {\n            reconstruct_row(Vd",
      ["single_token", "two_tokens"]),
+    ("latent_scale_uses_rank", "w_lat[t] = acc * inv_sqrt_d;",
+     "w_lat[t] = acc / sqrt((double)rK);", ["latent_is_sdpa_on_latent_rows"]),
+    ("latent_gqa_interleaved", "const long head = (long)b * Hq + (long)g * G + j;",
+     "const long head = (long)b * Hq + (long)j * Hkv + g;",
+     ["latent_is_sdpa_on_latent_rows", "latent_folding_identity"]),
+    ("latent_unnormalised", "const double p_lat = w_lat[t] / sum_lat;",
+     "const double p_lat = w_lat[t];", ["latent_is_sdpa_on_latent_rows"]),
+    ("latent_no_max_subtraction", "w_lat[t] = exp(w_lat[t] - mx);", "w_lat[t] = exp(w_lat[t]);",
+     ["latent_large_scores"]),
+    ("latent_values_from_keys", "oh[c] += p_lat * Vd[t * rV + c];",
+     "oh[c] += p_lat * Kd[t * rK + c];", ["latent_is_sdpa_on_latent_rows", "latent_edges"]),
     ("round_ties_away", "nearbyint(x / q)", "round(x / q)",
      ["round_bf16_edges", "round_bf16_matches_torch"]),
     ("append_off_by_one", "long dst = ((long)b * Hkv + h) * L_max + L;",
