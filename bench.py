@@ -210,9 +210,18 @@ def run_gpu(args, w: si.Workload):
     v_s = torch.randn((w.B, w.Hkv, 1, w.d), generator=g, device=dev).to(torch.bfloat16)
     out = torch.empty((len(layers), w.B, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
+    # latent mode (bases folded into the attention weights): q~ in, o~ out, per layer
+    qlat_s = [torch.randn((w.B, w.Hq, lay.rK), generator=g, device=dev).to(torch.bfloat16)
+              for lay in layers] if args.latent else []
+    olat = [torch.empty((w.B, w.Hq, lay.rV), dtype=torch.bfloat16, device=dev)
+            for lay in layers] if args.latent else []
 
     def layer_step(li, lay):
-        if args.unfused:  # the two separate calls (three kernels)
+        if args.latent:  # attention in the latent space only (no projections, no append)
+            stief.stief_decode_latent(qlat_s[li], lay.k_lat, lay.v_lat, lay.seq_lens, olat[li],
+                                      lay.ws, max_seq_len=L_max, num_splits=args.splits,
+                                      dev_status=status)
+        elif args.unfused:  # the two separate calls (three kernels)
             stief.stief_compress_append(k_s, v_s, lay.P_K, lay.P_V, lay.k_lat, lay.v_lat,
                                         lay.seq_lens, dev_status=status)
             stief.stief_decode_attention(q_s, lay.P_K, lay.P_V, lay.k_lat, lay.v_lat,
@@ -230,7 +239,7 @@ def run_gpu(args, w: si.Workload):
     def decode_only(lays):
         """One launch of the step's attention kernel on layer 0 (for the kernel's own timing)."""
         lay = lays[0]
-        if args.unfused:
+        if args.unfused and not args.latent:
             stief.stief_decode_attention(q_s, lay.P_K, lay.P_V, lay.k_lat, lay.v_lat,
                                          lay.seq_lens, out[0], lay.ws, max_seq_len=L_max,
                                          num_splits=args.splits, dev_status=status)
@@ -238,6 +247,8 @@ def run_gpu(args, w: si.Workload):
             layer_step(0, lay)
 
     def reset_lengths(L0):
+        if args.latent:  # nothing is appended: every step attends over the full context
+            L0 = w.L
         for lays in reps:
             for lay in lays:
                 lay.seq_lens.fill_(L0)
@@ -256,6 +267,8 @@ def run_gpu(args, w: si.Workload):
     h_k = k_s.cpu().pin_memory()
     h_v = v_s.cpu().pin_memory()
     h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h_qlat = [t.cpu().pin_memory() for t in qlat_s]
+    h_olat = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in olat]
     n_dec = max(8, R) // R * R
     cap = torch.cuda.Stream(device=dev)
     cap.wait_stream(torch.cuda.current_stream())
@@ -272,11 +285,18 @@ def run_gpu(args, w: si.Workload):
             step_graphs.append(gr)
             ge = torch.cuda.CUDAGraph()
             with torch.cuda.graph(ge, stream=cap):
-                q_s.copy_(h_q, non_blocking=True)
-                k_s.copy_(h_k, non_blocking=True)
-                v_s.copy_(h_v, non_blocking=True)
-                step(reps[r])
-                h_out.copy_(out, non_blocking=True)
+                if args.latent:
+                    for dst, src in zip(qlat_s, h_qlat):
+                        dst.copy_(src, non_blocking=True)
+                    step(reps[r])
+                    for dst, src in zip(h_olat, olat):
+                        dst.copy_(src, non_blocking=True)
+                else:
+                    q_s.copy_(h_q, non_blocking=True)
+                    k_s.copy_(h_k, non_blocking=True)
+                    v_s.copy_(h_v, non_blocking=True)
+                    step(reps[r])
+                    h_out.copy_(out, non_blocking=True)
             e2e_graphs.append(ge)
         dec_graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(dec_graph, stream=cap):
@@ -337,7 +357,8 @@ def run_gpu(args, w: si.Workload):
     # ---- decode kernel timing for the roofline: runs of n_dec back-to-back launches
     # (replicas rotating), averaged over the timed region; plus single launches.  The fused
     # kernel appends a token per launch: lengths restart at L_dec - 1 for each run.
-    L_run0 = L_dec - (0 if args.unfused else 1)
+    appends = not (args.unfused or args.latent)  # the step's kernel appends a token
+    L_run0 = L_dec - (1 if appends else 0)
     reset_lengths(L_run0)
     dec_reps = max(3, args.decode_iters // n_dec)
     torch.cuda.synchronize()
@@ -349,7 +370,7 @@ def run_gpu(args, w: si.Workload):
     d1.record(stream)
     torch.cuda.synchronize()
     dec_us = d0.elapsed_time(d1) * 1e3 / (dec_reps * n_dec)
-    L_dec_mean = L_dec + (0 if args.unfused else (dec_reps * n_dec // R) / 2)
+    L_dec_mean = L_dec + ((dec_reps * n_dec // R) / 2 if appends else 0)
     reset_lengths(L_run0)
     iso = []
     for j in range(max(5, min(args.decode_iters, 30))):
@@ -380,8 +401,9 @@ def run_gpu(args, w: si.Workload):
     torch.cuda.synchronize()
     barrier()
     e2e_ms = e0_ev.elapsed_time(e1_ev) / K
-    h2d = (q_s.numel() + k_s.numel() + v_s.numel()) * 2
-    d2h = out.numel() * 2
+    h2d = (sum(t.numel() for t in qlat_s) if args.latent
+           else q_s.numel() + k_s.numel() + v_s.numel()) * 2
+    d2h = (sum(t.numel() for t in olat) if args.latent else out.numel()) * 2
     st = stief.stief_read_device_status(status)
     if st != 0:
         raise RuntimeError(f"device status {st:#x} after the e2e steps")
@@ -425,12 +447,17 @@ def run_gpu(args, w: si.Workload):
             "workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "context": w.L,
             "layers": len(layers), "ranks": [list(r) for r in w.layer_ranks()][:4]
             + (["..."] if len(layers) > 4 else []),
-            "step": ("append 1 token per (sequence, KV head) + decode, every layer; the API "
-                     "calls captured in CUDA graphs (one step per replica, the timed region "
-                     "replays the replica cycle back to back); " +
-                     ("stief_compress_append + stief_decode_attention (3 kernels per layer)"
+            "step": (("latent decode only (bases folded into the attention weights: q~ in, "
+                      "o~ out; the new token's latent rows would come from the folded K/V "
+                      "projection), every layer; " if args.latent else
+                      "append 1 token per (sequence, KV head) + decode, every layer; ") +
+                     "the API calls captured in CUDA graphs (one step per replica, the timed "
+                     "region replays the replica cycle back to back); " +
+                     ("stief_decode_latent (1 kernel per layer)" if args.latent else
+                      "stief_compress_append + stief_decode_attention (3 kernels per layer)"
                       if args.unfused else "stief_append_decode (1 kernel per layer)")),
-            "context_growth": f"+1 token per step of a replica (contexts {ctx_first}..{ctx_last})",
+            "context_growth": (f"none (context {w.L} every step)" if args.latent else
+                               f"+1 token per step of a replica (contexts {ctx_first}..{ctx_last})"),
             "l2": (f"no flush: steps rotate over {R} copies of the layer caches "
                    f"({rot_mb:.0f} MiB in all, > 3x the 126 MB L2)" if R > 1 else
                    f"no flush: one step reads {rot_mb:.0f} MiB of caches (> 3x the 126 MB L2)"
@@ -440,7 +467,8 @@ def run_gpu(args, w: si.Workload):
         },
         "hbm_gbs_step": round(step_bytes / (ms_per_step / 1e3) / 1e9, 1),
         "roofline": {
-            "kernel": "stief_decode_kernel (" + ("stief_decode_attention" if args.unfused
+            "kernel": "stief_decode_kernel (" + ("stief_decode_latent" if args.latent else
+                                                 "stief_decode_attention" if args.unfused
                                                  else "stief_append_decode") + ")",
             "bound": "hbm",
             "achieved": round(achieved, 1),
@@ -448,7 +476,7 @@ def run_gpu(args, w: si.Workload):
             "peak_kind": f"{peak_kind} hbm_gbs (copy bandwidth, burst)",
             "unit": "GB/s",
             "frac": round(achieved / peak, 4),
-            "traffic": _traffic_per_launch(w.name),
+            "traffic": None if (args.latent or args.unfused) else _traffic_per_launch(w.name),
             "algorithmic_bytes": bytes_per_dec,
             "decode_us": round(dec_us, 3),
             "decode_timing": f"{dec_reps} replays of a graph of {n_dec} back-to-back decode "
@@ -460,13 +488,13 @@ def run_gpu(args, w: si.Workload):
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "how": "per step one CUDA-graph replay of the public API calls with the "
                        "pinned host copies (inputs H2D, outputs D2H) inside"},
-        "gpu_launches": (3 if args.unfused else 1) * len(layers) * K,
+        "gpu_launches": (3 if args.unfused and not args.latent else 1) * len(layers) * K,
         "clocks": clocks,
         "wall_s_timed_region": round(t_wall, 3),
     }
     if compress is not None:
         result["compress"] = compress
-    if rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
+    if rank == 0 and ws_n == 1 and not args.no_cpu_baseline and not args.latent:
         result["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     if ws_n > 1:
         torch.distributed.destroy_process_group()
@@ -604,9 +632,16 @@ def run_profile_launches(args, w: si.Workload):
     vn = torch.randn((w.B, w.Hkv, w.d), generator=g, device=dev).to(torch.bfloat16)
     out = torch.empty_like(q)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
+    q_lat = torch.randn((w.B, w.Hq, lay.rK), generator=g, device=dev).to(torch.bfloat16)
+    o_lat = torch.empty((w.B, w.Hq, lay.rV), dtype=torch.bfloat16, device=dev)
     for _ in range(args.profile_launches):
         lay.seq_lens.fill_(w.L - 1)
-        if args.unfused:
+        if args.latent:
+            lay.seq_lens.fill_(w.L)
+            stief.stief_decode_latent(q_lat, lay.k_lat, lay.v_lat, lay.seq_lens, o_lat, lay.ws,
+                                      max_seq_len=L_max, num_splits=args.splits,
+                                      dev_status=status)
+        elif args.unfused:
             lay.seq_lens.fill_(w.L)
             stief.stief_decode_attention(q, lay.P_K, lay.P_V, lay.k_lat, lay.v_lat, lay.seq_lens,
                                          out, lay.ws, max_seq_len=L_max, num_splits=args.splits,
@@ -669,6 +704,9 @@ def main():
                     help="diagnostics: run only the first N layers of the workload")
     ap.add_argument("--splits", type=int, default=0,
                     help="diagnostics: force the decode split count (0 = automatic)")
+    ap.add_argument("--latent", action="store_true",
+                    help="time stief_decode_latent (bases folded into the attention weights) "
+                         "instead of the fused append + decode step")
     ap.add_argument("--unfused", action="store_true",
                     help="time the step as the two separate calls (append kernel, length "
                          "update, decode) instead of stief_append_decode")

@@ -76,6 +76,9 @@ def library() -> ctypes.CDLL:
             lib.stief_append_decode.restype = _i
             lib.stief_append_decode.argtypes = ([vp] * 10 + [ctypes.c_size_t] + [_i] * 9
                                                 + [vp, vp])
+            lib.stief_decode_latent.restype = _i
+            lib.stief_decode_latent.argtypes = ([vp] * 6 + [ctypes.c_size_t] + [_i] * 9
+                                                + [vp, vp])
             lib.stief_decode_attention_noalloc.restype = _i
             lib.stief_decode_attention_noalloc.argtypes = [vp] * 7 + [_i] * 9 + [vp, vp]
             lib.stief_read_device_status.restype = _i
@@ -260,6 +263,39 @@ def stief_append_decode(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tenso
                                          _opt_status(dev_status), _stream_ptr(stream))
     _check("stief_append_decode", code)
     return out
+
+
+def stief_decode_latent(q_lat: torch.Tensor, k_lat: torch.Tensor, v_lat: torch.Tensor,
+                        seq_lens: torch.Tensor, out_lat: torch.Tensor, workspace: torch.Tensor,
+                        max_seq_len: int, num_splits: int = 0, d: int = 128,
+                        dev_status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """The decode step in the latent space (bases folded into the attention weights):
+    out_lat [B][Hq][rV] = softmax(q_lat k_lat^T / sqrt(d)) v_lat.
+
+    q_lat [B][Hq][rK] bf16; k_lat [B][Hkv][L_max][rK], v_lat [B][Hkv][L_max][rV] bf16;
+    seq_lens [B] int32; out_lat [B][Hq][rV] bf16 (written); d the head dimension (score
+    scale); workspace as for stief_decode_attention.
+    """
+    pq = _dev(q_lat, "q_lat", torch.bfloat16, 3)
+    pkl = _dev(k_lat, "k_lat", torch.bfloat16, 4)
+    pvl = _dev(v_lat, "v_lat", torch.bfloat16, 4)
+    psl = _dev(seq_lens, "seq_lens", torch.int32, 1)
+    po = _dev(out_lat, "out_lat", torch.bfloat16, 3)
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    B, Hq, rK = q_lat.shape
+    Hkv, L_max = k_lat.shape[1], k_lat.shape[2]
+    rV = v_lat.shape[3]
+    if tuple(k_lat.shape) != (B, Hkv, L_max, rK) or tuple(v_lat.shape) != (B, Hkv, L_max, rV) \
+            or seq_lens.shape[0] != B or tuple(out_lat.shape) != (B, Hq, rV):
+        raise ValueError("stief_decode_latent: inconsistent shapes")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    code = library().stief_decode_latent(pq, pkl, pvl, psl, po, workspace.data_ptr(), ws_bytes,
+                                         B, Hq, Hkv, int(d), rK, rV, L_max, int(max_seq_len),
+                                         int(num_splits), _opt_status(dev_status),
+                                         _stream_ptr(stream))
+    _check("stief_decode_latent", code)
+    return out_lat
 
 
 def stief_decode_attention_noalloc(q: torch.Tensor, P_K: torch.Tensor, P_V: torch.Tensor,

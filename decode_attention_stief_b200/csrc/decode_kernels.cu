@@ -229,7 +229,7 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int NW, int ns, int rK,
 // NKS >= rK/16; NMV >= rV/16.
 constexpr int kMaxConsumerWarps = 8;
 
-template <int NB, int NKS, int NMV, int TT>
+template <int NB, int NKS, int NMV, int TT, bool LAT>
 __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
     stief_decode_kernel(const __grid_constant__ DecodeArgs a) {
   constexpr int kTile = TT;
@@ -359,7 +359,10 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
   bool ok = true;
   if (producer) {
     if (lane < 12 && lane < a.nmaps) prefetch_tensormap(&a.maps[lane]);
-    if (lane == 0) {
+    if (lane == 0 && LAT) {  // latent decode: the rows of q~ are the input
+      mbar_arrive_expect_tx(setup_bar, 2u * gcount * rK);
+      bulk_g2s(smem + L.qraw, a.q + ((size_t)b * a.Hq + h0) * rK, 2u * gcount * rK, setup_bar);
+    } else if (lane == 0) {
       // q and P_K first (they gate q~), then every warp's ring
       const uint64_t keep = l2_policy_evict_last();  // bases are shared by many CTAs
       mbar_arrive_expect_tx(setup_bar, 2u * d * rK + 2u * gcount * d + (owns_new ? 4u * d : 0u));
@@ -380,6 +383,14 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
         issue(lane, k, stream);
     }
     __syncwarp();
+  } else if (LAT) {
+    // q~ is given (bf16 [heads][r_K]): widen and scale it into log2 units; absent heads are 0
+    ok = warp_wait(setup_bar, 0, a.dev_status);
+    const uint16_t* qr = reinterpret_cast<const uint16_t*>(smem + L.qraw);
+    for (int i = tid; i < 8 * rK; i += NW * 32) {
+      const int h = i / rK, j = i - h * rK;
+      qt[h * xs + j] = h < gcount ? bf16_to_f32(qr[h * rK + j]) * a.qscale : 0.f;
+    }
   } else {
     // q~ = q P_K on the MMA: q~^T[j][head] = sum_i P_K[i][j] q[head][i]
     // (M = the r_K columns of P_K, N = 8 heads, K = d), scaled into log2 units
@@ -448,7 +459,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
 
   if (producer) {
     // ---- producer: P_V, the rest of every ring, then refills as stages are released ----
-    if (lane == 0) {
+    if (lane == 0 && !LAT) {
       fence_proxy_async_smem();  // P_V replaces P_K, read through the generic proxy above
       const uint64_t keep = l2_policy_evict_last();
       mbar_arrive_expect_tx(setup_bar, 2u * d * rV);
@@ -798,12 +809,21 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
   }
   __syncthreads();
 
+  // output columns per head: d, or r_V for the latent decode (o~ itself is the result)
+  const int od = LAT ? rV : d;
+  const int rec = od + 4;  // floats per partial state
+  float* parts = a.ws_part + unit * (size_t)S * G_T * rec;
+  if (LAT) {
+    for (int i = tid; i < gcount * rV; i += NT) {
+      const int h = i / rV, j = i - h * rV;
+      if (S == 1) a.out[((size_t)b * a.Hq + h0 + h) * rV + j] = f32_to_bf16_rn(qt[h * xs + j]);
+      else parts[((size_t)s_idx * G_T + h) * rec + j] = qt[h * xs + j];
+    }
+  }
   // ---- up-projection o = o~ P_V^T on the MMA: o^T[i][n] = sum_j P_V[i][j] o~^T[j][n] ----
   // (M = d, N = heads, K = r_V); warp w takes rows 16 w, 16 (w + NW + 1), ...
-  const int rec = d + 4;  // floats per partial state
-  float* parts = a.ws_part + unit * (size_t)S * G_T * rec;
-  if (!warp_wait(setup_bar, 1, a.dev_status)) ok = false;
-  for (int mt = warp; mt < d / 16 && ok; mt += NW + 1) {
+  if (!LAT && !warp_wait(setup_bar, 1, a.dev_status)) ok = false;
+  for (int mt = warp; mt < d / 16 && ok && !LAT; mt += NW + 1) {
     float c[NB][4];
 #pragma unroll
     for (int ks = 0; ks < NMV; ++ks)
@@ -833,8 +853,8 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
 
   // ---- split merge: publish this split, take a ticket; the last CTA merges them all ---------
   if (tid < gcount) {
-    parts[((size_t)s_idx * G_T + tid) * rec + d] = fin[tid];
-    parts[((size_t)s_idx * G_T + tid) * rec + d + 1] = fin[8 + tid];
+    parts[((size_t)s_idx * G_T + tid) * rec + od] = fin[tid];
+    parts[((size_t)s_idx * G_T + tid) * rec + od + 1] = fin[8 + tid];
   }
   __syncthreads();  // every state of this CTA is written (block scope) ...
   if (tid == 0) {
@@ -854,7 +874,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
   // Thread groups of tpi consecutive lanes take one item = (head, 4 output columns); lane
   // `sub` of a group merges splits sub, sub + tpi, ... (sixteen loads in flight at a time),
   // then the group combines its tpi running states with shuffles.
-  const int nitems = gcount * (d / 4);
+  const int nitems = gcount * (od / 4);
   int tpi = 1;
   while (tpi < 8 && tpi * 2 * nitems <= NT) tpi *= 2;
   const int sub = tid & (tpi - 1);
@@ -881,7 +901,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
   for (int it = 0; it < iters; ++it) {
     const int item = (it * NT + tid) / tpi;
     const bool valid = item < nitems;
-    const int g = valid ? item / (d / 4) : 0, c4 = valid ? item - g * (d / 4) : 0;
+    const int g = valid ? item / (od / 4) : 0, c4 = valid ? item - g * (od / 4) : 0;
     float M = -INFINITY, Ls = 0.f;
     float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int s0 = sub; s0 < S; s0 += kBatch * tpi) {
@@ -892,7 +912,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
         const int s = s0 + u * tpi;
         if (valid && s < S) {
           const float* r = parts + ((size_t)s * G_T + g) * rec;
-          const float2 m2 = __ldcg(reinterpret_cast<const float2*>(r + d));
+          const float2 m2 = __ldcg(reinterpret_cast<const float2*>(r + od));
           ms[u] = m2.x;
           ls[u] = m2.y;
           os[u] = __ldcg(reinterpret_cast<const float4*>(r) + c4);
@@ -919,17 +939,17 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
       uint2 packed;
       packed.x = pack_bf16x2_rn(o.x * inv, o.y * inv);
       packed.y = pack_bf16x2_rn(o.z * inv, o.w * inv);
-      *reinterpret_cast<uint2*>(a.out + ((size_t)b * a.Hq + h0 + g) * d + 4 * c4) = packed;
+      *reinterpret_cast<uint2*>(a.out + ((size_t)b * a.Hq + h0 + g) * od + 4 * c4) = packed;
     }
   }
 }
 
 // ------------------------------------------------------------------------------ launch
 
-template <int NB, int NKS, int NMV, int TT>
-static cudaError_t launch_t(const DecodeArgs& a, cudaStream_t stream) {
+template <int NB, int NKS, int NMV, int TT, bool LAT>
+static cudaError_t launch_k(const DecodeArgs& a, cudaStream_t stream) {
   const DecodeSmem L = decode_smem_layout(a.nwarps, a.nstage, a.rK, a.rV, TT);
-  auto kern = stief_decode_kernel<NB, NKS, NMV, TT>;
+  auto kern = stief_decode_kernel<NB, NKS, NMV, TT, LAT>;
   static SmemLimit limit;
   cudaError_t e = limit.ensure(reinterpret_cast<const void*>(kern), a.device, (int)L.total);
   if (e != cudaSuccess) return e;
@@ -946,6 +966,13 @@ static cudaError_t launch_t(const DecodeArgs& a, cudaStream_t stream) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+// the latent decode is its own instantiation, so its branches cost the other paths nothing
+template <int NB, int NKS, int NMV, int TT>
+static cudaError_t launch_t(const DecodeArgs& a, cudaStream_t stream) {
+  return a.latent ? launch_k<NB, NKS, NMV, TT, true>(a, stream)
+                  : launch_k<NB, NKS, NMV, TT, false>(a, stream);
 }
 
 uint32_t decode_smem_bytes(int nwarps, int nstage, int rK, int rV, int tile) {

@@ -152,8 +152,9 @@ stief_status plan_decode(DecodeArgs& a, const uint16_t* q, const uint16_t* P_K,
                          const uint16_t* P_V, const uint16_t* k_lat, const uint16_t* v_lat,
                          const int32_t* seq_lens, uint16_t* out, int B, int Hq, int Hkv, int d,
                          int rK, int rV, int L_max, int max_seq_len, int num_splits,
-                         uint32_t* dev_status) {
-  if (!q || !P_K || !P_V || !k_lat || !v_lat || !seq_lens || !out) return STIEF_ERR_INVALID_ARG;
+                         uint32_t* dev_status, bool latent) {
+  if (!q || !k_lat || !v_lat || !seq_lens || !out) return STIEF_ERR_INVALID_ARG;
+  if (!latent && (!P_K || !P_V)) return STIEF_ERR_INVALID_ARG;
   if (B < 1 || B > 65535 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || Hq / Hkv > 64)
     return STIEF_ERR_INVALID_ARG;
   if (d != 128 || !rank_ok(rK) || !rank_ok(rV) || L_max < 1 || max_seq_len < 0)
@@ -161,9 +162,9 @@ stief_status plan_decode(DecodeArgs& a, const uint16_t* q, const uint16_t* P_K,
   if (max_seq_len > L_max) return STIEF_ERR_CAPACITY;
   const int smax = stief_decode_max_splits(max_seq_len);
   if (num_splits < 0 || num_splits > smax) return STIEF_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(P_K) || !aligned16(P_V) || !aligned16(k_lat) ||
-      !aligned16(v_lat) || !aligned16(out))
+  if (!aligned16(q) || !aligned16(k_lat) || !aligned16(v_lat) || !aligned16(out))
     return STIEF_ERR_ALIGNMENT;
+  if (!latent && (!aligned16(P_K) || !aligned16(P_V))) return STIEF_ERR_ALIGNMENT;
   const uint64_t rows = (uint64_t)B * Hkv * L_max;
   if (rows >= (1ull << 31)) return STIEF_ERR_INVALID_ARG;  // TMA row coordinates are int32
 
@@ -172,6 +173,7 @@ stief_status plan_decode(DecodeArgs& a, const uint16_t* q, const uint16_t* P_K,
   if (!query_device(&dev, &sms, &sm100)) return STIEF_ERR_CUDA;
   if (!sm100) return STIEF_ERR_UNSUPPORTED_DEVICE;
   a.device = dev;
+  a.latent = latent ? 1 : 0;
 
   a.q = q;
   a.seq_lens = seq_lens;
@@ -199,9 +201,10 @@ stief_status plan_decode(DecodeArgs& a, const uint16_t* q, const uint16_t* P_K,
   int nmaps = 0;
   const uint64_t prow = (uint64_t)Hkv * d;
   if (!plan_pieces(a, &nmaps, a.pk, k_lat, rK, rows, a.tile) ||
-      !plan_pieces(a, &nmaps, a.pv, v_lat, rV, rows, a.tile) ||
-      !plan_pieces(a, &nmaps, a.ppk, P_K, rK, prow, d) ||
-      !plan_pieces(a, &nmaps, a.ppv, P_V, rV, prow, d))
+      !plan_pieces(a, &nmaps, a.pv, v_lat, rV, rows, a.tile))
+    return STIEF_ERR_CUDA;
+  if (!latent && (!plan_pieces(a, &nmaps, a.ppk, P_K, rK, prow, d) ||
+                  !plan_pieces(a, &nmaps, a.ppv, P_V, rV, prow, d)))
     return STIEF_ERR_CUDA;
   a.nmaps = nmaps;
   return STIEF_OK;

@@ -135,24 +135,26 @@ stief_status decode_common(const uint16_t* q, const uint16_t* k_new, const uint1
                            uint16_t* v_lat, int32_t* seq_lens, uint16_t* out, void* workspace,
                            size_t workspace_bytes, int B, int Hq, int Hkv, int d, int rK, int rV,
                            int L_max, int max_seq_len, int num_splits, uint32_t* dev_status,
-                           stief_stream_t stream, bool append) {
+                           stief_stream_t stream, bool append, bool latent = false) {
   // cheap host checks first, so argument errors never touch CUDA
-  if (!q || !P_K || !P_V || !k_lat || !v_lat || !seq_lens || !out) return STIEF_ERR_INVALID_ARG;
+  if (!q || !k_lat || !v_lat || !seq_lens || !out) return STIEF_ERR_INVALID_ARG;
+  if (!latent && (!P_K || !P_V)) return STIEF_ERR_INVALID_ARG;
   if (append && (!k_new || !v_new)) return STIEF_ERR_INVALID_ARG;
   stief_status st = check_decode_shape(B, Hq, Hkv, d, rK, rV, L_max, max_seq_len);
   if (st != STIEF_OK) return st;
   const int smax = stief_decode_max_splits(max_seq_len);
   if (num_splits < 0 || num_splits > smax) return STIEF_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(P_K) || !aligned16(P_V) || !aligned16(k_lat) ||
-      !aligned16(v_lat) || !aligned16(out) || !aligned16(workspace))
+  if (!aligned16(q) || !aligned16(k_lat) || !aligned16(v_lat) || !aligned16(out) ||
+      !aligned16(workspace))
     return STIEF_ERR_ALIGNMENT;
+  if (!latent && (!aligned16(P_K) || !aligned16(P_V))) return STIEF_ERR_ALIGNMENT;
   if (append && (!aligned16(k_new) || !aligned16(v_new))) return STIEF_ERR_ALIGNMENT;
   const size_t need = stief_decode_workspace_bytes(B, Hq, Hkv, rV, max_seq_len);
   if (!workspace || workspace_bytes < need) return STIEF_ERR_WORKSPACE;
 
   stief::DecodeArgs a{};
   st = stief::plan_decode(a, q, P_K, P_V, k_lat, v_lat, seq_lens, out, B, Hq, Hkv, d, rK, rV,
-                          L_max, max_seq_len, num_splits, dev_status);
+                          L_max, max_seq_len, num_splits, dev_status, latent);
   if (st != STIEF_OK) return st;
   a.append = append ? 1 : 0;
   a.k_new = k_new;
@@ -196,6 +198,17 @@ stief_status stief_append_decode(const uint16_t* q, const uint16_t* k_new, const
   return decode_common(q, k_new, v_new, P_K, P_V, k_lat, v_lat, seq_lens, out, workspace,
                        workspace_bytes, B, Hq, Hkv, d, rK, rV, L_max, max_seq_len, num_splits,
                        dev_status, stream, true);
+}
+
+stief_status stief_decode_latent(const uint16_t* q_lat, const uint16_t* k_lat,
+                                 const uint16_t* v_lat, const int32_t* seq_lens, uint16_t* out_lat,
+                                 void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv,
+                                 int d, int rK, int rV, int L_max, int max_seq_len, int num_splits,
+                                 uint32_t* dev_status, stief_stream_t stream) {
+  return decode_common(q_lat, nullptr, nullptr, nullptr, nullptr, const_cast<uint16_t*>(k_lat),
+                       const_cast<uint16_t*>(v_lat), const_cast<int32_t*>(seq_lens), out_lat,
+                       workspace, workspace_bytes, B, Hq, Hkv, d, rK, rV, L_max, max_seq_len,
+                       num_splits, dev_status, stream, false, true);
 }
 
 stief_status stief_read_device_status(const uint32_t* dev_status, uint32_t* value,

@@ -56,6 +56,7 @@ struct DecodeArgs {
   int nstage;       // shared-memory stages per warp
   float qscale;     // log2(e) / sqrt(d), applied to q . P_K
   int device;       // current device at planning time (host bookkeeping only)
+  int latent;       // latent decode: q holds q~ [B][Hq][rK], out is o~ [B][Hq][rV], no bases
 };
 
 struct CompressArgs {
@@ -107,11 +108,13 @@ uint32_t compress_tc_smem_bytes(int rK, int rV);
 
 // Validates a decode call and fills everything in `a` except the workspace pointers
 // (split count, group tiling, CTA configuration, key tensor maps).  Host only.
+// With `latent`, q is q~ [B][Hq][rK], out is o~ [B][Hq][rV] and P_K, P_V are unused (may be
+// NULL): no base tensor maps are planned.
 stief_status plan_decode(DecodeArgs& a, const uint16_t* q, const uint16_t* P_K,
                          const uint16_t* P_V, const uint16_t* k_lat, const uint16_t* v_lat,
                          const int32_t* seq_lens, uint16_t* out, int B, int Hq, int Hkv, int d,
                          int rK, int rV, int L_max, int max_seq_len, int num_splits,
-                         uint32_t* dev_status);
+                         uint32_t* dev_status, bool latent = false);
 
 // Decode workspace layout: `units` = B * Hkv * qsub split-ticket counters, then B sequence
 // tickets (uint32, padded together to 256 bytes), then units * G_T * splits partial states

@@ -127,7 +127,8 @@ STIEF_API int stief_decode_auto_splits(int B, int Hq, int Hkv, int max_seq_len, 
  * per-split partial states: for each query head, the split's up-projected
  * unnormalised output (d floats), its running maximum and sum, and two pad words.
  * rV is validated but does not change the size.  The same workspace serves
- * stief_append_decode.  Pure host function.  Returns 0 for invalid arguments.
+ * stief_append_decode and stief_decode_latent (whose partial states hold r_V <= d
+ * columns in the same records).  Pure host function.  Returns 0 for invalid arguments.
  */
 STIEF_API size_t stief_decode_workspace_bytes(int B, int Hq, int Hkv, int rV, int max_seq_len);
 
@@ -221,6 +222,41 @@ STIEF_API stief_status stief_append_decode(const uint16_t* q, const uint16_t* k_
                                  size_t workspace_bytes, int B, int Hq, int Hkv, int d, int rK,
                                  int rV, int L_max, int max_seq_len, int num_splits,
                                  uint32_t* dev_status, stief_stream_t stream);
+
+/*
+ * stief_decode_latent -- the decode step in the latent space only, for models whose
+ * attention weights absorb the bases (StiefAttention technical summary, "Mecanismo
+ * Central" item 5, last sentence: the projection bases can be folded into the
+ * attention's linear weights, at no extra run time over standard low-rank methods).
+ * With W_Q P_K as the query weight and P_V^T W_O as the output weight, the model
+ * hands over q~ directly and consumes o~; the query projection and the up-projection
+ * of stief_decode_attention drop out.
+ *
+ * For every sequence b and query head h (KV head g = h / (Hq/Hkv), L = seq_lens[b]):
+ *     s_t = q_lat[b][h] . k_lat[b][g][t] / sqrt(d)          t < L
+ *     out_lat[b][h] = bf16_RNE( sum_t softmax(s)_t v_lat[b][g][t] )
+ * i.e. stief_decode_attention with q~ given and o~ returned: for q_lat = q . P_K,
+ * out_lat . P_V^T equals stief_decode_attention's output up to rounding (q~ enters
+ * here as bf16, there as fp32).  Same split-KV online softmax, precision (q~, the
+ * softmax weights and o~ enter the tensor-core products as bf16 pairs, fp32
+ * accumulation), masking and L == 0 behaviour.
+ *
+ *   q_lat        : bf16 [B][Hq][rK]
+ *   k_lat, v_lat : bf16 [B][Hkv][L_max][rK], [B][Hkv][L_max][rV] (only read)
+ *   out_lat      : bf16 [B][Hq][rV] (written)
+ *   d            : the head dimension; sets the score scale 1/sqrt(d) (d == 128)
+ *   seq_lens, workspace, max_seq_len, num_splits, dev_status, stream: as for
+ *                  stief_decode_attention (same workspace size and rules)
+ *
+ * One kernel, as stief_decode_attention's without the base loads.
+ * Returns STIEF_OK or an argument error (nothing launched).
+ */
+STIEF_API stief_status stief_decode_latent(const uint16_t* q_lat, const uint16_t* k_lat,
+                                 const uint16_t* v_lat, const int32_t* seq_lens,
+                                 uint16_t* out_lat, void* workspace, size_t workspace_bytes,
+                                 int B, int Hq, int Hkv, int d, int rK, int rV, int L_max,
+                                 int max_seq_len, int num_splits, uint32_t* dev_status,
+                                 stief_stream_t stream);
 
 /*
  * stief_decode_attention_noalloc -- stief_decode_attention without a workspace

@@ -89,6 +89,28 @@ def test_decode_argument_errors(lib, kw, code):
     assert _decode(lib, **kw) == code
 
 
+def _latent(lib, **kw):
+    a = dict(q=FAKE, k_lat=FAKE, v_lat=FAKE, seq_lens=FAKE, out=FAKE, ws=FAKE, ws_bytes=1 << 40,
+             B=1, Hq=32, Hkv=8, d=128, rK=64, rV=48, L_max=1024, max_seq_len=1024, num_splits=0)
+    a.update(kw)
+    return lib.stief_decode_latent(a["q"], a["k_lat"], a["v_lat"], a["seq_lens"], a["out"],
+                                   a["ws"], a["ws_bytes"], a["B"], a["Hq"], a["Hkv"], a["d"],
+                                   a["rK"], a["rV"], a["L_max"], a["max_seq_len"],
+                                   a["num_splits"], None, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), INVALID), (dict(k_lat=None), INVALID), (dict(out=None), INVALID),
+    (dict(d=64), INVALID), (dict(rV=40), INVALID), (dict(Hq=30), INVALID),
+    (dict(num_splits=9), INVALID), (dict(max_seq_len=2048), CAPACITY),
+    (dict(q=FAKE + 8), ALIGN), (dict(v_lat=FAKE + 2), ALIGN), (dict(out=FAKE + 4), ALIGN),
+    (dict(ws=None), WORKSPACE), (dict(ws_bytes=16), WORKSPACE),
+])
+def test_latent_decode_argument_errors(lib, kw, code):
+    """The latent decode takes no bases: its checks are the decode's minus P_K / P_V."""
+    assert _latent(lib, **kw) == code
+
+
 @pytest.mark.parametrize("kw,code", [
     (dict(k=None), INVALID), (dict(sl=None), INVALID), (dict(d=96), INVALID),
     (dict(rK=24), INVALID), (dict(T=-1), INVALID), (dict(B=0), INVALID),
