@@ -196,7 +196,11 @@ stief_status plan_decode(DecodeArgs& a, const uint16_t* q, const uint16_t* P_K,
   a.tile = choose_decode_tile(rK, rV);
   a.chunk = ((max_seq_len + a.S - 1) / a.S + a.tile - 1) / a.tile * a.tile;
   a.qscale = (float)(1.4426950408889634 / std::sqrt((double)d));
-  if (!choose_decode_config(rK, rV, a.tile, &a.nwarps, &a.nstage)) return STIEF_ERR_INVALID_ARG;
+  const long long units = (long long)B * a.Hkv * a.qsub;
+  const bool pair = a.S == 1 && units > sms &&
+                    choose_decode_config_pair(rK, rV, a.tile, &a.nwarps, &a.nstage);
+  if (!pair && !choose_decode_config(rK, rV, a.tile, &a.nwarps, &a.nstage))
+    return STIEF_ERR_INVALID_ARG;
 
   int nmaps = 0;
   const uint64_t prow = (uint64_t)Hkv * d;

@@ -133,6 +133,24 @@ inline int choose_decode_tile(int rK, int rV) { return rK <= 64 && rV <= 64 && r
 
 // Consumer warps per CTA and stages per warp for the decode kernel: 8 warps with as many
 // stages (up to 8) as shared memory allows, fewer warps only when 8 cannot have two each.
+// Grids of more than one wave (one split, more units than SMs) run two CTAs per SM with a
+// smaller ring, so that one CTA's prologue and epilogue overlap the other's streaming (at
+// batch 64 x 8 KV heads x 4096 tokens: 87.8 instead of 100.7 us per launch).  Two CTAs fit
+// when each takes at most half of the SM's 228 KB less the 1 KB the system reserves per CTA,
+// and when 2 x (warps + producer) x 32 threads x 168 registers fit in 64 K: at most five
+// consumer warps.  Fewer than four consumer warps per CTA is not worth it.
+constexpr int kPairSmemPerBlock = 233472 / 2 - 1024;
+constexpr int kPairMaxConsumerWarps = 5;
+inline bool choose_decode_config_pair(int rK, int rV, int tile, int* nwarps, int* nstage) {
+  for (int nw = kPairMaxConsumerWarps; nw >= 4; --nw)
+    for (int ns = 4; ns >= 2; --ns)
+      if (decode_smem_bytes(nw, ns, rK, rV, tile) <= (uint32_t)kPairSmemPerBlock) {
+        *nwarps = nw;
+        *nstage = ns;
+        return true;
+      }
+  return false;
+}
 inline bool choose_decode_config(int rK, int rV, int tile, int* nwarps, int* nstage) {
   for (int nw = 8; nw >= 2; --nw)
     for (int ns = 8; ns >= 2; --ns)

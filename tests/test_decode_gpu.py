@@ -152,3 +152,17 @@ def test_workspace_counters_return_to_zero_and_partials_may_hold_garbage():
         torch.cuda.synchronize()
         assert int(ws[:counter_bytes].count_nonzero()) == 0
         assert_decode_close(out.cpu(), want)
+
+
+@pytest.mark.parametrize("rK,rV", [(64, 64), (32, 96), (32, 48)])
+def test_multi_wave_grid_two_ctas_per_sm(rK, rV):
+    """More (sequence, KV head) units than SMs with one split: the planner runs two CTAs per
+    SM with a smaller ring; ragged lengths, an empty sequence and tile tails included."""
+    B = 40  # 40 x 8 KV heads = 320 units, more than the 148 SMs
+    rng = np.random.default_rng(990 + rK)
+    lens = rng.integers(1, 300, size=B).tolist()
+    lens[3] = 0
+    lens[7] = 300
+    got, want, _ = _run(B, 32, 8, rK, rV, 300, lens, 991 + rK + rV)
+    assert_decode_close(got, want)
+    assert torch.all(got[3].float() == 0)

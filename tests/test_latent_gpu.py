@@ -140,3 +140,11 @@ def test_full_size_one_layer(name):
     err = decode_error(got, want)
     print(f"\n  {name} latent decode: max|err| / ||o~||_inf = {err:.3e}")
     assert err <= DECODE_TOL
+
+
+def test_multi_wave_grid_two_ctas_per_sm():
+    """The latent decode on a grid of more units than SMs (two CTAs per SM)."""
+    lens = [257, 1, 0, 300] * 10
+    q, k, v = _case(40, 32, 8, 64, 64, 300, 4800)
+    got = _gpu_latent(q, k, v, lens)
+    assert_decode_close(got, _oracle(q, k, v, lens))
