@@ -28,11 +28,11 @@
 //   rescaled when a head's maximum passes its running reference by more than 8)
 //   mix     O^T[dim][n] += V_down^T[dim][token] . P^T[token][n]  (M = r_V dims, K = tokens)
 // where P^T comes from the score accumulators through an in-register 8x8 transpose
-// (movmatrix).  The epilogue merges the warps (log-sum-exp), up-projects with P_V^T
-// on the same MMA (M = d, K = r_V), and either writes the output (one split) or
-// stores an up-projected partial state and takes a ticket; the last CTA of the unit
-// merges the splits and resets the ticket counter, so the workspace counters stay
-// zero between calls.
+// (movmatrix).  The epilogue merges the warps (log-sum-exp); with one split it
+// up-projects with P_V^T on the same MMA (M = d, K = r_V) and writes the output,
+// otherwise it stores the latent partial state (o~, m, l) and takes a ticket: the last
+// CTA of the unit merges the splits, up-projects once and resets the ticket counter,
+// so the workspace counters stay zero between calls.
 #include <cfloat>
 #include <cmath>
 #include <cstdint>
@@ -809,52 +809,59 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
   }
   __syncthreads();
 
-  // output columns per head: d, or r_V for the latent decode (o~ itself is the result)
-  const int od = LAT ? rV : d;
-  const int rec = od + 4;  // floats per partial state
-  float* parts = a.ws_part + unit * (size_t)S * G_T * rec;
-  if (LAT) {
-    for (int i = tid; i < gcount * rV; i += NT) {
-      const int h = i / rV, j = i - h * rV;
-      if (S == 1) a.out[((size_t)b * a.Hq + h0 + h) * rV + j] = f32_to_bf16_rn(qt[h * xs + j]);
-      else parts[((size_t)s_idx * G_T + h) * rec + j] = qt[h * xs + j];
-    }
-  }
   // ---- up-projection o = o~ P_V^T on the MMA: o^T[i][n] = sum_j P_V[i][j] o~^T[j][n] ----
-  // (M = d, N = heads, K = r_V); warp w takes rows 16 w, 16 (w + NW + 1), ...
-  if (!LAT && !warp_wait(setup_bar, 1, a.dev_status)) ok = false;
-  for (int mt = warp; mt < d / 16 && ok && !LAT; mt += NW + 1) {
-    float c[NB][4];
+  // (M = d, N = heads, K = r_V) from the normalised o~ in qt; warp w takes rows 16 w,
+  // 16 (w + NW + 1), ...
+  auto up_project = [&]() {
+    if (!warp_wait(setup_bar, 1, a.dev_status)) return;
+    for (int mt = warp; mt < d / 16; mt += NW + 1) {
+      float c[NB][4];
 #pragma unroll
-    for (int ks = 0; ks < NMV; ++ks)
-      if (ks < nmv) {
-        uint32_t af[4];
-        const PieceLoc pl = locate(rV, d, 2 * ks + a_chunk(lane));
-        ldsm_x4(smem_u32(pmat) + swz(pl, 16 * mt + a_row(lane)), af);
-        uint32_t bf[NB][2];
-        bfrag_hilo<NB>(qt, xs, ks, lane, bf);
+      for (int ks = 0; ks < NMV; ++ks)
+        if (ks < nmv) {
+          uint32_t af[4];
+          const PieceLoc pl = locate(rV, d, 2 * ks + a_chunk(lane));
+          ldsm_x4(smem_u32(pmat) + swz(pl, 16 * mt + a_row(lane)), af);
+          uint32_t bf[NB][2];
+          bfrag_hilo<NB>(qt, xs, ks, lane, bf);
 #pragma unroll
-        for (int j = 0; j < NB; ++j) {
-          if (ks == 0) mma_bf16_z(c[j], af, bf[j][0], bf[j][1]);
-          else mma_bf16(c[j], af, bf[j][0], bf[j][1]);
+          for (int j = 0; j < NB; ++j) {
+            if (ks == 0) mma_bf16_z(c[j], af, bf[j][0], bf[j][1]);
+            else mma_bf16(c[j], af, bf[j][0], bf[j][1]);
+          }
         }
-      }
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float o = NB == 1 ? c[0][e] + __shfl_xor_sync(kFull, c[0][e], 2) : c[0][e] + c[NB - 1][e];
-      const int head = hA + (e & 1), i = 16 * mt + (lane >> 2) + 8 * (e >> 1);
-      if (!lo_lane && head < gcount) {
-        if (S == 1) a.out[((size_t)b * a.Hq + h0 + head) * d + i] = f32_to_bf16_rn(o);
-        else parts[((size_t)s_idx * G_T + head) * rec + i] = o;
+      for (int e = 0; e < 4; ++e) {
+        const float o = NB == 1 ? c[0][e] + __shfl_xor_sync(kFull, c[0][e], 2) : c[0][e] + c[NB - 1][e];
+        const int head = hA + (e & 1), i = 16 * mt + (lane >> 2) + 8 * (e >> 1);
+        if (!lo_lane && head < gcount) a.out[((size_t)b * a.Hq + h0 + head) * d + i] = f32_to_bf16_rn(o);
       }
     }
+  };
+  if (S == 1) {  // this CTA finishes the unit alone: qt holds the normalised o~
+    if (LAT) {
+      for (int i = tid; i < gcount * rV; i += NT) {
+        const int h = i / rV, j = i - h * rV;
+        a.out[((size_t)b * a.Hq + h0 + h) * rV + j] = f32_to_bf16_rn(qt[h * xs + j]);
+      }
+    } else if (ok) {
+      up_project();
+    }
+    return;
   }
-  if (S == 1) return;
+  // Split partial states stay in the latent space (o~ scaled to the CTA's maximum, r_V floats
+  // per head, then m and l): the last CTA merges them and up-projects once.
+  const int rec = rV + 4;  // floats per partial state
+  float* parts = a.ws_part + unit * (size_t)S * G_T * rec;
+  for (int i = tid; i < gcount * rV; i += NT) {
+    const int h = i / rV, j = i - h * rV;
+    parts[((size_t)s_idx * G_T + h) * rec + j] = qt[h * xs + j];
+  }
 
   // ---- split merge: publish this split, take a ticket; the last CTA merges them all ---------
   if (tid < gcount) {
-    parts[((size_t)s_idx * G_T + tid) * rec + od] = fin[tid];
-    parts[((size_t)s_idx * G_T + tid) * rec + od + 1] = fin[8 + tid];
+    parts[((size_t)s_idx * G_T + tid) * rec + rV] = fin[tid];
+    parts[((size_t)s_idx * G_T + tid) * rec + rV + 1] = fin[8 + tid];
   }
   __syncthreads();  // every state of this CTA is written (block scope) ...
   if (tid == 0) {
@@ -870,11 +877,16 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
     *flag = last;
   }
   __syncthreads();
-  if (!*flag) return;
+  if (!*flag) {
+    // P_V is only used by the merging CTA, but its copy must land before this CTA's shared
+    // memory is released (it was requested long before; the wait is bounded)
+    if (!LAT && tid == 0) mbar_wait_bounded(setup_bar, 1u, a.dev_status);
+    return;
+  }
   // Thread groups of tpi consecutive lanes take one item = (head, 4 output columns); lane
-  // `sub` of a group merges splits sub, sub + tpi, ... (sixteen loads in flight at a time),
+  // `sub` of a group merges splits sub, sub + tpi, ... (a batch of eight in flight at a time),
   // then the group combines its tpi running states with shuffles.
-  const int nitems = gcount * (od / 4);
+  const int nitems = gcount * (rV / 4);
   int tpi = 1;
   while (tpi < 8 && tpi * 2 * nitems <= NT) tpi *= 2;
   const int sub = tid & (tpi - 1);
@@ -897,11 +909,11 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
     o.z = fmaf(w, o2.z, o.z);
     o.w = fmaf(w, o2.w, o.w);
   };
-  constexpr int kBatch = 16;
+  constexpr int kBatch = 8;
   for (int it = 0; it < iters; ++it) {
     const int item = (it * NT + tid) / tpi;
     const bool valid = item < nitems;
-    const int g = valid ? item / (od / 4) : 0, c4 = valid ? item - g * (od / 4) : 0;
+    const int g = valid ? item / (rV / 4) : 0, c4 = valid ? item - g * (rV / 4) : 0;
     float M = -INFINITY, Ls = 0.f;
     float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int s0 = sub; s0 < S; s0 += kBatch * tpi) {
@@ -912,7 +924,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
         const int s = s0 + u * tpi;
         if (valid && s < S) {
           const float* r = parts + ((size_t)s * G_T + g) * rec;
-          const float2 m2 = __ldcg(reinterpret_cast<const float2*>(r + od));
+          const float2 m2 = __ldcg(reinterpret_cast<const float2*>(r + rV));
           ms[u] = m2.x;
           ls[u] = m2.y;
           os[u] = __ldcg(reinterpret_cast<const float4*>(r) + c4);
@@ -922,8 +934,22 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
           os[u] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
       }
+      // the batch's maximum first, then independent weights and sums (short dependency chains)
+      float Mb = -INFINITY;
 #pragma unroll
-      for (int u = 0; u < kBatch; ++u) merge(M, Ls, o, ms[u], ls[u], os[u]);
+      for (int u = 0; u < kBatch; ++u) Mb = fmaxf(Mb, ms[u]);
+      float Lb2 = 0.f;
+      float4 ob = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const float w = ms[u] == -INFINITY ? 0.f : ex2(ms[u] - Mb);
+        Lb2 = fmaf(w, ls[u], Lb2);
+        ob.x = fmaf(w, os[u].x, ob.x);
+        ob.y = fmaf(w, os[u].y, ob.y);
+        ob.z = fmaf(w, os[u].z, ob.z);
+        ob.w = fmaf(w, os[u].w, ob.w);
+      }
+      merge(M, Ls, o, Mb, Lb2, ob);
     }
     for (int off = 1; off < tpi; off <<= 1) {
       const float M2 = __shfl_xor_sync(kFull, M, off), L2 = __shfl_xor_sync(kFull, Ls, off);
@@ -936,11 +962,23 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
     }
     if (valid && sub == 0) {
       const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
-      uint2 packed;
-      packed.x = pack_bf16x2_rn(o.x * inv, o.y * inv);
-      packed.y = pack_bf16x2_rn(o.z * inv, o.w * inv);
-      *reinterpret_cast<uint2*>(a.out + ((size_t)b * a.Hq + h0 + g) * od + 4 * c4) = packed;
+      if (LAT) {  // o~ is the result
+        uint2 packed;
+        packed.x = pack_bf16x2_rn(o.x * inv, o.y * inv);
+        packed.y = pack_bf16x2_rn(o.z * inv, o.w * inv);
+        *reinterpret_cast<uint2*>(a.out + ((size_t)b * a.Hq + h0 + g) * rV + 4 * c4) = packed;
+      } else {  // the normalised o~ becomes the up-projection's operand
+        float* dst = qt + g * xs + 4 * c4;
+        dst[0] = o.x * inv;
+        dst[1] = o.y * inv;
+        dst[2] = o.z * inv;
+        dst[3] = o.w * inv;
+      }
     }
+  }
+  if (!LAT) {
+    __syncthreads();
+    up_project();
   }
 }
 

@@ -46,7 +46,7 @@ struct DecodeArgs {
   int32_t* seq_lens_w;
   uint32_t* ws_seq;  // [B] per-sequence finish tickets; zero between calls
   uint32_t* ws_cnt;  // [units] split tickets; zero between calls
-  float* ws_part;    // [units * S * G_T][d + 4] partial states: o[d] (up-projected), m, l, 0, 0
+  float* ws_part;    // [units * S * G_T][rV + 4] partial states: o~[rV] (latent), m, l, 0, 0
   uint32_t* dev_status;
   int B, Hq, Hkv, G, G_T, qsub, d, rK, rV, L_max, S;
   int max_seq_len;  // host bound of seq_lens; the splits partition [0, S * chunk)
@@ -118,7 +118,7 @@ stief_status plan_decode(DecodeArgs& a, const uint16_t* q, const uint16_t* P_K,
 
 // Decode workspace layout: `units` = B * Hkv * qsub split-ticket counters, then B sequence
 // tickets (uint32, padded together to 256 bytes), then units * G_T * splits partial states
-// of (d + 4) floats.
+// of (d + 4) floats (the kernel uses r_V + 4 <= d + 4 of each).
 inline size_t decode_ws_counter_bytes(size_t units, size_t B) {
   return ((units + B) * 4u + 255u) / 256u * 256u;
 }

@@ -124,11 +124,12 @@ STIEF_API int stief_decode_auto_splits(int B, int Hq, int Hkv, int max_seq_len, 
  * needs for these sizes, for any split count it may use (at most
  * stief_decode_max_splits(max_seq_len)).  The workspace holds one ticket counter
  * per (sequence, KV head, query sub-group) and one per sequence, followed by the
- * per-split partial states: for each query head, the split's up-projected
- * unnormalised output (d floats), its running maximum and sum, and two pad words.
- * rV is validated but does not change the size.  The same workspace serves
- * stief_append_decode and stief_decode_latent (whose partial states hold r_V <= d
- * columns in the same records).  Pure host function.  Returns 0 for invalid arguments.
+ * per-split partial states: for each query head, the split's unnormalised latent
+ * output o~ (r_V floats), its running maximum and sum, and two pad words; the last
+ * CTA of a (sequence, KV head, sub-group) merges them and up-projects once.  The size
+ * is computed for records of d + 4 floats (r_V <= d), so rV is validated but does not
+ * change it.  The same workspace serves stief_append_decode and stief_decode_latent.
+ * Pure host function.  Returns 0 for invalid arguments.
  */
 STIEF_API size_t stief_decode_workspace_bytes(int B, int Hq, int Hkv, int rV, int max_seq_len);
 
