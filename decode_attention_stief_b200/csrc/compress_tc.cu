@@ -10,14 +10,19 @@
 //   - X tiles arrive by 2-D TMA tensor copies with the 128-byte swizzle, in two 64-column
 //     atoms: exactly the canonical K-major SW128 operand layout of the MMA;
 //   - P[h] is written once per CTA, transposed into the same K-major SW128 layout
-//     (rows n = latent column, 128 bytes of k per row and atom);
+//     (rows n = latent column, 128 bytes of k per row and atom), all its loads in flight
+//     at once;
 //   - one thread issues tcgen05.mma; completion is signalled by tcgen05.commit on an
 //     mbarrier; the accumulators live in 256 columns of tensor memory (D_K at column
 //     0, D_V at column 128);
 //   - epilogue: each of 4 warps reads its 32 TMEM lanes (rows) with tcgen05.ld, rounds
 //     to bf16 (RNE) and stores its rows into the latent cache at seq_lens[b] + row.
-// A CTA loops over m-tiles of one (b, h) so P is staged once.  Every wait is bounded;
-// tensor memory is always released before the CTA exits.
+// A CTA loops over m-tiles of one (b, h) so P is staged once.  Its X tiles stream
+// through a two-stage ring: the first two are requested at kernel entry (the bases are
+// staged and the length is read while they fly), and the copy of tile i + 2 is issued as
+// soon as tile i's MMA has consumed its stage, so loads overlap the MMA and the epilogue.
+// Every wait is bounded; every requested copy lands and tensor memory is released before
+// the CTA exits.
 #include <cstdint>
 
 #include "stief_device.cuh"
@@ -28,14 +33,16 @@ namespace stief {
 namespace {
 
 constexpr int kTcRows = 128;     // M: rows (tokens) per MMA tile
+constexpr int kTcStages = 2;     // X tiles in flight per CTA
 constexpr int kTcThreads = 128;  // 4 warps: TMEM lanes 32w .. 32w + 31
 constexpr uint32_t kTmemCols = 256;
 
 // Shared-memory layout (byte offsets, all swizzled operands 1 KiB aligned).
 struct TcSmem {
-  uint32_t xk[2], xv[2];  // X tiles, two 64-column atoms each: 128 rows x 128 B
+  uint32_t xk[kTcStages][2], xv[kTcStages][2];  // X tiles per stage, two 64-column atoms:
+                                                // 128 rows x 128 B each
   uint32_t pk[2], pv[2];  // transposed bases, two atoms each: r rows x 128 B
-  uint32_t bars;          // tma, mma
+  uint32_t bars;          // tma[kTcStages], mma
   uint32_t tmem_slot;     // tcgen05.alloc writes the TMEM base address here
   uint32_t total;
 };
@@ -43,12 +50,15 @@ struct TcSmem {
 __host__ __device__ inline TcSmem tc_smem_layout(int rK, int rV) {
   TcSmem s;
   uint32_t off = 0;
-  for (int i = 0; i < 2; ++i) { s.xk[i] = off; off += kTcRows * 128; }
-  for (int i = 0; i < 2; ++i) { s.xv[i] = off; off += kTcRows * 128; }
+  for (int st = 0; st < kTcStages; ++st) {
+    for (int i = 0; i < 2; ++i) { s.xk[st][i] = off; off += kTcRows * 128; }
+    for (int i = 0; i < 2; ++i) { s.xv[st][i] = off; off += kTcRows * 128; }
+  }
   for (int i = 0; i < 2; ++i) { s.pk[i] = off; off += (uint32_t)rK * 128; off = (off + 1023) & ~1023u; }
   for (int i = 0; i < 2; ++i) { s.pv[i] = off; off += (uint32_t)rV * 128; off = (off + 1023) & ~1023u; }
   s.bars = off;
-  off += 16;
+  off += 8 * (kTcStages + 1);
+  off = (off + 15) & ~15u;
   s.tmem_slot = off;
   off += 16;
   s.total = off;
@@ -111,24 +121,34 @@ __device__ __forceinline__ void tc_fence_after() {
 }
 
 // P[h] ([128][r] row-major in global) -> shared [r rows][128 k] K-major SW128, two atoms.
-__device__ __forceinline__ void stage_basis(uint8_t* smem, const uint32_t (&atom)[2],
-                                            const uint16_t* P, int r, int tid) {
-  // thread = row k of P (128 threads, d = 128); each writes its k into every row n
+// Thread = row k of P (128 threads, d = 128): it reads its row of both bases first (all
+// loads in flight together), then writes its k into every row n of each.
+__device__ __forceinline__ void stage_bases(uint8_t* smem, const uint32_t (&atk)[2],
+                                            const uint32_t (&atv)[2], const uint16_t* PK,
+                                            const uint16_t* PV, int rK, int rV, int tid) {
+  constexpr int kMaxChunks = 16;  // r <= 128: 16 chunks of 8 columns
   const int k = tid;
-  const uint16_t* src = P + (size_t)k * r;
-  const uint32_t at = atom[k >> 6];
+  uint4 wk[kMaxChunks], wv[kMaxChunks];
+#pragma unroll
+  for (int q = 0; q < kMaxChunks; ++q) {
+    if (8 * q < rK) wk[q] = __ldg(reinterpret_cast<const uint4*>(PK + (size_t)k * rK) + q);
+    if (8 * q < rV) wv[q] = __ldg(reinterpret_cast<const uint4*>(PV + (size_t)k * rV) + q);
+  }
   const uint32_t kb = (uint32_t)(k & 63) * 2u;  // byte of k inside the 128-byte row
-  for (int n0 = 0; n0 < r; n0 += 8) {
-    const uint4 w = *reinterpret_cast<const uint4*>(src + n0);
-    const uint16_t v[8] = {(uint16_t)(w.x & 0xFFFF), (uint16_t)(w.x >> 16), (uint16_t)(w.y & 0xFFFF),
-                           (uint16_t)(w.y >> 16),    (uint16_t)(w.z & 0xFFFF), (uint16_t)(w.z >> 16),
-                           (uint16_t)(w.w & 0xFFFF), (uint16_t)(w.w >> 16)};
+  auto put = [&](const uint32_t (&atom)[2], const uint4& w, int n0) {
+    const uint32_t at = atom[k >> 6];
+    const uint32_t v[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int n = n0 + j;
       const uint32_t off = at + (uint32_t)n * 128u + ((((kb >> 4) ^ (uint32_t)(n & 7)) << 4) | (kb & 15u));
-      *reinterpret_cast<uint16_t*>(smem + off) = v[j];
+      *reinterpret_cast<uint16_t*>(smem + off) = (uint16_t)(v[j >> 1] >> (16 * (j & 1)));
     }
+  };
+#pragma unroll
+  for (int q = 0; q < kMaxChunks; ++q) {
+    if (8 * q < rK) put(atk, wk[q], 8 * q);
+    if (8 * q < rV) put(atv, wv[q], 8 * q);
   }
 }
 
@@ -149,24 +169,36 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int h = blockIdx.y, b = blockIdx.z;
   const int rK = a.rK, rV = a.rV, T = a.T;
   const TcSmem L = tc_smem_layout(rK, rV);
-  uint64_t* tma_bar = reinterpret_cast<uint64_t*>(smem + L.bars);
-  uint64_t* mma_bar = tma_bar + 1;
+  uint64_t* tma_bar = reinterpret_cast<uint64_t*>(smem + L.bars);  // [kTcStages]
+  uint64_t* mma_bar = tma_bar + kTcStages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.tmem_slot);
+  const int64_t head_row = ((int64_t)b * a.Hkv + h) * T;
+  const int my_tiles = (int)blockIdx.x < ta.tiles ? (ta.tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
+  auto tile_m0 = [&](int i) { return ((int)blockIdx.x + i * (int)gridDim.x) * kTcRows; };
+  int issued = 0;  // copies requested (thread 0 only)
+  auto issue = [&](int i) {  // thread 0: tile i of this CTA into stage i % kTcStages
+    const int st = i % kTcStages;
+    const uint64_t pol = l2_policy_evict_first();
+    mbar_arrive_expect_tx(&tma_bar[st], 4u * kTcRows * 128u);
+    const int y = (int)(head_row + tile_m0(i));
+    for (int at = 0; at < 2; ++at) {
+      tma_load_2d(smem + L.xk[st][at], &ta.mk, 64 * at, y, &tma_bar[st], pol);
+      tma_load_2d(smem + L.xv[st][at], &ta.mv, 64 * at, y, &tma_bar[st], pol);
+    }
+    issued = i + 1;
+  };
 
   pdl_launch_dependents();
-  const int Lb = a.seq_lens[b];
-  const bool bad = Lb < 0 || Lb > a.L_max;
-  const bool full = !bad && (long long)Lb + T > a.L_max;
-  if (tid == 0 && blockIdx.x == 0 && h == 0) {
-    if (bad) report(a.dev_status, STIEF_DEV_BAD_LENGTH);
-    if (full) report(a.dev_status, STIEF_DEV_CAPACITY_OVERFLOW);
-  }
-  if (bad || full) return;
   if ((smem_u32(smem) & 1023u) != 0) {  // swizzled operands need 1 KiB alignment
     if (tid == 0) report(a.dev_status, STIEF_DEV_SMEM_ALIGN);
     return;
   }
-
+  if (tid == 0) {
+    for (int st = 0; st < kTcStages + 1; ++st) mbar_init(&tma_bar[st], 1);
+    fence_barrier_init();
+    // the first tiles fly while the bases are staged and the length is read
+    for (int i = 0; i < kTcStages && i < my_tiles; ++i) issue(i);
+  }
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(tmem_slot)),
@@ -174,59 +206,55 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  if (tid == 0) {
-    mbar_init(tma_bar, 1);
-    mbar_init(mma_bar, 1);
-    fence_barrier_init();
+  stage_bases(smem, L.pk, L.pv, a.P_K + (size_t)h * 128 * rK, a.P_V + (size_t)h * 128 * rV, rK, rV,
+              tid);
+  const int Lb = a.seq_lens[b];
+  const bool bad = Lb < 0 || Lb > a.L_max;
+  const bool full = !bad && (long long)Lb + T > a.L_max;
+  if (tid == 0 && blockIdx.x == 0 && h == 0) {
+    if (bad) report(a.dev_status, STIEF_DEV_BAD_LENGTH);
+    if (full) report(a.dev_status, STIEF_DEV_CAPACITY_OVERFLOW);
   }
-  stage_basis(smem, L.pk, a.P_K + (size_t)h * 128 * rK, rK, tid);
-  stage_basis(smem, L.pv, a.P_V + (size_t)h * 128 * rV, rV, tid);
   fence_proxy_async_smem();  // the generic-proxy basis writes must be seen by the MMA
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t idK = idesc_bf16_f32(rK), idV = idesc_bf16_f32(rV);
-  const int64_t head_row = ((int64_t)b * a.Hkv + h) * T;
-  bool ok = true;
-  int phase = 0;
+  bool ok = !(bad || full);
+  int consumed = 0;  // tiles whose copy has been waited for
 
-  for (int mt = blockIdx.x; mt < ta.tiles && ok; mt += gridDim.x) {
-    const int m0 = mt * kTcRows;
-    if (tid == 0) {
-      const uint64_t pol = l2_policy_evict_first();
-      mbar_arrive_expect_tx(tma_bar, 4u * kTcRows * 128u);
-      const int y = (int)(head_row + m0);
-      for (int i = 0; i < 2; ++i) {
-        tma_load_2d(smem + L.xk[i], &ta.mk, 64 * i, y, tma_bar, pol);
-        tma_load_2d(smem + L.xv[i], &ta.mv, 64 * i, y, tma_bar, pol);
-      }
-    }
+  for (int i = 0; i < my_tiles && ok; ++i) {
+    const int st = i % kTcStages;
+    const uint32_t tphase = (uint32_t)((i / kTcStages) & 1);
     // a timed-out wait ends the loop for the whole CTA (tcgen05 ops below are warp-wide)
-    if (__syncthreads_or(!mbar_wait_bounded(tma_bar, phase, a.dev_status))) {
+    if (__syncthreads_or(!mbar_wait_bounded(&tma_bar[st], tphase, a.dev_status))) {
       ok = false;
       break;
     }
+    consumed = i + 1;
     if (tid == 0) {
       tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {  // K = 128 in steps of 16 (32 bytes inside an atom)
         const uint32_t koff = (uint32_t)(kk & 3) * 32u;
-        umma_bf16(tmem, sw128_desc(smem_u32(smem + L.xk[kk >> 2]) + koff),
+        umma_bf16(tmem, sw128_desc(smem_u32(smem + L.xk[st][kk >> 2]) + koff),
                   sw128_desc(smem_u32(smem + L.pk[kk >> 2]) + koff), idK, kk > 0);
-        umma_bf16(tmem + 128u, sw128_desc(smem_u32(smem + L.xv[kk >> 2]) + koff),
+        umma_bf16(tmem + 128u, sw128_desc(smem_u32(smem + L.xv[st][kk >> 2]) + koff),
                   sw128_desc(smem_u32(smem + L.pv[kk >> 2]) + koff), idV, kk > 0);
       }
       umma_commit(mma_bar);
     }
-    if (__syncthreads_or(!mbar_wait_bounded(mma_bar, phase, a.dev_status))) {
+    if (__syncthreads_or(!mbar_wait_bounded(mma_bar, (uint32_t)(i & 1), a.dev_status))) {
       ok = false;
       break;
     }
     tc_fence_after();
-    phase ^= 1;
+    // the MMA has read stage st: refill it with tile i + kTcStages
+    if (tid == 0 && i + kTcStages < my_tiles) issue(i + kTcStages);
 
     // epilogue: warp w owns rows 32w .. 32w + 31 (TMEM lanes); lane = row
+    const int m0 = tile_m0(i);
     const int row = warp * 32 + lane;
     const bool live = m0 + row < T;
     const size_t cache_row = ((size_t)b * a.Hkv + h) * a.L_max + Lb + m0 + row;
@@ -258,10 +286,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncthreads();
   }
 
-  if (!ok && tid == 0) {
-    // give an outstanding copy or MMA a bounded chance to finish before memory is released
-    mbar_wait_bounded(tma_bar, phase, nullptr);
-    mbar_wait_bounded(mma_bar, phase, nullptr);
+  if (tid == 0) {
+    // every requested copy must land before the shared memory is released (bounded waits;
+    // on the normal path nothing is outstanding), and an MMA left by a timeout gets a
+    // bounded chance to finish
+    for (int j = consumed; j < issued; ++j)
+      mbar_wait_bounded(&tma_bar[j % kTcStages], (uint32_t)((j / kTcStages) & 1), nullptr);
+    if (!ok && consumed > 0) mbar_wait_bounded(mma_bar, (uint32_t)((consumed - 1) & 1), nullptr);
   }
   tc_fence_before();
   __syncthreads();
