@@ -14,8 +14,11 @@ from ._binding import (  # noqa: F401
     library,
     library_path,
     stief_append_decode,
+    stief_append_decode_paged,
     stief_compress_append,
+    stief_compress_append_paged,
     stief_decode_attention,
+    stief_decode_attention_paged,
     stief_decode_attention_noalloc,
     stief_decode_auto_splits,
     stief_decode_latent,

@@ -76,6 +76,14 @@ def library() -> ctypes.CDLL:
             lib.stief_append_decode.restype = _i
             lib.stief_append_decode.argtypes = ([vp] * 10 + [ctypes.c_size_t] + [_i] * 9
                                                 + [vp, vp])
+            lib.stief_compress_append_paged.restype = _i
+            lib.stief_compress_append_paged.argtypes = [vp] * 8 + [_i] * 9 + [vp, vp]
+            lib.stief_decode_attention_paged.restype = _i
+            lib.stief_decode_attention_paged.argtypes = ([vp] * 9 + [ctypes.c_size_t] + [_i] * 11
+                                                         + [vp, vp])
+            lib.stief_append_decode_paged.restype = _i
+            lib.stief_append_decode_paged.argtypes = ([vp] * 11 + [ctypes.c_size_t] + [_i] * 11
+                                                      + [vp, vp])
             lib.stief_decode_latent.restype = _i
             lib.stief_decode_latent.argtypes = ([vp] * 6 + [ctypes.c_size_t] + [_i] * 9
                                                 + [vp, vp])
@@ -262,6 +270,99 @@ def stief_append_decode(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tenso
                                          L_max, int(max_seq_len), int(num_splits),
                                          _opt_status(dev_status), _stream_ptr(stream))
     _check("stief_append_decode", code)
+    return out
+
+
+def _pages(k_pages, v_pages, block_table, B):
+    """Pointers and sizes of a paged cache: pools [num_pages][Hkv][page_size][r] bf16 and a
+    block table [B][max_pages] int32."""
+    pkp = _dev(k_pages, "k_pages", torch.bfloat16, 4)
+    pvp = _dev(v_pages, "v_pages", torch.bfloat16, 4)
+    pbt = _dev(block_table, "block_table", torch.int32, 2)
+    num_pages, Hkv, page_size, rK = k_pages.shape
+    rV = v_pages.shape[3]
+    if tuple(v_pages.shape) != (num_pages, Hkv, page_size, rV) or block_table.shape[0] != B:
+        raise ValueError("paged cache: inconsistent shapes")
+    return pkp, pvp, pbt, num_pages, Hkv, page_size, rK, rV, block_table.shape[1]
+
+
+def stief_compress_append_paged(k_new, v_new, P_K, P_V, k_pages, v_pages, block_table, seq_lens,
+                                dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """stief_compress_append into a paged cache (pools [num_pages][Hkv][page_size][r], block
+    table [B][max_pages])."""
+    pk = _dev(k_new, "k_new", torch.bfloat16, 4)
+    pv = _dev(v_new, "v_new", torch.bfloat16, 4)
+    ppk = _dev(P_K, "P_K", torch.bfloat16, 3)
+    ppv = _dev(P_V, "P_V", torch.bfloat16, 3)
+    psl = _dev(seq_lens, "seq_lens", torch.int32, 1)
+    B, Hkv, T, d = k_new.shape
+    pkp, pvp, pbt, num_pages, Hkv2, page_size, rK, rV, max_pages = _pages(k_pages, v_pages,
+                                                                          block_table, B)
+    if Hkv2 != Hkv or tuple(P_K.shape) != (Hkv, d, rK) or tuple(P_V.shape) != (Hkv, d, rV) \
+            or tuple(v_new.shape) != (B, Hkv, T, d) or seq_lens.shape[0] != B:
+        raise ValueError("stief_compress_append_paged: inconsistent shapes")
+    code = library().stief_compress_append_paged(pk, pv, ppk, ppv, pkp, pvp, pbt, psl, B, Hkv, T,
+                                                 d, rK, rV, num_pages, page_size, max_pages,
+                                                 _opt_status(dev_status), _stream_ptr(stream))
+    _check("stief_compress_append_paged", code)
+
+
+def stief_decode_attention_paged(q, P_K, P_V, k_pages, v_pages, block_table, seq_lens, out,
+                                 workspace, max_seq_len: int, num_splits: int = 0,
+                                 dev_status: Optional[torch.Tensor] = None, stream=None):
+    """stief_decode_attention over a paged cache."""
+    pq = _dev(q, "q", torch.bfloat16, 3)
+    ppk = _dev(P_K, "P_K", torch.bfloat16, 3)
+    ppv = _dev(P_V, "P_V", torch.bfloat16, 3)
+    psl = _dev(seq_lens, "seq_lens", torch.int32, 1)
+    po = _dev(out, "out", torch.bfloat16, 3)
+    B, Hq, d = q.shape
+    pkp, pvp, pbt, num_pages, Hkv, page_size, rK, rV, max_pages = _pages(k_pages, v_pages,
+                                                                         block_table, B)
+    if tuple(P_K.shape) != (Hkv, d, rK) or tuple(P_V.shape) != (Hkv, d, rV) \
+            or seq_lens.shape[0] != B or tuple(out.shape) != (B, Hq, d):
+        raise ValueError("stief_decode_attention_paged: inconsistent shapes")
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    code = library().stief_decode_attention_paged(pq, ppk, ppv, pkp, pvp, pbt, psl, po,
+                                                  workspace.data_ptr(), ws_bytes, B, Hq, Hkv, d,
+                                                  rK, rV, num_pages, page_size, max_pages,
+                                                  int(max_seq_len), int(num_splits),
+                                                  _opt_status(dev_status), _stream_ptr(stream))
+    _check("stief_decode_attention_paged", code)
+    return out
+
+
+def stief_append_decode_paged(q, k_new, v_new, P_K, P_V, k_pages, v_pages, block_table, seq_lens,
+                              out, workspace, max_seq_len: int, num_splits: int = 0,
+                              dev_status: Optional[torch.Tensor] = None, stream=None):
+    """stief_append_decode over a paged cache."""
+    pq = _dev(q, "q", torch.bfloat16, 3)
+    kn = k_new.reshape(k_new.shape[0], k_new.shape[1], -1) if k_new.dim() == 4 else k_new
+    vn = v_new.reshape(v_new.shape[0], v_new.shape[1], -1) if v_new.dim() == 4 else v_new
+    pkn = _dev(kn, "k_new", torch.bfloat16, 3)
+    pvn = _dev(vn, "v_new", torch.bfloat16, 3)
+    ppk = _dev(P_K, "P_K", torch.bfloat16, 3)
+    ppv = _dev(P_V, "P_V", torch.bfloat16, 3)
+    psl = _dev(seq_lens, "seq_lens", torch.int32, 1)
+    po = _dev(out, "out", torch.bfloat16, 3)
+    B, Hq, d = q.shape
+    pkp, pvp, pbt, num_pages, Hkv, page_size, rK, rV, max_pages = _pages(k_pages, v_pages,
+                                                                         block_table, B)
+    if tuple(kn.shape) != (B, Hkv, d) or tuple(vn.shape) != (B, Hkv, d) \
+            or tuple(P_K.shape) != (Hkv, d, rK) or tuple(P_V.shape) != (Hkv, d, rV) \
+            or seq_lens.shape[0] != B or tuple(out.shape) != (B, Hq, d):
+        raise ValueError("stief_append_decode_paged: inconsistent shapes")
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    code = library().stief_append_decode_paged(pq, pkn, pvn, ppk, ppv, pkp, pvp, pbt, psl, po,
+                                               workspace.data_ptr(), ws_bytes, B, Hq, Hkv, d, rK,
+                                               rV, num_pages, page_size, max_pages,
+                                               int(max_seq_len), int(num_splits),
+                                               _opt_status(dev_status), _stream_ptr(stream))
+    _check("stief_append_decode_paged", code)
     return out
 
 

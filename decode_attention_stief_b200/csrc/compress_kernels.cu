@@ -63,7 +63,9 @@ __global__ void __launch_bounds__(kSmallThreads) stief_compress_rows_kernel(cons
 
   const int Lb = a.seq_lens[b];
   const bool bad = Lb < 0 || Lb > a.L_max;
-  const bool full = !bad && (long long)Lb + T > a.L_max;
+  const CacheRows cr{a.block_table, a.max_pages, a.page_size, a.num_pages, a.Hkv, a.L_max};
+  // no room, or (paged) a page of the new rows is not mapped: the sequence is not appended to
+  const bool full = !bad && ((long long)Lb + T > a.L_max || !pages_mapped(cr, b, Lb, Lb + T));
   if (tid == 0 && blockIdx.x == 0 && blockIdx.y == 0) {
     if (bad) report(a.dev_status, STIEF_DEV_BAD_LENGTH);
     if (full) report(a.dev_status, STIEF_DEV_CAPACITY_OVERFLOW);
@@ -96,8 +98,7 @@ __global__ void __launch_bounds__(kSmallThreads) stief_compress_rows_kernel(cons
     for (int t = 0; t < TT; ++t) red[(sl * TT + t) * pairs + cp] = acc[t];
   }
   __syncthreads();
-  uint32_t* dst = reinterpret_cast<uint32_t*>((is_v ? a.v_lat : a.k_lat) +
-                                              (((size_t)b * a.Hkv + h) * a.L_max + Lb + r0) * r);
+  uint32_t* lat = reinterpret_cast<uint32_t*>(is_v ? a.v_lat : a.k_lat);
   for (int o = tid; o < nrows * pairs; o += kSmallThreads) {
     const int t = o / pairs, c2 = o - t * pairs;
     float2 sum = make_float2(0.f, 0.f);
@@ -106,16 +107,17 @@ __global__ void __launch_bounds__(kSmallThreads) stief_compress_rows_kernel(cons
       sum.x += v.x;
       sum.y += v.y;
     }
-    dst[(size_t)t * pairs + c2] = pack_bf16x2_rn(sum.x, sum.y);
+    lat[cache_row(cr, b, h, Lb + r0 + t) * pairs + c2] = pack_bf16x2_rn(sum.x, sum.y);
   }
 }
 
-__global__ void __launch_bounds__(256) stief_seq_lens_kernel(int32_t* seq_lens, int B, int T,
-                                                             int L_max) {
+__global__ void __launch_bounds__(256) stief_seq_lens_kernel(const CompressArgs a) {
   pdl_wait();  // every projection CTA has finished reading the old lengths
-  for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < B; b += gridDim.x * blockDim.x) {
-    const int L = seq_lens[b];
-    if (L >= 0 && (long long)L + T <= L_max) seq_lens[b] = L + T;
+  const CacheRows cr{a.block_table, a.max_pages, a.page_size, a.num_pages, a.Hkv, a.L_max};
+  for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < a.B; b += gridDim.x * blockDim.x) {
+    const int L = a.seq_lens[b];
+    if (L >= 0 && (long long)L + a.T <= a.L_max && pages_mapped(cr, b, L, L + a.T))
+      a.seq_lens[b] = L + a.T;
   }
 }
 
@@ -129,7 +131,7 @@ static cudaError_t launch_seq_lens(const CompressArgs& a, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, stief_seq_lens_kernel, a.seq_lens, a.B, a.T, a.L_max);
+  return cudaLaunchKernelEx(&cfg, stief_seq_lens_kernel, a);
 }
 
 template <int TT>

@@ -210,7 +210,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               tid);
   const int Lb = a.seq_lens[b];
   const bool bad = Lb < 0 || Lb > a.L_max;
-  const bool full = !bad && (long long)Lb + T > a.L_max;
+  const CacheRows cr{a.block_table, a.max_pages, a.page_size, a.num_pages, a.Hkv, a.L_max};
+  // no room, or (paged) a page of the new rows is not mapped: the sequence is not appended to
+  const bool full = !bad && ((long long)Lb + T > a.L_max || !pages_mapped(cr, b, Lb, Lb + T));
   if (tid == 0 && blockIdx.x == 0 && h == 0) {
     if (bad) report(a.dev_status, STIEF_DEV_BAD_LENGTH);
     if (full) report(a.dev_status, STIEF_DEV_CAPACITY_OVERFLOW);
@@ -257,11 +259,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int m0 = tile_m0(i);
     const int row = warp * 32 + lane;
     const bool live = m0 + row < T;
-    const size_t cache_row = ((size_t)b * a.Hkv + h) * a.L_max + Lb + m0 + row;
+    const long long crow = live ? cache_row(cr, b, h, Lb + m0 + row) : 0;  // mapped (checked)
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
     for (int which = 0; which < 2; ++which) {
       const int r = which ? rV : rK;
-      uint16_t* dst = (which ? a.v_lat : a.k_lat) + cache_row * r;
+      uint16_t* dst = (which ? a.v_lat : a.k_lat) + crow * r;
       for (int c0 = 0; c0 < r; c0 += 16) {
         uint32_t v[16];
         tmem_ld16(lane_base + (which ? 128u : 0u) + (uint32_t)c0, v);

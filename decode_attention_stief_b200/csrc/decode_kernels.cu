@@ -229,7 +229,7 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int NW, int ns, int rK,
 // NKS >= rK/16; NMV >= rV/16.
 constexpr int kMaxConsumerWarps = 8;
 
-template <int NB, int NKS, int NMV, int TT, bool LAT>
+template <int NB, int NKS, int NMV, int TT, bool LAT, bool PG>
 __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
     stief_decode_kernel(const __grid_constant__ DecodeArgs a) {
   constexpr int kTile = TT;
@@ -254,6 +254,9 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
   const int h0 = kvh * a.G + qs * G_T;          // first query head of this CTA
   const int gcount = min(G_T, a.G - qs * G_T);  // valid query heads here
   const size_t unit = ((size_t)b * a.Hkv + kvh) * a.qsub + qs;
+  // PG: paged caches (the contiguous instantiations carry no page lookups)
+  const CacheRows cr{PG ? a.block_table : nullptr, a.max_pages, a.page_size, a.num_pages, a.Hkv,
+                     a.L_max};
 
   const DecodeSmem L = decode_smem_layout(NW, ns, rK, rV, TT);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);  // [NW][ns]: tile landed
@@ -302,10 +305,13 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
       if (tid == 0 && s_idx == 0 && blockIdx.y == 0) report(a.dev_status, STIEF_DEV_CAPACITY_OVERFLOW);
     } else if (Lb + 1 > a.max_seq_len) {
       if (tid == 0 && s_idx == 0 && blockIdx.y == 0) report(a.dev_status, STIEF_DEV_BAD_LENGTH);
+    } else if (PG && cache_row(cr, b, kvh, Lb) < 0) {  // the new token's page is not mapped
+      if (tid == 0 && s_idx == 0 && blockIdx.y == 0) report(a.dev_status, STIEF_DEV_CAPACITY_OVERFLOW);
     } else {
       appended = true;
     }
   }
+  const long long new_row = appended ? cache_row(cr, b, kvh, Lb) : 0;  // the appended row
   const int L_att = Lb + (appended ? 1 : 0);  // tokens attended to
   const bool owns_new = appended && Lb >= t0 && Lb < t0 + a.chunk;  // the new token is in range
   const int t1 = min(t0 + a.chunk, L_att);
@@ -324,7 +330,15 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
   };
   const int n_tiles = t1 > t0 ? (t1 - t0 + kTile - 1) / kTile : 0;
   auto warp_tiles = [NW](int w, int tiles) { return w < tiles ? (tiles - w + NW - 1) / NW : 0; };
-  const size_t head_row0 = ((size_t)b * a.Hkv + kvh) * a.L_max;
+  // a tile's first row (tiles never straddle a page: page_size is a multiple of the tile);
+  // a tile of an unmapped page is requested past the end of the pool, which the copy fills
+  // with zeros (such tokens lie past the sequence and are masked)
+  const long long pool_rows = PG ? (long long)a.num_pages * a.Hkv * a.page_size
+                                 : (long long)a.B * a.Hkv * a.L_max;
+  auto tile_row = [&](int t) {
+    const long long r = cache_row(cr, b, kvh, t);
+    return (int)(r < 0 ? pool_rows : r);
+  };
   // TMA parameters of the cache pieces (at most three per matrix), kept in registers
   const void* kmap[3];
   const void* vmap[3];
@@ -346,7 +360,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
     uint64_t* bar = &full[w * ns + (k % ns)];
     // whole 32-row boxes land (rows past the sequence are masked on chip)
     mbar_arrive_expect_tx(bar, st_bytes);
-    const int y = (int)(head_row0 + t0 + (w + k * NW) * kTile);
+    const int y = tile_row(t0 + (w + k * NW) * kTile);
 #pragma unroll
     for (int p = 0; p < 3; ++p)
       if (p < npk) tma_load_2d(dst + ko[p], kmap[p], kx[p], y, bar, policy);
@@ -436,7 +450,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
         kl[j] = f32_to_bf16_rn(c[0]);
         kl[j + 8] = f32_to_bf16_rn(c[2]);
         if (qs == 0) {  // the cache row itself (every sub-group computes the same values)
-          uint16_t* dst = a.k_lat_w + (head_row0 + Lb) * rK;
+          uint16_t* dst = a.k_lat_w + new_row * rK;
           dst[j] = kl[j];
           dst[j + 8] = kl[j + 8];
         }
@@ -505,8 +519,8 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
             vl[j] = f32_to_bf16_rn(cv[0]);
             vl[j + 8] = f32_to_bf16_rn(cv[2]);
             if (qs == 0) {
-              a.v_lat_w[(head_row0 + Lb) * rV + j] = vl[j];
-              a.v_lat_w[(head_row0 + Lb) * rV + j + 8] = vl[j + 8];
+              a.v_lat_w[new_row * rV + j] = vl[j];
+              a.v_lat_w[new_row * rV + j + 8] = vl[j + 8];
             }
           }
         }
@@ -984,10 +998,10 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
 
 // ------------------------------------------------------------------------------ launch
 
-template <int NB, int NKS, int NMV, int TT, bool LAT>
+template <int NB, int NKS, int NMV, int TT, bool LAT, bool PG>
 static cudaError_t launch_k(const DecodeArgs& a, cudaStream_t stream) {
   const DecodeSmem L = decode_smem_layout(a.nwarps, a.nstage, a.rK, a.rV, TT);
-  auto kern = stief_decode_kernel<NB, NKS, NMV, TT, LAT>;
+  auto kern = stief_decode_kernel<NB, NKS, NMV, TT, LAT, PG>;
   static SmemLimit limit;
   cudaError_t e = limit.ensure(reinterpret_cast<const void*>(kern), a.device, (int)L.total);
   if (e != cudaSuccess) return e;
@@ -1006,11 +1020,16 @@ static cudaError_t launch_k(const DecodeArgs& a, cudaStream_t stream) {
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
-// the latent decode is its own instantiation, so its branches cost the other paths nothing
+// the latent decode and the paged caches are their own instantiations, so their branches
+// cost the contiguous path nothing (a runtime flag cost it 0.5-0.8 us per launch)
 template <int NB, int NKS, int NMV, int TT>
 static cudaError_t launch_t(const DecodeArgs& a, cudaStream_t stream) {
-  return a.latent ? launch_k<NB, NKS, NMV, TT, true>(a, stream)
-                  : launch_k<NB, NKS, NMV, TT, false>(a, stream);
+  if (a.latent) {
+    if (a.block_table) return cudaErrorInvalidValue;  // no paged latent decode
+    return launch_k<NB, NKS, NMV, TT, true, false>(a, stream);
+  }
+  return a.block_table ? launch_k<NB, NKS, NMV, TT, false, true>(a, stream)
+                       : launch_k<NB, NKS, NMV, TT, false, false>(a, stream);
 }
 
 uint32_t decode_smem_bytes(int nwarps, int nstage, int rK, int rV, int tile) {

@@ -152,7 +152,8 @@ stief_status plan_decode(DecodeArgs& a, const uint16_t* q, const uint16_t* P_K,
                          const uint16_t* P_V, const uint16_t* k_lat, const uint16_t* v_lat,
                          const int32_t* seq_lens, uint16_t* out, int B, int Hq, int Hkv, int d,
                          int rK, int rV, int L_max, int max_seq_len, int num_splits,
-                         uint32_t* dev_status, bool latent) {
+                         uint32_t* dev_status, bool latent, const int32_t* block_table,
+                         int max_pages, int page_size, int num_pages) {
   if (!q || !k_lat || !v_lat || !seq_lens || !out) return STIEF_ERR_INVALID_ARG;
   if (!latent && (!P_K || !P_V)) return STIEF_ERR_INVALID_ARG;
   if (B < 1 || B > 65535 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || Hq / Hkv > 64)
@@ -165,7 +166,8 @@ stief_status plan_decode(DecodeArgs& a, const uint16_t* q, const uint16_t* P_K,
   if (!aligned16(q) || !aligned16(k_lat) || !aligned16(v_lat) || !aligned16(out))
     return STIEF_ERR_ALIGNMENT;
   if (!latent && (!aligned16(P_K) || !aligned16(P_V))) return STIEF_ERR_ALIGNMENT;
-  const uint64_t rows = (uint64_t)B * Hkv * L_max;
+  // rows of the cache tensors: contiguous [B][Hkv][L_max], or pools [num_pages][Hkv][page_size]
+  const uint64_t rows = block_table ? (uint64_t)num_pages * Hkv * page_size : (uint64_t)B * Hkv * L_max;
   if (rows >= (1ull << 31)) return STIEF_ERR_INVALID_ARG;  // TMA row coordinates are int32
 
   int dev = 0, sms = 0;
@@ -174,6 +176,10 @@ stief_status plan_decode(DecodeArgs& a, const uint16_t* q, const uint16_t* P_K,
   if (!sm100) return STIEF_ERR_UNSUPPORTED_DEVICE;
   a.device = dev;
   a.latent = latent ? 1 : 0;
+  a.block_table = block_table;
+  a.max_pages = max_pages;
+  a.page_size = page_size;
+  a.num_pages = num_pages;
 
   a.q = q;
   a.seq_lens = seq_lens;

@@ -41,6 +41,29 @@ stief_status check_decode_shape(int B, int Hq, int Hkv, int d, int rK, int rV, i
   return STIEF_OK;
 }
 
+// A paged cache: pools [num_pages][Hkv][page_size][r] and a block table [B][max_pages]
+// (null for the contiguous layout).
+struct Paging {
+  const int32_t* block_table = nullptr;
+  int num_pages = 0, page_size = 0, max_pages = 0;
+};
+
+constexpr int kPageQuantum = 64;  // page sizes are multiples of the largest decode tile
+
+// Host checks of a paged cache; on success *capacity = max_pages * page_size tokens.
+stief_status check_paging(const Paging& pg, int Hkv, int* capacity) {
+  if (!pg.block_table) return STIEF_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(pg.block_table) & 3u) != 0) return STIEF_ERR_ALIGNMENT;
+  if (pg.page_size < kPageQuantum || pg.page_size % kPageQuantum != 0 || pg.num_pages < 1 ||
+      pg.max_pages < 1 || Hkv < 1)
+    return STIEF_ERR_INVALID_ARG;
+  const long long cap = (long long)pg.max_pages * pg.page_size;
+  const long long rows = (long long)pg.num_pages * Hkv * pg.page_size;
+  if (cap > 0x7fffffffLL || rows >= (1LL << 31)) return STIEF_ERR_INVALID_ARG;
+  *capacity = (int)cap;
+  return STIEF_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -89,12 +112,20 @@ size_t stief_decode_workspace_bytes(int B, int Hq, int Hkv, int rV, int max_seq_
   return stief::decode_ws_bytes(units, (size_t)B, G_T, stief_decode_max_splits(max_seq_len), kHeadDim);
 }
 
-stief_status stief_compress_append(const uint16_t* k_new, const uint16_t* v_new,
-                                   const uint16_t* P_K, const uint16_t* P_V, uint16_t* k_lat,
-                                   uint16_t* v_lat, int32_t* seq_lens, int B, int Hkv, int T,
-                                   int d, int rK, int rV, int L_max, uint32_t* dev_status,
-                                   stief_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+stief_status compress_common(const uint16_t* k_new, const uint16_t* v_new, const uint16_t* P_K,
+                             const uint16_t* P_V, uint16_t* k_lat, uint16_t* v_lat,
+                             int32_t* seq_lens, int B, int Hkv, int T, int d, int rK, int rV,
+                             int L_max, uint32_t* dev_status, stief_stream_t stream,
+                             const Paging& pg) {
   if (!k_new || !v_new || !P_K || !P_V || !k_lat || !v_lat || !seq_lens) return STIEF_ERR_INVALID_ARG;
+  if (pg.block_table) {
+    const stief_status st = check_paging(pg, Hkv, &L_max);
+    if (st != STIEF_OK) return st;
+  }
   if (B < 1 || Hkv < 1 || T < 0 || d != kHeadDim || !rank_ok(rK) || !rank_ok(rV) || L_max < 1)
     return STIEF_ERR_INVALID_ARG;
   if (T > L_max) return STIEF_ERR_CAPACITY;
@@ -122,9 +153,43 @@ stief_status stief_compress_append(const uint16_t* k_new, const uint16_t* v_new,
   a.rK = rK;
   a.rV = rV;
   a.L_max = L_max;
+  a.block_table = pg.block_table;
+  a.max_pages = pg.max_pages;
+  a.page_size = pg.page_size;
+  a.num_pages = pg.num_pages;
   if (stief::launch_compress(a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return STIEF_ERR_CUDA;
   return STIEF_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+stief_status stief_compress_append(const uint16_t* k_new, const uint16_t* v_new,
+                                   const uint16_t* P_K, const uint16_t* P_V, uint16_t* k_lat,
+                                   uint16_t* v_lat, int32_t* seq_lens, int B, int Hkv, int T,
+                                   int d, int rK, int rV, int L_max, uint32_t* dev_status,
+                                   stief_stream_t stream) {
+  return compress_common(k_new, v_new, P_K, P_V, k_lat, v_lat, seq_lens, B, Hkv, T, d, rK, rV,
+                         L_max, dev_status, stream, Paging{});
+}
+
+stief_status stief_compress_append_paged(const uint16_t* k_new, const uint16_t* v_new,
+                                         const uint16_t* P_K, const uint16_t* P_V,
+                                         uint16_t* k_pages, uint16_t* v_pages,
+                                         const int32_t* block_table, int32_t* seq_lens, int B,
+                                         int Hkv, int T, int d, int rK, int rV, int num_pages,
+                                         int page_size, int max_pages, uint32_t* dev_status,
+                                         stief_stream_t stream) {
+  Paging pg;
+  pg.block_table = block_table;
+  pg.num_pages = num_pages;
+  pg.page_size = page_size;
+  pg.max_pages = max_pages;
+  if (!block_table) return STIEF_ERR_INVALID_ARG;
+  return compress_common(k_new, v_new, P_K, P_V, k_pages, v_pages, seq_lens, B, Hkv, T, d, rK,
+                         rV, 0, dev_status, stream, pg);
 }
 
 namespace {
@@ -135,9 +200,14 @@ stief_status decode_common(const uint16_t* q, const uint16_t* k_new, const uint1
                            uint16_t* v_lat, int32_t* seq_lens, uint16_t* out, void* workspace,
                            size_t workspace_bytes, int B, int Hq, int Hkv, int d, int rK, int rV,
                            int L_max, int max_seq_len, int num_splits, uint32_t* dev_status,
-                           stief_stream_t stream, bool append, bool latent = false) {
+                           stief_stream_t stream, bool append, bool latent = false,
+                           const Paging& pg = Paging{}) {
   // cheap host checks first, so argument errors never touch CUDA
   if (!q || !k_lat || !v_lat || !seq_lens || !out) return STIEF_ERR_INVALID_ARG;
+  if (pg.block_table) {  // paged: the capacity is max_pages * page_size tokens
+    const stief_status sp = check_paging(pg, Hkv, &L_max);
+    if (sp != STIEF_OK) return sp;
+  }
   if (!latent && (!P_K || !P_V)) return STIEF_ERR_INVALID_ARG;
   if (append && (!k_new || !v_new)) return STIEF_ERR_INVALID_ARG;
   stief_status st = check_decode_shape(B, Hq, Hkv, d, rK, rV, L_max, max_seq_len);
@@ -154,7 +224,8 @@ stief_status decode_common(const uint16_t* q, const uint16_t* k_new, const uint1
 
   stief::DecodeArgs a{};
   st = stief::plan_decode(a, q, P_K, P_V, k_lat, v_lat, seq_lens, out, B, Hq, Hkv, d, rK, rV,
-                          L_max, max_seq_len, num_splits, dev_status, latent);
+                          L_max, max_seq_len, num_splits, dev_status, latent, pg.block_table,
+                          pg.max_pages, pg.page_size, pg.num_pages);
   if (st != STIEF_OK) return st;
   a.append = append ? 1 : 0;
   a.k_new = k_new;
@@ -209,6 +280,46 @@ stief_status stief_decode_latent(const uint16_t* q_lat, const uint16_t* k_lat,
                        const_cast<uint16_t*>(v_lat), const_cast<int32_t*>(seq_lens), out_lat,
                        workspace, workspace_bytes, B, Hq, Hkv, d, rK, rV, L_max, max_seq_len,
                        num_splits, dev_status, stream, false, true);
+}
+
+stief_status stief_decode_attention_paged(const uint16_t* q, const uint16_t* P_K,
+                                          const uint16_t* P_V, const uint16_t* k_pages,
+                                          const uint16_t* v_pages, const int32_t* block_table,
+                                          const int32_t* seq_lens, uint16_t* out, void* workspace,
+                                          size_t workspace_bytes, int B, int Hq, int Hkv, int d,
+                                          int rK, int rV, int num_pages, int page_size,
+                                          int max_pages, int max_seq_len, int num_splits,
+                                          uint32_t* dev_status, stief_stream_t stream) {
+  Paging pg;
+  pg.block_table = block_table;
+  pg.num_pages = num_pages;
+  pg.page_size = page_size;
+  pg.max_pages = max_pages;
+  if (!block_table) return STIEF_ERR_INVALID_ARG;
+  return decode_common(q, nullptr, nullptr, P_K, P_V, const_cast<uint16_t*>(k_pages),
+                       const_cast<uint16_t*>(v_pages), const_cast<int32_t*>(seq_lens), out,
+                       workspace, workspace_bytes, B, Hq, Hkv, d, rK, rV, 0, max_seq_len,
+                       num_splits, dev_status, stream, false, false, pg);
+}
+
+stief_status stief_append_decode_paged(const uint16_t* q, const uint16_t* k_new,
+                                       const uint16_t* v_new, const uint16_t* P_K,
+                                       const uint16_t* P_V, uint16_t* k_pages, uint16_t* v_pages,
+                                       const int32_t* block_table, int32_t* seq_lens,
+                                       uint16_t* out, void* workspace, size_t workspace_bytes,
+                                       int B, int Hq, int Hkv, int d, int rK, int rV,
+                                       int num_pages, int page_size, int max_pages,
+                                       int max_seq_len, int num_splits, uint32_t* dev_status,
+                                       stief_stream_t stream) {
+  Paging pg;
+  pg.block_table = block_table;
+  pg.num_pages = num_pages;
+  pg.page_size = page_size;
+  pg.max_pages = max_pages;
+  if (!block_table) return STIEF_ERR_INVALID_ARG;
+  return decode_common(q, k_new, v_new, P_K, P_V, k_pages, v_pages, seq_lens, out, workspace,
+                       workspace_bytes, B, Hq, Hkv, d, rK, rV, 0, max_seq_len, num_splits,
+                       dev_status, stream, true, false, pg);
 }
 
 stief_status stief_read_device_status(const uint32_t* dev_status, uint32_t* value,

@@ -176,6 +176,33 @@ __device__ __forceinline__ void prefetch_tensormap(const void* map) {
 
 // Block until the preceding grid in the stream has completed and its memory is
 // visible (no-op when the kernel was not launched as a programmatic dependent).
+// Row of token t of (sequence b, KV head h) in a latent cache.  Contiguous caches hold
+// [B][Hkv][L_max] rows; paged caches hold [num_pages][Hkv][page_size] rows and map token t
+// through the sequence's block table (page block_table[b][t / page_size]).  Returns -1 for a
+// token whose page is not mapped (past max_pages, or an id outside [0, num_pages)).
+struct CacheRows {
+  const int32_t* block_table;  // [B][max_pages], or null for a contiguous cache
+  int max_pages, page_size, num_pages, Hkv, L_max;
+};
+__device__ __forceinline__ long long cache_row(const CacheRows& c, int b, int h, int t) {
+  if (c.block_table == nullptr) return ((long long)b * c.Hkv + h) * c.L_max + t;
+  const int pi = t / c.page_size;
+  if (pi >= c.max_pages) return -1;
+  const int pg = __ldg(c.block_table + (size_t)b * c.max_pages + pi);
+  if (pg < 0 || pg >= c.num_pages) return -1;
+  return ((long long)pg * c.Hkv + h) * c.page_size + (t - pi * c.page_size);
+}
+// Whether every page holding tokens [t0, t1) of sequence b is mapped (always, contiguous).
+__device__ __forceinline__ bool pages_mapped(const CacheRows& c, int b, int t0, int t1) {
+  if (c.block_table == nullptr || t1 <= t0) return true;
+  for (int pi = t0 / c.page_size; pi <= (t1 - 1) / c.page_size; ++pi) {
+    if (pi >= c.max_pages) return false;
+    const int pg = __ldg(c.block_table + (size_t)b * c.max_pages + pi);
+    if (pg < 0 || pg >= c.num_pages) return false;
+  }
+  return true;
+}
+
 __device__ __forceinline__ void pdl_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }

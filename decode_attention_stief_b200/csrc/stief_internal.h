@@ -57,6 +57,10 @@ struct DecodeArgs {
   float qscale;     // log2(e) / sqrt(d), applied to q . P_K
   int device;       // current device at planning time (host bookkeeping only)
   int latent;       // latent decode: q holds q~ [B][Hq][rK], out is o~ [B][Hq][rV], no bases
+  // paged caches: [num_pages][Hkv][page_size][r] pools addressed through block_table
+  // [B][max_pages] (null for a contiguous cache; L_max is then max_pages * page_size)
+  const int32_t* block_table;
+  int max_pages, page_size, num_pages;
 };
 
 struct CompressArgs {
@@ -70,6 +74,9 @@ struct CompressArgs {
   uint32_t* dev_status;
   int B, Hkv, T, d, rK, rV, L_max;
   int device;  // current device (host bookkeeping only)
+  // paged caches, as in DecodeArgs (block_table null: contiguous [B][Hkv][L_max] rows)
+  const int32_t* block_table;
+  int max_pages, page_size, num_pages;
 };
 
 constexpr int kMaxSmemPerBlock = 232448;  // 227 KB opt-in dynamic shared memory (sm_100)
@@ -109,12 +116,15 @@ uint32_t compress_tc_smem_bytes(int rK, int rV);
 // Validates a decode call and fills everything in `a` except the workspace pointers
 // (split count, group tiling, CTA configuration, key tensor maps).  Host only.
 // With `latent`, q is q~ [B][Hq][rK], out is o~ [B][Hq][rV] and P_K, P_V are unused (may be
-// NULL): no base tensor maps are planned.
+// NULL): no base tensor maps are planned.  With a block table, k_lat / v_lat are page pools
+// [num_pages][Hkv][page_size][r] and L_max is the capacity max_pages * page_size.
 stief_status plan_decode(DecodeArgs& a, const uint16_t* q, const uint16_t* P_K,
                          const uint16_t* P_V, const uint16_t* k_lat, const uint16_t* v_lat,
                          const int32_t* seq_lens, uint16_t* out, int B, int Hq, int Hkv, int d,
                          int rK, int rV, int L_max, int max_seq_len, int num_splits,
-                         uint32_t* dev_status, bool latent = false);
+                         uint32_t* dev_status, bool latent = false,
+                         const int32_t* block_table = nullptr, int max_pages = 0,
+                         int page_size = 0, int num_pages = 0);
 
 // Decode workspace layout: `units` = B * Hkv * qsub split-ticket counters, then B sequence
 // tickets (uint32, padded together to 256 bytes), then units * G_T * splits partial states

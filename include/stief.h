@@ -260,6 +260,54 @@ STIEF_API stief_status stief_decode_latent(const uint16_t* q_lat, const uint16_t
                                  stief_stream_t stream);
 
 /*
+ * Paged latent caches (serving-style block tables).  The pages give no memory layout;
+ * this library's paged form keeps each cache as a pool of pages,
+ *     k_pages : bf16 [num_pages][Hkv][page_size][rK]
+ *     v_pages : bf16 [num_pages][Hkv][page_size][rV]
+ * and gives every sequence b a row of the block table,
+ *     block_table : int32 [B][max_pages] (device), page ids in [0, num_pages),
+ * so that token t of (b, KV head h) is row t % page_size of page block_table[b][t /
+ * page_size], head h.  A sequence's capacity is max_pages * page_size tokens (the
+ * contiguous calls' L_max).  page_size is a multiple of 64 (>= 64); num_pages *
+ * Hkv * page_size < 2^31.  Entries for pages the sequence does not reach are never
+ * read for its tokens.  An append whose new rows need a page with an id outside
+ * [0, num_pages) (or past max_pages) is refused for that sequence as a full cache is:
+ * STIEF_DEV_CAPACITY_OVERFLOW, nothing written, the length unchanged.  A decode never
+ * checks the pages below the length (they read as zeros if unmapped, which masks
+ * nothing): the caller maps every page below the length.  block_table must be 4-byte
+ * aligned; the pools 16-byte.
+ * The calls below are their contiguous counterparts with k_lat / v_lat replaced by
+ * the pools and L_max by (num_pages, page_size, max_pages); everything else --
+ * results, workspace, status words, launch behaviour -- is the same.
+ */
+STIEF_API stief_status stief_compress_append_paged(const uint16_t* k_new, const uint16_t* v_new,
+                                         const uint16_t* P_K, const uint16_t* P_V,
+                                         uint16_t* k_pages, uint16_t* v_pages,
+                                         const int32_t* block_table, int32_t* seq_lens, int B,
+                                         int Hkv, int T, int d, int rK, int rV, int num_pages,
+                                         int page_size, int max_pages, uint32_t* dev_status,
+                                         stief_stream_t stream);
+
+STIEF_API stief_status stief_decode_attention_paged(const uint16_t* q, const uint16_t* P_K,
+                                          const uint16_t* P_V, const uint16_t* k_pages,
+                                          const uint16_t* v_pages, const int32_t* block_table,
+                                          const int32_t* seq_lens, uint16_t* out, void* workspace,
+                                          size_t workspace_bytes, int B, int Hq, int Hkv, int d,
+                                          int rK, int rV, int num_pages, int page_size,
+                                          int max_pages, int max_seq_len, int num_splits,
+                                          uint32_t* dev_status, stief_stream_t stream);
+
+STIEF_API stief_status stief_append_decode_paged(const uint16_t* q, const uint16_t* k_new,
+                                       const uint16_t* v_new, const uint16_t* P_K,
+                                       const uint16_t* P_V, uint16_t* k_pages, uint16_t* v_pages,
+                                       const int32_t* block_table, int32_t* seq_lens,
+                                       uint16_t* out, void* workspace, size_t workspace_bytes,
+                                       int B, int Hq, int Hkv, int d, int rK, int rV,
+                                       int num_pages, int page_size, int max_pages,
+                                       int max_seq_len, int num_splits, uint32_t* dev_status,
+                                       stief_stream_t stream);
+
+/*
  * stief_decode_attention_noalloc -- stief_decode_attention without a workspace
  * argument and without any device allocation.  The paper has no counterpart: this
  * is a deployment variant for callers that cannot obtain device memory when they

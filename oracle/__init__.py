@@ -210,3 +210,25 @@ def decode(q, P_K, P_V, k_lat, v_lat, seq_lens, num_threads: int = 0) -> np.ndar
 
 def decode_latent(q_lat, k_lat, v_lat, seq_lens, d: int = 128, num_threads: int = 0) -> np.ndarray:
     return default().decode_latent(q_lat, k_lat, v_lat, seq_lens, d, num_threads)
+
+
+def gather_pages(pages, block_table, seq_lens, L_max: int) -> np.ndarray:
+    """The contiguous cache [B][Hkv][L_max][r] (fp64) that a paged cache stands for.
+
+    The library's paged layout: a pool ``pages`` [num_pages][Hkv][page_size][r] and a block
+    table [B][max_pages]; token t of (sequence b, KV head h) is row t % page_size of page
+    block_table[b][t // page_size], head h.  Rows at and past seq_lens[b] are left zero.
+    Plain indexing, no arithmetic: the paged calls are defined as the contiguous ones on the
+    cache this returns.
+    """
+    pages = _f64(pages)
+    bt = np.asarray(block_table)
+    lens = np.asarray(seq_lens)
+    num_pages, Hkv, ps, r = pages.shape
+    B = bt.shape[0]
+    out = np.zeros((B, Hkv, L_max, r), dtype=np.float64)
+    for b in range(B):
+        for t in range(int(lens[b])):
+            out[b, :, t] = pages[int(bt[b, t // ps]), :, t % ps]
+    return out
+

@@ -280,6 +280,30 @@ def check_latent_edges(o, r: int = 32) -> None:
     assert np.array_equal(got[1], np.repeat(v[1, 0, :1], 3, axis=0))
 
 
+# ----------------------------------------------------------------------------- paged layout
+
+def check_paged_layout(o) -> None:
+    """gather_pages inverts a scatter of a known contiguous cache into shuffled pages, and
+    token t of sequence b comes from page block_table[b][t // page_size], row t % page_size."""
+    rng = np.random.default_rng(20)
+    B, Hkv, ps, r, max_pages = 3, 2, 64, 16, 4
+    lens = np.array([256, 70, 0], np.int32)
+    cont = rng.standard_normal((B, Hkv, max_pages * ps, r))
+    perm = rng.permutation(B * max_pages)
+    bt = perm.reshape(B, max_pages).astype(np.int32)
+    pages = np.zeros((B * max_pages, Hkv, ps, r))
+    for b in range(B):
+        for j in range(max_pages):
+            pages[bt[b, j]] = cont[b, :, j * ps:(j + 1) * ps]
+    import oracle  # gather_pages is plain indexing in the Python module (no C part)
+    got = oracle.gather_pages(pages, bt, lens, max_pages * ps)
+    for b in range(B):
+        assert np.array_equal(got[b, :, :lens[b]], cont[b, :, :lens[b]])
+        assert np.all(got[b, :, lens[b]:] == 0)
+    # one hand-picked token: sequence 1, token 69 -> page bt[1][1], row 5
+    assert np.array_equal(got[1, :, 69], pages[bt[1, 1], :, 5])
+
+
 # ----------------------------------------------------------------------------- compression
 
 def check_compress_identity_basis(o, r: int = 48, d: int = 128) -> None:
@@ -353,6 +377,7 @@ ALL_ORACLE_CHECKS = {
                                                                          tol=1e-10),
     "latent_folding_identity": check_latent_folding_identity,
     "latent_edges": check_latent_edges,
+    "paged_layout": check_paged_layout,
     "compress_identity_basis": check_compress_identity_basis,
     "compress_matches_exact_product": check_compress_matches_exact_product,
     "compress_append_bookkeeping": check_compress_append_bookkeeping,

@@ -111,6 +111,30 @@ def test_latent_decode_argument_errors(lib, kw, code):
     assert _latent(lib, **kw) == code
 
 
+def _paged(lib, **kw):
+    a = dict(q=FAKE, P_K=FAKE, P_V=FAKE, kp=FAKE, vp=FAKE, bt=FAKE, sl=FAKE, out=FAKE, ws=FAKE,
+             ws_bytes=1 << 40, B=2, Hq=32, Hkv=8, d=128, rK=64, rV=64, num_pages=64,
+             page_size=128, max_pages=16, max_seq_len=2048, num_splits=0)
+    a.update(kw)
+    return lib.stief_decode_attention_paged(a["q"], a["P_K"], a["P_V"], a["kp"], a["vp"], a["bt"],
+                                            a["sl"], a["out"], a["ws"], a["ws_bytes"], a["B"],
+                                            a["Hq"], a["Hkv"], a["d"], a["rK"], a["rV"],
+                                            a["num_pages"], a["page_size"], a["max_pages"],
+                                            a["max_seq_len"], a["num_splits"], None, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(bt=None), INVALID), (dict(page_size=96), INVALID), (dict(page_size=32), INVALID),
+    (dict(num_pages=0), INVALID), (dict(max_pages=0), INVALID),
+    (dict(max_seq_len=16 * 128 + 1), CAPACITY),  # beyond max_pages * page_size
+    (dict(num_pages=1 << 20, page_size=1 << 12), INVALID),  # pool rows >= 2^31
+    (dict(bt=FAKE + 2), ALIGN), (dict(kp=FAKE + 8), ALIGN), (dict(ws=None), WORKSPACE),
+])
+def test_paged_decode_argument_errors(lib, kw, code):
+    """The paged decode checks the pool geometry and the block table before any CUDA call."""
+    assert _paged(lib, **kw) == code
+
+
 @pytest.mark.parametrize("kw,code", [
     (dict(k=None), INVALID), (dict(sl=None), INVALID), (dict(d=96), INVALID),
     (dict(rK=24), INVALID), (dict(T=-1), INVALID), (dict(B=0), INVALID),
