@@ -232,3 +232,28 @@ def gather_pages(pages, block_table, seq_lens, L_max: int) -> np.ndarray:
             out[b, :, t] = pages[int(bt[b, t // ps]), :, t % ps]
     return out
 
+
+def quantize_rows(x):
+    """Per-row symmetric int8 quantisation of latent rows (the low-bit cache form).
+
+    The pages report the compressed cache to be robust to 4- and 8-bit quantisation but fix no
+    scheme; this library's reading: one fp32 scale per stored row (per token, KV head),
+        scale = fp32(max_c |x_c| / 127),  code_c = RNE(fp32(x_c / scale)) in [-127, 127],
+    with a zero row stored as scale 0 and codes 0.  x are the bf16 latent values (exact in
+    fp32).  The two divisions and the rounding to an integer are taken in IEEE fp32, the
+    kernel's precision, so the integer codes are decided identically on both sides.
+    Returns (codes int8 [..., r], scales float32 [...]).
+    """
+    x32 = np.asarray(x, dtype=np.float32)
+    amax = np.max(np.abs(x32), axis=-1)
+    scale = (amax / np.float32(127.0)).astype(np.float32)
+    safe = np.where(scale > 0, scale, np.float32(1.0)).astype(np.float32)
+    q = np.rint((x32 / safe[..., None]).astype(np.float32))
+    q = np.where(scale[..., None] > 0, q, 0.0)
+    return np.clip(q, -127, 127).astype(np.int8), scale
+
+
+def dequantize_rows(codes, scales) -> np.ndarray:
+    """code * scale per element, exact in fp64."""
+    return np.asarray(codes, np.float64) * np.asarray(scales, np.float64)[..., None]
+

@@ -304,6 +304,33 @@ def check_paged_layout(o) -> None:
     assert np.array_equal(got[1, :, 69], pages[bt[1, 1], :, 5])
 
 
+# ----------------------------------------------------------------------------- int8 rows
+
+def check_quantize_rows(o) -> None:
+    """Closed forms of the per-row int8 form: the largest magnitude maps to +-127 exactly;
+    a zero row is scale 0 and codes 0; codes are odd-symmetric; halfway cases round to even;
+    every element is within half a step (plus the fp32 division's rounding) of its code."""
+    import oracle
+    rng = np.random.default_rng(21)
+    x = oracle.round_bf16(rng.standard_normal((64, 48)) * rng.uniform(0.01, 10, (64, 1)))
+    q, s = oracle.quantize_rows(x)
+    assert q.dtype == np.int8 and s.dtype == np.float32
+    amax_idx = np.argmax(np.abs(x), axis=1)
+    assert np.all(np.abs(q[np.arange(64), amax_idx]) == 127)
+    assert np.all(np.sign(q[np.arange(64), amax_idx]) == np.sign(x[np.arange(64), amax_idx]))
+    err = np.abs(x - oracle.dequantize_rows(q, s))
+    assert np.all(err <= 0.5 * s[:, None] * (1 + 2.0 ** -22) + np.abs(x) * 2.0 ** -23)
+    qn, sn = oracle.quantize_rows(-x)
+    assert np.array_equal(qn, -q) and np.array_equal(sn, s)
+    z, zs = oracle.quantize_rows(np.zeros((2, 16)))
+    assert np.all(z == 0) and np.all(zs == 0)
+    # row max 127 gives scale exactly 1: x = k + 0.5 rounds to the even neighbour
+    row = np.array([[127.0, 2.5, 3.5, -2.5, -0.5, 0.5, 1.5, 126.5]])
+    qr, sr = oracle.quantize_rows(row)
+    assert sr[0] == 1.0
+    assert qr[0].tolist() == [127, 2, 4, -2, 0, 0, 2, 126]
+
+
 # ----------------------------------------------------------------------------- compression
 
 def check_compress_identity_basis(o, r: int = 48, d: int = 128) -> None:
@@ -378,6 +405,7 @@ ALL_ORACLE_CHECKS = {
     "latent_folding_identity": check_latent_folding_identity,
     "latent_edges": check_latent_edges,
     "paged_layout": check_paged_layout,
+    "quantize_rows": check_quantize_rows,
     "compress_identity_basis": check_compress_identity_basis,
     "compress_matches_exact_product": check_compress_matches_exact_product,
     "compress_append_bookkeeping": check_compress_append_bookkeeping,
