@@ -16,8 +16,10 @@ from ._binding import (  # noqa: F401
     stief_append_decode,
     stief_append_decode_paged,
     stief_compress_append,
+    stief_compress_append_q8,
     stief_compress_append_paged,
     stief_decode_attention,
+    stief_decode_attention_q8,
     stief_decode_attention_paged,
     stief_decode_attention_noalloc,
     stief_decode_auto_splits,

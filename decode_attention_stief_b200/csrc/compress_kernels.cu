@@ -99,6 +99,7 @@ __global__ void __launch_bounds__(kSmallThreads) stief_compress_rows_kernel(cons
   }
   __syncthreads();
   uint32_t* lat = reinterpret_cast<uint32_t*>(is_v ? a.v_lat : a.k_lat);
+  const bool q8 = a.k_scale != nullptr;
   for (int o = tid; o < nrows * pairs; o += kSmallThreads) {
     const int t = o / pairs, c2 = o - t * pairs;
     float2 sum = make_float2(0.f, 0.f);
@@ -107,7 +108,24 @@ __global__ void __launch_bounds__(kSmallThreads) stief_compress_rows_kernel(cons
       sum.x += v.x;
       sum.y += v.y;
     }
-    lat[cache_row(cr, b, h, Lb + r0 + t) * pairs + c2] = pack_bf16x2_rn(sum.x, sum.y);
+    if (q8)  // keep the bf16-rounded row for the quantisation below (slice 0's own slot)
+      red[t * pairs + c2] = make_float2(bf16_round(sum.x), bf16_round(sum.y));
+    else
+      lat[cache_row(cr, b, h, Lb + r0 + t) * pairs + c2] = pack_bf16x2_rn(sum.x, sum.y);
+  }
+  if (q8) {
+    // int8 cache: a thread per row: one fp32 scale (max / 127) and RNE codes
+    __syncthreads();
+    if (tid < nrows) {
+      const float* row = reinterpret_cast<const float*>(red + tid * pairs);
+      float amax = 0.f;
+      for (int c = 0; c < r; ++c) amax = fmaxf(amax, fabsf(row[c]));
+      const float scale = __fdiv_rn(amax, 127.f);
+      const long long crow = cache_row(cr, b, h, Lb + r0 + tid);
+      int8_t* dst = reinterpret_cast<int8_t*>(is_v ? a.v_lat : a.k_lat) + crow * r;
+      for (int c = 0; c < r; ++c) dst[c] = (int8_t)quantize_code(row[c], scale);
+      (is_v ? a.v_scale : a.k_scale)[crow] = scale;
+    }
   }
 }
 

@@ -261,7 +261,40 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const bool live = m0 + row < T;
     const long long crow = live ? cache_row(cr, b, h, Lb + m0 + row) : 0;  // mapped (checked)
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-    for (int which = 0; which < 2; ++which) {
+    for (int which = 0; which < 2 && a.k_scale != nullptr; ++which) {
+      // int8 cache: the row rounded to bf16, then one fp32 scale (max / 127) and RNE codes,
+      // divisions in IEEE fp32; the accumulators are read twice (maximum, then codes)
+      const int r = which ? rV : rK;
+      const uint32_t col0 = which ? 128u : 0u;
+      float amax = 0.f;
+      for (int c0 = 0; c0 < r; c0 += 16) {
+        uint32_t v[16];
+        tmem_ld16(lane_base + col0 + (uint32_t)c0, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(bf16_round(__uint_as_float(v[e]))));
+      }
+      const float scale = __fdiv_rn(amax, 127.f);
+      int8_t* dst = reinterpret_cast<int8_t*>(which ? a.v_lat : a.k_lat) + crow * r;
+      for (int c0 = 0; c0 < r; c0 += 16) {
+        uint32_t v[16];
+        tmem_ld16(lane_base + col0 + (uint32_t)c0, v);
+        tmem_wait_ld();
+        uint32_t packed[4];
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          uint32_t word = 0u;
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            word |= (uint32_t)(uint8_t)quantize_code(bf16_round(__uint_as_float(v[4 * g + e])), scale)
+                    << (8 * e);
+          packed[g] = word;
+        }
+        if (live) *reinterpret_cast<uint4*>(dst + c0) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+      }
+      if (live) (which ? a.v_scale : a.k_scale)[crow] = scale;
+    }
+    for (int which = 0; which < 2 && a.k_scale == nullptr; ++which) {
       const int r = which ? rV : rK;
       uint16_t* dst = (which ? a.v_lat : a.k_lat) + crow * r;
       for (int c0 = 0; c0 < r; c0 += 16) {

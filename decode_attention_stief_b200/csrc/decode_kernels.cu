@@ -135,6 +135,15 @@ __device__ __forceinline__ PieceLoc locate(int r, int rows, int chunk) {
   }
   return pl;
 }
+// Two int8 codes (bytes j and j + 1 of w) times a scale, rounded to bf16 and packed.  A
+// code c becomes exact fp32 through the bit pattern of 2^23 + (c + 128) less 2^23 + 128.
+__device__ __forceinline__ uint32_t deq_pair(uint32_t u, int j, float2 sc2) {
+  // u: the codes + 128 as unsigned bytes (w ^ 0x80808080)
+  float2 c = make_float2(__uint_as_float(__byte_perm(u, 0x4B000000u, 0x7540u | (uint32_t)j)),
+                         __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7540u | (uint32_t)(j + 1))));
+  c = __fmul2_rn(__fadd2_rn(c, make_float2(-8388736.f, -8388736.f)), sc2);
+  return pack_bf16x2_rn(c.x, c.y);
+}
 // Byte offset of (row, chunk) under the piece's TMA swizzle: 128-byte rows XOR the chunk
 // with row & 7, 64-byte rows with (row >> 1) & 3, 32-byte rows with (row >> 2) & 1.
 __device__ __forceinline__ uint32_t swz(const PieceLoc& pl, int row) {
@@ -193,11 +202,18 @@ struct DecodeSmem {
   uint32_t region;  // per warp a ring of stages (keys then values of a tile); later the
                     // cross-warp reduction and the split-merge staging
   uint32_t region_bytes;
+  // int8 caches: the region holds one bf16 tile per warp (the dequantised stage, laid out
+  // as a bf16 ring stage), then the rings of raw stages: codes K [tile][rK], codes V
+  // [tile][rV], scales K [tile], scales V [tile]
+  uint32_t ring;      // offset of the rings inside the region
+  uint32_t stage;     // bytes of one ring stage
+  uint32_t q8_v, q8_ks, q8_vs;  // offsets inside a raw int8 stage
   uint32_t total;
   int xs;  // row stride of qt in floats
 };
 
-__host__ __device__ inline DecodeSmem decode_smem_layout(int NW, int ns, int rK, int rV, int tile) {
+__host__ __device__ inline DecodeSmem decode_smem_layout(int NW, int ns, int rK, int rV, int tile,
+                                                          bool q8 = false) {
   DecodeSmem s;
   const int rmax = rK > rV ? rK : rV;
   uint32_t off = 0;
@@ -217,7 +233,19 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int NW, int ns, int rK,
   s.pmat = off;
   off += 256u * rmax;  // d = 128 rows x r bf16
   s.region = off;
-  s.region_bytes = (uint32_t)NW * ns * tile * (rK + rV) * 2u;
+  const uint32_t bf16_stage = (uint32_t)tile * (rK + rV) * 2u;  // a multiple of 1 KiB
+  if (q8) {
+    s.q8_v = align_up((uint32_t)tile * rK, 128);
+    s.q8_ks = s.q8_v + align_up((uint32_t)tile * rV, 128);
+    s.q8_vs = s.q8_ks + (uint32_t)tile * 4u;
+    s.stage = align_up(s.q8_vs + (uint32_t)tile * 4u, 128);
+    s.ring = (uint32_t)NW * bf16_stage;
+  } else {
+    s.q8_v = s.q8_ks = s.q8_vs = 0;
+    s.stage = bf16_stage;
+    s.ring = 0;
+  }
+  s.region_bytes = s.ring + (uint32_t)NW * ns * s.stage;
   off += s.region_bytes;
   s.total = off;
   return s;
@@ -229,9 +257,14 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int NW, int ns, int rK,
 // NKS >= rK/16; NMV >= rV/16.
 constexpr int kMaxConsumerWarps = 8;
 
-template <int NB, int NKS, int NMV, int TT, bool LAT, bool PG>
+// Kernel modes: the contiguous bf16 cache, the latent decode, paged caches, int8 caches.
+// Each is its own instantiation, so a mode's branches cost the others nothing.
+constexpr int kModePlain = 0, kModeLatent = 1, kModePaged = 2, kModeQ8 = 3;
+
+template <int NB, int NKS, int NMV, int TT, int MODE>
 __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
     stief_decode_kernel(const __grid_constant__ DecodeArgs a) {
+  constexpr bool LAT = MODE == kModeLatent, PG = MODE == kModePaged, Q8 = MODE == kModeQ8;
   constexpr int kTile = TT;
   constexpr int MT = TT / 16;              // 16-token m-tiles (scores) / k-steps (mix) per tile
   // score k-steps / value m-tiles whose fragments are loaded together (fewer where the
@@ -258,7 +291,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
   const CacheRows cr{PG ? a.block_table : nullptr, a.max_pages, a.page_size, a.num_pages, a.Hkv,
                      a.L_max};
 
-  const DecodeSmem L = decode_smem_layout(NW, ns, rK, rV, TT);
+  const DecodeSmem L = decode_smem_layout(NW, ns, rK, rV, TT, Q8);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);  // [NW][ns]: tile landed
   uint64_t* empty = full + NW * ns;                             // [NW][ns]: tile consumed
   uint64_t* setup_bar = empty + NW * ns;  // phase 0: q and P_K, phase 1: P_V
@@ -356,8 +389,18 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
   }
   const int npk = a.pk.n, npv = a.pv.n;
   auto issue = [&](int w, int k, uint64_t policy) {  // producer: tile k of consumer warp w
-    uint8_t* dst = smem + L.region + ((size_t)w * ns + (k % ns)) * st_bytes;
+    uint8_t* dst = smem + L.region + L.ring + ((size_t)w * ns + (k % ns)) * L.stage;
     uint64_t* bar = &full[w * ns + (k % ns)];
+    if (Q8) {  // int8 codes of K and V (one box each) and the tile's two rows of scales
+      const uint32_t tb = (uint32_t)kTile * (rK + rV) + 8u * kTile;
+      mbar_arrive_expect_tx(bar, tb);
+      const int y = tile_row(t0 + (w + k * NW) * kTile);
+      tma_load_2d(dst, kmap[0], 0, y, bar, policy);
+      tma_load_2d(dst + L.q8_v, vmap[0], 0, y, bar, policy);
+      bulk_g2s(dst + L.q8_ks, a.k_scale + y, 4u * kTile, bar);
+      bulk_g2s(dst + L.q8_vs, a.v_scale + y, 4u * kTile, bar);
+      return;
+    }
     // whole 32-row boxes land (rows past the sequence are masked on chip)
     mbar_arrive_expect_tx(bar, st_bytes);
     const int y = tile_row(t0 + (w + k * NW) * kTile);
@@ -560,7 +603,17 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
   } else {
     // ---- consumers: stream the warp's tiles ------------------------------------------------
     const int my_tiles = warp_tiles(warp, n_tiles);
-    uint8_t* ring = smem + L.region + (size_t)warp * ns * st_bytes;
+    uint8_t* ring = smem + L.region + L.ring + (size_t)warp * ns * L.stage;
+    uint8_t* staging = smem + L.region + (size_t)warp * st_bytes;  // int8 caches only
+    // int8 caches: in the dequantise pass a lane takes one 8-column chunk of each matrix and
+    // every (32 / chunks per row)-th row of it (no division per item); its chunk's place in
+    // the swizzled bf16 tile is fixed
+    const int kcpr = rK >> 3, vcpr = rV >> 3;  // 8-column chunks per row
+    const int krpp = 32 / kcpr, vrpp = 32 / vcpr;  // rows per pass
+    const bool klive = lane < krpp * kcpr, vlive = lane < vrpp * vcpr;
+    const int kc0 = lane % kcpr, vc0 = lane % vcpr;
+    const int kt0 = lane / kcpr, vt0 = lane / vcpr;
+    const PieceLoc kpl = locate(rK, kTile, kc0), vpl = locate(rV, kTile, vc0);
     uint32_t qf[NKS][NB][2];  // B fragments of Q^T (hi / lo parts)
 #pragma unroll
     for (int ks = 0; ks < NKS; ++ks)
@@ -585,7 +638,38 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
         ok = false;
         break;
       }
-      const uint32_t sbase = smem_u32(ring + (size_t)st * st_bytes);
+      uint32_t sbase = smem_u32(ring + (size_t)st * L.stage);
+      if (Q8) {
+        // dequantise the raw stage into this warp's bf16 tile (code x row scale, rounded to
+        // bf16, written at the positions the TMA swizzle would have given), then release
+        // the raw stage at once
+        const uint8_t* raw = ring + (size_t)st * L.stage;
+        __syncwarp();  // every lane is done reading the previous tile
+        for (int m = 0; m < 2; ++m) {
+          const int r = m ? rV : rK;
+          const int8_t* codes = reinterpret_cast<const int8_t*>(raw + (m ? L.q8_v : 0u)) + 8 * (m ? vc0 : kc0);
+          const float* scl = reinterpret_cast<const float*>(raw + (m ? L.q8_vs : L.q8_ks));
+          uint8_t* dstt = staging + (m ? kt_bytes : 0u);
+          const PieceLoc& pl = m ? vpl : kpl;
+          const int rpp = m ? vrpp : krpp;
+          if (m ? vlive : klive)
+            for (int t = m ? vt0 : kt0; t < kTile; t += rpp) {
+              const uint2 w8 = *reinterpret_cast<const uint2*>(codes + t * r);
+              const float sc = scl[t];
+              const float2 sc2 = make_float2(sc, sc);
+              const uint32_t ux = w8.x ^ 0x80808080u, uy = w8.y ^ 0x80808080u;
+              uint4 o;
+              o.x = deq_pair(ux, 0, sc2);
+              o.y = deq_pair(ux, 2, sc2);
+              o.z = deq_pair(uy, 0, sc2);
+              o.w = deq_pair(uy, 2, sc2);
+              *reinterpret_cast<uint4*>(dstt + swz(pl, t)) = o;
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[warp * ns + st]);  // the raw stage may be refilled
+        sbase = smem_u32(staging);
+      }
       const int tok0 = t0 + (warp + k * NW) * kTile;
       const int n = min(kTile, t1 - tok0);
       if (owns_new && tok0 <= Lb && Lb < tok0 + kTile) {
@@ -759,7 +843,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
             }
         }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[warp * ns + st]);  // the stage may be refilled
+      if (!Q8 && lane == 0) mbar_arrive(&empty[warp * ns + st]);  // the stage may be refilled
     }
   }
   pdl_launch_dependents();
@@ -998,10 +1082,10 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
 
 // ------------------------------------------------------------------------------ launch
 
-template <int NB, int NKS, int NMV, int TT, bool LAT, bool PG>
+template <int NB, int NKS, int NMV, int TT, int MODE>
 static cudaError_t launch_k(const DecodeArgs& a, cudaStream_t stream) {
-  const DecodeSmem L = decode_smem_layout(a.nwarps, a.nstage, a.rK, a.rV, TT);
-  auto kern = stief_decode_kernel<NB, NKS, NMV, TT, LAT, PG>;
+  const DecodeSmem L = decode_smem_layout(a.nwarps, a.nstage, a.rK, a.rV, TT, MODE == kModeQ8);
+  auto kern = stief_decode_kernel<NB, NKS, NMV, TT, MODE>;
   static SmemLimit limit;
   cudaError_t e = limit.ensure(reinterpret_cast<const void*>(kern), a.device, (int)L.total);
   if (e != cudaSuccess) return e;
@@ -1024,16 +1108,16 @@ static cudaError_t launch_k(const DecodeArgs& a, cudaStream_t stream) {
 // cost the contiguous path nothing (a runtime flag cost it 0.5-0.8 us per launch)
 template <int NB, int NKS, int NMV, int TT>
 static cudaError_t launch_t(const DecodeArgs& a, cudaStream_t stream) {
-  if (a.latent) {
-    if (a.block_table) return cudaErrorInvalidValue;  // no paged latent decode
-    return launch_k<NB, NKS, NMV, TT, true, false>(a, stream);
-  }
-  return a.block_table ? launch_k<NB, NKS, NMV, TT, false, true>(a, stream)
-                       : launch_k<NB, NKS, NMV, TT, false, false>(a, stream);
+  if ((a.latent != 0) + (a.block_table != nullptr) + (a.q8 != 0) > 1)
+    return cudaErrorInvalidValue;  // the modes do not combine
+  if (a.latent) return launch_k<NB, NKS, NMV, TT, kModeLatent>(a, stream);
+  if (a.block_table) return launch_k<NB, NKS, NMV, TT, kModePaged>(a, stream);
+  if (a.q8) return launch_k<NB, NKS, NMV, TT, kModeQ8>(a, stream);
+  return launch_k<NB, NKS, NMV, TT, kModePlain>(a, stream);
 }
 
-uint32_t decode_smem_bytes(int nwarps, int nstage, int rK, int rV, int tile) {
-  return decode_smem_layout(nwarps, nstage, rK, rV, tile).total;
+uint32_t decode_smem_bytes(int nwarps, int nstage, int rK, int rV, int tile, bool q8) {
+  return decode_smem_layout(nwarps, nstage, rK, rV, tile, q8).total;
 }
 
 template <int NB>

@@ -148,12 +148,29 @@ bool encode_tiled_bf16_2d(CUtensorMap* map, const void* base, uint64_t cols, uin
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D tiled map over an int8 matrix [rows][cols] (row stride = cols bytes), boxes of
+// box_cols x box_rows, no swizzle (the int8 stages are read row-major).
+static bool encode_tiled_u8_2d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
+                               uint32_t box_cols, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1u, 1u};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 stief_status plan_decode(DecodeArgs& a, const uint16_t* q, const uint16_t* P_K,
                          const uint16_t* P_V, const uint16_t* k_lat, const uint16_t* v_lat,
                          const int32_t* seq_lens, uint16_t* out, int B, int Hq, int Hkv, int d,
                          int rK, int rV, int L_max, int max_seq_len, int num_splits,
                          uint32_t* dev_status, bool latent, const int32_t* block_table,
-                         int max_pages, int page_size, int num_pages) {
+                         int max_pages, int page_size, int num_pages, const float* k_scale,
+                         const float* v_scale) {
+  const bool q8 = k_scale != nullptr;
   if (!q || !k_lat || !v_lat || !seq_lens || !out) return STIEF_ERR_INVALID_ARG;
   if (!latent && (!P_K || !P_V)) return STIEF_ERR_INVALID_ARG;
   if (B < 1 || B > 65535 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || Hq / Hkv > 64)
@@ -204,15 +221,31 @@ stief_status plan_decode(DecodeArgs& a, const uint16_t* q, const uint16_t* P_K,
   a.qscale = (float)(1.4426950408889634 / std::sqrt((double)d));
   const long long units = (long long)B * a.Hkv * a.qsub;
   const bool pair = a.S == 1 && units > sms &&
-                    choose_decode_config_pair(rK, rV, a.tile, &a.nwarps, &a.nstage);
-  if (!pair && !choose_decode_config(rK, rV, a.tile, &a.nwarps, &a.nstage))
+                    choose_decode_config_pair(rK, rV, a.tile, &a.nwarps, &a.nstage, q8);
+  if (!pair && !choose_decode_config(rK, rV, a.tile, &a.nwarps, &a.nstage, q8))
     return STIEF_ERR_INVALID_ARG;
 
   int nmaps = 0;
   const uint64_t prow = (uint64_t)Hkv * d;
-  if (!plan_pieces(a, &nmaps, a.pk, k_lat, rK, rows, a.tile) ||
-      !plan_pieces(a, &nmaps, a.pv, v_lat, rV, rows, a.tile))
+  a.q8 = q8 ? 1 : 0;
+  a.k_scale = k_scale;
+  a.v_scale = v_scale;
+  if (q8) {  // int8 codes: one box of r bytes x tile rows per matrix
+    if (!encode_tiled_u8_2d(&a.maps[0], k_lat, (uint64_t)rK, rows, (uint32_t)rK, (uint32_t)a.tile) ||
+        !encode_tiled_u8_2d(&a.maps[1], v_lat, (uint64_t)rV, rows, (uint32_t)rV, (uint32_t)a.tile))
+      return STIEF_ERR_CUDA;
+    a.pk.n = a.pv.n = 1;
+    a.pk.p[0] = Piece{};
+    a.pv.p[0] = Piece{};
+    a.pk.p[0].map = 0;
+    a.pv.p[0].map = 1;
+    a.pk.p[0].width = rK;
+    a.pv.p[0].width = rV;
+    nmaps = 2;
+  } else if (!plan_pieces(a, &nmaps, a.pk, k_lat, rK, rows, a.tile) ||
+             !plan_pieces(a, &nmaps, a.pv, v_lat, rV, rows, a.tile)) {
     return STIEF_ERR_CUDA;
+  }
   if (!latent && (!plan_pieces(a, &nmaps, a.ppk, P_K, rK, prow, d) ||
                   !plan_pieces(a, &nmaps, a.ppv, P_V, rV, prow, d)))
     return STIEF_ERR_CUDA;

@@ -49,6 +49,8 @@ struct Paging {
 };
 
 constexpr int kPageQuantum = 64;  // page sizes are multiples of the largest decode tile
+constexpr int kQ8RowQuantum = 64;  // int8 caches: L_max is a multiple of the largest tile,
+                                   // so a tile's scale copy never passes a head's rows
 
 // Host checks of a paged cache; on success *capacity = max_pages * page_size tokens.
 stief_status check_paging(const Paging& pg, int Hkv, int* capacity) {
@@ -120,7 +122,8 @@ stief_status compress_common(const uint16_t* k_new, const uint16_t* v_new, const
                              const uint16_t* P_V, uint16_t* k_lat, uint16_t* v_lat,
                              int32_t* seq_lens, int B, int Hkv, int T, int d, int rK, int rV,
                              int L_max, uint32_t* dev_status, stief_stream_t stream,
-                             const Paging& pg) {
+                             const Paging& pg, float* k_scale = nullptr,
+                             float* v_scale = nullptr) {
   if (!k_new || !v_new || !P_K || !P_V || !k_lat || !v_lat || !seq_lens) return STIEF_ERR_INVALID_ARG;
   if (pg.block_table) {
     const stief_status st = check_paging(pg, Hkv, &L_max);
@@ -157,6 +160,8 @@ stief_status compress_common(const uint16_t* k_new, const uint16_t* v_new, const
   a.max_pages = pg.max_pages;
   a.page_size = pg.page_size;
   a.num_pages = pg.num_pages;
+  a.k_scale = k_scale;
+  a.v_scale = v_scale;
   if (stief::launch_compress(a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return STIEF_ERR_CUDA;
   return STIEF_OK;
@@ -173,6 +178,19 @@ stief_status stief_compress_append(const uint16_t* k_new, const uint16_t* v_new,
                                    stief_stream_t stream) {
   return compress_common(k_new, v_new, P_K, P_V, k_lat, v_lat, seq_lens, B, Hkv, T, d, rK, rV,
                          L_max, dev_status, stream, Paging{});
+}
+
+stief_status stief_compress_append_q8(const uint16_t* k_new, const uint16_t* v_new,
+                                      const uint16_t* P_K, const uint16_t* P_V, int8_t* k_q,
+                                      int8_t* v_q, float* k_s, float* v_s, int32_t* seq_lens,
+                                      int B, int Hkv, int T, int d, int rK, int rV, int L_max,
+                                      uint32_t* dev_status, stief_stream_t stream) {
+  if (!k_s || !v_s) return STIEF_ERR_INVALID_ARG;
+  if (L_max % kQ8RowQuantum != 0) return STIEF_ERR_INVALID_ARG;
+  if (!aligned16(k_s) || !aligned16(v_s)) return STIEF_ERR_ALIGNMENT;
+  return compress_common(k_new, v_new, P_K, P_V, reinterpret_cast<uint16_t*>(k_q),
+                         reinterpret_cast<uint16_t*>(v_q), seq_lens, B, Hkv, T, d, rK, rV, L_max,
+                         dev_status, stream, Paging{}, k_s, v_s);
 }
 
 stief_status stief_compress_append_paged(const uint16_t* k_new, const uint16_t* v_new,
@@ -201,7 +219,8 @@ stief_status decode_common(const uint16_t* q, const uint16_t* k_new, const uint1
                            size_t workspace_bytes, int B, int Hq, int Hkv, int d, int rK, int rV,
                            int L_max, int max_seq_len, int num_splits, uint32_t* dev_status,
                            stief_stream_t stream, bool append, bool latent = false,
-                           const Paging& pg = Paging{}) {
+                           const Paging& pg = Paging{}, const float* k_scale = nullptr,
+                           const float* v_scale = nullptr) {
   // cheap host checks first, so argument errors never touch CUDA
   if (!q || !k_lat || !v_lat || !seq_lens || !out) return STIEF_ERR_INVALID_ARG;
   if (pg.block_table) {  // paged: the capacity is max_pages * page_size tokens
@@ -225,7 +244,7 @@ stief_status decode_common(const uint16_t* q, const uint16_t* k_new, const uint1
   stief::DecodeArgs a{};
   st = stief::plan_decode(a, q, P_K, P_V, k_lat, v_lat, seq_lens, out, B, Hq, Hkv, d, rK, rV,
                           L_max, max_seq_len, num_splits, dev_status, latent, pg.block_table,
-                          pg.max_pages, pg.page_size, pg.num_pages);
+                          pg.max_pages, pg.page_size, pg.num_pages, k_scale, v_scale);
   if (st != STIEF_OK) return st;
   a.append = append ? 1 : 0;
   a.k_new = k_new;
@@ -280,6 +299,25 @@ stief_status stief_decode_latent(const uint16_t* q_lat, const uint16_t* k_lat,
                        const_cast<uint16_t*>(v_lat), const_cast<int32_t*>(seq_lens), out_lat,
                        workspace, workspace_bytes, B, Hq, Hkv, d, rK, rV, L_max, max_seq_len,
                        num_splits, dev_status, stream, false, true);
+}
+
+stief_status stief_decode_attention_q8(const uint16_t* q, const uint16_t* P_K,
+                                       const uint16_t* P_V, const int8_t* k_q, const int8_t* v_q,
+                                       const float* k_s, const float* v_s,
+                                       const int32_t* seq_lens, uint16_t* out, void* workspace,
+                                       size_t workspace_bytes, int B, int Hq, int Hkv, int d,
+                                       int rK, int rV, int L_max, int max_seq_len,
+                                       int num_splits, uint32_t* dev_status,
+                                       stief_stream_t stream) {
+  if (!k_s || !v_s) return STIEF_ERR_INVALID_ARG;
+  if (L_max % kQ8RowQuantum != 0) return STIEF_ERR_INVALID_ARG;
+  if (!aligned16(k_s) || !aligned16(v_s)) return STIEF_ERR_ALIGNMENT;
+  return decode_common(q, nullptr, nullptr, P_K, P_V,
+                       reinterpret_cast<uint16_t*>(const_cast<int8_t*>(k_q)),
+                       reinterpret_cast<uint16_t*>(const_cast<int8_t*>(v_q)),
+                       const_cast<int32_t*>(seq_lens), out, workspace, workspace_bytes, B, Hq, Hkv,
+                       d, rK, rV, L_max, max_seq_len, num_splits, dev_status, stream, false, false,
+                       Paging{}, k_s, v_s);
 }
 
 stief_status stief_decode_attention_paged(const uint16_t* q, const uint16_t* P_K,

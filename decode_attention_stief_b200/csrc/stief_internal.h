@@ -61,6 +61,10 @@ struct DecodeArgs {
   // [B][max_pages] (null for a contiguous cache; L_max is then max_pages * page_size)
   const int32_t* block_table;
   int max_pages, page_size, num_pages;
+  // int8 caches: k_lat / v_lat hold int8 codes [rows][r] and these the fp32 row scales
+  int q8;
+  const float* k_scale;
+  const float* v_scale;
 };
 
 struct CompressArgs {
@@ -77,6 +81,9 @@ struct CompressArgs {
   // paged caches, as in DecodeArgs (block_table null: contiguous [B][Hkv][L_max] rows)
   const int32_t* block_table;
   int max_pages, page_size, num_pages;
+  // int8 caches: k_lat / v_lat take int8 codes and these the fp32 row scales (null: bf16)
+  float* k_scale;
+  float* v_scale;
 };
 
 constexpr int kMaxSmemPerBlock = 232448;  // 227 KB opt-in dynamic shared memory (sm_100)
@@ -102,7 +109,7 @@ struct SmemLimit {
   }
 };
 
-uint32_t decode_smem_bytes(int nwarps, int nstage, int rK, int rV, int tile);
+uint32_t decode_smem_bytes(int nwarps, int nstage, int rK, int rV, int tile, bool q8 = false);
 
 // 2-D tiled TMA tensor map over a row-major bf16 matrix [rows][cols] (row stride in
 // bytes), boxes of box_cols x box_rows with the given swizzle.  Host only.
@@ -117,14 +124,16 @@ uint32_t compress_tc_smem_bytes(int rK, int rV);
 // (split count, group tiling, CTA configuration, key tensor maps).  Host only.
 // With `latent`, q is q~ [B][Hq][rK], out is o~ [B][Hq][rV] and P_K, P_V are unused (may be
 // NULL): no base tensor maps are planned.  With a block table, k_lat / v_lat are page pools
-// [num_pages][Hkv][page_size][r] and L_max is the capacity max_pages * page_size.
+// [num_pages][Hkv][page_size][r] and L_max is the capacity max_pages * page_size.  With row
+// scales (k_scale, v_scale), k_lat / v_lat are int8 codes [B][Hkv][L_max][r].
 stief_status plan_decode(DecodeArgs& a, const uint16_t* q, const uint16_t* P_K,
                          const uint16_t* P_V, const uint16_t* k_lat, const uint16_t* v_lat,
                          const int32_t* seq_lens, uint16_t* out, int B, int Hq, int Hkv, int d,
                          int rK, int rV, int L_max, int max_seq_len, int num_splits,
                          uint32_t* dev_status, bool latent = false,
                          const int32_t* block_table = nullptr, int max_pages = 0,
-                         int page_size = 0, int num_pages = 0);
+                         int page_size = 0, int num_pages = 0, const float* k_scale = nullptr,
+                         const float* v_scale = nullptr);
 
 // Decode workspace layout: `units` = B * Hkv * qsub split-ticket counters, then B sequence
 // tickets (uint32, padded together to 256 bytes), then units * G_T * splits partial states
@@ -151,20 +160,22 @@ inline int choose_decode_tile(int rK, int rV) { return rK <= 64 && rV <= 64 && r
 // consumer warps.  Fewer than four consumer warps per CTA is not worth it.
 constexpr int kPairSmemPerBlock = 233472 / 2 - 1024;
 constexpr int kPairMaxConsumerWarps = 5;
-inline bool choose_decode_config_pair(int rK, int rV, int tile, int* nwarps, int* nstage) {
+inline bool choose_decode_config_pair(int rK, int rV, int tile, int* nwarps, int* nstage,
+                                      bool q8 = false) {
   for (int nw = kPairMaxConsumerWarps; nw >= 4; --nw)
     for (int ns = 4; ns >= 2; --ns)
-      if (decode_smem_bytes(nw, ns, rK, rV, tile) <= (uint32_t)kPairSmemPerBlock) {
+      if (decode_smem_bytes(nw, ns, rK, rV, tile, q8) <= (uint32_t)kPairSmemPerBlock) {
         *nwarps = nw;
         *nstage = ns;
         return true;
       }
   return false;
 }
-inline bool choose_decode_config(int rK, int rV, int tile, int* nwarps, int* nstage) {
+inline bool choose_decode_config(int rK, int rV, int tile, int* nwarps, int* nstage,
+                                 bool q8 = false) {
   for (int nw = 8; nw >= 2; --nw)
     for (int ns = 8; ns >= 2; --ns)
-      if (decode_smem_bytes(nw, ns, rK, rV, tile) <= (uint32_t)kMaxSmemPerBlock) {
+      if (decode_smem_bytes(nw, ns, rK, rV, tile, q8) <= (uint32_t)kMaxSmemPerBlock) {
         *nwarps = nw;
         *nstage = ns;
         return true;

@@ -308,6 +308,34 @@ STIEF_API stief_status stief_append_decode_paged(const uint16_t* q, const uint16
                                        stief_stream_t stream);
 
 /*
+ * int8 latent caches (the low-bit form).  The pages report the compressed cache to be
+ * robust to 4- and 8-bit quantisation but fix no scheme; this library stores each latent
+ * row (one token, one KV head) as int8 codes and one fp32 scale:
+ *     k_q : int8 [B][Hkv][L_max][rK],  k_s : float [B][Hkv][L_max]  (likewise v_q, v_s)
+ *     scale = max_c |x_c| / 127,  code_c = RNE(x_c / scale) in [-127, 127]
+ * where x is the row rounded to bf16 (what the bf16 cache would hold), both divisions in
+ * IEEE fp32; a zero row is scale 0 and codes 0.  A value stands for code * scale.
+ * A row takes r + 4 bytes instead of the bf16 cache's 2 r.  L_max must be a multiple of 64; k_s, v_s, k_q, v_q
+ * 16-byte aligned.  The calls are their bf16 counterparts on this form: the compress writes
+ * codes and scales; the decode attends over code * scale (dequantised on chip to bf16, then
+ * the same tensor-core path).  Paged int8 caches and the fused step are not provided.
+ */
+STIEF_API stief_status stief_compress_append_q8(const uint16_t* k_new, const uint16_t* v_new,
+                                      const uint16_t* P_K, const uint16_t* P_V, int8_t* k_q,
+                                      int8_t* v_q, float* k_s, float* v_s, int32_t* seq_lens,
+                                      int B, int Hkv, int T, int d, int rK, int rV, int L_max,
+                                      uint32_t* dev_status, stief_stream_t stream);
+
+STIEF_API stief_status stief_decode_attention_q8(const uint16_t* q, const uint16_t* P_K,
+                                       const uint16_t* P_V, const int8_t* k_q, const int8_t* v_q,
+                                       const float* k_s, const float* v_s,
+                                       const int32_t* seq_lens, uint16_t* out, void* workspace,
+                                       size_t workspace_bytes, int B, int Hq, int Hkv, int d,
+                                       int rK, int rV, int L_max, int max_seq_len,
+                                       int num_splits, uint32_t* dev_status,
+                                       stief_stream_t stream);
+
+/*
  * stief_decode_attention_noalloc -- stief_decode_attention without a workspace
  * argument and without any device allocation.  The paper has no counterpart: this
  * is a deployment variant for callers that cannot obtain device memory when they

@@ -135,6 +135,27 @@ def test_paged_decode_argument_errors(lib, kw, code):
     assert _paged(lib, **kw) == code
 
 
+def _q8(lib, **kw):
+    a = dict(q=FAKE, P_K=FAKE, P_V=FAKE, kq=FAKE, vq=FAKE, ks=FAKE, vs=FAKE, sl=FAKE, out=FAKE,
+             ws=FAKE, ws_bytes=1 << 40, B=1, Hq=32, Hkv=8, d=128, rK=64, rV=64, L_max=1024,
+             max_seq_len=1024, num_splits=0)
+    a.update(kw)
+    return lib.stief_decode_attention_q8(a["q"], a["P_K"], a["P_V"], a["kq"], a["vq"], a["ks"],
+                                         a["vs"], a["sl"], a["out"], a["ws"], a["ws_bytes"], a["B"],
+                                         a["Hq"], a["Hkv"], a["d"], a["rK"], a["rV"], a["L_max"],
+                                         a["max_seq_len"], a["num_splits"], None, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(ks=None), INVALID), (dict(vs=None), INVALID),
+    (dict(L_max=1000, max_seq_len=1000), INVALID),  # int8 caches: L_max a multiple of 64
+    (dict(ks=FAKE + 4), ALIGN), (dict(kq=FAKE + 8), ALIGN), (dict(rK=40), INVALID),
+    (dict(ws=None), WORKSPACE),
+])
+def test_q8_decode_argument_errors(lib, kw, code):
+    assert _q8(lib, **kw) == code
+
+
 @pytest.mark.parametrize("kw,code", [
     (dict(k=None), INVALID), (dict(sl=None), INVALID), (dict(d=96), INVALID),
     (dict(rK=24), INVALID), (dict(T=-1), INVALID), (dict(B=0), INVALID),

@@ -1,0 +1,154 @@
+"""int8 latent caches: stief_compress_append_q8 and stief_decode_attention_q8 (CUDA, through
+the C ABI) against the fp64 oracle.
+
+The stored form is the oracle's quantize_rows (one fp32 scale per row, RNE codes, both
+divisions in IEEE fp32) applied to the bf16-rounded latent row.  With the identity basis the
+latent rows are exact bf16 values on both sides, so the integer codes and the scales must be
+bit-identical; with general bases the GPU's bf16 row can differ from the oracle's by an ulp
+at a rounding boundary, so codes may differ by one there.  The decode is checked against
+the oracle's decode over code * scale, tolerance 2e-2 * ||o||_inf as for the bf16 cache.
+"""
+import numpy as np
+import pytest
+import torch
+
+import decode_attention_stief_b200 as stief
+import oracle
+import stief_inputs as si
+from gpu_util import assert_decode_close, f64
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda")
+
+
+def _identity_basis(Hkv, d, r):
+    P = np.zeros((Hkv, d, r))
+    for h in range(Hkv):
+        P[h, :r, :] = np.eye(r)
+    return si.to_bf16(P)
+
+
+def _compress_q8(k_new, v_new, P_K, P_V, B, Hkv, L_max, rK, rV, lens, expect_status=0):
+    kq = torch.zeros((B, Hkv, L_max, rK), dtype=torch.int8, device=DEV)
+    vq = torch.zeros((B, Hkv, L_max, rV), dtype=torch.int8, device=DEV)
+    ks = torch.full((B, Hkv, L_max), -1.0, dtype=torch.float32, device=DEV)
+    vs = torch.full((B, Hkv, L_max), -1.0, dtype=torch.float32, device=DEV)
+    lens_t = torch.as_tensor(np.asarray(lens, np.int32)).to(DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    stief.stief_compress_append_q8(k_new.to(DEV), v_new.to(DEV), P_K.to(DEV), P_V.to(DEV), kq, vq,
+                                   ks, vs, lens_t, dev_status=status)
+    assert stief.stief_read_device_status(status) == expect_status
+    return kq.cpu(), vq.cpu(), ks.cpu(), vs.cpu(), lens_t.cpu().numpy()
+
+
+@pytest.mark.parametrize("T", [1, 5, 8, 200])
+def test_identity_basis_codes_and_scales_are_bit_exact(T):
+    """P = [I; 0]: the latent row is the first r coordinates of the bf16 row exactly, so the
+    quantisation decisions are taken on identical inputs (CUDA-core path T < 128, tensor
+    cores from 128)."""
+    B, Hkv, rK, rV, L_max = 2, 2, 64, 48, 256
+    k_new, v_new = si.full_kv(6000 + T, B, Hkv, T, 128)
+    P_K, P_V = _identity_basis(Hkv, 128, rK), _identity_basis(Hkv, 128, rV)
+    lens = [0, 37]
+    kq, vq, ks, vs, glens = _compress_q8(k_new, v_new, P_K, P_V, B, Hkv, L_max, rK, rV, lens)
+    assert glens.tolist() == [L + T for L in lens]
+    for b, L in enumerate(lens):
+        wk, wks = oracle.quantize_rows(f64(k_new[b])[..., :rK])
+        wv, wvs = oracle.quantize_rows(f64(v_new[b])[..., :rV])
+        assert np.array_equal(kq[b, :, L:L + T].numpy(), wk)
+        assert np.array_equal(vq[b, :, L:L + T].numpy(), wv)
+        assert np.array_equal(ks[b, :, L:L + T].numpy(), wks)
+        assert np.array_equal(vs[b, :, L:L + T].numpy(), wvs)
+        assert torch.all(ks[b, :, :L] == -1) and torch.all(ks[b, :, L + T:] == -1)
+
+
+@pytest.mark.parametrize("T", [3, 130])
+def test_general_bases_codes_within_one(T):
+    B, Hkv, rK, rV, L_max = 1, 4, 64, 64, 192
+    k_new, v_new = si.full_kv(6100 + T, B, Hkv, T, 128)
+    P_K, P_V = si.bases_bf16(6100 + T, Hkv, 128, rK, rV)
+    kq, vq, ks, vs, _ = _compress_q8(k_new, v_new, P_K, P_V, B, Hkv, L_max, rK, rV, [10])
+    for m, (q, s, x, P) in enumerate(((kq, ks, k_new, P_K), (vq, vs, v_new, P_V))):
+        for h in range(Hkv):
+            lat = oracle.project(f64(x[0, h]), f64(P[h]), round_to_bf16=True)
+            wq, ws = oracle.quantize_rows(lat)
+            gq = q[0, h, 10:10 + T].numpy().astype(np.int32)
+            assert np.max(np.abs(gq - wq.astype(np.int32))) <= 1
+            assert np.mean(gq == wq) > 0.98
+            np.testing.assert_allclose(s[0, h, 10:10 + T].numpy(), ws, rtol=2 ** -7)
+
+
+def _random_q8_cache(seed, B, Hkv, L, r):
+    """Seeded codes and scales: the int8 form of a low-rank latent cache."""
+    lat = si.latent_cache(seed, B, Hkv, L, r, 0)
+    q, s = oracle.quantize_rows(f64(lat))
+    return torch.from_numpy(q), torch.from_numpy(s)
+
+
+def _decode_q8(q, P_K, P_V, kq, vq, ks, vs, lens, max_seq_len, num_splits=0):
+    B, Hq, d = q.shape
+    out = torch.full((B, Hq, d), float("nan"), dtype=torch.bfloat16, device=DEV)
+    ws = stief.workspace_for(B, Hq, P_K.shape[0], P_V.shape[2], max_seq_len)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    stief.stief_decode_attention_q8(q.to(DEV), P_K.to(DEV), P_V.to(DEV), kq.to(DEV), vq.to(DEV),
+                                    ks.to(DEV), vs.to(DEV),
+                                    torch.as_tensor(np.asarray(lens, np.int32)).to(DEV), out, ws,
+                                    max_seq_len, num_splits=num_splits, dev_status=status)
+    assert stief.stief_read_device_status(status) == 0
+    return out.cpu()
+
+
+@pytest.mark.parametrize("rK,rV", [(64, 64), (32, 48), (96, 128), (16, 16)])
+@pytest.mark.parametrize("num_splits", [0, 1, 3])
+def test_decode_q8_matches_oracle(rK, rV, num_splits):
+    B, Hq, Hkv, L = 3, 16, 4, 704
+    lens = [700, 33, 0]
+    q = si.queries(6200 + rK, B, Hq, 128)
+    P_K, P_V = si.bases_bf16(6200 + rV, Hkv, 128, rK, rV)
+    kq, ks = _random_q8_cache(6201 + rK, B, Hkv, L, rK)
+    vq, vs = _random_q8_cache(6202 + rV, B, Hkv, L, rV)
+    got = _decode_q8(q, P_K, P_V, kq, vq, ks, vs, lens, 700, num_splits)
+    want = oracle.decode(f64(q), f64(P_K), f64(P_V), oracle.dequantize_rows(kq.numpy(), ks.numpy()),
+                         oracle.dequantize_rows(vq.numpy(), vs.numpy()), np.asarray(lens, np.int32))
+    assert_decode_close(got, want)
+    assert torch.all(got[2].float() == 0)
+
+
+def test_compress_then_decode_q8_end_to_end():
+    """Prefill chunk into an int8 cache on the tensor cores, then a decode over it, against
+    the oracle's projection, quantisation and decode."""
+    B, Hq, Hkv, rK, rV, T, L_max = 2, 32, 8, 64, 64, 300, 320
+    k_new, v_new = si.full_kv(6300, B, Hkv, T, 128)
+    P_K, P_V = si.bases_bf16(6300, Hkv, 128, rK, rV)
+    kq, vq, ks, vs, glens = _compress_q8(k_new, v_new, P_K, P_V, B, Hkv, L_max, rK, rV, [0, 0])
+    q = si.queries(6301, B, Hq, 128)
+    lens = [300, 171]
+    got = _decode_q8(q, P_K, P_V, kq, vq, ks, vs, lens, L_max)
+    wk = np.zeros((B, Hkv, L_max, rK))
+    wv = np.zeros((B, Hkv, L_max, rV))
+    for b in range(B):
+        for h in range(Hkv):
+            c, s = oracle.quantize_rows(oracle.project(f64(k_new[b, h]), f64(P_K[h])))
+            wk[b, h, :T] = oracle.dequantize_rows(c, s)
+            c, s = oracle.quantize_rows(oracle.project(f64(v_new[b, h]), f64(P_V[h])))
+            wv[b, h, :T] = oracle.dequantize_rows(c, s)
+    want = oracle.decode(f64(q), f64(P_K), f64(P_V), wk, wv, np.asarray(lens, np.int32))
+    assert_decode_close(got, want)
+
+
+@pytest.mark.parametrize("name", ["llama3_8b_32k", "llama31_8b_128k"])
+def test_decode_q8_full_size(name):
+    """The benchmark shapes at full context over an int8 cache; sequence 0 checked exactly."""
+    w = si.WORKLOADS[name]
+    seed = si.sub_seed(w.seed, 48)
+    k = si.latent_cache_torch(seed, w.B, w.Hkv, w.L, w.rK, 0, DEV)
+    v = si.latent_cache_torch(seed, w.B, w.Hkv, w.L, w.rV, 1, DEV)
+    kq, ks = oracle.quantize_rows(f64(k))
+    vq, vs = oracle.quantize_rows(f64(v))
+    kq, ks, vq, vs = (torch.from_numpy(x) for x in (kq, ks, vq, vs))
+    q = si.queries_torch(seed + 1, w.B, w.Hq, w.d, DEV)
+    P_K, P_V = si.bases_bf16(seed, w.Hkv, w.d, w.rK, w.rV)
+    got = _decode_q8(q, P_K, P_V, kq, vq, ks, vs, [w.L] * w.B, w.L)
+    want = oracle.decode(f64(q), f64(P_K), f64(P_V), oracle.dequantize_rows(kq.numpy(), ks.numpy()),
+                         oracle.dequantize_rows(vq.numpy(), vs.numpy()), np.full(w.B, w.L, np.int32))
+    assert_decode_close(got, want)
