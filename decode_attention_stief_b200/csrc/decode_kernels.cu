@@ -37,6 +37,8 @@
 #include <cmath>
 #include <cstdint>
 
+#include <cuda_fp16.h>
+
 #include "stief_device.cuh"
 #include "stief_internal.h"
 
@@ -98,6 +100,52 @@ __device__ __forceinline__ void mma_bf16_z(float (&c)[4], const uint32_t (&a)[4]
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.f));
 }
 
+// The same two products with fp16 operands (the int8 caches' codes are exact in fp16).
+__device__ __forceinline__ void mma_f16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                        uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma_f16_z(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                          uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%10,%10,%10,%10};"
+      : "=f"(c[0]), "=f"(c[1]), "=f"(c[2]), "=f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.f));
+}
+template <bool F16>
+__device__ __forceinline__ void mma_op(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  if constexpr (F16) mma_f16(c, a, b0, b1);
+  else mma_bf16(c, a, b0, b1);
+}
+template <bool F16>
+__device__ __forceinline__ void mma_op_z(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  if constexpr (F16) mma_f16_z(c, a, b0, b1);
+  else mma_bf16_z(c, a, b0, b1);
+}
+
+// fp16 hi / lo parts of an fp32 pair, packed (first element in the low half)
+__device__ __forceinline__ uint32_t hi_pair_h(float x0, float x1) {
+  const __half2 h = __floats2half2_rn(x0, x1);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+__device__ __forceinline__ uint32_t lo_pair_h(float x0, float x1, uint32_t hi) {
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hi));
+  return hi_pair_h(x0 - f.x, x1 - f.y);
+}
+// Four int8 codes (w) as exact fp16 pairs: 0x64uu is 1024 + uu in fp16, uu = code + 128.
+__device__ __forceinline__ void codes_f16(uint32_t w, uint32_t& h01, uint32_t& h23) {
+  const uint32_t u = w ^ 0x80808080u;
+  const uint32_t a = __byte_perm(u, 0x64646464u, 0x5140u), b = __byte_perm(u, 0x64646464u, 0x7362u);
+  // minus 1152 = 1024 + 128 in both halves (0x6480 is 1152 in fp16)
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(h01) : "r"(a), "r"(0x64806480u));
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(h23) : "r"(b), "r"(0x64806480u));
+}
+
 // hi / lo bf16 parts of an fp32 pair, packed (first element in the low half)
 __device__ __forceinline__ uint32_t hi_pair(float x0, float x1) { return pack_bf16x2_rn(x0, x1); }
 __device__ __forceinline__ uint32_t lo_pair(float x0, float x1, uint32_t hi) {
@@ -135,15 +183,6 @@ __device__ __forceinline__ PieceLoc locate(int r, int rows, int chunk) {
   }
   return pl;
 }
-// Two int8 codes (bytes j and j + 1 of w) times a scale, rounded to bf16 and packed.  A
-// code c becomes exact fp32 through the bit pattern of 2^23 + (c + 128) less 2^23 + 128.
-__device__ __forceinline__ uint32_t deq_pair(uint32_t u, int j, float2 sc2) {
-  // u: the codes + 128 as unsigned bytes (w ^ 0x80808080)
-  float2 c = make_float2(__uint_as_float(__byte_perm(u, 0x4B000000u, 0x7540u | (uint32_t)j)),
-                         __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7540u | (uint32_t)(j + 1))));
-  c = __fmul2_rn(__fadd2_rn(c, make_float2(-8388736.f, -8388736.f)), sc2);
-  return pack_bf16x2_rn(c.x, c.y);
-}
 // Byte offset of (row, chunk) under the piece's TMA swizzle: 128-byte rows XOR the chunk
 // with row & 7, 64-byte rows with (row >> 1) & 3, 32-byte rows with (row >> 2) & 1.
 __device__ __forceinline__ uint32_t swz(const PieceLoc& pl, int row) {
@@ -167,14 +206,16 @@ __device__ __forceinline__ int at_chunk(int lane) { return (lane >> 3) & 1; }
 // top; k = cols 16 ks + 2 (lane & 3) + {0, 1} (first register) and + 8 (second).
 template <int NB>
 __device__ __forceinline__ void bfrag_hilo(const float* X, int xs, int ks, int lane,
-                                           uint32_t (&bf)[NB][2]) {
+                                           uint32_t (&bf)[NB][2], bool f16 = false) {
   const int n = lane >> 2;
   const int c = 16 * ks + 2 * (lane & 3);
   const int head = NB == 1 ? (n & 3) : n;
   const float2 x = *reinterpret_cast<const float2*>(X + head * xs + c);
   const float2 y = *reinterpret_cast<const float2*>(X + head * xs + c + 8);
-  const uint32_t hx = hi_pair(x.x, x.y), hy = hi_pair(y.x, y.y);
-  const uint32_t lx = lo_pair(x.x, x.y, hx), ly = lo_pair(y.x, y.y, hy);
+  const uint32_t hx = f16 ? hi_pair_h(x.x, x.y) : hi_pair(x.x, x.y);
+  const uint32_t hy = f16 ? hi_pair_h(y.x, y.y) : hi_pair(y.x, y.y);
+  const uint32_t lx = f16 ? lo_pair_h(x.x, x.y, hx) : lo_pair(x.x, x.y, hx);
+  const uint32_t ly = f16 ? lo_pair_h(y.x, y.y, hy) : lo_pair(y.x, y.y, hy);
   if constexpr (NB == 1) {
     const bool lo = (n >> 2) != 0;
     bf[0][0] = lo ? lx : hx;
@@ -202,10 +243,12 @@ struct DecodeSmem {
   uint32_t region;  // per warp a ring of stages (keys then values of a tile); later the
                     // cross-warp reduction and the split-merge staging
   uint32_t region_bytes;
-  // int8 caches: the region holds one bf16 tile per warp (the dequantised stage, laid out
-  // as a bf16 ring stage), then the rings of raw stages: codes K [tile][rK], codes V
+  // int8 caches: the region holds one 16-bit tile per warp (the stage's codes as fp16,
+  // row-major, rows padded by 16 bytes), then the rings of raw stages: codes K [tile][rK], codes V
   // [tile][rV], scales K [tile], scales V [tile]
   uint32_t ring;      // offset of the rings inside the region
+  uint32_t q8_sc;     // int8 caches: per warp the tile's key then value row scales (fp32)
+  uint32_t q8_tile;   // int8 caches: bytes of a warp's 16-bit tile
   uint32_t stage;     // bytes of one ring stage
   uint32_t q8_v, q8_ks, q8_vs;  // offsets inside a raw int8 stage
   uint32_t total;
@@ -239,9 +282,12 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int NW, int ns, int rK,
     s.q8_ks = s.q8_v + align_up((uint32_t)tile * rV, 128);
     s.q8_vs = s.q8_ks + (uint32_t)tile * 4u;
     s.stage = align_up(s.q8_vs + (uint32_t)tile * 4u, 128);
-    s.ring = (uint32_t)NW * bf16_stage;
+    // the 16-bit tile is row-major with rows padded by 16 bytes (conflict-free ldmatrix)
+    s.q8_tile = (uint32_t)tile * (2u * rK + 16u + 2u * rV + 16u);
+    s.q8_sc = (uint32_t)NW * s.q8_tile;
+    s.ring = align_up(s.q8_sc + (uint32_t)NW * 8u * tile, 128);
   } else {
-    s.q8_v = s.q8_ks = s.q8_vs = 0;
+    s.q8_v = s.q8_ks = s.q8_vs = s.q8_sc = s.q8_tile = 0;
     s.stage = bf16_stage;
     s.ring = 0;
   }
@@ -604,7 +650,9 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
     // ---- consumers: stream the warp's tiles ------------------------------------------------
     const int my_tiles = warp_tiles(warp, n_tiles);
     uint8_t* ring = smem + L.region + L.ring + (size_t)warp * ns * L.stage;
-    uint8_t* staging = smem + L.region + (size_t)warp * st_bytes;  // int8 caches only
+    uint8_t* staging = smem + L.region + (size_t)warp * L.q8_tile;  // int8 caches only
+    const uint32_t sK = 2u * rK + 16u, sV = 2u * rV + 16u;  // its row strides
+    const uint32_t q8_kt = (uint32_t)kTile * sK;            // its value rows' offset
     // int8 caches: in the dequantise pass a lane takes one 8-column chunk of each matrix and
     // every (32 / chunks per row)-th row of it (no division per item); its chunk's place in
     // the swizzled bf16 tile is fixed
@@ -613,20 +661,30 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
     const bool klive = lane < krpp * kcpr, vlive = lane < vrpp * vcpr;
     const int kc0 = lane % kcpr, vc0 = lane % vcpr;
     const int kt0 = lane / kcpr, vt0 = lane / vcpr;
-    const PieceLoc kpl = locate(rK, kTile, kc0), vpl = locate(rV, kTile, vc0);
+
     uint32_t qf[NKS][NB][2];  // B fragments of Q^T (hi / lo parts)
 #pragma unroll
     for (int ks = 0; ks < NKS; ++ks)
-      if (ks < nks) bfrag_hilo<NB>(qt, xs, ks, lane, qf[ks]);
+      if (ks < nks) bfrag_hilo<NB>(qt, xs, ks, lane, qf[ks], Q8);  // fp16 against int8 codes
     uint32_t koff[NKS], kstep[NKS], voff[NMV], vstep[NMV];
 #pragma unroll
     for (int ks = 0; ks < NKS; ++ks) {
+      if (Q8) {  // the row-major padded 16-bit tile
+        koff[ks] = (uint32_t)a_row(lane) * sK + (uint32_t)(2 * ks + a_chunk(lane)) * 16u;
+        kstep[ks] = 16u * sK;
+        continue;
+      }
       const PieceLoc pl = locate(rK, kTile, 2 * ks + a_chunk(lane));
       koff[ks] = swz(pl, a_row(lane));
       kstep[ks] = 32u * pl.w;  // 16 rows further (the swizzle repeats every 8 rows)
     }
 #pragma unroll
     for (int mt = 0; mt < NMV; ++mt) {
+      if (Q8) {
+        voff[mt] = q8_kt + (uint32_t)at_row(lane) * sV + (uint32_t)(2 * mt + at_chunk(lane)) * 16u;
+        vstep[mt] = 16u * sV;
+        continue;
+      }
       const PieceLoc pl = locate(rV, kTile, 2 * mt + at_chunk(lane));
       voff[mt] = kt_bytes + swz(pl, at_row(lane));
       vstep[mt] = 32u * pl.w;
@@ -639,39 +697,41 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
         break;
       }
       uint32_t sbase = smem_u32(ring + (size_t)st * L.stage);
+      const int tok0 = t0 + (warp + k * NW) * kTile;
+      const int n = min(kTile, t1 - tok0);
+      // int8 caches: the tile's row scales go to this warp's scale buffer (0 past the
+      // sequence, so that whatever the scale rows hold there reaches nothing) and the codes
+      // become exact fp16 in its 16-bit tile
+      float* scw = reinterpret_cast<float*>(smem + L.region + L.q8_sc) + warp * 2 * kTile;
       if (Q8) {
-        // dequantise the raw stage into this warp's bf16 tile (code x row scale, rounded to
-        // bf16, written at the positions the TMA swizzle would have given), then release
-        // the raw stage at once
         const uint8_t* raw = ring + (size_t)st * L.stage;
-        __syncwarp();  // every lane is done reading the previous tile
+        const float* scr = reinterpret_cast<const float*>(raw + L.q8_ks);  // K then V rows
+        __syncwarp();  // every lane is done reading the previous tile and its scales
+        for (int i = lane; i < 2 * kTile; i += 32)  // the V row follows the K row in the stage
+          scw[i] = (i < kTile ? i : i - kTile) < n ? scr[i] : 0.f;
         for (int m = 0; m < 2; ++m) {
           const int r = m ? rV : rK;
           const int8_t* codes = reinterpret_cast<const int8_t*>(raw + (m ? L.q8_v : 0u)) + 8 * (m ? vc0 : kc0);
-          const float* scl = reinterpret_cast<const float*>(raw + (m ? L.q8_vs : L.q8_ks));
-          uint8_t* dstt = staging + (m ? kt_bytes : 0u);
-          const PieceLoc& pl = m ? vpl : kpl;
+          const uint32_t stride = m ? sV : sK;
           const int rpp = m ? vrpp : krpp;
+          const int t0 = m ? vt0 : kt0;
+          uint8_t* dst = staging + (m ? q8_kt : 0u) + (uint32_t)t0 * stride + 16u * (uint32_t)(m ? vc0 : kc0);
+          const int8_t* src = codes + t0 * r;
+          const uint32_t dstep = (uint32_t)rpp * stride;
+          const int sstep = rpp * r;
           if (m ? vlive : klive)
-            for (int t = m ? vt0 : kt0; t < kTile; t += rpp) {
-              const uint2 w8 = *reinterpret_cast<const uint2*>(codes + t * r);
-              const float sc = scl[t];
-              const float2 sc2 = make_float2(sc, sc);
-              const uint32_t ux = w8.x ^ 0x80808080u, uy = w8.y ^ 0x80808080u;
+            for (int t = t0; t < kTile; t += rpp, dst += dstep, src += sstep) {
+              const uint2 w8 = *reinterpret_cast<const uint2*>(src);
               uint4 o;
-              o.x = deq_pair(ux, 0, sc2);
-              o.y = deq_pair(ux, 2, sc2);
-              o.z = deq_pair(uy, 0, sc2);
-              o.w = deq_pair(uy, 2, sc2);
-              *reinterpret_cast<uint4*>(dstt + swz(pl, t)) = o;
+              codes_f16(w8.x, o.x, o.y);
+              codes_f16(w8.y, o.z, o.w);
+              *reinterpret_cast<uint4*>(dst) = o;
             }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[warp * ns + st]);  // the raw stage may be refilled
         sbase = smem_u32(staging);
       }
-      const int tok0 = t0 + (warp + k * NW) * kTile;
-      const int n = min(kTile, t1 - tok0);
       if (owns_new && tok0 <= Lb && Lb < tok0 + kTile) {
         // This tile holds the new token, whose cache rows were not written yet when the tile
         // was fetched: put the projected rows (key row from the prologue, value row from
@@ -715,8 +775,8 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
               for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
                 for (int j = 0; j < NB; ++j) {
-                  if (g0 + u == 0) mma_bf16_z(c[mt][j], kf[u][mt], qf[0][j][0], qf[0][j][1]);
-                  else mma_bf16(c[mt][j], kf[u][mt], qf[g0 + u][j][0], qf[g0 + u][j][1]);
+                  if (g0 + u == 0) mma_op_z<Q8>(c[mt][j], kf[u][mt], qf[0][j][0], qf[0][j][1]);
+                  else mma_op<Q8>(c[mt][j], kf[u][mt], qf[g0 + u][j][0], qf[g0 + u][j][1]);
                 }
             }
         }
@@ -754,6 +814,12 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
         for (int e = 0; e < 4; ++e)
           s[mt][e] = NB == 1 ? c[mt][0][e] + __shfl_xor_sync(kFull, c[mt][0][e], 2)
                              : c[mt][0][e] + c[mt][NB - 1][e];
+      if (Q8) {  // scores of code rows times the rows' key scales
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) s[mt][e] *= scw[16 * mt + (lane >> 2) + 8 * (e >> 1)];
+      }
       if (n < kTile) {  // missing tokens take no weight
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt)
@@ -815,8 +881,11 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
         const float pA = ex2(s[mt][e0] - uA), pB = ex2(s[mt][e0 + 1] - uB);
         pa_sum += pA;
         pb_sum += pB;
-        const uint32_t hw = hi_pair(pA, pB);
-        const uint32_t lw = lo_pair(pA, pB, hw);
+        // int8 caches: the weights of code rows carry the rows' value scales (not in l)
+        const float sv = Q8 ? scw[kTile + 16 * mt + (lane >> 2) + 8 * (r & 1)] : 1.f;
+        const float wA = pA * sv, wB = pB * sv;
+        const uint32_t hw = Q8 ? hi_pair_h(wA, wB) : hi_pair(wA, wB);
+        const uint32_t lw = Q8 ? lo_pair_h(wA, wB, hw) : lo_pair(wA, wB, hw);
         if constexpr (NB == 1) {
           pb[0][r] = movm_t(lo_lane ? lw : hw);
         } else {
@@ -839,7 +908,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
               for (int kk = 0; kk < MT; ++kk)
 #pragma unroll
                 for (int j = 0; j < NB; ++j)
-                  mma_bf16(oacc[g0 + u][j], vf[u][kk], pb[j][2 * kk], pb[j][2 * kk + 1]);
+                  mma_op<Q8>(oacc[g0 + u][j], vf[u][kk], pb[j][2 * kk], pb[j][2 * kk + 1]);
             }
         }
       __syncwarp();
