@@ -33,6 +33,14 @@
 // otherwise it stores the latent partial state (o~, m, l) and takes a ticket: the last
 // CTA of the unit merges the splits, up-projects once and resets the ticket counter,
 // so the workspace counters stay zero between calls.
+//
+// Modes (compile-time, one instantiation each): the contiguous bf16 cache; the latent
+// decode (q~ given, o~ returned: no base loads, projections or up-projection, for bases
+// folded into the attention weights); paged caches (tiles addressed through a block
+// table); int8 caches (code boxes and row scales copied raw; each warp turns its codes into
+// exact fp16 in a padded row-major tile and the MMAs take fp16 operands, the row scales
+// multiplying the scores and the softmax weights).  Grids of more than one wave run two
+// CTAs per SM with a smaller ring.
 #include <cfloat>
 #include <cmath>
 #include <cstdint>
