@@ -367,6 +367,17 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
   if (tid == 0) {
     for (int i = 0; i < 2 * NW * ns + 2; ++i) mbar_init(&full[i], 1);
     fence_barrier_init();
+    if (!LAT) {
+      // P_K is requested before the dependency wait (its latency then overlaps the preceding
+      // kernel's tail): a weight, which the calls document the preceding kernel must not
+      // write.  Its bytes are added to the setup barrier's phase; q arrives after the wait.
+      asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(setup_bar)),
+                   "r"(2u * d * rK) : "memory");
+      const uint64_t keep = l2_policy_evict_last();
+      for (int p = 0; p < a.ppk.n; ++p)
+        tma_load_2d(pmat + a.ppk.p[p].smem_off, &a.maps[a.ppk.p[p].map], a.ppk.p[p].x, kvh * d,
+                    setup_bar, keep);
+    }
   }
   __syncthreads();
   // inputs may come from the preceding kernel in the stream: read nothing before this
@@ -474,18 +485,16 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
       mbar_arrive_expect_tx(setup_bar, 2u * gcount * rK);
       bulk_g2s(smem + L.qraw, a.q + ((size_t)b * a.Hq + h0) * rK, 2u * gcount * rK, setup_bar);
     } else if (lane == 0) {
-      // q and P_K first (they gate q~), then every warp's ring
+      // q (and, for the fused step, the new rows) first: they gate q~; then every warp's ring
       const uint64_t keep = l2_policy_evict_last();  // bases are shared by many CTAs
-      mbar_arrive_expect_tx(setup_bar, 2u * d * rK + 2u * gcount * d + (owns_new ? 4u * d : 0u));
+      mbar_arrive_expect_tx(setup_bar, 2u * gcount * d + (owns_new ? 4u * d : 0u));
       bulk_g2s(smem + L.qraw, a.q + ((size_t)b * a.Hq + h0) * d, 2u * gcount * d, setup_bar);
       if (owns_new) {
         const size_t row = ((size_t)b * a.Hkv + kvh) * d;
         bulk_g2s(smem + L.newraw, a.k_new + row, 2u * d, setup_bar);
         bulk_g2s(smem + L.newraw + 2u * d, a.v_new + row, 2u * d, setup_bar);
       }
-      for (int p = 0; p < a.ppk.n; ++p)
-        tma_load_2d(pmat + a.ppk.p[p].smem_off, &a.maps[a.ppk.p[p].map], a.ppk.p[p].x, kvh * d,
-                    setup_bar, keep);
+      (void)keep;  // P_K was requested before the dependency wait
     }
     __syncwarp();
     if (lane < NW) {  // lane w requests consumer warp w's tiles

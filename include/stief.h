@@ -179,7 +179,13 @@ STIEF_API size_t stief_decode_workspace_bytes(int B, int Hq, int Hkv, int rV, in
  * up-projection over its token range; the last CTA of each (sequence, KV head,
  * sub-group) to finish merges the splits (log-sum-exp).  The kernel is launched
  * as a programmatic dependent of the preceding work in the stream: it may be
- * scheduled while that work drains but reads no input before it has completed.
+ * scheduled while that work drains and reads no input before it has completed,
+ * except P_K, which it requests first so that its latency overlaps that work: P_K
+ * must not be written by the kernel that immediately precedes the call in the
+ * stream if that kernel lets its dependents start early (programmatic dependent
+ * launch).  This library's kernels never write the bases.  The same holds for the
+ * other calls that take P_K (stief_append_decode and the _noalloc, _paged and _q8
+ * decodes).
  * Returns STIEF_OK or an argument error (nothing launched).
  */
 STIEF_API stief_status stief_decode_attention(const uint16_t* q, const uint16_t* P_K,
