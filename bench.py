@@ -168,12 +168,13 @@ def build_state(w: si.Workload, total_steps: int, seed: int, dev):
     return layers, L_max
 
 
-def replica_count(w: si.Workload) -> int:
+def replica_count(w: si.Workload, int8: bool = False) -> int:
     """Copies of the workload's layer state that consecutive timed steps rotate over, so that
     the inputs of a step were last touched at least ROTATE_BYTES of cache reads earlier
     (more than 3x the 126 MB L2: every step streams its cache from HBM, and no flush is
     needed between steps)."""
-    per = sum(2 * (rK + rV) * w.B * w.Hkv * w.L for rK, rV in w.layer_ranks())
+    per = sum(((rK + rV + 8) if int8 else 2 * (rK + rV)) * w.B * w.Hkv * w.L
+              for rK, rV in w.layer_ranks())
     return 1 if per >= ROTATE_BYTES else min(MAX_REPLICAS, -(-ROTATE_BYTES // per))
 
 
@@ -195,7 +196,7 @@ def run_gpu(args, w: si.Workload):
                                              device_id=dev)
     seed = w.seed + 7919 * rank
     W, K = args.warmup, args.steps
-    R = replica_count(w)
+    R = replica_count(w, args.int8)
     reps = []
     for r in range(R):
         # room for every append of the warm-up, timed and kernel-timing runs of a replica
@@ -213,11 +214,28 @@ def run_gpu(args, w: si.Workload):
     # latent mode (bases folded into the attention weights): q~ in, o~ out, per layer
     qlat_s = [torch.randn((w.B, w.Hq, lay.rK), generator=g, device=dev).to(torch.bfloat16)
               for lay in layers] if args.latent else []
+    # int8 mode: every replica's layer caches as int8 codes and fp32 row scales (synthetic:
+    # the decode's cost does not depend on the values); L_max a multiple of 64
+    if args.int8:
+        for lays in reps:
+            for lay in lays:
+                L8 = (L_max + 63) // 64 * 64
+                lay.kq = torch.randint(-127, 128, (w.B, w.Hkv, L8, lay.rK), generator=g,
+                                       device=dev, dtype=torch.int8)
+                lay.vq = torch.randint(-127, 128, (w.B, w.Hkv, L8, lay.rV), generator=g,
+                                       device=dev, dtype=torch.int8)
+                lay.ks = torch.rand((w.B, w.Hkv, L8), generator=g, device=dev) * 0.02
+                lay.vs = torch.rand((w.B, w.Hkv, L8), generator=g, device=dev) * 0.02
+                lay.k_lat = lay.v_lat = None  # the bf16 caches are not used
     olat = [torch.empty((w.B, w.Hq, lay.rV), dtype=torch.bfloat16, device=dev)
             for lay in layers] if args.latent else []
 
     def layer_step(li, lay):
-        if args.latent:  # attention in the latent space only (no projections, no append)
+        if args.int8:  # decode over the int8 cache (no append)
+            stief.stief_decode_attention_q8(q_s, lay.P_K, lay.P_V, lay.kq, lay.vq, lay.ks, lay.vs,
+                                            lay.seq_lens, out[li], lay.ws, max_seq_len=L_max,
+                                            num_splits=args.splits, dev_status=status)
+        elif args.latent:  # attention in the latent space only (no projections, no append)
             stief.stief_decode_latent(qlat_s[li], lay.k_lat, lay.v_lat, lay.seq_lens, olat[li],
                                       lay.ws, max_seq_len=L_max, num_splits=args.splits,
                                       dev_status=status)
@@ -239,7 +257,7 @@ def run_gpu(args, w: si.Workload):
     def decode_only(lays):
         """One launch of the step's attention kernel on layer 0 (for the kernel's own timing)."""
         lay = lays[0]
-        if args.unfused and not args.latent:
+        if args.unfused and not args.latent and not args.int8:
             stief.stief_decode_attention(q_s, lay.P_K, lay.P_V, lay.k_lat, lay.v_lat,
                                          lay.seq_lens, out[0], lay.ws, max_seq_len=L_max,
                                          num_splits=args.splits, dev_status=status)
@@ -247,7 +265,7 @@ def run_gpu(args, w: si.Workload):
             layer_step(0, lay)
 
     def reset_lengths(L0):
-        if args.latent:  # nothing is appended: every step attends over the full context
+        if args.latent or args.int8:  # nothing is appended: every step attends over the full context
             L0 = w.L
         for lays in reps:
             for lay in lays:
@@ -307,9 +325,12 @@ def run_gpu(args, w: si.Workload):
         with torch.cuda.graph(warm_graph, stream=cap):
             for i in range(n_dec):
                 lay = reps[i % R][0]
-                stief.stief_decode_attention(q_s, lay.P_K, lay.P_V, lay.k_lat, lay.v_lat,
-                                             lay.seq_lens, out[0], lay.ws, max_seq_len=L_max,
-                                             dev_status=status)
+                if args.int8:
+                    layer_step(0, lay)
+                else:
+                    stief.stief_decode_attention(q_s, lay.P_K, lay.P_V, lay.k_lat, lay.v_lat,
+                                                 lay.seq_lens, out[0], lay.ws, max_seq_len=L_max,
+                                                 dev_status=status)
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
 
@@ -357,7 +378,7 @@ def run_gpu(args, w: si.Workload):
     # ---- decode kernel timing for the roofline: runs of n_dec back-to-back launches
     # (replicas rotating), averaged over the timed region; plus single launches.  The fused
     # kernel appends a token per launch: lengths restart at L_dec - 1 for each run.
-    appends = not (args.unfused or args.latent)  # the step's kernel appends a token
+    appends = not (args.unfused or args.latent or args.int8)  # the step's kernel appends a token
     L_run0 = L_dec - (1 if appends else 0)
     reset_lengths(L_run0)
     dec_reps = max(3, args.decode_iters // n_dec)
@@ -424,12 +445,13 @@ def run_gpu(args, w: si.Workload):
     tokens_per_step = w.B * ws_n
     value = tokens_per_step / (ms_per_step / 1e3)
     lay0 = layers[0]
-    bytes_per_dec = int(2 * (lay0.rK + lay0.rV) * w.B * w.Hkv * L_dec_mean)
+    row_bytes = (lambda rK, rV: rK + rV + 8) if args.int8 else (lambda rK, rV: 2 * (rK + rV))
+    bytes_per_dec = int(row_bytes(lay0.rK, lay0.rV) * w.B * w.Hkv * L_dec_mean)
     achieved = bytes_per_dec / (dec_us / 1e6) / 1e9
     peak, peak_kind = _hbm_peak()
-    step_bytes = sum(2 * (lay.rK + lay.rV) * w.B * w.Hkv for lay in layers) * (
+    step_bytes = sum(row_bytes(lay.rK, lay.rV) * w.B * w.Hkv for lay in layers) * (
         (ctx_first + ctx_last) / 2)
-    rot_mb = R * sum(2 * (rK + rV) * w.B * w.Hkv * w.L for rK, rV in w.layer_ranks()) / 2**20
+    rot_mb = R * sum(row_bytes(rK, rV) * w.B * w.Hkv * w.L for rK, rV in w.layer_ranks()) / 2**20
     result = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -441,22 +463,25 @@ def run_gpu(args, w: si.Workload):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": "int8" if args.int8 else "bf16",
         "data": "synthetic",
         "config": {
             "workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "context": w.L,
             "layers": len(layers), "ranks": [list(r) for r in w.layer_ranks()][:4]
             + (["..."] if len(layers) > 4 else []),
-            "step": (("latent decode only (bases folded into the attention weights: q~ in, "
+            "step": (("decode over an int8 latent cache (codes + fp32 row scales, synthetic "
+                      "values), no append, every layer; " if args.int8 else
+                      "latent decode only (bases folded into the attention weights: q~ in, "
                       "o~ out; the new token's latent rows would come from the folded K/V "
                       "projection), every layer; " if args.latent else
                       "append 1 token per (sequence, KV head) + decode, every layer; ") +
                      "the API calls captured in CUDA graphs (one step per replica, the timed "
                      "region replays the replica cycle back to back); " +
-                     ("stief_decode_latent (1 kernel per layer)" if args.latent else
+                     ("stief_decode_attention_q8 (1 kernel per layer)" if args.int8 else
+                      "stief_decode_latent (1 kernel per layer)" if args.latent else
                       "stief_compress_append + stief_decode_attention (3 kernels per layer)"
                       if args.unfused else "stief_append_decode (1 kernel per layer)")),
-            "context_growth": (f"none (context {w.L} every step)" if args.latent else
+            "context_growth": (f"none (context {w.L} every step)" if args.latent or args.int8 else
                                f"+1 token per step of a replica (contexts {ctx_first}..{ctx_last})"),
             "l2": (f"no flush: steps rotate over {R} copies of the layer caches "
                    f"({rot_mb:.0f} MiB in all, > 3x the 126 MB L2)" if R > 1 else
@@ -467,7 +492,8 @@ def run_gpu(args, w: si.Workload):
         },
         "hbm_gbs_step": round(step_bytes / (ms_per_step / 1e3) / 1e9, 1),
         "roofline": {
-            "kernel": "stief_decode_kernel (" + ("stief_decode_latent" if args.latent else
+            "kernel": "stief_decode_kernel (" + ("stief_decode_attention_q8" if args.int8 else
+                                                 "stief_decode_latent" if args.latent else
                                                  "stief_decode_attention" if args.unfused
                                                  else "stief_append_decode") + ")",
             "bound": "hbm",
@@ -476,7 +502,7 @@ def run_gpu(args, w: si.Workload):
             "peak_kind": f"{peak_kind} hbm_gbs (copy bandwidth, burst)",
             "unit": "GB/s",
             "frac": round(achieved / peak, 4),
-            "traffic": None if (args.latent or args.unfused) else _traffic_per_launch(w.name),
+            "traffic": None if (args.latent or args.unfused or args.int8) else _traffic_per_launch(w.name),
             "algorithmic_bytes": bytes_per_dec,
             "decode_us": round(dec_us, 3),
             "decode_timing": f"{dec_reps} replays of a graph of {n_dec} back-to-back decode "
@@ -494,7 +520,7 @@ def run_gpu(args, w: si.Workload):
     }
     if compress is not None:
         result["compress"] = compress
-    if rank == 0 and ws_n == 1 and not args.no_cpu_baseline and not args.latent:
+    if rank == 0 and ws_n == 1 and not args.no_cpu_baseline and not args.latent and not args.int8:
         result["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     if ws_n > 1:
         torch.distributed.destroy_process_group()
@@ -716,6 +742,8 @@ def main():
                     help="diagnostics: run only the first N layers of the workload")
     ap.add_argument("--splits", type=int, default=0,
                     help="diagnostics: force the decode split count (0 = automatic)")
+    ap.add_argument("--int8", action="store_true",
+                    help="time stief_decode_attention_q8 over an int8 latent cache (no append)")
     ap.add_argument("--latent", action="store_true",
                     help="time stief_decode_latent (bases folded into the attention weights) "
                          "instead of the fused append + decode step")

@@ -197,3 +197,23 @@ def test_paged_append_into_unmapped_page_is_refused():
                                     dev_status=status)
     assert stief.stief_read_device_status(status) & stief.DEV_CAPACITY_OVERFLOW
     assert lens_t.item() == 64
+
+
+def test_paged_decode_multi_wave_grid():
+    """More units than SMs (40 x 8 = 320): the paged decode in the two-CTAs-per-SM plan."""
+    rng = np.random.default_rng(13)
+    B, Hq, Hkv, rK, rV, page_size, max_pages = 40, 32, 8, 64, 64, 64, 5
+    Lc = page_size * max_pages
+    lens = rng.integers(1, Lc, size=B).tolist()
+    lens[2] = 0
+    q = si.queries(5800, B, Hq, 128)
+    P_K, P_V = si.bases_bf16(5800, Hkv, 128, rK, rV)
+    kpool, vpool, table = _pools(B, Hkv, rK, rV, page_size, max_pages, 4, rng)
+    kc = si.latent_cache(5801, B, Hkv, Lc, rK, 0)
+    vc = si.latent_cache(5801, B, Hkv, Lc, rV, 1)
+    _fill_pages(kpool, table, kc, page_size, [Lc] * B)
+    _fill_pages(vpool, table, vc, page_size, [Lc] * B)
+    got = _run_paged_decode(q, P_K, P_V, kpool, vpool, table, lens, Lc)
+    want = oracle.decode(f64(q), f64(P_K), f64(P_V), oracle.gather_pages(f64(kpool), table, lens, Lc),
+                         oracle.gather_pages(f64(vpool), table, lens, Lc), np.asarray(lens, np.int32))
+    assert_decode_close(got, want)

@@ -152,3 +152,21 @@ def test_decode_q8_full_size(name):
     want = oracle.decode(f64(q), f64(P_K), f64(P_V), oracle.dequantize_rows(kq.numpy(), ks.numpy()),
                          oracle.dequantize_rows(vq.numpy(), vs.numpy()), np.full(w.B, w.L, np.int32))
     assert_decode_close(got, want)
+
+
+def test_decode_q8_multi_wave_grid():
+    """More units than SMs (40 x 8 = 320): the int8 decode in the two-CTAs-per-SM plan."""
+    B, Hq, Hkv, rK, rV, L = 40, 32, 8, 64, 64, 320
+    rng = np.random.default_rng(6400)
+    lens = rng.integers(1, L, size=B).tolist()
+    lens[5] = 0
+    lens[9] = L
+    q = si.queries(6400, B, Hq, 128)
+    P_K, P_V = si.bases_bf16(6400, Hkv, 128, rK, rV)
+    kq, ks = _random_q8_cache(6401, B, Hkv, L, rK)
+    vq, vs = _random_q8_cache(6402, B, Hkv, L, rV)
+    got = _decode_q8(q, P_K, P_V, kq, vq, ks, vs, lens, L)
+    want = oracle.decode(f64(q), f64(P_K), f64(P_V), oracle.dequantize_rows(kq.numpy(), ks.numpy()),
+                         oracle.dequantize_rows(vq.numpy(), vs.numpy()), np.asarray(lens, np.int32))
+    assert_decode_close(got, want)
+    assert torch.all(got[5].float() == 0)
