@@ -670,10 +670,9 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
     uint8_t* staging = smem + L.region + (size_t)warp * L.q8_tile;  // int8 caches only
     const uint32_t sK = 2u * rK + 16u, sV = 2u * rV + 16u;  // its row strides
     const uint32_t q8_kt = (uint32_t)kTile * sK;            // its value rows' offset
-    // int8 caches: in the dequantise pass a lane takes one 8-column chunk of each matrix and
-    // every (32 / chunks per row)-th row of it (no division per item); its chunk's place in
-    // the swizzled bf16 tile is fixed
-    const int kcpr = rK >> 3, vcpr = rV >> 3;  // 8-column chunks per row
+    // int8 caches: in the conversion pass a lane takes one 16-column chunk of each matrix
+    // and every (32 / chunks per row)-th row of it (no division per item)
+    const int kcpr = rK >> 4, vcpr = rV >> 4;  // 16-column chunks per row
     const int krpp = 32 / kcpr, vrpp = 32 / vcpr;  // rows per pass
     const bool klive = lane < krpp * kcpr, vlive = lane < vrpp * vcpr;
     const int kc0 = lane % kcpr, vc0 = lane % vcpr;
@@ -728,21 +727,24 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
           scw[i] = (i < kTile ? i : i - kTile) < n ? scr[i] : 0.f;
         for (int m = 0; m < 2; ++m) {
           const int r = m ? rV : rK;
-          const int8_t* codes = reinterpret_cast<const int8_t*>(raw + (m ? L.q8_v : 0u)) + 8 * (m ? vc0 : kc0);
+          const int8_t* codes = reinterpret_cast<const int8_t*>(raw + (m ? L.q8_v : 0u)) + 16 * (m ? vc0 : kc0);
           const uint32_t stride = m ? sV : sK;
           const int rpp = m ? vrpp : krpp;
           const int t0 = m ? vt0 : kt0;
-          uint8_t* dst = staging + (m ? q8_kt : 0u) + (uint32_t)t0 * stride + 16u * (uint32_t)(m ? vc0 : kc0);
+          uint8_t* dst = staging + (m ? q8_kt : 0u) + (uint32_t)t0 * stride + 32u * (uint32_t)(m ? vc0 : kc0);
           const int8_t* src = codes + t0 * r;
           const uint32_t dstep = (uint32_t)rpp * stride;
           const int sstep = rpp * r;
           if (m ? vlive : klive)
             for (int t = t0; t < kTile; t += rpp, dst += dstep, src += sstep) {
-              const uint2 w8 = *reinterpret_cast<const uint2*>(src);
-              uint4 o;
-              codes_f16(w8.x, o.x, o.y);
-              codes_f16(w8.y, o.z, o.w);
-              *reinterpret_cast<uint4*>(dst) = o;
+              const uint4 w16 = *reinterpret_cast<const uint4*>(src);
+              uint4 o0, o1;
+              codes_f16(w16.x, o0.x, o0.y);
+              codes_f16(w16.y, o0.z, o0.w);
+              codes_f16(w16.z, o1.x, o1.y);
+              codes_f16(w16.w, o1.z, o1.w);
+              reinterpret_cast<uint4*>(dst)[0] = o0;
+              reinterpret_cast<uint4*>(dst)[1] = o1;
             }
         }
         __syncwarp();
