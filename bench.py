@@ -50,6 +50,29 @@ def _dist_env():
     return ws, rank, local
 
 
+def rank_seed(base: int, rank: int) -> int:
+    """Each rank decodes its own independent sequences (weak scaling: the (sequence, KV head)
+    units shard with no exchange), drawn from a rank-specific seed."""
+    return base + 7919 * rank
+
+
+def reduce_over_ranks(values, device=None):
+    """Per-rank timings -> their maximum over the ranks (the job ends with its slowest rank);
+    the identity without a process group."""
+    if not torch.distributed.is_available() or not torch.distributed.is_initialized() \
+            or torch.distributed.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def job_tokens_per_s(tokens_per_rank_step: int, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput: the tokens every rank decodes per step over the slowest rank's
+    step time."""
+    return tokens_per_rank_step * world / (ms_per_step / 1e3)
+
+
 def _hbm_peak():
     try:
         with open(PEAKS_FILE) as f:
@@ -194,7 +217,7 @@ def run_gpu(args, w: si.Workload):
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=dev)
-    seed = w.seed + 7919 * rank
+    seed = rank_seed(w.seed, rank)
     W, K = args.warmup, args.steps
     R = replica_count(w, args.int8)
     reps = []
@@ -429,10 +452,7 @@ def run_gpu(args, w: si.Workload):
     if st != 0:
         raise RuntimeError(f"device status {st:#x} after the e2e steps")
 
-    if ws_n > 1:
-        t = torch.tensor([ms_per_step, e2e_ms, dec_us], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_per_step, e2e_ms, dec_us = (float(x) for x in t.tolist())
+    ms_per_step, e2e_ms, dec_us = reduce_over_ranks([ms_per_step, e2e_ms, dec_us], dev)
     del step_graphs, e2e_graphs, dec_graph, warm_graph, cycle_graph
 
     # ---- prefill compress (the prefill + batched decode workload): one 4096-token chunk
@@ -442,8 +462,7 @@ def run_gpu(args, w: si.Workload):
         compress = time_prefill_compress(args, len(layers), dev, stream)
 
     # ---- numbers
-    tokens_per_step = w.B * ws_n
-    value = tokens_per_step / (ms_per_step / 1e3)
+    value = job_tokens_per_s(w.B, ws_n, ms_per_step)
     lay0 = layers[0]
     row_bytes = (lambda rK, rV: rK + rV + 8) if args.int8 else (lambda rK, rV: 2 * (rK + rV))
     bytes_per_dec = int(row_bytes(lay0.rK, lay0.rV) * w.B * w.Hkv * L_dec_mean)
@@ -510,7 +529,7 @@ def run_gpu(args, w: si.Workload):
             "decode_us_single_launch": round(dec_us_iso, 3),
             "frac_single_launch": round(bytes_per_dec / (dec_us_iso / 1e6) / 1e9 / peak, 4),
         },
-        "e2e": {"value": round(tokens_per_step / (e2e_ms / 1e3), 2), "unit": "tokens/s",
+        "e2e": {"value": round(job_tokens_per_s(w.B, ws_n, e2e_ms), 2), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "how": "per step one CUDA-graph replay of the public API calls with the "
                        "pinned host copies (inputs H2D, outputs D2H) inside"},
