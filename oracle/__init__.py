@@ -178,6 +178,97 @@ class Oracle:
             raise ValueError("decode_latent: a sequence length is outside [0, L_max]")
         return out
 
+    # ------------------------------------------------------------------ joint value latent
+    #
+    # STAR-KV technical summary, "Metodologia" item 2 (hybrid decomposition): the keys keep
+    # one basis per KV head, the values of all KV heads are factored together.  The joint
+    # value basis P_VJ is [Hkv*d][rV] over the concatenation v_cat = [v_0 | v_1 | ... ] of a
+    # token's KV-head value rows, and the cache stores one value latent per token,
+    # v_joint = v_cat . P_VJ, shared by every head.  Reconstruction gives the whole
+    # concatenation back, v_cat~ = v_joint . P_VJ^T, and KV head g reads its own block of d
+    # coordinates, [g*d, (g+1)*d).  The three helpers below are that layout and nothing else;
+    # every product runs in the C functions above.
+
+    @staticmethod
+    def _concat_heads(x):
+        """[Hkv][T][d] -> [T][Hkv*d]: a token's KV-head rows side by side, head 0 first."""
+        Hkv, T, d = x.shape
+        return np.ascontiguousarray(np.transpose(x, (1, 0, 2)).reshape(T, Hkv * d))
+
+    @staticmethod
+    def _head_blocks(P_VJ, Hkv):
+        """[Hkv*d][rV] -> [Hkv][d][rV]: block g holds rows [g*d, (g+1)*d) of P_VJ, the part of
+        the reconstruction that lands in KV head g's coordinates."""
+        HD, rV = P_VJ.shape
+        return np.ascontiguousarray(P_VJ.reshape(Hkv, HD // Hkv, rV))
+
+    @staticmethod
+    def _share_values(v_joint, Hkv):
+        """[B][L][rV] -> [B][Hkv][L][rV]: the one value latent of a token, seen by each head."""
+        B, L, rV = v_joint.shape
+        return np.ascontiguousarray(np.broadcast_to(v_joint[:, None], (B, Hkv, L, rV)))
+
+    def compress_append_joint_v(self, k_new, v_new, P_K, P_VJ, k_lat, v_joint, seq_lens,
+                                round_to_bf16: bool = True):
+        """Append T tokens per sequence: keys per KV head (k_lat[b][g] gets k_new[b][g] . P_K[g]),
+        values jointly (v_joint[b] gets concat_g(v_new[b][g]) . P_VJ), both bf16-rounded like
+        the per-head cache.  A sequence whose rows would pass L_max is left untouched and
+        counted.
+
+        Shapes: k_new/v_new [B][Hkv][T][d], P_K [Hkv][d][rK], P_VJ [Hkv*d][rV],
+        k_lat [B][Hkv][L_max][rK], v_joint [B][L_max][rV], seq_lens [B].
+        Returns updated copies (k_lat, v_joint, seq_lens, n_overflow).
+        """
+        k_new, v_new, P_K, P_VJ = map(_f64, (k_new, v_new, P_K, P_VJ))
+        k_lat = _f64(k_lat).copy()
+        v_joint = _f64(v_joint).copy()
+        lens = np.asarray(seq_lens, dtype=np.int32).copy()
+        B, Hkv, T, d = k_new.shape
+        L_max = k_lat.shape[2]
+        if v_new.shape != k_new.shape or P_K.shape[:2] != (Hkv, d) or P_VJ.shape[0] != Hkv * d:
+            raise ValueError("compress_append_joint_v: inconsistent shapes")
+        if k_lat.shape[:2] != (B, Hkv) or v_joint.shape[:2] != (B, L_max):
+            raise ValueError("compress_append_joint_v: inconsistent cache shapes")
+        n_bad = 0
+        for b in range(B):
+            L = int(lens[b])
+            if L < 0 or L + T > L_max:
+                n_bad += 1
+                continue
+            for g in range(Hkv):
+                k_lat[b, g, L:L + T] = self.project(k_new[b, g], P_K[g], round_to_bf16)
+            v_joint[b, L:L + T] = self.project(self._concat_heads(v_new[b]), P_VJ, round_to_bf16)
+            lens[b] = L + T
+        return k_lat, v_joint, lens, n_bad
+
+    def decode_joint_v(self, q, P_K, P_VJ, k_lat, v_joint, seq_lens,
+                       num_threads: int = 0) -> np.ndarray:
+        """One decode step with per-head keys and a joint value latent; returns [B][Hq][d].
+
+        Query head h of KV head g: scores against K_down[g] . P_K[g]^T as in decode(); its
+        values are block g of v_joint[t] . P_VJ^T.  That is decode() with P_V[g] = block g of
+        P_VJ and every head reading the shared value latent.
+        Shapes: q [B][Hq][d], P_K [Hkv][d][rK], P_VJ [Hkv*d][rV], k_lat [B][Hkv][L_max][rK],
+        v_joint [B][L_max][rV], seq_lens [B].
+        """
+        P_K, P_VJ, v_joint = map(_f64, (P_K, P_VJ, v_joint))
+        Hkv = P_K.shape[0]
+        if P_VJ.shape[0] != Hkv * P_K.shape[1] or v_joint.ndim != 3:
+            raise ValueError("decode_joint_v: inconsistent shapes")
+        return self.decode(q, P_K, self._head_blocks(P_VJ, Hkv), k_lat,
+                           self._share_values(v_joint, Hkv), seq_lens, num_threads)
+
+    def decode_latent_joint_v(self, q_lat, k_lat, v_joint, seq_lens, d: int = 128,
+                              num_threads: int = 0) -> np.ndarray:
+        """Latent-space decode with a joint value latent (bases folded into the weights; the
+        output projection absorbs block g of P_VJ); returns o~ [B][Hq][rV].
+
+        Shapes: q_lat [B][Hq][rK], k_lat [B][Hkv][L_max][rK], v_joint [B][L_max][rV].
+        """
+        k_lat, v_joint = _f64(k_lat), _f64(v_joint)
+        return self.decode_latent(q_lat, k_lat, self._share_values(v_joint, k_lat.shape[1]),
+                                  seq_lens, d, num_threads)
+
 def default() -> Oracle:
     """The oracle built from stief_oracle.c (compiled on first use)."""
     global _lib
@@ -257,3 +348,18 @@ def dequantize_rows(codes, scales) -> np.ndarray:
     """code * scale per element, exact in fp64."""
     return np.asarray(codes, np.float64) * np.asarray(scales, np.float64)[..., None]
 
+
+
+def compress_append_joint_v(k_new, v_new, P_K, P_VJ, k_lat, v_joint, seq_lens,
+                            round_to_bf16: bool = True):
+    return default().compress_append_joint_v(k_new, v_new, P_K, P_VJ, k_lat, v_joint, seq_lens,
+                                             round_to_bf16)
+
+
+def decode_joint_v(q, P_K, P_VJ, k_lat, v_joint, seq_lens, num_threads: int = 0) -> np.ndarray:
+    return default().decode_joint_v(q, P_K, P_VJ, k_lat, v_joint, seq_lens, num_threads)
+
+
+def decode_latent_joint_v(q_lat, k_lat, v_joint, seq_lens, d: int = 128,
+                          num_threads: int = 0) -> np.ndarray:
+    return default().decode_latent_joint_v(q_lat, k_lat, v_joint, seq_lens, d, num_threads)

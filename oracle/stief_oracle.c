@@ -20,7 +20,7 @@
  *   - attention itself is ordinary softmax attention over the reconstructed
  *     keys and values.
  *
- * Readings taken where the pages are silent (each listed in the design doc):
+ * Readings taken where the pages are silent:
  *   - one basis pair per KV head, stored [Hkv][d][r];
  *   - scores scaled by 1/sqrt(d) with d the full head dimension;
  *   - grouped-query attention with contiguous groups, query head h reads KV

@@ -11,8 +11,10 @@ Stiefel manifold", StiefAttention technical summary, "Mecanismo Central" /
 "Kernmechanismus": item 2 (orthonormal bases on the Stiefel manifold), item 3
 (QR orthonormalisation; R is only a change of coordinates inside the subspace),
 item 5 (stored K_down = K P_K, reconstruction K~ = K_down P_K^T before
-attention; the bases may be folded into the attention weights); "Resultados Experimentais" (the uncompressed FP16 baseline, i.e.
-plain attention, which the r = d case must reproduce).
+attention; the bases may be folded into the attention weights); "Resultados Experimentais"
+(the uncompressed FP16 baseline, i.e. plain attention, which the r = d case must reproduce).
+STAR-KV technical summary, "Metodologia" item 2 (values decomposed jointly over the heads,
+keys per head) for the joint-value calls.
 """
 from __future__ import annotations
 
@@ -385,6 +387,138 @@ def check_compress_append_bookkeeping(o, r: int = 32, d: int = 128) -> None:
             assert np.all(vl[b, h, keep] == -canary)
 
 
+# ----------------------------------------------------------------------------- joint value latent
+#
+# STAR-KV technical summary, "Metodologia" item 2: values decomposed jointly over the
+# concatenated heads, keys per head; the value reconstruction is absorbed into the output
+# projection.  The oracle's joint-value calls are layout over decode / decode_latent / project;
+# these pins fix the layout (concatenation order, the block of P_VJ each head reads, the shared
+# latent) against plain attention and against the per-head form.
+
+def _block_diag(P):
+    """[Hkv][d][r] -> the (Hkv*d) x (Hkv*r) block-diagonal matrix with block g = P[g]."""
+    Hkv, d, r = P.shape
+    out = np.zeros((Hkv * d, Hkv * r))
+    for g in range(Hkv):
+        out[g * d:(g + 1) * d, g * r:(g + 1) * r] = P[g]
+    return out
+
+
+def check_joint_v_full_rank_is_plain_attention(o, d: int = 32, tol: float = 1e-12) -> None:
+    """rK = d and rV = Hkv*d: both reconstructions are exact, so compress-then-decode with a
+    joint value basis is plain attention on the original rows (torch SDPA, float64).  A
+    concatenation order that differs between compression and reconstruction fails here."""
+    B, Hq, Hkv, L_max, T = 2, 6, 3, 24, 24
+    lens = np.array([24, 7], dtype=np.int32)
+    rng = np.random.default_rng(23)
+    K = rng.standard_normal((B, Hkv, T, d))
+    V = rng.standard_normal((B, Hkv, T, d))
+    q = rng.standard_normal((B, Hq, d))
+    P_K = si.bases(24, Hkv, d, d)
+    P_VJ = si.bases(25, 1, Hkv * d, Hkv * d)[0]
+    k_lat, v_joint, new_lens, nbad = o.compress_append_joint_v(
+        K, V, P_K, P_VJ, np.zeros((B, Hkv, L_max, d)), np.zeros((B, L_max, Hkv * d)),
+        np.zeros(B, np.int32), round_to_bf16=False)
+    assert nbad == 0 and new_lens.tolist() == [T, T]
+    got = o.decode_joint_v(q, P_K, P_VJ, k_lat, v_joint, lens)
+    want = _sdpa_reference(q, K, V, lens)
+    assert np.all(np.isfinite(got)), "non-finite output"
+    err = _rel_err(got, want)
+    assert err <= tol, f"joint values at full rank differ from plain attention: {err}"
+
+
+def check_joint_v_block_diagonal_is_per_head(o, r: int = 16, d: int = 128) -> None:
+    """P_VJ = blockdiag(P_V[0], ..., P_V[Hkv-1]): the joint latent of a token is the per-head
+    latents side by side, and decode_joint_v equals the per-head decode over them (the
+    products with the zero blocks add exact zeros, so the caches agree bit for bit)."""
+    B, Hq, Hkv, L_max, T = 2, 8, 4, 12, 9
+    rng = np.random.default_rng(26)
+    k_new = si.bf16_to_f64(si.to_bf16(rng.standard_normal((B, Hkv, T, d))))
+    v_new = si.bf16_to_f64(si.to_bf16(rng.standard_normal((B, Hkv, T, d))))
+    P_K = si.bases(27, Hkv, d, 24)
+    P_V = si.bases(28, Hkv, d, r)
+    lens0 = np.array([0, 3], np.int32)
+    kj, vj, lj, _ = o.compress_append_joint_v(k_new, v_new, P_K, _block_diag(P_V),
+                                              np.zeros((B, Hkv, L_max, 24)),
+                                              np.zeros((B, L_max, Hkv * r)), lens0)
+    kp, vp, lp, _ = o.compress_append(k_new, v_new, P_K, P_V, np.zeros((B, Hkv, L_max, 24)),
+                                      np.zeros((B, Hkv, L_max, r)), lens0)
+    assert np.array_equal(lj, lp) and np.array_equal(kj, kp)
+    for g in range(Hkv):
+        assert np.array_equal(vj[:, :, g * r:(g + 1) * r], vp[:, g])
+    q = rng.standard_normal((B, Hq, d))
+    got = o.decode_joint_v(q, P_K, _block_diag(P_V), kj, vj, lj)
+    want = o.decode(q, P_K, P_V, kp, vp, lp)
+    assert _rel_err(got, want) <= 1e-14
+
+
+def check_joint_v_latent_folding(o, d: int = 64) -> None:
+    """Folding: decode_latent_joint_v(q P_K[g]) followed by block g of P_VJ equals
+    decode_joint_v(q) (associativity of the products)."""
+    rng = np.random.default_rng(29)
+    B, Hq, Hkv, L, rK, rV = 2, 8, 2, 21, 32, 40
+    q = rng.standard_normal((B, Hq, d))
+    P_K = si.bases(30, Hkv, d, rK)
+    P_VJ = si.bases(31, 1, Hkv * d, rV)[0]
+    k = rng.standard_normal((B, Hkv, L, rK))
+    v = rng.standard_normal((B, L, rV))
+    lens = np.array([L, 4], np.int32)
+    G = Hq // Hkv
+    q_lat = np.stack([np.stack([q[b, h] @ P_K[h // G] for h in range(Hq)]) for b in range(B)])
+    o_lat = o.decode_latent_joint_v(q_lat, k, v, lens, d=d)
+    blk = lambda g: P_VJ[g * d:(g + 1) * d]
+    got = np.stack([np.stack([blk(h // G) @ o_lat[b, h] for h in range(Hq)]) for b in range(B)])
+    want = o.decode_joint_v(q, P_K, P_VJ, k, v, lens)
+    assert _rel_err(got, want) <= 1e-12
+
+
+def check_joint_v_edges(o, d: int = 16) -> None:
+    """One token: every query head of KV head g returns block g of v_joint[0] . P_VJ^T (its
+    softmax weight is 1); the latent form returns v_joint[0] itself.  Length 0 gives 0."""
+    rng = np.random.default_rng(32)
+    Hkv, Hq, rK, rV = 3, 6, 8, 12
+    P_K = si.bases(33, Hkv, d, rK)
+    P_VJ = si.bases(34, 1, Hkv * d, rV)[0]
+    k = rng.standard_normal((2, Hkv, 5, rK))
+    v = rng.standard_normal((2, 5, rV))
+    lens = np.array([0, 1], np.int32)
+    got = o.decode_joint_v(5.0 * rng.standard_normal((2, Hq, d)), P_K, P_VJ, k, v, lens)
+    assert np.all(got[0] == 0.0)
+    full = P_VJ @ v[1, 0]                      # the reconstructed concatenation, Hkv*d long
+    G = Hq // Hkv
+    for h in range(Hq):
+        g = h // G
+        assert np.allclose(got[1, h], full[g * d:(g + 1) * d], rtol=0, atol=1e-14)
+    lat = o.decode_latent_joint_v(rng.standard_normal((2, Hq, rK)), k, v, lens, d=d)
+    assert np.all(lat[0] == 0.0)
+    assert np.array_equal(lat[1], np.repeat(v[1, :1], Hq, axis=0))
+
+
+def check_joint_v_compress_bookkeeping(o, d: int = 16) -> None:
+    """Joint rows land exactly at [len, len+T) of the sequence's value latent, keys per head
+    as in compress_append; a sequence that would overflow is left untouched."""
+    rng = np.random.default_rng(35)
+    B, Hkv, T, L_max, rK = 3, 2, 3, 10, 8
+    lens = np.array([0, 7, 8], np.int32)
+    k_new = si.bf16_to_f64(si.to_bf16(rng.standard_normal((B, Hkv, T, d))))
+    v_new = si.bf16_to_f64(si.to_bf16(rng.standard_normal((B, Hkv, T, d))))
+    P_K = np.repeat(_identity_basis(d, rK)[None], Hkv, axis=0)
+    P_VJ = np.eye(Hkv * d)                      # the stored latent is the concatenation itself
+    kl, vj, new_lens, nbad = o.compress_append_joint_v(
+        k_new, v_new, P_K, P_VJ, np.full((B, Hkv, L_max, rK), 7.0),
+        np.full((B, L_max, Hkv * d), -7.0), lens)
+    assert nbad == 1 and new_lens.tolist() == [3, 10, 8]
+    for b in range(2):
+        s = int(lens[b])
+        for t in range(T):
+            assert np.array_equal(vj[b, s + t], np.concatenate([v_new[b, g, t] for g in range(Hkv)]))
+            assert np.array_equal(kl[b, :, s + t], k_new[b, :, t, :rK])
+        keep = np.ones(L_max, bool)
+        keep[s:s + T] = False
+        assert np.all(vj[b, keep] == -7.0) and np.all(kl[b, :, keep] == 7.0)
+    assert np.all(vj[2] == -7.0) and np.all(kl[2] == 7.0)
+
+
 ALL_ORACLE_CHECKS = {
     "round_bf16_matches_torch": check_round_bf16_matches_torch,
     "round_bf16_edges": check_round_bf16_edges,
@@ -409,4 +543,9 @@ ALL_ORACLE_CHECKS = {
     "compress_identity_basis": check_compress_identity_basis,
     "compress_matches_exact_product": check_compress_matches_exact_product,
     "compress_append_bookkeeping": check_compress_append_bookkeeping,
+    "joint_v_full_rank_is_plain_attention": check_joint_v_full_rank_is_plain_attention,
+    "joint_v_block_diagonal_is_per_head": check_joint_v_block_diagonal_is_per_head,
+    "joint_v_latent_folding": check_joint_v_latent_folding,
+    "joint_v_edges": check_joint_v_edges,
+    "joint_v_compress_bookkeeping": check_joint_v_compress_bookkeeping,
 }

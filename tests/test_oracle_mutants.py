@@ -11,6 +11,7 @@ import os
 import subprocess
 import sys
 
+import numpy as np
 import pytest
 
 import oracle
@@ -87,4 +88,60 @@ def test_mutant_is_caught(tmp_path, name, orig, repl, checks):
         return  # the planted mistake crashed the child (e.g. an out-of-bounds write): caught
     caught = json.loads(proc.stdout.strip().splitlines()[-1])
     missed = [c for c, ok in caught.items() if not ok]
+    assert not missed, f"mutant {name} passed pins {missed}"
+
+
+# The joint-value calls are layout (concatenation order, the block of P_VJ each KV head reads,
+# the value latent every head shares) over the C functions above.  Their planted mistakes are
+# subclasses that override one layout helper; they touch no memory, so they run in-process.
+
+def _interleaved_concat(x):
+    Hkv, T, d = x.shape
+    return np.ascontiguousarray(np.transpose(x, (1, 2, 0)).reshape(T, d * Hkv))
+
+
+def _interleaved_blocks(P_VJ, Hkv):
+    HD, rV = P_VJ.shape
+    return np.ascontiguousarray(np.transpose(P_VJ.reshape(HD // Hkv, Hkv, rV), (1, 0, 2)))
+
+
+def _block0_everywhere(P_VJ, Hkv):
+    HD, rV = P_VJ.shape
+    return np.ascontiguousarray(np.broadcast_to(P_VJ[:HD // Hkv][None], (Hkv, HD // Hkv, rV)))
+
+
+def _values_for_head0_only(v_joint, Hkv):
+    B, L, rV = v_joint.shape
+    out = np.zeros((B, Hkv, L, rV))
+    out[:, 0] = v_joint
+    return out
+
+
+JOINT_MUTANTS = [
+    ("joint_concat_interleaved", "_concat_heads", _interleaved_concat,
+     ["joint_v_full_rank_is_plain_attention", "joint_v_block_diagonal_is_per_head",
+      "joint_v_compress_bookkeeping"]),
+    ("joint_blocks_interleaved", "_head_blocks", _interleaved_blocks,
+     ["joint_v_full_rank_is_plain_attention", "joint_v_block_diagonal_is_per_head",
+      "joint_v_edges"]),
+    ("joint_every_head_reads_block0", "_head_blocks", _block0_everywhere,
+     ["joint_v_full_rank_is_plain_attention", "joint_v_block_diagonal_is_per_head",
+      "joint_v_edges"]),
+    ("joint_values_for_head0_only", "_share_values", _values_for_head0_only,
+     ["joint_v_full_rank_is_plain_attention", "joint_v_edges"]),
+]
+
+
+@pytest.mark.parametrize("name,helper,wrong,checks", JOINT_MUTANTS, ids=[m[0] for m in JOINT_MUTANTS])
+def test_joint_mutant_is_caught(name, helper, wrong, checks):
+    import oracle_checks as oc
+    mutant_cls = type("Mutant", (oracle.Oracle,), {helper: staticmethod(wrong)})
+    m = mutant_cls(oracle.build())
+    missed = []
+    for c in checks:
+        try:
+            oc.ALL_ORACLE_CHECKS[c](m)
+            missed.append(c)
+        except (AssertionError, ValueError):
+            pass
     assert not missed, f"mutant {name} passed pins {missed}"
