@@ -266,8 +266,11 @@ STIEF_API stief_status stief_decode_latent(const uint16_t* q_lat, const uint16_t
                                  stief_stream_t stream);
 
 /*
- * Paged latent caches (serving-style block tables).  The pages give no memory layout;
- * this library's paged form keeps each cache as a pool of pages,
+ * Paged latent caches (serving-style block tables).  StiefAttention's pages give no
+ * memory layout; the idea of fixed-size token blocks for regular, coalesced cache access
+ * comes from a neighbouring method's page (HyLRA technical summary, section 2.4,
+ * "hardware-efficient optimisations": block-level sparsity over fixed token blocks).
+ * This library's paged form keeps each cache as a pool of pages,
  *     k_pages : bf16 [num_pages][Hkv][page_size][rK]
  *     v_pages : bf16 [num_pages][Hkv][page_size][rV]
  * and gives every sequence b a row of the block table,
@@ -315,7 +318,9 @@ STIEF_API stief_status stief_append_decode_paged(const uint16_t* q, const uint16
 
 /*
  * int8 latent caches (the low-bit form).  The pages report the compressed cache to be
- * robust to 4- and 8-bit quantisation but fix no scheme; this library stores each latent
+ * robust to 4- and 8-bit quantisation (StiefAttention technical summary, "Resultados
+ * Experimentais", the quantisation-compatibility result) but fix no scheme; this library
+ * stores each latent
  * row (one token, one KV head) as int8 codes and one fp32 scale:
  *     k_q : int8 [B][Hkv][L_max][rK],  k_s : float [B][Hkv][L_max]  (likewise v_q, v_s)
  *     scale = max_c |x_c| / 127,  code_c = RNE(x_c / scale) in [-127, 127]
