@@ -36,6 +36,9 @@ METRIC = "decode attn tokens/s and achieved HBM GB/s (frac of peak) over latent 
 DEFAULT_WORKLOAD = "llama3_8b_32k"
 ROTATE_BYTES = 3 * (126 << 20)  # consecutive steps' inputs span more than 3x the L2
 MAX_REPLICAS = 64
+# tokens per page of the paged caches (the fixed token-block size a neighbouring page's
+# hardware-efficiency section gives as its example)
+PAGE_SIZE = 128
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 FALLBACK_HBM_GBS = 6650.0
@@ -201,6 +204,23 @@ def replica_count(w: si.Workload, int8: bool = False) -> int:
     return 1 if per >= ROTATE_BYTES else min(MAX_REPLICAS, -(-ROTATE_BYTES // per))
 
 
+def to_pages(cache: torch.Tensor, page_size: int, perm: torch.Tensor):
+    """A contiguous latent cache [B][Hkv][L][r] as a page pool and block table.
+
+    Page j of sequence b (its tokens [j*page_size, (j+1)*page_size), every KV head) goes to
+    pool entry perm[b*max_pages + j]; the cache is zero-padded to whole pages.  Returns
+    (pool [B*max_pages][Hkv][page_size][r], block_table [B][max_pages] int32).
+    """
+    B, Hkv, L, r = cache.shape
+    mp = -(-L // page_size)
+    if mp * page_size != L:
+        cache = torch.nn.functional.pad(cache, (0, 0, 0, mp * page_size - L))
+    blocks = cache.reshape(B, Hkv, mp, page_size, r).permute(0, 2, 1, 3, 4)
+    pool = torch.empty((B * mp, Hkv, page_size, r), dtype=cache.dtype, device=cache.device)
+    pool[perm.to(cache.device)] = blocks.reshape(B * mp, Hkv, page_size, r)
+    return pool, perm.reshape(B, mp).to(device=cache.device, dtype=torch.int32)
+
+
 def _backlog():
     """Queue ~50 us of GPU work so the events that follow are not exposed to host launch gaps."""
     torch.cuda._sleep(100000)
@@ -250,6 +270,17 @@ def run_gpu(args, w: si.Workload):
                 lay.ks = torch.rand((w.B, w.Hkv, L8), generator=g, device=dev) * 0.02
                 lay.vs = torch.rand((w.B, w.Hkv, L8), generator=g, device=dev) * 0.02
                 lay.k_lat = lay.v_lat = None  # the bf16 caches are not used
+    # paged mode: every replica's layer caches moved into pools of PAGE_SIZE-token pages, the
+    # pages of each sequence at shuffled pool positions (one block table per layer)
+    if args.paged:
+        gp = torch.Generator()
+        gp.manual_seed(seed + 2)
+        for lays in reps:
+            for lay in lays:
+                perm = torch.randperm(w.B * -(-L_max // PAGE_SIZE), generator=gp)
+                lay.k_pages, lay.block_table = to_pages(lay.k_lat, PAGE_SIZE, perm)
+                lay.v_pages, _ = to_pages(lay.v_lat, PAGE_SIZE, perm)
+                lay.k_lat = lay.v_lat = None  # the contiguous caches are not used
     olat = [torch.empty((w.B, w.Hq, lay.rV), dtype=torch.bfloat16, device=dev)
             for lay in layers] if args.latent else []
 
@@ -262,6 +293,11 @@ def run_gpu(args, w: si.Workload):
             stief.stief_decode_latent(qlat_s[li], lay.k_lat, lay.v_lat, lay.seq_lens, olat[li],
                                       lay.ws, max_seq_len=L_max, num_splits=args.splits,
                                       dev_status=status)
+        elif args.paged:  # append + decode in one kernel, over page pools
+            stief.stief_append_decode_paged(q_s, k_s, v_s, lay.P_K, lay.P_V, lay.k_pages,
+                                            lay.v_pages, lay.block_table, lay.seq_lens, out[li],
+                                            lay.ws, max_seq_len=L_max, num_splits=args.splits,
+                                            dev_status=status)
         elif args.unfused:  # the two separate calls (three kernels)
             stief.stief_compress_append(k_s, v_s, lay.P_K, lay.P_V, lay.k_lat, lay.v_lat,
                                         lay.seq_lens, dev_status=status)
@@ -350,6 +386,11 @@ def run_gpu(args, w: si.Workload):
                 lay = reps[i % R][0]
                 if args.int8:
                     layer_step(0, lay)
+                elif args.paged:
+                    stief.stief_decode_attention_paged(q_s, lay.P_K, lay.P_V, lay.k_pages,
+                                                       lay.v_pages, lay.block_table, lay.seq_lens,
+                                                       out[0], lay.ws, max_seq_len=L_max,
+                                                       dev_status=status)
                 else:
                     stief.stief_decode_attention(q_s, lay.P_K, lay.P_V, lay.k_lat, lay.v_lat,
                                                  lay.seq_lens, out[0], lay.ws, max_seq_len=L_max,
@@ -493,11 +534,15 @@ def run_gpu(args, w: si.Workload):
                       "latent decode only (bases folded into the attention weights: q~ in, "
                       "o~ out; the new token's latent rows would come from the folded K/V "
                       "projection), every layer; " if args.latent else
+                      f"append 1 token per (sequence, KV head) + decode over page pools "
+                      f"({PAGE_SIZE}-token pages at shuffled pool positions), every layer; "
+                      if args.paged else
                       "append 1 token per (sequence, KV head) + decode, every layer; ") +
                      "the API calls captured in CUDA graphs (one step per replica, the timed "
                      "region replays the replica cycle back to back); " +
                      ("stief_decode_attention_q8 (1 kernel per layer)" if args.int8 else
                       "stief_decode_latent (1 kernel per layer)" if args.latent else
+                      "stief_append_decode_paged (1 kernel per layer)" if args.paged else
                       "stief_compress_append + stief_decode_attention (3 kernels per layer)"
                       if args.unfused else "stief_append_decode (1 kernel per layer)")),
             "context_growth": (f"none (context {w.L} every step)" if args.latent or args.int8 else
@@ -513,6 +558,7 @@ def run_gpu(args, w: si.Workload):
         "roofline": {
             "kernel": "stief_decode_kernel (" + ("stief_decode_attention_q8" if args.int8 else
                                                  "stief_decode_latent" if args.latent else
+                                                 "stief_append_decode_paged" if args.paged else
                                                  "stief_decode_attention" if args.unfused
                                                  else "stief_append_decode") + ")",
             "bound": "hbm",
@@ -521,7 +567,8 @@ def run_gpu(args, w: si.Workload):
             "peak_kind": f"{peak_kind} hbm_gbs (copy bandwidth, burst)",
             "unit": "GB/s",
             "frac": round(achieved / peak, 4),
-            "traffic": None if (args.latent or args.unfused or args.int8) else _traffic_per_launch(w.name),
+            "traffic": (None if (args.latent or args.unfused or args.int8 or args.paged)
+                        else _traffic_per_launch(w.name)),
             "algorithmic_bytes": bytes_per_dec,
             "decode_us": round(dec_us, 3),
             "decode_timing": f"{dec_reps} replays of a graph of {n_dec} back-to-back decode "
@@ -539,7 +586,8 @@ def run_gpu(args, w: si.Workload):
     }
     if compress is not None:
         result["compress"] = compress
-    if rank == 0 and ws_n == 1 and not args.no_cpu_baseline and not args.latent and not args.int8:
+    if (rank == 0 and ws_n == 1 and not args.no_cpu_baseline
+            and not (args.latent or args.int8 or args.paged)):
         result["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     if ws_n > 1:
         torch.distributed.destroy_process_group()
@@ -766,6 +814,9 @@ def main():
     ap.add_argument("--latent", action="store_true",
                     help="time stief_decode_latent (bases folded into the attention weights) "
                          "instead of the fused append + decode step")
+    ap.add_argument("--paged", action="store_true",
+                    help="time stief_append_decode_paged: the fused step over page pools "
+                         f"({PAGE_SIZE}-token pages, shuffled block tables)")
     ap.add_argument("--unfused", action="store_true",
                     help="time the step as the two separate calls (append kernel, length "
                          "update, decode) instead of stief_append_decode")
@@ -777,6 +828,10 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if sum(map(bool, (args.int8, args.latent, args.paged, args.unfused))) > 1:
+        ap.error("--int8, --latent, --paged and --unfused are separate modes")
+    if args.paged and args.profile_launches > 0:
+        ap.error("--profile-launches has no paged mode")
     w = si.WORKLOADS[args.workload]
     if args.layers > 0:
         import dataclasses

@@ -1,0 +1,39 @@
+"""Host-side pieces of bench.py (CPU only): the paged-cache setup of ``--paged``.
+
+``to_pages`` moves a contiguous latent cache into a page pool at shuffled positions; the
+oracle's ``gather_pages`` (pinned by its own scatter/gather check) must give the contiguous
+cache back, so the paged bench times the same attention as the contiguous one.
+"""
+import numpy as np
+import torch
+
+import bench
+import oracle
+
+
+def test_to_pages_round_trip_through_the_oracle_gather():
+    B, Hkv, L, r, ps = 3, 2, 300, 16, 128          # 300 tokens: 3 pages, the last one partial
+    g = torch.Generator().manual_seed(5)
+    cache = torch.randn((B, Hkv, L, r), generator=g).to(torch.bfloat16)
+    mp = -(-L // ps)
+    perm = torch.randperm(B * mp, generator=g)
+    pool, bt = bench.to_pages(cache, ps, perm)
+    assert pool.shape == (B * mp, Hkv, ps, r) and pool.dtype == torch.bfloat16
+    assert bt.shape == (B, mp) and bt.dtype == torch.int32
+    assert sorted(bt.flatten().tolist()) == list(range(B * mp))   # every pool page used once
+    lens = np.array([L, 129, 0], np.int32)
+    back = oracle.gather_pages(pool.to(torch.float64).numpy(), bt.numpy(), lens, L)
+    want = cache.to(torch.float64).numpy()
+    for b in range(B):
+        assert np.array_equal(back[b, :, :lens[b]], want[b, :, :lens[b]])
+    # the padding past L in the last page is zero
+    last = pool[int(bt[0, mp - 1])]
+    assert torch.all(last[:, L - (mp - 1) * ps:] == 0)
+
+
+def test_to_pages_exact_pages_need_no_padding():
+    cache = torch.arange(2 * 1 * 256 * 8, dtype=torch.float32).reshape(2, 1, 256, 8)
+    perm = torch.tensor([3, 0, 2, 1])
+    pool, bt = bench.to_pages(cache, 128, perm)
+    assert bt.tolist() == [[3, 0], [2, 1]]
+    assert torch.equal(pool[3, 0], cache[0, 0, :128]) and torch.equal(pool[1, 0], cache[1, 0, 128:])
