@@ -20,10 +20,12 @@ from ._binding import (  # noqa: F401
     stief_compress_append_paged,
     stief_decode_attention,
     stief_decode_attention_q8,
+    stief_decode_attention_joint_v,
     stief_decode_attention_paged,
     stief_decode_attention_noalloc,
     stief_decode_auto_splits,
     stief_decode_latent,
+    stief_decode_latent_joint_v,
     stief_decode_max_splits,
     stief_decode_workspace_bytes,
     stief_read_device_status,

@@ -89,6 +89,12 @@ def library() -> ctypes.CDLL:
             lib.stief_decode_attention_q8.restype = _i
             lib.stief_decode_attention_q8.argtypes = ([vp] * 10 + [ctypes.c_size_t] + [_i] * 9
                                                       + [vp, vp])
+            lib.stief_decode_attention_joint_v.restype = _i
+            lib.stief_decode_attention_joint_v.argtypes = ([vp] * 8 + [ctypes.c_size_t] + [_i] * 9
+                                                           + [vp, vp])
+            lib.stief_decode_latent_joint_v.restype = _i
+            lib.stief_decode_latent_joint_v.argtypes = ([vp] * 6 + [ctypes.c_size_t] + [_i] * 9
+                                                        + [vp, vp])
             lib.stief_decode_latent.restype = _i
             lib.stief_decode_latent.argtypes = ([vp] * 6 + [ctypes.c_size_t] + [_i] * 9
                                                 + [vp, vp])
@@ -508,3 +514,69 @@ def stief_read_device_status(dev_status: torch.Tensor, stream=None) -> int:
     if code not in (0, 6):
         raise StiefError("stief_read_device_status", code)
     return int(v.value)
+
+
+def stief_decode_attention_joint_v(q: torch.Tensor, P_K: torch.Tensor, P_VJ: torch.Tensor,
+                                   k_lat: torch.Tensor, v_joint: torch.Tensor,
+                                   seq_lens: torch.Tensor, out: torch.Tensor,
+                                   workspace: torch.Tensor, max_seq_len: int, num_splits: int = 0,
+                                   dev_status: Optional[torch.Tensor] = None,
+                                   stream=None) -> torch.Tensor:
+    """stief_decode_attention with a joint value latent: P_VJ [Hkv*d][rV] bf16 over the
+    concatenated KV-head values, v_joint [B][L_max][rV] bf16 (one row per token, shared by the
+    KV heads); keys, q, out and the workspace as for stief_decode_attention."""
+    pq = _dev(q, "q", torch.bfloat16, 3)
+    ppk = _dev(P_K, "P_K", torch.bfloat16, 3)
+    ppv = _dev(P_VJ, "P_VJ", torch.bfloat16, 2)
+    pkl = _dev(k_lat, "k_lat", torch.bfloat16, 4)
+    pvl = _dev(v_joint, "v_joint", torch.bfloat16, 3)
+    psl = _dev(seq_lens, "seq_lens", torch.int32, 1)
+    po = _dev(out, "out", torch.bfloat16, 3)
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    B, Hq, d = q.shape
+    Hkv, _, rK = P_K.shape
+    rV = P_VJ.shape[1]
+    L_max = k_lat.shape[2]
+    if tuple(P_K.shape) != (Hkv, d, rK) or tuple(P_VJ.shape) != (Hkv * d, rV) \
+            or tuple(k_lat.shape) != (B, Hkv, L_max, rK) \
+            or tuple(v_joint.shape) != (B, L_max, rV) or seq_lens.shape[0] != B \
+            or tuple(out.shape) != (B, Hq, d):
+        raise ValueError("stief_decode_attention_joint_v: inconsistent shapes")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    code = library().stief_decode_attention_joint_v(pq, ppk, ppv, pkl, pvl, psl, po,
+                                                    workspace.data_ptr(), ws_bytes, B, Hq, Hkv, d,
+                                                    rK, rV, L_max, int(max_seq_len),
+                                                    int(num_splits), _opt_status(dev_status),
+                                                    _stream_ptr(stream))
+    _check("stief_decode_attention_joint_v", code)
+    return out
+
+
+def stief_decode_latent_joint_v(q_lat: torch.Tensor, k_lat: torch.Tensor, v_joint: torch.Tensor,
+                                seq_lens: torch.Tensor, out_lat: torch.Tensor,
+                                workspace: torch.Tensor, max_seq_len: int, num_splits: int = 0,
+                                d: int = 128, dev_status: Optional[torch.Tensor] = None,
+                                stream=None) -> torch.Tensor:
+    """stief_decode_latent with a joint value latent v_joint [B][L_max][rV] bf16 (one row per
+    token, shared by the KV heads)."""
+    pq = _dev(q_lat, "q_lat", torch.bfloat16, 3)
+    pkl = _dev(k_lat, "k_lat", torch.bfloat16, 4)
+    pvl = _dev(v_joint, "v_joint", torch.bfloat16, 3)
+    psl = _dev(seq_lens, "seq_lens", torch.int32, 1)
+    po = _dev(out_lat, "out_lat", torch.bfloat16, 3)
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    B, Hq, rK = q_lat.shape
+    Hkv, L_max = k_lat.shape[1], k_lat.shape[2]
+    rV = v_joint.shape[2]
+    if tuple(k_lat.shape) != (B, Hkv, L_max, rK) or tuple(v_joint.shape) != (B, L_max, rV) \
+            or seq_lens.shape[0] != B or tuple(out_lat.shape) != (B, Hq, rV):
+        raise ValueError("stief_decode_latent_joint_v: inconsistent shapes")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    code = library().stief_decode_latent_joint_v(pq, pkl, pvl, psl, po, workspace.data_ptr(),
+                                                 ws_bytes, B, Hq, Hkv, int(d), rK, rV, L_max,
+                                                 int(max_seq_len), int(num_splits),
+                                                 _opt_status(dev_status), _stream_ptr(stream))
+    _check("stief_decode_latent_joint_v", code)
+    return out_lat

@@ -311,14 +311,18 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int NW, int ns, int rK,
 // NKS >= rK/16; NMV >= rV/16.
 constexpr int kMaxConsumerWarps = 8;
 
-// Kernel modes: the contiguous bf16 cache, the latent decode, paged caches, int8 caches.
+// Kernel modes: the contiguous bf16 cache, the latent decode, paged caches, int8 caches, and
+// joint value latents (one value row per token shared by the KV heads; full or latent output).
 // Each is its own instantiation, so a mode's branches cost the others nothing.
-constexpr int kModePlain = 0, kModeLatent = 1, kModePaged = 2, kModeQ8 = 3;
+constexpr int kModePlain = 0, kModeLatent = 1, kModePaged = 2, kModeQ8 = 3, kModeJointV = 4,
+              kModeLatentJointV = 5;
 
 template <int NB, int NKS, int NMV, int TT, int MODE>
 __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
     stief_decode_kernel(const __grid_constant__ DecodeArgs a) {
-  constexpr bool LAT = MODE == kModeLatent, PG = MODE == kModePaged, Q8 = MODE == kModeQ8;
+  constexpr bool LAT = MODE == kModeLatent || MODE == kModeLatentJointV;
+  constexpr bool PG = MODE == kModePaged, Q8 = MODE == kModeQ8;
+  constexpr bool JV = MODE == kModeJointV || MODE == kModeLatentJointV;
   constexpr int kTile = TT;
   constexpr int MT = TT / 16;              // 16-token m-tiles (scores) / k-steps (mix) per tile
   // score k-steps / value m-tiles whose fragments are loaded together (fewer where the
@@ -468,13 +472,16 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
     }
     // whole 32-row boxes land (rows past the sequence are masked on chip)
     mbar_arrive_expect_tx(bar, st_bytes);
-    const int y = tile_row(t0 + (w + k * NW) * kTile);
+    const int tt = t0 + (w + k * NW) * kTile;
+    const int y = tile_row(tt);
+    // joint values: the value rows of sequence b are b * L_max + t, whatever the KV head
+    const int yv = JV ? b * a.L_max + tt : y;
 #pragma unroll
     for (int p = 0; p < 3; ++p)
       if (p < npk) tma_load_2d(dst + ko[p], kmap[p], kx[p], y, bar, policy);
 #pragma unroll
     for (int p = 0; p < 3; ++p)
-      if (p < npv) tma_load_2d(dst + vo[p], vmap[p], vx[p], y, bar, policy);
+      if (p < npv) tma_load_2d(dst + vo[p], vmap[p], vx[p], yv, bar, policy);
   };
 
   // ---- prologue ------------------------------------------------------------------------------
@@ -1198,6 +1205,11 @@ template <int NB, int NKS, int NMV, int TT>
 static cudaError_t launch_t(const DecodeArgs& a, cudaStream_t stream) {
   if ((a.latent != 0) + (a.block_table != nullptr) + (a.q8 != 0) > 1)
     return cudaErrorInvalidValue;  // the modes do not combine
+  if (a.joint_v) {
+    if (a.block_table != nullptr || a.q8 != 0 || a.append != 0) return cudaErrorInvalidValue;
+    return a.latent ? launch_k<NB, NKS, NMV, TT, kModeLatentJointV>(a, stream)
+                    : launch_k<NB, NKS, NMV, TT, kModeJointV>(a, stream);
+  }
   if (a.latent) return launch_k<NB, NKS, NMV, TT, kModeLatent>(a, stream);
   if (a.block_table) return launch_k<NB, NKS, NMV, TT, kModePaged>(a, stream);
   if (a.q8) return launch_k<NB, NKS, NMV, TT, kModeQ8>(a, stream);

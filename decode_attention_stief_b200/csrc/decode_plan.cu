@@ -169,8 +169,9 @@ stief_status plan_decode(DecodeArgs& a, const uint16_t* q, const uint16_t* P_K,
                          int rK, int rV, int L_max, int max_seq_len, int num_splits,
                          uint32_t* dev_status, bool latent, const int32_t* block_table,
                          int max_pages, int page_size, int num_pages, const float* k_scale,
-                         const float* v_scale) {
+                         const float* v_scale, bool joint_v) {
   const bool q8 = k_scale != nullptr;
+  if (joint_v && (block_table || q8)) return STIEF_ERR_INVALID_ARG;
   if (!q || !k_lat || !v_lat || !seq_lens || !out) return STIEF_ERR_INVALID_ARG;
   if (!latent && (!P_K || !P_V)) return STIEF_ERR_INVALID_ARG;
   if (B < 1 || B > 65535 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || Hq / Hkv > 64)
@@ -186,6 +187,8 @@ stief_status plan_decode(DecodeArgs& a, const uint16_t* q, const uint16_t* P_K,
   // rows of the cache tensors: contiguous [B][Hkv][L_max], or pools [num_pages][Hkv][page_size]
   const uint64_t rows = block_table ? (uint64_t)num_pages * Hkv * page_size : (uint64_t)B * Hkv * L_max;
   if (rows >= (1ull << 31)) return STIEF_ERR_INVALID_ARG;  // TMA row coordinates are int32
+  // joint values: one row per (sequence, token), [B][L_max][rV], read by every KV head
+  const uint64_t vrows = joint_v ? (uint64_t)B * L_max : rows;
 
   int dev = 0, sms = 0;
   bool sm100 = false;
@@ -197,6 +200,7 @@ stief_status plan_decode(DecodeArgs& a, const uint16_t* q, const uint16_t* P_K,
   a.max_pages = max_pages;
   a.page_size = page_size;
   a.num_pages = num_pages;
+  a.joint_v = joint_v ? 1 : 0;
 
   a.q = q;
   a.seq_lens = seq_lens;
@@ -243,7 +247,7 @@ stief_status plan_decode(DecodeArgs& a, const uint16_t* q, const uint16_t* P_K,
     a.pv.p[0].width = rV;
     nmaps = 2;
   } else if (!plan_pieces(a, &nmaps, a.pk, k_lat, rK, rows, a.tile) ||
-             !plan_pieces(a, &nmaps, a.pv, v_lat, rV, rows, a.tile)) {
+             !plan_pieces(a, &nmaps, a.pv, v_lat, rV, vrows, a.tile)) {
     return STIEF_ERR_CUDA;
   }
   if (!latent && (!plan_pieces(a, &nmaps, a.ppk, P_K, rK, prow, d) ||

@@ -220,7 +220,7 @@ stief_status decode_common(const uint16_t* q, const uint16_t* k_new, const uint1
                            int L_max, int max_seq_len, int num_splits, uint32_t* dev_status,
                            stief_stream_t stream, bool append, bool latent = false,
                            const Paging& pg = Paging{}, const float* k_scale = nullptr,
-                           const float* v_scale = nullptr) {
+                           const float* v_scale = nullptr, bool joint_v = false) {
   // cheap host checks first, so argument errors never touch CUDA
   if (!q || !k_lat || !v_lat || !seq_lens || !out) return STIEF_ERR_INVALID_ARG;
   if (pg.block_table) {  // paged: the capacity is max_pages * page_size tokens
@@ -244,7 +244,7 @@ stief_status decode_common(const uint16_t* q, const uint16_t* k_new, const uint1
   stief::DecodeArgs a{};
   st = stief::plan_decode(a, q, P_K, P_V, k_lat, v_lat, seq_lens, out, B, Hq, Hkv, d, rK, rV,
                           L_max, max_seq_len, num_splits, dev_status, latent, pg.block_table,
-                          pg.max_pages, pg.page_size, pg.num_pages, k_scale, v_scale);
+                          pg.max_pages, pg.page_size, pg.num_pages, k_scale, v_scale, joint_v);
   if (st != STIEF_OK) return st;
   a.append = append ? 1 : 0;
   a.k_new = k_new;
@@ -299,6 +299,35 @@ stief_status stief_decode_latent(const uint16_t* q_lat, const uint16_t* k_lat,
                        const_cast<uint16_t*>(v_lat), const_cast<int32_t*>(seq_lens), out_lat,
                        workspace, workspace_bytes, B, Hq, Hkv, d, rK, rV, L_max, max_seq_len,
                        num_splits, dev_status, stream, false, true);
+}
+
+stief_status stief_decode_attention_joint_v(const uint16_t* q, const uint16_t* P_K,
+                                            const uint16_t* P_VJ, const uint16_t* k_lat,
+                                            const uint16_t* v_joint, const int32_t* seq_lens,
+                                            uint16_t* out, void* workspace,
+                                            size_t workspace_bytes, int B, int Hq, int Hkv,
+                                            int d, int rK, int rV, int L_max, int max_seq_len,
+                                            int num_splits, uint32_t* dev_status,
+                                            stief_stream_t stream) {
+  return decode_common(q, nullptr, nullptr, P_K, P_VJ, const_cast<uint16_t*>(k_lat),
+                       const_cast<uint16_t*>(v_joint), const_cast<int32_t*>(seq_lens), out,
+                       workspace, workspace_bytes, B, Hq, Hkv, d, rK, rV, L_max, max_seq_len,
+                       num_splits, dev_status, stream, false, false, Paging{}, nullptr, nullptr,
+                       true);
+}
+
+stief_status stief_decode_latent_joint_v(const uint16_t* q_lat, const uint16_t* k_lat,
+                                         const uint16_t* v_joint, const int32_t* seq_lens,
+                                         uint16_t* out_lat, void* workspace,
+                                         size_t workspace_bytes, int B, int Hq, int Hkv, int d,
+                                         int rK, int rV, int L_max, int max_seq_len,
+                                         int num_splits, uint32_t* dev_status,
+                                         stief_stream_t stream) {
+  return decode_common(q_lat, nullptr, nullptr, nullptr, nullptr, const_cast<uint16_t*>(k_lat),
+                       const_cast<uint16_t*>(v_joint), const_cast<int32_t*>(seq_lens), out_lat,
+                       workspace, workspace_bytes, B, Hq, Hkv, d, rK, rV, L_max, max_seq_len,
+                       num_splits, dev_status, stream, false, true, Paging{}, nullptr, nullptr,
+                       true);
 }
 
 stief_status stief_decode_attention_q8(const uint16_t* q, const uint16_t* P_K,

@@ -63,6 +63,7 @@ struct DecodeArgs {
   int max_pages, page_size, num_pages;
   // int8 caches: k_lat / v_lat hold int8 codes [rows][r] and these the fp32 row scales
   int q8;
+  int joint_v;     // values: one row per (sequence, token) shared by the KV heads
   const float* k_scale;
   const float* v_scale;
 };
@@ -133,7 +134,7 @@ stief_status plan_decode(DecodeArgs& a, const uint16_t* q, const uint16_t* P_K,
                          uint32_t* dev_status, bool latent = false,
                          const int32_t* block_table = nullptr, int max_pages = 0,
                          int page_size = 0, int num_pages = 0, const float* k_scale = nullptr,
-                         const float* v_scale = nullptr);
+                         const float* v_scale = nullptr, bool joint_v = false);
 
 // Decode workspace layout: `units` = B * Hkv * qsub split-ticket counters, then B sequence
 // tickets (uint32, padded together to 256 bytes), then units * G_T * splits partial states

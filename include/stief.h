@@ -348,6 +348,35 @@ STIEF_API stief_status stief_decode_attention_q8(const uint16_t* q, const uint16
                                        stief_stream_t stream);
 
 /*
+ * Joint value latents (STAR-KV technical summary, "Metodologia" item 2, the hybrid
+ * decomposition: keys keep one basis per KV head, the values of all KV heads are factored
+ * together, and the value reconstruction is absorbed into the output projection).  The values
+ * of a token's Hkv heads, concatenated head 0 first, are projected by one basis
+ *     P_VJ : bf16 [Hkv*d][rV]
+ * and the cache holds one value latent per token, shared by every KV head:
+ *     v_joint : bf16 [B][L_max][rV]
+ * KV head g's values are rebuilt from rows [g*d, (g+1)*d) of P_VJ, so P_VJ read as
+ * [Hkv][d][rV] has the per-head P_V layout.  The keys, queries, outputs, workspace, status
+ * words and launch behaviour are those of the per-head calls:
+ *   stief_decode_attention_joint_v: stief_decode_attention with v_lat -> v_joint and
+ *       P_V -> P_VJ:  o_h = (sum_t p_t v_joint[t]) . (rows of KV head g of P_VJ)^T;
+ *   stief_decode_latent_joint_v: stief_decode_latent with v_lat -> v_joint:
+ *       o~_h = sum_t p_t v_joint[t].
+ * B * L_max < 2^31 as for the per-head cache.  No fused append, paged or int8 form.
+ */
+STIEF_API stief_status stief_decode_attention_joint_v(
+    const uint16_t* q, const uint16_t* P_K, const uint16_t* P_VJ, const uint16_t* k_lat,
+    const uint16_t* v_joint, const int32_t* seq_lens, uint16_t* out, void* workspace,
+    size_t workspace_bytes, int B, int Hq, int Hkv, int d, int rK, int rV, int L_max,
+    int max_seq_len, int num_splits, uint32_t* dev_status, stief_stream_t stream);
+
+STIEF_API stief_status stief_decode_latent_joint_v(
+    const uint16_t* q_lat, const uint16_t* k_lat, const uint16_t* v_joint,
+    const int32_t* seq_lens, uint16_t* out_lat, void* workspace, size_t workspace_bytes, int B,
+    int Hq, int Hkv, int d, int rK, int rV, int L_max, int max_seq_len, int num_splits,
+    uint32_t* dev_status, stief_stream_t stream);
+
+/*
  * stief_decode_attention_noalloc -- stief_decode_attention without a workspace
  * argument and without any device allocation.  The paper has no counterpart: this
  * is a deployment variant for callers that cannot obtain device memory when they

@@ -111,6 +111,37 @@ def test_latent_decode_argument_errors(lib, kw, code):
     assert _latent(lib, **kw) == code
 
 
+def _joint(lib, latent=False, **kw):
+    a = dict(q=FAKE, P_K=FAKE, P_VJ=FAKE, k_lat=FAKE, v_joint=FAKE, seq_lens=FAKE, out=FAKE,
+             ws=FAKE, ws_bytes=1 << 40, B=1, Hq=32, Hkv=8, d=128, rK=64, rV=64, L_max=1024,
+             max_seq_len=1024, num_splits=0)
+    a.update(kw)
+    tail = (a["ws"], a["ws_bytes"], a["B"], a["Hq"], a["Hkv"], a["d"], a["rK"], a["rV"],
+            a["L_max"], a["max_seq_len"], a["num_splits"], None, None)
+    if latent:
+        return lib.stief_decode_latent_joint_v(a["q"], a["k_lat"], a["v_joint"], a["seq_lens"],
+                                               a["out"], *tail)
+    return lib.stief_decode_attention_joint_v(a["q"], a["P_K"], a["P_VJ"], a["k_lat"],
+                                              a["v_joint"], a["seq_lens"], a["out"], *tail)
+
+
+@pytest.mark.parametrize("latent", [False, True])
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), INVALID), (dict(v_joint=None), INVALID), (dict(out=None), INVALID),
+    (dict(d=64), INVALID), (dict(rV=40), INVALID), (dict(Hq=30), INVALID),
+    (dict(max_seq_len=2048), CAPACITY), (dict(v_joint=FAKE + 2), ALIGN),
+    (dict(ws_bytes=16), WORKSPACE),
+])
+def test_joint_value_decode_argument_errors(lib, latent, kw, code):
+    """The joint-value calls check what the per-head decode and latent decode check."""
+    assert _joint(lib, latent=latent, **kw) == code
+
+
+@pytest.mark.parametrize("kw", [dict(P_K=None), dict(P_VJ=None)])
+def test_joint_value_decode_needs_both_bases(lib, kw):
+    assert _joint(lib, **kw) == INVALID
+
+
 def _paged(lib, **kw):
     a = dict(q=FAKE, P_K=FAKE, P_V=FAKE, kp=FAKE, vp=FAKE, bt=FAKE, sl=FAKE, out=FAKE, ws=FAKE,
              ws_bytes=1 << 40, B=2, Hq=32, Hkv=8, d=128, rK=64, rV=64, num_pages=64,
