@@ -194,13 +194,24 @@ def build_state(w: si.Workload, total_steps: int, seed: int, dev):
     return layers, L_max
 
 
-def replica_count(w: si.Workload, int8: bool = False) -> int:
+def row_bytes_fn(w: si.Workload, int8: bool = False, joint: bool = False):
+    """Cache bytes per (token, sequence, KV head) for a layer of ranks (rK, rV): bf16 rows, int8
+    rows with their two fp32 scales, or per-head keys with one joint value row shared by the
+    Hkv heads (its bytes split over them)."""
+    if int8:
+        return lambda rK, rV: rK + rV + 8
+    if joint:
+        return lambda rK, rV: 2 * rK + 2 * rV / w.Hkv
+    return lambda rK, rV: 2 * (rK + rV)
+
+
+def replica_count(w: si.Workload, int8: bool = False, joint: bool = False) -> int:
     """Copies of the workload's layer state that consecutive timed steps rotate over, so that
     the inputs of a step were last touched at least ROTATE_BYTES of cache reads earlier
     (more than 3x the 126 MB L2: every step streams its cache from HBM, and no flush is
     needed between steps)."""
-    per = sum(((rK + rV + 8) if int8 else 2 * (rK + rV)) * w.B * w.Hkv * w.L
-              for rK, rV in w.layer_ranks())
+    rb = row_bytes_fn(w, int8, joint)
+    per = int(sum(rb(rK, rV) * w.B * w.Hkv * w.L for rK, rV in w.layer_ranks()))
     return 1 if per >= ROTATE_BYTES else min(MAX_REPLICAS, -(-ROTATE_BYTES // per))
 
 
@@ -239,7 +250,7 @@ def run_gpu(args, w: si.Workload):
                                              device_id=dev)
     seed = rank_seed(w.seed, rank)
     W, K = args.warmup, args.steps
-    R = replica_count(w, args.int8)
+    R = replica_count(w, args.int8, args.joint)
     reps = []
     for r in range(R):
         # room for every append of the warm-up, timed and kernel-timing runs of a replica
@@ -281,6 +292,16 @@ def run_gpu(args, w: si.Workload):
                 lay.k_pages, lay.block_table = to_pages(lay.k_lat, PAGE_SIZE, perm)
                 lay.v_pages, _ = to_pages(lay.v_lat, PAGE_SIZE, perm)
                 lay.k_lat = lay.v_lat = None  # the contiguous caches are not used
+    # joint mode: per layer one joint value basis P_VJ [Hkv*d][rV] and one value latent per
+    # token v_joint [B][L_max][rV] shared by the KV heads (the per-head value caches dropped)
+    if args.joint:
+        for ri, lays in enumerate(reps):
+            for li, lay in enumerate(lays):
+                js = si.sub_seed(seed, 14, li, ri)
+                lay.P_VJ = si.to_bf16(si.bases(js, 1, w.Hkv * w.d, lay.rV)[0]).to(dev)
+                lay.v_joint = si.latent_cache_torch(js, w.B, 1, L_max, lay.rV, 1, dev)[:, 0]
+                lay.v_joint = lay.v_joint.contiguous()
+                lay.v_lat = None
     olat = [torch.empty((w.B, w.Hq, lay.rV), dtype=torch.bfloat16, device=dev)
             for lay in layers] if args.latent else []
 
@@ -293,6 +314,11 @@ def run_gpu(args, w: si.Workload):
             stief.stief_decode_latent(qlat_s[li], lay.k_lat, lay.v_lat, lay.seq_lens, olat[li],
                                       lay.ws, max_seq_len=L_max, num_splits=args.splits,
                                       dev_status=status)
+        elif args.joint:  # decode with per-head keys and the joint value latent (no append)
+            stief.stief_decode_attention_joint_v(q_s, lay.P_K, lay.P_VJ, lay.k_lat, lay.v_joint,
+                                                 lay.seq_lens, out[li], lay.ws,
+                                                 max_seq_len=L_max, num_splits=args.splits,
+                                                 dev_status=status)
         elif args.paged:  # append + decode in one kernel, over page pools
             stief.stief_append_decode_paged(q_s, k_s, v_s, lay.P_K, lay.P_V, lay.k_pages,
                                             lay.v_pages, lay.block_table, lay.seq_lens, out[li],
@@ -324,7 +350,7 @@ def run_gpu(args, w: si.Workload):
             layer_step(0, lay)
 
     def reset_lengths(L0):
-        if args.latent or args.int8:  # nothing is appended: every step attends over the full context
+        if args.latent or args.int8 or args.joint:  # no append: every step attends over the full context
             L0 = w.L
         for lays in reps:
             for lay in lays:
@@ -384,7 +410,7 @@ def run_gpu(args, w: si.Workload):
         with torch.cuda.graph(warm_graph, stream=cap):
             for i in range(n_dec):
                 lay = reps[i % R][0]
-                if args.int8:
+                if args.int8 or args.joint:
                     layer_step(0, lay)
                 elif args.paged:
                     stief.stief_decode_attention_paged(q_s, lay.P_K, lay.P_V, lay.k_pages,
@@ -442,7 +468,7 @@ def run_gpu(args, w: si.Workload):
     # ---- decode kernel timing for the roofline: runs of n_dec back-to-back launches
     # (replicas rotating), averaged over the timed region; plus single launches.  The fused
     # kernel appends a token per launch: lengths restart at L_dec - 1 for each run.
-    appends = not (args.unfused or args.latent or args.int8)  # the step's kernel appends a token
+    appends = not (args.unfused or args.latent or args.int8 or args.joint)  # the kernel appends
     L_run0 = L_dec - (1 if appends else 0)
     reset_lengths(L_run0)
     dec_reps = max(3, args.decode_iters // n_dec)
@@ -505,7 +531,7 @@ def run_gpu(args, w: si.Workload):
     # ---- numbers
     value = job_tokens_per_s(w.B, ws_n, ms_per_step)
     lay0 = layers[0]
-    row_bytes = (lambda rK, rV: rK + rV + 8) if args.int8 else (lambda rK, rV: 2 * (rK + rV))
+    row_bytes = row_bytes_fn(w, args.int8, args.joint)
     bytes_per_dec = int(row_bytes(lay0.rK, lay0.rV) * w.B * w.Hkv * L_dec_mean)
     achieved = bytes_per_dec / (dec_us / 1e6) / 1e9
     peak, peak_kind = _hbm_peak()
@@ -531,6 +557,8 @@ def run_gpu(args, w: si.Workload):
             + (["..."] if len(layers) > 4 else []),
             "step": (("decode over an int8 latent cache (codes + fp32 row scales, synthetic "
                       "values), no append, every layer; " if args.int8 else
+                      "decode with per-head keys and one joint value latent per token shared by "
+                      "the KV heads, no append, every layer; " if args.joint else
                       "latent decode only (bases folded into the attention weights: q~ in, "
                       "o~ out; the new token's latent rows would come from the folded K/V "
                       "projection), every layer; " if args.latent else
@@ -541,11 +569,13 @@ def run_gpu(args, w: si.Workload):
                      "the API calls captured in CUDA graphs (one step per replica, the timed "
                      "region replays the replica cycle back to back); " +
                      ("stief_decode_attention_q8 (1 kernel per layer)" if args.int8 else
+                      "stief_decode_attention_joint_v (1 kernel per layer)" if args.joint else
                       "stief_decode_latent (1 kernel per layer)" if args.latent else
                       "stief_append_decode_paged (1 kernel per layer)" if args.paged else
                       "stief_compress_append + stief_decode_attention (3 kernels per layer)"
                       if args.unfused else "stief_append_decode (1 kernel per layer)")),
-            "context_growth": (f"none (context {w.L} every step)" if args.latent or args.int8 else
+            "context_growth": (f"none (context {w.L} every step)"
+                               if args.latent or args.int8 or args.joint else
                                f"+1 token per step of a replica (contexts {ctx_first}..{ctx_last})"),
             "l2": (f"no flush: steps rotate over {R} copies of the layer caches "
                    f"({rot_mb:.0f} MiB in all, > 3x the 126 MB L2)" if R > 1 else
@@ -557,6 +587,7 @@ def run_gpu(args, w: si.Workload):
         "hbm_gbs_step": round(step_bytes / (ms_per_step / 1e3) / 1e9, 1),
         "roofline": {
             "kernel": "stief_decode_kernel (" + ("stief_decode_attention_q8" if args.int8 else
+                                                 "stief_decode_attention_joint_v" if args.joint else
                                                  "stief_decode_latent" if args.latent else
                                                  "stief_append_decode_paged" if args.paged else
                                                  "stief_decode_attention" if args.unfused
@@ -567,7 +598,8 @@ def run_gpu(args, w: si.Workload):
             "peak_kind": f"{peak_kind} hbm_gbs (copy bandwidth, burst)",
             "unit": "GB/s",
             "frac": round(achieved / peak, 4),
-            "traffic": (None if (args.latent or args.unfused or args.int8 or args.paged)
+            "traffic": (None if (args.latent or args.unfused or args.int8 or args.paged
+                                 or args.joint)
                         else _traffic_per_launch(w.name)),
             "algorithmic_bytes": bytes_per_dec,
             "decode_us": round(dec_us, 3),
@@ -587,7 +619,7 @@ def run_gpu(args, w: si.Workload):
     if compress is not None:
         result["compress"] = compress
     if (rank == 0 and ws_n == 1 and not args.no_cpu_baseline
-            and not (args.latent or args.int8 or args.paged)):
+            and not (args.latent or args.int8 or args.paged or args.joint)):
         result["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     if ws_n > 1:
         torch.distributed.destroy_process_group()
@@ -814,6 +846,9 @@ def main():
     ap.add_argument("--latent", action="store_true",
                     help="time stief_decode_latent (bases folded into the attention weights) "
                          "instead of the fused append + decode step")
+    ap.add_argument("--joint", action="store_true",
+                    help="time stief_decode_attention_joint_v: per-head keys, one value latent "
+                         "per token shared by the KV heads (no append)")
     ap.add_argument("--paged", action="store_true",
                     help="time stief_append_decode_paged: the fused step over page pools "
                          f"({PAGE_SIZE}-token pages, shuffled block tables)")
@@ -828,10 +863,10 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    if sum(map(bool, (args.int8, args.latent, args.paged, args.unfused))) > 1:
-        ap.error("--int8, --latent, --paged and --unfused are separate modes")
-    if args.paged and args.profile_launches > 0:
-        ap.error("--profile-launches has no paged mode")
+    if sum(map(bool, (args.int8, args.latent, args.paged, args.joint, args.unfused))) > 1:
+        ap.error("--int8, --latent, --paged, --joint and --unfused are separate modes")
+    if (args.paged or args.joint) and args.profile_launches > 0:
+        ap.error("--profile-launches has no paged or joint mode")
     w = si.WORKLOADS[args.workload]
     if args.layers > 0:
         import dataclasses

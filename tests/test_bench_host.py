@@ -37,3 +37,18 @@ def test_to_pages_exact_pages_need_no_padding():
     pool, bt = bench.to_pages(cache, 128, perm)
     assert bt.tolist() == [[3, 0], [2, 1]]
     assert torch.equal(pool[3, 0], cache[0, 0, :128]) and torch.equal(pool[1, 0], cache[1, 0, 128:])
+
+
+def test_row_bytes_of_each_cache_form():
+    """Bytes per (token, sequence, KV head): bf16 rows, int8 rows with two fp32 scales, and
+    per-head keys plus one joint value row shared by the Hkv heads."""
+    import stief_inputs as si
+    w = si.WORKLOADS["llama3_8b_32k"]
+    assert bench.row_bytes_fn(w)(64, 64) == 256
+    assert bench.row_bytes_fn(w, int8=True)(64, 64) == 64 + 64 + 8
+    assert bench.row_bytes_fn(w, joint=True)(64, 64) == 2 * 64 + 2 * 64 / w.Hkv
+    # fewer bytes per step: at least as many replicas to keep the rotation above 3x L2
+    assert bench.replica_count(w, joint=True) >= bench.replica_count(w)
+    total = bench.replica_count(w, joint=True) * sum(
+        bench.row_bytes_fn(w, joint=True)(rK, rV) * w.B * w.Hkv * w.L for rK, rV in w.layer_ranks())
+    assert total >= bench.ROTATE_BYTES or bench.replica_count(w, joint=True) == bench.MAX_REPLICAS
