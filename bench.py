@@ -739,6 +739,19 @@ def _oracle_tokens_per_s(w: si.Workload, L_s: int, t_step: float) -> float:
     return w.B / (t_step * (w.L / L_s) * len(w.layer_ranks()))
 
 
+def _cpu_model() -> str:
+    """The host CPU's model name (first "model name" line of /proc/cpuinfo)."""
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
 def cpu_baseline(w: si.Workload, budget_s: float = 20.0):
     """The fp64 oracle (as it stands) on host cores, on a bounded sample of one step:
     layer 0, all sequences and heads, append 1 token + decode, at a context shortened
@@ -748,7 +761,7 @@ def cpu_baseline(w: si.Workload, budget_s: float = 20.0):
     L_s = _sample_context(w, budget_s / 2)
     t = _time_oracle(w, L_s, 0, 2)
     return {"value": round(_oracle_tokens_per_s(w, L_s, t), 4), "unit": "tokens/s",
-            "cores": threads, "kind": "oracle",
+            "cores": threads, "kind": "oracle", "cpu_model": _cpu_model(),
             "sample": f"layer 0, all {w.B} sequences x {w.Hq} heads, append 1 + decode at "
                       f"context {L_s} (of {w.L}), 2 steps of {t:.2f} s; scaled "
                       f"x{w.L / L_s:.2f} to the context and x{len(w.layer_ranks())} layers"}
@@ -817,7 +830,8 @@ def run_reference(args, w: si.Workload):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
                    "context": w.L, "layers": len(w.layer_ranks())},
-        "cpu_baseline": {"kind": "oracle", "cores": threads, "value": round(value, 4),
+        "cpu_baseline": {"kind": "oracle", "cores": threads, "cpu_model": _cpu_model(),
+                         "value": round(value, 4),
                          "unit": "tokens/s", "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},

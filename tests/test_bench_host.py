@@ -52,3 +52,11 @@ def test_row_bytes_of_each_cache_form():
     total = bench.replica_count(w, joint=True) * sum(
         bench.row_bytes_fn(w, joint=True)(rK, rV) * w.B * w.Hkv * w.L for rK, rV in w.layer_ranks())
     assert total >= bench.ROTATE_BYTES or bench.replica_count(w, joint=True) == bench.MAX_REPLICAS
+
+
+def test_cpu_baseline_reports_cores_and_cpu_model():
+    """The oracle's timed baseline names what it ran on (a short budget keeps this quick)."""
+    import stief_inputs as si
+    res = bench.cpu_baseline(si.WORKLOADS["tiny"], budget_s=0.5)
+    assert res["kind"] == "oracle" and res["cores"] >= 1 and res["value"] > 0
+    assert isinstance(res["cpu_model"], str) and res["cpu_model"]
