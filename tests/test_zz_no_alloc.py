@@ -4,8 +4,8 @@ It keeps its split partial states in a fixed device array owned by the library
 instead of a caller workspace.  These tests call it through the C ABI and check
 its output against stief_decode_attention (the workspace entry point) within the
 parity tolerance, on two calls in a row with different inputs, and that sizes
-beyond its fixed scratch are refused before anything is launched.  This file is
-collected last on purpose; it passes alone in a fresh process as well.
+beyond its fixed scratch are refused before anything is launched.  It passes alone in a
+fresh process as well as after the other GPU files.
 """
 import ctypes
 
