@@ -17,6 +17,7 @@ from ._binding import (  # noqa: F401
     stief_append_decode_paged,
     stief_compress_append,
     stief_compress_append_q8,
+    stief_compress_append_joint_v,
     stief_compress_append_paged,
     stief_decode_attention,
     stief_decode_attention_q8,

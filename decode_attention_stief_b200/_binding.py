@@ -89,6 +89,8 @@ def library() -> ctypes.CDLL:
             lib.stief_decode_attention_q8.restype = _i
             lib.stief_decode_attention_q8.argtypes = ([vp] * 10 + [ctypes.c_size_t] + [_i] * 9
                                                       + [vp, vp])
+            lib.stief_compress_append_joint_v.restype = _i
+            lib.stief_compress_append_joint_v.argtypes = [vp] * 7 + [_i] * 7 + [vp, vp]
             lib.stief_decode_attention_joint_v.restype = _i
             lib.stief_decode_attention_joint_v.argtypes = ([vp] * 8 + [ctypes.c_size_t] + [_i] * 9
                                                            + [vp, vp])
@@ -580,3 +582,30 @@ def stief_decode_latent_joint_v(q_lat: torch.Tensor, k_lat: torch.Tensor, v_join
                                                  _opt_status(dev_status), _stream_ptr(stream))
     _check("stief_decode_latent_joint_v", code)
     return out_lat
+
+
+def stief_compress_append_joint_v(k_new: torch.Tensor, v_new: torch.Tensor, P_K: torch.Tensor,
+                                  P_VJ: torch.Tensor, k_lat: torch.Tensor, v_joint: torch.Tensor,
+                                  seq_lens: torch.Tensor, dev_status: Optional[torch.Tensor] = None,
+                                  stream=None) -> None:
+    """stief_compress_append with the values projected jointly over the KV heads: keys per head
+    into k_lat [B][Hkv][L_max][rK], values through P_VJ [Hkv*d][rV] into v_joint [B][L_max][rV]
+    (one row per token); k_new, v_new [B][Hkv][T][d] bf16; seq_lens [B] int32 advanced by T."""
+    pk = _dev(k_new, "k_new", torch.bfloat16, 4)
+    pv = _dev(v_new, "v_new", torch.bfloat16, 4)
+    ppk = _dev(P_K, "P_K", torch.bfloat16, 3)
+    ppv = _dev(P_VJ, "P_VJ", torch.bfloat16, 2)
+    pkl = _dev(k_lat, "k_lat", torch.bfloat16, 4)
+    pvl = _dev(v_joint, "v_joint", torch.bfloat16, 3)
+    psl = _dev(seq_lens, "seq_lens", torch.int32, 1)
+    B, Hkv, T, d = k_new.shape
+    rK, rV = P_K.shape[2], P_VJ.shape[1]
+    L_max = k_lat.shape[2]
+    if tuple(v_new.shape) != (B, Hkv, T, d) or tuple(P_K.shape) != (Hkv, d, rK) \
+            or tuple(P_VJ.shape) != (Hkv * d, rV) or tuple(k_lat.shape) != (B, Hkv, L_max, rK) \
+            or tuple(v_joint.shape) != (B, L_max, rV) or seq_lens.shape[0] != B:
+        raise ValueError("stief_compress_append_joint_v: inconsistent shapes")
+    code = library().stief_compress_append_joint_v(pk, pv, ppk, ppv, pkl, pvl, psl, B, Hkv, T, d,
+                                                   rK, rV, L_max, _opt_status(dev_status),
+                                                   _stream_ptr(stream))
+    _check("stief_compress_append_joint_v", code)

@@ -301,6 +301,47 @@ stief_status stief_decode_latent(const uint16_t* q_lat, const uint16_t* k_lat,
                        num_splits, dev_status, stream, false, true);
 }
 
+stief_status stief_compress_append_joint_v(const uint16_t* k_new, const uint16_t* v_new,
+                                           const uint16_t* P_K, const uint16_t* P_VJ,
+                                           uint16_t* k_lat, uint16_t* v_joint, int32_t* seq_lens,
+                                           int B, int Hkv, int T, int d, int rK, int rV,
+                                           int L_max, uint32_t* dev_status,
+                                           stief_stream_t stream) {
+  if (!k_new || !v_new || !P_K || !P_VJ || !k_lat || !v_joint || !seq_lens)
+    return STIEF_ERR_INVALID_ARG;
+  if (B < 1 || B > 65535 || Hkv < 1 || Hkv > 65534 || T < 0 || d != kHeadDim || !rank_ok(rK) ||
+      !rank_ok(rV) || L_max < 1)
+    return STIEF_ERR_INVALID_ARG;
+  if (T > L_max) return STIEF_ERR_CAPACITY;
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(P_K) || !aligned16(P_VJ) ||
+      !aligned16(k_lat) || !aligned16(v_joint))
+    return STIEF_ERR_ALIGNMENT;
+  if (T == 0) return STIEF_OK;
+  int dev = 0;
+  const stief_status st = device_check(&dev);
+  if (st != STIEF_OK) return st;
+  stief::CompressArgs a{};
+  a.device = dev;
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.P_K = P_K;
+  a.P_V = P_VJ;
+  a.k_lat = k_lat;
+  a.v_lat = v_joint;
+  a.seq_lens = seq_lens;
+  a.dev_status = dev_status;
+  a.B = B;
+  a.Hkv = Hkv;
+  a.T = T;
+  a.d = d;
+  a.rK = rK;
+  a.rV = rV;
+  a.L_max = L_max;
+  if (stief::launch_compress_joint(a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return STIEF_ERR_CUDA;
+  return STIEF_OK;
+}
+
 stief_status stief_decode_attention_joint_v(const uint16_t* q, const uint16_t* P_K,
                                             const uint16_t* P_VJ, const uint16_t* k_lat,
                                             const uint16_t* v_joint, const int32_t* seq_lens,

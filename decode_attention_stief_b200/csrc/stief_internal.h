@@ -184,5 +184,8 @@ inline bool choose_decode_config(int rK, int rV, int tile, int* nwarps, int* nst
   return false;
 }
 cudaError_t launch_compress(const CompressArgs& a, cudaStream_t stream);
+// Joint value latents: keys per head into k_lat, the values of all KV heads of a token
+// through P_V = P_VJ [Hkv*d][rV] into v_lat = v_joint [B][L_max][rV]; then the lengths.
+cudaError_t launch_compress_joint(const CompressArgs& a, cudaStream_t stream);
 
 }  // namespace stief

@@ -361,9 +361,19 @@ STIEF_API stief_status stief_decode_attention_q8(const uint16_t* q, const uint16
  *   stief_decode_attention_joint_v: stief_decode_attention with v_lat -> v_joint and
  *       P_V -> P_VJ:  o_h = (sum_t p_t v_joint[t]) . (rows of KV head g of P_VJ)^T;
  *   stief_decode_latent_joint_v: stief_decode_latent with v_lat -> v_joint:
- *       o~_h = sum_t p_t v_joint[t].
+ *       o~_h = sum_t p_t v_joint[t];
+ *   stief_compress_append_joint_v: stief_compress_append with the values projected jointly,
+ *       v_joint[b][seq_lens[b] + t] = bf16_RNE( [v_new[b][0][t] | ... | v_new[b][Hkv-1][t]] . P_VJ )
+ *       (fp32 accumulation), keys per head as in stief_compress_append, then
+ *       seq_lens[b] += T; the same skipping and status bits for a full cache or a bad length.
+ *       CUDA cores only (no tensor-core path); B <= 65535.
  * B * L_max < 2^31 as for the per-head cache.  No fused append, paged or int8 form.
  */
+STIEF_API stief_status stief_compress_append_joint_v(
+    const uint16_t* k_new, const uint16_t* v_new, const uint16_t* P_K, const uint16_t* P_VJ,
+    uint16_t* k_lat, uint16_t* v_joint, int32_t* seq_lens, int B, int Hkv, int T, int d, int rK,
+    int rV, int L_max, uint32_t* dev_status, stief_stream_t stream);
+
 STIEF_API stief_status stief_decode_attention_joint_v(
     const uint16_t* q, const uint16_t* P_K, const uint16_t* P_VJ, const uint16_t* k_lat,
     const uint16_t* v_joint, const int32_t* seq_lens, uint16_t* out, void* workspace,

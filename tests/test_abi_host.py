@@ -142,6 +142,28 @@ def test_joint_value_decode_needs_both_bases(lib, kw):
     assert _joint(lib, **kw) == INVALID
 
 
+def _joint_compress(lib, **kw):
+    a = dict(k=FAKE, v=FAKE, P_K=FAKE, P_VJ=FAKE, kl=FAKE, vj=FAKE, sl=FAKE, B=1, Hkv=8, T=1,
+             d=128, rK=64, rV=64, L_max=1024)
+    a.update(kw)
+    return lib.stief_compress_append_joint_v(a["k"], a["v"], a["P_K"], a["P_VJ"], a["kl"],
+                                             a["vj"], a["sl"], a["B"], a["Hkv"], a["T"], a["d"],
+                                             a["rK"], a["rV"], a["L_max"], None, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(k=None), INVALID), (dict(P_VJ=None), INVALID), (dict(vj=None), INVALID),
+    (dict(sl=None), INVALID), (dict(d=64), INVALID), (dict(rK=8), INVALID), (dict(rV=136), INVALID),
+    (dict(B=0), INVALID), (dict(B=65536), INVALID), (dict(Hkv=0), INVALID), (dict(T=-1), INVALID),
+    (dict(L_max=0), INVALID), (dict(T=2000), CAPACITY), (dict(vj=FAKE + 2), ALIGN),
+    (dict(P_VJ=FAKE + 8), ALIGN), (dict(T=0), OK),
+])
+def test_joint_compress_argument_errors(lib, kw, code):
+    """T = 0 is a no-op that returns OK without touching CUDA; everything else is refused
+    before anything is launched."""
+    assert _joint_compress(lib, **kw) == code
+
+
 def _paged(lib, **kw):
     a = dict(q=FAKE, P_K=FAKE, P_V=FAKE, kp=FAKE, vp=FAKE, bt=FAKE, sl=FAKE, out=FAKE, ws=FAKE,
              ws_bytes=1 << 40, B=2, Hq=32, Hkv=8, d=128, rK=64, rV=64, num_pages=64,

@@ -148,3 +148,127 @@ def test_shape_errors_are_refused_before_launch():
     q, P_K, P_VJ, k, v = _case(1, 8, 2, 32, 32, 64, 7800)
     with pytest.raises(ValueError):   # a per-head value cache where the joint one is expected
         _gpu_joint(q, P_K, P_VJ, k, k, [64])
+
+
+# ----------------------------------------------------------------------------- joint compress
+
+CANARY = 0x7FC1  # a quiet-NaN bf16 pattern: any stray write changes it
+
+
+def _canary(shape):
+    t = torch.full(shape, CANARY, dtype=torch.int16, device=DEV)
+    return t.view(torch.bfloat16)
+
+
+def _compress_joint(k_new, v_new, P_K, P_VJ, L_max, lens):
+    B, Hkv, T, d = k_new.shape
+    rK, rV = P_K.shape[2], P_VJ.shape[1]
+    k_lat = _canary((B, Hkv, L_max, rK))
+    v_joint = _canary((B, L_max, rV))
+    lens_t = torch.as_tensor(np.asarray(lens, np.int32)).to(DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    stief.stief_compress_append_joint_v(k_new.to(DEV), v_new.to(DEV), P_K.to(DEV), P_VJ.to(DEV),
+                                        k_lat, v_joint, lens_t, dev_status=status)
+    st = stief.stief_read_device_status(status)
+    return k_lat.cpu(), v_joint.cpu(), lens_t.cpu().numpy(), st
+
+
+def _selector_basis(Hkv, d, r):
+    """[Hkv*d][r] with column c = the unit vector of head c % Hkv, dimension c // Hkv: every
+    stored coordinate is one input coordinate, from heads in turn (exact in bf16)."""
+    P = np.zeros((Hkv * d, r))
+    for c in range(r):
+        P[(c % Hkv) * d + c // Hkv, c] = 1.0
+    return si.to_bf16(P)
+
+
+@pytest.mark.parametrize("T", [1, 5, 8, 20])
+def test_compress_selector_bases_bit_exact(T):
+    """Selector bases: each stored value is one input coordinate, so the GPU's rows equal the
+    oracle's bit for bit (which head each column reads is fixed by the concatenation order)."""
+    B, Hkv, d, rK, rV, L_max = 2, 4, 128, 32, 48, 40
+    k_new, v_new = si.full_kv(7900 + T, B, Hkv, T, d)
+    P_K = torch.stack([_selector_basis(1, d, rK) for _ in range(Hkv)])
+    P_VJ = _selector_basis(Hkv, d, rV)
+    lens = [0, 11]
+    gk, gv, glens, st = _compress_joint(k_new, v_new, P_K, P_VJ, L_max, lens)
+    assert st == 0 and glens.tolist() == [L + T for L in lens]
+    wk, wv, wl, nbad = oracle.compress_append_joint_v(
+        f64(k_new), f64(v_new), f64(P_K), f64(P_VJ), np.zeros((B, Hkv, L_max, rK)),
+        np.zeros((B, L_max, rV)), np.asarray(lens, np.int32))
+    assert nbad == 0 and wl.tolist() == glens.tolist()
+    for b, L in enumerate(lens):
+        assert np.array_equal(f64(gk[b, :, L:L + T]), wk[b, :, L:L + T])
+        assert np.array_equal(f64(gv[b, L:L + T]), wv[b, L:L + T])
+        keep = np.ones(L_max, bool)
+        keep[L:L + T] = False
+        assert torch.all(gk[b][:, keep].view(torch.int16) == CANARY)
+        assert torch.all(gv[b][keep].view(torch.int16) == CANARY)
+
+
+@pytest.mark.parametrize("T", [3, 130])
+def test_compress_general_bases_within_the_fp32_bound(T):
+    """General bases: the fp32 sum of Hkv*d products, rounded once to bf16, against the exact
+    product: within half a bf16 ulp plus the fp32 accumulation bound K * 2^-23 * sum|x||p|."""
+    B, Hkv, d, rK, rV, L_max = 1, 8, 128, 64, 64, 160
+    k_new, v_new = si.full_kv(8000 + T, B, Hkv, T, d)
+    P_K = si.to_bf16(si.bases(8000, Hkv, d, rK))
+    P_VJ = si.to_bf16(si.bases(8001, 1, Hkv * d, rV)[0])
+    gk, gv, glens, st = _compress_joint(k_new, v_new, P_K, P_VJ, L_max, [7])
+    assert st == 0 and glens.tolist() == [7 + T]
+    x = np.ascontiguousarray(np.transpose(f64(v_new[0]), (1, 0, 2)).reshape(T, Hkv * d))
+    P = f64(P_VJ)
+    exact = x @ P
+    bound = 2.0 ** -8 * np.abs(exact) + Hkv * d * 2.0 ** -23 * (np.abs(x) @ np.abs(P)) + 1e-30
+    got = f64(gv[0, 7:7 + T])
+    assert np.all(np.abs(got - exact) <= bound)
+    want = oracle.compress_append_joint_v(f64(k_new), f64(v_new), f64(P_K), f64(P_VJ),
+                                          np.zeros((B, Hkv, L_max, rK)), np.zeros((B, L_max, rV)),
+                                          np.array([7], np.int32))[1][0, 7:7 + T]
+    assert np.mean(got == want) > 0.95
+    for h in range(Hkv):
+        ek = f64(k_new[0, h]) @ f64(P_K[h])
+        kb = 2.0 ** -8 * np.abs(ek) + d * 2.0 ** -23 * (np.abs(f64(k_new[0, h])) @ np.abs(f64(P_K[h])))
+        assert np.all(np.abs(f64(gk[0, h, 7:7 + T]) - ek) <= kb + 1e-30)
+
+
+def test_compress_refuses_full_and_bad_sequences():
+    """A sequence whose rows would pass L_max, and one with a negative length, are skipped
+    (nothing written, length unchanged) and reported; the others are appended."""
+    B, Hkv, d, rK, rV, L_max, T = 3, 2, 128, 32, 32, 16, 4
+    k_new, v_new = si.full_kv(8100, B, Hkv, T, d)
+    P_K = si.to_bf16(si.bases(8100, Hkv, d, rK))
+    P_VJ = si.to_bf16(si.bases(8101, 1, Hkv * d, rV)[0])
+    gk, gv, glens, st = _compress_joint(k_new, v_new, P_K, P_VJ, L_max, [13, -1, 12])
+    assert st == (stief.DEV_CAPACITY_OVERFLOW | stief.DEV_BAD_LENGTH)
+    assert glens.tolist() == [13, -1, 16]
+    for b in (0, 1):
+        assert torch.all(gk[b].view(torch.int16) == CANARY)
+        assert torch.all(gv[b].view(torch.int16) == CANARY)
+    assert not torch.any(gv[2, 12:16].view(torch.int16) == CANARY)
+
+
+def test_compress_then_decode_joint_end_to_end():
+    """A prefill chunk and one decode-step token into a joint cache, then the joint decode,
+    against the oracle's joint compress and decode."""
+    B, Hq, Hkv, d, rK, rV, L_max = 2, 32, 8, 128, 64, 96, 200
+    k_pre, v_pre = si.full_kv(8200, B, Hkv, 150, d)
+    k_new, v_new = si.full_kv(8201, B, Hkv, 1, d)
+    P_K = si.to_bf16(si.bases(8200, Hkv, d, rK))
+    P_VJ = si.to_bf16(si.bases(8202, 1, Hkv * d, rV)[0])
+    k_lat = torch.zeros((B, Hkv, L_max, rK), dtype=torch.bfloat16, device=DEV)
+    v_joint = torch.zeros((B, L_max, rV), dtype=torch.bfloat16, device=DEV)
+    lens = torch.tensor([0, 40], dtype=torch.int32, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    wk, wv = np.zeros((B, Hkv, L_max, rK)), np.zeros((B, L_max, rV))
+    wl = np.array([0, 40], np.int32)
+    for kk, vv in ((k_pre, v_pre), (k_new, v_new)):
+        stief.stief_compress_append_joint_v(kk.to(DEV), vv.to(DEV), P_K.to(DEV), P_VJ.to(DEV),
+                                            k_lat, v_joint, lens, dev_status=status)
+        wk, wv, wl, _ = oracle.compress_append_joint_v(f64(kk), f64(vv), f64(P_K), f64(P_VJ),
+                                                       wk, wv, wl)
+    assert stief.stief_read_device_status(status) == 0
+    assert lens.cpu().tolist() == wl.tolist() == [151, 191]
+    q = si.queries(8203, B, Hq, d)
+    got = _gpu_joint(q, P_K, P_VJ, k_lat, v_joint, wl.tolist(), max_seq_len=L_max)
+    assert_decode_close(got, oracle.decode_joint_v(f64(q), f64(P_K), f64(P_VJ), wk, wv, wl))
