@@ -40,6 +40,11 @@ def test_every_declared_symbol_is_exported(lib):
     assert not missing, f"not exported: {missing}"
 
 
+def test_every_declared_call_has_a_binding_of_the_same_name():
+    missing = [n for n in declared_functions() if not callable(getattr(stief, n, None))]
+    assert not missing, f"no Python binding: {missing}"
+
+
 def test_only_declared_symbols_are_exported():
     out = os.popen(f"nm -D --defined-only {stief.library_path()}").read()
     exported = set(re.findall(r"\b(stief_[a-z_0-9]+)\b", out))
