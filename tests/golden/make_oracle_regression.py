@@ -61,12 +61,14 @@ def results(o=None):
         x["k_new"], x["v_new"], x["P_K"], x["P_VJ"], np.zeros((B, Hkv, L_max, rK)),
         np.zeros((B, L_max, 2 * rV)), lens0)
     out_j = o.decode_joint_v(x["q"], x["P_K"], x["P_VJ"], kj, vj, dl)
+    codes, scales = oracle.quantize_rows(k_lat)  # the int8 form of the key cache
     return {
         "compress_k_lat": k_lat, "compress_v_lat": v_lat,
         "compress_lens": lens.astype(np.float64), "compress_overflow": np.array([float(nbad)]),
         "decode_out": out, "decode_latent_out": out_lat,
         "joint_v_cache": vj, "joint_v_lens": lj.astype(np.float64),
         "joint_v_overflow": np.array([float(nbj)]), "decode_joint_v_out": out_j,
+        "int8_codes": codes.astype(np.float64), "int8_scales": scales.astype(np.float64),
     }
 
 
