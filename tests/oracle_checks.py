@@ -128,6 +128,25 @@ def check_full_rank_is_plain_attention(o, q_scale: float = 1.0, d: int = 128,
     assert err <= tol, f"r=d differs from plain attention: rel err {err}"
 
 
+def check_tiny_compressed_is_sdpa_on_reconstructed_rows(o) -> None:
+    """Brute force on tiny inputs with r < d (d = 16, r_K = 8, r_V = 4, up to 5 tokens): the
+    rows K~ = K_down P_K^T and V~ = V_down P_V^T formed explicitly (numpy products), then torch
+    SDPA in float64 over them, must equal the oracle's decode to 1e-13."""
+    d, rK, rV, B, Hq, Hkv, L_max = 16, 8, 4, 3, 4, 2, 5
+    rng = np.random.default_rng(40)
+    lens = np.array([5, 1, 3], np.int32)
+    P_K = si.bases(41, Hkv, d, rK)
+    P_V = si.bases(42, Hkv, d, rV)
+    k = rng.standard_normal((B, Hkv, L_max, rK))
+    v = rng.standard_normal((B, Hkv, L_max, rV))
+    q = rng.standard_normal((B, Hq, d))
+    K = np.einsum("bhtr,hdr->bhtd", k, P_K)
+    V = np.einsum("bhtr,hdr->bhtd", v, P_V)
+    want = _sdpa_reference(q, K, V, lens)
+    got = o.decode(q, P_K, P_V, k, v, lens)
+    assert _rel_err(got, want) <= 1e-13
+
+
 def check_gauge_invariance(o, r: int = 48, d: int = 128) -> None:
     """P -> P.O (O orthogonal r x r) leaves the output unchanged (QR: R is a change of coordinates)."""
     B, Hq, Hkv, L = 2, 4, 2, 29
@@ -526,6 +545,8 @@ ALL_ORACLE_CHECKS = {
     # scores in the hundreds: exp() overflows unless the maximum is subtracted first
     "full_rank_large_scores": lambda o: check_full_rank_is_plain_attention(o, q_scale=400.0,
                                                                            tol=1e-10),
+    "tiny_compressed_is_sdpa_on_reconstructed_rows":
+        check_tiny_compressed_is_sdpa_on_reconstructed_rows,
     "gauge_invariance": check_gauge_invariance,
     "single_token": check_single_token,
     "two_tokens": check_two_tokens,

@@ -60,3 +60,20 @@ def test_cpu_baseline_reports_cores_and_cpu_model():
     res = bench.cpu_baseline(si.WORKLOADS["tiny"], budget_s=0.5)
     assert res["kind"] == "oracle" and res["cores"] >= 1 and res["value"] > 0
     assert isinstance(res["cpu_model"], str) and res["cpu_model"]
+
+
+def test_algorithmic_bytes_follow_the_footprint_formula():
+    """The bench's algorithmic bytes per decode are the latent footprint 2 (r_K + r_V) bytes per
+    (token, KV head, sequence): 64 MiB at batch 1, 8 KV heads, 32768 tokens, ranks 64/64;
+    160 MiB at 131072 tokens, ranks 32/48; 512 MiB at batch 64, 4096 tokens, ranks 64/64;
+    256 KiB for one KV head at 1024 tokens.  Against the full bf16 cache (2 * d * 2 bytes per
+    token and KV head) the ranks 64/64 keep half the bytes."""
+    import stief_inputs as si
+    W = si.WORKLOADS
+    per_launch = lambda w: bench.row_bytes_fn(w)(*w.layer_ranks()[0]) * w.B * w.Hkv * w.L
+    assert per_launch(W["llama3_8b_32k"]) == 64 * 2**20
+    assert per_launch(W["llama31_8b_128k"]) == 160 * 2**20
+    assert per_launch(W["prefill_b64"]) == 512 * 2**20
+    assert per_launch(W["tiny"]) == 256 * 2**10
+    w = W["llama3_8b_32k"]
+    assert bench.row_bytes_fn(w)(64, 64) * 2 == 2 * w.d * 2

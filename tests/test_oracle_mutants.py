@@ -22,23 +22,28 @@ ROOT = os.path.dirname(TESTS)
 
 # (name, original text, replacement, checks expected to fail)
 MUTANTS = [
-    ("scale_uses_rank", "1.0 / sqrt((double)d)", "1.0 / sqrt((double)rK)", ["two_tokens"]),
-    ("gqa_interleaved", "(long)g * G + j", "(long)j * Hkv + g", ["full_rank_is_plain_attention"]),
+    ("scale_uses_rank", "1.0 / sqrt((double)d)", "1.0 / sqrt((double)rK)",
+     ["two_tokens", "tiny_compressed_is_sdpa_on_reconstructed_rows"]),
+    ("gqa_interleaved", "(long)g * G + j", "(long)j * Hkv + g",
+     ["full_rank_is_plain_attention", "tiny_compressed_is_sdpa_on_reconstructed_rows"]),
     ("reconstruct_transposed", "acc += lat[c] * P[(long)i * r + c];",
-     "acc += lat[c] * P[(long)c * d + i];", ["single_token", "gauge_invariance"]),
+     "acc += lat[c] * P[(long)c * d + i];",
+     ["single_token", "gauge_invariance", "tiny_compressed_is_sdpa_on_reconstructed_rows"]),
     ("compress_transposed", "acc += x[t * d + i] * P[(long)i * r + c];",
      "acc += x[t * d + i] * P[(long)c * d + i];",
      ["compress_identity_basis", "full_rank_is_plain_attention"]),
     ("no_max_subtraction", "sj[t] = exp(sj[t] - mx);", "sj[t] = exp(sj[t]);",
      ["full_rank_large_scores"]),
     ("unnormalised_weights", "double p = s[(long)j * L + t] / denom[j];",
-     "double p = s[(long)j * L + t];", ["two_tokens", "uniform_keys"]),
+     "double p = s[(long)j * L + t];",
+     ["two_tokens", "uniform_keys", "tiny_compressed_is_sdpa_on_reconstructed_rows"]),
     ("values_use_key_basis", "reconstruct_row(Vd + t * rV, PV, d, rV, row);",
-     "reconstruct_row(Vd + t * rV, PK, d, rV, row);", ["full_rank_is_plain_attention"]),
+     "reconstruct_row(Vd + t * rV, PK, d, rV, row);",
+     ["full_rank_is_plain_attention", "tiny_compressed_is_sdpa_on_reconstructed_rows"]),
     ("first_value_dropped",
      "for (long t = 0; t < L; ++t) {\n            reconstruct_row(Vd",
      "for (long t = 1; t < L; ++t) {\n            reconstruct_row(Vd",
-     ["single_token", "two_tokens"]),
+     ["single_token", "two_tokens", "tiny_compressed_is_sdpa_on_reconstructed_rows"]),
     ("latent_scale_uses_rank", "w_lat[t] = acc * inv_sqrt_d;",
      "w_lat[t] = acc / sqrt((double)rK);", ["latent_is_sdpa_on_latent_rows"]),
     ("latent_gqa_interleaved", "const long head = (long)b * Hq + (long)g * G + j;",
