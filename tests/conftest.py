@@ -10,7 +10,8 @@ if ROOT not in sys.path:
 # Files collected after all others, in this order: the no-allocation entry point, then the
 # newest GPU paths (whose cases had not yet run on a GPU when they were written).  With -x a
 # failure in one of the newest then cannot hide the results of the established files.
-RUN_LAST = ("test_zz_no_alloc.py", "test_joint_gpu.py", "test_bench_modes_gpu.py")
+RUN_LAST = ("test_zz_no_alloc.py", "test_gauge_gpu.py", "test_joint_gpu.py",
+            "test_bench_modes_gpu.py")
 
 
 def pytest_configure(config):
