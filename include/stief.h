@@ -26,7 +26,8 @@
  *   - Calls are asynchronous on `stream` (NULL = the legacy default stream).
  *     A call that returns an error from argument checking launches nothing.
  *   - Supported: d == 128; 16 <= r_K, r_V <= 128 with r % 16 == 0; Hq % Hkv == 0;
- *     1 <= Hq / Hkv <= 64; B, Hkv >= 1.
+ *     1 <= Hq / Hkv <= 64; B, Hkv >= 1; for the decode calls B <= 65535 and
+ *     B * Hkv * L_max < 2^31 (cache rows are addressed with 32-bit copy coordinates).
  *   - `dev_status` (may be NULL) is a device uint32 word.  Kernels OR the
  *     STIEF_DEV_* bits below into it when they meet a condition that host-side
  *     checks cannot see.  The library never clears it: the caller zeroes it
@@ -367,7 +368,8 @@ STIEF_API stief_status stief_decode_attention_q8(const uint16_t* q, const uint16
  *       (fp32 accumulation), keys per head as in stief_compress_append, then
  *       seq_lens[b] += T; the same skipping and status bits for a full cache or a bad length.
  *       CUDA cores only (no tensor-core path); B <= 65535.
- * B * L_max < 2^31 as for the per-head cache.  No fused append, paged or int8 form.
+ * The key cache has the per-head limits (B * Hkv * L_max < 2^31).  No fused append, paged or
+ * int8 form.
  */
 STIEF_API stief_status stief_compress_append_joint_v(
     const uint16_t* k_new, const uint16_t* v_new, const uint16_t* P_K, const uint16_t* P_VJ,
