@@ -194,6 +194,19 @@ def build_state(w: si.Workload, total_steps: int, seed: int, dev):
     return layers, L_max
 
 
+def step_call(args) -> str:
+    """The API call whose kernel a step of the chosen mode runs (one per layer)."""
+    if args.int8:
+        return "stief_decode_attention_q8"
+    if args.joint:
+        return "stief_decode_latent_joint_v" if args.latent else "stief_decode_attention_joint_v"
+    if args.latent:
+        return "stief_decode_latent"
+    if args.paged:
+        return "stief_append_decode_paged"
+    return "stief_decode_attention" if args.unfused else "stief_append_decode"
+
+
 def row_bytes_fn(w: si.Workload, int8: bool = False, joint: bool = False):
     """Cache bytes per (token, sequence, KV head) for a layer of ranks (rK, rV): bf16 rows, int8
     rows with their two fp32 scales, or per-head keys with one joint value row shared by the
@@ -310,6 +323,10 @@ def run_gpu(args, w: si.Workload):
             stief.stief_decode_attention_q8(q_s, lay.P_K, lay.P_V, lay.kq, lay.vq, lay.ks, lay.vs,
                                             lay.seq_lens, out[li], lay.ws, max_seq_len=L_max,
                                             num_splits=args.splits, dev_status=status)
+        elif args.latent and args.joint:  # latent output over the joint value latent
+            stief.stief_decode_latent_joint_v(qlat_s[li], lay.k_lat, lay.v_joint, lay.seq_lens,
+                                              olat[li], lay.ws, max_seq_len=L_max,
+                                              num_splits=args.splits, dev_status=status)
         elif args.latent:  # attention in the latent space only (no projections, no append)
             stief.stief_decode_latent(qlat_s[li], lay.k_lat, lay.v_lat, lay.seq_lens, olat[li],
                                       lay.ws, max_seq_len=L_max, num_splits=args.splits,
@@ -558,7 +575,8 @@ def run_gpu(args, w: si.Workload):
             "step": (("decode over an int8 latent cache (codes + fp32 row scales, synthetic "
                       "values), no append, every layer; " if args.int8 else
                       "decode with per-head keys and one joint value latent per token shared by "
-                      "the KV heads, no append, every layer; " if args.joint else
+                      "the KV heads" + (" (latent output)" if args.latent else "") +
+                      ", no append, every layer; " if args.joint else
                       "latent decode only (bases folded into the attention weights: q~ in, "
                       "o~ out; the new token's latent rows would come from the folded K/V "
                       "projection), every layer; " if args.latent else
@@ -568,12 +586,8 @@ def run_gpu(args, w: si.Workload):
                       "append 1 token per (sequence, KV head) + decode, every layer; ") +
                      "the API calls captured in CUDA graphs (one step per replica, the timed "
                      "region replays the replica cycle back to back); " +
-                     ("stief_decode_attention_q8 (1 kernel per layer)" if args.int8 else
-                      "stief_decode_attention_joint_v (1 kernel per layer)" if args.joint else
-                      "stief_decode_latent (1 kernel per layer)" if args.latent else
-                      "stief_append_decode_paged (1 kernel per layer)" if args.paged else
-                      "stief_compress_append + stief_decode_attention (3 kernels per layer)"
-                      if args.unfused else "stief_append_decode (1 kernel per layer)")),
+                     ("stief_compress_append + stief_decode_attention (3 kernels per layer)"
+                      if args.unfused else f"{step_call(args)} (1 kernel per layer)")),
             "context_growth": (f"none (context {w.L} every step)"
                                if args.latent or args.int8 or args.joint else
                                f"+1 token per step of a replica (contexts {ctx_first}..{ctx_last})"),
@@ -586,12 +600,7 @@ def run_gpu(args, w: si.Workload):
         },
         "hbm_gbs_step": round(step_bytes / (ms_per_step / 1e3) / 1e9, 1),
         "roofline": {
-            "kernel": "stief_decode_kernel (" + ("stief_decode_attention_q8" if args.int8 else
-                                                 "stief_decode_attention_joint_v" if args.joint else
-                                                 "stief_decode_latent" if args.latent else
-                                                 "stief_append_decode_paged" if args.paged else
-                                                 "stief_decode_attention" if args.unfused
-                                                 else "stief_append_decode") + ")",
+            "kernel": f"stief_decode_kernel ({step_call(args)})",
             "bound": "hbm",
             "achieved": round(achieved, 1),
             "peak": peak,
@@ -877,8 +886,10 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    if sum(map(bool, (args.int8, args.latent, args.paged, args.joint, args.unfused))) > 1:
-        ap.error("--int8, --latent, --paged, --joint and --unfused are separate modes")
+    modes = [m for m in ("int8", "latent", "paged", "joint", "unfused") if getattr(args, m)]
+    if len(modes) > 1 and modes != ["latent", "joint"]:
+        ap.error("--int8, --latent, --paged, --joint and --unfused are separate modes "
+                 "(--latent --joint together time the latent joint-value decode)")
     if (args.paged or args.joint) and args.profile_launches > 0:
         ap.error("--profile-launches has no paged or joint mode")
     w = si.WORKLOADS[args.workload]

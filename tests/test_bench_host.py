@@ -77,3 +77,18 @@ def test_algorithmic_bytes_follow_the_footprint_formula():
     assert per_launch(W["tiny"]) == 256 * 2**10
     w = W["llama3_8b_32k"]
     assert bench.row_bytes_fn(w)(64, 64) * 2 == 2 * w.d * 2
+
+
+def test_step_call_names_the_api_call_of_each_mode():
+    class A:
+        int8 = latent = paged = joint = unfused = False
+    cases = [({}, "stief_append_decode"), ({"unfused": True}, "stief_decode_attention"),
+             ({"latent": True}, "stief_decode_latent"), ({"int8": True}, "stief_decode_attention_q8"),
+             ({"paged": True}, "stief_append_decode_paged"),
+             ({"joint": True}, "stief_decode_attention_joint_v"),
+             ({"joint": True, "latent": True}, "stief_decode_latent_joint_v")]
+    for flags, want in cases:
+        a = A()
+        for k, v in flags.items():
+            setattr(a, k, v)
+        assert bench.step_call(a) == want

@@ -1,5 +1,5 @@
-"""bench.py's paged and joint-value modes run end to end on a small workload and print one
-JSON line with the contract's keys (the timing itself is not checked here)."""
+"""bench.py's paged and joint-value modes (full and latent output) run end to end on a small
+workload and print one JSON line with the contract's keys (the timing itself is not checked)."""
 import json
 import os
 import subprocess
@@ -11,10 +11,11 @@ pytestmark = pytest.mark.gpu
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-@pytest.mark.parametrize("mode,call", [("--paged", "stief_append_decode_paged"),
-                                       ("--joint", "stief_decode_attention_joint_v")])
+@pytest.mark.parametrize("mode,call", [(["--paged"], "stief_append_decode_paged"),
+                                       (["--joint"], "stief_decode_attention_joint_v"),
+                                       (["--latent", "--joint"], "stief_decode_latent_joint_v")])
 def test_bench_mode_runs(mode, call):
-    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), mode, "--workload", "tiny",
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), *mode, "--workload", "tiny",
            "--steps", "3", "--warmup", "3", "--decode-iters", "3", "--no-cpu-baseline",
            "--clock-window", "0"]
     run = subprocess.run(cmd, capture_output=True, text=True, timeout=600, cwd=ROOT)
