@@ -17,10 +17,13 @@
 //     0, D_V at column 128);
 //   - epilogue: each of 4 warps reads its 32 TMEM lanes (rows) with tcgen05.ld, rounds
 //     to bf16 (RNE) and stores its rows into the latent cache at seq_lens[b] + row.
-// A CTA loops over m-tiles of one (b, h) so P is staged once.  Its X tiles stream
-// through a two-stage ring: the first two are requested at kernel entry (the bases are
-// staged and the length is read while they fly), and the copy of tile i + 2 is issued as
-// soon as tile i's MMA has consumed its stage, so loads overlap the MMA and the epilogue.
+// A CTA loops over m-tiles of one (b, h) so P is staged once.  The kernel is launched as a
+// programmatic dependent: barrier set-up, the tensor-memory allocation and the staging of
+// the bases (weights, which the preceding kernel must not write) overlap the preceding
+// kernel's tail; the new rows and the lengths are read only after the dependency wait.  Its
+// X tiles stream through a two-stage ring: the first two are requested right after the wait
+// (the length is read while they fly), and the copy of tile i + 2 is issued as soon as tile
+// i's MMA has consumed its stage, so loads overlap the MMA and the epilogue.
 // Every wait is bounded; every requested copy lands and tensor memory is released before
 // the CTA exits.
 #include <cstdint>
@@ -196,8 +199,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (tid == 0) {
     for (int st = 0; st < kTcStages + 1; ++st) mbar_init(&tma_bar[st], 1);
     fence_barrier_init();
-    // the first tiles fly while the bases are staged and the length is read
-    for (int i = 0; i < kTcStages && i < my_tiles; ++i) issue(i);
   }
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -208,6 +209,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
   stage_bases(smem, L.pk, L.pv, a.P_K + (size_t)h * 128 * rK, a.P_V + (size_t)h * 128 * rV, rK, rV,
               tid);
+  __syncthreads();  // the barriers are initialised
+  // the new rows and the lengths may come from the preceding kernel: read nothing before this
+  pdl_wait();
+  if (tid == 0)  // the first tiles fly while the length is read
+    for (int i = 0; i < kTcStages && i < my_tiles; ++i) issue(i);
   const int Lb = a.seq_lens[b];
   const bool bad = Lb < 0 || Lb > a.L_max;
   const CacheRows cr{a.block_table, a.max_pages, a.page_size, a.num_pages, a.Hkv, a.L_max};
@@ -361,8 +367,19 @@ cudaError_t launch_compress_tc(const CompressArgs& a, cudaStream_t stream) {
   static SmemLimit limit;
   cudaError_t e = limit.ensure(reinterpret_cast<const void*>(stief_compress_tc_kernel), dev, (int)smem);
   if (e != cudaSuccess) return e;
-  stief_compress_tc_kernel<<<dim3(gx, a.Hkv, a.B), kTcThreads, smem, stream>>>(ta);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(gx, a.Hkv, a.B);
+  cfg.blockDim = dim3(kTcThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  // programmatic dependent launch: the CTAs may start while the preceding kernel drains and
+  // wait for it (griddepcontrol.wait) before reading the new rows or the lengths
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, stief_compress_tc_kernel, ta);
 }
 
 }  // namespace stief
