@@ -86,8 +86,11 @@ def _hbm_peak():
 
 
 def _kernel_source_hash() -> str:
-    p = os.path.join(ROOT, "decode_attention_stief_b200", "csrc", "decode_kernels.cu")
-    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+    """Hash of the decode kernel's device code (the kernel template and its device helpers)."""
+    h = hashlib.sha256()
+    for name in ("decode_kernel.cuh", "stief_device.cuh"):
+        h.update(open(os.path.join(ROOT, "decode_attention_stief_b200", "csrc", name), "rb").read())
+    return h.hexdigest()[:16]
 
 
 def _traffic_per_launch(workload: str):
@@ -228,6 +231,53 @@ def replica_count(w: si.Workload, int8: bool = False, joint: bool = False) -> in
     return 1 if per >= ROTATE_BYTES else min(MAX_REPLICAS, -(-ROTATE_BYTES // per))
 
 
+def step_description(args) -> str:
+    """What one timed step runs, in words (the same text in both arms)."""
+    if args.int8:
+        what = ("decode over an int8 latent cache (codes + fp32 row scales, synthetic values), "
+                "no append, every layer; ")
+    elif args.joint:
+        what = ("decode with per-head keys and one joint value latent per token shared by the "
+                "KV heads" + (" (latent output)" if args.latent else "") + ", no append, every "
+                "layer; ")
+    elif args.latent:
+        what = ("latent decode only (bases folded into the attention weights: q~ in, o~ out; the "
+                "new token's latent rows would come from the folded K/V projection), every "
+                "layer; ")
+    elif args.paged:
+        what = (f"append 1 token per (sequence, KV head) + decode over page pools ({PAGE_SIZE}-"
+                f"token pages at shuffled pool positions), every layer; ")
+    else:
+        what = "append 1 token per (sequence, KV head) + decode, every layer; "
+    how = ("the API calls captured in CUDA graphs (one step per replica, the timed region "
+           "replays the replica cycle back to back); ")
+    calls = ("stief_compress_append + stief_decode_attention (3 kernels per layer)"
+             if args.unfused else f"{step_call(args)} (1 kernel per layer)")
+    return what + how + calls
+
+
+def config_dict(w: si.Workload, args, world: int) -> dict:
+    """The workload and how it is run: identical in the GPU arm and the reference arm."""
+    R = replica_count(w, args.int8, args.joint)
+    rb = row_bytes_fn(w, args.int8, args.joint)
+    rot_mb = R * sum(rb(rK, rV) * w.B * w.Hkv * w.L for rK, rV in w.layer_ranks()) / 2**20
+    appends = not (args.latent or args.int8 or args.joint)
+    ranks = [list(r) for r in w.layer_ranks()]
+    return {
+        "workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "context": w.L,
+        "layers": len(ranks), "ranks": ranks[:4] + (["..."] if len(ranks) > 4 else []),
+        "step": step_description(args),
+        "context_growth": (f"+1 token per step of a replica, from context {w.L}" if appends
+                           else f"none (context {w.L} every step)"),
+        "l2": (f"no flush: steps rotate over {R} copies of the layer caches ({rot_mb:.0f} MiB in "
+               f"all, > 3x the 126 MB L2)" if R > 1 else
+               f"no flush: one step reads {rot_mb:.0f} MiB of caches (> 3x the 126 MB L2)"
+               if rot_mb * 2**20 >= ROTATE_BYTES else
+               f"inputs ({rot_mb:.1f} MiB in {R} copies) fit in L2: a latency case"),
+        "parallelism": f"independent sequences per GPU x{world}",
+    }
+
+
 def to_pages(cache: torch.Tensor, page_size: int, perm: torch.Tensor):
     """A contiguous latent cache [B][Hkv][L][r] as a page pool and block table.
 
@@ -272,15 +322,26 @@ def run_gpu(args, w: si.Workload):
     layers = reps[0]
     g = torch.Generator(device=dev)
     g.manual_seed(seed + 1)
-    # the step's inputs live in fixed device buffers (filled by H2D copies in the e2e path)
-    q_s = torch.randn((w.B, w.Hq, w.d), generator=g, device=dev).to(torch.bfloat16)
-    k_s = torch.randn((w.B, w.Hkv, 1, w.d), generator=g, device=dev).to(torch.bfloat16)
-    v_s = torch.randn((w.B, w.Hkv, 1, w.d), generator=g, device=dev).to(torch.bfloat16)
+    # The step's inputs live in one device staging buffer, filled by one H2D copy per step in
+    # the end-to-end timing: q [B][Hq][d], then the new token's k and v rows [B][Hkv][1][d]
+    # (latent mode: q~ [B][Hq][r_K] of every layer, one after the other).  Every view starts
+    # on a 32-byte boundary.
+    if args.latent:
+        sizes = [w.B * w.Hq * lay.rK for lay in layers]
+    else:
+        sizes = [w.B * w.Hq * w.d, w.B * w.Hkv * w.d, w.B * w.Hkv * w.d]
+    inp = torch.randn((sum(sizes),), generator=g, device=dev).to(torch.bfloat16)
+    views = list(torch.split(inp, sizes))
+    if args.latent:
+        qlat_s = [v.view(w.B, w.Hq, lay.rK) for v, lay in zip(views, layers)]
+        q_s = k_s = v_s = None
+    else:
+        qlat_s = []
+        q_s = views[0].view(w.B, w.Hq, w.d)
+        k_s = views[1].view(w.B, w.Hkv, 1, w.d)
+        v_s = views[2].view(w.B, w.Hkv, 1, w.d)
     out = torch.empty((len(layers), w.B, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
-    # latent mode (bases folded into the attention weights): q~ in, o~ out, per layer
-    qlat_s = [torch.randn((w.B, w.Hq, lay.rK), generator=g, device=dev).to(torch.bfloat16)
-              for lay in layers] if args.latent else []
     # int8 mode: every replica's layer caches as int8 codes and fp32 row scales (synthetic:
     # the decode's cost does not depend on the values); L_max a multiple of 64
     if args.int8:
@@ -315,8 +376,15 @@ def run_gpu(args, w: si.Workload):
                 lay.v_joint = si.latent_cache_torch(js, w.B, 1, L_max, lay.rV, 1, dev)[:, 0]
                 lay.v_joint = lay.v_joint.contiguous()
                 lay.v_lat = None
-    olat = [torch.empty((w.B, w.Hq, lay.rV), dtype=torch.bfloat16, device=dev)
-            for lay in layers] if args.latent else []
+    # outputs: one device buffer read back by one D2H copy per step (latent mode: o~ of every
+    # layer, one after the other)
+    if args.latent:
+        osizes = [w.B * w.Hq * lay.rV for lay in layers]
+        out_all = torch.empty((sum(osizes),), dtype=torch.bfloat16, device=dev)
+        olat = [v.view(w.B, w.Hq, lay.rV) for v, lay in zip(torch.split(out_all, osizes), layers)]
+    else:
+        out_all = out
+        olat = []
 
     def layer_step(li, lay):
         if args.int8:  # decode over the int8 cache (no append)
@@ -383,12 +451,15 @@ def run_gpu(args, w: si.Workload):
     for i in range(W):
         step(reps[i % R])
     torch.cuda.synchronize()
-    h_q = q_s.cpu().pin_memory()
-    h_k = k_s.cpu().pin_memory()
-    h_v = v_s.cpu().pin_memory()
-    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    h_qlat = [t.cpu().pin_memory() for t in qlat_s]
-    h_olat = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in olat]
+    h_inp = inp.cpu().pin_memory()
+    h_out = torch.empty(out_all.shape, dtype=out_all.dtype).pin_memory()
+
+    def e2e_step(lays):
+        """One step as a user runs it: the inputs H2D (one copy from pinned memory), the API
+        calls, the outputs D2H (one copy into pinned memory)."""
+        inp.copy_(h_inp, non_blocking=True)
+        step(lays)
+        h_out.copy_(out_all, non_blocking=True)
     n_dec = max(8, R) // R * R
     cap = torch.cuda.Stream(device=dev)
     cap.wait_stream(torch.cuda.current_stream())
@@ -405,18 +476,7 @@ def run_gpu(args, w: si.Workload):
             step_graphs.append(gr)
             ge = torch.cuda.CUDAGraph()
             with torch.cuda.graph(ge, stream=cap):
-                if args.latent:
-                    for dst, src in zip(qlat_s, h_qlat):
-                        dst.copy_(src, non_blocking=True)
-                    step(reps[r])
-                    for dst, src in zip(h_olat, olat):
-                        dst.copy_(src, non_blocking=True)
-                else:
-                    q_s.copy_(h_q, non_blocking=True)
-                    k_s.copy_(h_k, non_blocking=True)
-                    v_s.copy_(h_v, non_blocking=True)
-                    step(reps[r])
-                    h_out.copy_(out, non_blocking=True)
+                e2e_step(reps[r])
             e2e_graphs.append(ge)
         dec_graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(dec_graph, stream=cap):
@@ -427,7 +487,7 @@ def run_gpu(args, w: si.Workload):
         with torch.cuda.graph(warm_graph, stream=cap):
             for i in range(n_dec):
                 lay = reps[i % R][0]
-                if args.int8 or args.joint:
+                if args.int8 or args.joint or args.latent:
                     layer_step(0, lay)
                 elif args.paged:
                     stief.stief_decode_attention_paged(q_s, lay.P_K, lay.P_V, lay.k_pages,
@@ -512,31 +572,36 @@ def run_gpu(args, w: si.Workload):
     iso.sort()
     dec_us_iso = iso[len(iso) // 2]
 
-    # ---- end to end through the public API: per step one replay of the captured API calls
-    # with the host copies: inputs H2D from pinned memory, append + decode, outputs D2H
-    reset_lengths(w.L - 1 - W)
-    for i in range(W):
-        e2e_graphs[i % R].replay()
-    reset_lengths(w.L - 1)
-    e0_ev, e1_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
-    torch.cuda.synchronize()
-    _backlog()
-    e0_ev.record(stream)
-    for j in range(K):
-        e2e_graphs[j % R].replay()
-    e1_ev.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    e2e_ms = e0_ev.elapsed_time(e1_ev) / K
-    h2d = (sum(t.numel() for t in qlat_s) if args.latent
-           else q_s.numel() + k_s.numel() + v_s.numel()) * 2
-    d2h = (sum(t.numel() for t in olat) if args.latent else out.numel()) * 2
+    # ---- end to end through the public API, two ways, each step with one H2D copy of its
+    # inputs from pinned memory and one D2H copy of its outputs into pinned memory:
+    #  - api: the Python binding calls the C entry points every step (host cost included);
+    #  - graph: the same calls captured once in a CUDA graph, one replay per step.
+    def time_e2e(run_one):
+        reset_lengths(w.L - 1 - W)
+        for i in range(W):
+            run_one(i)
+        reset_lengths(w.L - 1)
+        e0_ev, e1_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        e0_ev.record(stream)
+        for j in range(K):
+            run_one(j)
+        e1_ev.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        return e0_ev.elapsed_time(e1_ev) / K
+
+    e2e_api_ms = time_e2e(lambda j: e2e_step(reps[j % R]))
+    e2e_graph_ms = time_e2e(lambda j: e2e_graphs[j % R].replay())
+    h2d = h_inp.numel() * h_inp.element_size()
+    d2h = h_out.numel() * h_out.element_size()
     st = stief.stief_read_device_status(status)
     if st != 0:
         raise RuntimeError(f"device status {st:#x} after the e2e steps")
 
-    ms_per_step, e2e_ms, dec_us = reduce_over_ranks([ms_per_step, e2e_ms, dec_us], dev)
+    ms_per_step, e2e_api_ms, e2e_graph_ms, dec_us = reduce_over_ranks(
+        [ms_per_step, e2e_api_ms, e2e_graph_ms, dec_us], dev)
     del step_graphs, e2e_graphs, dec_graph, warm_graph, cycle_graph
 
     # ---- prefill compress (the prefill + batched decode workload): one 4096-token chunk
@@ -554,7 +619,6 @@ def run_gpu(args, w: si.Workload):
     peak, peak_kind = _hbm_peak()
     step_bytes = sum(row_bytes(lay.rK, lay.rV) * w.B * w.Hkv for lay in layers) * (
         (ctx_first + ctx_last) / 2)
-    rot_mb = R * sum(row_bytes(rK, rV) * w.B * w.Hkv * w.L for rK, rV in w.layer_ranks()) / 2**20
     result = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -568,36 +632,7 @@ def run_gpu(args, w: si.Workload):
         "vs_baseline": None,
         "dtype": "int8" if args.int8 else "bf16",
         "data": "synthetic",
-        "config": {
-            "workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "context": w.L,
-            "layers": len(layers), "ranks": [list(r) for r in w.layer_ranks()][:4]
-            + (["..."] if len(layers) > 4 else []),
-            "step": (("decode over an int8 latent cache (codes + fp32 row scales, synthetic "
-                      "values), no append, every layer; " if args.int8 else
-                      "decode with per-head keys and one joint value latent per token shared by "
-                      "the KV heads" + (" (latent output)" if args.latent else "") +
-                      ", no append, every layer; " if args.joint else
-                      "latent decode only (bases folded into the attention weights: q~ in, "
-                      "o~ out; the new token's latent rows would come from the folded K/V "
-                      "projection), every layer; " if args.latent else
-                      f"append 1 token per (sequence, KV head) + decode over page pools "
-                      f"({PAGE_SIZE}-token pages at shuffled pool positions), every layer; "
-                      if args.paged else
-                      "append 1 token per (sequence, KV head) + decode, every layer; ") +
-                     "the API calls captured in CUDA graphs (one step per replica, the timed "
-                     "region replays the replica cycle back to back); " +
-                     ("stief_compress_append + stief_decode_attention (3 kernels per layer)"
-                      if args.unfused else f"{step_call(args)} (1 kernel per layer)")),
-            "context_growth": (f"none (context {w.L} every step)"
-                               if args.latent or args.int8 or args.joint else
-                               f"+1 token per step of a replica (contexts {ctx_first}..{ctx_last})"),
-            "l2": (f"no flush: steps rotate over {R} copies of the layer caches "
-                   f"({rot_mb:.0f} MiB in all, > 3x the 126 MB L2)" if R > 1 else
-                   f"no flush: one step reads {rot_mb:.0f} MiB of caches (> 3x the 126 MB L2)"
-                   if rot_mb * 2**20 >= ROTATE_BYTES else
-                   f"inputs ({rot_mb:.1f} MiB in {R} copies) fit in L2: a latency case"),
-            "parallelism": f"independent sequences per GPU x{ws_n}",
-        },
+        "config": config_dict(w, args, ws_n),
         "hbm_gbs_step": round(step_bytes / (ms_per_step / 1e3) / 1e9, 1),
         "roofline": {
             "kernel": f"stief_decode_kernel ({step_call(args)})",
@@ -617,16 +652,27 @@ def run_gpu(args, w: si.Workload):
             "decode_us_single_launch": round(dec_us_iso, 3),
             "frac_single_launch": round(bytes_per_dec / (dec_us_iso / 1e6) / 1e9 / peak, 4),
         },
-        "e2e": {"value": round(job_tokens_per_s(w.B, ws_n, e2e_ms), 2), "unit": "tokens/s",
+        "e2e": {"value": round(job_tokens_per_s(w.B, ws_n, e2e_api_ms), 2), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "how": "per step one CUDA-graph replay of the public API calls with the "
-                       "pinned host copies (inputs H2D, outputs D2H) inside"},
+                "ms_per_step": round(e2e_api_ms, 6),
+                "how": "value: every step calls the public API from Python (ctypes into the C "
+                       "entry points) between one H2D copy of the step's inputs from pinned "
+                       "memory and one D2H copy of its outputs into pinned memory, CUDA events "
+                       "around the K steps; graph_value: the same step captured once in a CUDA "
+                       "graph, one replay per step",
+                "graph_value": round(job_tokens_per_s(w.B, ws_n, e2e_graph_ms), 2),
+                "graph_ms_per_step": round(e2e_graph_ms, 6)},
         "gpu_launches": (3 if args.unfused and not args.latent else 1) * len(layers) * K,
         "clocks": clocks,
         "wall_s_timed_region": round(t_wall, 3),
     }
     if compress is not None:
         result["compress"] = compress
+    extra = [n for n in args.extra.split(",") if n] if args.extra != "auto" else (
+        ["llama31_8b_128k", "llama3_8b_32layer_b16"]
+        if w.name == DEFAULT_WORKLOAD and step_call(args) == "stief_append_decode" else [])
+    if extra and ws_n == 1:
+        result["rooflines"] = [workload_roofline(args, n, dev) for n in extra]
     if (rank == 0 and ws_n == 1 and not args.no_cpu_baseline
             and not (args.latent or args.int8 or args.paged or args.joint)):
         result["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
@@ -634,6 +680,88 @@ def run_gpu(args, w: si.Workload):
         torch.distributed.destroy_process_group()
     if rank == 0:
         print(json.dumps(result), flush=True)
+
+
+def workload_roofline(args, name: str, dev) -> dict:
+    """The fused step's roofline on another workload, measured in the same run: its decode
+    kernel (stief_append_decode on layer 0, launches back to back over rotating replicas, like
+    the headline's) and its whole step (every layer), each from CUDA-graph replays."""
+    import decode_attention_stief_b200 as stief
+    w = si.WORKLOADS[name]
+    R = replica_count(w)
+    n_dec = max(8, R) // R * R
+    dec_reps, step_reps = 4, max(3, 12 // R) * R
+    grow = 2 * (args.warmup + dec_reps * n_dec // R + step_reps // R) + 64
+    reps = [build_state(w, grow, w.seed + 104729 * r, dev) for r in range(R)]
+    L_max = reps[0][1]
+    reps = [lays for lays, _ in reps]
+    g = torch.Generator(device=dev)
+    g.manual_seed(w.seed + 1)
+    q = torch.randn((w.B, w.Hq, w.d), generator=g, device=dev).to(torch.bfloat16)
+    kn = torch.randn((w.B, w.Hkv, 1, w.d), generator=g, device=dev).to(torch.bfloat16)
+    vn = torch.randn((w.B, w.Hkv, 1, w.d), generator=g, device=dev).to(torch.bfloat16)
+    out = torch.empty((w.B, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def launch(lay):
+        stief.stief_append_decode(q, kn, vn, lay.P_K, lay.P_V, lay.k_lat, lay.v_lat, lay.seq_lens,
+                                  out, lay.ws, max_seq_len=L_max, dev_status=status)
+
+    def reset():
+        for lays in reps:
+            for lay in lays:
+                lay.seq_lens.fill_(w.L - 1)
+
+    reset()
+    for i in range(args.warmup):
+        for lay in reps[i % R]:
+            launch(lay)
+    torch.cuda.synchronize()
+    cap = torch.cuda.Stream(device=dev)
+    cap.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(cap):
+        dec_graph, cycle = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(dec_graph, stream=cap):
+            for i in range(n_dec):
+                launch(reps[i % R][0])
+        with torch.cuda.graph(cycle, stream=cap):
+            for r in range(R):
+                for lay in reps[r]:
+                    launch(lay)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+
+    def timed(graph, n):
+        reset()
+        torch.cuda.synchronize()
+        _backlog()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            graph.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) * 1e3 / n  # us per replay
+
+    dec_us = timed(dec_graph, dec_reps) / n_dec
+    step_us = timed(cycle, step_reps // R) / R
+    st = stief.stief_read_device_status(status)
+    if st != 0:
+        raise RuntimeError(f"device status {st:#x} in the {name} roofline")
+    del dec_graph, cycle
+    rK, rV = w.layer_ranks()[0]
+    nbytes = int(2 * (rK + rV) * w.B * w.Hkv * (w.L + dec_reps * n_dec // R / 2))
+    peak, kind = _hbm_peak()
+    achieved = nbytes / (dec_us / 1e6) / 1e9
+    return {"workload": name, "B": w.B, "context": w.L, "layers": len(w.layer_ranks()),
+            "ranks_layer0": [rK, rV],
+            "decode_us": round(dec_us, 3), "algorithmic_bytes": nbytes,
+            "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "traffic": _traffic_per_launch(name),
+            "step_ms": round(step_us / 1e3, 6),
+            "tokens_per_s": round(w.B / (step_us / 1e6), 2),
+            "how": f"stief_append_decode on layer 0, {dec_reps} replays of {n_dec} launches back "
+                   f"to back over {R} replica(s); step = every layer, {step_reps} steps"}
 
 
 def time_prefill_compress(args, n_layers: int, dev, stream):
@@ -837,8 +965,7 @@ def run_reference(args, w: si.Workload):
         "n_gpus": ws_n, "steps": K, "warmup": W,
         "ms_per_step": round(w.B / value * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
-                   "context": w.L, "layers": len(w.layer_ranks())},
+        "config": config_dict(w, args, ws_n),
         "cpu_baseline": {"kind": "oracle", "cores": threads, "cpu_model": _cpu_model(),
                          "value": round(value, 4),
                          "unit": "tokens/s", "sample": sample},
@@ -846,6 +973,22 @@ def run_reference(args, w: si.Workload):
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(res), flush=True)
+
+
+def _free_port() -> int:
+    import socket
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def launch_ranks(n: int, argv) -> int:
+    """Run this script as n ranks of one node (torch.distributed.run on 127.0.0.1); returns the
+    launcher's exit code."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", f"--master-port={_free_port()}",
+           os.path.abspath(__file__), *argv]
+    return subprocess.call(cmd)
 
 
 def main():
@@ -883,7 +1026,17 @@ def main():
                          "kernel on layer 0 and exit (no timing, no JSON line)")
     ap.add_argument("--clock-window", type=float, default=0.6,
                     help="seconds of untimed decode load before the timed region")
+    ap.add_argument("--extra", default="auto",
+                    help="comma-separated workloads whose fused-step roofline is measured after "
+                         "the headline (auto: the 128k and 32-layer batch-16 workloads beside "
+                         "the default 32k one; empty: none)")
     args = ap.parse_args()
+    env_world = os.environ.get("WORLD_SIZE")
+    if env_world is None and args.gpus > 1:
+        # one process per GPU: start the ranks ourselves, as the driver's torchrun would
+        sys.exit(launch_ranks(args.gpus, sys.argv[1:]))
+    if env_world is not None and int(env_world) != args.gpus:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={env_world}: run N ranks with --gpus N")
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     modes = [m for m in ("int8", "latent", "paged", "joint", "unfused") if getattr(args, m)]

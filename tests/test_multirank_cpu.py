@@ -73,7 +73,7 @@ def test_ranks_decode_distinct_sequences():
 def test_reference_arm_prints_on_rank_0_only(rank):
     env = dict(os.environ, WORLD_SIZE="2", RANK=str(rank), LOCAL_RANK=str(rank))
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
-                          "--workload", "tiny", "--steps", "2", "--warmup", "3",
+                          "--gpus", "2", "--workload", "tiny", "--steps", "2", "--warmup", "3",
                           "--cpu-seconds", "0.5"], env=env, capture_output=True, text=True,
                          timeout=300, cwd=ROOT)
     assert out.returncode == 0, out.stderr[-2000:]
@@ -84,3 +84,37 @@ def test_reference_arm_prints_on_rank_0_only(rank):
         assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     else:
         assert lines == []
+
+
+def test_gpus_flag_launches_the_ranks_itself():
+    # no WORLD_SIZE in the environment: bench.py --gpus 2 starts two ranks (torch.distributed.run
+    # on 127.0.0.1) and rank 0 prints the one line
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--gpus", "2", "--workload", "tiny", "--steps", "2", "--warmup", "3",
+                          "--cpu-seconds", "0.5"], env=env, capture_output=True, text=True,
+                         timeout=300, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.strip().startswith("{")]
+    assert len(lines) == 1, out.stdout[-2000:]
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2
+
+
+def test_world_size_must_match_the_gpus_flag():
+    env = dict(os.environ, WORLD_SIZE="2", RANK="0", LOCAL_RANK="0")
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--workload", "tiny", "--steps", "2", "--warmup", "3"], env=env,
+                         capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert out.returncode != 0 and "WORLD_SIZE" in out.stderr
+
+
+def test_reference_arm_config_is_the_gpu_arms():
+    import argparse
+    import bench
+    import stief_inputs as si
+    args = argparse.Namespace(int8=False, latent=False, joint=False, paged=False, unfused=False)
+    c = bench.config_dict(si.WORKLOADS["llama3_8b_32k"], args, 1)
+    assert c["workload"] == "llama3_8b_32k" and c["context"] == 32768 and c["ranks"] == [[64, 64]]
+    assert "stief_append_decode" in c["step"] and "6 copies" in c["l2"]
