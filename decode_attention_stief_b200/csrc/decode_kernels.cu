@@ -1,1240 +1,30 @@
-// decode_kernels.cu -- split-KV decode attention over the latent (Stiefel-projected)
-// KV cache, for sm_100a.
-//
-// Operation (StiefAttention technical summary, "Mecanismo Central" item 5): keys
-// and values are stored as K_down = K P_K, V_down = V P_V and attention runs over
-// the reconstructions K~ = K_down P_K^T, V~ = V_down P_V^T.  The kernel never forms
-// K~ or V~; it uses the equal products
-//     s_t = (q P_K) . K_down[t] / sqrt(d)          (query projected once per CTA)
-//     o   = (sum_t softmax(s)_t V_down[t]) P_V^T   (up-projection after the mix)
-// so the HBM stream is the bf16 latent cache, read once per KV head.
-//
-// One kernel, grid (splits, Hkv * qsub, B).  A CTA serves up to G_T <= 8 query heads
-// of one KV head (a "unit") over one token range, with nwarps warps that each stream
-// their own 32-token tiles (warp w takes tiles w, w + nwarps, ...) through a private
-// ring of shared-memory stages.  Every stage holds the keys and the values of one tile,
-// fetched by 2-D TMA tensor copies in 64/32/16-column pieces with the matching swizzle
-// and completing on the stage's mbarrier.
-//
-// The contractions run on the warp-level tensor-core MMA (m16n8k16, bf16 operands,
-// fp32 accumulators), with the query heads as the N = 8 dimension: column n of the
-// MMA is head n & 3 for groups of up to 4 heads (part n >> 2), or head n with the part
-// given by the n-tile for groups of 8.  Part 0 carries the bf16 rounding hi(x) of an
-// fp32 operand x and part 1 its residual lo(x) = bf16(x - hi(x)); the two products are
-// added in fp32, which keeps q~, the softmax weights and o~ at about 16 significant
-// bits although the MMA takes bf16.  Per tile and warp:
-//   scores  S[token][n]  = K_down[token][:] . Q^T[:][n]     (M = tokens, K = r_K)
-//   online softmax over the tile (log2 domain, lazy rescale: accumulators are only
-//   rescaled when a head's maximum passes its running reference by more than 8)
-//   mix     O^T[dim][n] += V_down^T[dim][token] . P^T[token][n]  (M = r_V dims, K = tokens)
-// where P^T comes from the score accumulators through an in-register 8x8 transpose
-// (movmatrix).  The epilogue merges the warps (log-sum-exp); with one split it
-// up-projects with P_V^T on the same MMA (M = d, K = r_V) and writes the output,
-// otherwise it stores the latent partial state (o~, m, l) and takes a ticket: the last
-// CTA of the unit merges the splits, up-projects once and resets the ticket counter,
-// so the workspace counters stay zero between calls.
-//
-// Modes (compile-time, one instantiation each): the contiguous bf16 cache; the latent
-// decode (q~ given, o~ returned: no base loads, projections or up-projection, for bases
-// folded into the attention weights); paged caches (tiles addressed through a block
-// table); int8 caches (code boxes and row scales copied raw; each warp turns its codes into
-// exact fp16 in a padded row-major tile and the MMAs take fp16 operands, the row scales
-// multiplying the scores and the softmax weights).  Grids of more than one wave run two
-// CTAs per SM with a smaller ring.
-#include <cfloat>
-#include <cmath>
-#include <cstdint>
-
-#include <cuda_fp16.h>
-
-#include "stief_device.cuh"
-#include "stief_internal.h"
+// decode_kernels.cu -- dispatch of a planned decode call to the kernel instantiation of its
+// mode (each mode's instantiations live in their own translation unit, decode_mode_*.cu).
+#include "decode_kernel.cuh"
 
 namespace stief {
-
-constexpr int kPreIssue = 1;         // stages per warp requested before q~ is ready
-constexpr float kRescaleTau = 8.0f;  // lazy-rescale threshold (log2 units)
-constexpr uint32_t kFull = 0xffffffffu;
-
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-// A bounded mbarrier wait whose outcome is the same in every lane of the warp (the
-// warp-wide MMA and ldmatrix instructions that follow need all 32 lanes).
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint32_t* dev_status) {
-  return __all_sync(kFull, mbar_wait_bounded(bar, parity, dev_status));
-}
-
-// ---------------------------------------------------------------------------- warp MMA
-
-// Four 8x8 b16 matrices; lanes 8i..8i+7 give the row addresses of matrix i.
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-// Same, each matrix transposed on the way.
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-// Transpose of an 8x8 b16 matrix held in the warp's registers (one pair per lane).
-__device__ __forceinline__ uint32_t movm_t(uint32_t x) {
-  uint32_t y;
-  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
-  return y;
-}
-// c += A(16x16, row) . B(16x8, col), bf16 in, fp32 accumulate.
-__device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
-                                         uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// c = A . B (accumulators start at zero).
-__device__ __forceinline__ void mma_bf16_z(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
-                                           uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%10,%10,%10,%10};"
-      : "=f"(c[0]), "=f"(c[1]), "=f"(c[2]), "=f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.f));
-}
-
-// The same two products with fp16 operands (the int8 caches' codes are exact in fp16).
-__device__ __forceinline__ void mma_f16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
-                                        uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ void mma_f16_z(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
-                                          uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%10,%10,%10,%10};"
-      : "=f"(c[0]), "=f"(c[1]), "=f"(c[2]), "=f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.f));
-}
-template <bool F16>
-__device__ __forceinline__ void mma_op(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  if constexpr (F16) mma_f16(c, a, b0, b1);
-  else mma_bf16(c, a, b0, b1);
-}
-template <bool F16>
-__device__ __forceinline__ void mma_op_z(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  if constexpr (F16) mma_f16_z(c, a, b0, b1);
-  else mma_bf16_z(c, a, b0, b1);
-}
-
-// fp16 hi / lo parts of an fp32 pair, packed (first element in the low half)
-__device__ __forceinline__ uint32_t hi_pair_h(float x0, float x1) {
-  const __half2 h = __floats2half2_rn(x0, x1);
-  return *reinterpret_cast<const uint32_t*>(&h);
-}
-__device__ __forceinline__ uint32_t lo_pair_h(float x0, float x1, uint32_t hi) {
-  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hi));
-  return hi_pair_h(x0 - f.x, x1 - f.y);
-}
-// Four int8 codes (w) as exact fp16 pairs: 0x64uu is 1024 + uu in fp16, uu = code + 128.
-__device__ __forceinline__ void codes_f16(uint32_t w, uint32_t& h01, uint32_t& h23) {
-  const uint32_t u = w ^ 0x80808080u;
-  const uint32_t a = __byte_perm(u, 0x64646464u, 0x5140u), b = __byte_perm(u, 0x64646464u, 0x7362u);
-  // minus 1152 = 1024 + 128 in both halves (0x6480 is 1152 in fp16)
-  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(h01) : "r"(a), "r"(0x64806480u));
-  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(h23) : "r"(b), "r"(0x64806480u));
-}
-
-// hi / lo bf16 parts of an fp32 pair, packed (first element in the low half)
-__device__ __forceinline__ uint32_t hi_pair(float x0, float x1) { return pack_bf16x2_rn(x0, x1); }
-__device__ __forceinline__ uint32_t lo_pair(float x0, float x1, uint32_t hi) {
-  return pack_bf16x2_rn(x0 - bf16lo(hi), x1 - bf16hi(hi));
-}
-
-// ---------------------------------------------------------------------------- tile addressing
-
-// Where 16-byte column chunk `chunk` of a row lives inside a tile of `rows` rows stacked
-// from the pieces of a rank-r matrix: r / 64 pieces 64 columns wide, then one 32 wide if
-// r % 64 >= 32, then one 16 wide if r % 32 == 16 (the order the host plans them in).
-struct PieceLoc {
-  uint32_t off;  // piece offset in the tile
-  uint32_t w;    // piece width (columns)
-  uint32_t lc;   // chunk index inside the piece
-};
-__device__ __forceinline__ PieceLoc locate(int r, int rows, int chunk) {
-  const int col = chunk * 8;
-  const int x64 = r & ~63;
-  const bool has32 = r - x64 >= 32;
-  PieceLoc pl;
-  if (col < x64) {
-    pl.w = 64u;
-    pl.off = (uint32_t)((col >> 6) * rows * 128);
-    pl.lc = (uint32_t)((col & 63) >> 3);
-  } else if (has32 && col < x64 + 32) {
-    pl.w = 32u;
-    pl.off = (uint32_t)(x64 * rows * 2);
-    pl.lc = (uint32_t)((col - x64) >> 3);
-  } else {
-    const int x16 = x64 + (has32 ? 32 : 0);
-    pl.w = 16u;
-    pl.off = (uint32_t)(x16 * rows * 2);
-    pl.lc = (uint32_t)((col - x16) >> 3);
-  }
-  return pl;
-}
-// Byte offset of (row, chunk) under the piece's TMA swizzle: 128-byte rows XOR the chunk
-// with row & 7, 64-byte rows with (row >> 1) & 3, 32-byte rows with (row >> 2) & 1.
-__device__ __forceinline__ uint32_t swz(const PieceLoc& pl, int row) {
-  const uint32_t sw = pl.w == 64u ? (uint32_t)(row & 7)
-                      : pl.w == 32u ? (uint32_t)((row >> 1) & 3)
-                                    : (uint32_t)((row >> 2) & 1);
-  return pl.off + (uint32_t)row * pl.w * 2u + ((pl.lc ^ sw) << 4);
-}
-// Lane row / chunk for an x4 ldmatrix of a 16x16 block read as an A operand:
-//  - row-major (no transpose; the block's rows are the MMA's M): matrices
-//    (rows 0-7, chunk 0), (rows 8-15, chunk 0), (rows 0-7, chunk 1), (rows 8-15, chunk 1)
-//  - transposed (the block's rows are the MMA's K): matrices
-//    (rows 0-7, chunk 0), (rows 0-7, chunk 1), (rows 8-15, chunk 0), (rows 8-15, chunk 1)
-__device__ __forceinline__ int a_row(int lane) { return (lane & 7) + ((lane >> 3) & 1) * 8; }
-__device__ __forceinline__ int a_chunk(int lane) { return lane >> 4; }
-__device__ __forceinline__ int at_row(int lane) { return (lane & 7) + (lane >> 4) * 8; }
-__device__ __forceinline__ int at_chunk(int lane) { return (lane >> 3) & 1; }
-
-// B fragments (k-step ks) of X^T for an fp32 matrix X[head][col] in shared memory (row
-// stride xs floats): column n = lane >> 2 of n-tile j is (head, part) as described at the
-// top; k = cols 16 ks + 2 (lane & 3) + {0, 1} (first register) and + 8 (second).
-template <int NB>
-__device__ __forceinline__ void bfrag_hilo(const float* X, int xs, int ks, int lane,
-                                           uint32_t (&bf)[NB][2], bool f16 = false) {
-  const int n = lane >> 2;
-  const int c = 16 * ks + 2 * (lane & 3);
-  const int head = NB == 1 ? (n & 3) : n;
-  const float2 x = *reinterpret_cast<const float2*>(X + head * xs + c);
-  const float2 y = *reinterpret_cast<const float2*>(X + head * xs + c + 8);
-  const uint32_t hx = f16 ? hi_pair_h(x.x, x.y) : hi_pair(x.x, x.y);
-  const uint32_t hy = f16 ? hi_pair_h(y.x, y.y) : hi_pair(y.x, y.y);
-  const uint32_t lx = f16 ? lo_pair_h(x.x, x.y, hx) : lo_pair(x.x, x.y, hx);
-  const uint32_t ly = f16 ? lo_pair_h(y.x, y.y, hy) : lo_pair(y.x, y.y, hy);
-  if constexpr (NB == 1) {
-    const bool lo = (n >> 2) != 0;
-    bf[0][0] = lo ? lx : hx;
-    bf[0][1] = lo ? ly : hy;
-  } else {
-    bf[0][0] = hx;
-    bf[0][1] = hy;
-    bf[NB - 1][0] = lx;
-    bf[NB - 1][1] = ly;
-  }
-}
-
-__host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
-
-// Shared-memory carve-up (byte offsets from the dynamic base).
-struct DecodeSmem {
-  uint32_t bars;    // nwarps*nstage "full" and nwarps*nstage "empty" stage barriers, then
-                    // the setup barrier (q and P_K, then P_V) and the new-row barrier
-  uint32_t ml;      // [nwarps][8] (m, l); then [8] M, [8] L; then a flag
-  uint32_t qraw;    // [G_T][d] bf16 query rows
-  uint32_t newraw;  // append: the new token's k and v rows, bf16 [2][d]
-  uint32_t newlat;  // append: its projected key and value rows, bf16 [rK] then [rV]
-  uint32_t qt;      // [8][xs] fp32: q~ (prologue), o~ (epilogue)
-  uint32_t pmat;    // P_K (prologue), then P_V: d rows, pieces, swizzled
-  uint32_t region;  // per warp a ring of stages (keys then values of a tile); later the
-                    // cross-warp reduction and the split-merge staging
-  uint32_t region_bytes;
-  // int8 caches: the region holds one 16-bit tile per warp (the stage's codes as fp16,
-  // row-major, rows padded by 16 bytes), then the rings of raw stages: codes K [tile][rK], codes V
-  // [tile][rV], scales K [tile], scales V [tile]
-  uint32_t ring;      // offset of the rings inside the region
-  uint32_t q8_sc;     // int8 caches: per warp the tile's key then value row scales (fp32)
-  uint32_t q8_tile;   // int8 caches: bytes of a warp's 16-bit tile
-  uint32_t stage;     // bytes of one ring stage
-  uint32_t q8_v, q8_ks, q8_vs;  // offsets inside a raw int8 stage
-  uint32_t total;
-  int xs;  // row stride of qt in floats
-};
-
-__host__ __device__ inline DecodeSmem decode_smem_layout(int NW, int ns, int rK, int rV, int tile,
-                                                          bool q8 = false) {
-  DecodeSmem s;
-  const int rmax = rK > rV ? rK : rV;
-  uint32_t off = 0;
-  s.bars = off;
-  off = align_up(off + 8u * (2 * NW * ns + 2), 16);
-  s.ml = off;
-  off = align_up(off + 4u * (NW * 16 + 16 + 4), 16);
-  s.qraw = off;
-  off = align_up(off + 2u * 8u * 128u, 16);  // up to 8 heads of d = 128
-  s.newraw = off;
-  off = align_up(off + 2u * 2u * 128u, 16);
-  s.newlat = off;
-  off = align_up(off + 2u * (uint32_t)(rK + rV), 16);
-  s.xs = rmax + 4;
-  s.qt = off;
-  off = align_up(off + 4u * 8u * s.xs, 1024);
-  s.pmat = off;
-  off += 256u * rmax;  // d = 128 rows x r bf16
-  s.region = off;
-  const uint32_t bf16_stage = (uint32_t)tile * (rK + rV) * 2u;  // a multiple of 1 KiB
-  if (q8) {
-    s.q8_v = align_up((uint32_t)tile * rK, 128);
-    s.q8_ks = s.q8_v + align_up((uint32_t)tile * rV, 128);
-    s.q8_vs = s.q8_ks + (uint32_t)tile * 4u;
-    s.stage = align_up(s.q8_vs + (uint32_t)tile * 4u, 128);
-    // the 16-bit tile is row-major with rows padded by 16 bytes (conflict-free ldmatrix)
-    s.q8_tile = (uint32_t)tile * (2u * rK + 16u + 2u * rV + 16u);
-    s.q8_sc = (uint32_t)NW * s.q8_tile;
-    s.ring = align_up(s.q8_sc + (uint32_t)NW * 8u * tile, 128);
-  } else {
-    s.q8_v = s.q8_ks = s.q8_vs = s.q8_sc = s.q8_tile = 0;
-    s.stage = bf16_stage;
-    s.ring = 0;
-  }
-  s.region_bytes = s.ring + (uint32_t)NW * ns * s.stage;
-  off += s.region_bytes;
-  s.total = off;
-  return s;
-}
-
-// One CTA = nwarps consumer warps + 1 producer warp.  Lane w of the producer requests the
-// tiles (TMA) of consumer warp w and refills its stages as the warp releases them; the
-// consumer warps only compute.  NB: B n-tiles (1: up to 4 heads, 2: up to 8);
-// NKS >= rK/16; NMV >= rV/16.
-constexpr int kMaxConsumerWarps = 8;
-
-// Kernel modes: the contiguous bf16 cache, the latent decode, paged caches, int8 caches, and
-// joint value latents (one value row per token shared by the KV heads; full or latent output).
-// Each is its own instantiation, so a mode's branches cost the others nothing.
-constexpr int kModePlain = 0, kModeLatent = 1, kModePaged = 2, kModeQ8 = 3, kModeJointV = 4,
-              kModeLatentJointV = 5;
-
-template <int NB, int NKS, int NMV, int TT, int MODE>
-__global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
-    stief_decode_kernel(const __grid_constant__ DecodeArgs a) {
-  constexpr bool LAT = MODE == kModeLatent || MODE == kModeLatentJointV;
-  constexpr bool PG = MODE == kModePaged, Q8 = MODE == kModeQ8;
-  constexpr bool JV = MODE == kModeJointV || MODE == kModeLatentJointV;
-  constexpr int kTile = TT;
-  constexpr int MT = TT / 16;              // 16-token m-tiles (scores) / k-steps (mix) per tile
-  // score k-steps / value m-tiles whose fragments are loaded together (fewer where the
-  // accumulators already take many registers)
-  constexpr int KG = NB == 1 && TT == 32 ? 2 : 1;
-  constexpr int VG = NB == 1 && TT == 32 ? 2 : 1;
-  extern __shared__ __align__(1024) uint8_t smem[];
-  const int tid = threadIdx.x;
-  const int lane = tid & 31;
-  const int warp = tid >> 5;
-  const int NW = a.nwarps, ns = a.nstage;
-  const int NT = (NW + 1) * 32;  // all threads, the producer warp included
-  const bool producer = warp == NW;
-  const int s_idx = blockIdx.x;              // split
-  const int kvh = blockIdx.y / a.qsub;       // KV head
-  const int qs = blockIdx.y - kvh * a.qsub;  // query sub-group of that head
-  const int b = blockIdx.z;
-  const int d = a.d, rK = a.rK, rV = a.rV, S = a.S, G_T = a.G_T;
-  const int nks = rK >> 4, nmv = rV >> 4;
-  const int h0 = kvh * a.G + qs * G_T;          // first query head of this CTA
-  const int gcount = min(G_T, a.G - qs * G_T);  // valid query heads here
-  const size_t unit = ((size_t)b * a.Hkv + kvh) * a.qsub + qs;
-  // PG: paged caches (the contiguous instantiations carry no page lookups)
-  const CacheRows cr{PG ? a.block_table : nullptr, a.max_pages, a.page_size, a.num_pages, a.Hkv,
-                     a.L_max};
-
-  const DecodeSmem L = decode_smem_layout(NW, ns, rK, rV, TT, Q8);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);  // [NW][ns]: tile landed
-  uint64_t* empty = full + NW * ns;                             // [NW][ns]: tile consumed
-  uint64_t* setup_bar = empty + NW * ns;  // phase 0: q and P_K, phase 1: P_V
-  uint64_t* newrow_bar = setup_bar + 1;   // append: the new value row is in shared memory
-  float* ml = reinterpret_cast<float*>(smem + L.ml);
-  float* fin = ml + NW * 16;  // [8] M, [8] L
-  int* flag = reinterpret_cast<int*>(fin + 16);
-  float* qt = reinterpret_cast<float*>(smem + L.qt);
-  const int xs = L.xs;
-  uint8_t* pmat = smem + L.pmat;
-  const uint32_t kt_bytes = (uint32_t)kTile * rK * 2u;
-  const uint32_t st_bytes = kt_bytes + (uint32_t)kTile * rV * 2u;
-
-  // the swizzle patterns assume 1 KiB-aligned tiles
-  if (((smem_u32(smem + L.pmat) | smem_u32(smem + L.region)) & 1023u) != 0) {
-    if (tid == 0) report(a.dev_status, STIEF_DEV_SMEM_ALIGN);
-    return;
-  }
-  if (tid == 0) {
-    for (int i = 0; i < 2 * NW * ns + 2; ++i) mbar_init(&full[i], 1);
-    fence_barrier_init();
-    if (!LAT) {
-      // P_K is requested before the dependency wait (its latency then overlaps the preceding
-      // kernel's tail): a weight, which the calls document the preceding kernel must not
-      // write.  Its bytes are added to the setup barrier's phase; q arrives after the wait.
-      asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(setup_bar)),
-                   "r"(2u * d * rK) : "memory");
-      const uint64_t keep = l2_policy_evict_last();
-      for (int p = 0; p < a.ppk.n; ++p)
-        tma_load_2d(pmat + a.ppk.p[p].smem_off, &a.maps[a.ppk.p[p].map], a.ppk.p[p].x, kvh * d,
-                    setup_bar, keep);
-    }
-  }
-  __syncthreads();
-  // inputs may come from the preceding kernel in the stream: read nothing before this
-  pdl_wait();
-
-  // ---- split range and tiles --------------------------------------------------------------
-  // Splits partition [0, S * chunk) by the host bound max_seq_len (the grid was sized by it),
-  // so the first tiles can be requested before seq_lens has been read.  Consumer warp w takes
-  // the split's tiles w, w + NW, ...
-  const int t0 = s_idx * a.chunk;
-  const int t_spec = min(t0 + a.chunk, a.max_seq_len);
-  const int spec_tiles = t_spec > t0 ? (t_spec - t0 + kTile - 1) / kTile : 0;
-  int Lb = __ldcg(a.seq_lens + b);
-  if (Lb < 0 || Lb > a.max_seq_len) {
-    if (tid == 0 && s_idx == 0 && blockIdx.y == 0) report(a.dev_status, STIEF_DEV_BAD_LENGTH);
-    Lb = 0;
-  }
-  // append path: the new token becomes row Lb and is attended to, when the cache has room
-  // (Lb + 1 <= L_max; the host bound max_seq_len must cover the grown length too)
-  bool appended = false;
-  if (a.append) {
-    if (Lb + 1 > a.L_max) {
-      if (tid == 0 && s_idx == 0 && blockIdx.y == 0) report(a.dev_status, STIEF_DEV_CAPACITY_OVERFLOW);
-    } else if (Lb + 1 > a.max_seq_len) {
-      if (tid == 0 && s_idx == 0 && blockIdx.y == 0) report(a.dev_status, STIEF_DEV_BAD_LENGTH);
-    } else if (PG && cache_row(cr, b, kvh, Lb) < 0) {  // the new token's page is not mapped
-      if (tid == 0 && s_idx == 0 && blockIdx.y == 0) report(a.dev_status, STIEF_DEV_CAPACITY_OVERFLOW);
-    } else {
-      appended = true;
-    }
-  }
-  const long long new_row = appended ? cache_row(cr, b, kvh, Lb) : 0;  // the appended row
-  const int L_att = Lb + (appended ? 1 : 0);  // tokens attended to
-  const bool owns_new = appended && Lb >= t0 && Lb < t0 + a.chunk;  // the new token is in range
-  const int t1 = min(t0 + a.chunk, L_att);
-  // append path: each CTA of a sequence takes a ticket once it has read the old length;
-  // the CTA holding the last ticket (every CTA of the sequence has read it by then) stores
-  // the grown length.  The ticket is requested here by an idle producer lane and only looked
-  // at when the producer is done, so its round trip is off every critical path.
-  const bool seq_lane = a.append && warp == NW && lane == 31;
-  uint32_t seq_ticket = 0u;
-  if (seq_lane) seq_ticket = atomicAdd(a.ws_seq + b, 1u);
-  auto finish_sequence = [&]() {
-    if (seq_lane && seq_ticket == (uint32_t)gridDim.x * gridDim.y - 1u) {
-      a.ws_seq[b] = 0u;
-      if (appended) a.seq_lens_w[b] = Lb + 1;
-    }
-  };
-  const int n_tiles = t1 > t0 ? (t1 - t0 + kTile - 1) / kTile : 0;
-  auto warp_tiles = [NW](int w, int tiles) { return w < tiles ? (tiles - w + NW - 1) / NW : 0; };
-  // a tile's first row (tiles never straddle a page: page_size is a multiple of the tile);
-  // a tile of an unmapped page is requested past the end of the pool, which the copy fills
-  // with zeros (such tokens lie past the sequence and are masked)
-  const long long pool_rows = PG ? (long long)a.num_pages * a.Hkv * a.page_size
-                                 : (long long)a.B * a.Hkv * a.L_max;
-  auto tile_row = [&](int t) {
-    const long long r = cache_row(cr, b, kvh, t);
-    return (int)(r < 0 ? pool_rows : r);
-  };
-  // TMA parameters of the cache pieces (at most three per matrix), kept in registers
-  const void* kmap[3];
-  const void* vmap[3];
-  int kx[3], vx[3];
-  uint32_t ko[3], vo[3];
-#pragma unroll
-  for (int p = 0; p < 3; ++p) {
-    const int pk = p < a.pk.n ? p : 0, pv = p < a.pv.n ? p : 0;
-    kmap[p] = &a.maps[a.pk.p[pk].map];
-    kx[p] = a.pk.p[pk].x;
-    ko[p] = (uint32_t)a.pk.p[pk].smem_off;
-    vmap[p] = &a.maps[a.pv.p[pv].map];
-    vx[p] = a.pv.p[pv].x;
-    vo[p] = kt_bytes + (uint32_t)a.pv.p[pv].smem_off;
-  }
-  const int npk = a.pk.n, npv = a.pv.n;
-  auto issue = [&](int w, int k, uint64_t policy) {  // producer: tile k of consumer warp w
-    uint8_t* dst = smem + L.region + L.ring + ((size_t)w * ns + (k % ns)) * L.stage;
-    uint64_t* bar = &full[w * ns + (k % ns)];
-    if (Q8) {  // int8 codes of K and V (one box each) and the tile's two rows of scales
-      const uint32_t tb = (uint32_t)kTile * (rK + rV) + 8u * kTile;
-      mbar_arrive_expect_tx(bar, tb);
-      const int y = tile_row(t0 + (w + k * NW) * kTile);
-      tma_load_2d(dst, kmap[0], 0, y, bar, policy);
-      tma_load_2d(dst + L.q8_v, vmap[0], 0, y, bar, policy);
-      bulk_g2s(dst + L.q8_ks, a.k_scale + y, 4u * kTile, bar);
-      bulk_g2s(dst + L.q8_vs, a.v_scale + y, 4u * kTile, bar);
-      return;
-    }
-    // whole 32-row boxes land (rows past the sequence are masked on chip)
-    mbar_arrive_expect_tx(bar, st_bytes);
-    const int tt = t0 + (w + k * NW) * kTile;
-    const int y = tile_row(tt);
-    // joint values: the value rows of sequence b are b * L_max + t, whatever the KV head
-    const int yv = JV ? b * a.L_max + tt : y;
-#pragma unroll
-    for (int p = 0; p < 3; ++p)
-      if (p < npk) tma_load_2d(dst + ko[p], kmap[p], kx[p], y, bar, policy);
-#pragma unroll
-    for (int p = 0; p < 3; ++p)
-      if (p < npv) tma_load_2d(dst + vo[p], vmap[p], vx[p], yv, bar, policy);
-  };
-
-  // ---- prologue ------------------------------------------------------------------------------
-  bool ok = true;
-  if (producer) {
-    if (lane < 12 && lane < a.nmaps) prefetch_tensormap(&a.maps[lane]);
-    if (lane == 0 && LAT) {  // latent decode: the rows of q~ are the input
-      mbar_arrive_expect_tx(setup_bar, 2u * gcount * rK);
-      bulk_g2s(smem + L.qraw, a.q + ((size_t)b * a.Hq + h0) * rK, 2u * gcount * rK, setup_bar);
-    } else if (lane == 0) {
-      // q (and, for the fused step, the new rows) first: they gate q~; then every warp's ring
-      const uint64_t keep = l2_policy_evict_last();  // bases are shared by many CTAs
-      mbar_arrive_expect_tx(setup_bar, 2u * gcount * d + (owns_new ? 4u * d : 0u));
-      bulk_g2s(smem + L.qraw, a.q + ((size_t)b * a.Hq + h0) * d, 2u * gcount * d, setup_bar);
-      if (owns_new) {
-        const size_t row = ((size_t)b * a.Hkv + kvh) * d;
-        bulk_g2s(smem + L.newraw, a.k_new + row, 2u * d, setup_bar);
-        bulk_g2s(smem + L.newraw + 2u * d, a.v_new + row, 2u * d, setup_bar);
-      }
-      (void)keep;  // P_K was requested before the dependency wait
-    }
-    __syncwarp();
-    if (lane < NW) {  // lane w requests consumer warp w's tiles
-      const uint64_t stream = l2_policy_evict_first();
-      for (int k = 0; k < min(min(kPreIssue, ns), warp_tiles(lane, spec_tiles)); ++k)
-        issue(lane, k, stream);
-    }
-    __syncwarp();
-  } else if (LAT) {
-    // q~ is given (bf16 [heads][r_K]): widen and scale it into log2 units; absent heads are 0
-    ok = warp_wait(setup_bar, 0, a.dev_status);
-    const uint16_t* qr = reinterpret_cast<const uint16_t*>(smem + L.qraw);
-    for (int i = tid; i < 8 * rK; i += NW * 32) {
-      const int h = i / rK, j = i - h * rK;
-      qt[h * xs + j] = h < gcount ? bf16_to_f32(qr[h * rK + j]) * a.qscale : 0.f;
-    }
-  } else {
-    // q~ = q P_K on the MMA: q~^T[j][head] = sum_i P_K[i][j] q[head][i]
-    // (M = the r_K columns of P_K, N = 8 heads, K = d), scaled into log2 units
-    const int n = lane >> 2;  // B column = head
-    ok = warp_wait(setup_bar, 0, a.dev_status);
-    uint32_t qb[8][2];  // d / 16 k-steps
-    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(smem + L.qraw) + min(n, gcount - 1) * (d / 2);
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      qb[ks][0] = n < gcount ? qrow[8 * ks + (lane & 3)] : 0u;
-      qb[ks][1] = n < gcount ? qrow[8 * ks + 4 + (lane & 3)] : 0u;
-    }
-    // append: the new key row k_down = k_new P_K is the same contraction with B column 0 =
-    // k_new (fp32 accumulation, one rounding to bf16).  Tasks 0..nks-1 are the q~ m-tiles,
-    // nks..2 nks-1 the k_down m-tiles; the warps share them out.
-    const uint32_t* krow = reinterpret_cast<const uint32_t*>(smem + L.newraw);
-    const int ntasks = owns_new ? 2 * nks : nks;
-    for (int task = warp; task < ntasks && ok; task += NW) {
-      const bool key = task >= nks;
-      const int mt = key ? task - nks : task;
-      float c[4];
-      const PieceLoc pl = locate(rK, d, 2 * mt + at_chunk(lane));
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        uint32_t af[4];
-        ldsm_x4_t(smem_u32(pmat) + swz(pl, 16 * ks + at_row(lane)), af);
-        uint32_t b0 = qb[ks][0], b1 = qb[ks][1];
-        if (key) {
-          b0 = n == 0 ? krow[8 * ks + (lane & 3)] : 0u;
-          b1 = n == 0 ? krow[8 * ks + 4 + (lane & 3)] : 0u;
-        }
-        if (ks == 0) mma_bf16_z(c, af, b0, b1);
-        else mma_bf16(c, af, b0, b1);
-      }
-      const int j = 16 * mt + (lane >> 2), hh = 2 * (lane & 3);
-      if (!key) {
-        qt[hh * xs + j] = c[0] * a.qscale;
-        qt[(hh + 1) * xs + j] = c[1] * a.qscale;
-        qt[hh * xs + j + 8] = c[2] * a.qscale;
-        qt[(hh + 1) * xs + j + 8] = c[3] * a.qscale;
-      } else if ((lane & 3) == 0) {  // column 0: k_down[j], k_down[j + 8]
-        uint16_t* kl = reinterpret_cast<uint16_t*>(smem + L.newlat);
-        kl[j] = f32_to_bf16_rn(c[0]);
-        kl[j + 8] = f32_to_bf16_rn(c[2]);
-        if (qs == 0) {  // the cache row itself (every sub-group computes the same values)
-          uint16_t* dst = a.k_lat_w + new_row * rK;
-          dst[j] = kl[j];
-          dst[j + 8] = kl[j + 8];
-        }
-      }
-    }
-  }
-  __syncthreads();  // q~ is in shared memory and every read of P_K is done
-
-  // this lane's two heads (hA, hB = hA + 1) and, for NB == 1, its part of the MMA columns
-  const int hA = NB == 1 ? 2 * (lane & 1) : 2 * (lane & 3);
-  const bool lo_lane = NB == 1 && (lane & 2) != 0;
-  float mA = -INFINITY, mB = -INFINITY, lA = 0.f, lB = 0.f;
-  float oacc[NMV][NB][4];
-#pragma unroll
-  for (int mt = 0; mt < NMV; ++mt)
-#pragma unroll
-    for (int j = 0; j < NB; ++j)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) oacc[mt][j][e] = 0.f;
-
-  if (producer) {
-    // ---- producer: P_V, the rest of every ring, then refills as stages are released ----
-    if (lane == 0 && !LAT) {
-      fence_proxy_async_smem();  // P_V replaces P_K, read through the generic proxy above
-      const uint64_t keep = l2_policy_evict_last();
-      mbar_arrive_expect_tx(setup_bar, 2u * d * rV);
-      for (int p = 0; p < a.ppv.n; ++p)
-        tma_load_2d(pmat + a.ppv.p[p].smem_off, &a.maps[a.ppv.p[p].map], a.ppv.p[p].x, kvh * d,
-                    setup_bar, keep);
-    }
-    __syncwarp();
-    {
-      // Lane w serves consumer warp w: tile k goes into the stage the warp released after
-      // tile k - ns.  The lanes stay converged: every pass tests all their stages at once
-      // (non-blocking) and issues whatever is free, so one slow warp holds up no other.
-      const int w = lane;
-      const uint64_t stream = l2_policy_evict_first();
-      const int pre = min(kPreIssue, ns);
-      const int tiles_w = lane < NW ? warp_tiles(w, n_tiles) : 0;
-      for (int k = pre; k < min(ns, tiles_w); ++k) issue(w, k, stream);
-      int k = ns;
-      uint64_t last_progress = global_timer_ns();
-      // append: once P_V has landed, the new value row v_down = v_new P_V is projected on
-      // the MMA (B column 0) into shared memory (and the cache) for the tile that holds it
-      // (one 16-row m-tile per call, so the refills in between are not held up)
-      int vrow_next = owns_new ? 0 : nmv;  // next m-tile of the new value row to project
-      auto project_vrow = [&]() {
-        const uint32_t* vrow = reinterpret_cast<const uint32_t*>(smem + L.newraw + 2u * d);
-        const bool vcol = (lane >> 2) == 0;  // lanes holding B column 0
-        uint16_t* vl = reinterpret_cast<uint16_t*>(smem + L.newlat) + rK;
-        {
-          const int mv = vrow_next;
-          float cv[4];
-          const PieceLoc pl = locate(rV, d, 2 * mv + at_chunk(lane));
-#pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {
-            uint32_t af[4];
-            ldsm_x4_t(smem_u32(pmat) + swz(pl, 16 * ks + at_row(lane)), af);
-            const uint32_t v0 = vcol ? vrow[8 * ks + (lane & 3)] : 0u;
-            const uint32_t v1 = vcol ? vrow[8 * ks + 4 + (lane & 3)] : 0u;
-            if (ks == 0) mma_bf16_z(cv, af, v0, v1);
-            else mma_bf16(cv, af, v0, v1);
-          }
-          if ((lane & 3) == 0) {  // column 0: v_down[j], v_down[j + 8]
-            const int j = 16 * mv + (lane >> 2);
-            vl[j] = f32_to_bf16_rn(cv[0]);
-            vl[j + 8] = f32_to_bf16_rn(cv[2]);
-            if (qs == 0) {
-              a.v_lat_w[new_row * rV + j] = vl[j];
-              a.v_lat_w[new_row * rV + j + 8] = vl[j + 8];
-            }
-          }
-        }
-        if (++vrow_next == nmv) {
-          __syncwarp();
-          if (lane == 0) mbar_arrive(newrow_bar);  // release: the row is visible to the consumers
-        }
-      };
-      while (__any_sync(kFull, k < tiles_w)) {
-        if (vrow_next < nmv && mbar_test(setup_bar, 1u)) project_vrow();
-        const bool ready = k < tiles_w && mbar_test(&empty[w * ns + (k % ns)], (uint32_t)((k / ns - 1) & 1));
-        if (ready) {
-          issue(w, k, stream);
-          ++k;
-        }
-        if (__any_sync(kFull, ready)) {
-          last_progress = global_timer_ns();
-        } else {
-          __nanosleep(64);
-          if (global_timer_ns() - last_progress > kWaitLimitNs) {  // the consumers gave up
-            if (lane == 0) report(a.dev_status, STIEF_DEV_WAIT_TIMEOUT);
-            break;
-          }
-        }
-      }
-      if (vrow_next < nmv && mbar_wait_bounded(setup_bar, 1u, a.dev_status))
-        while (vrow_next < nmv) project_vrow();
-      finish_sequence();
-      // tiles requested before seq_lens was known but past the sequence are never consumed:
-      // they must land before the region is reused
-      if (lane < NW) {
-        const int requested = min(pre, warp_tiles(w, spec_tiles));
-        for (int kk = tiles_w; kk < requested; ++kk) mbar_wait_bounded(&full[w * ns + kk], 0u, nullptr);
-      }
-    }
-    __syncwarp();
-  } else {
-    // ---- consumers: stream the warp's tiles ------------------------------------------------
-    const int my_tiles = warp_tiles(warp, n_tiles);
-    uint8_t* ring = smem + L.region + L.ring + (size_t)warp * ns * L.stage;
-    uint8_t* staging = smem + L.region + (size_t)warp * L.q8_tile;  // int8 caches only
-    const uint32_t sK = 2u * rK + 16u, sV = 2u * rV + 16u;  // its row strides
-    const uint32_t q8_kt = (uint32_t)kTile * sK;            // its value rows' offset
-    // int8 caches: in the conversion pass a lane takes one 16-column chunk of each matrix
-    // and every (32 / chunks per row)-th row of it (no division per item)
-    const int kcpr = rK >> 4, vcpr = rV >> 4;  // 16-column chunks per row
-    const int krpp = 32 / kcpr, vrpp = 32 / vcpr;  // rows per pass
-    const bool klive = lane < krpp * kcpr, vlive = lane < vrpp * vcpr;
-    const int kc0 = lane % kcpr, vc0 = lane % vcpr;
-    const int kt0 = lane / kcpr, vt0 = lane / vcpr;
-
-    uint32_t qf[NKS][NB][2];  // B fragments of Q^T (hi / lo parts)
-#pragma unroll
-    for (int ks = 0; ks < NKS; ++ks)
-      if (ks < nks) bfrag_hilo<NB>(qt, xs, ks, lane, qf[ks], Q8);  // fp16 against int8 codes
-    uint32_t koff[NKS], kstep[NKS], voff[NMV], vstep[NMV];
-#pragma unroll
-    for (int ks = 0; ks < NKS; ++ks) {
-      if (Q8) {  // the row-major padded 16-bit tile
-        koff[ks] = (uint32_t)a_row(lane) * sK + (uint32_t)(2 * ks + a_chunk(lane)) * 16u;
-        kstep[ks] = 16u * sK;
-        continue;
-      }
-      const PieceLoc pl = locate(rK, kTile, 2 * ks + a_chunk(lane));
-      koff[ks] = swz(pl, a_row(lane));
-      kstep[ks] = 32u * pl.w;  // 16 rows further (the swizzle repeats every 8 rows)
-    }
-#pragma unroll
-    for (int mt = 0; mt < NMV; ++mt) {
-      if (Q8) {
-        voff[mt] = q8_kt + (uint32_t)at_row(lane) * sV + (uint32_t)(2 * mt + at_chunk(lane)) * 16u;
-        vstep[mt] = 16u * sV;
-        continue;
-      }
-      const PieceLoc pl = locate(rV, kTile, 2 * mt + at_chunk(lane));
-      voff[mt] = kt_bytes + swz(pl, at_row(lane));
-      vstep[mt] = 32u * pl.w;
-    }
-
-    for (int k = 0; k < my_tiles && ok; ++k) {
-      const int st = k % ns;
-      if (!warp_wait(&full[warp * ns + st], (uint32_t)((k / ns) & 1), a.dev_status)) {
-        ok = false;
-        break;
-      }
-      uint32_t sbase = smem_u32(ring + (size_t)st * L.stage);
-      const int tok0 = t0 + (warp + k * NW) * kTile;
-      const int n = min(kTile, t1 - tok0);
-      // int8 caches: the tile's row scales go to this warp's scale buffer (0 past the
-      // sequence, so that whatever the scale rows hold there reaches nothing) and the codes
-      // become exact fp16 in its 16-bit tile
-      float* scw = reinterpret_cast<float*>(smem + L.region + L.q8_sc) + warp * 2 * kTile;
-      if (Q8) {
-        const uint8_t* raw = ring + (size_t)st * L.stage;
-        const float* scr = reinterpret_cast<const float*>(raw + L.q8_ks);  // K then V rows
-        __syncwarp();  // every lane is done reading the previous tile and its scales
-        for (int i = lane; i < 2 * kTile; i += 32)  // the V row follows the K row in the stage
-          scw[i] = (i < kTile ? i : i - kTile) < n ? scr[i] : 0.f;
-        for (int m = 0; m < 2; ++m) {
-          const int r = m ? rV : rK;
-          const int8_t* codes = reinterpret_cast<const int8_t*>(raw + (m ? L.q8_v : 0u)) + 16 * (m ? vc0 : kc0);
-          const uint32_t stride = m ? sV : sK;
-          const int rpp = m ? vrpp : krpp;
-          const int t0 = m ? vt0 : kt0;
-          uint8_t* dst = staging + (m ? q8_kt : 0u) + (uint32_t)t0 * stride + 32u * (uint32_t)(m ? vc0 : kc0);
-          const int8_t* src = codes + t0 * r;
-          const uint32_t dstep = (uint32_t)rpp * stride;
-          const int sstep = rpp * r;
-          if (m ? vlive : klive)
-            for (int t = t0; t < kTile; t += rpp, dst += dstep, src += sstep) {
-              const uint4 w16 = *reinterpret_cast<const uint4*>(src);
-              uint4 o0, o1;
-              codes_f16(w16.x, o0.x, o0.y);
-              codes_f16(w16.y, o0.z, o0.w);
-              codes_f16(w16.z, o1.x, o1.y);
-              codes_f16(w16.w, o1.z, o1.w);
-              reinterpret_cast<uint4*>(dst)[0] = o0;
-              reinterpret_cast<uint4*>(dst)[1] = o1;
-            }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[warp * ns + st]);  // the raw stage may be refilled
-        sbase = smem_u32(staging);
-      }
-      if (owns_new && tok0 <= Lb && Lb < tok0 + kTile) {
-        // This tile holds the new token, whose cache rows were not written yet when the tile
-        // was fetched: put the projected rows (key row from the prologue, value row from
-        // the producer) into the tile.
-        if (!warp_wait(newrow_bar, 0, a.dev_status)) {
-          ok = false;
-          break;
-        }
-        const int r_new = Lb - tok0;
-        const uint16_t* kl = reinterpret_cast<const uint16_t*>(smem + L.newlat);
-        for (int cch = lane; cch < (rK + rV) / 8; cch += 32) {
-          const bool key = cch < rK / 8;
-          const PieceLoc pt = key ? locate(rK, kTile, cch) : locate(rV, kTile, cch - rK / 8);
-          *reinterpret_cast<uint4*>(ring + (size_t)st * st_bytes + (key ? 0u : kt_bytes) +
-                                    swz(pt, r_new)) = *reinterpret_cast<const uint4*>(kl + 8 * cch);
-        }
-        fence_proxy_async_smem();  // generic writes into a stage the TMA engine fills
-        __syncwarp();
-      }
-
-      // Fragments are requested a group of k-steps (m-tiles) at a time, so their latencies
-      // overlap; asm volatile keeps the order written here.
-      // scores: c[mt][j][e] is token 16 mt + (lane >> 2) + 8 (e >> 1), column
-      // 2 (lane & 3) + (e & 1)
-      float c[MT][NB][4];
-#pragma unroll
-      for (int g0 = 0; g0 < NKS; g0 += KG)
-        if (g0 < nks) {
-          uint32_t kf[KG][MT][4];
-#pragma unroll
-          for (int u = 0; u < KG; ++u)
-            if (g0 + u < nks) {
-#pragma unroll
-              for (int mt = 0; mt < MT; ++mt)
-                ldsm_x4(sbase + koff[g0 + u] + mt * kstep[g0 + u], kf[u][mt]);
-            }
-#pragma unroll
-          for (int u = 0; u < KG; ++u)
-            if (g0 + u < nks) {
-#pragma unroll
-              for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                for (int j = 0; j < NB; ++j) {
-                  if (g0 + u == 0) mma_op_z<Q8>(c[mt][j], kf[u][mt], qf[0][j][0], qf[0][j][1]);
-                  else mma_op<Q8>(c[mt][j], kf[u][mt], qf[g0 + u][j][0], qf[g0 + u][j][1]);
-                }
-            }
-        }
-      // value fragments do not depend on the scores: request the first group now
-      uint32_t vf[VG][MT][4];
-      auto load_v = [&](int g0) {
-#pragma unroll
-        for (int u = 0; u < VG; ++u)
-          if (g0 + u < nmv) {
-#pragma unroll
-            for (int kk = 0; kk < MT; ++kk)
-              ldsm_x4_t(sbase + voff[g0 + u] + kk * vstep[g0 + u], vf[u][kk]);
-          }
-        if (n < kTile) {
-          // the sequence ends inside this tile: the value rows past it may hold anything
-          // (0 * NaN would reach the accumulators), so their fragment halves become zero.
-          // Register r of a fragment holds tokens 16 kk + 8 (r >> 1) + 2 (lane & 3) + {0, 1}.
-#pragma unroll
-          for (int u = 0; u < VG; ++u)
-#pragma unroll
-            for (int kk = 0; kk < MT; ++kk)
-#pragma unroll
-              for (int r = 0; r < 4; ++r) {
-                const int tok = 16 * kk + 8 * (r >> 1) + 2 * (lane & 3);
-                vf[u][kk][r] = tok + 1 < n ? vf[u][kk][r] : (tok < n ? (vf[u][kk][r] & 0xffffu) : 0u);
-              }
-        }
-      };
-      load_v(0);
-      // add the hi and lo parts: s[mt][e] is the score of head hA + (e & 1)
-      float s[MT][4];
-#pragma unroll
-      for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          s[mt][e] = NB == 1 ? c[mt][0][e] + __shfl_xor_sync(kFull, c[mt][0][e], 2)
-                             : c[mt][0][e] + c[mt][NB - 1][e];
-      if (Q8) {  // scores of code rows times the rows' key scales
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) s[mt][e] *= scw[16 * mt + (lane >> 2) + 8 * (e >> 1)];
-      }
-      if (n < kTile) {  // missing tokens take no weight
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            if (16 * mt + (lane >> 2) + 8 * (e >> 1) >= n) s[mt][e] = -INFINITY;
-      }
-
-      // online softmax, log2 domain.  The lane maxima are voted on first: only when some
-      // head passes its reference by more than the threshold are the maxima over the 8
-      // lanes sharing the heads formed and the accumulators rescaled.
-      float tA = fmaxf(s[0][0], s[0][2]), tB = fmaxf(s[0][1], s[0][3]);
-#pragma unroll
-      for (int mt = 1; mt < MT; ++mt) {
-        tA = fmaxf(tA, fmaxf(s[mt][0], s[mt][2]));
-        tB = fmaxf(tB, fmaxf(s[mt][1], s[mt][3]));
-      }
-      if (__any_sync(kFull, tA > mA + kRescaleTau || tB > mB + kRescaleTau)) {
-#pragma unroll
-        for (int o = 4; o < 32; o <<= 1) {
-          tA = fmaxf(tA, __shfl_xor_sync(kFull, tA, o));
-          tB = fmaxf(tB, __shfl_xor_sync(kFull, tB, o));
-        }
-        if (tA > mA + kRescaleTau) {
-          const float mn = fmaxf(mA, tA);
-          const float f = ex2(mA - mn);  // 0 while mA is -inf
-          lA *= f;
-          mA = mn;
-#pragma unroll
-          for (int mt = 0; mt < NMV; ++mt)
-#pragma unroll
-            for (int j = 0; j < NB; ++j) {
-              oacc[mt][j][0] *= f;
-              oacc[mt][j][2] *= f;
-            }
-        }
-        if (tB > mB + kRescaleTau) {
-          const float mn = fmaxf(mB, tB);
-          const float f = ex2(mB - mn);
-          lB *= f;
-          mB = mn;
-#pragma unroll
-          for (int mt = 0; mt < NMV; ++mt)
-#pragma unroll
-            for (int j = 0; j < NB; ++j) {
-              oacc[mt][j][1] *= f;
-              oacc[mt][j][3] *= f;
-            }
-        }
-      }
-      const float uA = mA == -INFINITY ? 0.f : mA, uB = mB == -INFINITY ? 0.f : mB;
-      // weights of the tile as B fragments of P^T: block r = tokens 8r..8r+7 in the score
-      // layout (row = token, columns = this lane's two heads), transposed to (token pairs, head)
-      uint32_t pb[NB][2 * MT];
-      float pa_sum = 0.f, pb_sum = 0.f;
-#pragma unroll
-      for (int r = 0; r < 2 * MT; ++r) {
-        const int mt = r >> 1, e0 = (r & 1) * 2;
-        const float pA = ex2(s[mt][e0] - uA), pB = ex2(s[mt][e0 + 1] - uB);
-        pa_sum += pA;
-        pb_sum += pB;
-        // int8 caches: the weights of code rows carry the rows' value scales (not in l)
-        const float sv = Q8 ? scw[kTile + 16 * mt + (lane >> 2) + 8 * (r & 1)] : 1.f;
-        const float wA = pA * sv, wB = pB * sv;
-        const uint32_t hw = Q8 ? hi_pair_h(wA, wB) : hi_pair(wA, wB);
-        const uint32_t lw = Q8 ? lo_pair_h(wA, wB, hw) : lo_pair(wA, wB, hw);
-        if constexpr (NB == 1) {
-          pb[0][r] = movm_t(lo_lane ? lw : hw);
-        } else {
-          pb[0][r] = movm_t(hw);
-          pb[NB - 1][r] = movm_t(lw);
-        }
-      }
-      lA += pa_sum;
-      lB += pb_sum;
-
-      // value mix: O^T[dim][n] += V^T[dim][token] P^T[token][n]
-#pragma unroll
-      for (int g0 = 0; g0 < NMV; g0 += VG)
-        if (g0 < nmv) {
-          if (g0 > 0) load_v(g0);
-#pragma unroll
-          for (int u = 0; u < VG; ++u)
-            if (g0 + u < nmv) {
-#pragma unroll
-              for (int kk = 0; kk < MT; ++kk)
-#pragma unroll
-                for (int j = 0; j < NB; ++j)
-                  mma_op<Q8>(oacc[g0 + u][j], vf[u][kk], pb[j][2 * kk], pb[j][2 * kk + 1]);
-            }
-        }
-      __syncwarp();
-      if (!Q8 && lane == 0) mbar_arrive(&empty[warp * ns + st]);  // the stage may be refilled
-    }
-  }
-  pdl_launch_dependents();
-
-  // ---- merge the warps ------------------------------------------------------------------
-#pragma unroll
-  for (int o = 4; o < 32; o <<= 1) {
-    lA += __shfl_xor_sync(kFull, lA, o);
-    lB += __shfl_xor_sync(kFull, lB, o);
-  }
-  float ov[NMV][4];  // o~ of (dim 16 mt + (lane >> 2) + 8 (e >> 1), head hA + (e & 1))
-#pragma unroll
-  for (int mt = 0; mt < NMV; ++mt)
-#pragma unroll
-    for (int e = 0; e < 4; ++e)
-      ov[mt][e] = NB == 1 ? oacc[mt][0][e] + __shfl_xor_sync(kFull, oacc[mt][0][e], 2)
-                          : oacc[mt][0][e] + oacc[mt][NB - 1][e];
-  __syncthreads();  // every warp is done with its ring: the region becomes the reduction buffer
-  float* red = reinterpret_cast<float*>(smem + L.region);  // [NW][8][rV]
-  const int HR = NB == 1 ? 4 : 8;                          // heads the MMA columns carry
-  if (!producer && !lo_lane) {
-#pragma unroll
-    for (int mt = 0; mt < NMV; ++mt)
-      if (mt < nmv)
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          red[(warp * 8 + hA + (e & 1)) * rV + 16 * mt + (lane >> 2) + 8 * (e >> 1)] = ov[mt][e];
-    if ((lane >> 2) == 0) {
-      ml[(warp * 8 + hA) * 2] = mA;
-      ml[(warp * 8 + hA) * 2 + 1] = lA;
-      ml[(warp * 8 + hA + 1) * 2] = mB;
-      ml[(warp * 8 + hA + 1) * 2 + 1] = lB;
-    }
-  }
-  __syncthreads();
-  // o~ of the CTA (normalised when this CTA finishes the unit alone) becomes the B operand
-  // of the up-projection
-  for (int idx = tid; idx < HR * rV; idx += NT) {
-    const int h = idx / rV, jj = idx - h * rV;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kMaxConsumerWarps; ++w)
-      if (w < NW) M = fmaxf(M, ml[(w * 8 + h) * 2]);
-    float o = 0.f, lsum = 0.f;
-#pragma unroll
-    for (int w = 0; w < kMaxConsumerWarps; ++w)
-      if (w < NW) {
-        const float mw = ml[(w * 8 + h) * 2];
-        if (mw != -INFINITY) {
-          const float f = ex2(mw - M);
-          o = fmaf(f, red[(w * 8 + h) * rV + jj], o);
-          lsum = fmaf(f, ml[(w * 8 + h) * 2 + 1], lsum);
-        }
-      }
-    if (S == 1) o = lsum > 0.f ? o / lsum : 0.f;
-    qt[h * xs + jj] = o;
-    if (jj == 0) {
-      fin[h] = M;
-      fin[8 + h] = lsum;
-    }
-  }
-  __syncthreads();
-
-  // ---- up-projection o = o~ P_V^T on the MMA: o^T[i][n] = sum_j P_V[i][j] o~^T[j][n] ----
-  // (M = d, N = heads, K = r_V) from the normalised o~ in qt; warp w takes rows 16 w,
-  // 16 (w + NW + 1), ...
-  auto up_project = [&]() {
-    if (!warp_wait(setup_bar, 1, a.dev_status)) return;
-    for (int mt = warp; mt < d / 16; mt += NW + 1) {
-      float c[NB][4];
-#pragma unroll
-      for (int ks = 0; ks < NMV; ++ks)
-        if (ks < nmv) {
-          uint32_t af[4];
-          const PieceLoc pl = locate(rV, d, 2 * ks + a_chunk(lane));
-          ldsm_x4(smem_u32(pmat) + swz(pl, 16 * mt + a_row(lane)), af);
-          uint32_t bf[NB][2];
-          bfrag_hilo<NB>(qt, xs, ks, lane, bf);
-#pragma unroll
-          for (int j = 0; j < NB; ++j) {
-            if (ks == 0) mma_bf16_z(c[j], af, bf[j][0], bf[j][1]);
-            else mma_bf16(c[j], af, bf[j][0], bf[j][1]);
-          }
-        }
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float o = NB == 1 ? c[0][e] + __shfl_xor_sync(kFull, c[0][e], 2) : c[0][e] + c[NB - 1][e];
-        const int head = hA + (e & 1), i = 16 * mt + (lane >> 2) + 8 * (e >> 1);
-        if (!lo_lane && head < gcount) a.out[((size_t)b * a.Hq + h0 + head) * d + i] = f32_to_bf16_rn(o);
-      }
-    }
-  };
-  if (S == 1) {  // this CTA finishes the unit alone: qt holds the normalised o~
-    if (LAT) {
-      for (int i = tid; i < gcount * rV; i += NT) {
-        const int h = i / rV, j = i - h * rV;
-        a.out[((size_t)b * a.Hq + h0 + h) * rV + j] = f32_to_bf16_rn(qt[h * xs + j]);
-      }
-    } else if (ok) {
-      up_project();
-    }
-    return;
-  }
-  // Split partial states stay in the latent space (o~ scaled to the CTA's maximum, r_V floats
-  // per head, then m and l): the last CTA merges them and up-projects once.
-  const int rec = rV + 4;  // floats per partial state
-  float* parts = a.ws_part + unit * (size_t)S * G_T * rec;
-  for (int i = tid; i < gcount * rV; i += NT) {
-    const int h = i / rV, j = i - h * rV;
-    parts[((size_t)s_idx * G_T + h) * rec + j] = qt[h * xs + j];
-  }
-
-  // ---- split merge: publish this split, take a ticket; the last CTA merges them all ---------
-  if (tid < gcount) {
-    parts[((size_t)s_idx * G_T + tid) * rec + rV] = fin[tid];
-    parts[((size_t)s_idx * G_T + tid) * rec + rV + 1] = fin[8 + tid];
-  }
-  __syncthreads();  // every state of this CTA is written (block scope) ...
-  if (tid == 0) {
-    // ... and the acquire-release ticket makes them, by cumulativity, visible device-wide
-    // before the count moves; the last CTA's acquire orders its reads of the others' states
-    uint32_t ticket;
-    asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], 1;"
-                 : "=r"(ticket)
-                 : "l"(a.ws_cnt + unit)
-                 : "memory");
-    const int last = ticket == (uint32_t)(S - 1);
-    if (last) a.ws_cnt[unit] = 0u;  // ready for the next call
-    *flag = last;
-  }
-  __syncthreads();
-  if (!*flag) {
-    // P_V is only used by the merging CTA, but its copy must land before this CTA's shared
-    // memory is released (it was requested long before; the wait is bounded)
-    if (!LAT && tid == 0) mbar_wait_bounded(setup_bar, 1u, a.dev_status);
-    return;
-  }
-  // Thread groups of tpi consecutive lanes take one item = (head, 4 output columns); lane
-  // `sub` of a group merges splits sub, sub + tpi, ... (a batch of eight in flight at a time),
-  // then the group combines its tpi running states with shuffles.
-  const int nitems = gcount * (rV / 4);
-  int tpi = 1;
-  while (tpi < 8 && tpi * 2 * nitems <= NT) tpi *= 2;
-  const int sub = tid & (tpi - 1);
-  const int iters = (nitems * tpi + NT - 1) / NT;
-  auto merge = [](float& M, float& Ls, float4& o, float m2, float l2, const float4& o2) {
-    if (m2 == -INFINITY) return;
-    if (m2 > M) {
-      const float f = ex2(M - m2);  // 0 while M is -inf
-      Ls *= f;
-      o.x *= f;
-      o.y *= f;
-      o.z *= f;
-      o.w *= f;
-      M = m2;
-    }
-    const float w = ex2(m2 - M);
-    Ls = fmaf(w, l2, Ls);
-    o.x = fmaf(w, o2.x, o.x);
-    o.y = fmaf(w, o2.y, o.y);
-    o.z = fmaf(w, o2.z, o.z);
-    o.w = fmaf(w, o2.w, o.w);
-  };
-  constexpr int kBatch = 8;
-  for (int it = 0; it < iters; ++it) {
-    const int item = (it * NT + tid) / tpi;
-    const bool valid = item < nitems;
-    const int g = valid ? item / (rV / 4) : 0, c4 = valid ? item - g * (rV / 4) : 0;
-    float M = -INFINITY, Ls = 0.f;
-    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s0 = sub; s0 < S; s0 += kBatch * tpi) {
-      float ms[kBatch], ls[kBatch];
-      float4 os[kBatch];
-#pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        const int s = s0 + u * tpi;
-        if (valid && s < S) {
-          const float* r = parts + ((size_t)s * G_T + g) * rec;
-          const float2 m2 = __ldcg(reinterpret_cast<const float2*>(r + rV));
-          ms[u] = m2.x;
-          ls[u] = m2.y;
-          os[u] = __ldcg(reinterpret_cast<const float4*>(r) + c4);
-        } else {
-          ms[u] = -INFINITY;
-          ls[u] = 0.f;
-          os[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-      }
-      // the batch's maximum first, then independent weights and sums (short dependency chains)
-      float Mb = -INFINITY;
-#pragma unroll
-      for (int u = 0; u < kBatch; ++u) Mb = fmaxf(Mb, ms[u]);
-      float Lb2 = 0.f;
-      float4 ob = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        const float w = ms[u] == -INFINITY ? 0.f : ex2(ms[u] - Mb);
-        Lb2 = fmaf(w, ls[u], Lb2);
-        ob.x = fmaf(w, os[u].x, ob.x);
-        ob.y = fmaf(w, os[u].y, ob.y);
-        ob.z = fmaf(w, os[u].z, ob.z);
-        ob.w = fmaf(w, os[u].w, ob.w);
-      }
-      merge(M, Ls, o, Mb, Lb2, ob);
-    }
-    for (int off = 1; off < tpi; off <<= 1) {
-      const float M2 = __shfl_xor_sync(kFull, M, off), L2 = __shfl_xor_sync(kFull, Ls, off);
-      float4 o2;
-      o2.x = __shfl_xor_sync(kFull, o.x, off);
-      o2.y = __shfl_xor_sync(kFull, o.y, off);
-      o2.z = __shfl_xor_sync(kFull, o.z, off);
-      o2.w = __shfl_xor_sync(kFull, o.w, off);
-      merge(M, Ls, o, M2, L2, o2);
-    }
-    if (valid && sub == 0) {
-      const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
-      if (LAT) {  // o~ is the result
-        uint2 packed;
-        packed.x = pack_bf16x2_rn(o.x * inv, o.y * inv);
-        packed.y = pack_bf16x2_rn(o.z * inv, o.w * inv);
-        *reinterpret_cast<uint2*>(a.out + ((size_t)b * a.Hq + h0 + g) * rV + 4 * c4) = packed;
-      } else {  // the normalised o~ becomes the up-projection's operand
-        float* dst = qt + g * xs + 4 * c4;
-        dst[0] = o.x * inv;
-        dst[1] = o.y * inv;
-        dst[2] = o.z * inv;
-        dst[3] = o.w * inv;
-      }
-    }
-  }
-  if (!LAT) {
-    __syncthreads();
-    up_project();
-  }
-}
-
-// ------------------------------------------------------------------------------ launch
-
-template <int NB, int NKS, int NMV, int TT, int MODE>
-static cudaError_t launch_k(const DecodeArgs& a, cudaStream_t stream) {
-  const DecodeSmem L = decode_smem_layout(a.nwarps, a.nstage, a.rK, a.rV, TT, MODE == kModeQ8);
-  auto kern = stief_decode_kernel<NB, NKS, NMV, TT, MODE>;
-  static SmemLimit limit;
-  cudaError_t e = limit.ensure(reinterpret_cast<const void*>(kern), a.device, (int)L.total);
-  if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(a.S, a.Hkv * a.qsub, a.B);
-  cfg.blockDim = dim3((a.nwarps + 1) * 32);  // consumer warps + the producer warp
-  cfg.dynamicSmemBytes = L.total;
-  cfg.stream = stream;
-  // programmatic dependent launch: the CTAs may be scheduled while the previous kernel in
-  // the stream drains; they wait for it (griddepcontrol.wait) before reading any input
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, a);
-}
-
-// the latent decode and the paged caches are their own instantiations, so their branches
-// cost the contiguous path nothing (a runtime flag cost it 0.5-0.8 us per launch)
-template <int NB, int NKS, int NMV, int TT>
-static cudaError_t launch_t(const DecodeArgs& a, cudaStream_t stream) {
-  if ((a.latent != 0) + (a.block_table != nullptr) + (a.q8 != 0) > 1)
-    return cudaErrorInvalidValue;  // the modes do not combine
-  if (a.joint_v) {
-    if (a.block_table != nullptr || a.q8 != 0 || a.append != 0) return cudaErrorInvalidValue;
-    return a.latent ? launch_k<NB, NKS, NMV, TT, kModeLatentJointV>(a, stream)
-                    : launch_k<NB, NKS, NMV, TT, kModeJointV>(a, stream);
-  }
-  if (a.latent) return launch_k<NB, NKS, NMV, TT, kModeLatent>(a, stream);
-  if (a.block_table) return launch_k<NB, NKS, NMV, TT, kModePaged>(a, stream);
-  if (a.q8) return launch_k<NB, NKS, NMV, TT, kModeQ8>(a, stream);
-  return launch_k<NB, NKS, NMV, TT, kModePlain>(a, stream);
-}
 
 uint32_t decode_smem_bytes(int nwarps, int nstage, int rK, int rV, int tile, bool q8) {
   return decode_smem_layout(nwarps, nstage, rK, rV, tile, q8).total;
 }
 
-template <int NB>
-static cudaError_t launch_nb(const DecodeArgs& a, cudaStream_t stream) {
-  const bool wk = a.rK > 64, wv = a.rV > 64;
-  if (a.tile == 64) {  // only small ranks (both <= 64, rK + rV <= 96) take 64-token tiles
-    if (wk || wv) return cudaErrorInvalidValue;
-    return launch_t<NB, 4, 4, 64>(a, stream);
-  }
-  if (!wk && !wv) return launch_t<NB, 4, 4, 32>(a, stream);
-  if (!wk) return launch_t<NB, 4, 8, 32>(a, stream);
-  if (!wv) return launch_t<NB, 8, 4, 32>(a, stream);
-  return launch_t<NB, 8, 8, 32>(a, stream);
+uint32_t decode_region_bytes(int nwarps, int nstage, int rK, int rV, int tile, bool q8) {
+  return decode_smem_layout(nwarps, nstage, rK, rV, tile, q8).region_bytes;
 }
 
+// the latent decode, paged, int8 and joint-value caches are their own instantiations, so their
+// branches cost the contiguous path nothing (a runtime flag cost it 0.5-0.8 us per launch)
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
-  return a.G_T <= 4 ? launch_nb<1>(a, stream) : launch_nb<2>(a, stream);
+  if ((a.latent != 0) + (a.block_table != nullptr) + (a.q8 != 0) > 1)
+    return cudaErrorInvalidValue;  // the modes do not combine
+  if (a.joint_v) {
+    if (a.block_table != nullptr || a.q8 != 0 || a.append != 0) return cudaErrorInvalidValue;
+    return a.latent ? launch_decode_latent_joint_v(a, stream) : launch_decode_joint_v(a, stream);
+  }
+  if (a.latent) return launch_decode_latent(a, stream);
+  if (a.block_table) return launch_decode_paged(a, stream);
+  if (a.q8) return launch_decode_q8(a, stream);
+  return launch_decode_plain(a, stream);
 }
 
 }  // namespace stief

@@ -2,6 +2,7 @@
 // argument checks, split count, CTA configuration and the key-cache tensor maps.
 #include <cmath>
 #include <cstdint>
+#include <atomic>
 #include <mutex>
 
 #include <cuda.h>
@@ -114,7 +115,15 @@ struct DevInfo {
 DevInfo g_dev_info[kMaxDevices];
 std::once_flag g_dev_once[kMaxDevices];
 
+#ifdef STIEF_TEST_HOOKS
+std::atomic<uint32_t> g_test_stall{0};
+#endif
+
 }  // namespace
+
+#ifdef STIEF_TEST_HOOKS
+uint32_t test_stall_bytes() { return g_test_stall.load(); }
+#endif
 
 bool query_device(int* dev_out, int* sms, bool* sm100) {
   int dev = 0;
@@ -228,6 +237,15 @@ stief_status plan_decode(DecodeArgs& a, const uint16_t* q, const uint16_t* P_K,
                     choose_decode_config_pair(rK, rV, a.tile, &a.nwarps, &a.nstage, q8);
   if (!pair && !choose_decode_config(rK, rV, a.tile, &a.nwarps, &a.nstage, q8))
     return STIEF_ERR_INVALID_ARG;
+  // Split merge: through tagged words when the whole grid is on the GPU at once (one CTA per
+  // SM at most, so every split of a unit runs while its merging CTA reads their records) and
+  // the merging CTA's staging fits its shared memory; otherwise by tickets (no CTA waits for
+  // another).
+  a.merge_tagged = 0;
+  if (a.S > 1 && (long long)a.S * units <= sms &&
+      decode_tagged_stage_bytes(a.G_T, a.S, rV) <=
+          decode_region_bytes(a.nwarps, a.nstage, rK, rV, a.tile, q8))
+    a.merge_tagged = 1;
 
   int nmaps = 0;
   const uint64_t prow = (uint64_t)Hkv * d;
@@ -254,7 +272,18 @@ stief_status plan_decode(DecodeArgs& a, const uint16_t* q, const uint16_t* P_K,
                   !plan_pieces(a, &nmaps, a.ppv, P_V, rV, prow, d)))
     return STIEF_ERR_CUDA;
   a.nmaps = nmaps;
+#ifdef STIEF_TEST_HOOKS
+  a.test_stall_bytes = test_stall_bytes();
+#endif
   return STIEF_OK;
 }
 
 }  // namespace stief
+
+#ifdef STIEF_TEST_HOOKS
+// Test build only (libstief_testhooks.so, used by the timeout tests; not part of the public
+// header): every decode planned after this call waits for `bytes` more on its setup barrier
+// than any copy delivers, so its bounded waits run out (0 turns it off).  The bytes must be a
+// multiple of 16.
+extern "C" STIEF_API void stief_test_set_stall(uint32_t bytes) { stief::g_test_stall.store(bytes); }
+#endif

@@ -259,6 +259,7 @@ stief_status decode_common(const uint16_t* q, const uint16_t* k_new, const uint1
   a.ws_seq = a.ws_cnt + units;
   a.ws_part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
                                        stief::decode_ws_counter_bytes(units, (size_t)B));
+  a.ws_words = reinterpret_cast<uint64_t*>(a.ws_part);
   if (stief::launch_decode(a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return STIEF_ERR_CUDA;
   return STIEF_OK;

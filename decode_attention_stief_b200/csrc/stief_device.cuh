@@ -28,8 +28,13 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
-// A bounded wait gives up after this long (nanoseconds of the global timer).
+// A bounded wait gives up after this long (nanoseconds of the global timer).  The test build
+// (STIEF_TEST_HOOKS, a separate library used only by the timeout tests) gives up sooner.
+#ifdef STIEF_TEST_HOOKS
+constexpr uint64_t kWaitLimitNs = 50000000ull;  // 50 ms
+#else
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+#endif
 
 // ---------------------------------------------------------------------------- mbarrier
 
@@ -172,6 +177,17 @@ __device__ __forceinline__ void prefetch_tensormap(const void* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }
 
+// ---------------------------------------------------------------------------- named barriers
+
+// Hardware barrier `id` (1..15; 0 is __syncthreads) among `count` threads (a multiple of 32):
+// wait for all of them, or arrive without waiting.
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+__device__ __forceinline__ void named_bar_arrive(int id, int count) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // ---------------------------------------------------------------------------- PDL
 
 // Block until the preceding grid in the stream has completed and its memory is
@@ -210,6 +226,29 @@ __device__ __forceinline__ void pdl_wait() {
 // to start its prologue now.
 __device__ __forceinline__ void pdl_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------- tagged words
+
+// Values passed between CTAs without a fence: each 64-bit word holds an fp32 value in its
+// low half and a tag in its high half.  An aligned 64-bit access is single-copy atomic, so
+// a reader that sees the tag also sees the value written with it; a vector access of two
+// words is two such accesses (each word is checked on its own).
+__device__ __forceinline__ uint64_t tagged(float v, uint32_t tag) {
+  return ((uint64_t)tag << 32) | (uint64_t)__float_as_uint(v);
+}
+__device__ __forceinline__ float tagged_value(uint64_t w) { return __uint_as_float((uint32_t)w); }
+__device__ __forceinline__ uint32_t tagged_tag(uint64_t w) { return (uint32_t)(w >> 32); }
+
+// Store two tagged words (16-byte aligned) at GPU scope, bypassing L1.
+__device__ __forceinline__ void st_tagged2(uint64_t* p, uint64_t w0, uint64_t w1) {
+  asm volatile("st.relaxed.gpu.global.v2.b64 [%0], {%1, %2};" ::"l"(p), "l"(w0), "l"(w1)
+               : "memory");
+}
+// Load two tagged words (16-byte aligned) at GPU scope (every call reads L2 again).
+__device__ __forceinline__ void ld_tagged2(const uint64_t* p, uint64_t& w0, uint64_t& w1) {
+  asm volatile("ld.relaxed.gpu.global.v2.b64 {%0, %1}, [%2];" : "=l"(w0), "=l"(w1) : "l"(p)
+               : "memory");
 }
 
 // ---------------------------------------------------------------------------- loads

@@ -46,7 +46,13 @@ struct DecodeArgs {
   int32_t* seq_lens_w;
   uint32_t* ws_seq;  // [B] per-sequence finish tickets; zero between calls
   uint32_t* ws_cnt;  // [units] split tickets; zero between calls
-  float* ws_part;    // [units * S * G_T][rV + 4] partial states: o~[rV] (latent), m, l, 0, 0
+  // Split partial states, in one of two forms over the same bytes:
+  //  - ticket merge: float [units * S * G_T][rV + 4]: o~[rV] (latent), m, l, 0, 0
+  //  - tagged merge: uint64 [units * S * G_T][rV + 2]: o~[rV], m, l as tagged words (value,
+  //    tag 1 when written); every word is zero between calls
+  float* ws_part;
+  uint64_t* ws_words;
+  int merge_tagged;  // 1: the tagged merge (the grid fits on the GPU at once), 0: tickets
   uint32_t* dev_status;
   int B, Hq, Hkv, G, G_T, qsub, d, rK, rV, L_max, S;
   int max_seq_len;  // host bound of seq_lens; the splits partition [0, S * chunk)
@@ -66,6 +72,11 @@ struct DecodeArgs {
   int joint_v;     // values: one row per (sequence, token) shared by the KV heads
   const float* k_scale;
   const float* v_scale;
+#ifdef STIEF_TEST_HOOKS
+  // test build only: bytes added to the setup barrier's expected count that no copy delivers,
+  // so that its phase never completes and the waits for it run out (0: off)
+  uint32_t test_stall_bytes;
+#endif
 };
 
 struct CompressArgs {
@@ -111,6 +122,8 @@ struct SmemLimit {
 };
 
 uint32_t decode_smem_bytes(int nwarps, int nstage, int rK, int rV, int tile, bool q8 = false);
+// Bytes of the region (rings, then the warp-merge and split-merge staging) in that layout.
+uint32_t decode_region_bytes(int nwarps, int nstage, int rK, int rV, int tile, bool q8 = false);
 
 // 2-D tiled TMA tensor map over a row-major bf16 matrix [rows][cols] (row stride in
 // bytes), boxes of box_cols x box_rows with the given swizzle.  Host only.
@@ -137,13 +150,26 @@ stief_status plan_decode(DecodeArgs& a, const uint16_t* q, const uint16_t* P_K,
                          const float* v_scale = nullptr, bool joint_v = false);
 
 // Decode workspace layout: `units` = B * Hkv * qsub split-ticket counters, then B sequence
-// tickets (uint32, padded together to 256 bytes), then units * G_T * splits partial states
-// of (d + 4) floats (the kernel uses r_V + 4 <= d + 4 of each).
+// tickets (uint32, padded together to 256 bytes), then units * G_T * splits partial-state
+// records of (d + 2) 8-byte words (a tagged record uses r_V + 2 <= d + 2 words, a ticket
+// record r_V + 4 <= 2 d + 4 floats).
 inline size_t decode_ws_counter_bytes(size_t units, size_t B) {
   return ((units + B) * 4u + 255u) / 256u * 256u;
 }
 inline size_t decode_ws_bytes(size_t units, size_t B, int G_T, int splits, int d) {
-  return decode_ws_counter_bytes(units, B) + units * (size_t)G_T * splits * (size_t)(d + 4) * 4u;
+  return decode_ws_counter_bytes(units, B) + units * (size_t)G_T * splits * (size_t)(d + 2) * 8u;
+}
+// Bytes of the tagged partial-state words a call with this plan writes (the prefix of the
+// record area that must be zero when it starts).
+inline size_t decode_ws_tagged_bytes(size_t units, int G_T, int splits, int rV) {
+  return units * (size_t)G_T * splits * (size_t)(rV + 2) * 8u;
+}
+// Shared-memory bytes the merging CTA of the tagged merge stages the records in: its heads'
+// records [nh][S][rV + 2], their weights [nh][S], eight inverse sums and the merged o~
+// [nh][rV], where nh <= ceil(G_T / S) heads are merged by one CTA.
+inline size_t decode_tagged_stage_bytes(int G_T, int splits, int rV) {
+  const int nh = (G_T + splits - 1) / splits;
+  return 4u * ((size_t)nh * splits * (rV + 2) + (size_t)nh * splits + 8 + (size_t)nh * rV);
 }
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
 
@@ -184,6 +210,10 @@ inline bool choose_decode_config(int rK, int rV, int tile, int* nwarps, int* nst
   return false;
 }
 cudaError_t launch_compress(const CompressArgs& a, cudaStream_t stream);
+#ifdef STIEF_TEST_HOOKS
+// test build only: the stall the next decode launches are planned with (see DecodeArgs)
+uint32_t test_stall_bytes();
+#endif
 // Joint value latents: keys per head into k_lat, the values of all KV heads of a token
 // through P_V = P_VJ [Hkv*d][rV] into v_lat = v_joint [B][L_max][rV]; then the lengths.
 cudaError_t launch_compress_joint(const CompressArgs& a, cudaStream_t stream);

@@ -20,12 +20,15 @@
 // before any stream capture.  All calls share the one array per device:
 // concurrent calls whose kernels overlap on the GPU (different streams, or
 // several host threads) race on it and must be serialised by the caller.  The
-// array keeps the previous call's contents.  Only the ticket counters must be
-// zero when a call starts: the array is zero when the library is loaded, and
-// every call that runs to completion leaves its counters at zero again (the
-// partial states are always written before they are read).  Sizes whose partial states do not fit are rejected with
-// STIEF_ERR_WORKSPACE before anything is launched.  No cudaMalloc, cudaFree or
-// allocating library routine is called.
+// array keeps the previous call's contents.  The ticket counters and the tagged
+// words of the split merge must be zero when a call starts; a call that runs to
+// completion leaves them so, but one that stopped early (a wait timeout) may not,
+// and the caller cannot reach the array to clear it.  So every call zeroes the
+// part it will use with cudaMemsetAsync on its stream before the launch (the
+// partial states themselves are always written before they are read).  Sizes
+// whose partial states do not fit are rejected with STIEF_ERR_WORKSPACE before
+// anything is launched.  No cudaMalloc, cudaFree or allocating library routine
+// is called.
 #include <cmath>
 #include <cstdint>
 #include <mutex>
@@ -84,7 +87,25 @@ extern "C" STIEF_API stief_status stief_decode_attention_noalloc(
   a.ws_seq = a.ws_cnt + units;
   a.ws_part = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) +
                                        stief::decode_ws_counter_bytes(units, (size_t)B));
-  if (stief::launch_decode(a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
-    return STIEF_ERR_CUDA;
+  a.ws_words = reinterpret_cast<uint64_t*>(a.ws_part);
+  // The ticket counters (and the tagged words of the split merge) must be zero when the
+  // kernel starts.  A call that completes leaves them so, but one that stopped early (a wait
+  // timeout) may not, and the caller cannot reach this array to clear it: zero them here, in
+  // stream order, before every launch (a memset, not an allocation).
+  size_t clear = stief::decode_ws_counter_bytes(units, (size_t)B);
+  if (a.merge_tagged) clear += stief::decode_ws_tagged_bytes(units, a.G_T, a.S, a.rV);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(scratch, 0, clear, s) != cudaSuccess) return STIEF_ERR_CUDA;
+  if (stief::launch_decode(a, s) != cudaSuccess) return STIEF_ERR_CUDA;
   return STIEF_OK;
 }
+
+#ifdef STIEF_TEST_HOOKS
+// Test build only: the device address of this library's scratch array on the current device,
+// so that a test can plant stale counters in it (the public calls never expose it).
+extern "C" STIEF_API stief_status stief_test_noalloc_scratch(void** ptr, size_t* bytes) {
+  if (!ptr || !bytes) return STIEF_ERR_INVALID_ARG;
+  *bytes = kScratchBytes;
+  return scratch_address(ptr);
+}
+#endif

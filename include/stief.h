@@ -96,8 +96,12 @@ typedef enum stief_status {
  * A sequence whose seq_lens[b] + T exceeds L_max (or whose length is negative)
  * is skipped entirely -- no row written, length unchanged -- and
  * STIEF_DEV_CAPACITY_OVERFLOW (or STIEF_DEV_BAD_LENGTH) is set in *dev_status.
- * Small T runs on CUDA cores; prefill-sized T runs as a tcgen05 tensor-core
- * GEMM with the accumulator in tensor memory.
+ * Small T runs on CUDA cores; prefill-sized T (>= 128) runs as a tcgen05
+ * tensor-core GEMM with the accumulator in tensor memory.  That kernel is
+ * launched as a programmatic dependent of the preceding work in the stream and
+ * stages P_K and P_V before waiting for it: the bases must not be written by the
+ * kernel that immediately precedes the call if that kernel lets its dependents
+ * start early (this library's kernels never write the bases).
  * Returns STIEF_OK or an argument error (nothing launched).
  */
 STIEF_API stief_status stief_compress_append(const uint16_t* k_new, const uint16_t* v_new,
@@ -124,13 +128,18 @@ STIEF_API int stief_decode_auto_splits(int B, int Hq, int Hkv, int max_seq_len, 
  * stief_decode_workspace_bytes -- bytes of device workspace stief_decode_attention
  * needs for these sizes, for any split count it may use (at most
  * stief_decode_max_splits(max_seq_len)).  The workspace holds one ticket counter
- * per (sequence, KV head, query sub-group) and one per sequence, followed by the
- * per-split partial states: for each query head, the split's unnormalised latent
- * output o~ (r_V floats), its running maximum and sum, and two pad words; the last
- * CTA of a (sequence, KV head, sub-group) merges them and up-projects once.  The size
- * is computed for records of d + 4 floats (r_V <= d), so rV is validated but does not
- * change it.  The same workspace serves stief_append_decode and stief_decode_latent.
- * Pure host function.  Returns 0 for invalid arguments.
+ * per (sequence, KV head, query sub-group) and one per sequence (padded together to
+ * 256 bytes), followed by the per-split partial states: for each query head, the
+ * split's latent output o~ scaled to its running maximum (r_V values), that maximum
+ * and its sum.  When the whole grid fits on the GPU at once they are 8-byte words
+ * (an fp32 value and a tag saying it was written; the CTA of split s merges heads
+ * s, s + S, ... as soon as every split's words are there, then zeroes them); otherwise
+ * r_V + 4 floats, merged by the last CTA to take a ticket.  Either way the size is
+ * B*Hkv*ceil(G/G_T)*G_T*splits*(d+2)*8 bytes after the counters (G = Hq/Hkv, G_T the
+ * smallest of 1, 2, 4, 8 that is >= min(G, 8), splits = stief_decode_max_splits), so
+ * rV is validated but does not change it.  The same workspace serves
+ * stief_append_decode and stief_decode_latent.  Pure host function.  Returns 0 for
+ * invalid arguments.
  */
 STIEF_API size_t stief_decode_workspace_bytes(int B, int Hq, int Hkv, int rV, int max_seq_len);
 
@@ -166,19 +175,23 @@ STIEF_API size_t stief_decode_workspace_bytes(int B, int Hq, int Hkv, int rV, in
  *   workspace    : device scratch of at least workspace_bytes >=
  *                  stief_decode_workspace_bytes(B, Hq, Hkv, rV, max_seq_len)
  *                  bytes.  Zero-fill it once before its first use: its ticket
- *                  counters must be zero when a call starts, and every call that
- *                  runs to completion leaves them at zero again, so the same
- *                  workspace serves any later call (any sizes) on the same
- *                  stream without clearing.  After a call whose dev_status reports
- *                  a timeout, zero it again
+ *                  counters and merge words must be zero when a call starts, and
+ *                  every call that runs to completion leaves them at zero again,
+ *                  so the same workspace serves any later call (any sizes) on the
+ *                  same stream without clearing.  After a call whose dev_status
+ *                  reports a timeout, zero it again
  *   max_seq_len  : host-side upper bound of seq_lens (<= L_max); sizes the grid
  *   num_splits   : 0 = automatic, otherwise the number of KV splits per sequence
  *                  (1 .. stief_decode_max_splits(max_seq_len))
  *
  * One kernel runs on `stream`, a CTA per (split, KV head, query sub-group,
- * sequence): query projection, scores, online softmax, latent value mix and
- * up-projection over its token range; the last CTA of each (sequence, KV head,
- * sub-group) to finish merges the splits (log-sum-exp).  The kernel is launched
+ * sequence): query projection, scores, online softmax and latent value mix over
+ * its token range; the splits of each (sequence, KV head, sub-group) are merged
+ * (log-sum-exp) and up-projected once, through the workspace (see
+ * stief_decode_workspace_bytes).  The merge that waits for the other splits' words
+ * assumes every CTA of the grid can run at once, as on an otherwise idle GPU; a
+ * kernel on another stream that holds SMs until this one finishes would make that
+ * wait run out (STIEF_DEV_WAIT_TIMEOUT after 2 s).  The kernel is launched
  * as a programmatic dependent of the preceding work in the stream: it may be
  * scheduled while that work drains and reads no input before it has completed,
  * except P_K, which it requests first so that its latency overlaps that work: P_K
@@ -400,17 +413,19 @@ STIEF_API stief_status stief_decode_latent_joint_v(
  * workspace / workspace_bytes.  The per-split partial states live in a fixed 8 MiB
  * array of device memory owned by the library (one per GPU that loads it, held
  * until the process exits).  Sizes whose partial states, for the split count
- * actually used, exceed 8 MiB -- B*Hkv*ceil(G/G_T)*G_T*splits*(d+4)*4 bytes with
+ * actually used, exceed 8 MiB -- B*Hkv*ceil(G/G_T)*G_T*splits*(d+2)*8 bytes with
  * G = Hq/Hkv and G_T the smallest of 1, 2, 4, 8 that is >= min(G, 8) -- plus the
  * ticket counters, return
  * STIEF_ERR_WORKSPACE and launch nothing.  The first call on each device looks up
  * the array's device address (cudaGetSymbolAddress) with that device current; make
  * that first call before any stream capture.  All calls on a device share the
  * array: calls whose kernels overlap on the GPU race on it, so the caller must
- * order them (e.g. one stream).  The array keeps the last call's contents; its
- * ticket counters are zero at load and every call that runs to completion leaves
- * them at zero, so nothing needs clearing between calls.  Calls no cudaMalloc,
- * cudaFree or allocating library routine.
+ * order them (e.g. one stream).  The array keeps the last call's contents.  Its
+ * ticket counters and merge words must be zero when a kernel starts; a call that
+ * stopped early (STIEF_DEV_WAIT_TIMEOUT) may leave them otherwise, and the caller
+ * cannot reach the array, so every call zeroes the part it uses with
+ * cudaMemsetAsync on `stream` before its launch (a memset, not an allocation).
+ * Calls no cudaMalloc, cudaFree or allocating library routine.
  */
 STIEF_API stief_status stief_decode_attention_noalloc(
     const uint16_t* q, const uint16_t* P_K, const uint16_t* P_V, const uint16_t* k_lat,

@@ -7,11 +7,10 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-# Files collected after all others, in this order: the no-allocation entry point, then the
-# newest GPU paths (whose cases had not yet run on a GPU when they were written).  With -x a
-# failure in one of the newest then cannot hide the results of the established files.
-RUN_LAST = ("test_zz_no_alloc.py", "test_gauge_gpu.py", "test_joint_gpu.py",
-            "test_bench_modes_gpu.py")
+# Files collected after all others, in this order.  The file of the no-allocation entry point
+# comes last of all, so that with -x a failure there cannot hide any other file's results.
+RUN_LAST = ("test_gauge_gpu.py", "test_joint_gpu.py", "test_bench_modes_gpu.py",
+            "test_wait_timeout_gpu.py", "test_zz_no_alloc.py")
 
 
 def pytest_configure(config):

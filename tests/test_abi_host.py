@@ -246,12 +246,12 @@ def test_split_planning():
 
 
 def test_workspace_bytes():
-    # ticket counters (uint32 per unit, padded to 256 B), then
-    # (units + B) ticket counters padded to 256 bytes, then [units * G_T * max_splits]
-    # partial states of (d + 4) floats: the up-projected output row, m, l and two pad
-    # words (the value rank does not change the size)
-    assert stief.stief_decode_workspace_bytes(1, 32, 8, 64, 32768) == 256 + 8 * 4 * 256 * 132 * 4
-    assert stief.stief_decode_workspace_bytes(2, 24, 8, 48, 100) == 256 + 16 * 4 * 1 * 132 * 4
-    assert stief.stief_decode_workspace_bytes(64, 32, 8, 64, 4096) == 2304 + 512 * 4 * 32 * 132 * 4
+    # (units + B) uint32 ticket counters padded to 256 bytes, then [units * G_T * max_splits]
+    # partial-state records of (d + 2) 8-byte words: a tagged record holds o~[r_V], m and l
+    # as (value, tag) words, a ticket record r_V + 4 floats (the value rank does not change
+    # the size)
+    assert stief.stief_decode_workspace_bytes(1, 32, 8, 64, 32768) == 256 + 8 * 4 * 256 * 130 * 8
+    assert stief.stief_decode_workspace_bytes(2, 24, 8, 48, 100) == 256 + 16 * 4 * 1 * 130 * 8
+    assert stief.stief_decode_workspace_bytes(64, 32, 8, 64, 4096) == 2304 + 512 * 4 * 32 * 130 * 8
     assert stief.stief_decode_workspace_bytes(1, 32, 8, 72, 100) == 0
     assert stief.stief_decode_workspace_bytes(1, 30, 8, 64, 100) == 0

@@ -1,11 +1,14 @@
 """stief_decode_attention_noalloc: the decode entry point for callers that cannot allocate.
 
-It keeps its split partial states in a fixed device array owned by the library
-instead of a caller workspace.  These tests call it through the C ABI and check
-its output against stief_decode_attention (the workspace entry point) within the
-parity tolerance, on two calls in a row with different inputs, and that sizes
-beyond its fixed scratch are refused before anything is launched.  It passes alone in a
-fresh process as well as after the other GPU files.
+Some callers cannot allocate device memory where they decode: a serving engine whose
+KV-cache pool already holds nearly all of HBM, an operator interface that passes only
+inputs and outputs, or a loop that must not call cudaMalloc.  This entry point keeps its
+split partial states in a fixed device array owned by the library instead of a caller
+workspace.  These tests call it through the C ABI and check its output against
+stief_decode_attention (the workspace entry point) and against the fp64 oracle, within the
+parity tolerance, on two calls in a row with different inputs, and that sizes beyond its
+fixed scratch are refused before anything is launched.  They pass alone in a fresh process
+as well as after the other GPU files.
 """
 import ctypes
 
@@ -13,7 +16,7 @@ import pytest
 import torch
 
 import decode_attention_stief_b200 as stief
-from gpu_util import DECODE_TOL, decode_error, f64, make_decode_case
+from gpu_util import DECODE_TOL, decode_error, f64, make_decode_case, oracle_decode
 
 pytestmark = pytest.mark.gpu
 
@@ -39,10 +42,12 @@ def test_noalloc_matches_workspace_entry_point_two_calls():
     case1 = make_decode_case(2, 32, 8, 64, 48, 3000, 4242)
     got1, ref1 = _both(case1, [3000, 1777], 3000)
     assert decode_error(got1, f64(ref1)) <= DECODE_TOL
+    assert decode_error(got1, oracle_decode(*case1, [3000, 1777])) <= DECODE_TOL
     # second call right after, different sizes: the scratch holds the first call's data
     case2 = make_decode_case(3, 16, 2, 32, 96, 700, 4343)
     got2, ref2 = _both(case2, [700, 0, 129], 700)
     assert decode_error(got2, f64(ref2)) <= DECODE_TOL
+    assert decode_error(got2, oracle_decode(*case2, [700, 0, 129])) <= DECODE_TOL
     assert torch.all(got2[1].float() == 0)
 
 
