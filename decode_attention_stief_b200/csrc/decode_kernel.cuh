@@ -1087,7 +1087,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
   // ---- up-projection o = o~ P_V^T on the MMA: o^T[i][n] = sum_j P_V[i][j] o~^T[j][n] ----
   // (M = d, N = heads, K = r_V) from the normalised o~ in qt; warp w takes rows 16 w,
   // 16 (w + NW + 1), ...
-  auto up_project = [&]() {
+  auto up_project = [&](int nheads, int hbase, int hstride) {
     if (!setup_ok || !warp_wait(setup_bar, 1, a.dev_status)) return;
     for (int mt = warp; mt < d / 16; mt += NW + 1) {
       float c[NB][4];
@@ -1109,7 +1109,8 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
       for (int e = 0; e < 4; ++e) {
         const float o = NB == 1 ? c[0][e] + __shfl_xor_sync(kFull, c[0][e], 2) : c[0][e] + c[NB - 1][e];
         const int head = hA + (e & 1), i = 16 * mt + (lane >> 2) + 8 * (e >> 1);
-        if (!lo_lane && head < gcount) a.out[((size_t)b * a.Hq + h0 + head) * d + i] = f32_to_bf16_rn(o);
+        if (!lo_lane && head < nheads)
+          a.out[((size_t)b * a.Hq + h0 + hbase + head * hstride) * d + i] = f32_to_bf16_rn(o);
       }
     }
   };
@@ -1120,7 +1121,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
         a.out[((size_t)b * a.Hq + h0 + h) * rV + j] = f32_to_bf16_rn(qt[h * xs + j]);
       }
     } else if (ok) {
-      up_project();
+      up_project(gcount, 0, 1);
     }
     return;
   }
@@ -1140,9 +1141,6 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
     const int nh = (gcount - s_idx + S - 1) / S;  // heads s_idx + hh S, hh < nh
     const int RP = RW / 2;                        // 16-byte word pairs per record
     float* stg = reinterpret_cast<float*>(smem + L.region);  // [nh][S][RW] the records' values
-    float* wts = stg + nh * S * RW;                           // [nh][S] weights of the splits
-    float* invl = wts + nh * S;                               // [8] 1 / merged sum
-    float* ob = invl + 8;                                     // [nh][rV] merged o~
     const uint64_t* ubase = a.ws_words + (size_t)unit * S * G_T * RW;
     const int items = nh * S * RP;
     auto item_src = [&](int i) {
@@ -1176,68 +1174,41 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
       }
     }
     __syncthreads();
-    if (warp < nh) {  // warp hh: the maximum over the splits, their weights and the sum
-      const float* r = stg + warp * S * RW;
+    // the words read are in shared memory now: zero them for the next call (these stores
+    // drain while the merge below runs)
+    for (int i = tid; i < items; i += NT) st_tagged2(const_cast<uint64_t*>(item_src(i)), 0ull, 0ull);
+    // merged, normalised o~ of head s_idx + hh S, columns 2p and 2p + 1: each thread forms
+    // the splits' maximum and weights itself (no separate pass), into row hh of qt
+    for (int t = tid; t < nh * (rV / 2); t += NT) {
+      const int hh = t / (rV / 2), p2 = 2 * (t - hh * (rV / 2));
+      const float* r = stg + hh * S * RW;
       float M = -INFINITY;
-      for (int sp = lane; sp < S; sp += 32) M = fmaxf(M, r[sp * RW + rV]);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
-      float Ls = 0.f;
-      for (int sp = lane; sp < S; sp += 32) {
-        const float m = r[sp * RW + rV];
+#pragma unroll 4
+      for (int sp = 0; sp < S; ++sp) M = fmaxf(M, r[sp * RW + rV]);
+      float o0 = 0.f, o1 = 0.f, Ls = 0.f;
+#pragma unroll 4
+      for (int sp = 0; sp < S; ++sp) {
+        const float* rs = r + sp * RW;
+        const float m = rs[rV];
         const float wgt = m == -INFINITY ? 0.f : ex2(m - M);  // 0 for a split with no token
-        wts[warp * S + sp] = wgt;
-        Ls = fmaf(wgt, r[sp * RW + rV + 1], Ls);
+        const float2 v = *reinterpret_cast<const float2*>(rs + p2);
+        o0 = fmaf(wgt, v.x, o0);
+        o1 = fmaf(wgt, v.y, o1);
+        Ls = fmaf(wgt, rs[rV + 1], Ls);
       }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) Ls += __shfl_xor_sync(kFull, Ls, o);
-      if (lane == 0) invl[warp] = Ls > 0.f ? 1.f / Ls : 0.f;
-    }
-    __syncthreads();
-    for (int i = tid; i < nh * rV; i += NT) {  // merged, normalised o~
-      const int hh = i / rV, j = i - hh * rV;
-      const float* r = stg + hh * S * RW + j;
-      const float* wv = wts + hh * S;
-      float oa = 0.f, obb = 0.f;  // two chains
-      int sp = 0;
-      for (; sp + 1 < S; sp += 2) {
-        oa = fmaf(wv[sp], r[sp * RW], oa);
-        obb = fmaf(wv[sp + 1], r[(sp + 1) * RW], obb);
-      }
-      if (sp < S) oa = fmaf(wv[sp], r[sp * RW], oa);
-      ob[i] = (oa + obb) * invl[hh];
+      const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+      qt[hh * xs + p2] = o0 * inv;
+      qt[hh * xs + p2 + 1] = o1 * inv;
     }
     __syncthreads();
     if (LAT) {  // o~ is the result
       for (int i = tid; i < nh * rV; i += NT) {
         const int hh = i / rV, j = i - hh * rV;
-        a.out[((size_t)b * a.Hq + h0 + s_idx + hh * S) * rV + j] = f32_to_bf16_rn(ob[i]);
+        a.out[((size_t)b * a.Hq + h0 + s_idx + hh * S) * rV + j] = f32_to_bf16_rn(qt[hh * xs + j]);
       }
-    } else if (setup_ok && mbar_wait_bounded(setup_bar, 1u, a.dev_status)) {
-      // o = o~ P_V^T on the CUDA cores in fp32: two lanes per output row, each taking every
-      // other 16-byte chunk of the row of P_V (whole warps: nh d 2 is a multiple of 32)
-      for (int i = tid; i < nh * d * 2; i += NT) {
-        const int half = i & 1, ri = i >> 1, hh = ri / d, row = ri - hh * d;
-        const float* o8 = ob + hh * rV;
-        float acc = 0.f;
-        for (int c = half; c < rV / 8; c += 2) {
-          const uint4 pv = lds128(smem_u32(pmat) + swz(locate(rV, d, c), row));
-          const float* x = o8 + 8 * c;
-          acc = fmaf(bf16lo(pv.x), x[0], acc);
-          acc = fmaf(bf16hi(pv.x), x[1], acc);
-          acc = fmaf(bf16lo(pv.y), x[2], acc);
-          acc = fmaf(bf16hi(pv.y), x[3], acc);
-          acc = fmaf(bf16lo(pv.z), x[4], acc);
-          acc = fmaf(bf16hi(pv.z), x[5], acc);
-          acc = fmaf(bf16lo(pv.w), x[6], acc);
-          acc = fmaf(bf16hi(pv.w), x[7], acc);
-        }
-        acc += __shfl_xor_sync(kFull, acc, 1);
-        if (half == 0) a.out[((size_t)b * a.Hq + h0 + s_idx + hh * S) * d + row] = f32_to_bf16_rn(acc);
-      }
+    } else {
+      up_project(nh, s_idx, S);  // MMA columns 0 .. nh-1 carry the merged heads
     }
-    // the words read here are zero again for the next call
-    for (int i = tid; i < items; i += NT) st_tagged2(const_cast<uint64_t*>(item_src(i)), 0ull, 0ull);
     return;
   }
   // Split partial states stay in the latent space (o~ scaled to the CTA's maximum, r_V floats
@@ -1369,7 +1340,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
   }
   if (!LAT) {
     __syncthreads();
-    up_project();
+    up_project(gcount, 0, 1);
   }
 }
 
