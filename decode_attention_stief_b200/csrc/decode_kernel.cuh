@@ -54,7 +54,7 @@
 
 namespace stief {
 
-constexpr int kPreIssue = 1;         // stages per warp requested together with q
+constexpr int kPreIssue = 1;         // stages per warp requested before the length is known
 constexpr float kRescaleTau = 8.0f;  // lazy-rescale threshold (log2 units)
 constexpr uint32_t kFull = 0xffffffffu;
 
@@ -394,8 +394,6 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
   // the tensor maps are kernel parameters, not inputs: bring them in before the wait
   if (producer && lane < 12 && lane < a.nmaps) prefetch_tensormap(&a.maps[lane]);
   __syncthreads();
-  // inputs may come from the preceding kernel in the stream: read nothing before this
-  pdl_wait();
 
   // ---- split range and tiles --------------------------------------------------------------
   // Splits partition [0, S * chunk) by the host bound max_seq_len (the grid was sized by it),
@@ -457,20 +455,41 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
       if (p < npv) tma_load_2d(dst + vo[p], vmap[p], vx[p], yv, bar, policy);
   };
 
-  // q and each warp's first tile are requested before the length is read (its latency then
-  // overlaps theirs): the producer's lane 0 sends q (its bytes join P_K's on the setup
-  // barrier, whose one arrival waits for the length), lane w the first tile of consumer warp
-  // w by the host bound.  The rest of the rings follows once q has landed (requested with it,
-  // their flood of misses would hold up q's copy for microseconds).  Tiles past the sequence
-  // are never consumed and are waited for before the ring is reused.
+  // Contiguous bf16 caches (plain and latent modes): every warp's first tile is requested
+  // before the dependency wait, like P_K, so that it streams while the preceding kernel
+  // finishes (requesting whole rings there measured slower: the flood delays some CTAs'
+  // data by microseconds).  The calls document that the kernel immediately preceding them
+  // must not write the cache rows below the lengths, except the row just below each length
+  // (the one a preceding fused step on the same caches appends), which is read again after
+  // the wait.
+  constexpr bool EARLY = MODE == kModePlain || MODE == kModeLatent;
   int ring_issued = 0;  // producer lane w: tiles [0, ring_issued) of warp w are requested
+  if (EARLY && producer && lane < NW) {
+    const uint64_t stream = l2_policy_evict_first();
+    ring_issued = min(min(kPreIssue, ns), warp_tiles(lane, spec_tiles));
+    for (int k = 0; k < ring_issued; ++k) issue(lane, k, stream);
+  }
+  // inputs may come from the preceding kernel in the stream: read nothing else before this
+  pdl_wait();
+  // the next kernel in the stream may be scheduled now (its CTAs take SMs as ours exit)
+  pdl_launch_dependents();
+
+  // q is requested before the length is read (its latency then overlaps the length's): the
+  // producer's lane 0 sends q (its bytes join P_K's on the setup barrier, whose one arrival
+  // waits for the length; the latent mode's q~ rows complete the barrier at once).  The other
+  // modes' warps get their first tile now by the host bound and the rest of the rings once q
+  // has landed (requested with it, their flood of misses would hold up q's copy).  Tiles past
+  // the sequence are never consumed and are waited for before the ring is reused.
   if (producer) {
-    if (lane == 0 && !LAT) {
+    if (lane == 0 && LAT) {
+      mbar_arrive_expect_tx(setup_bar, 2u * gcount * rK + stall);
+      bulk_g2s(smem + L.qraw, a.q + ((size_t)b * a.Hq + h0) * rK, 2u * gcount * rK, setup_bar);
+    } else if (lane == 0) {
       asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(setup_bar)),
                    "r"(2u * gcount * d) : "memory");
       bulk_g2s(smem + L.qraw, a.q + ((size_t)b * a.Hq + h0) * d, 2u * gcount * d, setup_bar);
     }
-    if (lane < NW) {
+    if (!EARLY && lane < NW) {
       const uint64_t stream = l2_policy_evict_first();
       ring_issued = min(min(kPreIssue, ns), warp_tiles(lane, spec_tiles));
       for (int k = 0; k < ring_issued; ++k) issue(lane, k, stream);
@@ -518,11 +537,8 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
   // ---- prologue ------------------------------------------------------------------------------
   bool ok = true;
   if (producer) {
-    if (LAT) {  // latent decode: the rows of q~ are the input (no new rows: no append)
-      if (lane == 0) {
-        mbar_arrive_expect_tx(setup_bar, 2u * gcount * rK + stall);
-        bulk_g2s(smem + L.qraw, a.q + ((size_t)b * a.Hq + h0) * rK, 2u * gcount * rK, setup_bar);
-      }
+    if (LAT) {
+      // latent decode: the rows of q~ (requested above) are the input; no new rows, no append
     } else if (lane == 0) {
       // the new rows of the fused step follow once the length says which CTA holds the new
       // token: their bytes and the barrier's one arrival are added then
@@ -811,6 +827,22 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
         if (lane == 0) mbar_arrive(&empty[warp * ns + st]);  // the raw stage may be refilled
         sbase = smem_u32(staging);
       }
+      if (EARLY && k < kPreIssue && Lb >= 1 && tok0 <= Lb - 1 && Lb - 1 < tok0 + kTile) {
+        // this tile was requested before the dependency wait: the row just below the length
+        // may have been appended by the preceding kernel (a fused step on the same caches),
+        // so it is read again now (L2; the wait made it visible)
+        const int r_prev = Lb - 1 - tok0;
+        const long long prow = cache_row(cr, b, kvh, Lb - 1);
+        for (int cch = lane; cch < (rK + rV) / 8; cch += 32) {
+          const bool key = cch < rK / 8;
+          const uint4 v = key ? __ldcg(reinterpret_cast<const uint4*>(a.k_lat_w + prow * rK) + cch)
+                              : __ldcg(reinterpret_cast<const uint4*>(a.v_lat_w + prow * rV) + (cch - rK / 8));
+          const PieceLoc pt = key ? locate(rK, kTile, cch) : locate(rV, kTile, cch - rK / 8);
+          *reinterpret_cast<uint4*>(ring + (size_t)st * st_bytes + (key ? 0u : kt_bytes) + swz(pt, r_prev)) = v;
+        }
+        fence_proxy_async_smem();  // generic writes into a stage the TMA engine fills
+        __syncwarp();
+      }
       if (owns_new && tok0 <= Lb && Lb < tok0 + kTile) {
         // This tile holds the new token, whose cache rows were not written yet when the tile
         // was fetched: put the projected rows (key row from the prologue, value row from
@@ -994,7 +1026,6 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
       if (!Q8 && lane == 0) mbar_arrive(&empty[warp * ns + st]);  // the stage may be refilled
     }
   }
-  pdl_launch_dependents();
 
   // ---- merge the warps ------------------------------------------------------------------
   // (a) every warp's running maximum and sum per head; (b) the CTA's maximum per head, to

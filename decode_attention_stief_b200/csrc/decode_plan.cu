@@ -214,6 +214,10 @@ stief_status plan_decode(DecodeArgs& a, const uint16_t* q, const uint16_t* P_K,
   a.q = q;
   a.seq_lens = seq_lens;
   a.out = out;
+  // the caches' base pointers (the tiles come through the tensor maps; the fused step writes
+  // its new rows here, and the kernel reads the row just below each length again here)
+  a.k_lat_w = const_cast<uint16_t*>(k_lat);
+  a.v_lat_w = const_cast<uint16_t*>(v_lat);
   a.dev_status = dev_status;
   a.B = B;
   a.Hq = Hq;

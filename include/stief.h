@@ -194,12 +194,18 @@ STIEF_API size_t stief_decode_workspace_bytes(int B, int Hq, int Hkv, int rV, in
  * wait run out (STIEF_DEV_WAIT_TIMEOUT after 2 s).  The kernel is launched
  * as a programmatic dependent of the preceding work in the stream: it may be
  * scheduled while that work drains and reads no input before it has completed,
- * except P_K, which it requests first so that its latency overlaps that work: P_K
- * must not be written by the kernel that immediately precedes the call in the
- * stream if that kernel lets its dependents start early (programmatic dependent
- * launch).  This library's kernels never write the bases.  The same holds for the
- * other calls that take P_K (stief_append_decode and the _noalloc, _paged and _q8
- * decodes).
+ * except P_K and the first tiles of k_lat and v_lat, which it requests first so
+ * that their latency overlaps that work.  So if the kernel that immediately
+ * precedes the call in the stream lets its dependents start early (programmatic
+ * dependent launch), it must write neither P_K nor any row of k_lat or v_lat
+ * below seq_lens[b] - 1; the row just below each length is read again after the
+ * wait, so stief_append_decode calls may follow one another on the same caches.
+ * This library's kernels never write the bases, and its compress calls end with a
+ * kernel that lets no dependent start early.  The rule on P_K holds for every call
+ * that takes it (stief_append_decode and the _noalloc, _paged and _q8 decodes);
+ * the rule on the cache rows for stief_append_decode, stief_decode_latent and
+ * stief_decode_attention_noalloc (the _paged, _q8 and _joint_v calls read no cache
+ * row before the wait).
  * Returns STIEF_OK or an argument error (nothing launched).
  */
 STIEF_API stief_status stief_decode_attention(const uint16_t* q, const uint16_t* P_K,

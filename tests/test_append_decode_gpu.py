@@ -201,3 +201,42 @@ def test_append_decode_equals_two_calls():
     assert np.max(np.abs(ulps)) <= 1.0
     ref = f64(out2.cpu())
     assert np.max(np.abs(f64(got) - ref)) <= DECODE_TOL * np.max(np.abs(ref))
+
+
+@pytest.mark.parametrize("num_splits", [0, 6])
+def test_back_to_back_steps_without_host_sync(num_splits):
+    """Fused steps queued back to back on the same caches (nothing between them, no host
+    synchronisation) equal the oracle's steps in sequence.  Each launch requests its first
+    tiles before its dependency wait, while the launch before it may still be appending the
+    row just below the new length; the kernel reads that row again after the wait.  A latent
+    decode queued right after the last step sees the grown caches as well."""
+    dev = torch.device("cuda")
+    lens = [700, 129, 0]
+    B, Hq, Hkv, rK, rV, L_max = 3, 8, 2, 64, 64, 800
+    q, _, _, P_K, P_V, k_lat, v_lat = _case(B, Hq, Hkv, rK, rV, L_max, lens, 3800)
+    qd, Pk, Pv, gk, gv = (x.to(dev).contiguous() for x in (q, P_K, P_V, k_lat, v_lat))
+    lens_t = torch.as_tensor(np.asarray(lens, np.int32)).to(dev)
+    ws = stief.workspace_for(B, Hq, Hkv, rV, L_max)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    steps = []
+    for step in range(5):
+        kn, vn = si.full_kv(3900 + step, B, Hkv, 1, 128)
+        kn, vn = kn[:, :, 0].contiguous(), vn[:, :, 0].contiguous()
+        out = torch.full((B, Hq, 128), float("nan"), dtype=torch.bfloat16, device=dev)
+        stief.stief_append_decode(qd, kn.to(dev), vn.to(dev), Pk, Pv, gk, gv, lens_t, out, ws,
+                                  L_max, num_splits=num_splits, dev_status=status)
+        steps.append((kn, vn, out))
+    q_lat = si.queries(3950, B, Hq, rK).to(dev)
+    o_lat = torch.empty((B, Hq, rV), dtype=torch.bfloat16, device=dev)
+    stief.stief_decode_latent(q_lat, gk, gv, lens_t, o_lat, ws, L_max, num_splits=num_splits,
+                              dev_status=status)
+    assert stief.stief_read_device_status(status) == 0
+    wk, wv, wl = f64(k_lat), f64(v_lat), np.asarray(lens, np.int32)
+    for kn, vn, out in steps:
+        wk, wv, wl, _ = oracle.compress_append(f64(kn)[:, :, None], f64(vn)[:, :, None],
+                                               f64(P_K), f64(P_V), wk, wv, wl)
+        want = oracle.decode(f64(q), f64(P_K), f64(P_V), wk, wv, wl)
+        assert decode_error(out.cpu(), want) <= DECODE_TOL
+    assert lens_t.cpu().tolist() == wl.tolist() == [L + 5 for L in lens]
+    want_l = oracle.decode_latent(f64(q_lat), wk, wv, wl, d=128)
+    assert decode_error(o_lat.cpu(), want_l) <= DECODE_TOL
