@@ -220,8 +220,9 @@ __device__ __forceinline__ void bfrag_hilo(const float* X, int xs, int ks, int l
   const int n = lane >> 2;
   const int c = 16 * ks + 2 * (lane & 3);
   const int head = NB == 1 ? (n & 3) : n;
-  const float2 x = *reinterpret_cast<const float2*>(X + head * xs + c);
-  const float2 y = *reinterpret_cast<const float2*>(X + head * xs + c + 8);
+  const uint32_t xa = smem_u32(X + head * xs + c);
+  const float2 x = lds_f32x2(xa);
+  const float2 y = lds_f32x2(xa + 32u);
   const uint32_t hx = f16 ? hi_pair_h(x.x, x.y) : hi_pair(x.x, x.y);
   const uint32_t hy = f16 ? hi_pair_h(y.x, y.y) : hi_pair(y.x, y.y);
   const uint32_t lx = f16 ? lo_pair_h(x.x, x.y, hx) : lo_pair(x.x, x.y, hx);
@@ -576,12 +577,16 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
     const int n = lane >> 2;  // B column = head
     ok = warp_wait(setup_bar, 0, a.dev_status);
     if (!ok && lane == 0) flag[1] = 1;
-    uint32_t qb[8][2];  // d / 16 k-steps
-    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(smem + L.qraw) + min(n, gcount - 1) * (d / 2);
+    uint32_t qb[8][2];  // d / 16 k-steps (explicit shared loads issued together)
+    const uint32_t qrowb = smem_u32(smem + L.qraw) + 4u * (uint32_t)(min(n, gcount - 1) * (d / 2) + (lane & 3));
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
-      qb[ks][0] = n < gcount ? qrow[8 * ks + (lane & 3)] : 0u;
-      qb[ks][1] = n < gcount ? qrow[8 * ks + 4 + (lane & 3)] : 0u;
+      qb[ks][0] = lds_u32(qrowb + 32u * ks);
+      qb[ks][1] = lds_u32(qrowb + 32u * ks + 16u);
+    }
+    if (n >= gcount) {  // absent heads are zero columns
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) qb[ks][0] = qb[ks][1] = 0u;
     }
     // append: the new key row k_down = k_new P_K is the same contraction with B column 0 =
     // k_new (fp32 accumulation, one rounding to bf16).  Tasks 0..nks-1 are the q~ m-tiles,
@@ -607,10 +612,11 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
       }
       const int j = 16 * mt + (lane >> 2), hh = 2 * (lane & 3);
       if (!key) {
-        qt[hh * xs + j] = c[0] * a.qscale;
-        qt[(hh + 1) * xs + j] = c[1] * a.qscale;
-        qt[hh * xs + j + 8] = c[2] * a.qscale;
-        qt[(hh + 1) * xs + j + 8] = c[3] * a.qscale;
+        const uint32_t qtb = smem_u32(qt);
+        sts_f32(qtb + 4u * (uint32_t)(hh * xs + j), c[0] * a.qscale);
+        sts_f32(qtb + 4u * (uint32_t)((hh + 1) * xs + j), c[1] * a.qscale);
+        sts_f32(qtb + 4u * (uint32_t)(hh * xs + j + 8), c[2] * a.qscale);
+        sts_f32(qtb + 4u * (uint32_t)((hh + 1) * xs + j + 8), c[3] * a.qscale);
       } else if ((lane & 3) == 0) {  // column 0: k_down[j], k_down[j + 8]
         uint16_t* kl = reinterpret_cast<uint16_t*>(smem + L.newlat);
         kl[j] = f32_to_bf16_rn(c[0]);
@@ -1051,14 +1057,22 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
   }
   __syncthreads();  // every warp is done with its ring: the region becomes the reduction buffer
   float* red = reinterpret_cast<float*>(smem + L.region);  // [NW][8][rV]
+  // (explicit shared accesses issued in batches: see lds_f32)
+  const uint32_t mlb = smem_u32(ml), redb = smem_u32(red);
   if (!producer) {
-    float MA = -INFINITY, MB = -INFINITY;
+    float va[kMaxConsumerWarps], vb[kMaxConsumerWarps];
 #pragma unroll
-    for (int w = 0; w < kMaxConsumerWarps; ++w)
-      if (w < NW) {
-        MA = fmaxf(MA, ml[(w * 8 + hA) * 2]);
-        MB = fmaxf(MB, ml[(w * 8 + hA + 1) * 2]);
-      }
+    for (int w = 0; w < kMaxConsumerWarps; ++w) {
+      const int ww = w < NW ? w : 0;  // a repeat of warp 0 changes no maximum
+      va[w] = lds_f32(mlb + 8u * (uint32_t)(ww * 8 + hA));
+      vb[w] = lds_f32(mlb + 8u * (uint32_t)(ww * 8 + hA + 1));
+    }
+    float MA = va[0], MB = vb[0];
+#pragma unroll
+    for (int w = 1; w < kMaxConsumerWarps; ++w) {
+      MA = fmaxf(MA, va[w]);
+      MB = fmaxf(MB, vb[w]);
+    }
     const float fA = mA == -INFINITY ? 0.f : ex2(mA - MA);  // 0 for a warp that saw no token
     const float fB = mB == -INFINITY ? 0.f : ex2(mB - MB);
     if (!lo_lane) {
@@ -1067,11 +1081,12 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
         if (mt < nmv)
 #pragma unroll
           for (int e = 0; e < 4; ++e)
-            red[(warp * 8 + hA + (e & 1)) * rV + 16 * mt + (lane >> 2) + 8 * (e >> 1)] =
-                ov[mt][e] * ((e & 1) ? fB : fA);
+            sts_f32(redb + 4u * (uint32_t)((warp * 8 + hA + (e & 1)) * rV + 16 * mt + (lane >> 2) +
+                                           8 * (e >> 1)),
+                    ov[mt][e] * ((e & 1) ? fB : fA));
       if ((lane >> 2) == 0) {  // the sums rescaled in place (only the maxima were read above)
-        ml[(warp * 8 + hA) * 2 + 1] = lA * fA;
-        ml[(warp * 8 + hA + 1) * 2 + 1] = lB * fB;
+        sts_f32(mlb + 8u * (uint32_t)(warp * 8 + hA) + 4u, lA * fA);
+        sts_f32(mlb + 8u * (uint32_t)(warp * 8 + hA + 1) + 4u, lB * fB);
         if (warp == 0) {
           fin[hA] = MA;
           fin[hA + 1] = MB;
@@ -1088,14 +1103,21 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
   uint64_t* my_words = tagged_merge ? a.ws_words + ((size_t)unit * S + s_idx) * G_T * RW : nullptr;
   for (int idx = tid; idx < HR * (rV / 2); idx += NT) {
     const int h = idx / (rV / 2), jj = 2 * (idx - h * (rV / 2));
+    float2 v[kMaxConsumerWarps];
+    float lw[kMaxConsumerWarps];
+#pragma unroll
+    for (int w = 0; w < kMaxConsumerWarps; ++w) {
+      const int ww = w < NW ? w : 0;
+      v[w] = lds_f32x2(redb + 4u * (uint32_t)((ww * 8 + h) * rV + jj));
+      lw[w] = lds_f32(mlb + 8u * (uint32_t)(ww * 8 + h) + 4u);
+    }
     float o0 = 0.f, o1 = 0.f, lsum = 0.f;
 #pragma unroll
     for (int w = 0; w < kMaxConsumerWarps; ++w)
       if (w < NW) {
-        const float2 v = *reinterpret_cast<const float2*>(red + (w * 8 + h) * rV + jj);
-        o0 += v.x;
-        o1 += v.y;
-        lsum += ml[(w * 8 + h) * 2 + 1];
+        o0 += v[w].x;
+        o1 += v[w].y;
+        lsum += lw[w];
       }
     if (S == 1) {
       o0 = lsum > 0.f ? o0 / lsum : 0.f;
@@ -1171,25 +1193,63 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
     }
     const int nh = (gcount - s_idx + S - 1) / S;  // heads s_idx + hh S, hh < nh
     const int RP = RW / 2;                        // 16-byte word pairs per record
-    float* stg = reinterpret_cast<float*>(smem + L.region);  // [nh][S][RW] the records' values
+    const int SP = (S + 3) & ~3;                  // splits padded to whole float4s
+    // The records' values, split-major per column: stg[(hh * RW + col) * SP + sp], so that a
+    // column's splits are contiguous (float4 loads); splits [S, SP) hold m = -inf, l = o = 0.
+    const uint32_t stgb = smem_u32(smem + L.region);
     const uint64_t* ubase = a.ws_words + (size_t)unit * S * G_T * RW;
-    const int items = nh * S * RP;
-    auto item_src = [&](int i) {
-      const int hh = i / (S * RP), r = i - hh * (S * RP), sp = r / RP, pr = r - sp * RP;
-      return ubase + ((size_t)sp * G_T + s_idx + hh * S) * RW + 2 * pr;
+    const int items = nh * S * RP;  // (record hh * S + sp, word pair)
+    for (int i = tid; i < nh * RW * (SP - S); i += NT) {
+      const int col = i / (SP - S), hh = col / RW;
+      sts_f32(stgb + 4u * (uint32_t)(col * SP + S + (i - col * (SP - S))),
+              col - hh * RW == rV ? -INFINITY : 0.f);
+    }
+    // A thread's items are tid, tid + NT, ...: their (hh, sp, pair) advance by fixed steps,
+    // so no item needs a division.
+    const int q_rec = NT / RP, q_pr = NT - q_rec * RP;
+    int c_pr, c_sp, c_hh;
+    auto first_item = [&]() {
+      c_pr = tid % RP;
+      const int rec = tid / RP;
+      c_hh = rec / S;
+      c_sp = rec - c_hh * S;
+    };
+    auto next_item = [&]() {
+      c_pr += q_pr;
+      int inc = q_rec;
+      if (c_pr >= RP) {
+        c_pr -= RP;
+        ++inc;
+      }
+      c_sp += inc;
+      while (c_sp >= S) {
+        c_sp -= S;
+        ++c_hh;
+      }
+    };
+    auto item_src = [&]() {
+      return ubase + ((size_t)c_sp * G_T + s_idx + c_hh * S) * RW + 2 * c_pr;
     };
     uint64_t t_wait = 0;  // when this thread first found a word not yet written
     bool gave_up = false;
     constexpr int kLd = 4;  // word pairs in flight per thread
+    first_item();
     for (int i0 = tid; i0 < items; i0 += kLd * NT) {
       uint64_t w0[kLd], w1[kLd];
-#pragma unroll
-      for (int u = 0; u < kLd; ++u)
-        if (i0 + u * NT < items) ld_tagged2(item_src(i0 + u * NT), w0[u], w1[u]);
+      const uint64_t* src[kLd];
+      uint32_t dst[kLd];
 #pragma unroll
       for (int u = 0; u < kLd; ++u) {
-        const int i = i0 + u * NT;
-        if (i >= items) continue;
+        if (i0 + u * NT < items) {
+          src[u] = item_src();
+          dst[u] = stgb + 4u * (uint32_t)((c_hh * RW + 2 * c_pr) * SP + c_sp);
+          ld_tagged2(src[u], w0[u], w1[u]);
+        }
+        next_item();
+      }
+#pragma unroll
+      for (int u = 0; u < kLd; ++u) {
+        if (i0 + u * NT >= items) continue;
         while ((tagged_tag(w0[u]) & tagged_tag(w1[u])) != 1u && !gave_up) {
           const uint64_t now = global_timer_ns();
           if (t_wait == 0) {
@@ -1198,44 +1258,51 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
             report(a.dev_status, STIEF_DEV_WAIT_TIMEOUT);
             gave_up = true;
           }
-          ld_tagged2(item_src(i), w0[u], w1[u]);
+          ld_tagged2(src[u], w0[u], w1[u]);
         }
-        stg[2 * i] = tagged_value(w0[u]);
-        stg[2 * i + 1] = tagged_value(w1[u]);
+        sts_f32(dst[u], tagged_value(w0[u]));
+        sts_f32(dst[u] + 4u * (uint32_t)SP, tagged_value(w1[u]));
       }
     }
     __syncthreads();
     // the words read are in shared memory now: zero them for the next call (these stores
     // drain while the merge below runs)
-    for (int i = tid; i < items; i += NT) st_tagged2(const_cast<uint64_t*>(item_src(i)), 0ull, 0ull);
-    // merged, normalised o~ of head s_idx + hh S, columns 2p and 2p + 1: each thread forms
-    // the splits' maximum and weights itself (no separate pass), into row hh of qt
-    for (int t = tid; t < nh * (rV / 2); t += NT) {
-      const int hh = t / (rV / 2), p2 = 2 * (t - hh * (rV / 2));
-      const float* r = stg + hh * S * RW;
+    first_item();
+    for (int i = tid; i < items; i += NT) {
+      st_tagged2(const_cast<uint64_t*>(item_src()), 0ull, 0ull);
+      next_item();
+    }
+    // merged, normalised o~ of head s_idx + hh S, column c: each thread forms the splits'
+    // maximum and weights itself, into row hh of qt
+    const uint32_t qtb = smem_u32(qt);
+    for (int t = tid; t < nh * rV; t += NT) {
+      const int hh = t / rV, c = t - hh * rV;
+      const uint32_t mrow = stgb + 4u * (uint32_t)((hh * RW + rV) * SP);
+      const uint32_t lrow = mrow + 4u * (uint32_t)SP, crow = stgb + 4u * (uint32_t)((hh * RW + c) * SP);
       float M = -INFINITY;
 #pragma unroll 4
-      for (int sp = 0; sp < S; ++sp) M = fmaxf(M, r[sp * RW + rV]);
-      float o0 = 0.f, o1 = 0.f, Ls = 0.f;
-#pragma unroll 4
-      for (int sp = 0; sp < S; ++sp) {
-        const float* rs = r + sp * RW;
-        const float m = rs[rV];
-        const float wgt = m == -INFINITY ? 0.f : ex2(m - M);  // 0 for a split with no token
-        const float2 v = *reinterpret_cast<const float2*>(rs + p2);
-        o0 = fmaf(wgt, v.x, o0);
-        o1 = fmaf(wgt, v.y, o1);
-        Ls = fmaf(wgt, rs[rV + 1], Ls);
+      for (int s4 = 0; s4 < SP; s4 += 4) {
+        const float4 m4 = lds128f(mrow + 4u * (uint32_t)s4);
+        M = fmaxf(M, fmaxf(fmaxf(m4.x, m4.y), fmaxf(m4.z, m4.w)));
       }
-      const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
-      qt[hh * xs + p2] = o0 * inv;
-      qt[hh * xs + p2 + 1] = o1 * inv;
+      float o = 0.f, Ls = 0.f;
+      auto wgt = [&](float m) { return m == -INFINITY ? 0.f : ex2(m - M); };  // 0: no token
+#pragma unroll 4
+      for (int s4 = 0; s4 < SP; s4 += 4) {
+        const uint32_t off = 4u * (uint32_t)s4;
+        const float4 m4 = lds128f(mrow + off), l4 = lds128f(lrow + off), v4 = lds128f(crow + off);
+        const float w0 = wgt(m4.x), w1 = wgt(m4.y), w2 = wgt(m4.z), w3 = wgt(m4.w);
+        o = fmaf(w0, v4.x, fmaf(w1, v4.y, fmaf(w2, v4.z, fmaf(w3, v4.w, o))));
+        Ls = fmaf(w0, l4.x, fmaf(w1, l4.y, fmaf(w2, l4.z, fmaf(w3, l4.w, Ls))));
+      }
+      sts_f32(qtb + 4u * (uint32_t)(hh * xs + c), Ls > 0.f ? o / Ls : 0.f);
     }
     __syncthreads();
     if (LAT) {  // o~ is the result
       for (int i = tid; i < nh * rV; i += NT) {
         const int hh = i / rV, j = i - hh * rV;
-        a.out[((size_t)b * a.Hq + h0 + s_idx + hh * S) * rV + j] = f32_to_bf16_rn(qt[hh * xs + j]);
+        a.out[((size_t)b * a.Hq + h0 + s_idx + hh * S) * rV + j] =
+            f32_to_bf16_rn(lds_f32(qtb + 4u * (uint32_t)(hh * xs + j)));
       }
     } else {
       up_project(nh, s_idx, S);  // MMA columns 0 .. nh-1 carry the merged heads

@@ -165,11 +165,11 @@ inline size_t decode_ws_tagged_bytes(size_t units, int G_T, int splits, int rV) 
   return units * (size_t)G_T * splits * (size_t)(rV + 2) * 8u;
 }
 // Shared-memory bytes the merging CTA of the tagged merge stages the records in: its heads'
-// records [nh][S][rV + 2], their weights [nh][S], eight inverse sums and the merged o~
-// [nh][rV], where nh <= ceil(G_T / S) heads are merged by one CTA.
+// records as [nh][rV + 2 columns][splits padded to a multiple of 4] floats, where
+// nh <= ceil(G_T / S) heads are merged by one CTA.
 inline size_t decode_tagged_stage_bytes(int G_T, int splits, int rV) {
   const int nh = (G_T + splits - 1) / splits;
-  return 4u * ((size_t)nh * splits * (rV + 2) + (size_t)nh * splits + 8 + (size_t)nh * rV);
+  return 4u * (size_t)nh * (rV + 2) * (size_t)((splits + 3) & ~3);
 }
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
 
