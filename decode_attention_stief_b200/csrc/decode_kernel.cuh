@@ -214,15 +214,17 @@ __device__ __forceinline__ int at_chunk(int lane) { return (lane >> 3) & 1; }
 // B fragments (k-step ks) of X^T for an fp32 matrix X[head][col] in shared memory (row
 // stride xs floats): column n = lane >> 2 of n-tile j is (head, part) as described at the
 // top; k = cols 16 ks + 2 (lane & 3) + {0, 1} (first register) and + 8 (second).
-template <int NB>
-__device__ __forceinline__ void bfrag_hilo(const float* X, int xs, int ks, int lane,
-                                           uint32_t (&bf)[NB][2], bool f16 = false) {
+// (split into the loads and the conversion, so that callers can put the loads of several
+// k-steps in flight before the first conversion waits for them)
+__device__ __forceinline__ uint32_t bfrag_addr(const float* X, int xs, int ks, int lane, int nb) {
   const int n = lane >> 2;
-  const int c = 16 * ks + 2 * (lane & 3);
-  const int head = NB == 1 ? (n & 3) : n;
-  const uint32_t xa = smem_u32(X + head * xs + c);
-  const float2 x = lds_f32x2(xa);
-  const float2 y = lds_f32x2(xa + 32u);
+  const int head = nb == 1 ? (n & 3) : n;
+  return smem_u32(X + head * xs + 16 * ks + 2 * (lane & 3));
+}
+template <int NB>
+__device__ __forceinline__ void bfrag_from(float2 x, float2 y, int lane, uint32_t (&bf)[NB][2],
+                                           bool f16 = false) {
+  const int n = lane >> 2;
   const uint32_t hx = f16 ? hi_pair_h(x.x, x.y) : hi_pair(x.x, x.y);
   const uint32_t hy = f16 ? hi_pair_h(y.x, y.y) : hi_pair(y.x, y.y);
   const uint32_t lx = f16 ? lo_pair_h(x.x, x.y, hx) : lo_pair(x.x, x.y, hx);
@@ -237,6 +239,12 @@ __device__ __forceinline__ void bfrag_hilo(const float* X, int xs, int ks, int l
     bf[NB - 1][0] = lx;
     bf[NB - 1][1] = ly;
   }
+}
+template <int NB>
+__device__ __forceinline__ void bfrag_hilo(const float* X, int xs, int ks, int lane,
+                                           uint32_t (&bf)[NB][2], bool f16 = false) {
+  const uint32_t xa = bfrag_addr(X, xs, ks, lane, NB);
+  bfrag_from<NB>(lds_f32x2(xa), lds_f32x2(xa + 32u), lane, bf, f16);
 }
 
 __host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
@@ -596,20 +604,25 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
     for (int task = warp; task < ntasks && ok; task += NW) {
       const bool key = task >= nks;
       const int mt = key ? task - nks : task;
-      float c[4];
       const PieceLoc pl = locate(rK, d, 2 * mt + at_chunk(lane));
+      uint32_t af[8][4];  // all eight k-steps' fragments in flight together
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) ldsm_x4_t(smem_u32(pmat) + swz(pl, 16 * ks + at_row(lane)), af[ks]);
+      float c[4], c2[4];  // even and odd k-steps: two MMA chains of four
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
-        uint32_t af[4];
-        ldsm_x4_t(smem_u32(pmat) + swz(pl, 16 * ks + at_row(lane)), af);
         uint32_t b0 = qb[ks][0], b1 = qb[ks][1];
         if (key) {
           b0 = n == 0 ? krow[8 * ks + (lane & 3)] : 0u;
           b1 = n == 0 ? krow[8 * ks + 4 + (lane & 3)] : 0u;
         }
-        if (ks == 0) mma_bf16_z(c, af, b0, b1);
-        else mma_bf16(c, af, b0, b1);
+        if (ks == 0) mma_bf16_z(c, af[ks], b0, b1);
+        else if (ks == 1) mma_bf16_z(c2, af[ks], b0, b1);
+        else if (ks & 1) mma_bf16(c2, af[ks], b0, b1);
+        else mma_bf16(c, af[ks], b0, b1);
       }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) c[e] += c2[e];
       const int j = 16 * mt + (lane >> 2), hh = 2 * (lane & 3);
       if (!key) {
         const uint32_t qtb = smem_u32(qt);
@@ -760,10 +773,20 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
     const int kc0 = lane % kcpr, vc0 = lane % vcpr;
     const int kt0 = lane / kcpr, vt0 = lane / vcpr;
 
-    uint32_t qf[NKS][NB][2];  // B fragments of Q^T (hi / lo parts)
+    uint32_t qf[NKS][NB][2];  // B fragments of Q^T (hi / lo parts; fp16 against int8 codes)
+    {
+      float2 qx[NKS], qy[NKS];
 #pragma unroll
-    for (int ks = 0; ks < NKS; ++ks)
-      if (ks < nks) bfrag_hilo<NB>(qt, xs, ks, lane, qf[ks], Q8);  // fp16 against int8 codes
+      for (int ks = 0; ks < NKS; ++ks)
+        if (ks < nks) {
+          const uint32_t xa = bfrag_addr(qt, xs, ks, lane, NB);
+          qx[ks] = lds_f32x2(xa);
+          qy[ks] = lds_f32x2(xa + 32u);
+        }
+#pragma unroll
+      for (int ks = 0; ks < NKS; ++ks)
+        if (ks < nks) bfrag_from<NB>(qx[ks], qy[ks], lane, qf[ks], Q8);
+    }
     uint32_t koff[NKS], kstep[NKS], voff[NMV], vstep[NMV];
 #pragma unroll
     for (int ks = 0; ks < NKS; ++ks) {
@@ -1144,20 +1167,32 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
     if (!setup_ok || !warp_wait(setup_bar, 1, a.dev_status)) return;
     for (int mt = warp; mt < d / 16; mt += NW + 1) {
       float c[NB][4];
+      constexpr int KB = 4;  // k-steps whose fragments are loaded together
 #pragma unroll
-      for (int ks = 0; ks < NMV; ++ks)
-        if (ks < nmv) {
-          uint32_t af[4];
-          const PieceLoc pl = locate(rV, d, 2 * ks + a_chunk(lane));
-          ldsm_x4(smem_u32(pmat) + swz(pl, 16 * mt + a_row(lane)), af);
-          uint32_t bf[NB][2];
-          bfrag_hilo<NB>(qt, xs, ks, lane, bf);
+      for (int k0 = 0; k0 < NMV; k0 += KB) {
+        uint32_t af[KB][4];
+        float2 bx[KB], by[KB];
 #pragma unroll
-          for (int j = 0; j < NB; ++j) {
-            if (ks == 0) mma_bf16_z(c[j], af, bf[j][0], bf[j][1]);
-            else mma_bf16(c[j], af, bf[j][0], bf[j][1]);
+        for (int u = 0; u < KB; ++u)
+          if (k0 + u < nmv) {
+            const PieceLoc pl = locate(rV, d, 2 * (k0 + u) + a_chunk(lane));
+            ldsm_x4(smem_u32(pmat) + swz(pl, 16 * mt + a_row(lane)), af[u]);
+            const uint32_t xa = bfrag_addr(qt, xs, k0 + u, lane, NB);
+            bx[u] = lds_f32x2(xa);
+            by[u] = lds_f32x2(xa + 32u);
           }
-        }
+#pragma unroll
+        for (int u = 0; u < KB; ++u)
+          if (k0 + u < nmv) {
+            uint32_t bf[NB][2];
+            bfrag_from<NB>(bx[u], by[u], lane, bf);
+#pragma unroll
+            for (int j = 0; j < NB; ++j) {
+              if (k0 + u == 0) mma_bf16_z(c[j], af[u], bf[j][0], bf[j][1]);
+              else mma_bf16(c[j], af[u], bf[j][0], bf[j][1]);
+            }
+          }
+      }
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float o = NB == 1 ? c[0][e] + __shfl_xor_sync(kFull, c[0][e], 2) : c[0][e] + c[NB - 1][e];
