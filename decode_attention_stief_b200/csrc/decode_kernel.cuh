@@ -37,17 +37,16 @@
 // Modes (compile-time, one instantiation each): the contiguous bf16 cache; the latent
 // decode (q~ given, o~ returned: no base loads, projections or up-projection, for bases
 // folded into the attention weights); paged caches (tiles addressed through a block
-// table); int8 caches (code boxes and row scales copied raw; each warp turns its codes into
-// exact fp16 in a padded row-major tile and the MMAs take fp16 operands, the row scales
-// multiplying the scores and the softmax weights).  Grids of more than one wave run two
+// table); int8 caches (the codes go straight into the integer MMA, m16n8k32 with s32
+// accumulators: q~ and the softmax weights enter as 16-bit fixed point split into two 8-bit
+// parts, per head and per head and tile respectively, so both products are exact in integers;
+// the row scales multiply the scores and the weights).  Grids of more than one wave run two
 // CTAs per SM with a smaller ring.
 #pragma once
 
 #include <cfloat>
 #include <cmath>
 #include <cstdint>
-
-#include <cuda_fp16.h>
 
 #include "stief_device.cuh"
 #include "stief_internal.h"
@@ -110,50 +109,64 @@ __device__ __forceinline__ void mma_bf16_z(float (&c)[4], const uint32_t (&a)[4]
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.f));
 }
 
-// The same two products with fp16 operands (the int8 caches' codes are exact in fp16).
-__device__ __forceinline__ void mma_f16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
-                                        uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ void mma_f16_z(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
-                                          uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%10,%10,%10,%10};"
-      : "=f"(c[0]), "=f"(c[1]), "=f"(c[2]), "=f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.f));
-}
-template <bool F16>
-__device__ __forceinline__ void mma_op(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  if constexpr (F16) mma_f16(c, a, b0, b1);
-  else mma_bf16(c, a, b0, b1);
-}
-template <bool F16>
-__device__ __forceinline__ void mma_op_z(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  if constexpr (F16) mma_f16_z(c, a, b0, b1);
-  else mma_bf16_z(c, a, b0, b1);
+// Two 8x8 b16 matrices (lanes 0-15 give the row addresses).
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];"
+               : "=r"(r0), "=r"(r1)
+               : "r"(addr));
 }
 
-// fp16 hi / lo parts of an fp32 pair, packed (first element in the low half)
-__device__ __forceinline__ uint32_t hi_pair_h(float x0, float x1) {
-  const __half2 h = __floats2half2_rn(x0, x1);
-  return *reinterpret_cast<const uint32_t*>(&h);
+// Integer products for the int8 caches, exact in s32:
+// c (+)= A(16x32, s8, row) . B(32x8, s8 or u8, col)  and  c (+)= A(16x16, s8) . B(16x8, s8).
+// Register i of A holds 4 consecutive k of row (lane >> 2) + 8 (i & 1), k from
+// 4 (lane & 3) + 16 (i >> 1); register i of B 4 consecutive k from 4 (lane & 3) + 16 i of
+// column lane >> 2.
+template <bool ZERO, bool BU8>
+__device__ __forceinline__ void mma_i8_k32(int (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  if constexpr (ZERO && BU8)
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%10,%10,%10};"
+        : "=r"(c[0]), "=r"(c[1]), "=r"(c[2]), "=r"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "r"(0));
+  else if constexpr (ZERO)
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%10,%10,%10};"
+        : "=r"(c[0]), "=r"(c[1]), "=r"(c[2]), "=r"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "r"(0));
+  else if constexpr (BU8)
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  else
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
-__device__ __forceinline__ uint32_t lo_pair_h(float x0, float x1, uint32_t hi) {
-  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hi));
-  return hi_pair_h(x0 - f.x, x1 - f.y);
+template <bool ZERO>
+__device__ __forceinline__ void mma_i8_k16(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
+  if constexpr (ZERO)
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5}, {%6}, "
+        "{%7,%7,%7,%7};"
+        : "=r"(c[0]), "=r"(c[1]), "=r"(c[2]), "=r"(c[3])
+        : "r"(a0), "r"(a1), "r"(b0), "r"(0));
+  else
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5}, {%6}, "
+        "{%0,%1,%2,%3};"
+        : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+        : "r"(a0), "r"(a1), "r"(b0));
 }
-// Four int8 codes (w) as exact fp16 pairs: 0x64uu is 1024 + uu in fp16, uu = code + 128.
-__device__ __forceinline__ void codes_f16(uint32_t w, uint32_t& h01, uint32_t& h23) {
-  const uint32_t u = w ^ 0x80808080u;
-  const uint32_t a = __byte_perm(u, 0x64646464u, 0x5140u), b = __byte_perm(u, 0x64646464u, 0x7362u);
-  // minus 1152 = 1024 + 128 in both halves (0x6480 is 1152 in fp16)
-  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(h01) : "r"(a), "r"(0x64806480u));
-  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(h23) : "r"(b), "r"(0x64806480u));
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 // hi / lo bf16 parts of an fp32 pair, packed (first element in the low half)
@@ -165,8 +178,9 @@ __device__ __forceinline__ uint32_t lo_pair(float x0, float x1, uint32_t hi) {
 // ---------------------------------------------------------------------------- tile addressing
 
 // Where 16-byte column chunk `chunk` of a row lives inside a tile of `rows` rows stacked
-// from the pieces of a rank-r matrix: r / 64 pieces 64 columns wide, then one 32 wide if
-// r % 64 >= 32, then one 16 wide if r % 32 == 16 (the order the host plans them in).
+// from the pieces of a matrix r 16-bit columns wide: r / 64 pieces 64 columns wide, then one
+// 32 wide if r % 64 >= 32, then one 16 wide if r % 32 == 16 (the order the host plans them
+// in).
 struct PieceLoc {
   uint32_t off;  // piece offset in the tile
   uint32_t w;    // piece width (columns)
@@ -175,30 +189,42 @@ struct PieceLoc {
 __device__ __forceinline__ PieceLoc locate(int r, int rows, int chunk) {
   const int col = chunk * 8;
   const int x64 = r & ~63;
-  const bool has32 = r - x64 >= 32;
+  const int x32 = x64 + (r - x64 >= 32 ? 32 : 0);
   PieceLoc pl;
   if (col < x64) {
     pl.w = 64u;
     pl.off = (uint32_t)((col >> 6) * rows * 128);
     pl.lc = (uint32_t)((col & 63) >> 3);
-  } else if (has32 && col < x64 + 32) {
+  } else if (col < x32) {
     pl.w = 32u;
     pl.off = (uint32_t)(x64 * rows * 2);
     pl.lc = (uint32_t)((col - x64) >> 3);
   } else {
-    const int x16 = x64 + (has32 ? 32 : 0);
     pl.w = 16u;
-    pl.off = (uint32_t)(x16 * rows * 2);
-    pl.lc = (uint32_t)((col - x16) >> 3);
+    pl.off = (uint32_t)(x32 * rows * 2);
+    pl.lc = (uint32_t)((col - x32) >> 3);
   }
   return pl;
 }
+// The same for int8 rows, whose r_bytes are addressed as r = r_bytes / 2 16-bit columns (r a
+// multiple of 8): after the pieces above, one 8 columns (16 bytes) wide if r % 16 == 8.
+__device__ __forceinline__ PieceLoc locate_i8(int r, int rows, int chunk) {
+  const int x16 = r & ~15;
+  if (chunk * 8 < x16) return locate(x16, rows, chunk);
+  PieceLoc pl;
+  pl.w = 8u;
+  pl.off = (uint32_t)(x16 * rows * 2);
+  pl.lc = 0u;
+  return pl;
+}
 // Byte offset of (row, chunk) under the piece's TMA swizzle: 128-byte rows XOR the chunk
-// with row & 7, 64-byte rows with (row >> 1) & 3, 32-byte rows with (row >> 2) & 1.
+// with row & 7, 64-byte rows with (row >> 1) & 3, 32-byte rows with (row >> 2) & 1; 16-byte
+// rows are not swizzled (8 consecutive rows already fill the 32 banks).
 __device__ __forceinline__ uint32_t swz(const PieceLoc& pl, int row) {
-  const uint32_t sw = pl.w == 64u ? (uint32_t)(row & 7)
+  const uint32_t sw = pl.w == 64u   ? (uint32_t)(row & 7)
                       : pl.w == 32u ? (uint32_t)((row >> 1) & 3)
-                                    : (uint32_t)((row >> 2) & 1);
+                      : pl.w == 16u ? (uint32_t)((row >> 2) & 1)
+                                    : 0u;
   return pl.off + (uint32_t)row * pl.w * 2u + ((pl.lc ^ sw) << 4);
 }
 // Lane row / chunk for an x4 ldmatrix of a 16x16 block read as an A operand:
@@ -222,13 +248,10 @@ __device__ __forceinline__ uint32_t bfrag_addr(const float* X, int xs, int ks, i
   return smem_u32(X + head * xs + 16 * ks + 2 * (lane & 3));
 }
 template <int NB>
-__device__ __forceinline__ void bfrag_from(float2 x, float2 y, int lane, uint32_t (&bf)[NB][2],
-                                           bool f16 = false) {
+__device__ __forceinline__ void bfrag_from(float2 x, float2 y, int lane, uint32_t (&bf)[NB][2]) {
   const int n = lane >> 2;
-  const uint32_t hx = f16 ? hi_pair_h(x.x, x.y) : hi_pair(x.x, x.y);
-  const uint32_t hy = f16 ? hi_pair_h(y.x, y.y) : hi_pair(y.x, y.y);
-  const uint32_t lx = f16 ? lo_pair_h(x.x, x.y, hx) : lo_pair(x.x, x.y, hx);
-  const uint32_t ly = f16 ? lo_pair_h(y.x, y.y, hy) : lo_pair(y.x, y.y, hy);
+  const uint32_t hx = hi_pair(x.x, x.y), hy = hi_pair(y.x, y.y);
+  const uint32_t lx = lo_pair(x.x, x.y, hx), ly = lo_pair(y.x, y.y, hy);
   if constexpr (NB == 1) {
     const bool lo = (n >> 2) != 0;
     bf[0][0] = lo ? lx : hx;
@@ -242,9 +265,9 @@ __device__ __forceinline__ void bfrag_from(float2 x, float2 y, int lane, uint32_
 }
 template <int NB>
 __device__ __forceinline__ void bfrag_hilo(const float* X, int xs, int ks, int lane,
-                                           uint32_t (&bf)[NB][2], bool f16 = false) {
+                                           uint32_t (&bf)[NB][2]) {
   const uint32_t xa = bfrag_addr(X, xs, ks, lane, NB);
-  bfrag_from<NB>(lds_f32x2(xa), lds_f32x2(xa + 32u), lane, bf, f16);
+  bfrag_from<NB>(lds_f32x2(xa), lds_f32x2(xa + 32u), lane, bf);
 }
 
 __host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
@@ -262,14 +285,11 @@ struct DecodeSmem {
   uint32_t region;  // per warp a ring of stages (keys then values of a tile); later the
                     // cross-warp reduction and the split-merge staging
   uint32_t region_bytes;
-  // int8 caches: the region holds one 16-bit tile per warp (the stage's codes as fp16,
-  // row-major, rows padded by 16 bytes), then the rings of raw stages: codes K [tile][rK], codes V
-  // [tile][rV], scales K [tile], scales V [tile]
-  uint32_t ring;      // offset of the rings inside the region
-  uint32_t q8_sc;     // int8 caches: per warp the tile's key then value row scales (fp32)
-  uint32_t q8_tile;   // int8 caches: bytes of a warp's 16-bit tile
-  uint32_t stage;     // bytes of one ring stage
-  uint32_t q8_v, q8_ks, q8_vs;  // offsets inside a raw int8 stage
+  uint32_t stage;             // bytes of one ring stage (a multiple of 1 KiB)
+  // int8 caches: a stage holds the key codes [tile][rK] and the value codes [tile][rV] in
+  // column pieces like the bf16 tiles (the rows' bytes read as 16-bit columns), then the
+  // tile's key and value row scales (fp32)
+  uint32_t q8_v, q8_ks, q8_vs;  // offsets inside an int8 stage
   uint32_t total;
   int xs;  // row stride of qt in floats
 };
@@ -295,22 +315,16 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int NW, int ns, int rK,
   s.pmat = off;
   off += 256u * rmax;  // d = 128 rows x r bf16
   s.region = off;
-  const uint32_t bf16_stage = (uint32_t)tile * (rK + rV) * 2u;  // a multiple of 1 KiB
   if (q8) {
-    s.q8_v = align_up((uint32_t)tile * rK, 128);
-    s.q8_ks = s.q8_v + align_up((uint32_t)tile * rV, 128);
+    s.q8_v = align_up((uint32_t)tile * rK, 1024);  // the swizzle patterns need 1 KiB alignment
+    s.q8_ks = s.q8_v + (uint32_t)tile * rV;
     s.q8_vs = s.q8_ks + (uint32_t)tile * 4u;
-    s.stage = align_up(s.q8_vs + (uint32_t)tile * 4u, 128);
-    // the 16-bit tile is row-major with rows padded by 16 bytes (conflict-free ldmatrix)
-    s.q8_tile = (uint32_t)tile * (2u * rK + 16u + 2u * rV + 16u);
-    s.q8_sc = (uint32_t)NW * s.q8_tile;
-    s.ring = align_up(s.q8_sc + (uint32_t)NW * 8u * tile, 128);
+    s.stage = align_up(s.q8_vs + (uint32_t)tile * 4u, 1024);
   } else {
-    s.q8_v = s.q8_ks = s.q8_vs = s.q8_sc = s.q8_tile = 0;
-    s.stage = bf16_stage;
-    s.ring = 0;
+    s.q8_v = s.q8_ks = s.q8_vs = 0;
+    s.stage = (uint32_t)tile * (rK + rV) * 2u;  // a multiple of 1 KiB
   }
-  s.region_bytes = s.ring + (uint32_t)NW * ns * s.stage;
+  s.region_bytes = (uint32_t)NW * ns * s.stage;
   off += s.region_bytes;
   s.total = off;
   return s;
@@ -371,8 +385,9 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
   float* qt = reinterpret_cast<float*>(smem + L.qt);
   const int xs = L.xs;
   uint8_t* pmat = smem + L.pmat;
-  const uint32_t kt_bytes = (uint32_t)kTile * rK * 2u;
-  const uint32_t st_bytes = kt_bytes + (uint32_t)kTile * rV * 2u;
+  // a stage: the key tile, then the value tile at kt_bytes (int8 caches: then the row scales)
+  const uint32_t kt_bytes = Q8 ? L.q8_v : (uint32_t)kTile * rK * 2u;
+  const uint32_t st_bytes = Q8 ? (uint32_t)kTile * (rK + rV + 8) : kt_bytes + (uint32_t)kTile * rV * 2u;
 
   // the swizzle patterns assume 1 KiB-aligned tiles
   if (((smem_u32(smem + L.pmat) | smem_u32(smem + L.region)) & 1023u) != 0) {
@@ -438,19 +453,9 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
   }
   const int npk = a.pk.n, npv = a.pv.n;
   auto issue = [&](int w, int k, uint64_t policy) {  // producer: tile k of consumer warp w
-    uint8_t* dst = smem + L.region + L.ring + ((size_t)w * ns + (k % ns)) * L.stage;
+    uint8_t* dst = smem + L.region + ((size_t)w * ns + (k % ns)) * L.stage;
     uint64_t* bar = &full[w * ns + (k % ns)];
-    if (Q8) {  // int8 codes of K and V (one box each) and the tile's two rows of scales
-      const uint32_t tb = (uint32_t)kTile * (rK + rV) + 8u * kTile;
-      mbar_arrive_expect_tx(bar, tb);
-      const int y = tile_row(t0 + (w + k * NW) * kTile);
-      tma_load_2d(dst, kmap[0], 0, y, bar, policy);
-      tma_load_2d(dst + L.q8_v, vmap[0], 0, y, bar, policy);
-      bulk_g2s(dst + L.q8_ks, a.k_scale + y, 4u * kTile, bar);
-      bulk_g2s(dst + L.q8_vs, a.v_scale + y, 4u * kTile, bar);
-      return;
-    }
-    // whole 32-row boxes land (rows past the sequence are masked on chip)
+    // whole boxes land (rows past the sequence are masked on chip)
     mbar_arrive_expect_tx(bar, st_bytes);
     const int tt = t0 + (w + k * NW) * kTile;
     const int y = tile_row(tt);
@@ -462,6 +467,10 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
 #pragma unroll
     for (int p = 0; p < 3; ++p)
       if (p < npv) tma_load_2d(dst + vo[p], vmap[p], vx[p], yv, bar, policy);
+    if (Q8) {  // the tile's two rows of scales
+      bulk_g2s(dst + L.q8_ks, a.k_scale + y, 4u * kTile, bar);
+      bulk_g2s(dst + L.q8_vs, a.v_scale + y, 4u * kTile, bar);
+    }
   };
 
   // Contiguous bf16 caches (plain and latent modes): every warp's first tile is requested
@@ -761,20 +770,16 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
   } else {
     // ---- consumers: stream the warp's tiles ------------------------------------------------
     const int my_tiles = warp_tiles(warp, n_tiles);
-    uint8_t* ring = smem + L.region + L.ring + (size_t)warp * ns * L.stage;
-    uint8_t* staging = smem + L.region + (size_t)warp * L.q8_tile;  // int8 caches only
-    const uint32_t sK = 2u * rK + 16u, sV = 2u * rV + 16u;  // its row strides
-    const uint32_t q8_kt = (uint32_t)kTile * sK;            // its value rows' offset
-    // int8 caches: in the conversion pass a lane takes one 16-column chunk of each matrix
-    // and every (32 / chunks per row)-th row of it (no division per item)
-    const int kcpr = rK >> 4, vcpr = rV >> 4;  // 16-column chunks per row
-    const int krpp = 32 / kcpr, vrpp = 32 / vcpr;  // rows per pass
-    const bool klive = lane < krpp * kcpr, vlive = lane < vrpp * vcpr;
-    const int kc0 = lane % kcpr, vc0 = lane % vcpr;
-    const int kt0 = lane / kcpr, vt0 = lane / vcpr;
+    uint8_t* ring = smem + L.region + (size_t)warp * ns * L.stage;
+    // int8 caches: a row's bytes are addressed as 16-bit columns (r / 2 of them); the scores
+    // take k-steps of 32 codes (the last one 16 when r_K % 32 == 16)
+    const int rKc = Q8 ? rK / 2 : rK, rVc = Q8 ? rV / 2 : rV;
+    const int nks8 = (rK + 31) >> 5;
 
-    uint32_t qf[NKS][NB][2];  // B fragments of Q^T (hi / lo parts; fp16 against int8 codes)
-    {
+    uint32_t qf[NKS][NB][2];       // bf16 caches: B fragments of Q^T (hi / lo parts)
+    uint32_t qf8[NKS / 2][NB][2];  // int8 caches: the same as 8-bit parts
+    float sqA = 0.f, sqB = 0.f;    // int8 caches: fixed-point scales of q~ for heads hA, hA + 1
+    if constexpr (!Q8) {
       float2 qx[NKS], qy[NKS];
 #pragma unroll
       for (int ks = 0; ks < NKS; ++ks)
@@ -785,25 +790,68 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
         }
 #pragma unroll
       for (int ks = 0; ks < NKS; ++ks)
-        if (ks < nks) bfrag_from<NB>(qx[ks], qy[ks], lane, qf[ks], Q8);
+        if (ks < nks) bfrag_from<NB>(qx[ks], qy[ks], lane, qf[ks]);
+    } else {
+      // q~ in 16-bit fixed point per head, q16 = rint(q~ / s_q) with s_q = max_j |q~_j| / 32512,
+      // split as q16 = 256 hi + lo (hi in [-127, 127], lo in [-128, 127]), so that a score is
+      // s_q k_scale (256 K.hi + K.lo) with both integer products exact.  B column n carries
+      // part n >> 2 of head n & 3 (groups of up to 4) or, for groups of 8, n-tile 0 the hi and
+      // n-tile 1 the lo parts of head n.
+      const int n = lane >> 2;
+      const int hcol = NB == 1 ? (n & 3) : n;
+      const uint32_t qrow = smem_u32(qt) + 4u * (uint32_t)(hcol * xs);
+      float amax = 0.f;
+      for (int j = lane & 3; j < rK; j += 4) amax = fmaxf(amax, fabsf(lds_f32(qrow + 4u * (uint32_t)j)));
+      amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
+      const float inv = amax > 0.f ? 32512.f / amax : 0.f;  // absent heads are zero rows
+      const float sq = amax * (1.f / 32512.f);
+      sqA = __shfl_sync(kFull, sq, 4 * hA);  // lanes 4 h .. 4 h + 3 hold column h: head h
+      sqB = __shfl_sync(kFull, sq, 4 * (hA + 1));
+      const bool part_lo = NB == 1 && (n >> 2) != 0;
+#pragma unroll
+      for (int ks = 0; ks < NKS / 2; ++ks)
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int k0 = 32 * ks + 16 * half + 4 * (lane & 3);
+          uint32_t hb = 0u, lb = 0u;
+          if (ks < nks8 && k0 < rK) {
+            const float4 x = lds128f(qrow + 4u * (uint32_t)k0);
+            const float xv[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int q16 = __float2int_rn(xv[i] * inv);
+              const int hi = (q16 + 128) >> 8, lo = q16 - hi * 256;
+              hb |= ((uint32_t)hi & 0xffu) << (8 * i);
+              lb |= ((uint32_t)lo & 0xffu) << (8 * i);
+            }
+          }
+          if constexpr (NB == 1) {
+            qf8[ks][0][half] = part_lo ? lb : hb;
+          } else {
+            qf8[ks][0][half] = hb;
+            qf8[ks][NB - 1][half] = lb;
+          }
+        }
     }
+    // ldmatrix lane offsets.  Keys: the x4 (x2 for a 16-wide k-step) of m-tile 0 of each
+    // k-step, kstep bytes further per m-tile.  Values, bf16: the transposed x4 of each 16-dim
+    // m-tile over tokens 0-15, vstep further per 16 tokens; int8: the transposed x4 of rows
+    // (tokens) 0-31 of the m-tile's 16-byte column, vstep further per 32 tokens.
     uint32_t koff[NKS], kstep[NKS], voff[NMV], vstep[NMV];
 #pragma unroll
     for (int ks = 0; ks < NKS; ++ks) {
-      if (Q8) {  // the row-major padded 16-bit tile
-        koff[ks] = (uint32_t)a_row(lane) * sK + (uint32_t)(2 * ks + a_chunk(lane)) * 16u;
-        kstep[ks] = 16u * sK;
-        continue;
-      }
-      const PieceLoc pl = locate(rK, kTile, 2 * ks + a_chunk(lane));
+      const int ch = min(2 * ks + a_chunk(lane), rKc / 8 - 1);
+      const PieceLoc pl = Q8 ? locate_i8(rKc, kTile, ch) : locate(rKc, kTile, ch);
       koff[ks] = swz(pl, a_row(lane));
       kstep[ks] = 32u * pl.w;  // 16 rows further (the swizzle repeats every 8 rows)
     }
 #pragma unroll
     for (int mt = 0; mt < NMV; ++mt) {
       if (Q8) {
-        voff[mt] = q8_kt + (uint32_t)at_row(lane) * sV + (uint32_t)(2 * mt + at_chunk(lane)) * 16u;
-        vstep[mt] = 16u * sV;
+        const PieceLoc pl = locate_i8(rVc, kTile, min(mt, rVc / 8 - 1));
+        voff[mt] = kt_bytes + swz(pl, lane);
+        vstep[mt] = 64u * pl.w;
         continue;
       }
       const PieceLoc pl = locate(rV, kTile, 2 * mt + at_chunk(lane));
@@ -817,45 +865,9 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
         ok = false;
         break;
       }
-      uint32_t sbase = smem_u32(ring + (size_t)st * L.stage);
+      const uint32_t sbase = smem_u32(ring + (size_t)st * L.stage);
       const int tok0 = t0 + (warp + k * NW) * kTile;
       const int n = min(kTile, t1 - tok0);
-      // int8 caches: the tile's row scales go to this warp's scale buffer (0 past the
-      // sequence, so that whatever the scale rows hold there reaches nothing) and the codes
-      // become exact fp16 in its 16-bit tile
-      float* scw = reinterpret_cast<float*>(smem + L.region + L.q8_sc) + warp * 2 * kTile;
-      if (Q8) {
-        const uint8_t* raw = ring + (size_t)st * L.stage;
-        const float* scr = reinterpret_cast<const float*>(raw + L.q8_ks);  // K then V rows
-        __syncwarp();  // every lane is done reading the previous tile and its scales
-        for (int i = lane; i < 2 * kTile; i += 32)  // the V row follows the K row in the stage
-          scw[i] = (i < kTile ? i : i - kTile) < n ? scr[i] : 0.f;
-        for (int m = 0; m < 2; ++m) {
-          const int r = m ? rV : rK;
-          const int8_t* codes = reinterpret_cast<const int8_t*>(raw + (m ? L.q8_v : 0u)) + 16 * (m ? vc0 : kc0);
-          const uint32_t stride = m ? sV : sK;
-          const int rpp = m ? vrpp : krpp;
-          const int t0 = m ? vt0 : kt0;
-          uint8_t* dst = staging + (m ? q8_kt : 0u) + (uint32_t)t0 * stride + 32u * (uint32_t)(m ? vc0 : kc0);
-          const int8_t* src = codes + t0 * r;
-          const uint32_t dstep = (uint32_t)rpp * stride;
-          const int sstep = rpp * r;
-          if (m ? vlive : klive)
-            for (int t = t0; t < kTile; t += rpp, dst += dstep, src += sstep) {
-              const uint4 w16 = *reinterpret_cast<const uint4*>(src);
-              uint4 o0, o1;
-              codes_f16(w16.x, o0.x, o0.y);
-              codes_f16(w16.y, o0.z, o0.w);
-              codes_f16(w16.z, o1.x, o1.y);
-              codes_f16(w16.w, o1.z, o1.w);
-              reinterpret_cast<uint4*>(dst)[0] = o0;
-              reinterpret_cast<uint4*>(dst)[1] = o1;
-            }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[warp * ns + st]);  // the raw stage may be refilled
-        sbase = smem_u32(staging);
-      }
       if (EARLY && k < kPreIssue && Lb >= 1 && tok0 <= Lb - 1 && Lb - 1 < tok0 + kTile) {
         // this tile was requested before the dependency wait: the row just below the length
         // may have been appended by the preceding kernel (a fused step on the same caches),
@@ -867,7 +879,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
           const uint4 v = key ? __ldcg(reinterpret_cast<const uint4*>(a.k_lat_w + prow * rK) + cch)
                               : __ldcg(reinterpret_cast<const uint4*>(a.v_lat_w + prow * rV) + (cch - rK / 8));
           const PieceLoc pt = key ? locate(rK, kTile, cch) : locate(rV, kTile, cch - rK / 8);
-          *reinterpret_cast<uint4*>(ring + (size_t)st * st_bytes + (key ? 0u : kt_bytes) + swz(pt, r_prev)) = v;
+          *reinterpret_cast<uint4*>(ring + (size_t)st * L.stage + (key ? 0u : kt_bytes) + swz(pt, r_prev)) = v;
         }
         fence_proxy_async_smem();  // generic writes into a stage the TMA engine fills
         __syncwarp();
@@ -885,7 +897,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
         for (int cch = lane; cch < (rK + rV) / 8; cch += 32) {
           const bool key = cch < rK / 8;
           const PieceLoc pt = key ? locate(rK, kTile, cch) : locate(rV, kTile, cch - rK / 8);
-          *reinterpret_cast<uint4*>(ring + (size_t)st * st_bytes + (key ? 0u : kt_bytes) +
+          *reinterpret_cast<uint4*>(ring + (size_t)st * L.stage + (key ? 0u : kt_bytes) +
                                     swz(pt, r_new)) = *reinterpret_cast<const uint4*>(kl + 8 * cch);
         }
         fence_proxy_async_smem();  // generic writes into a stage the TMA engine fills
@@ -894,34 +906,9 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
 
       // Fragments are requested a group of k-steps (m-tiles) at a time, so their latencies
       // overlap; asm volatile keeps the order written here.
-      // scores: c[mt][j][e] is token 16 mt + (lane >> 2) + 8 (e >> 1), column
-      // 2 (lane & 3) + (e & 1)
-      float c[MT][NB][4];
-#pragma unroll
-      for (int g0 = 0; g0 < NKS; g0 += KG)
-        if (g0 < nks) {
-          uint32_t kf[KG][MT][4];
-#pragma unroll
-          for (int u = 0; u < KG; ++u)
-            if (g0 + u < nks) {
-#pragma unroll
-              for (int mt = 0; mt < MT; ++mt)
-                ldsm_x4(sbase + koff[g0 + u] + mt * kstep[g0 + u], kf[u][mt]);
-            }
-#pragma unroll
-          for (int u = 0; u < KG; ++u)
-            if (g0 + u < nks) {
-#pragma unroll
-              for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                for (int j = 0; j < NB; ++j) {
-                  if (g0 + u == 0) mma_op_z<Q8>(c[mt][j], kf[u][mt], qf[0][j][0], qf[0][j][1]);
-                  else mma_op<Q8>(c[mt][j], kf[u][mt], qf[g0 + u][j][0], qf[g0 + u][j][1]);
-                }
-            }
-        }
-      // value fragments do not depend on the scores: request the first group now
-      uint32_t vf[VG][MT][4];
+      // scores: s[mt][e] is token 16 mt + (lane >> 2) + 8 (e >> 1), head hA + (e & 1)
+      float s[MT][4];
+      uint32_t vf[VG][MT][4];  // bf16 caches: value fragments
       auto load_v = [&](int g0) {
 #pragma unroll
         for (int u = 0; u < VG; ++u)
@@ -945,20 +932,98 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
               }
         }
       };
-      load_v(0);
-      // add the hi and lo parts: s[mt][e] is the score of head hA + (e & 1)
-      float s[MT][4];
+      // int8 caches: value fragments of the first m-tiles (raw ldmatrix words, k32 steps)
+      constexpr int VG8 = MT == 4 ? 1 : 2;
+      uint32_t vx8[VG8][MT / 2][4];
+      if constexpr (!Q8) {
+        // c[mt][j][e] is token 16 mt + (lane >> 2) + 8 (e >> 1), column 2 (lane & 3) + (e & 1)
+        float c[MT][NB][4];
 #pragma unroll
-      for (int mt = 0; mt < MT; ++mt)
+        for (int g0 = 0; g0 < NKS; g0 += KG)
+          if (g0 < nks) {
+            uint32_t kf[KG][MT][4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-          s[mt][e] = NB == 1 ? c[mt][0][e] + __shfl_xor_sync(kFull, c[mt][0][e], 2)
-                             : c[mt][0][e] + c[mt][NB - 1][e];
-      if (Q8) {  // scores of code rows times the rows' key scales
+            for (int u = 0; u < KG; ++u)
+              if (g0 + u < nks) {
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt)
+                  ldsm_x4(sbase + koff[g0 + u] + mt * kstep[g0 + u], kf[u][mt]);
+              }
+#pragma unroll
+            for (int u = 0; u < KG; ++u)
+              if (g0 + u < nks) {
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                  for (int j = 0; j < NB; ++j) {
+                    if (g0 + u == 0) mma_bf16_z(c[mt][j], kf[u][mt], qf[0][j][0], qf[0][j][1]);
+                    else mma_bf16(c[mt][j], kf[u][mt], qf[g0 + u][j][0], qf[g0 + u][j][1]);
+                  }
+              }
+          }
+        // value fragments do not depend on the scores: request the first group now
+        load_v(0);
+        // add the hi and lo parts
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) s[mt][e] *= scw[16 * mt + (lane >> 2) + 8 * (e >> 1)];
+          for (int e = 0; e < 4; ++e)
+            s[mt][e] = NB == 1 ? c[mt][0][e] + __shfl_xor_sync(kFull, c[mt][0][e], 2)
+                               : c[mt][0][e] + c[mt][NB - 1][e];
+      } else {
+        // integer scores of the codes against the two parts of q~
+        int ci[MT][NB][4];
+#pragma unroll
+        for (int ks = 0; ks < NKS / 2; ++ks)
+          if (ks < nks8) {
+            const bool k32 = 32 * ks + 32 <= rK;
+            uint32_t kf[MT][4];
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+              if (k32) ldsm_x4(sbase + koff[ks] + mt * kstep[ks], kf[mt]);
+              else ldsm_x2(sbase + koff[ks] + mt * kstep[ks], kf[mt][0], kf[mt][1]);
+            }
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+              for (int j = 0; j < NB; ++j) {
+                if (k32) {
+                  if (ks == 0) mma_i8_k32<true, false>(ci[mt][j], kf[mt], qf8[ks][j][0], qf8[ks][j][1]);
+                  else mma_i8_k32<false, false>(ci[mt][j], kf[mt], qf8[ks][j][0], qf8[ks][j][1]);
+                } else {
+                  if (ks == 0) mma_i8_k16<true>(ci[mt][j], kf[mt][0], kf[mt][1], qf8[ks][j][0]);
+                  else mma_i8_k16<false>(ci[mt][j], kf[mt][0], kf[mt][1], qf8[ks][j][0]);
+                }
+              }
+          }
+        // the first value m-tiles' fragments do not depend on the scores: request them now
+#pragma unroll
+        for (int u = 0; u < VG8; ++u)
+          if (u < nmv) {
+#pragma unroll
+            for (int kk = 0; kk < MT / 2; ++kk) ldsm_x4_t(sbase + voff[u] + kk * vstep[u], vx8[u][kk]);
+          }
+        // the tile's key scales: tokens 16 mt + (lane >> 2) + 8 h
+        float skt[MT][2];
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            skt[mt][h] = lds_f32(sbase + L.q8_ks + 4u * (uint32_t)(16 * mt + (lane >> 2) + 8 * h));
+        // s = s_q k_scale (256 hi + lo), the parts added exactly in s32 (|256 hi + lo| < 2^30)
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            int v;
+            if constexpr (NB == 1) {
+              const int o = __shfl_xor_sync(kFull, ci[mt][0][e], 2);
+              v = lo_lane ? ci[mt][0][e] + o * 256 : ci[mt][0][e] * 256 + o;
+            } else {
+              v = ci[mt][0][e] * 256 + ci[mt][NB - 1][e];
+            }
+            s[mt][e] = (float)v * (skt[mt][e >> 1] * ((e & 1) ? sqB : sqA));
+          }
       }
       if (n < kTile) {  // missing tokens take no weight
 #pragma unroll
@@ -1011,48 +1076,143 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
         }
       }
       const float uA = mA == -INFINITY ? 0.f : mA, uB = mB == -INFINITY ? 0.f : mB;
-      // weights of the tile as B fragments of P^T: block r = tokens 8r..8r+7 in the score
-      // layout (row = token, columns = this lane's two heads), transposed to (token pairs, head)
-      uint32_t pb[NB][2 * MT];
       float pa_sum = 0.f, pb_sum = 0.f;
+      if constexpr (!Q8) {
+        // weights of the tile as B fragments of P^T: block r = tokens 8r..8r+7 in the score
+        // layout (row = token, columns = this lane's two heads), transposed to (token pairs, head)
+        uint32_t pb[NB][2 * MT];
 #pragma unroll
-      for (int r = 0; r < 2 * MT; ++r) {
-        const int mt = r >> 1, e0 = (r & 1) * 2;
-        const float pA = ex2(s[mt][e0] - uA), pB = ex2(s[mt][e0 + 1] - uB);
-        pa_sum += pA;
-        pb_sum += pB;
-        // int8 caches: the weights of code rows carry the rows' value scales (not in l)
-        const float sv = Q8 ? scw[kTile + 16 * mt + (lane >> 2) + 8 * (r & 1)] : 1.f;
-        const float wA = pA * sv, wB = pB * sv;
-        const uint32_t hw = Q8 ? hi_pair_h(wA, wB) : hi_pair(wA, wB);
-        const uint32_t lw = Q8 ? lo_pair_h(wA, wB, hw) : lo_pair(wA, wB, hw);
-        if constexpr (NB == 1) {
-          pb[0][r] = movm_t(lo_lane ? lw : hw);
-        } else {
-          pb[0][r] = movm_t(hw);
-          pb[NB - 1][r] = movm_t(lw);
+        for (int r = 0; r < 2 * MT; ++r) {
+          const int mt = r >> 1, e0 = (r & 1) * 2;
+          const float pA = ex2(s[mt][e0] - uA), pB = ex2(s[mt][e0 + 1] - uB);
+          pa_sum += pA;
+          pb_sum += pB;
+          const uint32_t hw = hi_pair(pA, pB);
+          const uint32_t lw = lo_pair(pA, pB, hw);
+          if constexpr (NB == 1) {
+            pb[0][r] = movm_t(lo_lane ? lw : hw);
+          } else {
+            pb[0][r] = movm_t(hw);
+            pb[NB - 1][r] = movm_t(lw);
+          }
         }
-      }
-      lA += pa_sum;
-      lB += pb_sum;
-
-      // value mix: O^T[dim][n] += V^T[dim][token] P^T[token][n]
+        lA += pa_sum;
+        lB += pb_sum;
+        // value mix: O^T[dim][n] += V^T[dim][token] P^T[token][n]
 #pragma unroll
-      for (int g0 = 0; g0 < NMV; g0 += VG)
-        if (g0 < nmv) {
-          if (g0 > 0) load_v(g0);
+        for (int g0 = 0; g0 < NMV; g0 += VG)
+          if (g0 < nmv) {
+            if (g0 > 0) load_v(g0);
 #pragma unroll
-          for (int u = 0; u < VG; ++u)
-            if (g0 + u < nmv) {
+            for (int u = 0; u < VG; ++u)
+              if (g0 + u < nmv) {
 #pragma unroll
-              for (int kk = 0; kk < MT; ++kk)
+                for (int kk = 0; kk < MT; ++kk)
+#pragma unroll
+                  for (int j = 0; j < NB; ++j)
+                    mma_bf16(oacc[g0 + u][j], vf[u][kk], pb[j][2 * kk], pb[j][2 * kk + 1]);
+              }
+          }
+      } else {
+        // int8 caches: a token's weight in the mix is p v_scale (the scale is not in l).  Per
+        // head and tile the weights become 16-bit fixed point, w16 = rint(w / sigma) with
+        // sigma = max w / 65535, split into two unsigned bytes (w16 = 256 hi + lo): the mix
+        // of the codes against each part is exact in s32 and sigma (256 for the hi part)
+        // brings it back into the fp32 accumulators.  Rows past the sequence take weight 0
+        // whatever their scale holds.
+        float svt[2 * MT];
+#pragma unroll
+        for (int r = 0; r < 2 * MT; ++r)
+          svt[r] = lds_f32(sbase + L.q8_vs + 4u * (uint32_t)(16 * (r >> 1) + (lane >> 2) + 8 * (r & 1)));
+        float wA[2 * MT], wB[2 * MT];
+        float xA = 0.f, xB = 0.f;
+#pragma unroll
+        for (int r = 0; r < 2 * MT; ++r) {
+          const int mt = r >> 1, e0 = (r & 1) * 2;
+          const float pA = ex2(s[mt][e0] - uA), pB = ex2(s[mt][e0 + 1] - uB);
+          pa_sum += pA;
+          pb_sum += pB;
+          const float sv = n < kTile && 16 * mt + (lane >> 2) + 8 * (r & 1) >= n ? 0.f : svt[r];
+          wA[r] = pA * sv;
+          wB[r] = pB * sv;
+          xA = fmaxf(xA, wA[r]);
+          xB = fmaxf(xB, wB[r]);
+        }
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+          xA = fmaxf(xA, __shfl_xor_sync(kFull, xA, o));
+          xB = fmaxf(xB, __shfl_xor_sync(kFull, xB, o));
+        }
+        lA += pa_sum;
+        lB += pb_sum;
+        const float fA = xA > 0.f ? 65535.f * rcp_approx(xA) : 0.f;
+        const float fB = xB > 0.f ? 65535.f * rcp_approx(xB) : 0.f;
+        // B fragments of W^T: per score m-tile, the lane's (token g, token g + 8) byte pairs of
+        // its two columns, transposed (movmatrix) to 4 tokens of one column.  Register r of a
+        // k32 step then holds tokens 2 (lane & 3) + {0, 8, 1, 9} + 16 r of column lane >> 2;
+        // the value fragments below put their tokens in the same order.
+        uint32_t pb8[NB][MT];
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          const uint32_t a0 = __float2uint_rn(wA[2 * mt] * fA), a1 = __float2uint_rn(wA[2 * mt + 1] * fA);
+          const uint32_t b0 = __float2uint_rn(wB[2 * mt] * fB), b1 = __float2uint_rn(wB[2 * mt + 1] * fB);
+          const uint32_t u = __byte_perm(a0, b0, 0x5410), v = __byte_perm(a1, b1, 0x5410);
+          // hi bytes: u.1 v.1 u.3 v.3; lo bytes: u.0 v.0 u.2 v.2
+          if constexpr (NB == 1) {
+            pb8[0][mt] = movm_t(__byte_perm(u, v, lo_lane ? 0x6240 : 0x7351));
+          } else {
+            pb8[0][mt] = movm_t(__byte_perm(u, v, 0x7351));
+            pb8[NB - 1][mt] = movm_t(__byte_perm(u, v, 0x6240));
+          }
+        }
+        const float sA = xA * (1.f / 65535.f), sB = xB * (1.f / 65535.f);
+        float zA[NB], zB[NB];  // sigma of the lane's two columns per n-tile (256 sigma: hi part)
+#pragma unroll
+        for (int j = 0; j < NB; ++j) {
+          const bool hi = NB == 1 ? !lo_lane : j == 0;
+          zA[j] = hi ? 256.f * sA : sA;
+          zB[j] = hi ? 256.f * sB : sB;
+        }
+        // value mix: the transposed x4 gives each lane, per 8 tokens, a 16-bit pair of dims
+        // (2 g, 2 g + 1) of tokens 2 (lane & 3) + {0, 1}; byte permutes make A rows of 4 tokens
+        // in the weights' order: row g is dim 2 g of the m-tile, row g + 8 dim 2 g + 1.
+#pragma unroll
+        for (int g0 = 0; g0 < NMV; g0 += VG8)
+          if (g0 < nmv) {
+            if (g0 > 0) {
+#pragma unroll
+              for (int u = 0; u < VG8; ++u)
+                if (g0 + u < nmv) {
+#pragma unroll
+                  for (int kk = 0; kk < MT / 2; ++kk)
+                    ldsm_x4_t(sbase + voff[g0 + u] + kk * vstep[g0 + u], vx8[u][kk]);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < VG8; ++u)
+              if (g0 + u < nmv) {
+                int acc[NB][4];
+#pragma unroll
+                for (int kk = 0; kk < MT / 2; ++kk) {
+                  const uint32_t* x = vx8[u][kk];
+                  const uint32_t af[4] = {__byte_perm(x[0], x[1], 0x6240), __byte_perm(x[0], x[1], 0x7351),
+                                          __byte_perm(x[2], x[3], 0x6240), __byte_perm(x[2], x[3], 0x7351)};
+#pragma unroll
+                  for (int j = 0; j < NB; ++j) {
+                    if (kk == 0) mma_i8_k32<true, true>(acc[j], af, pb8[j][2 * kk], pb8[j][2 * kk + 1]);
+                    else mma_i8_k32<false, true>(acc[j], af, pb8[j][2 * kk], pb8[j][2 * kk + 1]);
+                  }
+                }
 #pragma unroll
                 for (int j = 0; j < NB; ++j)
-                  mma_op<Q8>(oacc[g0 + u][j], vf[u][kk], pb[j][2 * kk], pb[j][2 * kk + 1]);
-            }
-        }
+#pragma unroll
+                  for (int e = 0; e < 4; ++e)
+                    oacc[g0 + u][j][e] = fmaf((float)acc[j][e], (e & 1) ? zB[j] : zA[j], oacc[g0 + u][j][e]);
+              }
+          }
+      }
       __syncwarp();
-      if (!Q8 && lane == 0) mbar_arrive(&empty[warp * ns + st]);  // the stage may be refilled
+      if (lane == 0) mbar_arrive(&empty[warp * ns + st]);  // the stage may be refilled
     }
   }
 
@@ -1064,7 +1224,9 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
     lA += __shfl_xor_sync(kFull, lA, o);
     lB += __shfl_xor_sync(kFull, lB, o);
   }
-  float ov[NMV][4];  // o~ of (dim 16 mt + (lane >> 2) + 8 (e >> 1), head hA + (e & 1))
+  // o~ of (dim 16 mt + (lane >> 2) + 8 (e >> 1), head hA + (e & 1)); int8 caches: dim
+  // 16 mt + 2 (lane >> 2) + (e >> 1)
+  float ov[NMV][4];
 #pragma unroll
   for (int mt = 0; mt < NMV; ++mt)
 #pragma unroll
@@ -1104,8 +1266,8 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
         if (mt < nmv)
 #pragma unroll
           for (int e = 0; e < 4; ++e)
-            sts_f32(redb + 4u * (uint32_t)((warp * 8 + hA + (e & 1)) * rV + 16 * mt + (lane >> 2) +
-                                           8 * (e >> 1)),
+            sts_f32(redb + 4u * (uint32_t)((warp * 8 + hA + (e & 1)) * rV + 16 * mt +
+                                           (Q8 ? 2 * (lane >> 2) + (e >> 1) : (lane >> 2) + 8 * (e >> 1))),
                     ov[mt][e] * ((e & 1) ? fB : fA));
       if ((lane >> 2) == 0) {  // the sums rescaled in place (only the maxima were read above)
         sts_f32(mlb + 8u * (uint32_t)(warp * 8 + hA) + 4u, lA * fA);

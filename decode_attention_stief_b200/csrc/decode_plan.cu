@@ -68,7 +68,8 @@ bool cached_map(CUtensorMap* out, const void* base, int r, uint64_t rows, int bo
   }
   const CUtensorMapSwizzle sw = width == 64   ? CU_TENSOR_MAP_SWIZZLE_128B
                                 : width == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
-                                              : CU_TENSOR_MAP_SWIZZLE_32B;
+                                : width == 16 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                              : CU_TENSOR_MAP_SWIZZLE_NONE;
   if (!encode_tiled_bf16_2d(out, base, (uint64_t)r, rows, (uint64_t)r * 2u, (uint32_t)width,
                             (uint32_t)box_rows, sw))
     return false;
@@ -79,23 +80,26 @@ bool cached_map(CUtensorMap* out, const void* base, int r, uint64_t rows, int bo
   return true;
 }
 
-// Column pieces of a rank-r matrix (r a multiple of 16): widths 64, 64, 32, 16 taken in
-// that order while they fit, each with its own tensor map (one per width, shared by
-// the pieces of that width) over `base` viewed as [rows][r] bf16, boxes of
-// width x box_rows.  Pieces are stacked in shared memory in the same order.
+// Column pieces of a matrix r 16-bit columns wide (r a multiple of 8): widths 64, 64, 32,
+// 16, 8 taken in that order while they fit, each with its own tensor map (one per width,
+// shared by the pieces of that width) over `base` viewed as [rows][r] 16-bit elements, boxes
+// of width x box_rows, swizzled 128, 64 or 32 bytes (the 8-wide piece, 16 bytes, is not
+// swizzled).  Pieces are stacked in shared memory in the same order.  A bf16 matrix of rank r
+// is r columns; an int8 matrix of rank r is viewed as r / 2 columns (the copy moves bytes).
 bool plan_pieces(DecodeArgs& a, int* nmaps, PieceSet& ps, const void* base, int r, uint64_t rows,
                  int box_rows) {
-  int map_of_width[3] = {-1, -1, -1};  // for 64, 32, 16
+  int map_of_width[4] = {-1, -1, -1, -1};  // for 64, 32, 16, 8
   int x = 0, off = 0;
   ps.n = 0;
-  for (int w : {64, 64, 32, 16}) {
+  for (int w : {64, 64, 32, 16, 8}) {
     if (r - x < w) continue;
-    const int wi = w == 64 ? 0 : w == 32 ? 1 : 2;
+    const int wi = w == 64 ? 0 : w == 32 ? 1 : w == 16 ? 2 : 3;
     if (map_of_width[wi] < 0) {
       if (*nmaps >= 12) return false;
       if (!cached_map(&a.maps[*nmaps], base, r, rows, box_rows, w)) return false;
       map_of_width[wi] = (*nmaps)++;
     }
+    if (ps.n >= 3) return false;
     Piece& p = ps.p[ps.n++];
     p.x = x;
     p.width = w;
@@ -155,21 +159,6 @@ bool encode_tiled_bf16_2d(CUtensorMap* map, const void* base, uint64_t cols, uin
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// 2-D tiled map over an int8 matrix [rows][cols] (row stride = cols bytes), boxes of
-// box_cols x box_rows, no swizzle (the int8 stages are read row-major).
-static bool encode_tiled_u8_2d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
-                               uint32_t box_cols, uint32_t box_rows) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)cols};
-  const cuuint32_t box[2] = {box_cols, box_rows};
-  const cuuint32_t estr[2] = {1u, 1u};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 stief_status plan_decode(DecodeArgs& a, const uint16_t* q, const uint16_t* P_K,
@@ -233,7 +222,7 @@ stief_status plan_decode(DecodeArgs& a, const uint16_t* q, const uint16_t* P_K,
   a.max_seq_len = max_seq_len;
   // tokens per split: the split's share rounded up to whole 32-token tiles, so that only
   // the last tile of a sequence can be partial
-  a.tile = choose_decode_tile(rK, rV);
+  a.tile = q8 ? choose_decode_tile_q8(rK, rV) : choose_decode_tile(rK, rV);
   a.chunk = ((max_seq_len + a.S - 1) / a.S + a.tile - 1) / a.tile * a.tile;
   a.qscale = (float)(1.4426950408889634 / std::sqrt((double)d));
   const long long units = (long long)B * a.Hkv * a.qsub;
@@ -256,22 +245,10 @@ stief_status plan_decode(DecodeArgs& a, const uint16_t* q, const uint16_t* P_K,
   a.q8 = q8 ? 1 : 0;
   a.k_scale = k_scale;
   a.v_scale = v_scale;
-  if (q8) {  // int8 codes: one box of r bytes x tile rows per matrix
-    if (!encode_tiled_u8_2d(&a.maps[0], k_lat, (uint64_t)rK, rows, (uint32_t)rK, (uint32_t)a.tile) ||
-        !encode_tiled_u8_2d(&a.maps[1], v_lat, (uint64_t)rV, rows, (uint32_t)rV, (uint32_t)a.tile))
-      return STIEF_ERR_CUDA;
-    a.pk.n = a.pv.n = 1;
-    a.pk.p[0] = Piece{};
-    a.pv.p[0] = Piece{};
-    a.pk.p[0].map = 0;
-    a.pv.p[0].map = 1;
-    a.pk.p[0].width = rK;
-    a.pv.p[0].width = rV;
-    nmaps = 2;
-  } else if (!plan_pieces(a, &nmaps, a.pk, k_lat, rK, rows, a.tile) ||
-             !plan_pieces(a, &nmaps, a.pv, v_lat, rV, vrows, a.tile)) {
+  // the caches' column pieces (int8 codes: rows of r bytes, moved as r / 2 16-bit columns)
+  if (!plan_pieces(a, &nmaps, a.pk, k_lat, q8 ? rK / 2 : rK, rows, a.tile) ||
+      !plan_pieces(a, &nmaps, a.pv, v_lat, q8 ? rV / 2 : rV, vrows, a.tile))
     return STIEF_ERR_CUDA;
-  }
   if (!latent && (!plan_pieces(a, &nmaps, a.ppk, P_K, rK, prow, d) ||
                   !plan_pieces(a, &nmaps, a.ppv, P_V, rV, prow, d)))
     return STIEF_ERR_CUDA;

@@ -176,6 +176,8 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
 // Tokens per tile: 64 for small ranks (an SM sustains a roughly fixed number of tiles per
 // microsecond, so small tiles would leave the memory system idle), 32 otherwise.
 inline int choose_decode_tile(int rK, int rV) { return rK <= 64 && rV <= 64 && rK + rV <= 96 ? 64 : 32; }
+// int8 caches: rows take half the bytes, so 64-token tiles whenever both ranks are <= 64.
+inline int choose_decode_tile_q8(int rK, int rV) { return rK <= 64 && rV <= 64 ? 64 : 32; }
 
 // Consumer warps per CTA and stages per warp for the decode kernel: 8 warps with as many
 // stages (up to 8) as shared memory allows, fewer warps only when 8 cannot have two each.

@@ -348,9 +348,12 @@ STIEF_API stief_status stief_append_decode_paged(const uint16_t* q, const uint16
  * IEEE fp32; a zero row is scale 0 and codes 0.  A value stands for code * scale.
  * A row takes r + 4 bytes instead of the bf16 cache's 2 r.  L_max must be a multiple of 64; k_s, v_s, k_q, v_q
  * 16-byte aligned.  The calls are their bf16 counterparts on this form: the compress writes
- * codes and scales; the decode attends over code * scale (codes become exact fp16 on chip;
- * the row scales multiply the scores and the softmax weights).  Paged int8 caches and the
- * fused step are not provided.
+ * codes and scales; the decode attends over code * scale.  On chip the codes enter the integer
+ * tensor-core MMA as they are: q~ is held per head as 16-bit fixed point (relative step
+ * 2^-15 of its largest element) and each tile's softmax weights per head as 16-bit fixed point
+ * of the tile's largest weight, each split into two 8-bit parts, so both products are exact
+ * in 32-bit integers; the row scales multiply the scores and the weights.  Paged int8 caches
+ * and the fused step are not provided.
  */
 STIEF_API stief_status stief_compress_append_q8(const uint16_t* k_new, const uint16_t* v_new,
                                       const uint16_t* P_K, const uint16_t* P_V, int8_t* k_q,

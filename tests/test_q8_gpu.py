@@ -170,3 +170,107 @@ def test_decode_q8_multi_wave_grid():
                          oracle.dequantize_rows(vq.numpy(), vs.numpy()), np.asarray(lens, np.int32))
     assert_decode_close(got, want)
     assert torch.all(got[5].float() == 0)
+
+
+def _q8_case(seed, B, Hq, Hkv, L, rK, rV, q_scale=1.0):
+    q = si.queries(seed, B, Hq, 128, scale=q_scale)
+    P_K, P_V = si.bases_bf16(seed + 1, Hkv, 128, rK, rV)
+    kq, ks = _random_q8_cache(seed + 2, B, Hkv, L, rK)
+    vq, vs = _random_q8_cache(seed + 3, B, Hkv, L, rV)
+    return q, P_K, P_V, kq, vq, ks, vs
+
+
+def _oracle_q8(q, P_K, P_V, kq, vq, ks, vs, lens):
+    return oracle.decode(f64(q), f64(P_K), f64(P_V), oracle.dequantize_rows(kq.numpy(), ks.numpy()),
+                         oracle.dequantize_rows(vq.numpy(), vs.numpy()), np.asarray(lens, np.int32))
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(32, 4), (8, 4), (24, 4), (4, 4)])
+@pytest.mark.parametrize("num_splits", [0, 2])
+def test_decode_q8_group_sizes(Hq, Hkv, num_splits):
+    """Query groups of 8 (the hi and lo parts in two n-tiles), 2, 6 (padded to 8) and 1."""
+    B, L, rK, rV = 2, 448, 64, 64
+    lens = [445, 130]
+    args = _q8_case(6500 + Hq, B, Hq, Hkv, L, rK, rV)
+    got = _decode_q8(*args, lens, 445, num_splits)
+    assert_decode_close(got, _oracle_q8(*args, lens))
+
+
+@pytest.mark.parametrize("rK,rV", [(48, 16), (80, 112), (112, 48), (16, 96), (128, 128)])
+def test_decode_q8_odd_ranks(rK, rV):
+    """Ranks whose rows are 16 x odd bytes: a 16-code last k-step for the scores, and 16-byte
+    (unswizzled) column pieces for the values and keys."""
+    B, Hq, Hkv, L = 2, 16, 4, 320
+    lens = [317, 64]
+    args = _q8_case(6600 + rK + rV, B, Hq, Hkv, L, rK, rV)
+    got = _decode_q8(*args, lens, 317, 0)
+    assert_decode_close(got, _oracle_q8(*args, lens))
+
+
+@pytest.mark.parametrize("lens", [[63, 64, 65], [127, 128, 129], [1, 31, 32]])
+def test_decode_q8_tile_boundaries(lens):
+    """Lengths at the 32- and 64-token tile edges (the 64/64 ranks take 64-token tiles)."""
+    B, Hq, Hkv, L, rK, rV = 3, 16, 4, 192, 64, 64
+    args = _q8_case(6700 + sum(lens), B, Hq, Hkv, L, rK, rV)
+    got = _decode_q8(*args, lens, 129, 0)
+    assert_decode_close(got, _oracle_q8(*args, lens))
+
+
+@pytest.mark.parametrize("q_scale", [4.0, 16.0])
+def test_decode_q8_peaked_scores(q_scale):
+    """Large queries make the softmax peaked (a few tokens carry the weight; the running
+    maximum is rescaled often)."""
+    B, Hq, Hkv, L, rK, rV = 2, 32, 8, 1024, 64, 64
+    lens = [1024, 517]
+    args = _q8_case(6800, B, Hq, Hkv, L, rK, rV, q_scale=q_scale)
+    got = _decode_q8(*args, lens, 1024, 0)
+    assert_decode_close(got, _oracle_q8(*args, lens))
+
+
+def test_decode_q8_needle_and_spread_mass():
+    """One needle token per (sequence, KV head) whose score is 12 above the other tokens' best,
+    so that it carries most of the weight while the rest still hold a few per cent: the
+    per-tile fixed point of the weights must keep both."""
+    B, Hq, Hkv, L, rK, rV = 2, 16, 4, 2048, 64, 64
+    G = Hq // Hkv
+    lens = [2048, 1500]
+    q, P_K, P_V, kq, vq, ks, vs = _q8_case(6900, B, Hq, Hkv, L, rK, rV)
+    kq, ks = kq.clone(), ks.clone()
+    rng = np.random.default_rng(6901)
+    k_deq = oracle.dequantize_rows(kq.numpy(), ks.numpy())
+    for b in range(B):
+        for h in range(Hkv):
+            qt = f64(q[b, h * G]) @ f64(P_K[h])  # q~ of the group's first head
+            s = k_deq[b, h, :lens[b]] @ qt / np.sqrt(128.0)
+            pos = int(rng.integers(0, lens[b]))
+            codes = np.where(qt >= 0, 127, -127).astype(np.int8)
+            scale = (s.max() + 12.0) * np.sqrt(128.0) / (127.0 * np.abs(qt).sum())
+            kq[b, h, pos] = torch.from_numpy(codes)
+            ks[b, h, pos] = float(np.float32(scale))
+    args = (q, P_K, P_V, kq, vq, ks, vs)
+    got = _decode_q8(*args, lens, 2048, 0)
+    assert_decode_close(got, _oracle_q8(*args, lens))
+
+
+@pytest.mark.parametrize("num_splits", [0, 3])
+def test_decode_q8_rows_past_length_hold_garbage(num_splits):
+    """Codes and scales past each length are arbitrary (NaN and inf scales included): they
+    must reach neither the scores nor the mix."""
+    B, Hq, Hkv, L, rK, rV = 3, 16, 4, 384, 48, 64
+    lens = [300, 33, 0]
+    q, P_K, P_V, kq, vq, ks, vs = _q8_case(7000, B, Hq, Hkv, L, rK, rV)
+    kq, vq, ks, vs = kq.clone(), vq.clone(), ks.clone(), vs.clone()
+    rng = np.random.default_rng(7001)
+    bad = np.array([np.nan, np.inf, -np.inf, 3e38], np.float32)
+    for b in range(B):
+        n = L - lens[b]
+        kq[b, :, lens[b]:] = torch.from_numpy(rng.integers(-128, 128, (Hkv, n, rK), dtype=np.int8))
+        vq[b, :, lens[b]:] = torch.from_numpy(rng.integers(-128, 128, (Hkv, n, rV), dtype=np.int8))
+        ks[b, :, lens[b]:] = torch.from_numpy(rng.choice(bad, (Hkv, n)))
+        vs[b, :, lens[b]:] = torch.from_numpy(rng.choice(bad, (Hkv, n)))
+    args = (q, P_K, P_V, kq, vq, ks, vs)
+    got = _decode_q8(*args, lens, 384, num_splits)
+    want = _oracle_q8(q, P_K, P_V, kq, vq, torch.nan_to_num(ks, 0.0, 0.0, 0.0),
+                      torch.nan_to_num(vs, 0.0, 0.0, 0.0), lens)
+    assert_decode_close(got, want)
+    assert torch.all(got[2].float() == 0)
