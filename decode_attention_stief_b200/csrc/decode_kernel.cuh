@@ -285,11 +285,11 @@ struct DecodeSmem {
   uint32_t region;  // per warp a ring of stages (keys then values of a tile); later the
                     // cross-warp reduction and the split-merge staging
   uint32_t region_bytes;
-  uint32_t stage;             // bytes of one ring stage (a multiple of 1 KiB)
-  // int8 caches: a stage holds the key codes [tile][rK] and the value codes [tile][rV] in
-  // column pieces like the bf16 tiles (the rows' bytes read as 16-bit columns), then the
-  // tile's key and value row scales (fp32)
-  uint32_t q8_v, q8_ks, q8_vs;  // offsets inside an int8 stage
+  uint32_t stage;  // bytes of one ring stage (a multiple of 1 KiB)
+  // int8 caches: a stage holds the key codes [tile][rK] and, from q8_v, the value codes
+  // [tile][rV], in column pieces like the bf16 tiles (the rows' bytes read as 16-bit
+  // columns); the row scales are not staged (the consumer lanes load them)
+  uint32_t q8_v;
   uint32_t total;
   int xs;  // row stride of qt in floats
 };
@@ -317,11 +317,9 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int NW, int ns, int rK,
   s.region = off;
   if (q8) {
     s.q8_v = align_up((uint32_t)tile * rK, 1024);  // the swizzle patterns need 1 KiB alignment
-    s.q8_ks = s.q8_v + (uint32_t)tile * rV;
-    s.q8_vs = s.q8_ks + (uint32_t)tile * 4u;
-    s.stage = align_up(s.q8_vs + (uint32_t)tile * 4u, 1024);
+    s.stage = align_up(s.q8_v + (uint32_t)tile * rV, 1024);
   } else {
-    s.q8_v = s.q8_ks = s.q8_vs = 0;
+    s.q8_v = 0;
     s.stage = (uint32_t)tile * (rK + rV) * 2u;  // a multiple of 1 KiB
   }
   s.region_bytes = (uint32_t)NW * ns * s.stage;
@@ -385,9 +383,9 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
   float* qt = reinterpret_cast<float*>(smem + L.qt);
   const int xs = L.xs;
   uint8_t* pmat = smem + L.pmat;
-  // a stage: the key tile, then the value tile at kt_bytes (int8 caches: then the row scales)
+  // a stage: the key tile, then the value tile at kt_bytes
   const uint32_t kt_bytes = Q8 ? L.q8_v : (uint32_t)kTile * rK * 2u;
-  const uint32_t st_bytes = Q8 ? (uint32_t)kTile * (rK + rV + 8) : kt_bytes + (uint32_t)kTile * rV * 2u;
+  const uint32_t st_bytes = Q8 ? (uint32_t)kTile * (rK + rV) : kt_bytes + (uint32_t)kTile * rV * 2u;
 
   // the swizzle patterns assume 1 KiB-aligned tiles
   if (((smem_u32(smem + L.pmat) | smem_u32(smem + L.region)) & 1023u) != 0) {
@@ -467,10 +465,6 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
 #pragma unroll
     for (int p = 0; p < 3; ++p)
       if (p < npv) tma_load_2d(dst + vo[p], vmap[p], vx[p], yv, bar, policy);
-    if (Q8) {  // the tile's two rows of scales
-      bulk_g2s(dst + L.q8_ks, a.k_scale + y, 4u * kTile, bar);
-      bulk_g2s(dst + L.q8_vs, a.v_scale + y, 4u * kTile, bar);
-    }
   };
 
   // Contiguous bf16 caches (plain and latent modes): every warp's first tile is requested
@@ -552,6 +546,21 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
     }
   };
   const int n_tiles = t1 > t0 ? (t1 - t0 + kTile - 1) / kTile : 0;
+  // int8 caches: the row scales of a tile come by coalesced loads, requested one tile ahead
+  // (a TMA or bulk copy per tile costs more than its bytes): lane i holds the scales of
+  // tokens i + 32 j of the tile.  The first tile's are requested before the setup wait.
+  constexpr int SJ = Q8 ? TT / 32 : 1;
+  float skc[SJ], svc[SJ], skn[SJ], svn[SJ];
+  auto load_scales = [&](int kk) {
+    if (kk < warp_tiles(warp, n_tiles)) {
+      const long long row = cache_row(cr, b, kvh, t0 + (warp + kk * NW) * kTile) + lane;
+#pragma unroll
+      for (int j = 0; j < SJ; ++j) {
+        skn[j] = __ldg(a.k_scale + row + 32 * j);
+        svn[j] = __ldg(a.v_scale + row + 32 * j);
+      }
+    }
+  };
   // ---- prologue ------------------------------------------------------------------------------
   bool ok = true;
   if (producer) {
@@ -592,6 +601,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
     // q~ = q P_K on the MMA: q~^T[j][head] = sum_i P_K[i][j] q[head][i]
     // (M = the r_K columns of P_K, N = 8 heads, K = d), scaled into log2 units
     const int n = lane >> 2;  // B column = head
+    if constexpr (Q8) load_scales(0);
     ok = warp_wait(setup_bar, 0, a.dev_status);
     if (!ok && lane == 0) flag[1] = 1;
     uint32_t qb[8][2];  // d / 16 k-steps (explicit shared loads issued together)
@@ -859,8 +869,17 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
       vstep[mt] = 32u * pl.w;
     }
 
+
     for (int k = 0; k < my_tiles && ok; ++k) {
       const int st = k % ns;
+      if constexpr (Q8) {
+#pragma unroll
+        for (int j = 0; j < SJ; ++j) {
+          skc[j] = skn[j];
+          svc[j] = svn[j];
+        }
+        load_scales(k + 1);
+      }
       if (!warp_wait(&full[warp * ns + st], (uint32_t)((k / ns) & 1), a.dev_status)) {
         ok = false;
         break;
@@ -1009,7 +1028,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
         for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
           for (int h = 0; h < 2; ++h)
-            skt[mt][h] = lds_f32(sbase + L.q8_ks + 4u * (uint32_t)(16 * mt + (lane >> 2) + 8 * h));
+            skt[mt][h] = __shfl_sync(kFull, skc[(16 * mt + 8 * h) >> 5], ((16 * mt + 8 * h) & 31) + (lane >> 2));
         // s = s_q k_scale (256 hi + lo), the parts added exactly in s32 (|256 hi + lo| < 2^30)
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt)
@@ -1123,7 +1142,8 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
         float svt[2 * MT];
 #pragma unroll
         for (int r = 0; r < 2 * MT; ++r)
-          svt[r] = lds_f32(sbase + L.q8_vs + 4u * (uint32_t)(16 * (r >> 1) + (lane >> 2) + 8 * (r & 1)));
+          svt[r] = __shfl_sync(kFull, svc[(16 * (r >> 1) + 8 * (r & 1)) >> 5],
+                               ((16 * (r >> 1) + 8 * (r & 1)) & 31) + (lane >> 2));
         float wA[2 * MT], wB[2 * MT];
         float xA = 0.f, xB = 0.f;
 #pragma unroll
