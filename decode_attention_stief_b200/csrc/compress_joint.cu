@@ -101,7 +101,10 @@ cudaError_t launch_compress_joint(const CompressArgs& a, cudaStream_t stream) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   stief_joint_lens_kernel<<<(a.B + 255) / 256, 256, 0, stream>>>(a);
-  return cudaGetLastError();
+  e = cudaGetLastError();
+  // these kernels let no dependent start early: a decode that follows may read ahead
+  if (e == cudaSuccess) mark_stream_compress(a.device, stream, false);
+  return e;
 }
 
 }  // namespace stief

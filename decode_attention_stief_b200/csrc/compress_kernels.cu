@@ -130,6 +130,10 @@ __global__ void __launch_bounds__(kSmallThreads) stief_compress_rows_kernel(cons
 }
 
 __global__ void __launch_bounds__(256) stief_seq_lens_kernel(const CompressArgs a) {
+  // the next kernel may start now: its inputs are read only after its own dependency wait
+  // (which waits for this grid, and so for the projection), and a decode launched right after
+  // a compress reads no cache tile before that wait (the library marks the stream)
+  pdl_launch_dependents();
   pdl_wait();  // every projection CTA has finished reading the old lengths
   const CacheRows cr{a.block_table, a.max_pages, a.page_size, a.num_pages, a.Hkv, a.L_max};
   for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < a.B; b += gridDim.x * blockDim.x) {
@@ -174,7 +178,9 @@ cudaError_t launch_compress(const CompressArgs& a, cudaStream_t stream) {
   else
     e = (a.T == 1) ? launch_rows<1>(a, stream) : launch_rows<kRowsPerCta>(a, stream);
   if (e != cudaSuccess) return e;
-  return launch_seq_lens(a, stream);
+  e = launch_seq_lens(a, stream);
+  if (e == cudaSuccess) mark_stream_compress(a.device, stream, true);
+  return e;
 }
 
 }  // namespace stief

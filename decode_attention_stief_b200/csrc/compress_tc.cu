@@ -15,8 +15,9 @@
 //   - one thread issues tcgen05.mma; completion is signalled by tcgen05.commit on an
 //     mbarrier; the accumulators live in 256 columns of tensor memory (D_K at column
 //     0, D_V at column 128);
-//   - epilogue: each of 4 warps reads its 32 TMEM lanes (rows) with tcgen05.ld, rounds
-//     to bf16 (RNE) and stores its rows into the latent cache at seq_lens[b] + row.
+//   - epilogue: each of 8 warps reads 32 TMEM lanes (rows) of the keys' or the values'
+//     columns with tcgen05.ld, rounds to bf16 (RNE) and stores its rows into the latent
+//     cache at seq_lens[b] + row.
 // A CTA loops over m-tiles of one (b, h) so P is staged once.  The kernel is launched as a
 // programmatic dependent: barrier set-up, the tensor-memory allocation and the staging of
 // the bases (weights, which the preceding kernel must not write) overlap the preceding
@@ -37,7 +38,9 @@ namespace {
 
 constexpr int kTcRows = 128;     // M: rows (tokens) per MMA tile
 constexpr int kTcStages = 2;     // X tiles in flight per CTA
-constexpr int kTcThreads = 128;  // 4 warps: TMEM lanes 32w .. 32w + 31
+// 8 warps: warp w reads TMEM lanes 32 (w & 3) .. + 31 (rows), the keys' columns for w < 4 and
+// the values' for w >= 4
+constexpr int kTcThreads = 256;
 constexpr uint32_t kTmemCols = 256;
 
 // Shared-memory layout (byte offsets, all swizzled operands 1 KiB aligned).
@@ -124,34 +127,33 @@ __device__ __forceinline__ void tc_fence_after() {
 }
 
 // P[h] ([128][r] row-major in global) -> shared [r rows][128 k] K-major SW128, two atoms.
-// Thread = row k of P (128 threads, d = 128): it reads its row of both bases first (all
-// loads in flight together), then writes its k into every row n of each.
+// Threads 0-127 stage P_K and threads 128-255 P_V; thread = row k of its basis (d = 128): it
+// reads its row first (all loads in flight together), then writes its k into every row n.
 __device__ __forceinline__ void stage_bases(uint8_t* smem, const uint32_t (&atk)[2],
                                             const uint32_t (&atv)[2], const uint16_t* PK,
                                             const uint16_t* PV, int rK, int rV, int tid) {
   constexpr int kMaxChunks = 16;  // r <= 128: 16 chunks of 8 columns
-  const int k = tid;
-  uint4 wk[kMaxChunks], wv[kMaxChunks];
+  const int k = tid & 127;
+  const bool vals = tid >= 128;
+  const int r = vals ? rV : rK;
+  const uint16_t* P = vals ? PV : PK;
+  const uint32_t(&atom)[2] = vals ? atv : atk;
+  uint4 w[kMaxChunks];
+#pragma unroll
+  for (int q = 0; q < kMaxChunks; ++q)
+    if (8 * q < r) w[q] = __ldg(reinterpret_cast<const uint4*>(P + (size_t)k * r) + q);
+  const uint32_t kb = (uint32_t)(k & 63) * 2u;  // byte of k inside the 128-byte row
+  const uint32_t at = atom[k >> 6];
 #pragma unroll
   for (int q = 0; q < kMaxChunks; ++q) {
-    if (8 * q < rK) wk[q] = __ldg(reinterpret_cast<const uint4*>(PK + (size_t)k * rK) + q);
-    if (8 * q < rV) wv[q] = __ldg(reinterpret_cast<const uint4*>(PV + (size_t)k * rV) + q);
-  }
-  const uint32_t kb = (uint32_t)(k & 63) * 2u;  // byte of k inside the 128-byte row
-  auto put = [&](const uint32_t (&atom)[2], const uint4& w, int n0) {
-    const uint32_t at = atom[k >> 6];
-    const uint32_t v[4] = {w.x, w.y, w.z, w.w};
+    if (8 * q >= r) continue;
+    const uint32_t v[4] = {w[q].x, w[q].y, w[q].z, w[q].w};
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      const int n = n0 + j;
+      const int n = 8 * q + j;
       const uint32_t off = at + (uint32_t)n * 128u + ((((kb >> 4) ^ (uint32_t)(n & 7)) << 4) | (kb & 15u));
       *reinterpret_cast<uint16_t*>(smem + off) = (uint16_t)(v[j >> 1] >> (16 * (j & 1)));
     }
-  };
-#pragma unroll
-  for (int q = 0; q < kMaxChunks; ++q) {
-    if (8 * q < rK) put(atk, wk[q], 8 * q);
-    if (8 * q < rV) put(atv, wv[q], 8 * q);
   }
 }
 
@@ -261,13 +263,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // the MMA has read stage st: refill it with tile i + kTcStages
     if (tid == 0 && i + kTcStages < my_tiles) issue(i + kTcStages);
 
-    // epilogue: warp w owns rows 32w .. 32w + 31 (TMEM lanes); lane = row
+    // epilogue: warp w owns rows 32 (w & 3) .. + 31 (TMEM lanes; lane = row) of the keys
+    // (w < 4) or of the values (w >= 4)
     const int m0 = tile_m0(i);
-    const int row = warp * 32 + lane;
+    const int row = (warp & 3) * 32 + lane;
+    const int which = warp >> 2;  // 0: keys, 1: values
     const bool live = m0 + row < T;
     const long long crow = live ? cache_row(cr, b, h, Lb + m0 + row) : 0;  // mapped (checked)
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-    for (int which = 0; which < 2 && a.k_scale != nullptr; ++which) {
+    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    if (a.k_scale != nullptr) {
       // int8 cache: the row rounded to bf16, then one fp32 scale (max / 127) and RNE codes,
       // divisions in IEEE fp32; the accumulators are read twice (maximum, then codes)
       const int r = which ? rV : rK;
@@ -300,7 +304,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       if (live) (which ? a.v_scale : a.k_scale)[crow] = scale;
     }
-    for (int which = 0; which < 2 && a.k_scale == nullptr; ++which) {
+    if (a.k_scale == nullptr) {
       const int r = which ? rV : rK;
       uint16_t* dst = (which ? a.v_lat : a.k_lat) + crow * r;
       for (int c0 = 0; c0 < r; c0 += 16) {

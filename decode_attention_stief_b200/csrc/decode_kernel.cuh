@@ -473,10 +473,11 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
   // data by microseconds).  The calls document that the kernel immediately preceding them
   // must not write the cache rows below the lengths, except the row just below each length
   // (the one a preceding fused step on the same caches appends), which is read again after
-  // the wait.
-  constexpr bool EARLY = MODE == kModePlain || MODE == kModeLatent;
+  // the wait.  Right after a compress of this library (whose new rows may still be in flight)
+  // the host clears `early` and nothing is requested before the wait.
+  const bool early_tiles = (MODE == kModePlain || MODE == kModeLatent) && a.early != 0;
   int ring_issued = 0;  // producer lane w: tiles [0, ring_issued) of warp w are requested
-  if (EARLY && producer && lane < NW) {
+  if (early_tiles && producer && lane < NW) {
     const uint64_t stream = l2_policy_evict_first();
     ring_issued = min(min(kPreIssue, ns), warp_tiles(lane, spec_tiles));
     for (int k = 0; k < ring_issued; ++k) issue(lane, k, stream);
@@ -501,7 +502,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
                    "r"(2u * gcount * d) : "memory");
       bulk_g2s(smem + L.qraw, a.q + ((size_t)b * a.Hq + h0) * d, 2u * gcount * d, setup_bar);
     }
-    if (!EARLY && lane < NW) {
+    if (!early_tiles && lane < NW) {
       const uint64_t stream = l2_policy_evict_first();
       ring_issued = min(min(kPreIssue, ns), warp_tiles(lane, spec_tiles));
       for (int k = 0; k < ring_issued; ++k) issue(lane, k, stream);
@@ -887,7 +888,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
       const uint32_t sbase = smem_u32(ring + (size_t)st * L.stage);
       const int tok0 = t0 + (warp + k * NW) * kTile;
       const int n = min(kTile, t1 - tok0);
-      if (EARLY && k < kPreIssue && Lb >= 1 && tok0 <= Lb - 1 && Lb - 1 < tok0 + kTile) {
+      if (early_tiles && k < kPreIssue && Lb >= 1 && tok0 <= Lb - 1 && Lb - 1 < tok0 + kTile) {
         // this tile was requested before the dependency wait: the row just below the length
         // may have been appended by the preceding kernel (a fused step on the same caches),
         // so it is read again now (L2; the wait made it visible)

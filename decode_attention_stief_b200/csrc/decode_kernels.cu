@@ -14,7 +14,11 @@ uint32_t decode_region_bytes(int nwarps, int nstage, int rK, int rV, int tile, b
 
 // the latent decode, paged, int8 and joint-value caches are their own instantiations, so their
 // branches cost the contiguous path nothing (a runtime flag cost it 0.5-0.8 us per launch)
-cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
+cudaError_t launch_decode(const DecodeArgs& planned, cudaStream_t stream) {
+  DecodeArgs a = planned;
+  // right after a compress of this library the new rows may still be in flight when this
+  // kernel starts: no cache tile is requested before the dependency wait then
+  a.early = take_stream_compress_mark(a.device, stream) ? 0 : 1;
   if ((a.latent != 0) + (a.block_table != nullptr) + (a.q8 != 0) > 1)
     return cudaErrorInvalidValue;  // the modes do not combine
   if (a.joint_v) {

@@ -3,7 +3,9 @@
 #include <cmath>
 #include <cstdint>
 #include <atomic>
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -128,6 +130,22 @@ std::atomic<uint32_t> g_test_stall{0};
 #ifdef STIEF_TEST_HOOKS
 uint32_t test_stall_bytes() { return g_test_stall.load(); }
 #endif
+
+namespace {
+std::mutex g_mark_mu;
+std::map<std::pair<int, cudaStream_t>, bool> g_compress_mark;  // (device, stream) -> marked
+}  // namespace
+
+void mark_stream_compress(int device, cudaStream_t s, bool marked) {
+  std::lock_guard<std::mutex> lock(g_mark_mu);
+  if (marked) g_compress_mark[{device, s}] = true;
+  else g_compress_mark.erase({device, s});
+}
+
+bool take_stream_compress_mark(int device, cudaStream_t s) {
+  std::lock_guard<std::mutex> lock(g_mark_mu);
+  return g_compress_mark.erase({device, s}) != 0;
+}
 
 bool query_device(int* dev_out, int* sms, bool* sm100) {
   int dev = 0;

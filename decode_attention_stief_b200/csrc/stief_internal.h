@@ -70,6 +70,10 @@ struct DecodeArgs {
   // int8 caches: k_lat / v_lat hold int8 codes [rows][r] and these the fp32 row scales
   int q8;
   int joint_v;     // values: one row per (sequence, token) shared by the KV heads
+  // 1: the contiguous bf16 and latent modes request each warp's first tile before the
+  // dependency wait; 0 when the library's previous launch in the stream was a compress (its
+  // length kernel lets the next kernel start while the new rows are still being written)
+  int early;
   const float* k_scale;
   const float* v_scale;
 #ifdef STIEF_TEST_HOOKS
@@ -172,6 +176,13 @@ inline size_t decode_tagged_stage_bytes(int G_T, int splits, int rV) {
   return 4u * (size_t)nh * (rV + 2) * (size_t)((splits + 3) & ~3);
 }
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+
+// Per (device, stream): whether the library's last launch there was a compress whose length
+// kernel lets its dependent start early.  A compress marks its stream; a decode reads and
+// clears the mark (it then requests no cache tile before its dependency wait); the joint
+// compress, whose kernels do not let dependents start early, clears it.  Host only.
+void mark_stream_compress(int device, cudaStream_t s, bool marked);
+bool take_stream_compress_mark(int device, cudaStream_t s);
 
 // Tokens per tile: 64 for small ranks (an SM sustains a roughly fixed number of tiles per
 // microsecond, so small tiles would leave the memory system idle), 32 otherwise.

@@ -101,7 +101,12 @@ typedef enum stief_status {
  * launched as a programmatic dependent of the preceding work in the stream and
  * stages P_K and P_V before waiting for it: the bases must not be written by the
  * kernel that immediately precedes the call if that kernel lets its dependents
- * start early (this library's kernels never write the bases).
+ * start early (this library's kernels never write the bases).  The call ends with
+ * a small kernel that advances the lengths once every projection CTA has read
+ * them; it lets the next kernel in the stream start early (that kernel's inputs
+ * are read after its own dependency wait).  The library notes per stream that its
+ * last launch there was a compress, and the decode call that follows requests no
+ * cache row before its wait.
  * Returns STIEF_OK or an argument error (nothing launched).
  */
 STIEF_API stief_status stief_compress_append(const uint16_t* k_new, const uint16_t* v_new,
@@ -200,8 +205,9 @@ STIEF_API size_t stief_decode_workspace_bytes(int B, int Hq, int Hkv, int rV, in
  * dependent launch), it must write neither P_K nor any row of k_lat or v_lat
  * below seq_lens[b] - 1; the row just below each length is read again after the
  * wait, so stief_append_decode calls may follow one another on the same caches.
- * This library's kernels never write the bases, and its compress calls end with a
- * kernel that lets no dependent start early.  The rule on P_K holds for every call
+ * This library's kernels never write the bases, and a decode call issued right after
+ * one of its compress calls in the same stream reads no cache row before the wait
+ * (the library keeps that note per stream).  The rule on P_K holds for every call
  * that takes it (stief_append_decode and the _noalloc, _paged and _q8 decodes);
  * the rule on the cache rows for stief_append_decode, stief_decode_latent and
  * stief_decode_attention_noalloc (the _paged, _q8 and _joint_v calls read no cache

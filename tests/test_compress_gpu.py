@@ -188,3 +188,46 @@ def test_prefill_chunk_full_size():
     for h in range(Hkv):
         assert _check_latent(gk[0, h], f64(k_new[0, h]), f64(P_K[h])) > 0.98
         assert _check_latent(gv[0, h], f64(v_new[0, h]), f64(P_V[h])) > 0.98
+
+
+@pytest.mark.parametrize("rK,rV", [(64, 64), (32, 48)])
+def test_decode_right_after_compress_same_stream(rK, rV):
+    """Compress chunks (tensor-core and CUDA-core paths) and decodes issued back to back on one
+    stream with no host synchronisation and no other work in between.  The compress call's
+    length kernel lets the next kernel start early, so the decode that follows must request no
+    cache row before its dependency wait: the caches start as NaN, so a row read before the
+    compress wrote it would show in the output."""
+    B, Hq, Hkv, d, L_max = 2, 16, 4, 128, 2048
+    seed = 91
+    dev = torch.device("cuda")
+    chunks = [640, 300, 1, 128, 7, 900]
+    P_K, P_V = si.bases_bf16(seed, Hkv, d, rK, rV)
+    gPK, gPV = P_K.to(dev), P_V.to(dev)
+    gk = torch.full((B, Hkv, L_max, rK), float("nan"), dtype=torch.bfloat16, device=dev)
+    gv = torch.full((B, Hkv, L_max, rV), float("nan"), dtype=torch.bfloat16, device=dev)
+    glens = torch.zeros(B, dtype=torch.int32, device=dev)
+    news = [si.full_kv(seed + i, B, Hkv, T, d) for i, T in enumerate(chunks)]
+    gnews = [(k.to(dev), v.to(dev)) for k, v in news]
+    qs = [si.queries(seed + 50 + i, B, Hq, d) for i in range(len(chunks))]
+    gqs = [q.to(dev) for q in qs]
+    outs = [torch.empty((B, Hq, d), dtype=torch.bfloat16, device=dev) for _ in chunks]
+    max_seq = sum(chunks)
+    ws = stief.workspace_for(B, Hq, Hkv, rV, max_seq)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    torch.cuda.synchronize()
+    for i in range(len(chunks)):
+        stief.stief_compress_append(gnews[i][0], gnews[i][1], gPK, gPV, gk, gv, glens,
+                                    dev_status=status)
+        stief.stief_decode_attention(gqs[i], gPK, gPV, gk, gv, glens, outs[i], ws, max_seq,
+                                     dev_status=status)
+    assert stief.stief_read_device_status(status) == 0
+    ok_lat = np.zeros((B, Hkv, L_max, rK))
+    ov_lat = np.zeros((B, Hkv, L_max, rV))
+    olens = np.zeros(B, np.int32)
+    for i in range(len(chunks)):
+        ok_lat, ov_lat, olens, nbad = oracle.compress_append(
+            f64(news[i][0]), f64(news[i][1]), f64(P_K), f64(P_V), ok_lat, ov_lat, olens)
+        assert nbad == 0
+        want = oracle.decode(f64(qs[i]), f64(P_K), f64(P_V), ok_lat, ov_lat, olens)
+        assert_decode_close(outs[i].cpu(), want)
+    assert glens.cpu().numpy().tolist() == olens.tolist() == [max_seq] * B
