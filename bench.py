@@ -642,9 +642,8 @@ def run_gpu(args, w: si.Workload):
             "peak_kind": f"{peak_kind} hbm_gbs (copy bandwidth, burst)",
             "unit": "GB/s",
             "frac": round(achieved / peak, 4),
-            "traffic": (None if (args.latent or args.unfused or args.int8 or args.paged
-                                 or args.joint)
-                        else _traffic_per_launch(w.name)),
+            "traffic": (None if (args.latent or args.unfused or args.paged or args.joint)
+                        else _traffic_per_launch(w.name + ("/int8" if args.int8 else ""))),
             "algorithmic_bytes": bytes_per_dec,
             "decode_us": round(dec_us, 3),
             "decode_timing": f"{dec_reps} replays of a graph of {n_dec} back-to-back decode "
@@ -921,9 +920,20 @@ def run_profile_launches(args, w: si.Workload):
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     q_lat = torch.randn((w.B, w.Hq, lay.rK), generator=g, device=dev).to(torch.bfloat16)
     o_lat = torch.empty((w.B, w.Hq, lay.rV), dtype=torch.bfloat16, device=dev)
+    if args.int8:  # int8 codes and row scales of layer 0 (synthetic values), L_max % 64 == 0
+        L8 = (L_max + 63) // 64 * 64
+        kq = torch.randint(-127, 128, (w.B, w.Hkv, L8, lay.rK), generator=g, device=dev, dtype=torch.int8)
+        vq = torch.randint(-127, 128, (w.B, w.Hkv, L8, lay.rV), generator=g, device=dev, dtype=torch.int8)
+        ks = torch.rand((w.B, w.Hkv, L8), generator=g, device=dev) * 0.02
+        vs = torch.rand((w.B, w.Hkv, L8), generator=g, device=dev) * 0.02
     for _ in range(args.profile_launches):
         lay.seq_lens.fill_(w.L - 1)
-        if args.latent:
+        if args.int8:
+            lay.seq_lens.fill_(w.L)
+            stief.stief_decode_attention_q8(q, lay.P_K, lay.P_V, kq, vq, ks, vs, lay.seq_lens, out,
+                                            lay.ws, max_seq_len=L_max, num_splits=args.splits,
+                                            dev_status=status)
+        elif args.latent:
             lay.seq_lens.fill_(w.L)
             stief.stief_decode_latent(q_lat, lay.k_lat, lay.v_lat, lay.seq_lens, o_lat, lay.ws,
                                       max_seq_len=L_max, num_splits=args.splits,
