@@ -197,10 +197,15 @@ def build_state(w: si.Workload, total_steps: int, seed: int, dev):
     return layers, L_max
 
 
+def _int4(args) -> bool:
+    """The 4-bit form of the int8 mode (argument namespaces built elsewhere may lack the flag)."""
+    return bool(getattr(args, "int4", False))
+
+
 def step_call(args) -> str:
     """The API call whose kernel a step of the chosen mode runs (one per layer)."""
     if args.int8:
-        return "stief_decode_attention_q8"
+        return "stief_decode_attention_q4" if _int4(args) else "stief_decode_attention_q8"
     if args.joint:
         return "stief_decode_latent_joint_v" if args.latent else "stief_decode_attention_joint_v"
     if args.latent:
@@ -210,10 +215,12 @@ def step_call(args) -> str:
     return "stief_decode_attention" if args.unfused else "stief_append_decode"
 
 
-def row_bytes_fn(w: si.Workload, int8: bool = False, joint: bool = False):
+def row_bytes_fn(w: si.Workload, int8: bool = False, joint: bool = False, int4: bool = False):
     """Cache bytes per (token, sequence, KV head) for a layer of ranks (rK, rV): bf16 rows, int8
-    rows with their two fp32 scales, or per-head keys with one joint value row shared by the
-    Hkv heads (its bytes split over them)."""
+    or 4-bit rows with their two fp32 scales, or per-head keys with one joint value row shared
+    by the Hkv heads (its bytes split over them)."""
+    if int4:
+        return lambda rK, rV: (rK + rV) // 2 + 8
     if int8:
         return lambda rK, rV: rK + rV + 8
     if joint:
@@ -221,12 +228,12 @@ def row_bytes_fn(w: si.Workload, int8: bool = False, joint: bool = False):
     return lambda rK, rV: 2 * (rK + rV)
 
 
-def replica_count(w: si.Workload, int8: bool = False, joint: bool = False) -> int:
+def replica_count(w: si.Workload, int8: bool = False, joint: bool = False, int4: bool = False) -> int:
     """Copies of the workload's layer state that consecutive timed steps rotate over, so that
     the inputs of a step were last touched at least ROTATE_BYTES of cache reads earlier
     (more than 3x the 126 MB L2: every step streams its cache from HBM, and no flush is
     needed between steps)."""
-    rb = row_bytes_fn(w, int8, joint)
+    rb = row_bytes_fn(w, int8, joint, int4)
     per = int(sum(rb(rK, rV) * w.B * w.Hkv * w.L for rK, rV in w.layer_ranks()))
     return 1 if per >= ROTATE_BYTES else min(MAX_REPLICAS, -(-ROTATE_BYTES // per))
 
@@ -234,8 +241,9 @@ def replica_count(w: si.Workload, int8: bool = False, joint: bool = False) -> in
 def step_description(args) -> str:
     """What one timed step runs, in words (the same text in both arms)."""
     if args.int8:
-        what = ("decode over an int8 latent cache (codes + fp32 row scales, synthetic values), "
-                "no append, every layer; ")
+        what = (("decode over a 4-bit latent cache (two codes per byte + fp32 row scales"
+                 if _int4(args) else "decode over an int8 latent cache (codes + fp32 row scales")
+                + ", synthetic values), no append, every layer; ")
     elif args.joint:
         what = ("decode with per-head keys and one joint value latent per token shared by the "
                 "KV heads" + (" (latent output)" if args.latent else "") + ", no append, every "
@@ -258,8 +266,8 @@ def step_description(args) -> str:
 
 def config_dict(w: si.Workload, args, world: int) -> dict:
     """The workload and how it is run: identical in the GPU arm and the reference arm."""
-    R = replica_count(w, args.int8, args.joint)
-    rb = row_bytes_fn(w, args.int8, args.joint)
+    R = replica_count(w, args.int8, args.joint, _int4(args))
+    rb = row_bytes_fn(w, args.int8, args.joint, _int4(args))
     rot_mb = R * sum(rb(rK, rV) * w.B * w.Hkv * w.L for rK, rV in w.layer_ranks()) / 2**20
     appends = not (args.latent or args.int8 or args.joint)
     ranks = [list(r) for r in w.layer_ranks()]
@@ -313,7 +321,7 @@ def run_gpu(args, w: si.Workload):
                                              device_id=dev)
     seed = rank_seed(w.seed, rank)
     W, K = args.warmup, args.steps
-    R = replica_count(w, args.int8, args.joint)
+    R = replica_count(w, args.int8, args.joint, _int4(args))
     reps = []
     for r in range(R):
         # room for every append of the warm-up, timed and kernel-timing runs of a replica
@@ -348,10 +356,16 @@ def run_gpu(args, w: si.Workload):
         for lays in reps:
             for lay in lays:
                 L8 = (L_max + 63) // 64 * 64
-                lay.kq = torch.randint(-127, 128, (w.B, w.Hkv, L8, lay.rK), generator=g,
-                                       device=dev, dtype=torch.int8)
-                lay.vq = torch.randint(-127, 128, (w.B, w.Hkv, L8, lay.rV), generator=g,
-                                       device=dev, dtype=torch.int8)
+                if _int4(args):  # two 4-bit codes per byte: any byte is a valid pair
+                    lay.kq = torch.randint(0, 256, (w.B, w.Hkv, L8, lay.rK // 2), generator=g,
+                                           device=dev, dtype=torch.uint8)
+                    lay.vq = torch.randint(0, 256, (w.B, w.Hkv, L8, lay.rV // 2), generator=g,
+                                           device=dev, dtype=torch.uint8)
+                else:
+                    lay.kq = torch.randint(-127, 128, (w.B, w.Hkv, L8, lay.rK), generator=g,
+                                           device=dev, dtype=torch.int8)
+                    lay.vq = torch.randint(-127, 128, (w.B, w.Hkv, L8, lay.rV), generator=g,
+                                           device=dev, dtype=torch.int8)
                 lay.ks = torch.rand((w.B, w.Hkv, L8), generator=g, device=dev) * 0.02
                 lay.vs = torch.rand((w.B, w.Hkv, L8), generator=g, device=dev) * 0.02
                 lay.k_lat = lay.v_lat = None  # the bf16 caches are not used
@@ -387,8 +401,8 @@ def run_gpu(args, w: si.Workload):
         olat = []
 
     def layer_step(li, lay):
-        if args.int8:  # decode over the int8 cache (no append)
-            stief.stief_decode_attention_q8(q_s, lay.P_K, lay.P_V, lay.kq, lay.vq, lay.ks, lay.vs,
+        if args.int8:  # decode over the int8 (or 4-bit) cache (no append)
+            (stief.stief_decode_attention_q4 if _int4(args) else stief.stief_decode_attention_q8)(q_s, lay.P_K, lay.P_V, lay.kq, lay.vq, lay.ks, lay.vs,
                                             lay.seq_lens, out[li], lay.ws, max_seq_len=L_max,
                                             num_splits=args.splits, dev_status=status)
         elif args.latent and args.joint:  # latent output over the joint value latent
@@ -613,7 +627,7 @@ def run_gpu(args, w: si.Workload):
     # ---- numbers
     value = job_tokens_per_s(w.B, ws_n, ms_per_step)
     lay0 = layers[0]
-    row_bytes = row_bytes_fn(w, args.int8, args.joint)
+    row_bytes = row_bytes_fn(w, args.int8, args.joint, _int4(args))
     bytes_per_dec = int(row_bytes(lay0.rK, lay0.rV) * w.B * w.Hkv * L_dec_mean)
     achieved = bytes_per_dec / (dec_us / 1e6) / 1e9
     peak, peak_kind = _hbm_peak()
@@ -630,7 +644,7 @@ def run_gpu(args, w: si.Workload):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "int8" if args.int8 else "bf16",
+        "dtype": ("int4" if _int4(args) else "int8") if args.int8 else "bf16",
         "data": "synthetic",
         "config": config_dict(w, args, ws_n),
         "hbm_gbs_step": round(step_bytes / (ms_per_step / 1e3) / 1e9, 1),
@@ -643,7 +657,8 @@ def run_gpu(args, w: si.Workload):
             "unit": "GB/s",
             "frac": round(achieved / peak, 4),
             "traffic": (None if (args.latent or args.unfused or args.paged or args.joint)
-                        else _traffic_per_launch(w.name + ("/int8" if args.int8 else ""))),
+                        else _traffic_per_launch(w.name + (("/int4" if _int4(args) else "/int8")
+                                                           if args.int8 else ""))),
             "algorithmic_bytes": bytes_per_dec,
             "decode_us": round(dec_us, 3),
             "decode_timing": f"{dec_reps} replays of a graph of {n_dec} back-to-back decode "
@@ -920,17 +935,21 @@ def run_profile_launches(args, w: si.Workload):
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     q_lat = torch.randn((w.B, w.Hq, lay.rK), generator=g, device=dev).to(torch.bfloat16)
     o_lat = torch.empty((w.B, w.Hq, lay.rV), dtype=torch.bfloat16, device=dev)
-    if args.int8:  # int8 codes and row scales of layer 0 (synthetic values), L_max % 64 == 0
+    if args.int8:  # int8 (4-bit) codes and row scales of layer 0 (synthetic), L_max % 64 == 0
         L8 = (L_max + 63) // 64 * 64
-        kq = torch.randint(-127, 128, (w.B, w.Hkv, L8, lay.rK), generator=g, device=dev, dtype=torch.int8)
-        vq = torch.randint(-127, 128, (w.B, w.Hkv, L8, lay.rV), generator=g, device=dev, dtype=torch.int8)
+        if _int4(args):
+            kq = torch.randint(0, 256, (w.B, w.Hkv, L8, lay.rK // 2), generator=g, device=dev, dtype=torch.uint8)
+            vq = torch.randint(0, 256, (w.B, w.Hkv, L8, lay.rV // 2), generator=g, device=dev, dtype=torch.uint8)
+        else:
+            kq = torch.randint(-127, 128, (w.B, w.Hkv, L8, lay.rK), generator=g, device=dev, dtype=torch.int8)
+            vq = torch.randint(-127, 128, (w.B, w.Hkv, L8, lay.rV), generator=g, device=dev, dtype=torch.int8)
         ks = torch.rand((w.B, w.Hkv, L8), generator=g, device=dev) * 0.02
         vs = torch.rand((w.B, w.Hkv, L8), generator=g, device=dev) * 0.02
     for _ in range(args.profile_launches):
         lay.seq_lens.fill_(w.L - 1)
         if args.int8:
             lay.seq_lens.fill_(w.L)
-            stief.stief_decode_attention_q8(q, lay.P_K, lay.P_V, kq, vq, ks, vs, lay.seq_lens, out,
+            (stief.stief_decode_attention_q4 if _int4(args) else stief.stief_decode_attention_q8)(q, lay.P_K, lay.P_V, kq, vq, ks, vs, lay.seq_lens, out,
                                             lay.ws, max_seq_len=L_max, num_splits=args.splits,
                                             dev_status=status)
         elif args.latent:
@@ -1017,6 +1036,9 @@ def main():
                     help="diagnostics: run only the first N layers of the workload")
     ap.add_argument("--splits", type=int, default=0,
                     help="diagnostics: force the decode split count (0 = automatic)")
+    ap.add_argument("--int4", action="store_true",
+                    help="time stief_decode_attention_q4 over a 4-bit latent cache (no append; "
+                         "ranks multiples of 32)")
     ap.add_argument("--int8", action="store_true",
                     help="time stief_decode_attention_q8 over an int8 latent cache (no append)")
     ap.add_argument("--latent", action="store_true",
@@ -1049,13 +1071,17 @@ def main():
         ap.error(f"--gpus {args.gpus} but WORLD_SIZE={env_world}: run N ranks with --gpus N")
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    modes = [m for m in ("int8", "latent", "paged", "joint", "unfused") if getattr(args, m)]
+    modes = [m for m in ("int8", "int4", "latent", "paged", "joint", "unfused") if getattr(args, m)]
     if len(modes) > 1 and modes != ["latent", "joint"]:
-        ap.error("--int8, --latent, --paged, --joint and --unfused are separate modes "
+        ap.error("--int8, --int4, --latent, --paged, --joint and --unfused are separate modes "
                  "(--latent --joint together time the latent joint-value decode)")
     if (args.paged or args.joint) and args.profile_launches > 0:
         ap.error("--profile-launches has no paged or joint mode")
     w = si.WORKLOADS[args.workload]
+    if args.int4:
+        if any(rK % 32 or rV % 32 for rK, rV in w.layer_ranks()):
+            ap.error(f"--int4 needs ranks that are multiples of 32; {w.name} has {w.layer_ranks()}")
+        args.int8 = True  # the 4-bit form runs the int8 mode's step with 4-bit codes
     if args.layers > 0:
         import dataclasses
         w = dataclasses.replace(w, layers=min(args.layers, w.layers),

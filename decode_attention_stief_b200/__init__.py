@@ -21,6 +21,8 @@ from ._binding import (  # noqa: F401
     stief_compress_append_paged,
     stief_decode_attention,
     stief_decode_attention_q8,
+    stief_compress_append_q4,
+    stief_decode_attention_q4,
     stief_decode_attention_joint_v,
     stief_decode_attention_paged,
     stief_decode_attention_noalloc,

@@ -89,6 +89,11 @@ def library() -> ctypes.CDLL:
             lib.stief_decode_attention_q8.restype = _i
             lib.stief_decode_attention_q8.argtypes = ([vp] * 10 + [ctypes.c_size_t] + [_i] * 9
                                                       + [vp, vp])
+            lib.stief_compress_append_q4.restype = _i
+            lib.stief_compress_append_q4.argtypes = [vp] * 9 + [_i] * 7 + [vp, vp]
+            lib.stief_decode_attention_q4.restype = _i
+            lib.stief_decode_attention_q4.argtypes = ([vp] * 10 + [ctypes.c_size_t] + [_i] * 9
+                                                      + [vp, vp])
             lib.stief_compress_append_joint_v.restype = _i
             lib.stief_compress_append_joint_v.argtypes = [vp] * 7 + [_i] * 7 + [vp, vp]
             lib.stief_decode_attention_joint_v.restype = _i
@@ -437,6 +442,68 @@ def stief_decode_attention_q8(q, P_K, P_V, k_q, v_q, k_s, v_s, seq_lens, out, wo
                                                rV, L_max, int(max_seq_len), int(num_splits),
                                                _opt_status(dev_status), _stream_ptr(stream))
     _check("stief_decode_attention_q8", code)
+    return out
+
+
+def stief_compress_append_q4(k_new, v_new, P_K, P_V, k_q, v_q, k_s, v_s, seq_lens,
+                             dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """stief_compress_append into a 4-bit cache: codes k_q [B][Hkv][L_max][rK / 2] (uint8, two
+    per byte) and row scales k_s [B][Hkv][L_max] (float32), likewise v_q, v_s; ranks multiples
+    of 32, L_max a multiple of 64."""
+    pk = _dev(k_new, "k_new", torch.bfloat16, 4)
+    pv = _dev(v_new, "v_new", torch.bfloat16, 4)
+    ppk = _dev(P_K, "P_K", torch.bfloat16, 3)
+    ppv = _dev(P_V, "P_V", torch.bfloat16, 3)
+    pkq = _dev(k_q, "k_q", torch.uint8, 4)
+    pvq = _dev(v_q, "v_q", torch.uint8, 4)
+    pks = _dev(k_s, "k_s", torch.float32, 3)
+    pvs = _dev(v_s, "v_s", torch.float32, 3)
+    psl = _dev(seq_lens, "seq_lens", torch.int32, 1)
+    B, Hkv, T, d = k_new.shape
+    rK, rV = P_K.shape[2], P_V.shape[2]
+    L_max = k_q.shape[2]
+    if tuple(v_new.shape) != (B, Hkv, T, d) or tuple(P_K.shape) != (Hkv, d, rK) \
+            or tuple(P_V.shape) != (Hkv, d, rV) or tuple(k_q.shape) != (B, Hkv, L_max, rK // 2) \
+            or tuple(v_q.shape) != (B, Hkv, L_max, rV // 2) or tuple(k_s.shape) != (B, Hkv, L_max) \
+            or tuple(v_s.shape) != (B, Hkv, L_max) or seq_lens.shape[0] != B:
+        raise ValueError("stief_compress_append_q4: inconsistent shapes")
+    code = library().stief_compress_append_q4(pk, pv, ppk, ppv, pkq, pvq, pks, pvs, psl, B, Hkv, T,
+                                              d, rK, rV, L_max, _opt_status(dev_status),
+                                              _stream_ptr(stream))
+    _check("stief_compress_append_q4", code)
+
+
+def stief_decode_attention_q4(q, P_K, P_V, k_q, v_q, k_s, v_s, seq_lens, out, workspace,
+                              max_seq_len: int, num_splits: int = 0,
+                              dev_status: Optional[torch.Tensor] = None, stream=None):
+    """stief_decode_attention over a 4-bit cache (codes and row scales as for
+    stief_compress_append_q4)."""
+    pq = _dev(q, "q", torch.bfloat16, 3)
+    ppk = _dev(P_K, "P_K", torch.bfloat16, 3)
+    ppv = _dev(P_V, "P_V", torch.bfloat16, 3)
+    pkq = _dev(k_q, "k_q", torch.uint8, 4)
+    pvq = _dev(v_q, "v_q", torch.uint8, 4)
+    pks = _dev(k_s, "k_s", torch.float32, 3)
+    pvs = _dev(v_s, "v_s", torch.float32, 3)
+    psl = _dev(seq_lens, "seq_lens", torch.int32, 1)
+    po = _dev(out, "out", torch.bfloat16, 3)
+    B, Hq, d = q.shape
+    Hkv, _, rK = P_K.shape
+    rV = P_V.shape[2]
+    L_max = k_q.shape[2]
+    if tuple(P_V.shape) != (Hkv, d, rV) or tuple(k_q.shape) != (B, Hkv, L_max, rK // 2) \
+            or tuple(v_q.shape) != (B, Hkv, L_max, rV // 2) or tuple(k_s.shape) != (B, Hkv, L_max) \
+            or tuple(v_s.shape) != (B, Hkv, L_max) or seq_lens.shape[0] != B \
+            or tuple(out.shape) != (B, Hq, d):
+        raise ValueError("stief_decode_attention_q4: inconsistent shapes")
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    code = library().stief_decode_attention_q4(pq, ppk, ppv, pkq, pvq, pks, pvs, psl, po,
+                                               workspace.data_ptr(), ws_bytes, B, Hq, Hkv, d, rK,
+                                               rV, L_max, int(max_seq_len), int(num_splits),
+                                               _opt_status(dev_status), _stream_ptr(stream))
+    _check("stief_decode_attention_q4", code)
     return out
 
 

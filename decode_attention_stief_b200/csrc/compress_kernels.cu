@@ -114,16 +114,25 @@ __global__ void __launch_bounds__(kSmallThreads) stief_compress_rows_kernel(cons
       lat[cache_row(cr, b, h, Lb + r0 + t) * pairs + c2] = pack_bf16x2_rn(sum.x, sum.y);
   }
   if (q8) {
-    // int8 cache: a thread per row: one fp32 scale (max / 127) and RNE codes
+    // int8 / 4-bit cache: a thread per row: one fp32 scale (max / 127, or max / 7) and RNE
+    // codes; 4-bit codes two per byte, column 2 j in the low nibble of byte j
     __syncthreads();
     if (tid < nrows) {
       const float* row = reinterpret_cast<const float*>(red + tid * pairs);
+      const int qmax = a.q4 ? 7 : 127;
       float amax = 0.f;
       for (int c = 0; c < r; ++c) amax = fmaxf(amax, fabsf(row[c]));
-      const float scale = __fdiv_rn(amax, 127.f);
+      const float scale = __fdiv_rn(amax, (float)qmax);
       const long long crow = cache_row(cr, b, h, Lb + r0 + tid);
-      int8_t* dst = reinterpret_cast<int8_t*>(is_v ? a.v_lat : a.k_lat) + crow * r;
-      for (int c = 0; c < r; ++c) dst[c] = (int8_t)quantize_code(row[c], scale);
+      if (a.q4) {
+        uint8_t* dst = reinterpret_cast<uint8_t*>(is_v ? a.v_lat : a.k_lat) + crow * (r / 2);
+        for (int c = 0; c < r; c += 2)
+          dst[c / 2] = (uint8_t)((quantize_code(row[c], scale, 7) & 0xF) |
+                                 ((quantize_code(row[c + 1], scale, 7) & 0xF) << 4));
+      } else {
+        int8_t* dst = reinterpret_cast<int8_t*>(is_v ? a.v_lat : a.k_lat) + crow * r;
+        for (int c = 0; c < r; ++c) dst[c] = (int8_t)quantize_code(row[c], scale);
+      }
       (is_v ? a.v_scale : a.k_scale)[crow] = scale;
     }
   }

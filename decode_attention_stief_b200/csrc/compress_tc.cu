@@ -272,10 +272,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const long long crow = live ? cache_row(cr, b, h, Lb + m0 + row) : 0;  // mapped (checked)
     const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     if (a.k_scale != nullptr) {
-      // int8 cache: the row rounded to bf16, then one fp32 scale (max / 127) and RNE codes,
-      // divisions in IEEE fp32; the accumulators are read twice (maximum, then codes)
+      // int8 / 4-bit cache: the row rounded to bf16, then one fp32 scale (max / 127, or max / 7)
+      // and RNE codes, divisions in IEEE fp32; the accumulators are read twice (maximum, then
+      // codes).  4-bit codes go two per byte, column 2 j in the low nibble of byte j.
       const int r = which ? rV : rK;
       const uint32_t col0 = which ? 128u : 0u;
+      const int qmax = a.q4 ? 7 : 127;
       float amax = 0.f;
       for (int c0 = 0; c0 < r; c0 += 16) {
         uint32_t v[16];
@@ -284,23 +286,34 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
         for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(bf16_round(__uint_as_float(v[e]))));
       }
-      const float scale = __fdiv_rn(amax, 127.f);
-      int8_t* dst = reinterpret_cast<int8_t*>(which ? a.v_lat : a.k_lat) + crow * r;
+      const float scale = __fdiv_rn(amax, (float)qmax);
+      uint8_t* dst = reinterpret_cast<uint8_t*>(which ? a.v_lat : a.k_lat) + crow * (a.q4 ? r / 2 : r);
       for (int c0 = 0; c0 < r; c0 += 16) {
         uint32_t v[16];
         tmem_ld16(lane_base + col0 + (uint32_t)c0, v);
         tmem_wait_ld();
-        uint32_t packed[4];
+        int code[16];
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          uint32_t word = 0u;
+        for (int e = 0; e < 16; ++e) code[e] = quantize_code(bf16_round(__uint_as_float(v[e])), scale, qmax);
+        if (a.q4) {
+          uint32_t w0 = 0u, w1 = 0u;
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            word |= (uint32_t)(uint8_t)quantize_code(bf16_round(__uint_as_float(v[4 * g + e])), scale)
-                    << (8 * e);
-          packed[g] = word;
+          for (int e = 0; e < 8; ++e) {
+            w0 |= (uint32_t)(code[e] & 0xF) << (4 * e);
+            w1 |= (uint32_t)(code[8 + e] & 0xF) << (4 * e);
+          }
+          if (live) *reinterpret_cast<uint2*>(dst + c0 / 2) = make_uint2(w0, w1);
+        } else {
+          uint32_t packed[4];
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            uint32_t word = 0u;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) word |= (uint32_t)(uint8_t)code[4 * g + e] << (8 * e);
+            packed[g] = word;
+          }
+          if (live) *reinterpret_cast<uint4*>(dst + c0) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
         }
-        if (live) *reinterpret_cast<uint4*>(dst + c0) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
       }
       if (live) (which ? a.v_scale : a.k_scale)[crow] = scale;
     }

@@ -163,6 +163,11 @@ __device__ __forceinline__ void mma_i8_k16(int (&c)[4], uint32_t a0, uint32_t a1
         : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
         : "r"(a0), "r"(a1), "r"(b0));
 }
+// 4-bit codes, two per byte (low nibble first): each byte's low / high nibble moved to the top
+// of the byte, i.e. 16 x the signed code, as four s8 lanes.
+__device__ __forceinline__ uint32_t nib_lo(uint32_t p) { return (p << 4) & 0xF0F0F0F0u; }
+__device__ __forceinline__ uint32_t nib_hi(uint32_t p) { return p & 0xF0F0F0F0u; }
+
 __device__ __forceinline__ float rcp_approx(float x) {
   float y;
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -294,8 +299,9 @@ struct DecodeSmem {
   int xs;  // row stride of qt in floats
 };
 
+// `code`: the cache form, 0 bf16 rows, 1 int8 codes (r bytes per row), 2 4-bit codes (r / 2).
 __host__ __device__ inline DecodeSmem decode_smem_layout(int NW, int ns, int rK, int rV, int tile,
-                                                          bool q8 = false) {
+                                                          int code = 0) {
   DecodeSmem s;
   const int rmax = rK > rV ? rK : rV;
   uint32_t off = 0;
@@ -315,9 +321,11 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int NW, int ns, int rK,
   s.pmat = off;
   off += 256u * rmax;  // d = 128 rows x r bf16
   s.region = off;
-  if (q8) {
-    s.q8_v = align_up((uint32_t)tile * rK, 1024);  // the swizzle patterns need 1 KiB alignment
-    s.stage = align_up(s.q8_v + (uint32_t)tile * rV, 1024);
+  if (code) {
+    const uint32_t kb = code == 1 ? (uint32_t)rK : (uint32_t)rK / 2u;  // code bytes per row
+    const uint32_t vb = code == 1 ? (uint32_t)rV : (uint32_t)rV / 2u;
+    s.q8_v = align_up((uint32_t)tile * kb, 1024);  // the swizzle patterns need 1 KiB alignment
+    s.stage = align_up(s.q8_v + (uint32_t)tile * vb, 1024);
   } else {
     s.q8_v = 0;
     s.stage = (uint32_t)tile * (rK + rV) * 2u;  // a multiple of 1 KiB
@@ -338,13 +346,14 @@ constexpr int kMaxConsumerWarps = 8;
 // joint value latents (one value row per token shared by the KV heads; full or latent output).
 // Each is its own instantiation, so a mode's branches cost the others nothing.
 constexpr int kModePlain = 0, kModeLatent = 1, kModePaged = 2, kModeQ8 = 3, kModeJointV = 4,
-              kModeLatentJointV = 5;
+              kModeLatentJointV = 5, kModeQ4 = 6;
 
 template <int NB, int NKS, int NMV, int TT, int MODE>
 __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
     stief_decode_kernel(const __grid_constant__ DecodeArgs a) {
   constexpr bool LAT = MODE == kModeLatent || MODE == kModeLatentJointV;
-  constexpr bool PG = MODE == kModePaged, Q8 = MODE == kModeQ8;
+  constexpr bool PG = MODE == kModePaged, Q8 = MODE == kModeQ8, Q4 = MODE == kModeQ4;
+  constexpr bool QI = Q8 || Q4;  // integer codes with row scales
   constexpr bool JV = MODE == kModeJointV || MODE == kModeLatentJointV;
   constexpr int kTile = TT;
   constexpr int MT = TT / 16;              // 16-token m-tiles (scores) / k-steps (mix) per tile
@@ -372,7 +381,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
   const CacheRows cr{PG ? a.block_table : nullptr, a.max_pages, a.page_size, a.num_pages, a.Hkv,
                      a.L_max};
 
-  const DecodeSmem L = decode_smem_layout(NW, ns, rK, rV, TT, Q8);
+  const DecodeSmem L = decode_smem_layout(NW, ns, rK, rV, TT, Q8 ? 1 : Q4 ? 2 : 0);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);  // [NW][ns]: tile landed
   uint64_t* empty = full + NW * ns;                             // [NW][ns]: tile consumed
   uint64_t* setup_bar = empty + NW * ns;  // phase 0: q and P_K, phase 1: P_V
@@ -384,8 +393,10 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
   const int xs = L.xs;
   uint8_t* pmat = smem + L.pmat;
   // a stage: the key tile, then the value tile at kt_bytes
-  const uint32_t kt_bytes = Q8 ? L.q8_v : (uint32_t)kTile * rK * 2u;
-  const uint32_t st_bytes = Q8 ? (uint32_t)kTile * (rK + rV) : kt_bytes + (uint32_t)kTile * rV * 2u;
+  const uint32_t kt_bytes = QI ? L.q8_v : (uint32_t)kTile * rK * 2u;
+  const uint32_t st_bytes = Q8   ? (uint32_t)kTile * (rK + rV)
+                            : Q4 ? (uint32_t)kTile * (rK + rV) / 2u
+                                 : kt_bytes + (uint32_t)kTile * rV * 2u;
 
   // the swizzle patterns assume 1 KiB-aligned tiles
   if (((smem_u32(smem + L.pmat) | smem_u32(smem + L.region)) & 1023u) != 0) {
@@ -550,7 +561,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
   // int8 caches: the row scales of a tile come by coalesced loads, requested one tile ahead
   // (a TMA or bulk copy per tile costs more than its bytes): lane i holds the scales of
   // tokens i + 32 j of the tile.  The first tile's are requested before the setup wait.
-  constexpr int SJ = Q8 ? TT / 32 : 1;
+  constexpr int SJ = QI ? TT / 32 : 1;
   float skc[SJ], svc[SJ], skn[SJ], svn[SJ];
   auto load_scales = [&](int kk) {
     if (kk < warp_tiles(warp, n_tiles)) {
@@ -602,7 +613,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
     // q~ = q P_K on the MMA: q~^T[j][head] = sum_i P_K[i][j] q[head][i]
     // (M = the r_K columns of P_K, N = 8 heads, K = d), scaled into log2 units
     const int n = lane >> 2;  // B column = head
-    if constexpr (Q8) load_scales(0);
+    if constexpr (QI) load_scales(0);
     ok = warp_wait(setup_bar, 0, a.dev_status);
     if (!ok && lane == 0) flag[1] = 1;
     uint32_t qb[8][2];  // d / 16 k-steps (explicit shared loads issued together)
@@ -782,15 +793,15 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
     // ---- consumers: stream the warp's tiles ------------------------------------------------
     const int my_tiles = warp_tiles(warp, n_tiles);
     uint8_t* ring = smem + L.region + (size_t)warp * ns * L.stage;
-    // int8 caches: a row's bytes are addressed as 16-bit columns (r / 2 of them); the scores
-    // take k-steps of 32 codes (the last one 16 when r_K % 32 == 16)
-    const int rKc = Q8 ? rK / 2 : rK, rVc = Q8 ? rV / 2 : rV;
+    // int8 / 4-bit caches: a row's bytes are addressed as 16-bit columns (r / 2 or r / 4 of
+    // them); the scores take k-steps of 32 codes (int8: the last one 16 when r_K % 32 == 16)
+    const int rKc = Q8 ? rK / 2 : Q4 ? rK / 4 : rK, rVc = Q8 ? rV / 2 : Q4 ? rV / 4 : rV;
     const int nks8 = (rK + 31) >> 5;
 
     uint32_t qf[NKS][NB][2];       // bf16 caches: B fragments of Q^T (hi / lo parts)
-    uint32_t qf8[NKS / 2][NB][2];  // int8 caches: the same as 8-bit parts
-    float sqA = 0.f, sqB = 0.f;    // int8 caches: fixed-point scales of q~ for heads hA, hA + 1
-    if constexpr (!Q8) {
+    uint32_t qf8[NKS / 2][NB][2];  // int8 / 4-bit caches: the same as 8-bit parts
+    float sqA = 0.f, sqB = 0.f;    // int8 / 4-bit caches: fixed-point scales of q~, heads hA, hA + 1
+    if constexpr (!QI) {
       float2 qx[NKS], qy[NKS];
 #pragma unroll
       for (int ks = 0; ks < NKS; ++ks)
@@ -807,7 +818,9 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
       // split as q16 = 256 hi + lo (hi in [-127, 127], lo in [-128, 127]), so that a score is
       // s_q k_scale (256 K.hi + K.lo) with both integer products exact.  B column n carries
       // part n >> 2 of head n & 3 (groups of up to 4) or, for groups of 8, n-tile 0 the hi and
-      // n-tile 1 the lo parts of head n.
+      // n-tile 1 the lo parts of head n.  4-bit caches: the key fragments carry 16 x the codes
+      // (s_q takes the 1/16) and their k order within a k-step is the nibble order: register 0
+      // slot i is column 8 (lane & 3) + 2 i, register 1 slot i column 8 (lane & 3) + 2 i + 1.
       const int n = lane >> 2;
       const int hcol = NB == 1 ? (n & 3) : n;
       const uint32_t qrow = smem_u32(qt) + 4u * (uint32_t)(hcol * xs);
@@ -816,7 +829,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
       amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
       amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
       const float inv = amax > 0.f ? 32512.f / amax : 0.f;  // absent heads are zero rows
-      const float sq = amax * (1.f / 32512.f);
+      const float sq = amax * (1.f / 32512.f) * (Q4 ? 0.0625f : 1.f);
       sqA = __shfl_sync(kFull, sq, 4 * hA);  // lanes 4 h .. 4 h + 3 hold column h: head h
       sqB = __shfl_sync(kFull, sq, 4 * (hA + 1));
       const bool part_lo = NB == 1 && (n >> 2) != 0;
@@ -824,11 +837,23 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
       for (int ks = 0; ks < NKS / 2; ++ks)
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-          const int k0 = 32 * ks + 16 * half + 4 * (lane & 3);
+          const int k0 = Q4 ? 32 * ks + 8 * (lane & 3) : 32 * ks + 16 * half + 4 * (lane & 3);
           uint32_t hb = 0u, lb = 0u;
           if (ks < nks8 && k0 < rK) {
-            const float4 x = lds128f(qrow + 4u * (uint32_t)k0);
-            const float xv[4] = {x.x, x.y, x.z, x.w};
+            float xv[4];
+            if constexpr (Q4) {
+              const float4 x0 = lds128f(qrow + 4u * (uint32_t)k0), x1 = lds128f(qrow + 4u * (uint32_t)(k0 + 4));
+              xv[0] = half ? x0.y : x0.x;
+              xv[1] = half ? x0.w : x0.z;
+              xv[2] = half ? x1.y : x1.x;
+              xv[3] = half ? x1.w : x1.z;
+            } else {
+              const float4 x = lds128f(qrow + 4u * (uint32_t)k0);
+              xv[0] = x.x;
+              xv[1] = x.y;
+              xv[2] = x.z;
+              xv[3] = x.w;
+            }
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const int q16 = __float2int_rn(xv[i] * inv);
@@ -846,20 +871,28 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
         }
     }
     // ldmatrix lane offsets.  Keys: the x4 (x2 for a 16-wide k-step) of m-tile 0 of each
-    // k-step, kstep bytes further per m-tile.  Values, bf16: the transposed x4 of each 16-dim
-    // m-tile over tokens 0-15, vstep further per 16 tokens; int8: the transposed x4 of rows
-    // (tokens) 0-31 of the m-tile's 16-byte column, vstep further per 32 tokens.
+    // k-step, kstep bytes further per m-tile (4-bit: the x4 of rows 0-31 of the k-step's
+    // 16-byte column, kstep further per 32 rows).  Values, bf16: the transposed x4 of each
+    // 16-dim m-tile over tokens 0-15, vstep further per 16 tokens; int8: the transposed x4 of
+    // rows (tokens) 0-31 of the m-tile's 16-byte column, vstep further per 32 tokens; 4-bit:
+    // the same per 16-byte column (32 dims, two m-tiles).
     uint32_t koff[NKS], kstep[NKS], voff[NMV], vstep[NMV];
 #pragma unroll
     for (int ks = 0; ks < NKS; ++ks) {
+      if (Q4) {
+        const PieceLoc pl = locate_i8(rKc, kTile, min(ks, rKc / 8 - 1));
+        koff[ks] = swz(pl, lane);
+        kstep[ks] = 64u * pl.w;
+        continue;
+      }
       const int ch = min(2 * ks + a_chunk(lane), rKc / 8 - 1);
-      const PieceLoc pl = Q8 ? locate_i8(rKc, kTile, ch) : locate(rKc, kTile, ch);
+      const PieceLoc pl = QI ? locate_i8(rKc, kTile, ch) : locate(rKc, kTile, ch);
       koff[ks] = swz(pl, a_row(lane));
       kstep[ks] = 32u * pl.w;  // 16 rows further (the swizzle repeats every 8 rows)
     }
 #pragma unroll
     for (int mt = 0; mt < NMV; ++mt) {
-      if (Q8) {
+      if (QI) {
         const PieceLoc pl = locate_i8(rVc, kTile, min(mt, rVc / 8 - 1));
         voff[mt] = kt_bytes + swz(pl, lane);
         vstep[mt] = 64u * pl.w;
@@ -873,7 +906,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
 
     for (int k = 0; k < my_tiles && ok; ++k) {
       const int st = k % ns;
-      if constexpr (Q8) {
+      if constexpr (QI) {
 #pragma unroll
         for (int j = 0; j < SJ; ++j) {
           skc[j] = skn[j];
@@ -955,7 +988,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
       // int8 caches: value fragments of the first m-tiles (raw ldmatrix words, k32 steps)
       constexpr int VG8 = MT == 4 ? 1 : 2;
       uint32_t vx8[VG8][MT / 2][4];
-      if constexpr (!Q8) {
+      if constexpr (!QI) {
         // c[mt][j][e] is token 16 mt + (lane >> 2) + 8 (e >> 1), column 2 (lane & 3) + (e & 1)
         float c[MT][NB][4];
 #pragma unroll
@@ -995,7 +1028,23 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
         int ci[MT][NB][4];
 #pragma unroll
         for (int ks = 0; ks < NKS / 2; ++ks)
-          if (ks < nks8) {
+          if (Q4 && ks < nks8) {
+            // 4-bit: one x4 gives 32 rows of the k-step's 16-byte column; a byte's low and high
+            // nibbles, moved to the top of the byte, are 16 x the two codes as exact s8
+            uint32_t kp[MT / 2][4];
+#pragma unroll
+            for (int gq = 0; gq < MT / 2; ++gq) ldsm_x4(sbase + koff[ks] + gq * kstep[ks], kp[gq]);
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+              const uint32_t p0 = kp[mt >> 1][2 * (mt & 1)], p1 = kp[mt >> 1][2 * (mt & 1) + 1];
+              const uint32_t af[4] = {nib_lo(p0), nib_lo(p1), nib_hi(p0), nib_hi(p1)};
+#pragma unroll
+              for (int j = 0; j < NB; ++j) {
+                if (ks == 0) mma_i8_k32<true, false>(ci[mt][j], af, qf8[ks][j][0], qf8[ks][j][1]);
+                else mma_i8_k32<false, false>(ci[mt][j], af, qf8[ks][j][0], qf8[ks][j][1]);
+              }
+            }
+          } else if (!Q4 && ks < nks8) {
             const bool k32 = 32 * ks + 32 <= rK;
             uint32_t kf[MT][4];
 #pragma unroll
@@ -1016,10 +1065,11 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
                 }
               }
           }
-        // the first value m-tiles' fragments do not depend on the scores: request them now
+        // the first value m-tiles' (4-bit: 16-byte columns') fragments do not depend on the
+        // scores: request them now
 #pragma unroll
         for (int u = 0; u < VG8; ++u)
-          if (u < nmv) {
+          if (Q4 ? 2 * u < nmv : u < nmv) {
 #pragma unroll
             for (int kk = 0; kk < MT / 2; ++kk) ldsm_x4_t(sbase + voff[u] + kk * vstep[u], vx8[u][kk]);
           }
@@ -1097,7 +1147,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
       }
       const float uA = mA == -INFINITY ? 0.f : mA, uB = mB == -INFINITY ? 0.f : mB;
       float pa_sum = 0.f, pb_sum = 0.f;
-      if constexpr (!Q8) {
+      if constexpr (!QI) {
         // weights of the tile as B fragments of P^T: block r = tokens 8r..8r+7 in the score
         // layout (row = token, columns = this lane's two heads), transposed to (token pairs, head)
         uint32_t pb[NB][2 * MT];
@@ -1186,7 +1236,9 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
             pb8[NB - 1][mt] = movm_t(__byte_perm(u, v, 0x6240));
           }
         }
-        const float sA = xA * (1.f / 65535.f), sB = xB * (1.f / 65535.f);
+        // (4-bit: the value fragments carry 16 x the codes, so sigma takes 1/16)
+        const float sA = xA * (Q4 ? 1.f / (16.f * 65535.f) : 1.f / 65535.f);
+        const float sB = xB * (Q4 ? 1.f / (16.f * 65535.f) : 1.f / 65535.f);
         float zA[NB], zB[NB];  // sigma of the lane's two columns per n-tile (256 sigma: hi part)
 #pragma unroll
         for (int j = 0; j < NB; ++j) {
@@ -1194,6 +1246,58 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
           zA[j] = hi ? 256.f * sA : sA;
           zB[j] = hi ? 256.f * sB : sB;
         }
+        if constexpr (Q4) {
+        // 4-bit: the transposed x4 of a 16-byte column gives each lane, per 8 tokens, the bytes
+        // 2 g (dims 4 g, 4 g + 1) and 2 g + 1 (dims 4 g + 2, 4 g + 3) of tokens 2 (lane & 3) + {0, 1};
+        // byte permutes gather 4 tokens in the weights' order and the nibble masks split the
+        // dims: m-tile 2 c has rows g = dim 4 g, g + 8 = dim 4 g + 1 of column c, m-tile 2 c + 1
+        // rows g = dim 4 g + 2, g + 8 = dim 4 g + 3.
+#pragma unroll
+        for (int c0 = 0; c0 < NMV / 2; c0 += VG8)
+          if (2 * c0 < nmv) {
+            if (c0 > 0) {
+#pragma unroll
+              for (int u = 0; u < VG8; ++u)
+                if (2 * (c0 + u) < nmv) {
+#pragma unroll
+                  for (int kk = 0; kk < MT / 2; ++kk)
+                    ldsm_x4_t(sbase + voff[c0 + u] + kk * vstep[c0 + u], vx8[u][kk]);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < VG8; ++u)
+              if (2 * (c0 + u) < nmv) {
+                const int c = c0 + u;
+                int accP[NB][4], accQ[NB][4];
+#pragma unroll
+                for (int kk = 0; kk < MT / 2; ++kk) {
+                  const uint32_t* x = vx8[u][kk];
+                  const uint32_t p0 = __byte_perm(x[0], x[1], 0x6240), q0 = __byte_perm(x[0], x[1], 0x7351);
+                  const uint32_t p1 = __byte_perm(x[2], x[3], 0x6240), q1 = __byte_perm(x[2], x[3], 0x7351);
+                  const uint32_t afP[4] = {nib_lo(p0), nib_hi(p0), nib_lo(p1), nib_hi(p1)};
+                  const uint32_t afQ[4] = {nib_lo(q0), nib_hi(q0), nib_lo(q1), nib_hi(q1)};
+#pragma unroll
+                  for (int j = 0; j < NB; ++j) {
+                    if (kk == 0) {
+                      mma_i8_k32<true, true>(accP[j], afP, pb8[j][2 * kk], pb8[j][2 * kk + 1]);
+                      mma_i8_k32<true, true>(accQ[j], afQ, pb8[j][2 * kk], pb8[j][2 * kk + 1]);
+                    } else {
+                      mma_i8_k32<false, true>(accP[j], afP, pb8[j][2 * kk], pb8[j][2 * kk + 1]);
+                      mma_i8_k32<false, true>(accQ[j], afQ, pb8[j][2 * kk], pb8[j][2 * kk + 1]);
+                    }
+                  }
+                }
+#pragma unroll
+                for (int j = 0; j < NB; ++j)
+#pragma unroll
+                  for (int e = 0; e < 4; ++e) {
+                    const float z = (e & 1) ? zB[j] : zA[j];
+                    oacc[2 * c][j][e] = fmaf((float)accP[j][e], z, oacc[2 * c][j][e]);
+                    oacc[2 * c + 1][j][e] = fmaf((float)accQ[j][e], z, oacc[2 * c + 1][j][e]);
+                  }
+              }
+          }
+        } else {
         // value mix: the transposed x4 gives each lane, per 8 tokens, a 16-bit pair of dims
         // (2 g, 2 g + 1) of tokens 2 (lane & 3) + {0, 1}; byte permutes make A rows of 4 tokens
         // in the weights' order: row g is dim 2 g of the m-tile, row g + 8 dim 2 g + 1.
@@ -1231,6 +1335,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
                     oacc[g0 + u][j][e] = fmaf((float)acc[j][e], (e & 1) ? zB[j] : zA[j], oacc[g0 + u][j][e]);
               }
           }
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[warp * ns + st]);  // the stage may be refilled
@@ -1246,7 +1351,8 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
     lB += __shfl_xor_sync(kFull, lB, o);
   }
   // o~ of (dim 16 mt + (lane >> 2) + 8 (e >> 1), head hA + (e & 1)); int8 caches: dim
-  // 16 mt + 2 (lane >> 2) + (e >> 1)
+  // 16 mt + 2 (lane >> 2) + (e >> 1); 4-bit caches: dim 32 (mt >> 1) + 4 (lane >> 2) +
+  // 2 (mt & 1) + (e >> 1)
   float ov[NMV][4];
 #pragma unroll
   for (int mt = 0; mt < NMV; ++mt)
@@ -1287,8 +1393,10 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
         if (mt < nmv)
 #pragma unroll
           for (int e = 0; e < 4; ++e)
-            sts_f32(redb + 4u * (uint32_t)((warp * 8 + hA + (e & 1)) * rV + 16 * mt +
-                                           (Q8 ? 2 * (lane >> 2) + (e >> 1) : (lane >> 2) + 8 * (e >> 1))),
+            sts_f32(redb + 4u * (uint32_t)((warp * 8 + hA + (e & 1)) * rV +
+                                           (Q4   ? 32 * (mt >> 1) + 4 * (lane >> 2) + 2 * (mt & 1) + (e >> 1)
+                                            : Q8 ? 16 * mt + 2 * (lane >> 2) + (e >> 1)
+                                                 : 16 * mt + (lane >> 2) + 8 * (e >> 1))),
                     ov[mt][e] * ((e & 1) ? fB : fA));
       if ((lane >> 2) == 0) {  // the sums rescaled in place (only the maxima were read above)
         sts_f32(mlb + 8u * (uint32_t)(warp * 8 + hA) + 4u, lA * fA);
@@ -1664,7 +1772,8 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
 
 template <int NB, int NKS, int NMV, int TT, int MODE>
 static cudaError_t launch_k(const DecodeArgs& a, cudaStream_t stream) {
-  const DecodeSmem L = decode_smem_layout(a.nwarps, a.nstage, a.rK, a.rV, TT, MODE == kModeQ8);
+  const DecodeSmem L = decode_smem_layout(a.nwarps, a.nstage, a.rK, a.rV, TT,
+                                          MODE == kModeQ8 ? 1 : MODE == kModeQ4 ? 2 : 0);
   auto kern = stief_decode_kernel<NB, NKS, NMV, TT, MODE>;
   static SmemLimit limit;
   cudaError_t e = limit.ensure(reinterpret_cast<const void*>(kern), a.device, (int)L.total);
@@ -1709,6 +1818,7 @@ cudaError_t launch_decode_plain(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_latent(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_paged(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_q8(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_decode_q4(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_joint_v(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_latent_joint_v(const DecodeArgs& a, cudaStream_t stream);
 

@@ -4,12 +4,12 @@
 
 namespace stief {
 
-uint32_t decode_smem_bytes(int nwarps, int nstage, int rK, int rV, int tile, bool q8) {
-  return decode_smem_layout(nwarps, nstage, rK, rV, tile, q8).total;
+uint32_t decode_smem_bytes(int nwarps, int nstage, int rK, int rV, int tile, int code) {
+  return decode_smem_layout(nwarps, nstage, rK, rV, tile, code).total;
 }
 
-uint32_t decode_region_bytes(int nwarps, int nstage, int rK, int rV, int tile, bool q8) {
-  return decode_smem_layout(nwarps, nstage, rK, rV, tile, q8).region_bytes;
+uint32_t decode_region_bytes(int nwarps, int nstage, int rK, int rV, int tile, int code) {
+  return decode_smem_layout(nwarps, nstage, rK, rV, tile, code).region_bytes;
 }
 
 // the latent decode, paged, int8 and joint-value caches are their own instantiations, so their
@@ -19,15 +19,16 @@ cudaError_t launch_decode(const DecodeArgs& planned, cudaStream_t stream) {
   // right after a compress of this library the new rows may still be in flight when this
   // kernel starts: no cache tile is requested before the dependency wait then
   a.early = take_stream_compress_mark(a.device, stream) ? 0 : 1;
-  if ((a.latent != 0) + (a.block_table != nullptr) + (a.q8 != 0) > 1)
+  if ((a.latent != 0) + (a.block_table != nullptr) + (a.q8 != 0) + (a.q4 != 0) > 1)
     return cudaErrorInvalidValue;  // the modes do not combine
   if (a.joint_v) {
-    if (a.block_table != nullptr || a.q8 != 0 || a.append != 0) return cudaErrorInvalidValue;
+    if (a.block_table != nullptr || a.q8 != 0 || a.q4 != 0 || a.append != 0) return cudaErrorInvalidValue;
     return a.latent ? launch_decode_latent_joint_v(a, stream) : launch_decode_joint_v(a, stream);
   }
   if (a.latent) return launch_decode_latent(a, stream);
   if (a.block_table) return launch_decode_paged(a, stream);
   if (a.q8) return launch_decode_q8(a, stream);
+  if (a.q4) return launch_decode_q4(a, stream);
   return launch_decode_plain(a, stream);
 }
 

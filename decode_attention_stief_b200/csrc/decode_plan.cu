@@ -185,9 +185,11 @@ stief_status plan_decode(DecodeArgs& a, const uint16_t* q, const uint16_t* P_K,
                          int rK, int rV, int L_max, int max_seq_len, int num_splits,
                          uint32_t* dev_status, bool latent, const int32_t* block_table,
                          int max_pages, int page_size, int num_pages, const float* k_scale,
-                         const float* v_scale, bool joint_v) {
-  const bool q8 = k_scale != nullptr;
-  if (joint_v && (block_table || q8)) return STIEF_ERR_INVALID_ARG;
+                         const float* v_scale, bool joint_v, bool q4) {
+  const bool q8 = k_scale != nullptr && !q4;  // int8 codes
+  if (q4 && (k_scale == nullptr || rK % 32 != 0 || rV % 32 != 0)) return STIEF_ERR_INVALID_ARG;
+  if (joint_v && (block_table || q8 || q4)) return STIEF_ERR_INVALID_ARG;
+  const int code = q8 ? 1 : q4 ? 2 : 0;  // the stage layout's code form
   if (!q || !k_lat || !v_lat || !seq_lens || !out) return STIEF_ERR_INVALID_ARG;
   if (!latent && (!P_K || !P_V)) return STIEF_ERR_INVALID_ARG;
   if (B < 1 || B > 65535 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || Hq / Hkv > 64)
@@ -240,13 +242,13 @@ stief_status plan_decode(DecodeArgs& a, const uint16_t* q, const uint16_t* P_K,
   a.max_seq_len = max_seq_len;
   // tokens per split: the split's share rounded up to whole 32-token tiles, so that only
   // the last tile of a sequence can be partial
-  a.tile = q8 ? choose_decode_tile_q8(rK, rV) : choose_decode_tile(rK, rV);
+  a.tile = (q8 || q4) ? choose_decode_tile_q8(rK, rV) : choose_decode_tile(rK, rV);
   a.chunk = ((max_seq_len + a.S - 1) / a.S + a.tile - 1) / a.tile * a.tile;
   a.qscale = (float)(1.4426950408889634 / std::sqrt((double)d));
   const long long units = (long long)B * a.Hkv * a.qsub;
   const bool pair = a.S == 1 && units > sms &&
-                    choose_decode_config_pair(rK, rV, a.tile, &a.nwarps, &a.nstage, q8);
-  if (!pair && !choose_decode_config(rK, rV, a.tile, &a.nwarps, &a.nstage, q8))
+                    choose_decode_config_pair(rK, rV, a.tile, &a.nwarps, &a.nstage, code);
+  if (!pair && !choose_decode_config(rK, rV, a.tile, &a.nwarps, &a.nstage, code))
     return STIEF_ERR_INVALID_ARG;
   // Split merge: through tagged words when the whole grid is on the GPU at once (one CTA per
   // SM at most, so every split of a unit runs while its merging CTA reads their records) and
@@ -255,17 +257,20 @@ stief_status plan_decode(DecodeArgs& a, const uint16_t* q, const uint16_t* P_K,
   a.merge_tagged = 0;
   if (a.S > 1 && (long long)a.S * units <= sms &&
       decode_tagged_stage_bytes(a.G_T, a.S, rV) <=
-          decode_region_bytes(a.nwarps, a.nstage, rK, rV, a.tile, q8))
+          decode_region_bytes(a.nwarps, a.nstage, rK, rV, a.tile, code))
     a.merge_tagged = 1;
 
   int nmaps = 0;
   const uint64_t prow = (uint64_t)Hkv * d;
   a.q8 = q8 ? 1 : 0;
+  a.q4 = q4 ? 1 : 0;
   a.k_scale = k_scale;
   a.v_scale = v_scale;
-  // the caches' column pieces (int8 codes: rows of r bytes, moved as r / 2 16-bit columns)
-  if (!plan_pieces(a, &nmaps, a.pk, k_lat, q8 ? rK / 2 : rK, rows, a.tile) ||
-      !plan_pieces(a, &nmaps, a.pv, v_lat, q8 ? rV / 2 : rV, vrows, a.tile))
+  // the caches' column pieces (int8 codes: rows of r bytes, moved as r / 2 16-bit columns;
+  // 4-bit codes: r / 2 bytes, r / 4 columns)
+  const int kc = q8 ? rK / 2 : q4 ? rK / 4 : rK, vc = q8 ? rV / 2 : q4 ? rV / 4 : rV;
+  if (!plan_pieces(a, &nmaps, a.pk, k_lat, kc, rows, a.tile) ||
+      !plan_pieces(a, &nmaps, a.pv, v_lat, vc, vrows, a.tile))
     return STIEF_ERR_CUDA;
   if (!latent && (!plan_pieces(a, &nmaps, a.ppk, P_K, rK, prow, d) ||
                   !plan_pieces(a, &nmaps, a.ppv, P_V, rV, prow, d)))

@@ -123,7 +123,7 @@ stief_status compress_common(const uint16_t* k_new, const uint16_t* v_new, const
                              int32_t* seq_lens, int B, int Hkv, int T, int d, int rK, int rV,
                              int L_max, uint32_t* dev_status, stief_stream_t stream,
                              const Paging& pg, float* k_scale = nullptr,
-                             float* v_scale = nullptr) {
+                             float* v_scale = nullptr, bool q4 = false) {
   if (!k_new || !v_new || !P_K || !P_V || !k_lat || !v_lat || !seq_lens) return STIEF_ERR_INVALID_ARG;
   if (pg.block_table) {
     const stief_status st = check_paging(pg, Hkv, &L_max);
@@ -162,6 +162,7 @@ stief_status compress_common(const uint16_t* k_new, const uint16_t* v_new, const
   a.num_pages = pg.num_pages;
   a.k_scale = k_scale;
   a.v_scale = v_scale;
+  a.q4 = q4 ? 1 : 0;
   if (stief::launch_compress(a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return STIEF_ERR_CUDA;
   return STIEF_OK;
@@ -193,6 +194,19 @@ stief_status stief_compress_append_q8(const uint16_t* k_new, const uint16_t* v_n
                          dev_status, stream, Paging{}, k_s, v_s);
 }
 
+stief_status stief_compress_append_q4(const uint16_t* k_new, const uint16_t* v_new,
+                                      const uint16_t* P_K, const uint16_t* P_V, uint8_t* k_q,
+                                      uint8_t* v_q, float* k_s, float* v_s, int32_t* seq_lens,
+                                      int B, int Hkv, int T, int d, int rK, int rV, int L_max,
+                                      uint32_t* dev_status, stief_stream_t stream) {
+  if (!k_s || !v_s) return STIEF_ERR_INVALID_ARG;
+  if (L_max % kQ8RowQuantum != 0 || rK % 32 != 0 || rV % 32 != 0) return STIEF_ERR_INVALID_ARG;
+  if (!aligned16(k_s) || !aligned16(v_s)) return STIEF_ERR_ALIGNMENT;
+  return compress_common(k_new, v_new, P_K, P_V, reinterpret_cast<uint16_t*>(k_q),
+                         reinterpret_cast<uint16_t*>(v_q), seq_lens, B, Hkv, T, d, rK, rV, L_max,
+                         dev_status, stream, Paging{}, k_s, v_s, true);
+}
+
 stief_status stief_compress_append_paged(const uint16_t* k_new, const uint16_t* v_new,
                                          const uint16_t* P_K, const uint16_t* P_V,
                                          uint16_t* k_pages, uint16_t* v_pages,
@@ -220,7 +234,8 @@ stief_status decode_common(const uint16_t* q, const uint16_t* k_new, const uint1
                            int L_max, int max_seq_len, int num_splits, uint32_t* dev_status,
                            stief_stream_t stream, bool append, bool latent = false,
                            const Paging& pg = Paging{}, const float* k_scale = nullptr,
-                           const float* v_scale = nullptr, bool joint_v = false) {
+                           const float* v_scale = nullptr, bool joint_v = false,
+                           bool q4 = false) {
   // cheap host checks first, so argument errors never touch CUDA
   if (!q || !k_lat || !v_lat || !seq_lens || !out) return STIEF_ERR_INVALID_ARG;
   if (pg.block_table) {  // paged: the capacity is max_pages * page_size tokens
@@ -244,7 +259,8 @@ stief_status decode_common(const uint16_t* q, const uint16_t* k_new, const uint1
   stief::DecodeArgs a{};
   st = stief::plan_decode(a, q, P_K, P_V, k_lat, v_lat, seq_lens, out, B, Hq, Hkv, d, rK, rV,
                           L_max, max_seq_len, num_splits, dev_status, latent, pg.block_table,
-                          pg.max_pages, pg.page_size, pg.num_pages, k_scale, v_scale, joint_v);
+                          pg.max_pages, pg.page_size, pg.num_pages, k_scale, v_scale, joint_v,
+                          q4);
   if (st != STIEF_OK) return st;
   a.append = append ? 1 : 0;
   a.k_new = k_new;
@@ -389,6 +405,25 @@ stief_status stief_decode_attention_q8(const uint16_t* q, const uint16_t* P_K,
                        const_cast<int32_t*>(seq_lens), out, workspace, workspace_bytes, B, Hq, Hkv,
                        d, rK, rV, L_max, max_seq_len, num_splits, dev_status, stream, false, false,
                        Paging{}, k_s, v_s);
+}
+
+stief_status stief_decode_attention_q4(const uint16_t* q, const uint16_t* P_K,
+                                       const uint16_t* P_V, const uint8_t* k_q, const uint8_t* v_q,
+                                       const float* k_s, const float* v_s,
+                                       const int32_t* seq_lens, uint16_t* out, void* workspace,
+                                       size_t workspace_bytes, int B, int Hq, int Hkv, int d,
+                                       int rK, int rV, int L_max, int max_seq_len,
+                                       int num_splits, uint32_t* dev_status,
+                                       stief_stream_t stream) {
+  if (!k_s || !v_s) return STIEF_ERR_INVALID_ARG;
+  if (L_max % kQ8RowQuantum != 0 || rK % 32 != 0 || rV % 32 != 0) return STIEF_ERR_INVALID_ARG;
+  if (!aligned16(k_s) || !aligned16(v_s)) return STIEF_ERR_ALIGNMENT;
+  return decode_common(q, nullptr, nullptr, P_K, P_V,
+                       reinterpret_cast<uint16_t*>(const_cast<uint8_t*>(k_q)),
+                       reinterpret_cast<uint16_t*>(const_cast<uint8_t*>(v_q)),
+                       const_cast<int32_t*>(seq_lens), out, workspace, workspace_bytes, B, Hq, Hkv,
+                       d, rK, rV, L_max, max_seq_len, num_splits, dev_status, stream, false, false,
+                       Paging{}, k_s, v_s, false, true);
 }
 
 stief_status stief_decode_attention_paged(const uint16_t* q, const uint16_t* P_K,

@@ -315,12 +315,12 @@ __device__ __forceinline__ uint16_t f32_to_bf16_rn(float f) {
 __device__ __forceinline__ float bf16_round(float x) {
   return __uint_as_float((uint32_t)f32_to_bf16_rn(x) << 16);
 }
-// The int8 code of x under a row scale: RNE(x / scale) in [-127, 127] (IEEE fp32 division);
-// a zero scale (a zero row) gives 0.
-__device__ __forceinline__ int quantize_code(float x, float scale) {
+// The integer code of x under a row scale: RNE(x / scale) in [-qmax, qmax] (IEEE fp32
+// division; qmax 127 for int8, 7 for 4-bit codes); a zero scale (a zero row) gives 0.
+__device__ __forceinline__ int quantize_code(float x, float scale, int qmax = 127) {
   if (!(scale > 0.f)) return 0;
   const int c = __float2int_rn(__fdiv_rn(x, scale));
-  return c > 127 ? 127 : (c < -127 ? -127 : c);
+  return c > qmax ? qmax : (c < -qmax ? -qmax : c);
 }
 __device__ __forceinline__ uint32_t pack_bf16x2_rn(float lo, float hi) {
   uint32_t r;

@@ -67,8 +67,10 @@ struct DecodeArgs {
   // [B][max_pages] (null for a contiguous cache; L_max is then max_pages * page_size)
   const int32_t* block_table;
   int max_pages, page_size, num_pages;
-  // int8 caches: k_lat / v_lat hold int8 codes [rows][r] and these the fp32 row scales
+  // int8 caches: k_lat / v_lat hold int8 codes [rows][r] and these the fp32 row scales;
+  // 4-bit caches (q4): two codes per byte, [rows][r / 2], with the same row scales
   int q8;
+  int q4;
   int joint_v;     // values: one row per (sequence, token) shared by the KV heads
   // 1: the contiguous bf16 and latent modes request each warp's first tile before the
   // dependency wait; 0 when the library's previous launch in the stream was a compress (its
@@ -97,9 +99,11 @@ struct CompressArgs {
   // paged caches, as in DecodeArgs (block_table null: contiguous [B][Hkv][L_max] rows)
   const int32_t* block_table;
   int max_pages, page_size, num_pages;
-  // int8 caches: k_lat / v_lat take int8 codes and these the fp32 row scales (null: bf16)
+  // int8 caches: k_lat / v_lat take int8 codes and these the fp32 row scales (null: bf16);
+  // with q4 the codes are 4-bit, two per byte ([rows][r / 2])
   float* k_scale;
   float* v_scale;
+  int q4;
 };
 
 constexpr int kMaxSmemPerBlock = 232448;  // 227 KB opt-in dynamic shared memory (sm_100)
@@ -125,9 +129,10 @@ struct SmemLimit {
   }
 };
 
-uint32_t decode_smem_bytes(int nwarps, int nstage, int rK, int rV, int tile, bool q8 = false);
+// code: 0 bf16 cache, 1 int8 codes, 2 4-bit codes
+uint32_t decode_smem_bytes(int nwarps, int nstage, int rK, int rV, int tile, int code = 0);
 // Bytes of the region (rings, then the warp-merge and split-merge staging) in that layout.
-uint32_t decode_region_bytes(int nwarps, int nstage, int rK, int rV, int tile, bool q8 = false);
+uint32_t decode_region_bytes(int nwarps, int nstage, int rK, int rV, int tile, int code = 0);
 
 // 2-D tiled TMA tensor map over a row-major bf16 matrix [rows][cols] (row stride in
 // bytes), boxes of box_cols x box_rows with the given swizzle.  Host only.
@@ -151,7 +156,7 @@ stief_status plan_decode(DecodeArgs& a, const uint16_t* q, const uint16_t* P_K,
                          uint32_t* dev_status, bool latent = false,
                          const int32_t* block_table = nullptr, int max_pages = 0,
                          int page_size = 0, int num_pages = 0, const float* k_scale = nullptr,
-                         const float* v_scale = nullptr, bool joint_v = false);
+                         const float* v_scale = nullptr, bool joint_v = false, bool q4 = false);
 
 // Decode workspace layout: `units` = B * Hkv * qsub split-ticket counters, then B sequence
 // tickets (uint32, padded together to 256 bytes), then units * G_T * splits partial-state
@@ -201,10 +206,10 @@ inline int choose_decode_tile_q8(int rK, int rV) { return rK <= 64 && rV <= 64 ?
 constexpr int kPairSmemPerBlock = 233472 / 2 - 1024;
 constexpr int kPairMaxConsumerWarps = 5;
 inline bool choose_decode_config_pair(int rK, int rV, int tile, int* nwarps, int* nstage,
-                                      bool q8 = false) {
+                                      int code = 0) {
   for (int nw = kPairMaxConsumerWarps; nw >= 4; --nw)
     for (int ns = 4; ns >= 2; --ns)
-      if (decode_smem_bytes(nw, ns, rK, rV, tile, q8) <= (uint32_t)kPairSmemPerBlock) {
+      if (decode_smem_bytes(nw, ns, rK, rV, tile, code) <= (uint32_t)kPairSmemPerBlock) {
         *nwarps = nw;
         *nstage = ns;
         return true;
@@ -212,10 +217,10 @@ inline bool choose_decode_config_pair(int rK, int rV, int tile, int* nwarps, int
   return false;
 }
 inline bool choose_decode_config(int rK, int rV, int tile, int* nwarps, int* nstage,
-                                 bool q8 = false) {
+                                 int code = 0) {
   for (int nw = 8; nw >= 2; --nw)
     for (int ns = 8; ns >= 2; --ns)
-      if (decode_smem_bytes(nw, ns, rK, rV, tile, q8) <= (uint32_t)kMaxSmemPerBlock) {
+      if (decode_smem_bytes(nw, ns, rK, rV, tile, code) <= (uint32_t)kMaxSmemPerBlock) {
         *nwarps = nw;
         *nstage = ns;
         return true;

@@ -377,6 +377,35 @@ STIEF_API stief_status stief_decode_attention_q8(const uint16_t* q, const uint16
                                        stief_stream_t stream);
 
 /*
+ * 4-bit latent caches (the pages' other quantisation width; same per-row reading as the int8
+ * form): each latent row (one token, one KV head) as symmetric 4-bit codes and one fp32 scale,
+ *     scale = max_c |x_c| / 7,  code_c = RNE(x_c / scale) in [-7, 7]
+ * (x the bf16-rounded row, both divisions in IEEE fp32; a zero row is scale 0, codes 0), two
+ * codes per byte, column 2j in the low nibble of byte j (4-bit two's complement):
+ *     k_q : uint8 [B][Hkv][L_max][rK / 2],  k_s : float [B][Hkv][L_max]  (likewise v_q, v_s)
+ * A row takes r / 2 + 4 bytes.  rK and rV must be multiples of 32 (rows of whole 16-byte
+ * units), L_max a multiple of 64; k_s, v_s, k_q, v_q 16-byte aligned.  The calls are the int8
+ * ones on this form: the compress writes codes and scales; the decode attends over
+ * code * scale, the codes entering the integer MMA as 16 x code (each byte's nibbles moved to
+ * the top of a byte), q~ and the weights as 16-bit fixed point in two 8-bit parts as for the
+ * int8 form.  Paged 4-bit caches and the fused step are not provided.
+ */
+STIEF_API stief_status stief_compress_append_q4(const uint16_t* k_new, const uint16_t* v_new,
+                                      const uint16_t* P_K, const uint16_t* P_V, uint8_t* k_q,
+                                      uint8_t* v_q, float* k_s, float* v_s, int32_t* seq_lens,
+                                      int B, int Hkv, int T, int d, int rK, int rV, int L_max,
+                                      uint32_t* dev_status, stief_stream_t stream);
+
+STIEF_API stief_status stief_decode_attention_q4(const uint16_t* q, const uint16_t* P_K,
+                                       const uint16_t* P_V, const uint8_t* k_q, const uint8_t* v_q,
+                                       const float* k_s, const float* v_s,
+                                       const int32_t* seq_lens, uint16_t* out, void* workspace,
+                                       size_t workspace_bytes, int B, int Hq, int Hkv, int d,
+                                       int rK, int rV, int L_max, int max_seq_len,
+                                       int num_splits, uint32_t* dev_status,
+                                       stief_stream_t stream);
+
+/*
  * Joint value latents (STAR-KV technical summary, "Metodologia" item 2, the hybrid
  * decomposition: keys keep one basis per KV head, the values of all KV heads are factored
  * together, and the value reconstruction is absorbed into the output projection).  The values

@@ -324,24 +324,47 @@ def gather_pages(pages, block_table, seq_lens, L_max: int) -> np.ndarray:
     return out
 
 
-def quantize_rows(x):
-    """Per-row symmetric int8 quantisation of latent rows (the low-bit cache form).
+def quantize_rows(x, qmax: int = 127):
+    """Per-row symmetric quantisation of latent rows (the low-bit cache forms).
 
     The pages report the compressed cache to be robust to 4- and 8-bit quantisation but fix no
     scheme; this library's reading: one fp32 scale per stored row (per token, KV head),
-        scale = fp32(max_c |x_c| / 127),  code_c = RNE(fp32(x_c / scale)) in [-127, 127],
-    with a zero row stored as scale 0 and codes 0.  x are the bf16 latent values (exact in
-    fp32).  The two divisions and the rounding to an integer are taken in IEEE fp32, the
-    kernel's precision, so the integer codes are decided identically on both sides.
+        scale = fp32(max_c |x_c| / qmax),  code_c = RNE(fp32(x_c / scale)) in [-qmax, qmax],
+    qmax = 127 for the int8 form and 7 for the 4-bit form, with a zero row stored as scale 0
+    and codes 0.  x are the bf16 latent values (exact in fp32).  The two divisions and the
+    rounding to an integer are taken in IEEE fp32, the kernel's precision, so the integer codes
+    are decided identically on both sides.
     Returns (codes int8 [..., r], scales float32 [...]).
     """
     x32 = np.asarray(x, dtype=np.float32)
     amax = np.max(np.abs(x32), axis=-1)
-    scale = (amax / np.float32(127.0)).astype(np.float32)
+    scale = (amax / np.float32(qmax)).astype(np.float32)
     safe = np.where(scale > 0, scale, np.float32(1.0)).astype(np.float32)
     q = np.rint((x32 / safe[..., None]).astype(np.float32))
     q = np.where(scale[..., None] > 0, q, 0.0)
-    return np.clip(q, -127, 127).astype(np.int8), scale
+    return np.clip(q, -qmax, qmax).astype(np.int8), scale
+
+
+def pack_q4(codes) -> np.ndarray:
+    """4-bit codes in [-8, 7] (int8 [..., r], r even) two per byte: byte j holds column 2j in
+    its low nibble and column 2j + 1 in its high nibble, each as a 4-bit two's complement."""
+    c = np.asarray(codes, dtype=np.int16)
+    lo = c[..., 0::2] & 0xF
+    hi = c[..., 1::2] & 0xF
+    return (lo | (hi << 4)).astype(np.uint8)
+
+
+def unpack_q4(packed) -> np.ndarray:
+    """The inverse of pack_q4: uint8 [..., r / 2] -> int8 codes [..., r]."""
+    p = np.asarray(packed, dtype=np.int16)
+    lo = p & 0xF
+    hi = (p >> 4) & 0xF
+    lo = np.where(lo >= 8, lo - 16, lo)
+    hi = np.where(hi >= 8, hi - 16, hi)
+    out = np.empty(p.shape[:-1] + (2 * p.shape[-1],), dtype=np.int8)
+    out[..., 0::2] = lo
+    out[..., 1::2] = hi
+    return out
 
 
 def dequantize_rows(codes, scales) -> np.ndarray:

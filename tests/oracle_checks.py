@@ -352,6 +352,37 @@ def check_quantize_rows(o) -> None:
     assert qr[0].tolist() == [127, 2, 4, -2, 0, 0, 2, 126]
 
 
+def check_quantize_rows_q4(o) -> None:
+    """The 4-bit form: the largest magnitude maps to +-7 exactly; codes stay in [-7, 7]; halfway
+    cases round to even; every element is within half a step of its code; and the packing puts
+    column 2j in the low and 2j + 1 in the high nibble of byte j (hand-packed bytes below),
+    round-tripping every code of [-8, 7]."""
+    import oracle
+    rng = np.random.default_rng(22)
+    x = oracle.round_bf16(rng.standard_normal((64, 64)) * rng.uniform(0.01, 10, (64, 1)))
+    q, s = oracle.quantize_rows(x, qmax=7)
+    assert q.dtype == np.int8 and s.dtype == np.float32
+    assert q.min() >= -7 and q.max() <= 7
+    amax_idx = np.argmax(np.abs(x), axis=1)
+    assert np.all(np.abs(q[np.arange(64), amax_idx]) == 7)
+    err = np.abs(x - oracle.dequantize_rows(q, s))
+    assert np.all(err <= 0.5 * s[:, None] * (1 + 2.0 ** -22) + np.abs(x) * 2.0 ** -23)
+    # row max 7 gives scale exactly 1: x = k + 0.5 rounds to the even neighbour
+    row = np.array([[7.0, 2.5, 3.5, -2.5, -0.5, 0.5, 1.5, -6.5]])
+    qr, sr = oracle.quantize_rows(row, qmax=7)
+    assert sr[0] == 1.0
+    assert qr[0].tolist() == [7, 2, 4, -2, 0, 0, 2, -6]
+    # packing: (lo, hi) = (7, 2) -> 0x27; (4, -2) -> 0xE4; (0, 0) -> 0x00; (2, -6) -> 0xA2
+    packed = oracle.pack_q4(qr)
+    assert packed.dtype == np.uint8 and packed.shape == (1, 4)
+    assert packed[0].tolist() == [0x27, 0xE4, 0x00, 0xA2]
+    allc = np.arange(-8, 8, dtype=np.int8)
+    grid = np.stack(np.meshgrid(allc, allc, indexing="ij"), -1).reshape(-1, 2)  # every (lo, hi)
+    assert np.array_equal(oracle.unpack_q4(oracle.pack_q4(grid)), grid)
+    assert sorted(oracle.pack_q4(grid)[:, 0].tolist()) == list(range(256))
+    assert np.array_equal(oracle.unpack_q4(oracle.pack_q4(q)), q)
+
+
 # ----------------------------------------------------------------------------- compression
 
 def check_compress_identity_basis(o, r: int = 48, d: int = 128) -> None:
@@ -561,6 +592,7 @@ ALL_ORACLE_CHECKS = {
     "latent_edges": check_latent_edges,
     "paged_layout": check_paged_layout,
     "quantize_rows": check_quantize_rows,
+    "quantize_rows_q4": check_quantize_rows_q4,
     "compress_identity_basis": check_compress_identity_basis,
     "compress_matches_exact_product": check_compress_matches_exact_product,
     "compress_append_bookkeeping": check_compress_append_bookkeeping,

@@ -81,9 +81,10 @@ def test_algorithmic_bytes_follow_the_footprint_formula():
 
 def test_step_call_names_the_api_call_of_each_mode():
     class A:
-        int8 = latent = paged = joint = unfused = False
+        int8 = int4 = latent = paged = joint = unfused = False
     cases = [({}, "stief_append_decode"), ({"unfused": True}, "stief_decode_attention"),
              ({"latent": True}, "stief_decode_latent"), ({"int8": True}, "stief_decode_attention_q8"),
+             ({"int8": True, "int4": True}, "stief_decode_attention_q4"),
              ({"paged": True}, "stief_append_decode_paged"),
              ({"joint": True}, "stief_decode_attention_joint_v"),
              ({"joint": True, "latent": True}, "stief_decode_latent_joint_v")]
