@@ -168,6 +168,15 @@ __device__ __forceinline__ void mma_i8_k16(int (&c)[4], uint32_t a0, uint32_t a1
 __device__ __forceinline__ uint32_t nib_lo(uint32_t p) { return (p << 4) & 0xF0F0F0F0u; }
 __device__ __forceinline__ uint32_t nib_hi(uint32_t p) { return p & 0xF0F0F0F0u; }
 
+// Exact conversions of small integers through the fp32 bit pattern (integer and fp32 adds instead
+// of the conversion pipe): 12582912 = 1.5 * 2^23 is the fp32 whose integers [2^23, 2^24) have
+// spacing 1, so for |x| < 2^22 the pattern 0x4B400000 + x is the fp32 value 12582912 + x.
+__device__ __forceinline__ float i2f_small(int x) { return __int_as_float(x + 0x4B400000) - 12582912.f; }
+// rint(w * f) for 0 <= w * f < 2^22: the sum with 12582912 rounds once to an integer (RNE).
+__device__ __forceinline__ uint32_t rint_small(float w, float f) {
+  return __float_as_uint(fmaf(w, f, 12582912.f)) - 0x4B400000u;
+}
+
 __device__ __forceinline__ float rcp_approx(float x) {
   float y;
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -1080,19 +1089,21 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
 #pragma unroll
           for (int h = 0; h < 2; ++h)
             skt[mt][h] = __shfl_sync(kFull, skc[(16 * mt + 8 * h) >> 5], ((16 * mt + 8 * h) & 31) + (lane >> 2));
-        // s = s_q k_scale (256 hi + lo), the parts added exactly in s32 (|256 hi + lo| < 2^30)
+        // s = s_q k_scale (256 hi + lo): each part is below 2^21 in magnitude (r <= 128 codes of
+        // at most 127 times at most 128), so it converts exactly; the sum rounds once in fp32
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            int v;
+            float v;
+            const float fc = i2f_small(ci[mt][0][e]);
             if constexpr (NB == 1) {
-              const int o = __shfl_xor_sync(kFull, ci[mt][0][e], 2);
-              v = lo_lane ? ci[mt][0][e] + o * 256 : ci[mt][0][e] * 256 + o;
+              const float fo = __shfl_xor_sync(kFull, fc, 2);
+              v = lo_lane ? fmaf(fo, 256.f, fc) : fmaf(fc, 256.f, fo);
             } else {
-              v = ci[mt][0][e] * 256 + ci[mt][NB - 1][e];
+              v = fmaf(fc, 256.f, i2f_small(ci[mt][NB - 1][e]));
             }
-            s[mt][e] = (float)v * (skt[mt][e >> 1] * ((e & 1) ? sqB : sqA));
+            s[mt][e] = v * (skt[mt][e >> 1] * ((e & 1) ? sqB : sqA));
           }
       }
       if (n < kTile) {  // missing tokens take no weight
@@ -1225,8 +1236,9 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
         uint32_t pb8[NB][MT];
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt) {
-          const uint32_t a0 = __float2uint_rn(wA[2 * mt] * fA), a1 = __float2uint_rn(wA[2 * mt + 1] * fA);
-          const uint32_t b0 = __float2uint_rn(wB[2 * mt] * fB), b1 = __float2uint_rn(wB[2 * mt + 1] * fB);
+          // w16 = rint(w f) in [0, 65535] (w f <= 65535 (1 + 2^-22))
+          const uint32_t a0 = rint_small(wA[2 * mt], fA), a1 = rint_small(wA[2 * mt + 1], fA);
+          const uint32_t b0 = rint_small(wB[2 * mt], fB), b1 = rint_small(wB[2 * mt + 1], fB);
           const uint32_t u = __byte_perm(a0, b0, 0x5410), v = __byte_perm(a1, b1, 0x5410);
           // hi bytes: u.1 v.1 u.3 v.3; lo bytes: u.0 v.0 u.2 v.2
           if constexpr (NB == 1) {
@@ -1292,8 +1304,8 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
 #pragma unroll
                   for (int e = 0; e < 4; ++e) {
                     const float z = (e & 1) ? zB[j] : zA[j];
-                    oacc[2 * c][j][e] = fmaf((float)accP[j][e], z, oacc[2 * c][j][e]);
-                    oacc[2 * c + 1][j][e] = fmaf((float)accQ[j][e], z, oacc[2 * c + 1][j][e]);
+                    oacc[2 * c][j][e] = fmaf(i2f_small(accP[j][e]), z, oacc[2 * c][j][e]);
+                    oacc[2 * c + 1][j][e] = fmaf(i2f_small(accQ[j][e]), z, oacc[2 * c + 1][j][e]);
                   }
               }
           }
@@ -1332,7 +1344,8 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
                 for (int j = 0; j < NB; ++j)
 #pragma unroll
                   for (int e = 0; e < 4; ++e)
-                    oacc[g0 + u][j][e] = fmaf((float)acc[j][e], (e & 1) ? zB[j] : zA[j], oacc[g0 + u][j][e]);
+                    // a tile's s32 mix is below 2^21 (64 tokens x 127 x 255): exact conversion
+                    oacc[g0 + u][j][e] = fmaf(i2f_small(acc[j][e]), (e & 1) ? zB[j] : zA[j], oacc[g0 + u][j][e]);
               }
           }
         }

@@ -231,3 +231,34 @@ def test_decode_right_after_compress_same_stream(rK, rV):
         want = oracle.decode(f64(qs[i]), f64(P_K), f64(P_V), ok_lat, ov_lat, olens)
         assert_decode_close(outs[i].cpu(), want)
     assert glens.cpu().numpy().tolist() == olens.tolist() == [max_seq] * B
+
+
+@pytest.mark.parametrize("name", ["llama3_8b_32k", "llama31_8b_128k"])
+def test_compress_then_decode_full_size(name):
+    """A benchmark shape built the way the model would build it: the whole context compressed by
+    one stief_compress_append call (tensor-core path), then a decode over that cache; the
+    stored latents are checked against the exact products and the decode against the oracle's
+    decode over the oracle's own compressed cache."""
+    w = si.WORKLOADS[name]
+    B, Hq, Hkv, d, L, rK, rV = w.B, w.Hq, w.Hkv, w.d, w.L, w.rK, w.rV
+    dev = torch.device("cuda")
+    seed = si.sub_seed(w.seed, 61)
+    k_new = si.low_rank_rows_torch(si.sub_seed(seed, 1), B * Hkv, L, d, dev).view(B, Hkv, L, d)
+    v_new = si.low_rank_rows_torch(si.sub_seed(seed, 2), B * Hkv, L, d, dev).view(B, Hkv, L, d)
+    P_K, P_V = si.bases_bf16(seed, Hkv, d, rK, rV)
+    gk, gv, glens = _run_append(k_new, v_new, P_K, P_V,
+                                torch.zeros((B, Hkv, L, rK), dtype=torch.bfloat16),
+                                torch.zeros((B, Hkv, L, rV), dtype=torch.bfloat16), [0] * B)
+    assert glens.tolist() == [L] * B
+    kn, vn = f64(k_new.cpu()), f64(v_new.cpu())
+    for h in (0, Hkv - 1):  # two heads checked element by element (the decode covers all)
+        assert _check_latent(gk[0, h], kn[0, h], f64(P_K[h])) > 0.98
+        assert _check_latent(gv[0, h], vn[0, h], f64(P_V[h])) > 0.98
+    q = si.queries_torch(seed + 3, B, Hq, d, dev)
+    got = gpu_decode(q, P_K, P_V, gk, gv, [L] * B)
+    ok_lat, ov_lat, olens, nbad = oracle.compress_append(
+        kn, vn, f64(P_K), f64(P_V), np.zeros((B, Hkv, L, rK)), np.zeros((B, Hkv, L, rV)),
+        np.zeros(B, np.int32))
+    assert nbad == 0 and olens.tolist() == [L] * B
+    want = oracle.decode(f64(q.cpu()), f64(P_K), f64(P_V), ok_lat, ov_lat, olens)
+    assert_decode_close(got, want)
