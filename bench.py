@@ -945,9 +945,18 @@ def run_profile_launches(args, w: si.Workload):
             vq = torch.randint(-127, 128, (w.B, w.Hkv, L8, lay.rV), generator=g, device=dev, dtype=torch.int8)
         ks = torch.rand((w.B, w.Hkv, L8), generator=g, device=dev) * 0.02
         vs = torch.rand((w.B, w.Hkv, L8), generator=g, device=dev) * 0.02
+    if args.joint:  # one joint value basis and one value latent per token (synthetic values)
+        js = si.sub_seed(w.seed, 14, 0, 0)
+        P_VJ = si.to_bf16(si.bases(js, 1, w.Hkv * w.d, lay.rV)[0]).to(dev)
+        v_joint = si.latent_cache_torch(js, w.B, 1, L_max, lay.rV, 1, dev)[:, 0].contiguous()
     for _ in range(args.profile_launches):
         lay.seq_lens.fill_(w.L - 1)
-        if args.int8:
+        if args.joint:
+            lay.seq_lens.fill_(w.L)
+            stief.stief_decode_attention_joint_v(q, lay.P_K, P_VJ, lay.k_lat, v_joint, lay.seq_lens,
+                                                 out, lay.ws, max_seq_len=L_max,
+                                                 num_splits=args.splits, dev_status=status)
+        elif args.int8:
             lay.seq_lens.fill_(w.L)
             (stief.stief_decode_attention_q4 if _int4(args) else stief.stief_decode_attention_q8)(q, lay.P_K, lay.P_V, kq, vq, ks, vs, lay.seq_lens, out,
                                             lay.ws, max_seq_len=L_max, num_splits=args.splits,
@@ -1075,8 +1084,8 @@ def main():
     if len(modes) > 1 and modes != ["latent", "joint"]:
         ap.error("--int8, --int4, --latent, --paged, --joint and --unfused are separate modes "
                  "(--latent --joint together time the latent joint-value decode)")
-    if (args.paged or args.joint) and args.profile_launches > 0:
-        ap.error("--profile-launches has no paged or joint mode")
+    if args.paged and args.profile_launches > 0:
+        ap.error("--profile-launches has no paged mode")
     w = si.WORKLOADS[args.workload]
     if args.int4:
         if any(rK % 32 or rV % 32 for rK, rV in w.layer_ranks()):
