@@ -22,6 +22,8 @@ from ._binding import (  # noqa: F401
     stief_decode_attention,
     stief_decode_attention_q8,
     stief_compress_append_q4,
+    stief_compress_append_q8_paged,
+    stief_decode_attention_q8_paged,
     stief_decode_attention_q4,
     stief_decode_attention_joint_v,
     stief_decode_attention_paged,

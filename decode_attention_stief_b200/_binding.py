@@ -89,6 +89,11 @@ def library() -> ctypes.CDLL:
             lib.stief_decode_attention_q8.restype = _i
             lib.stief_decode_attention_q8.argtypes = ([vp] * 10 + [ctypes.c_size_t] + [_i] * 9
                                                       + [vp, vp])
+            lib.stief_compress_append_q8_paged.restype = _i
+            lib.stief_compress_append_q8_paged.argtypes = [vp] * 10 + [_i] * 9 + [vp, vp]
+            lib.stief_decode_attention_q8_paged.restype = _i
+            lib.stief_decode_attention_q8_paged.argtypes = ([vp] * 11 + [ctypes.c_size_t] + [_i] * 11
+                                                            + [vp, vp])
             lib.stief_compress_append_q4.restype = _i
             lib.stief_compress_append_q4.argtypes = [vp] * 9 + [_i] * 7 + [vp, vp]
             lib.stief_decode_attention_q4.restype = _i
@@ -442,6 +447,79 @@ def stief_decode_attention_q8(q, P_K, P_V, k_q, v_q, k_s, v_s, seq_lens, out, wo
                                                rV, L_max, int(max_seq_len), int(num_splits),
                                                _opt_status(dev_status), _stream_ptr(stream))
     _check("stief_decode_attention_q8", code)
+    return out
+
+
+def stief_compress_append_q8_paged(k_new, v_new, P_K, P_V, k_pages, v_pages, k_s_pages,
+                                   v_s_pages, block_table, seq_lens,
+                                   dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """stief_compress_append into int8 page pools: codes k_pages [num_pages][Hkv][page_size][rK]
+    (int8) and row scales k_s_pages [num_pages][Hkv][page_size] (float32), likewise the values;
+    block_table [B][max_pages] int32."""
+    pk = _dev(k_new, "k_new", torch.bfloat16, 4)
+    pv = _dev(v_new, "v_new", torch.bfloat16, 4)
+    ppk = _dev(P_K, "P_K", torch.bfloat16, 3)
+    ppv = _dev(P_V, "P_V", torch.bfloat16, 3)
+    pkq = _dev(k_pages, "k_pages", torch.int8, 4)
+    pvq = _dev(v_pages, "v_pages", torch.int8, 4)
+    pks = _dev(k_s_pages, "k_s_pages", torch.float32, 3)
+    pvs = _dev(v_s_pages, "v_s_pages", torch.float32, 3)
+    pbt = _dev(block_table, "block_table", torch.int32, 2)
+    psl = _dev(seq_lens, "seq_lens", torch.int32, 1)
+    B, Hkv, T, d = k_new.shape
+    rK, rV = P_K.shape[2], P_V.shape[2]
+    num_pages, _, page_size, _ = k_pages.shape
+    max_pages = block_table.shape[1]
+    if tuple(v_new.shape) != (B, Hkv, T, d) or tuple(P_K.shape) != (Hkv, d, rK) \
+            or tuple(P_V.shape) != (Hkv, d, rV) \
+            or tuple(k_pages.shape) != (num_pages, Hkv, page_size, rK) \
+            or tuple(v_pages.shape) != (num_pages, Hkv, page_size, rV) \
+            or tuple(k_s_pages.shape) != (num_pages, Hkv, page_size) \
+            or tuple(v_s_pages.shape) != (num_pages, Hkv, page_size) \
+            or block_table.shape[0] != B or seq_lens.shape[0] != B:
+        raise ValueError("stief_compress_append_q8_paged: inconsistent shapes")
+    code = library().stief_compress_append_q8_paged(pk, pv, ppk, ppv, pkq, pvq, pks, pvs, pbt, psl,
+                                                    B, Hkv, T, d, rK, rV, num_pages, page_size,
+                                                    max_pages, _opt_status(dev_status),
+                                                    _stream_ptr(stream))
+    _check("stief_compress_append_q8_paged", code)
+
+
+def stief_decode_attention_q8_paged(q, P_K, P_V, k_pages, v_pages, k_s_pages, v_s_pages,
+                                    block_table, seq_lens, out, workspace, max_seq_len: int,
+                                    num_splits: int = 0,
+                                    dev_status: Optional[torch.Tensor] = None, stream=None):
+    """stief_decode_attention over int8 page pools (as for stief_compress_append_q8_paged)."""
+    pq = _dev(q, "q", torch.bfloat16, 3)
+    ppk = _dev(P_K, "P_K", torch.bfloat16, 3)
+    ppv = _dev(P_V, "P_V", torch.bfloat16, 3)
+    pkq = _dev(k_pages, "k_pages", torch.int8, 4)
+    pvq = _dev(v_pages, "v_pages", torch.int8, 4)
+    pks = _dev(k_s_pages, "k_s_pages", torch.float32, 3)
+    pvs = _dev(v_s_pages, "v_s_pages", torch.float32, 3)
+    pbt = _dev(block_table, "block_table", torch.int32, 2)
+    psl = _dev(seq_lens, "seq_lens", torch.int32, 1)
+    po = _dev(out, "out", torch.bfloat16, 3)
+    B, Hq, d = q.shape
+    Hkv, _, rK = P_K.shape
+    rV = P_V.shape[2]
+    num_pages, _, page_size, _ = k_pages.shape
+    max_pages = block_table.shape[1]
+    if tuple(P_V.shape) != (Hkv, d, rV) or tuple(k_pages.shape) != (num_pages, Hkv, page_size, rK) \
+            or tuple(v_pages.shape) != (num_pages, Hkv, page_size, rV) \
+            or tuple(k_s_pages.shape) != (num_pages, Hkv, page_size) \
+            or tuple(v_s_pages.shape) != (num_pages, Hkv, page_size) \
+            or block_table.shape[0] != B or seq_lens.shape[0] != B or tuple(out.shape) != (B, Hq, d):
+        raise ValueError("stief_decode_attention_q8_paged: inconsistent shapes")
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    code = library().stief_decode_attention_q8_paged(pq, ppk, ppv, pkq, pvq, pks, pvs, pbt, psl, po,
+                                                     workspace.data_ptr(), ws_bytes, B, Hq, Hkv, d,
+                                                     rK, rV, num_pages, page_size, max_pages,
+                                                     int(max_seq_len), int(num_splits),
+                                                     _opt_status(dev_status), _stream_ptr(stream))
+    _check("stief_decode_attention_q8_paged", code)
     return out
 
 

@@ -355,13 +355,14 @@ constexpr int kMaxConsumerWarps = 8;
 // joint value latents (one value row per token shared by the KV heads; full or latent output).
 // Each is its own instantiation, so a mode's branches cost the others nothing.
 constexpr int kModePlain = 0, kModeLatent = 1, kModePaged = 2, kModeQ8 = 3, kModeJointV = 4,
-              kModeLatentJointV = 5, kModeQ4 = 6;
+              kModeLatentJointV = 5, kModeQ4 = 6, kModePagedQ8 = 7;
 
 template <int NB, int NKS, int NMV, int TT, int MODE>
 __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
     stief_decode_kernel(const __grid_constant__ DecodeArgs a) {
   constexpr bool LAT = MODE == kModeLatent || MODE == kModeLatentJointV;
-  constexpr bool PG = MODE == kModePaged, Q8 = MODE == kModeQ8, Q4 = MODE == kModeQ4;
+  constexpr bool PG = MODE == kModePaged || MODE == kModePagedQ8;
+  constexpr bool Q8 = MODE == kModeQ8 || MODE == kModePagedQ8, Q4 = MODE == kModeQ4;
   constexpr bool QI = Q8 || Q4;  // integer codes with row scales
   constexpr bool JV = MODE == kModeJointV || MODE == kModeLatentJointV;
   constexpr int kTile = TT;
@@ -574,7 +575,8 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
   float skc[SJ], svc[SJ], skn[SJ], svn[SJ];
   auto load_scales = [&](int kk) {
     if (kk < warp_tiles(warp, n_tiles)) {
-      const long long row = cache_row(cr, b, kvh, t0 + (warp + kk * NW) * kTile) + lane;
+      // (a consumed tile lies below the length: its page is mapped and holds the whole tile)
+      const long long row = max(cache_row(cr, b, kvh, t0 + (warp + kk * NW) * kTile), 0ll) + lane;
 #pragma unroll
       for (int j = 0; j < SJ; ++j) {
         skn[j] = __ldg(a.k_scale + row + 32 * j);
@@ -1786,7 +1788,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
 template <int NB, int NKS, int NMV, int TT, int MODE>
 static cudaError_t launch_k(const DecodeArgs& a, cudaStream_t stream) {
   const DecodeSmem L = decode_smem_layout(a.nwarps, a.nstage, a.rK, a.rV, TT,
-                                          MODE == kModeQ8 ? 1 : MODE == kModeQ4 ? 2 : 0);
+                                          MODE == kModeQ8 || MODE == kModePagedQ8 ? 1 : MODE == kModeQ4 ? 2 : 0);
   auto kern = stief_decode_kernel<NB, NKS, NMV, TT, MODE>;
   static SmemLimit limit;
   cudaError_t e = limit.ensure(reinterpret_cast<const void*>(kern), a.device, (int)L.total);
@@ -1832,6 +1834,7 @@ cudaError_t launch_decode_latent(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_paged(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_q8(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_q4(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_decode_paged_q8(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_joint_v(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_latent_joint_v(const DecodeArgs& a, cudaStream_t stream);
 

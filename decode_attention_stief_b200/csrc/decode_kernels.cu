@@ -19,8 +19,10 @@ cudaError_t launch_decode(const DecodeArgs& planned, cudaStream_t stream) {
   // right after a compress of this library the new rows may still be in flight when this
   // kernel starts: no cache tile is requested before the dependency wait then
   a.early = take_stream_compress_mark(a.device, stream) ? 0 : 1;
+  if (a.block_table != nullptr && a.q8 != 0 && a.latent == 0 && a.q4 == 0 && a.append == 0)
+    return launch_decode_paged_q8(a, stream);  // int8 codes in page pools
   if ((a.latent != 0) + (a.block_table != nullptr) + (a.q8 != 0) + (a.q4 != 0) > 1)
-    return cudaErrorInvalidValue;  // the modes do not combine
+    return cudaErrorInvalidValue;  // the other modes do not combine
   if (a.joint_v) {
     if (a.block_table != nullptr || a.q8 != 0 || a.q4 != 0 || a.append != 0) return cudaErrorInvalidValue;
     return a.latent ? launch_decode_latent_joint_v(a, stream) : launch_decode_joint_v(a, stream);

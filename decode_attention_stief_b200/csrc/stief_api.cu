@@ -194,6 +194,26 @@ stief_status stief_compress_append_q8(const uint16_t* k_new, const uint16_t* v_n
                          dev_status, stream, Paging{}, k_s, v_s);
 }
 
+stief_status stief_compress_append_q8_paged(const uint16_t* k_new, const uint16_t* v_new,
+                                            const uint16_t* P_K, const uint16_t* P_V,
+                                            int8_t* k_pages, int8_t* v_pages, float* k_s_pages,
+                                            float* v_s_pages, const int32_t* block_table,
+                                            int32_t* seq_lens, int B, int Hkv, int T, int d,
+                                            int rK, int rV, int num_pages, int page_size,
+                                            int max_pages, uint32_t* dev_status,
+                                            stief_stream_t stream) {
+  Paging pg;
+  pg.block_table = block_table;
+  pg.num_pages = num_pages;
+  pg.page_size = page_size;
+  pg.max_pages = max_pages;
+  if (!block_table || !k_s_pages || !v_s_pages) return STIEF_ERR_INVALID_ARG;
+  if (!aligned16(k_s_pages) || !aligned16(v_s_pages)) return STIEF_ERR_ALIGNMENT;
+  return compress_common(k_new, v_new, P_K, P_V, reinterpret_cast<uint16_t*>(k_pages),
+                         reinterpret_cast<uint16_t*>(v_pages), seq_lens, B, Hkv, T, d, rK, rV, 0,
+                         dev_status, stream, pg, k_s_pages, v_s_pages);
+}
+
 stief_status stief_compress_append_q4(const uint16_t* k_new, const uint16_t* v_new,
                                       const uint16_t* P_K, const uint16_t* P_V, uint8_t* k_q,
                                       uint8_t* v_q, float* k_s, float* v_s, int32_t* seq_lens,
@@ -405,6 +425,31 @@ stief_status stief_decode_attention_q8(const uint16_t* q, const uint16_t* P_K,
                        const_cast<int32_t*>(seq_lens), out, workspace, workspace_bytes, B, Hq, Hkv,
                        d, rK, rV, L_max, max_seq_len, num_splits, dev_status, stream, false, false,
                        Paging{}, k_s, v_s);
+}
+
+stief_status stief_decode_attention_q8_paged(const uint16_t* q, const uint16_t* P_K,
+                                             const uint16_t* P_V, const int8_t* k_pages,
+                                             const int8_t* v_pages, const float* k_s_pages,
+                                             const float* v_s_pages, const int32_t* block_table,
+                                             const int32_t* seq_lens, uint16_t* out,
+                                             void* workspace, size_t workspace_bytes, int B,
+                                             int Hq, int Hkv, int d, int rK, int rV, int num_pages,
+                                             int page_size, int max_pages, int max_seq_len,
+                                             int num_splits, uint32_t* dev_status,
+                                             stief_stream_t stream) {
+  Paging pg;
+  pg.block_table = block_table;
+  pg.num_pages = num_pages;
+  pg.page_size = page_size;
+  pg.max_pages = max_pages;
+  if (!block_table || !k_s_pages || !v_s_pages) return STIEF_ERR_INVALID_ARG;
+  if (!aligned16(k_s_pages) || !aligned16(v_s_pages)) return STIEF_ERR_ALIGNMENT;
+  return decode_common(q, nullptr, nullptr, P_K, P_V,
+                       reinterpret_cast<uint16_t*>(const_cast<int8_t*>(k_pages)),
+                       reinterpret_cast<uint16_t*>(const_cast<int8_t*>(v_pages)),
+                       const_cast<int32_t*>(seq_lens), out, workspace, workspace_bytes, B, Hq, Hkv,
+                       d, rK, rV, 0, max_seq_len, num_splits, dev_status, stream, false, false, pg,
+                       k_s_pages, v_s_pages);
 }
 
 stief_status stief_decode_attention_q4(const uint16_t* q, const uint16_t* P_K,

@@ -359,7 +359,7 @@ STIEF_API stief_status stief_append_decode_paged(const uint16_t* q, const uint16
  * 2^-15 of its largest element) and each tile's softmax weights per head as 16-bit fixed point
  * of the tile's largest weight, each split into two 8-bit parts, so both products are exact
  * in 32-bit integers; the row scales multiply the scores and the weights.  Paged int8 caches
- * and the fused step are not provided.
+ * are the _q8_paged calls below; the fused step is not provided for int8 caches.
  */
 STIEF_API stief_status stief_compress_append_q8(const uint16_t* k_new, const uint16_t* v_new,
                                       const uint16_t* P_K, const uint16_t* P_V, int8_t* k_q,
@@ -375,6 +375,34 @@ STIEF_API stief_status stief_decode_attention_q8(const uint16_t* q, const uint16
                                        int rK, int rV, int L_max, int max_seq_len,
                                        int num_splits, uint32_t* dev_status,
                                        stief_stream_t stream);
+
+/*
+ * int8 caches in page pools: the int8 form above with the paged layout of the _paged calls.
+ *     k_pages : int8 [num_pages][Hkv][page_size][rK],  k_s_pages : float [num_pages][Hkv][page_size]
+ * (likewise v_pages, v_s_pages): token t of (sequence b, KV head h) is row t % page_size of page
+ * block_table[b][t / page_size], head h, in both the code and the scale pools.  page_size a
+ * multiple of 64; the capacity is max_pages * page_size.  Everything else is as for the
+ * _paged and _q8 calls.
+ */
+STIEF_API stief_status stief_compress_append_q8_paged(const uint16_t* k_new, const uint16_t* v_new,
+                                            const uint16_t* P_K, const uint16_t* P_V,
+                                            int8_t* k_pages, int8_t* v_pages, float* k_s_pages,
+                                            float* v_s_pages, const int32_t* block_table,
+                                            int32_t* seq_lens, int B, int Hkv, int T, int d,
+                                            int rK, int rV, int num_pages, int page_size,
+                                            int max_pages, uint32_t* dev_status,
+                                            stief_stream_t stream);
+
+STIEF_API stief_status stief_decode_attention_q8_paged(const uint16_t* q, const uint16_t* P_K,
+                                             const uint16_t* P_V, const int8_t* k_pages,
+                                             const int8_t* v_pages, const float* k_s_pages,
+                                             const float* v_s_pages, const int32_t* block_table,
+                                             const int32_t* seq_lens, uint16_t* out,
+                                             void* workspace, size_t workspace_bytes, int B,
+                                             int Hq, int Hkv, int d, int rK, int rV, int num_pages,
+                                             int page_size, int max_pages, int max_seq_len,
+                                             int num_splits, uint32_t* dev_status,
+                                             stief_stream_t stream);
 
 /*
  * 4-bit latent caches (the pages' other quantisation width; same per-row reading as the int8

@@ -274,3 +274,105 @@ def test_decode_q8_rows_past_length_hold_garbage(num_splits):
                       torch.nan_to_num(vs, 0.0, 0.0, 0.0), lens)
     assert_decode_close(got, want)
     assert torch.all(got[2].float() == 0)
+
+
+# ----------------------------------------------------------------------------- int8 page pools
+
+def _q8_pools(B, Hkv, rK, rV, page_size, max_pages, spare, rng):
+    num_pages = B * max_pages + spare
+    table = rng.permutation(num_pages)[: B * max_pages].reshape(B, max_pages).astype(np.int32)
+    kp = torch.full((num_pages, Hkv, page_size, rK), -128, dtype=torch.int8)
+    vp = torch.full((num_pages, Hkv, page_size, rV), -128, dtype=torch.int8)
+    ksp = torch.full((num_pages, Hkv, page_size), float("nan"), dtype=torch.float32)
+    vsp = torch.full((num_pages, Hkv, page_size), float("nan"), dtype=torch.float32)
+    return kp, vp, ksp, vsp, table
+
+
+def _fill(pool, table, cache, page_size, upto):
+    for b in range(table.shape[0]):
+        for j in range(table.shape[1]):
+            if j * page_size < upto[b]:
+                pool[table[b, j]] = cache[b, :, j * page_size:(j + 1) * page_size]
+
+
+def _decode_q8_paged(q, P_K, P_V, kp, vp, ksp, vsp, table, lens, max_seq_len, num_splits=0):
+    B, Hq, d = q.shape
+    out = torch.full((B, Hq, d), float("nan"), dtype=torch.bfloat16, device=DEV)
+    ws = stief.workspace_for(B, Hq, P_K.shape[0], P_V.shape[2], max_seq_len)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    stief.stief_decode_attention_q8_paged(q.to(DEV), P_K.to(DEV), P_V.to(DEV), kp.to(DEV), vp.to(DEV),
+                                          ksp.to(DEV), vsp.to(DEV), torch.as_tensor(table).to(DEV),
+                                          torch.as_tensor(np.asarray(lens, np.int32)).to(DEV), out, ws,
+                                          max_seq_len, num_splits=num_splits, dev_status=status)
+    assert stief.stief_read_device_status(status) == 0
+    return out.cpu()
+
+
+@pytest.mark.parametrize("page_size", [64, 128])
+@pytest.mark.parametrize("num_splits", [0, 3])
+def test_paged_q8_decode_matches_oracle(page_size, num_splits):
+    """int8 codes and scales in shuffled page pools (NaN scales and -128 codes in every unused
+    row): the decode over the pages equals the oracle's over the contiguous cache they stand
+    for; block-table entries past each sequence's pages are -1."""
+    rng = np.random.default_rng(8100 + page_size + num_splits)
+    B, Hq, Hkv, rK, rV = 3, 16, 4, 64, 32
+    max_pages = 1024 // page_size
+    Lc = page_size * max_pages
+    lens = [1000, 65, 0]
+    q = si.queries(8100, B, Hq, 128)
+    P_K, P_V = si.bases_bf16(8101, Hkv, 128, rK, rV)
+    kq, ks = _random_q8_cache(8102, B, Hkv, Lc, rK)
+    vq, vs = _random_q8_cache(8103, B, Hkv, Lc, rV)
+    kp, vp, ksp, vsp, table = _q8_pools(B, Hkv, rK, rV, page_size, max_pages, 3, rng)
+    for pool, cache in ((kp, kq), (vp, vq), (ksp, ks), (vsp, vs)):
+        _fill(pool, table, cache, page_size, lens)
+    for b in range(B):
+        table[b, -(-lens[b] // page_size):] = -1
+    got = _decode_q8_paged(q, P_K, P_V, kp, vp, ksp, vsp, table, lens, Lc, num_splits)
+    want = oracle.decode(f64(q), f64(P_K), f64(P_V), oracle.dequantize_rows(kq.numpy(), ks.numpy()),
+                         oracle.dequantize_rows(vq.numpy(), vs.numpy()), np.asarray(lens, np.int32))
+    assert_decode_close(got, want)
+    assert torch.all(got[2].float() == 0)
+
+
+@pytest.mark.parametrize("T", [5, 200])
+def test_paged_q8_compress_then_decode(T):
+    """Compress chunks into int8 page pools (CUDA-core path for T < 128, tensor cores above),
+    crossing pages, then decode over the pools; codes and scales equal the oracle's on the
+    identity basis and the decode matches the oracle."""
+    rng = np.random.default_rng(8200 + T)
+    B, Hq, Hkv, rK, rV, page_size, max_pages = 2, 8, 2, 64, 64, 64, 8
+    kp, vp, ksp, vsp, table = _q8_pools(B, Hkv, rK, rV, page_size, max_pages, 2, rng)
+    # the rows below the starting lengths are attended to: valid codes and scales everywhere
+    kp = torch.from_numpy(rng.integers(-127, 128, tuple(kp.shape), dtype=np.int8))
+    vp = torch.from_numpy(rng.integers(-127, 128, tuple(vp.shape), dtype=np.int8))
+    ksp = torch.from_numpy(rng.uniform(0.001, 0.02, tuple(ksp.shape)).astype(np.float32))
+    vsp = torch.from_numpy(rng.uniform(0.001, 0.02, tuple(vsp.shape)).astype(np.float32))
+    P_K, P_V = _identity_basis(Hkv, 128, rK), _identity_basis(Hkv, 128, rV)
+    gk, gv, gks, gvs = kp.to(DEV), vp.to(DEV), ksp.to(DEV), vsp.to(DEV)
+    gtab = torch.as_tensor(table).to(DEV)
+    glens = torch.as_tensor(np.asarray([10, 50], np.int32)).to(DEV)
+    k_new, v_new = si.full_kv(8200 + T, B, Hkv, T, 128)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    stief.stief_compress_append_q8_paged(k_new.to(DEV), v_new.to(DEV), P_K.to(DEV), P_V.to(DEV), gk,
+                                         gv, gks, gvs, gtab, glens, dev_status=status)
+    assert stief.stief_read_device_status(status) == 0
+    assert glens.cpu().tolist() == [10 + T, 50 + T]
+    for b, L0 in enumerate([10, 50]):
+        wk, wks = oracle.quantize_rows(f64(k_new[b])[..., :rK])
+        for t in range(T):
+            pg, row = table[b, (L0 + t) // page_size], (L0 + t) % page_size
+            assert np.array_equal(gk[pg, :, row].cpu().numpy(), wk[:, t])
+            assert np.array_equal(gks[pg, :, row].cpu().numpy(), wks[:, t])
+    q = si.queries(8201, B, Hq, 128)
+    lens = glens.cpu().tolist()
+    got = _decode_q8_paged(q, P_K, P_V, gk.cpu(), gv.cpu(), gks.cpu(), gvs.cpu(), table, lens,
+                           page_size * max_pages)
+    Lc = page_size * max_pages
+    kc = oracle.gather_pages(f64(gk.cpu()), table, lens, Lc)
+    kcs = oracle.gather_pages(f64(gks.cpu())[..., None], table, lens, Lc)[..., 0]
+    vc = oracle.gather_pages(f64(gv.cpu()), table, lens, Lc)
+    vcs = oracle.gather_pages(f64(gvs.cpu())[..., None], table, lens, Lc)[..., 0]
+    want = oracle.decode(f64(q), f64(P_K), f64(P_V), kc * kcs[..., None], vc * vcs[..., None],
+                         np.asarray(lens, np.int32))
+    assert_decode_close(got, want)
