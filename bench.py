@@ -474,6 +474,21 @@ def run_gpu(args, w: si.Workload):
         inp.copy_(h_inp, non_blocking=True)
         step(lays)
         h_out.copy_(out_all, non_blocking=True)
+
+    # the same step with prepared calls (stief.prepare: the binding's checks once per
+    # buffer set; every step still goes through the C entry points): what a serving loop
+    # that reuses its buffers runs
+    try:
+        prepared = [[stief.prepare(layer_step, li, lay) for li, lay in enumerate(lays)]
+                    for lays in reps]
+    except ValueError:  # a mode with more than one library call per layer
+        prepared = None
+
+    def e2e_step_prepared(r):
+        inp.copy_(h_inp, non_blocking=True)
+        for call in prepared[r]:
+            call()
+        h_out.copy_(out_all, non_blocking=True)
     n_dec = max(8, R) // R * R
     cap = torch.cuda.Stream(device=dev)
     cap.wait_stream(torch.cuda.current_stream())
@@ -606,7 +621,8 @@ def run_gpu(args, w: si.Workload):
         barrier()
         return e0_ev.elapsed_time(e1_ev) / K
 
-    e2e_api_ms = time_e2e(lambda j: e2e_step(reps[j % R]))
+    e2e_plain_ms = time_e2e(lambda j: e2e_step(reps[j % R]))
+    e2e_api_ms = time_e2e(lambda j: e2e_step_prepared(j % R)) if prepared is not None else e2e_plain_ms
     e2e_graph_ms = time_e2e(lambda j: e2e_graphs[j % R].replay())
     h2d = h_inp.numel() * h_inp.element_size()
     d2h = h_out.numel() * h_out.element_size()
@@ -614,8 +630,8 @@ def run_gpu(args, w: si.Workload):
     if st != 0:
         raise RuntimeError(f"device status {st:#x} after the e2e steps")
 
-    ms_per_step, e2e_api_ms, e2e_graph_ms, dec_us = reduce_over_ranks(
-        [ms_per_step, e2e_api_ms, e2e_graph_ms, dec_us], dev)
+    ms_per_step, e2e_api_ms, e2e_graph_ms, dec_us, e2e_plain_ms = reduce_over_ranks(
+        [ms_per_step, e2e_api_ms, e2e_graph_ms, dec_us, e2e_plain_ms], dev)
     del step_graphs, e2e_graphs, dec_graph, warm_graph, cycle_graph
 
     # ---- prefill compress (the prefill + batched decode workload): one 4096-token chunk
@@ -669,11 +685,15 @@ def run_gpu(args, w: si.Workload):
         "e2e": {"value": round(job_tokens_per_s(w.B, ws_n, e2e_api_ms), 2), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(e2e_api_ms, 6),
-                "how": "value: every step calls the public API from Python (ctypes into the C "
-                       "entry points) between one H2D copy of the step's inputs from pinned "
+                "how": "value: every step calls the public API from Python through prepared "
+                       "calls (stief.prepare: the binding's argument checks once per buffer "
+                       "set, then ctypes into the C entry points, which validate and plan on "
+                       "every call) between one H2D copy of the step's inputs from pinned "
                        "memory and one D2H copy of its outputs into pinned memory, CUDA events "
-                       "around the K steps; graph_value: the same step captured once in a CUDA "
-                       "graph, one replay per step",
+                       "around the K steps; unprepared_value: the same loop with the plain "
+                       "binding calls (checks on every call); graph_value: the step captured "
+                       "once in a CUDA graph, one replay per step",
+                "unprepared_value": round(job_tokens_per_s(w.B, ws_n, e2e_plain_ms), 2),
                 "graph_value": round(job_tokens_per_s(w.B, ws_n, e2e_graph_ms), 2),
                 "graph_ms_per_step": round(e2e_graph_ms, 6)},
         "gpu_launches": (3 if args.unfused and not args.latent else 1) * len(layers) * K,

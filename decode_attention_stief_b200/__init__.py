@@ -6,6 +6,7 @@ stream) into those calls.  There is no CPU fallback: if the library cannot be
 loaded, every call raises.
 """
 from ._binding import (  # noqa: F401
+    Prepared,
     StiefError,
     STATUS,
     DEV_CAPACITY_OVERFLOW,
@@ -13,6 +14,7 @@ from ._binding import (  # noqa: F401
     DEV_BAD_LENGTH,
     library,
     library_path,
+    prepare,
     stief_append_decode,
     stief_append_decode_paged,
     stief_compress_append,

@@ -125,6 +125,56 @@ def _check(func: str, code: int) -> None:
         raise StiefError(func, code)
 
 
+
+class Prepared:
+    """A library call validated once (see prepare): calling it launches the same call again with
+    the same device pointers, sizes and stream, at the C call's own host cost.  It keeps the
+    argument tensors alive; their storage, shapes and contents-to-be are the caller's to keep
+    as they were when it was prepared (in-place updates of their values are what it is for)."""
+
+    __slots__ = ("name", "_fn", "_cargs", "_keep")
+
+    def __init__(self, name, cargs, keep):
+        self.name = name
+        self._fn = getattr(library(), name)
+        self._cargs = cargs
+        self._keep = keep
+
+    def __call__(self):
+        code = self._fn(*self._cargs)
+        if code != 0:
+            raise StiefError(self.name, code)
+
+
+_capture = threading.local()
+
+
+def _invoke(name: str, cargs: tuple) -> None:
+    """Calls the library entry point `name` with the marshalled arguments, or, while prepare()
+    is capturing, records them instead."""
+    if getattr(_capture, "calls", None) is not None:
+        _capture.calls.append((name, cargs))
+        return
+    _check(name, getattr(library(), name)(*cargs))
+
+
+def prepare(fn, *args, **kwargs) -> Prepared:
+    """Validates and marshals the arguments of the binding function `fn` (e.g.
+    stief_append_decode) exactly as calling it would, without launching anything, and returns
+    a Prepared call: a serving loop that reuses the same buffers every step calls that object
+    instead, skipping the per-call checks (the library still validates sizes on every call).
+    The stream is the one given, or the current stream at preparation."""
+    _capture.calls = []
+    try:
+        fn(*args, **kwargs)
+        calls = _capture.calls
+    finally:
+        _capture.calls = None
+    if len(calls) != 1:
+        raise ValueError(f"{getattr(fn, '__name__', fn)} makes {len(calls)} library calls; prepare takes one")
+    name, cargs = calls[0]
+    return Prepared(name, cargs, (args, kwargs))
+
 def _stream_ptr(stream) -> int:
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -207,10 +257,9 @@ def stief_compress_append(k_new: torch.Tensor, v_new: torch.Tensor, P_K: torch.T
             or tuple(P_V.shape) != (Hkv, d, rV) or tuple(k_lat.shape) != (B, Hkv, L_max, rK) \
             or tuple(v_lat.shape) != (B, Hkv, L_max, rV) or seq_lens.shape[0] != B:
         raise ValueError("stief_compress_append: inconsistent shapes")
-    code = library().stief_compress_append(pk, pv, ppk, ppv, pkl, pvl, psl, B, Hkv, T, d, rK,
+    _invoke("stief_compress_append", (pk, pv, ppk, ppv, pkl, pvl, psl, B, Hkv, T, d, rK,
                                            rV, L_max, _opt_status(dev_status),
-                                           _stream_ptr(stream))
-    _check("stief_compress_append", code)
+                                           _stream_ptr(stream),))
 
 
 def stief_decode_attention(q: torch.Tensor, P_K: torch.Tensor, P_V: torch.Tensor,
@@ -244,11 +293,10 @@ def stief_decode_attention(q: torch.Tensor, P_K: torch.Tensor, P_V: torch.Tensor
             or tuple(out.shape) != (B, Hq, d):
         raise ValueError("stief_decode_attention: inconsistent shapes")
     ws_bytes = workspace.numel() * workspace.element_size()
-    code = library().stief_decode_attention(pq, ppk, ppv, pkl, pvl, psl, po,
+    _invoke("stief_decode_attention", (pq, ppk, ppv, pkl, pvl, psl, po,
                                             workspace.data_ptr(), ws_bytes, B, Hq, Hkv, d, rK,
                                             rV, L_max, int(max_seq_len), int(num_splits),
-                                            _opt_status(dev_status), _stream_ptr(stream))
-    _check("stief_decode_attention", code)
+                                            _opt_status(dev_status), _stream_ptr(stream),))
     return out
 
 
@@ -288,11 +336,10 @@ def stief_append_decode(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tenso
             or tuple(out.shape) != (B, Hq, d):
         raise ValueError("stief_append_decode: inconsistent shapes")
     ws_bytes = workspace.numel() * workspace.element_size()
-    code = library().stief_append_decode(pq, pkn, pvn, ppk, ppv, pkl, pvl, psl, po,
+    _invoke("stief_append_decode", (pq, pkn, pvn, ppk, ppv, pkl, pvl, psl, po,
                                          workspace.data_ptr(), ws_bytes, B, Hq, Hkv, d, rK, rV,
                                          L_max, int(max_seq_len), int(num_splits),
-                                         _opt_status(dev_status), _stream_ptr(stream))
-    _check("stief_append_decode", code)
+                                         _opt_status(dev_status), _stream_ptr(stream),))
     return out
 
 
@@ -324,10 +371,9 @@ def stief_compress_append_paged(k_new, v_new, P_K, P_V, k_pages, v_pages, block_
     if Hkv2 != Hkv or tuple(P_K.shape) != (Hkv, d, rK) or tuple(P_V.shape) != (Hkv, d, rV) \
             or tuple(v_new.shape) != (B, Hkv, T, d) or seq_lens.shape[0] != B:
         raise ValueError("stief_compress_append_paged: inconsistent shapes")
-    code = library().stief_compress_append_paged(pk, pv, ppk, ppv, pkp, pvp, pbt, psl, B, Hkv, T,
+    _invoke("stief_compress_append_paged", (pk, pv, ppk, ppv, pkp, pvp, pbt, psl, B, Hkv, T,
                                                  d, rK, rV, num_pages, page_size, max_pages,
-                                                 _opt_status(dev_status), _stream_ptr(stream))
-    _check("stief_compress_append_paged", code)
+                                                 _opt_status(dev_status), _stream_ptr(stream),))
 
 
 def stief_decode_attention_paged(q, P_K, P_V, k_pages, v_pages, block_table, seq_lens, out,
@@ -348,12 +394,11 @@ def stief_decode_attention_paged(q, P_K, P_V, k_pages, v_pages, block_table, seq
     if not workspace.is_cuda or not workspace.is_contiguous():
         raise ValueError("workspace must be a contiguous CUDA tensor")
     ws_bytes = workspace.numel() * workspace.element_size()
-    code = library().stief_decode_attention_paged(pq, ppk, ppv, pkp, pvp, pbt, psl, po,
+    _invoke("stief_decode_attention_paged", (pq, ppk, ppv, pkp, pvp, pbt, psl, po,
                                                   workspace.data_ptr(), ws_bytes, B, Hq, Hkv, d,
                                                   rK, rV, num_pages, page_size, max_pages,
                                                   int(max_seq_len), int(num_splits),
-                                                  _opt_status(dev_status), _stream_ptr(stream))
-    _check("stief_decode_attention_paged", code)
+                                                  _opt_status(dev_status), _stream_ptr(stream),))
     return out
 
 
@@ -380,12 +425,11 @@ def stief_append_decode_paged(q, k_new, v_new, P_K, P_V, k_pages, v_pages, block
     if not workspace.is_cuda or not workspace.is_contiguous():
         raise ValueError("workspace must be a contiguous CUDA tensor")
     ws_bytes = workspace.numel() * workspace.element_size()
-    code = library().stief_append_decode_paged(pq, pkn, pvn, ppk, ppv, pkp, pvp, pbt, psl, po,
+    _invoke("stief_append_decode_paged", (pq, pkn, pvn, ppk, ppv, pkp, pvp, pbt, psl, po,
                                                workspace.data_ptr(), ws_bytes, B, Hq, Hkv, d, rK,
                                                rV, num_pages, page_size, max_pages,
                                                int(max_seq_len), int(num_splits),
-                                               _opt_status(dev_status), _stream_ptr(stream))
-    _check("stief_append_decode_paged", code)
+                                               _opt_status(dev_status), _stream_ptr(stream),))
     return out
 
 
@@ -410,10 +454,9 @@ def stief_compress_append_q8(k_new, v_new, P_K, P_V, k_q, v_q, k_s, v_s, seq_len
             or tuple(v_q.shape) != (B, Hkv, L_max, rV) or tuple(k_s.shape) != (B, Hkv, L_max) \
             or tuple(v_s.shape) != (B, Hkv, L_max) or seq_lens.shape[0] != B:
         raise ValueError("stief_compress_append_q8: inconsistent shapes")
-    code = library().stief_compress_append_q8(pk, pv, ppk, ppv, pkq, pvq, pks, pvs, psl, B, Hkv, T,
+    _invoke("stief_compress_append_q8", (pk, pv, ppk, ppv, pkq, pvq, pks, pvs, psl, B, Hkv, T,
                                               d, rK, rV, L_max, _opt_status(dev_status),
-                                              _stream_ptr(stream))
-    _check("stief_compress_append_q8", code)
+                                              _stream_ptr(stream),))
 
 
 def stief_decode_attention_q8(q, P_K, P_V, k_q, v_q, k_s, v_s, seq_lens, out, workspace,
@@ -442,11 +485,10 @@ def stief_decode_attention_q8(q, P_K, P_V, k_q, v_q, k_s, v_s, seq_lens, out, wo
     if not workspace.is_cuda or not workspace.is_contiguous():
         raise ValueError("workspace must be a contiguous CUDA tensor")
     ws_bytes = workspace.numel() * workspace.element_size()
-    code = library().stief_decode_attention_q8(pq, ppk, ppv, pkq, pvq, pks, pvs, psl, po,
+    _invoke("stief_decode_attention_q8", (pq, ppk, ppv, pkq, pvq, pks, pvs, psl, po,
                                                workspace.data_ptr(), ws_bytes, B, Hq, Hkv, d, rK,
                                                rV, L_max, int(max_seq_len), int(num_splits),
-                                               _opt_status(dev_status), _stream_ptr(stream))
-    _check("stief_decode_attention_q8", code)
+                                               _opt_status(dev_status), _stream_ptr(stream),))
     return out
 
 
@@ -478,11 +520,10 @@ def stief_compress_append_q8_paged(k_new, v_new, P_K, P_V, k_pages, v_pages, k_s
             or tuple(v_s_pages.shape) != (num_pages, Hkv, page_size) \
             or block_table.shape[0] != B or seq_lens.shape[0] != B:
         raise ValueError("stief_compress_append_q8_paged: inconsistent shapes")
-    code = library().stief_compress_append_q8_paged(pk, pv, ppk, ppv, pkq, pvq, pks, pvs, pbt, psl,
+    _invoke("stief_compress_append_q8_paged", (pk, pv, ppk, ppv, pkq, pvq, pks, pvs, pbt, psl,
                                                     B, Hkv, T, d, rK, rV, num_pages, page_size,
                                                     max_pages, _opt_status(dev_status),
-                                                    _stream_ptr(stream))
-    _check("stief_compress_append_q8_paged", code)
+                                                    _stream_ptr(stream),))
 
 
 def stief_decode_attention_q8_paged(q, P_K, P_V, k_pages, v_pages, k_s_pages, v_s_pages,
@@ -514,12 +555,11 @@ def stief_decode_attention_q8_paged(q, P_K, P_V, k_pages, v_pages, k_s_pages, v_
     if not workspace.is_cuda or not workspace.is_contiguous():
         raise ValueError("workspace must be a contiguous CUDA tensor")
     ws_bytes = workspace.numel() * workspace.element_size()
-    code = library().stief_decode_attention_q8_paged(pq, ppk, ppv, pkq, pvq, pks, pvs, pbt, psl, po,
+    _invoke("stief_decode_attention_q8_paged", (pq, ppk, ppv, pkq, pvq, pks, pvs, pbt, psl, po,
                                                      workspace.data_ptr(), ws_bytes, B, Hq, Hkv, d,
                                                      rK, rV, num_pages, page_size, max_pages,
                                                      int(max_seq_len), int(num_splits),
-                                                     _opt_status(dev_status), _stream_ptr(stream))
-    _check("stief_decode_attention_q8_paged", code)
+                                                     _opt_status(dev_status), _stream_ptr(stream),))
     return out
 
 
@@ -545,10 +585,9 @@ def stief_compress_append_q4(k_new, v_new, P_K, P_V, k_q, v_q, k_s, v_s, seq_len
             or tuple(v_q.shape) != (B, Hkv, L_max, rV // 2) or tuple(k_s.shape) != (B, Hkv, L_max) \
             or tuple(v_s.shape) != (B, Hkv, L_max) or seq_lens.shape[0] != B:
         raise ValueError("stief_compress_append_q4: inconsistent shapes")
-    code = library().stief_compress_append_q4(pk, pv, ppk, ppv, pkq, pvq, pks, pvs, psl, B, Hkv, T,
+    _invoke("stief_compress_append_q4", (pk, pv, ppk, ppv, pkq, pvq, pks, pvs, psl, B, Hkv, T,
                                               d, rK, rV, L_max, _opt_status(dev_status),
-                                              _stream_ptr(stream))
-    _check("stief_compress_append_q4", code)
+                                              _stream_ptr(stream),))
 
 
 def stief_decode_attention_q4(q, P_K, P_V, k_q, v_q, k_s, v_s, seq_lens, out, workspace,
@@ -577,11 +616,10 @@ def stief_decode_attention_q4(q, P_K, P_V, k_q, v_q, k_s, v_s, seq_lens, out, wo
     if not workspace.is_cuda or not workspace.is_contiguous():
         raise ValueError("workspace must be a contiguous CUDA tensor")
     ws_bytes = workspace.numel() * workspace.element_size()
-    code = library().stief_decode_attention_q4(pq, ppk, ppv, pkq, pvq, pks, pvs, psl, po,
+    _invoke("stief_decode_attention_q4", (pq, ppk, ppv, pkq, pvq, pks, pvs, psl, po,
                                                workspace.data_ptr(), ws_bytes, B, Hq, Hkv, d, rK,
                                                rV, L_max, int(max_seq_len), int(num_splits),
-                                               _opt_status(dev_status), _stream_ptr(stream))
-    _check("stief_decode_attention_q4", code)
+                                               _opt_status(dev_status), _stream_ptr(stream),))
     return out
 
 
@@ -610,11 +648,10 @@ def stief_decode_latent(q_lat: torch.Tensor, k_lat: torch.Tensor, v_lat: torch.T
             or seq_lens.shape[0] != B or tuple(out_lat.shape) != (B, Hq, rV):
         raise ValueError("stief_decode_latent: inconsistent shapes")
     ws_bytes = workspace.numel() * workspace.element_size()
-    code = library().stief_decode_latent(pq, pkl, pvl, psl, po, workspace.data_ptr(), ws_bytes,
+    _invoke("stief_decode_latent", (pq, pkl, pvl, psl, po, workspace.data_ptr(), ws_bytes,
                                          B, Hq, Hkv, int(d), rK, rV, L_max, int(max_seq_len),
                                          int(num_splits), _opt_status(dev_status),
-                                         _stream_ptr(stream))
-    _check("stief_decode_latent", code)
+                                         _stream_ptr(stream),))
     return out_lat
 
 
@@ -645,11 +682,10 @@ def stief_decode_attention_noalloc(q: torch.Tensor, P_K: torch.Tensor, P_V: torc
             or tuple(v_lat.shape) != (B, Hkv, L_max, rV) or seq_lens.shape[0] != B \
             or tuple(out.shape) != (B, Hq, d):
         raise ValueError("stief_decode_attention_noalloc: inconsistent shapes")
-    code = library().stief_decode_attention_noalloc(pq, ppk, ppv, pkl, pvl, psl, po, B, Hq, Hkv,
+    _invoke("stief_decode_attention_noalloc", (pq, ppk, ppv, pkl, pvl, psl, po, B, Hq, Hkv,
                                                     d, rK, rV, L_max, int(max_seq_len),
                                                     int(num_splits), _opt_status(dev_status),
-                                                    _stream_ptr(stream))
-    _check("stief_decode_attention_noalloc", code)
+                                                    _stream_ptr(stream),))
     return out
 
 
@@ -691,12 +727,11 @@ def stief_decode_attention_joint_v(q: torch.Tensor, P_K: torch.Tensor, P_VJ: tor
             or tuple(out.shape) != (B, Hq, d):
         raise ValueError("stief_decode_attention_joint_v: inconsistent shapes")
     ws_bytes = workspace.numel() * workspace.element_size()
-    code = library().stief_decode_attention_joint_v(pq, ppk, ppv, pkl, pvl, psl, po,
+    _invoke("stief_decode_attention_joint_v", (pq, ppk, ppv, pkl, pvl, psl, po,
                                                     workspace.data_ptr(), ws_bytes, B, Hq, Hkv, d,
                                                     rK, rV, L_max, int(max_seq_len),
                                                     int(num_splits), _opt_status(dev_status),
-                                                    _stream_ptr(stream))
-    _check("stief_decode_attention_joint_v", code)
+                                                    _stream_ptr(stream),))
     return out
 
 
@@ -721,11 +756,10 @@ def stief_decode_latent_joint_v(q_lat: torch.Tensor, k_lat: torch.Tensor, v_join
             or seq_lens.shape[0] != B or tuple(out_lat.shape) != (B, Hq, rV):
         raise ValueError("stief_decode_latent_joint_v: inconsistent shapes")
     ws_bytes = workspace.numel() * workspace.element_size()
-    code = library().stief_decode_latent_joint_v(pq, pkl, pvl, psl, po, workspace.data_ptr(),
+    _invoke("stief_decode_latent_joint_v", (pq, pkl, pvl, psl, po, workspace.data_ptr(),
                                                  ws_bytes, B, Hq, Hkv, int(d), rK, rV, L_max,
                                                  int(max_seq_len), int(num_splits),
-                                                 _opt_status(dev_status), _stream_ptr(stream))
-    _check("stief_decode_latent_joint_v", code)
+                                                 _opt_status(dev_status), _stream_ptr(stream),))
     return out_lat
 
 
@@ -750,7 +784,6 @@ def stief_compress_append_joint_v(k_new: torch.Tensor, v_new: torch.Tensor, P_K:
             or tuple(P_VJ.shape) != (Hkv * d, rV) or tuple(k_lat.shape) != (B, Hkv, L_max, rK) \
             or tuple(v_joint.shape) != (B, L_max, rV) or seq_lens.shape[0] != B:
         raise ValueError("stief_compress_append_joint_v: inconsistent shapes")
-    code = library().stief_compress_append_joint_v(pk, pv, ppk, ppv, pkl, pvl, psl, B, Hkv, T, d,
+    _invoke("stief_compress_append_joint_v", (pk, pv, ppk, ppv, pkl, pvl, psl, B, Hkv, T, d,
                                                    rK, rV, L_max, _opt_status(dev_status),
-                                                   _stream_ptr(stream))
-    _check("stief_compress_append_joint_v", code)
+                                                   _stream_ptr(stream),))

@@ -255,3 +255,15 @@ def test_workspace_bytes():
     assert stief.stief_decode_workspace_bytes(64, 32, 8, 64, 4096) == 2304 + 512 * 4 * 32 * 130 * 8
     assert stief.stief_decode_workspace_bytes(1, 32, 8, 72, 100) == 0
     assert stief.stief_decode_workspace_bytes(1, 30, 8, 64, 100) == 0
+
+
+def test_prepare_validates_like_the_call():
+    """stief.prepare runs the binding function's own checks (no launch): a CPU tensor is
+    refused with the same error as the direct call, and the capture state is cleared after."""
+    import torch
+    import decode_attention_stief_b200 as stief
+    from decode_attention_stief_b200 import _binding
+    q = torch.zeros(1, 4, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="q must be on a CUDA device"):
+        stief.prepare(stief.stief_decode_attention, q, None, None, None, None, None, None, None, 0)
+    assert getattr(_binding._capture, "calls", None) is None

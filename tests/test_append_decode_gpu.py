@@ -14,7 +14,7 @@ import torch
 import decode_attention_stief_b200 as stief
 import oracle
 import stief_inputs as si
-from gpu_util import DECODE_TOL, bf16_ulp, decode_error, f64
+from gpu_util import DECODE_TOL, bf16_ulp, decode_error, f64, make_decode_case
 
 pytestmark = pytest.mark.gpu
 
@@ -240,3 +240,37 @@ def test_back_to_back_steps_without_host_sync(num_splits):
     assert lens_t.cpu().tolist() == wl.tolist() == [L + 5 for L in lens]
     want_l = oracle.decode_latent(f64(q_lat), wk, wv, wl, d=128)
     assert decode_error(o_lat.cpu(), want_l) <= DECODE_TOL
+
+
+def test_prepared_call_matches_direct_calls():
+    """stief.prepare(stief_append_decode, ...) validates once; calling the prepared object
+    repeats the same launch.  Three prepared steps and three direct steps on twin caches give
+    identical outputs, caches and lengths."""
+    B, Hq, Hkv, d, rK, rV, L_max = 2, 16, 4, 128, 64, 64, 512
+    dev = torch.device("cuda")
+    q, P_K, P_V, k_lat, v_lat = make_decode_case(B, Hq, Hkv, rK, rV, L_max, 9100)
+    q, P_K, P_V = q.to(dev), P_K.to(dev), P_V.to(dev)
+    caches = [(k_lat.to(dev).clone(), v_lat.to(dev).clone(),
+               torch.tensor([300, 41], dtype=torch.int32, device=dev)) for _ in range(2)]
+    kn = torch.empty((B, Hkv, d), dtype=torch.bfloat16, device=dev)
+    vn = torch.empty_like(kn)
+    outs = [torch.empty((B, Hq, d), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    ws = [stief.workspace_for(B, Hq, Hkv, rV, L_max) for _ in range(2)]
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    kl, vl, lens = caches[0]
+    prepared = stief.prepare(stief.stief_append_decode, q, kn, vn, P_K, P_V, kl, vl, lens, outs[0],
+                             ws[0], max_seq_len=L_max, dev_status=status)
+    assert isinstance(prepared, stief.Prepared) and prepared.name == "stief_append_decode"
+    g = torch.Generator(device=dev)
+    g.manual_seed(9101)
+    for step in range(3):
+        kn.copy_(torch.randn((B, Hkv, d), generator=g, device=dev).to(torch.bfloat16))
+        vn.copy_(torch.randn((B, Hkv, d), generator=g, device=dev).to(torch.bfloat16))
+        prepared()
+        kl2, vl2, lens2 = caches[1]
+        stief.stief_append_decode(q, kn, vn, P_K, P_V, kl2, vl2, lens2, outs[1], ws[1],
+                                  max_seq_len=L_max, dev_status=status)
+        assert torch.equal(outs[0], outs[1])
+    assert stief.stief_read_device_status(status) == 0
+    assert torch.equal(caches[0][2], caches[1][2]) and caches[0][2].tolist() == [303, 44]
+    assert torch.equal(caches[0][0], caches[1][0]) and torch.equal(caches[0][1], caches[1][1])
