@@ -800,9 +800,9 @@ def workload_roofline(args, name: str, dev) -> dict:
 
 def time_prefill_compress(args, n_layers: int, dev, stream):
     """Time stief_compress_append of one prefill chunk (B=1, Hkv=8, T=4096, ranks 64/64)
-    for every layer.  Each layer has its own chunk and cache (the chunks of all layers,
-    537 MB, exceed L2, so every layer's chunk streams from HBM without a flush).  Returns
-    a summary dict."""
+    for every layer, then stief_compress_append_joint_v of the same chunks.  Each layer has
+    its own chunk and cache (the chunks of all layers, 537 MB, exceed L2, so every layer's
+    chunk streams from HBM without a flush).  Returns a summary dict."""
     import decode_attention_stief_b200 as stief
     c = si.PREFILL_CHUNK
     B, Hkv, T, d, rK, rV = c["B"], c["Hkv"], c["T"], c["d"], c["rK"], c["rV"]
@@ -820,44 +820,69 @@ def time_prefill_compress(args, n_layers: int, dev, stream):
         for li in range(n_layers):
             stief.stief_compress_append(ks[li], vs[li], P_K, P_V, kl[li], vl[li], lens[li])
 
-    for _ in range(args.warmup):
-        lens.zero_()
-        chunk()
-    # the calls of all layers captured in one CUDA graph: the timing is the device's, not
-    # the host's launch rate
-    torch.cuda.synchronize()
-    cap = torch.cuda.Stream(device=dev)
-    cap.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(cap):
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph, stream=cap):
-            chunk()
-    torch.cuda.synchronize()
-    reps = max(3, min(args.steps, 20))
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(reps)]
-    for r in range(reps):
-        lens.zero_()  # every replay appends each layer's chunk to an empty cache
-        _backlog()
-        evs[r][0].record(stream)
-        graph.replay()
-        evs[r][1].record(stream)
-    torch.cuda.synchronize()
-    del graph
-    ms = sorted(a.elapsed_time(b) for a, b in evs)
-    ms_med = ms[len(ms) // 2]
+    def timed(fn):
+        """Median device time (ms) of one graph replay of fn over every layer."""
+        for _ in range(args.warmup):
+            lens.zero_()
+            fn()
+        # the calls of all layers captured in one CUDA graph: the timing is the device's, not
+        # the host's launch rate
+        torch.cuda.synchronize()
+        cap = torch.cuda.Stream(device=dev)
+        cap.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(cap):
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=cap):
+                fn()
+        torch.cuda.synchronize()
+        reps = max(3, min(args.steps, 20))
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(reps)]
+        for r in range(reps):
+            lens.zero_()  # every replay appends each layer's chunk to an empty cache
+            _backlog()
+            evs[r][0].record(stream)
+            graph.replay()
+            evs[r][1].record(stream)
+        torch.cuda.synchronize()
+        del graph
+        ms = sorted(a.elapsed_time(b) for a, b in evs)
+        return ms[len(ms) // 2]
+
+    peak, kind = _hbm_peak()
+
+    def summary(ms_med, bytes_moved, flops):
+        return {"us_total": round(ms_med * 1e3, 2), "us_per_layer": round(ms_med * 1e3 / n_layers, 3),
+                "algorithmic_bytes": bytes_moved,
+                "GBs": round(bytes_moved / (ms_med / 1e3) / 1e9, 1),
+                "frac_of_hbm_peak": round(bytes_moved / (ms_med / 1e3) / 1e9 / peak, 4),
+                "TFLOPs": round(flops / (ms_med / 1e3) / 1e12, 2),
+                "kernel_launches_per_layer": 2}
+
+    ms_med = timed(chunk)
     bytes_moved = n_layers * B * Hkv * T * (2 * d * 2 + 2 * (rK + rV))
     flops = n_layers * B * Hkv * T * 2 * d * (rK + rV)
-    peak, kind = _hbm_peak()
-    return {"what": f"stief_compress_append of a {T}-token chunk, {Hkv} KV heads, ranks {rK}/{rV}, "
-                    f"x{n_layers} layers (tcgen05 path), per-layer chunks (537 MB in all) stream from HBM; "
-                    f"the calls of all layers replayed from one CUDA graph",
-            "us_total": round(ms_med * 1e3, 2), "us_per_layer": round(ms_med * 1e3 / n_layers, 3),
-            "algorithmic_bytes": bytes_moved,
-            "GBs": round(bytes_moved / (ms_med / 1e3) / 1e9, 1),
-            "frac_of_hbm_peak": round(bytes_moved / (ms_med / 1e3) / 1e9 / peak, 4),
-            "TFLOPs": round(flops / (ms_med / 1e3) / 1e12, 2),
-            "kernel_launches_per_layer": 2}
+    out = {"what": f"stief_compress_append of a {T}-token chunk, {Hkv} KV heads, ranks {rK}/{rV}, "
+                   f"x{n_layers} layers (tcgen05 path), per-layer chunks (537 MB in all) stream from HBM; "
+                   f"the calls of all layers replayed from one CUDA graph"}
+    out.update(summary(ms_med, bytes_moved, flops))
+
+    # the same chunks into joint value latents (keys per head, one value row per token over
+    # the concatenated heads: a K = Hkv*d contraction), through stief_compress_append_joint_v
+    P_VJ = si.to_bf16(si.bases(c["seed"] + 7, 1, Hkv * d, rV)[0]).to(dev)
+    vj = [torch.empty((B, T, rV), dtype=torch.bfloat16, device=dev) for _ in range(n_layers)]
+
+    def chunk_joint():
+        for li in range(n_layers):
+            stief.stief_compress_append_joint_v(ks[li], vs[li], P_K, P_VJ, kl[li], vj[li], lens[li])
+
+    ms_joint = timed(chunk_joint)
+    bytes_joint = n_layers * B * T * (Hkv * (2 * d * 2 + 2 * rK) + 2 * rV)
+    out["joint"] = {"what": f"stief_compress_append_joint_v of the same chunks (joint value basis "
+                            f"[{Hkv * d}][{rV}], tcgen05 path)"}
+    out["joint"].update(summary(ms_joint, bytes_joint, flops))
+    del vj
+    return out
 
 
 # ----------------------------------------------------------------------------- CPU oracle

@@ -12,6 +12,9 @@
 //                                  the columns) from L2.
 //   stief_joint_lens_kernel     -- the length update, launched after the projection in stream
 //                                  order (every projection block has read the old lengths).
+// Prefill-sized chunks (T >= 128) go to the tcgen05 projection instead
+// (stief_compress_joint_tc_kernel, compress_joint_tc.cu) when its shared memory holds the
+// whole joint basis, followed by the compress length kernel as a programmatic dependent.
 //
 // Every store is checked against the size of its tensor and skipped (reported as a capacity
 // overflow) if it would fall outside; with valid lengths that never happens.
@@ -25,6 +28,7 @@ namespace stief {
 constexpr int kJointRows = 8;       // new tokens per block
 constexpr int kJointThreads = 128;  // one thread per output column (r <= 128)
 constexpr int kJointChunk = 256;    // reduction elements staged per pass
+constexpr int kJointTensorCoreMinRows = 128;  // T from which the tcgen05 path is used
 
 __global__ void __launch_bounds__(kJointThreads) stief_compress_joint_kernel(const CompressArgs a) {
   __shared__ float xs[kJointRows][kJointChunk];
@@ -96,6 +100,14 @@ __global__ void __launch_bounds__(256) stief_joint_lens_kernel(const CompressArg
 }
 
 cudaError_t launch_compress_joint(const CompressArgs& a, cudaStream_t stream) {
+  if (a.T >= kJointTensorCoreMinRows && compress_joint_tc_fits(a.Hkv, a.rK, a.rV)) {
+    cudaError_t e = launch_compress_joint_tc(a, stream);
+    if (e == cudaSuccess) e = launch_seq_lens(a, stream);
+    // the length kernel lets its dependents start early: a decode that follows must not
+    // request cache tiles before its dependency wait
+    if (e == cudaSuccess) mark_stream_compress(a.device, stream, true);
+    return e;
+  }
   const dim3 grid((a.T + kJointRows - 1) / kJointRows, a.Hkv + 1, a.B);
   stief_compress_joint_kernel<<<grid, kJointThreads, 0, stream>>>(a);
   cudaError_t e = cudaGetLastError();

@@ -152,7 +152,7 @@ __global__ void __launch_bounds__(256) stief_seq_lens_kernel(const CompressArgs 
   }
 }
 
-static cudaError_t launch_seq_lens(const CompressArgs& a, cudaStream_t stream) {
+cudaError_t launch_seq_lens(const CompressArgs& a, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((a.B + 255) / 256);
   cfg.blockDim = dim3(256);

@@ -31,12 +31,13 @@
 
 #include "stief_device.cuh"
 #include "stief_internal.h"
+#include "umma.cuh"
 
 namespace stief {
 
 namespace {
 
-constexpr int kTcRows = 128;     // M: rows (tokens) per MMA tile
+constexpr int kTcRows = kUmmaRows;  // M: rows (tokens) per MMA tile
 constexpr int kTcStages = 2;     // X tiles in flight per CTA
 // 8 warps: warp w reads TMEM lanes 32 (w & 3) .. + 31 (rows), the keys' columns for w < 4 and
 // the values' for w >= 4
@@ -69,61 +70,6 @@ __host__ __device__ inline TcSmem tc_smem_layout(int rK, int rV) {
   off += 16;
   s.total = off;
   return s;
-}
-
-// UMMA shared-memory descriptor: K-major, 128-byte swizzle, 8-row groups 1024 B apart.
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_addr) {
-  uint64_t d = 0;
-  d |= (uint64_t)((smem_addr >> 4) & 0x3FFFu);  // start address
-  d |= (uint64_t)1u << 16;                      // leading byte offset (unused for swizzled K-major)
-  d |= (uint64_t)(1024u >> 4) << 32;            // stride byte offset
-  d |= (uint64_t)1u << 46;                      // descriptor version (sm_100)
-  d |= (uint64_t)2u << 61;                      // layout: 128-byte swizzle
-  return d;
-}
-
-// Instruction descriptor: bf16 x bf16 -> fp32, A and B K-major, M = 128, N = n.
-__device__ __forceinline__ uint32_t idesc_bf16_f32(int n) {
-  return (1u << 4)                      // D format: f32
-         | (1u << 7)                    // A format: bf16
-         | (1u << 10)                   // B format: bf16
-         | ((uint32_t)(n >> 3) << 17)   // N / 8
-         | ((uint32_t)(kTcRows >> 4) << 24);  // M / 16
-}
-
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
-                                          uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   smem_u32(bar))
-               : "memory");
-}
-
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, "
-      "[%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_wait_ld() {
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
 // P[h] ([128][r] row-major in global) -> shared [r rows][128 k] K-major SW128, two atoms.

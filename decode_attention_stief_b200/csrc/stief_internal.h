@@ -235,5 +235,12 @@ uint32_t test_stall_bytes();
 // Joint value latents: keys per head into k_lat, the values of all KV heads of a token
 // through P_V = P_VJ [Hkv*d][rV] into v_lat = v_joint [B][L_max][rV]; then the lengths.
 cudaError_t launch_compress_joint(const CompressArgs& a, cudaStream_t stream);
+// The length update seq_lens[b] += T of a compress (contiguous or paged rows), launched as a
+// programmatic dependent of the projection; it lets its own dependents start early.
+cudaError_t launch_seq_lens(const CompressArgs& a, cudaStream_t stream);
+// The tcgen05 joint-value projection of prefill-sized chunks (d = 128), and whether its
+// shared memory (the whole joint basis plus a ring of at least two input chunks) fits.
+bool compress_joint_tc_fits(int Hkv, int rK, int rV);
+cudaError_t launch_compress_joint_tc(const CompressArgs& a, cudaStream_t stream);
 
 }  // namespace stief

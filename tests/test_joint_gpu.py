@@ -272,3 +272,135 @@ def test_compress_then_decode_joint_end_to_end():
     q = si.queries(8203, B, Hq, d)
     got = _gpu_joint(q, P_K, P_VJ, k_lat, v_joint, wl.tolist(), max_seq_len=L_max)
     assert_decode_close(got, oracle.decode_joint_v(f64(q), f64(P_K), f64(P_VJ), wk, wv, wl))
+
+
+# ------------------------------------------------- joint compress, prefill-sized chunks (tcgen05)
+
+def _check_within_fp32_bound(k_new, v_new, P_K, P_VJ, gk, gv, lens):
+    """Every stored row against the exact products: within half a bf16 ulp plus the fp32
+    accumulation bound K * 2^-23 * sum|x||p| (K = d for the keys, Hkv*d for the values)."""
+    B, Hkv, T, d = k_new.shape
+    P = f64(P_VJ)
+    for b, L in enumerate(lens):
+        x = np.ascontiguousarray(np.transpose(f64(v_new[b]), (1, 0, 2)).reshape(T, Hkv * d))
+        exact = x @ P
+        bound = 2.0 ** -8 * np.abs(exact) + Hkv * d * 2.0 ** -23 * (np.abs(x) @ np.abs(P)) + 1e-30
+        assert np.all(np.abs(f64(gv[b, L:L + T]) - exact) <= bound)
+        for h in range(Hkv):
+            xk, pk = f64(k_new[b, h]), f64(P_K[h])
+            ek = xk @ pk
+            kb = 2.0 ** -8 * np.abs(ek) + d * 2.0 ** -23 * (np.abs(xk) @ np.abs(pk)) + 1e-30
+            assert np.all(np.abs(f64(gk[b, h, L:L + T]) - ek) <= kb)
+
+
+@pytest.mark.parametrize("T", [128, 129, 300, 1000])
+def test_compress_tc_selector_bases_bit_exact(T):
+    """Chunks of 128 rows or more take the tensor-core projection: with selector bases every
+    stored value is one input coordinate, bit for bit the oracle's, at the rows the lengths
+    name, nothing written elsewhere (ragged last tiles included)."""
+    B, Hkv, d, rK, rV = 2, 4, 128, 32, 48
+    L_max = T + 40
+    k_new, v_new = si.full_kv(8300 + T, B, Hkv, T, d)
+    P_K = torch.stack([_selector_basis(1, d, rK) for _ in range(Hkv)])
+    P_VJ = _selector_basis(Hkv, d, rV)
+    lens = [0, 37]
+    gk, gv, glens, st = _compress_joint(k_new, v_new, P_K, P_VJ, L_max, lens)
+    assert st == 0 and glens.tolist() == [L + T for L in lens]
+    wk, wv, wl, nbad = oracle.compress_append_joint_v(
+        f64(k_new), f64(v_new), f64(P_K), f64(P_VJ), np.zeros((B, Hkv, L_max, rK)),
+        np.zeros((B, L_max, rV)), np.asarray(lens, np.int32))
+    assert nbad == 0 and wl.tolist() == glens.tolist()
+    for b, L in enumerate(lens):
+        assert np.array_equal(f64(gk[b, :, L:L + T]), wk[b, :, L:L + T])
+        assert np.array_equal(f64(gv[b, L:L + T]), wv[b, L:L + T])
+        keep = np.ones(L_max, bool)
+        keep[L:L + T] = False
+        assert torch.all(gk[b][:, keep].view(torch.int16) == CANARY)
+        assert torch.all(gv[b][keep].view(torch.int16) == CANARY)
+
+
+@pytest.mark.parametrize("B,Hkv,T,rK,rV", [
+    (1, 8, 4096, 64, 64),    # one prefill chunk of the 8B-class models (K = 1024 for the values)
+    (1, 8, 4096, 32, 48),
+    (2, 2, 10240, 64, 64),   # several tiles per CTA, the ring wrapping many times
+    (1, 1, 1153, 128, 128),  # one KV head, the widest ranks, a ragged tail
+    (3, 4, 640, 16, 112),
+    (1, 8, 256, 64, 128),    # the joint basis (256 KB) does not fit: the CUDA-core projection
+])
+def test_compress_tc_general_bases_within_the_fp32_bound(B, Hkv, T, rK, rV):
+    """General bases at prefill sizes: every stored key and joint value row within the fp32
+    bound of the exact product, lengths advanced, and (as a check on the accumulation
+    order only) almost every row equal to the oracle's bf16 rounding."""
+    d = 128
+    lens = [5 + 17 * b for b in range(B)]
+    L_max = T + 64
+    k_new, v_new = si.full_kv(8400 + T + Hkv, B, Hkv, T, d)
+    P_K = si.to_bf16(si.bases(8400 + rK, Hkv, d, rK))
+    P_VJ = si.to_bf16(si.bases(8401 + rV, 1, Hkv * d, rV)[0])
+    gk, gv, glens, st = _compress_joint(k_new, v_new, P_K, P_VJ, L_max, lens)
+    assert st == 0 and glens.tolist() == [L + T for L in lens]
+    _check_within_fp32_bound(k_new, v_new, P_K, P_VJ, gk, gv, lens)
+    want = oracle.compress_append_joint_v(f64(k_new), f64(v_new), f64(P_K), f64(P_VJ),
+                                          np.zeros((B, Hkv, L_max, rK)), np.zeros((B, L_max, rV)),
+                                          np.asarray(lens, np.int32))[1]
+    same = [np.mean(f64(gv[b, L:L + T]) == want[b, L:L + T]) for b, L in enumerate(lens)]
+    assert min(same) > 0.95
+    for b, L in enumerate(lens):
+        keep = np.ones(L_max, bool)
+        keep[L:L + T] = False
+        assert torch.all(gv[b][keep].view(torch.int16) == CANARY)
+        assert torch.all(gk[b][:, keep].view(torch.int16) == CANARY)
+
+
+def test_compress_tc_refuses_full_and_bad_sequences():
+    """On the tensor-core path too: a sequence with no room for the chunk and one with a
+    negative length are skipped (nothing written, length unchanged) and reported; the
+    others are appended."""
+    B, Hkv, d, rK, rV, T = 3, 8, 128, 64, 64, 200
+    L_max = 300
+    k_new, v_new = si.full_kv(8500, B, Hkv, T, d)
+    P_K = si.to_bf16(si.bases(8500, Hkv, d, rK))
+    P_VJ = si.to_bf16(si.bases(8501, 1, Hkv * d, rV)[0])
+    lens = [L_max - T + 1, -1, L_max - T]
+    gk, gv, glens, st = _compress_joint(k_new, v_new, P_K, P_VJ, L_max, lens)
+    assert st == (stief.DEV_CAPACITY_OVERFLOW | stief.DEV_BAD_LENGTH)
+    assert glens.tolist() == [lens[0], -1, L_max]
+    for b in (0, 1):
+        assert torch.all(gk[b].view(torch.int16) == CANARY)
+        assert torch.all(gv[b].view(torch.int16) == CANARY)
+    _check_within_fp32_bound(k_new[2:], v_new[2:], P_K, P_VJ, gk[2:], gv[2:], [lens[2]])
+
+
+def test_compress_tc_then_decode_same_stream():
+    """A 2048-token joint chunk compressed and decoded right after it on the same stream (the
+    compress's length kernel lets the decode start early; the decode must still see the new
+    rows and lengths), against the oracle's joint compress and decode."""
+    B, Hq, Hkv, d, rK, rV, T = 2, 32, 8, 128, 64, 64, 2048
+    L_max = T + 64
+    k_new, v_new = si.full_kv(8600, B, Hkv, T, d)
+    P_K = si.to_bf16(si.bases(8600, Hkv, d, rK))
+    P_VJ = si.to_bf16(si.bases(8602, 1, Hkv * d, rV)[0])
+    q = si.queries(8603, B, Hq, d)
+    k_lat = torch.zeros((B, Hkv, L_max, rK), dtype=torch.bfloat16, device=DEV)
+    v_joint = torch.zeros((B, L_max, rV), dtype=torch.bfloat16, device=DEV)
+    lens0 = [3, 60]
+    lens = torch.tensor(lens0, dtype=torch.int32, device=DEV)
+    qd, P_Kd, P_VJd = q.to(DEV), P_K.to(DEV), P_VJ.to(DEV)
+    out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=DEV)
+    ws = _ws(B, Hq, Hkv, rV, L_max)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    stief.stief_compress_append_joint_v(k_new.to(DEV), v_new.to(DEV), P_Kd, P_VJd, k_lat, v_joint,
+                                        lens, dev_status=status)
+    stief.stief_decode_attention_joint_v(qd, P_Kd, P_VJd, k_lat, v_joint, lens, out, ws,
+                                         max_seq_len=L_max, dev_status=status)
+    torch.cuda.synchronize()
+    assert stief.stief_read_device_status(status) == 0
+    wk, wv, wl, _ = oracle.compress_append_joint_v(
+        f64(k_new), f64(v_new), f64(P_K), f64(P_VJ), f64(k_lat.cpu()) * 0, f64(v_joint.cpu()) * 0,
+        np.asarray(lens0, np.int32))
+    assert lens.cpu().tolist() == wl.tolist()
+    # the decode reads the GPU's stored rows: compare it with the oracle on those rows, and the
+    # rows with the oracle's compress within the accumulation bound
+    _check_within_fp32_bound(k_new, v_new, P_K, P_VJ, k_lat.cpu(), v_joint.cpu(), lens0)
+    want = oracle.decode_joint_v(f64(q), f64(P_K), f64(P_VJ), f64(k_lat.cpu()), f64(v_joint.cpu()), wl)
+    assert_decode_close(out.cpu(), want)
