@@ -451,8 +451,8 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
   // with zeros (such tokens lie past the sequence and are masked)
   const long long pool_rows = PG ? (long long)a.num_pages * a.Hkv * a.page_size
                                  : (long long)a.B * a.Hkv * a.L_max;
-  auto tile_row = [&](int t) {
-    const long long r = cache_row(cr, b, kvh, t);
+  auto tile_row = [&](int t, bool before_wait = false) {
+    const long long r = cache_row(cr, b, kvh, t, before_wait);
     return (int)(r < 0 ? pool_rows : r);
   };
   // TMA parameters of the cache pieces (at most three per matrix), kept in registers
@@ -471,13 +471,13 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
     vo[p] = kt_bytes + (uint32_t)a.pv.p[pv].smem_off;
   }
   const int npk = a.pk.n, npv = a.pv.n;
-  auto issue = [&](int w, int k, uint64_t policy) {  // producer: tile k of consumer warp w
+  auto issue = [&](int w, int k, uint64_t policy, bool before_wait = false) {  // producer: tile k of consumer warp w
     uint8_t* dst = smem + L.region + ((size_t)w * ns + (k % ns)) * L.stage;
     uint64_t* bar = &full[w * ns + (k % ns)];
     // whole boxes land (rows past the sequence are masked on chip)
     mbar_arrive_expect_tx(bar, st_bytes);
     const int tt = t0 + (w + k * NW) * kTile;
-    const int y = tile_row(tt);
+    const int y = tile_row(tt, before_wait);
     // joint values: the value rows of sequence b are b * L_max + t, whatever the KV head
     const int yv = JV ? b * a.L_max + tt : y;
 #pragma unroll
@@ -488,20 +488,23 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
       if (p < npv) tma_load_2d(dst + vo[p], vmap[p], vx[p], yv, bar, policy);
   };
 
-  // Contiguous bf16 caches (plain and latent modes): every warp's first tile is requested
-  // before the dependency wait, like P_K, so that it streams while the preceding kernel
-  // finishes (requesting whole rings there measured slower: the flood delays some CTAs'
-  // data by microseconds).  The calls document that the kernel immediately preceding them
-  // must not write the cache rows below the lengths, except the row just below each length
-  // (the one a preceding fused step on the same caches appends), which is read again after
-  // the wait.  Right after a compress of this library (whose new rows may still be in flight)
-  // the host clears `early` and nothing is requested before the wait.
-  const bool early_tiles = (MODE == kModePlain || MODE == kModeLatent) && a.early != 0;
+  // Every warp's first tile is requested before the dependency wait, like P_K, so that it
+  // streams while the preceding kernel finishes (requesting whole rings there measured
+  // slower: the flood delays q and some CTAs' data by microseconds).  The calls document that
+  // the kernel immediately preceding them must not write the cache rows below the lengths
+  // (nor, for page pools, the block-table entries of their pages), except, for bf16
+  // per-head caches, the row just below each length (the one a preceding fused step on the
+  // same caches appends), which is read again after the wait.  Paged caches look the early
+  // tiles' pages up around the L1 cache, so that no line read before the wait can hide an
+  // entry the preceding kernel writes.  Right after a compress of this library (whose new
+  // rows may still be in flight) the host clears `early` and nothing is requested before the
+  // wait.
+  const bool early_tiles = a.early != 0;
   int ring_issued = 0;  // producer lane w: tiles [0, ring_issued) of warp w are requested
   if (early_tiles && producer && lane < NW) {
     const uint64_t stream = l2_policy_evict_first();
     ring_issued = min(min(kPreIssue, ns), warp_tiles(lane, spec_tiles));
-    for (int k = 0; k < ring_issued; ++k) issue(lane, k, stream);
+    for (int k = 0; k < ring_issued; ++k) issue(lane, k, stream, true);
   }
   // inputs may come from the preceding kernel in the stream: read nothing else before this
   pdl_wait();
@@ -932,7 +935,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
       const uint32_t sbase = smem_u32(ring + (size_t)st * L.stage);
       const int tok0 = t0 + (warp + k * NW) * kTile;
       const int n = min(kTile, t1 - tok0);
-      if (early_tiles && k < kPreIssue && Lb >= 1 && tok0 <= Lb - 1 && Lb - 1 < tok0 + kTile) {
+      if (!QI && !JV && early_tiles && k < kPreIssue && Lb >= 1 && tok0 <= Lb - 1 && Lb - 1 < tok0 + kTile) {
         // this tile was requested before the dependency wait: the row just below the length
         // may have been appended by the preceding kernel (a fused step on the same caches),
         // so it is read again now (L2; the wait made it visible)

@@ -196,15 +196,19 @@ __device__ __forceinline__ void named_bar_arrive(int id, int count) {
 // [B][Hkv][L_max] rows; paged caches hold [num_pages][Hkv][page_size] rows and map token t
 // through the sequence's block table (page block_table[b][t / page_size]).  Returns -1 for a
 // token whose page is not mapped (past max_pages, or an id outside [0, num_pages)).
+// `coherent` reads the block table through L2 only (for reads that may precede the
+// dependency wait: the read-only path could keep a line that the preceding kernel rewrites).
 struct CacheRows {
   const int32_t* block_table;  // [B][max_pages], or null for a contiguous cache
   int max_pages, page_size, num_pages, Hkv, L_max;
 };
-__device__ __forceinline__ long long cache_row(const CacheRows& c, int b, int h, int t) {
+__device__ __forceinline__ long long cache_row(const CacheRows& c, int b, int h, int t,
+                                              bool coherent = false) {
   if (c.block_table == nullptr) return ((long long)b * c.Hkv + h) * c.L_max + t;
   const int pi = t / c.page_size;
   if (pi >= c.max_pages) return -1;
-  const int pg = __ldg(c.block_table + (size_t)b * c.max_pages + pi);
+  const int* e = c.block_table + (size_t)b * c.max_pages + pi;
+  const int pg = coherent ? __ldcg(e) : __ldg(e);
   if (pg < 0 || pg >= c.num_pages) return -1;
   return ((long long)pg * c.Hkv + h) * c.page_size + (t - pi * c.page_size);
 }

@@ -208,10 +208,12 @@ STIEF_API size_t stief_decode_workspace_bytes(int B, int Hq, int Hkv, int rV, in
  * This library's kernels never write the bases, and a decode call issued right after
  * one of its compress calls in the same stream reads no cache row before the wait
  * (the library keeps that note per stream).  The rule on P_K holds for every call
- * that takes it (stief_append_decode and the _noalloc, _paged and _q8 decodes);
- * the rule on the cache rows for stief_append_decode, stief_decode_latent and
- * stief_decode_attention_noalloc (the _paged, _q8 and _joint_v calls read no cache
- * row before the wait).
+ * that takes it; the rule on the cache rows for every decode call, with two
+ * differences: the _paged calls also read the block-table entries of their first
+ * tiles before the wait (the preceding kernel must not write the entries of pages
+ * that hold rows below seq_lens[b]), and the int8, 4-bit and joint-value calls
+ * read no row again after the wait (the preceding kernel must write no row below
+ * seq_lens[b], the row just below it included).
  * Returns STIEF_OK or an argument error (nothing launched).
  */
 STIEF_API stief_status stief_decode_attention(const uint16_t* q, const uint16_t* P_K,
