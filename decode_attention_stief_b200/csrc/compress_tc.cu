@@ -24,7 +24,10 @@
 // kernel's tail; the new rows and the lengths are read only after the dependency wait.  Its
 // X tiles stream through a two-stage ring: the first two are requested right after the wait
 // (the length is read while they fly), and the copy of tile i + 2 is issued as soon as tile
-// i's MMA has consumed its stage, so loads overlap the MMA and the epilogue.
+// i's MMA has consumed its stage, so loads overlap the MMA and the epilogue.  Two accumulator
+// sets (all 512 TMEM columns): tile i + 1's MMAs are issued into the other set before tile
+// i's epilogue when its copy is already in, so they run during that epilogue; the epilogue
+// requests up to four 16-column TMEM loads before each wait.
 // Every wait is bounded; every requested copy lands and tensor memory is released before
 // the CTA exits.
 #include <cstdint>
@@ -42,7 +45,11 @@ constexpr int kTcStages = 2;     // X tiles in flight per CTA
 // 8 warps: warp w reads TMEM lanes 32 (w & 3) .. + 31 (rows), the keys' columns for w < 4 and
 // the values' for w >= 4
 constexpr int kTcThreads = 256;
-constexpr uint32_t kTmemCols = 256;
+// two accumulator sets of 256 columns (keys at 0, values at 128): tile i + 1's MMAs run into
+// one while tile i's epilogue reads the other.  All 512 columns of the SM: the shared memory
+// keeps this kernel at one CTA per SM
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kAccCols = 256;
 
 // Shared-memory layout (byte offsets, all swizzled operands 1 KiB aligned).
 struct TcSmem {
@@ -64,7 +71,7 @@ __host__ __device__ inline TcSmem tc_smem_layout(int rK, int rV) {
   for (int i = 0; i < 2; ++i) { s.pk[i] = off; off += (uint32_t)rK * 128; off = (off + 1023) & ~1023u; }
   for (int i = 0; i < 2; ++i) { s.pv[i] = off; off += (uint32_t)rV * 128; off = (off + 1023) & ~1023u; }
   s.bars = off;
-  off += 8 * (kTcStages + 1);
+  off += 8 * (2 * kTcStages + 1);  // copies landed [stages], MMAs done [2], drain
   off = (off + 15) & ~15u;
   s.tmem_slot = off;
   off += 16;
@@ -121,7 +128,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int rK = a.rK, rV = a.rV, T = a.T;
   const TcSmem L = tc_smem_layout(rK, rV);
   uint64_t* tma_bar = reinterpret_cast<uint64_t*>(smem + L.bars);  // [kTcStages]
-  uint64_t* mma_bar = tma_bar + kTcStages;
+  uint64_t* mma_bar = tma_bar + kTcStages;  // [2]: the MMAs of tile i are done (set i & 1)
+  uint64_t* drain_bar = mma_bar + 2;        // exit after a failed wait: every MMA is done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.tmem_slot);
   const int64_t head_row = ((int64_t)b * a.Hkv + h) * T;
   const int my_tiles = (int)blockIdx.x < ta.tiles ? (ta.tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
@@ -145,7 +153,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     return;
   }
   if (tid == 0) {
-    for (int st = 0; st < kTcStages + 1; ++st) mbar_init(&tma_bar[st], 1);
+    for (int st = 0; st < 2 * kTcStages + 1; ++st) mbar_init(&tma_bar[st], 1);
     fence_barrier_init();
   }
   if (warp == 0) {
@@ -178,36 +186,50 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t idK = idesc_bf16_f32(rK), idV = idesc_bf16_f32(rV);
   bool ok = !(bad || full);
-  int consumed = 0;  // tiles whose copy has been waited for
+  int consumed = 0;     // tiles whose copy has been waited for (thread 0)
+  int mma_next = 0;     // thread 0: tiles [0, mma_next) have their MMAs issued
+  // thread 0: tile i's MMAs into accumulator set i & 1, once its copy has landed
+  auto issue_mma = [&](int i) -> bool {
+    const int st = i % kTcStages;
+    if (!mbar_wait_bounded(&tma_bar[st], (uint32_t)((i / kTcStages) & 1), a.dev_status)) return false;
+    consumed = i + 1;
+    tc_fence_after();
+    const uint32_t acc = tmem + (uint32_t)(i & 1) * kAccCols;
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {  // K = 128 in steps of 16 (32 bytes inside an atom)
+      const uint32_t koff = (uint32_t)(kk & 3) * 32u;
+      umma_bf16(acc, sw128_desc(smem_u32(smem + L.xk[st][kk >> 2]) + koff),
+                sw128_desc(smem_u32(smem + L.pk[kk >> 2]) + koff), idK, kk > 0);
+      umma_bf16(acc + 128u, sw128_desc(smem_u32(smem + L.xv[st][kk >> 2]) + koff),
+                sw128_desc(smem_u32(smem + L.pv[kk >> 2]) + koff), idV, kk > 0);
+    }
+    umma_commit(&mma_bar[i & 1]);
+    mma_next = i + 1;
+    return true;
+  };
 
   for (int i = 0; i < my_tiles && ok; ++i) {
-    const int st = i % kTcStages;
-    const uint32_t tphase = (uint32_t)((i / kTcStages) & 1);
+    bool fail = false;  // thread 0: a copy did not land in time
+    if (tid == 0 && mma_next == i) fail = !issue_mma(i);
     // a timed-out wait ends the loop for the whole CTA (tcgen05 ops below are warp-wide)
-    if (__syncthreads_or(!mbar_wait_bounded(&tma_bar[st], tphase, a.dev_status))) {
+    if (__syncthreads_or(fail)) {
       ok = false;
       break;
     }
-    consumed = i + 1;
-    if (tid == 0) {
-      tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {  // K = 128 in steps of 16 (32 bytes inside an atom)
-        const uint32_t koff = (uint32_t)(kk & 3) * 32u;
-        umma_bf16(tmem, sw128_desc(smem_u32(smem + L.xk[st][kk >> 2]) + koff),
-                  sw128_desc(smem_u32(smem + L.pk[kk >> 2]) + koff), idK, kk > 0);
-        umma_bf16(tmem + 128u, sw128_desc(smem_u32(smem + L.xv[st][kk >> 2]) + koff),
-                  sw128_desc(smem_u32(smem + L.pv[kk >> 2]) + koff), idV, kk > 0);
-      }
-      umma_commit(mma_bar);
-    }
-    if (__syncthreads_or(!mbar_wait_bounded(mma_bar, (uint32_t)(i & 1), a.dev_status))) {
+    if (__syncthreads_or(!mbar_wait_bounded(&mma_bar[i & 1], (uint32_t)((i >> 1) & 1), a.dev_status))) {
       ok = false;
       break;
     }
     tc_fence_after();
-    // the MMA has read stage st: refill it with tile i + kTcStages
-    if (tid == 0 && i + kTcStages < my_tiles) issue(i + kTcStages);
+    if (tid == 0) {
+      // the MMAs have read stage i % kTcStages: refill it with tile i + kTcStages
+      if (i + kTcStages < my_tiles) issue(i + kTcStages);
+      // the next tile's MMAs run during this tile's epilogue (into the other accumulator set,
+      // whose tile's epilogue ended with the previous iteration) if its copy is already in
+      if (i + 1 < my_tiles &&
+          mbar_test(&tma_bar[(i + 1) % kTcStages], (uint32_t)(((i + 1) / kTcStages) & 1)))
+        issue_mma(i + 1);
+    }
 
     // epilogue: warp w owns rows 32 (w & 3) .. + 31 (TMEM lanes; lane = row) of the keys
     // (w < 4) or of the values (w >= 4)
@@ -216,7 +238,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int which = warp >> 2;  // 0: keys, 1: values
     const bool live = m0 + row < T;
     const long long crow = live ? cache_row(cr, b, h, Lb + m0 + row) : 0;  // mapped (checked)
-    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    const uint32_t lane_base = tmem + (uint32_t)(i & 1) * kAccCols + ((uint32_t)((warp & 3) * 32) << 16);
     if (a.k_scale != nullptr) {
       // int8 / 4-bit cache: the row rounded to bf16, then one fp32 scale (max / 127, or max / 7)
       // and RNE codes, divisions in IEEE fp32; the accumulators are read twice (maximum, then
@@ -266,22 +288,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (a.k_scale == nullptr) {
       const int r = which ? rV : rK;
       uint16_t* dst = (which ? a.v_lat : a.k_lat) + crow * r;
-      for (int c0 = 0; c0 < r; c0 += 16) {
-        uint32_t v[16];
-        tmem_ld16(lane_base + (which ? 128u : 0u) + (uint32_t)c0, v);
+      const uint32_t col0 = lane_base + (which ? 128u : 0u);
+      for (int g0 = 0; g0 < r; g0 += 64) {  // up to four 16-column loads in flight, one wait
+        uint32_t v[4][16];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (g0 + 16 * q < r) tmem_ld16(col0 + (uint32_t)(g0 + 16 * q), v[q]);
         tmem_wait_ld();
         if (live) {
-          uint4 lo, hi;
-          lo.x = pack_bf16x2_rn(__uint_as_float(v[0]), __uint_as_float(v[1]));
-          lo.y = pack_bf16x2_rn(__uint_as_float(v[2]), __uint_as_float(v[3]));
-          lo.z = pack_bf16x2_rn(__uint_as_float(v[4]), __uint_as_float(v[5]));
-          lo.w = pack_bf16x2_rn(__uint_as_float(v[6]), __uint_as_float(v[7]));
-          hi.x = pack_bf16x2_rn(__uint_as_float(v[8]), __uint_as_float(v[9]));
-          hi.y = pack_bf16x2_rn(__uint_as_float(v[10]), __uint_as_float(v[11]));
-          hi.z = pack_bf16x2_rn(__uint_as_float(v[12]), __uint_as_float(v[13]));
-          hi.w = pack_bf16x2_rn(__uint_as_float(v[14]), __uint_as_float(v[15]));
-          *reinterpret_cast<uint4*>(dst + c0) = lo;
-          *reinterpret_cast<uint4*>(dst + c0 + 8) = hi;
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if (g0 + 16 * q < r) store_bf16x16(dst + g0 + 16 * q, v[q]);
         }
       }
     }
@@ -296,7 +313,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // bounded chance to finish
     for (int j = consumed; j < issued; ++j)
       mbar_wait_bounded(&tma_bar[j % kTcStages], (uint32_t)((j / kTcStages) & 1), nullptr);
-    if (!ok && consumed > 0) mbar_wait_bounded(mma_bar, (uint32_t)((consumed - 1) & 1), nullptr);
+    if (!ok && mma_next > 0) {  // MMAs left by a timeout get a bounded chance to finish
+      umma_commit(drain_bar);
+      mbar_wait_bounded(drain_bar, 0u, nullptr);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -324,9 +344,9 @@ cudaError_t launch_compress_tc(const CompressArgs& a, cudaStream_t stream) {
   const int heads = a.B * a.Hkv;
   int gx = heads >= sms ? 1 : sms / heads;
   if (gx > ta.tiles) gx = ta.tiles;
-  // at least 80 KiB so no more than two CTAs (2 x 256 TMEM columns) share an SM
+  // more than half an SM's shared memory: one CTA per SM (it holds all 512 TMEM columns)
   uint32_t smem = tc_smem_layout(a.rK, a.rV).total;
-  if (smem < 80u * 1024u) smem = 80u * 1024u;
+  if (smem < 120u * 1024u) smem = 120u * 1024u;
   static SmemLimit limit;
   cudaError_t e = limit.ensure(reinterpret_cast<const void*>(stief_compress_tc_kernel), dev, (int)smem);
   if (e != cudaSuccess) return e;
