@@ -12,12 +12,13 @@
 //   - P[h] is written once per CTA, transposed into the same K-major SW128 layout
 //     (rows n = latent column, 128 bytes of k per row and atom), all its loads in flight
 //     at once;
-//   - one thread issues tcgen05.mma; completion is signalled by tcgen05.commit on an
-//     mbarrier; the accumulators live in 256 columns of tensor memory (D_K at column
-//     0, D_V at column 128);
-//   - epilogue: each of 8 warps reads 32 TMEM lanes (rows) of the keys' or the values'
-//     columns with tcgen05.ld, rounds to bf16 (RNE) and stores its rows into the latent
-//     cache at seq_lens[b] + row.
+//   - the keys and the values run as two halves of the CTA (warps 0-3 and 4-7), each with
+//     its own copies, barriers and MMAs, issued by the half's first thread; completion is
+//     signalled by tcgen05.commit on an mbarrier; the accumulators live in tensor memory
+//     (D_K at column 0, D_V at column 128 of an accumulator set);
+//   - epilogue: each of a half's 4 warps reads 32 TMEM lanes (rows) of its half's columns
+//     with tcgen05.ld, rounds to bf16 (RNE) and stores its rows into the latent cache at
+//     seq_lens[b] + row; the halves meet only at the start and at the end.
 // A CTA loops over m-tiles of one (b, h) so P is staged once.  The kernel is launched as a
 // programmatic dependent: barrier set-up, the tensor-memory allocation and the staging of
 // the bases (weights, which the preceding kernel must not write) overlap the preceding
@@ -56,7 +57,7 @@ struct TcSmem {
   uint32_t xk[kTcStages][2], xv[kTcStages][2];  // X tiles per stage, two 64-column atoms:
                                                 // 128 rows x 128 B each
   uint32_t pk[2], pv[2];  // transposed bases, two atoms each: r rows x 128 B
-  uint32_t bars;          // tma[kTcStages], mma
+  uint32_t bars;          // per half (keys, values): tma[kTcStages], mma[2], drain
   uint32_t tmem_slot;     // tcgen05.alloc writes the TMEM base address here
   uint32_t total;
 };
@@ -71,7 +72,7 @@ __host__ __device__ inline TcSmem tc_smem_layout(int rK, int rV) {
   for (int i = 0; i < 2; ++i) { s.pk[i] = off; off += (uint32_t)rK * 128; off = (off + 1023) & ~1023u; }
   for (int i = 0; i < 2; ++i) { s.pv[i] = off; off += (uint32_t)rV * 128; off = (off + 1023) & ~1023u; }
   s.bars = off;
-  off += 8 * (2 * kTcStages + 1);  // copies landed [stages], MMAs done [2], drain
+  off += 8 * 2 * (kTcStages + 3);  // per half: copies landed [stages], MMAs done [2], drain
   off = (off + 15) & ~15u;
   s.tmem_slot = off;
   off += 16;
@@ -110,6 +111,20 @@ __device__ __forceinline__ void stage_bases(uint8_t* smem, const uint32_t (&atk)
   }
 }
 
+// Named barrier `id` over `count` threads that also returns whether any of them passed true.
+__device__ __forceinline__ bool bar_red_or(int id, int count, bool p) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)p), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
+}
+
 }  // namespace
 
 struct CompressTcArgs {
@@ -127,23 +142,29 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int h = blockIdx.y, b = blockIdx.z;
   const int rK = a.rK, rV = a.rV, T = a.T;
   const TcSmem L = tc_smem_layout(rK, rV);
-  uint64_t* tma_bar = reinterpret_cast<uint64_t*>(smem + L.bars);  // [kTcStages]
-  uint64_t* mma_bar = tma_bar + kTcStages;  // [2]: the MMAs of tile i are done (set i & 1)
+  // The keys (warps 0-3) and the values (warps 4-7) run as two halves with their own copies,
+  // MMAs, barriers and epilogue; each half's first thread issues its copies and MMAs.
+  const int half = warp >> 2;            // 0: keys, 1: values
+  const bool issuer = (tid & 127) == 0;
+  const int bar_id = 1 + half;           // the half's named barrier (128 threads)
+  uint64_t* bars0 = reinterpret_cast<uint64_t*>(smem + L.bars);
+  uint64_t* tma_bar = bars0 + half * (kTcStages + 3);  // [kTcStages]: the half's copy landed
+  uint64_t* mma_bar = tma_bar + kTcStages;  // [2]: the half's MMAs of tile i are done (set i & 1)
   uint64_t* drain_bar = mma_bar + 2;        // exit after a failed wait: every MMA is done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.tmem_slot);
   const int64_t head_row = ((int64_t)b * a.Hkv + h) * T;
   const int my_tiles = (int)blockIdx.x < ta.tiles ? (ta.tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
   auto tile_m0 = [&](int i) { return ((int)blockIdx.x + i * (int)gridDim.x) * kTcRows; };
-  int issued = 0;  // copies requested (thread 0 only)
-  auto issue = [&](int i) {  // thread 0: tile i of this CTA into stage i % kTcStages
+  // stage st of this half: two 64-column atoms
+  auto x_atom = [&](int st, int at) { return half ? L.xv[st][at] : L.xk[st][at]; };
+  int issued = 0;  // copies requested (issuer only)
+  auto issue = [&](int i) {  // issuer: tile i of this half into stage i % kTcStages
     const int st = i % kTcStages;
     const uint64_t pol = l2_policy_evict_first();
-    mbar_arrive_expect_tx(&tma_bar[st], 4u * kTcRows * 128u);
+    mbar_arrive_expect_tx(&tma_bar[st], 2u * kTcRows * 128u);
     const int y = (int)(head_row + tile_m0(i));
-    for (int at = 0; at < 2; ++at) {
-      tma_load_2d(smem + L.xk[st][at], &ta.mk, 64 * at, y, &tma_bar[st], pol);
-      tma_load_2d(smem + L.xv[st][at], &ta.mv, 64 * at, y, &tma_bar[st], pol);
-    }
+    for (int at = 0; at < 2; ++at)
+      tma_load_2d(smem + x_atom(st, at), half ? &ta.mv : &ta.mk, 64 * at, y, &tma_bar[st], pol);
     issued = i + 1;
   };
 
@@ -153,7 +174,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     return;
   }
   if (tid == 0) {
-    for (int st = 0; st < 2 * kTcStages + 1; ++st) mbar_init(&tma_bar[st], 1);
+    for (int i = 0; i < 2 * (kTcStages + 3); ++i) mbar_init(&bars0[i], 1);
     fence_barrier_init();
   }
   if (warp == 0) {
@@ -168,7 +189,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();  // the barriers are initialised
   // the new rows and the lengths may come from the preceding kernel: read nothing before this
   pdl_wait();
-  if (tid == 0)  // the first tiles fly while the length is read
+  if (issuer)  // the first tiles fly while the length is read
     for (int i = 0; i < kTcStages && i < my_tiles; ++i) issue(i);
   const int Lb = a.seq_lens[b];
   const bool bad = Lb < 0 || Lb > a.L_max;
@@ -184,24 +205,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t idK = idesc_bf16_f32(rK), idV = idesc_bf16_f32(rV);
+  const int r_h = half ? rV : rK;
+  const uint32_t idesc = idesc_bf16_f32(r_h);
+  const uint32_t p0 = half ? L.pv[0] : L.pk[0], p1 = half ? L.pv[1] : L.pk[1];
   bool ok = !(bad || full);
-  int consumed = 0;     // tiles whose copy has been waited for (thread 0)
-  int mma_next = 0;     // thread 0: tiles [0, mma_next) have their MMAs issued
-  // thread 0: tile i's MMAs into accumulator set i & 1, once its copy has landed
+  int consumed = 0;  // tiles whose copy has been waited for (issuer)
+  int mma_next = 0;  // issuer: tiles [0, mma_next) have their MMAs issued
+  // issuer: tile i's MMAs into the half's columns of accumulator set i & 1 (keys at 0, values
+  // at 128), once its copy has landed
   auto issue_mma = [&](int i) -> bool {
     const int st = i % kTcStages;
     if (!mbar_wait_bounded(&tma_bar[st], (uint32_t)((i / kTcStages) & 1), a.dev_status)) return false;
     consumed = i + 1;
     tc_fence_after();
-    const uint32_t acc = tmem + (uint32_t)(i & 1) * kAccCols;
+    const uint32_t acc = tmem + (uint32_t)(i & 1) * kAccCols + (half ? 128u : 0u);
+    const uint32_t x0 = x_atom(st, 0), x1 = x_atom(st, 1);
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {  // K = 128 in steps of 16 (32 bytes inside an atom)
       const uint32_t koff = (uint32_t)(kk & 3) * 32u;
-      umma_bf16(acc, sw128_desc(smem_u32(smem + L.xk[st][kk >> 2]) + koff),
-                sw128_desc(smem_u32(smem + L.pk[kk >> 2]) + koff), idK, kk > 0);
-      umma_bf16(acc + 128u, sw128_desc(smem_u32(smem + L.xv[st][kk >> 2]) + koff),
-                sw128_desc(smem_u32(smem + L.pv[kk >> 2]) + koff), idV, kk > 0);
+      umma_bf16(acc, sw128_desc(smem_u32(smem + (kk < 4 ? x0 : x1)) + koff),
+                sw128_desc(smem_u32(smem + (kk < 4 ? p0 : p1)) + koff), idesc, kk > 0);
     }
     umma_commit(&mma_bar[i & 1]);
     mma_next = i + 1;
@@ -209,19 +232,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   };
 
   for (int i = 0; i < my_tiles && ok; ++i) {
-    bool fail = false;  // thread 0: a copy did not land in time
-    if (tid == 0 && mma_next == i) fail = !issue_mma(i);
-    // a timed-out wait ends the loop for the whole CTA (tcgen05 ops below are warp-wide)
-    if (__syncthreads_or(fail)) {
+    bool fail = false;  // issuer: a copy did not land in time
+    if (issuer && mma_next == i) fail = !issue_mma(i);
+    // a timed-out wait ends the loop for the whole half (tcgen05 ops below are warp-wide)
+    if (bar_red_or(bar_id, 128, fail)) {
       ok = false;
       break;
     }
-    if (__syncthreads_or(!mbar_wait_bounded(&mma_bar[i & 1], (uint32_t)((i >> 1) & 1), a.dev_status))) {
+    if (bar_red_or(bar_id, 128, !mbar_wait_bounded(&mma_bar[i & 1], (uint32_t)((i >> 1) & 1), a.dev_status))) {
       ok = false;
       break;
     }
     tc_fence_after();
-    if (tid == 0) {
+    if (issuer) {
       // the MMAs have read stage i % kTcStages: refill it with tile i + kTcStages
       if (i + kTcStages < my_tiles) issue(i + kTcStages);
       // the next tile's MMAs run during this tile's epilogue (into the other accumulator set,
@@ -235,7 +258,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // (w < 4) or of the values (w >= 4)
     const int m0 = tile_m0(i);
     const int row = (warp & 3) * 32 + lane;
-    const int which = warp >> 2;  // 0: keys, 1: values
+    const int which = half;
     const bool live = m0 + row < T;
     const long long crow = live ? cache_row(cr, b, h, Lb + m0 + row) : 0;  // mapped (checked)
     const uint32_t lane_base = tmem + (uint32_t)(i & 1) * kAccCols + ((uint32_t)((warp & 3) * 32) << 16);
@@ -302,15 +325,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       }
     }
-    // every warp is done reading the accumulators before the next tile overwrites them
+    // every warp of the half is done reading the accumulators before its next tile
+    // overwrites them
     tc_fence_before();
-    __syncthreads();
+    named_bar_sync(bar_id, 128);
   }
 
-  if (tid == 0) {
+  if (issuer) {
     // every requested copy must land before the shared memory is released (bounded waits;
-    // on the normal path nothing is outstanding), and an MMA left by a timeout gets a
-    // bounded chance to finish
+    // on the normal path nothing is outstanding)
     for (int j = consumed; j < issued; ++j)
       mbar_wait_bounded(&tma_bar[j % kTcStages], (uint32_t)((j / kTcStages) & 1), nullptr);
     if (!ok && mma_next > 0) {  // MMAs left by a timeout get a bounded chance to finish
