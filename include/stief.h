@@ -454,8 +454,10 @@ STIEF_API stief_status stief_decode_attention_q4(const uint16_t* q, const uint16
  *       v_joint[b][seq_lens[b] + t] = bf16_RNE( [v_new[b][0][t] | ... | v_new[b][Hkv-1][t]] . P_VJ )
  *       (fp32 accumulation), keys per head as in stief_compress_append, then
  *       seq_lens[b] += T; the same skipping and status bits for a full cache or a bad length.
- *       T >= 128 runs on the tensor cores when the whole joint basis and two 32 KB input
- *       stages fit one CTA's shared memory (Hkv * rV <= 651), with the launch behaviour of
+ *       T >= 128 runs on the tensor cores when the joint basis (half of it per CTA when an
+ *       even Hkv lets the value tiles be split over CTA pairs, with a 512 * rV-byte exchange
+ *       area) and two 32 KB input stages fit one CTA's shared memory (e.g. Hkv = 8: rV <= 96;
+ *       Hkv = 4: rV <= 128), with the launch behaviour of
  *       stief_compress_append's tensor-core path (a decode issued next on the same stream
  *       waits for it before reading any cache tile); otherwise CUDA cores.  B <= 65535.
  * The key cache has the per-head limits (B * Hkv * L_max < 2^31).  No fused append, paged or
