@@ -46,7 +46,7 @@ namespace stief {
 namespace {
 
 constexpr int kJtThreads = 256;
-constexpr uint32_t kJtTmemCols = 128;          // one accumulator, N = r <= 128 fp32 columns
+constexpr uint32_t kJtTmemCols = 256;  // two accumulator sets of 128 columns (N = r <= 128)
 constexpr int kJtMaxStages = 4;
 constexpr uint32_t kAtomBytes = kUmmaRows * 128u;  // 128 rows x 64 bf16 columns
 constexpr uint32_t kChunkBytes = 2u * kAtomBytes;  // one 128 x 128 input chunk
@@ -250,9 +250,67 @@ __global__ void __launch_bounds__(kJtThreads, 1)
   int consumed = 0;  // chunk copies waited for (thread 0)
   bool mma_issued = false;
 
+  // Key CTAs (one chunk per tile): two accumulator sets, so that tile i + 1's MMAs run
+  // during tile i's epilogue when its copy is already in; the stages' "empty" barriers serve
+  // as the two sets' "MMAs done" barriers (stage i % S is free once tile i's MMAs are done).
+  int mma_next = 0;  // thread 0: key tiles [0, mma_next) have their MMAs issued
+  auto key_mma = [&](int i) -> bool {
+    const int st = i % S;
+    if (!mbar_wait_bounded(&full[st], (uint32_t)((i / S) & 1), a.dev_status)) return false;
+    consumed = i + 1;
+    tc_fence_after();
+    const uint32_t xa = smem_u32(smem + L.x0 + (uint32_t)st * kChunkBytes);
+    const uint32_t pa = smem_u32(smem + L.basis);
+    const uint32_t acc = tmem + (uint32_t)(i & 1) * 128u;
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {  // K = 128 in steps of 16 (32 bytes inside an atom)
+      const uint32_t koff = (uint32_t)(kk & 3) * 32u;
+      umma_bf16(acc, sw128_desc(xa + (uint32_t)(kk >> 2) * kAtomBytes + koff),
+                sw128_desc(pa + (uint32_t)(kk >> 2) * atom_b + koff), idesc, kk > 0 ? 1u : 0u);
+    }
+    mma_issued = true;
+    umma_commit(&empty[i & 1]);
+    mma_next = i + 1;
+    return true;
+  };
+  for (int i = 0; !values && i < my_tiles && ok; ++i) {
+    bool fail = false;
+    if (tid == 0 && mma_next == i) fail = !key_mma(i);
+    if (__syncthreads_or(fail)) {
+      ok = false;
+      break;
+    }
+    if (__syncthreads_or(!mbar_wait_bounded(&empty[i & 1], (uint32_t)((i >> 1) & 1), a.dev_status))) {
+      ok = false;
+      break;
+    }
+    tc_fence_after();
+    if (tid == 0) {
+      if (i + S < my_tiles) issue(i + S);  // tile i's MMAs have read its stage
+      if (i + 1 < my_tiles && mbar_test(&full[(i + 1) % S], (uint32_t)(((i + 1) / S) & 1)))
+        key_mma(i + 1);
+    }
+    const int m0 = tile_m0(i);
+    const int row = (warp & 3) * 32 + lane;
+    const bool live = m0 + row < T;
+    const uint32_t lane_base = tmem + (uint32_t)(i & 1) * 128u + ((uint32_t)((warp & 3) * 32) << 16);
+    const size_t crow = ((size_t)b * Hkv + h) * a.L_max + (size_t)(Lb + m0 + row);
+    uint16_t* dst = a.k_lat + (live ? crow * (size_t)r : 0);
+    for (int c0 = 16 * (warp >> 2); c0 < r; c0 += 32) {
+      uint32_t v[16];
+      tmem_ld16(lane_base + (uint32_t)c0, v);
+      tmem_wait_ld();
+      if (live) store_bf16x16(dst + c0, v);
+    }
+    // every warp is done reading this set before tile i + 2 overwrites it
+    tc_fence_before();
+    __syncthreads();
+  }
+
+  // Value CTAs (one accumulator, set 0).
   // A pair runs every iteration (its two cluster barriers per tile must match in both CTAs);
   // after a failed wait a CTA only skips the work.  Other CTAs stop at the first failure.
-  for (int i = 0; i < my_tiles && (ok || paired); ++i) {
+  for (int i = 0; values && i < my_tiles && (ok || paired); ++i) {
     bool fail = false;
     if (ok && tid == 0) {
       for (int c = 0; c < nch; ++c) {
