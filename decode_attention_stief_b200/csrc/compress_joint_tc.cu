@@ -179,6 +179,11 @@ __global__ void __launch_bounds__(kJtThreads, 1)
   const CUtensorMap* map = values ? &ja.mv : &ja.mk;
   auto tile_m0 = [&](int i) { return (x + i * ctas) * kUmmaRows; };
 
+#ifdef STIEF_TEST_HOOKS
+  const uint32_t stall = a.test_stall_bytes;  // test build: chunk 0's copy never completes
+#else
+  constexpr uint32_t stall = 0u;
+#endif
   int issued = 0;  // chunk copies requested (thread 0 only)
   auto issue = [&](int s) {  // thread 0: chunk s % nch of tile s / nch into stage s % S
     const int st = s % S, i = s / nch, c = s - i * nch;
@@ -186,7 +191,7 @@ __global__ void __launch_bounds__(kJtThreads, 1)
     const int y = (int)(((int64_t)b * Hkv + g) * T + tile_m0(i));
     const uint64_t pol = l2_policy_evict_first();
     uint8_t* dst = smem + L.x0 + (uint32_t)st * kChunkBytes;
-    mbar_arrive_expect_tx(&full[st], kChunkBytes);
+    mbar_arrive_expect_tx(&full[st], kChunkBytes + (s == 0 ? stall : 0u));
     tma_load_2d(dst, map, 0, y, &full[st], pol);
     tma_load_2d(dst + kAtomBytes, map, 64, y, &full[st], pol);
     issued = s + 1;
@@ -428,6 +433,9 @@ bool compress_joint_tc_fits(int Hkv, int rK, int rV) {
 cudaError_t launch_compress_joint_tc(const CompressArgs& a, cudaStream_t stream) {
   JointTcArgs ja{};
   ja.a = a;
+#ifdef STIEF_TEST_HOOKS
+  ja.a.test_stall_bytes = test_stall_bytes();
+#endif
   ja.tiles = (a.T + kUmmaRows - 1) / kUmmaRows;
   ja.pair = jt_pair_fits(a.Hkv, a.rK, a.rV) ? 1 : 0;
   const int vch = ja.pair ? a.Hkv / 2 : a.Hkv;

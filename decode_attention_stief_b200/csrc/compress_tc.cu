@@ -157,11 +157,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   auto tile_m0 = [&](int i) { return ((int)blockIdx.x + i * (int)gridDim.x) * kTcRows; };
   // stage st of this half: two 64-column atoms
   auto x_atom = [&](int st, int at) { return half ? L.xv[st][at] : L.xk[st][at]; };
+#ifdef STIEF_TEST_HOOKS
+  const uint32_t stall = a.test_stall_bytes;  // test build: tile 0's copy never completes
+#else
+  constexpr uint32_t stall = 0u;
+#endif
   int issued = 0;  // copies requested (issuer only)
   auto issue = [&](int i) {  // issuer: tile i of this half into stage i % kTcStages
     const int st = i % kTcStages;
     const uint64_t pol = l2_policy_evict_first();
-    mbar_arrive_expect_tx(&tma_bar[st], 2u * kTcRows * 128u);
+    mbar_arrive_expect_tx(&tma_bar[st], 2u * kTcRows * 128u + (i == 0 ? stall : 0u));
     const int y = (int)(head_row + tile_m0(i));
     for (int at = 0; at < 2; ++at)
       tma_load_2d(smem + x_atom(st, at), half ? &ta.mv : &ta.mk, 64 * at, y, &tma_bar[st], pol);
@@ -355,6 +360,9 @@ uint32_t compress_tc_smem_bytes(int rK, int rV) { return tc_smem_layout(rK, rV).
 cudaError_t launch_compress_tc(const CompressArgs& a, cudaStream_t stream) {
   CompressTcArgs ta{};
   ta.a = a;
+#ifdef STIEF_TEST_HOOKS
+  ta.a.test_stall_bytes = test_stall_bytes();
+#endif
   ta.tiles = (a.T + kTcRows - 1) / kTcRows;
   const uint64_t rows = (uint64_t)a.B * a.Hkv * a.T;
   if (rows >= (1ull << 31)) return cudaErrorInvalidValue;  // TMA row coordinates are int32

@@ -287,7 +287,8 @@ stief_status plan_decode(DecodeArgs& a, const uint16_t* q, const uint16_t* P_K,
 #ifdef STIEF_TEST_HOOKS
 // Test build only (libstief_testhooks.so, used by the timeout tests; not part of the public
 // header): every decode planned after this call waits for `bytes` more on its setup barrier
-// than any copy delivers, so its bounded waits run out (0 turns it off).  The bytes must be a
-// multiple of 16.
+// than any copy delivers, and every tensor-core compress launched after it for `bytes` more on
+// each CTA's (half's) first copy, so their bounded waits run out (0 turns it off).  The bytes
+// must be a multiple of 16.
 extern "C" STIEF_API void stief_test_set_stall(uint32_t bytes) { stief::g_test_stall.store(bytes); }
 #endif

@@ -104,6 +104,11 @@ struct CompressArgs {
   float* k_scale;
   float* v_scale;
   int q4;
+#ifdef STIEF_TEST_HOOKS
+  // test build only: bytes added to the first copy's expected count in every CTA (half) of
+  // the tensor-core projections, which no copy delivers, so that the waits for it run out
+  uint32_t test_stall_bytes;
+#endif
 };
 
 constexpr int kMaxSmemPerBlock = 232448;  // 227 KB opt-in dynamic shared memory (sm_100)

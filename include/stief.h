@@ -69,7 +69,10 @@ typedef enum stief_status {
 #define STIEF_DEV_CAPACITY_OVERFLOW 0x1u /* compress: seq_lens[b] + T > L_max; that
                                             sequence was left untouched */
 #define STIEF_DEV_WAIT_TIMEOUT 0x2u      /* a bounded wait on an asynchronous copy or
-                                            tensor-core completion gave up */
+                                            tensor-core completion gave up; the call's
+                                            results are undefined (a compress may still
+                                            have advanced the lengths: put them back and
+                                            call again; a decode: zero the workspace) */
 #define STIEF_DEV_BAD_LENGTH 0x4u        /* a seq_lens entry was negative or > L_max
                                             (decode: that sequence's output is zero;
                                             compress: it is left untouched) */

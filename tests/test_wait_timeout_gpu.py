@@ -4,7 +4,8 @@ the kernel returns, the context stays usable, and the next call is correct again
 These tests load libstief_testhooks.so, the library built from the same sources with
 STIEF_TEST_HOOKS: its bounded waits give up after 50 ms instead of 2 s, and
 stief_test_set_stall(bytes) makes every decode planned afterwards expect `bytes` more on its
-setup barrier (q, P_K) than any copy delivers.  That phase then never completes, like a flag
+setup barrier (q, P_K) than any copy delivers, and every tensor-core compress launched
+afterwards `bytes` more on each CTA's (or CTA half's) first copy.  That phase then never completes, like a flag
 that nothing sets: every wait for it runs out, the kernel reports the timeout, waits (bounded)
 for the copies it has in flight and returns.  Nothing faults, traps or waits without a limit.
 
@@ -41,6 +42,10 @@ def hooks():
     lib.stief_decode_latent.argtypes = [_vp] * 6 + [_sz] + [_i] * 9 + [_vp, _vp]
     lib.stief_decode_attention_noalloc.restype = _i
     lib.stief_decode_attention_noalloc.argtypes = [_vp] * 7 + [_i] * 9 + [_vp, _vp]
+    for name in ("stief_compress_append", "stief_compress_append_joint_v"):
+        fn = getattr(lib, name)
+        fn.restype = _i
+        fn.argtypes = [_vp] * 7 + [_i] * 7 + [_vp, _vp]
     lib.stief_test_set_stall.restype = None
     lib.stief_test_set_stall.argtypes = [ctypes.c_uint32]
     lib.stief_test_noalloc_scratch.restype = _i
@@ -182,3 +187,78 @@ def test_noalloc_scratch_cleared_before_each_launch(hooks):
     call(status)
     assert _read(status) == 0
     assert decode_error(out.cpu(), want) <= DECODE_TOL
+
+
+# ---------------------------------------------------------------- tensor-core compress kernels
+
+# (joint, B, Hkv, T, rK, rV): the per-head projection (key and value halves of each CTA), the
+# joint one with value tiles over CTA pairs (an even Hkv; the pair runs every tile and both of
+# its CTAs meet at every cluster barrier after the timeout) and with one CTA per value tile
+# (Hkv = 1)
+COMPRESS_CASES = [(False, 2, 4, 300, 64, 48), (True, 2, 8, 300, 64, 64), (True, 1, 1, 700, 64, 128),
+                  (True, 1, 2, 2600, 32, 64)]
+
+
+@pytest.mark.parametrize("joint,B,Hkv,T,rK,rV", COMPRESS_CASES)
+def test_compress_timeout_reported_then_recovered(hooks, joint, B, Hkv, T, rK, rV):
+    """A stalled first copy in every CTA: the tensor-core compress reports the timeout and
+    returns (the rows and lengths of that call are undefined); with the lengths put back, the
+    next call writes the oracle's rows again."""
+    import stief_inputs as si
+    d, L_max = 128, T + 40
+    k_new, v_new = si.full_kv(9400 + T, B, Hkv, T, d)
+    P_K = si.to_bf16(si.bases(9400, Hkv, d, rK))
+    if joint:
+        P_V = si.to_bf16(si.bases(9401, 1, Hkv * d, rV)[0])
+        v_shape = (B, L_max, rV)
+        fn = hooks.stief_compress_append_joint_v
+    else:
+        P_V = si.to_bf16(si.bases(9401, Hkv, d, rV))
+        v_shape = (B, Hkv, L_max, rV)
+        fn = hooks.stief_compress_append
+    kn, vn, pk, pv = (x.cuda().contiguous() for x in (k_new, v_new, P_K, P_V))
+    k_lat = torch.zeros((B, Hkv, L_max, rK), dtype=torch.bfloat16, device="cuda")
+    v_lat = torch.zeros(v_shape, dtype=torch.bfloat16, device="cuda")
+    lens0 = [5 + 11 * b for b in range(B)]
+    lens = torch.tensor(lens0, dtype=torch.int32, device="cuda")
+
+    def call(status):
+        code = fn(kn.data_ptr(), vn.data_ptr(), pk.data_ptr(), pv.data_ptr(), k_lat.data_ptr(),
+                  v_lat.data_ptr(), lens.data_ptr(), B, Hkv, T, d, rK, rV, L_max,
+                  status.data_ptr(), _stream())
+        assert code == 0, stief.stief_status_string(code)
+
+    status = _status_word()
+    hooks.stief_test_set_stall(STALL_BYTES)
+    try:
+        call(status)
+        assert _read(status) & DEV_WAIT_TIMEOUT, "the stalled compress did not report a timeout"
+    finally:
+        hooks.stief_test_set_stall(0)
+    lens.copy_(torch.tensor(lens0, dtype=torch.int32))
+    status.zero_()
+    call(status)
+    assert _read(status) == 0
+    assert lens.cpu().tolist() == [L + T for L in lens0]
+    # every stored row within half a bf16 ulp of the exact product plus the fp32 accumulation
+    # bound K * 2^-23 * sum |x||p| (K = d per head, Hkv * d for the joint values); nothing else
+    # written
+    gk, gv = f64(k_lat.cpu()), f64(v_lat.cpu())
+
+    def within(got, x, P):
+        exact = x @ P
+        bound = 2.0 ** -8 * np.abs(exact) + P.shape[0] * 2.0 ** -23 * (np.abs(x) @ np.abs(P))
+        return np.all(np.abs(got - exact) <= bound + 1e-30)
+
+    for bb, L in enumerate(lens0):
+        for h in range(Hkv):
+            assert within(gk[bb, h, L:L + T], f64(k_new[bb, h]), f64(P_K[h]))
+            if not joint:
+                assert within(gv[bb, h, L:L + T], f64(v_new[bb, h]), f64(P_V[h]))
+        if joint:
+            x = np.ascontiguousarray(np.transpose(f64(v_new[bb]), (1, 0, 2)).reshape(T, Hkv * d))
+            assert within(gv[bb, L:L + T], x, f64(P_V))
+        keep = np.ones(L_max, bool)
+        keep[L:L + T] = False
+        assert not np.any(gk[bb][:, keep])
+        assert not np.any(gv[bb][keep] if joint else gv[bb][:, keep])
