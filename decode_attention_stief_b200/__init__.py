@@ -23,6 +23,7 @@ from ._binding import (  # noqa: F401
     stief_compress_append_paged,
     stief_decode_attention,
     stief_decode_attention_q8,
+    stief_append_decode_q8,
     stief_compress_append_q4,
     stief_compress_append_q8_paged,
     stief_decode_attention_q8_paged,

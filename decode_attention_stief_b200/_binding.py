@@ -89,6 +89,9 @@ def library() -> ctypes.CDLL:
             lib.stief_decode_attention_q8.restype = _i
             lib.stief_decode_attention_q8.argtypes = ([vp] * 10 + [ctypes.c_size_t] + [_i] * 9
                                                       + [vp, vp])
+            lib.stief_append_decode_q8.restype = _i
+            lib.stief_append_decode_q8.argtypes = ([vp] * 12 + [ctypes.c_size_t] + [_i] * 9
+                                                   + [vp, vp])
             lib.stief_compress_append_q8_paged.restype = _i
             lib.stief_compress_append_q8_paged.argtypes = [vp] * 10 + [_i] * 9 + [vp, vp]
             lib.stief_decode_attention_q8_paged.restype = _i
@@ -489,6 +492,46 @@ def stief_decode_attention_q8(q, P_K, P_V, k_q, v_q, k_s, v_s, seq_lens, out, wo
                                                workspace.data_ptr(), ws_bytes, B, Hq, Hkv, d, rK,
                                                rV, L_max, int(max_seq_len), int(num_splits),
                                                _opt_status(dev_status), _stream_ptr(stream),))
+    return out
+
+
+def stief_append_decode_q8(q, k_new, v_new, P_K, P_V, k_q, v_q, k_s, v_s, seq_lens, out,
+                           workspace, max_seq_len: int, num_splits: int = 0,
+                           dev_status: Optional[torch.Tensor] = None, stream=None):
+    """stief_append_decode on an int8 cache: the new token's rows are quantised into k_q, v_q
+    (codes) and k_s, v_s (row scales) at row seq_lens[b] as stief_compress_append_q8 stores
+    them, the decode attends over the grown cache, and seq_lens is incremented.  k_new, v_new
+    [B][Hkv][d] (or [B][Hkv][1][d]) bf16; the rest as for stief_decode_attention_q8."""
+    pq = _dev(q, "q", torch.bfloat16, 3)
+    kn = k_new.reshape(k_new.shape[0], k_new.shape[1], -1) if k_new.dim() == 4 else k_new
+    vn = v_new.reshape(v_new.shape[0], v_new.shape[1], -1) if v_new.dim() == 4 else v_new
+    pkn = _dev(kn, "k_new", torch.bfloat16, 3)
+    pvn = _dev(vn, "v_new", torch.bfloat16, 3)
+    ppk = _dev(P_K, "P_K", torch.bfloat16, 3)
+    ppv = _dev(P_V, "P_V", torch.bfloat16, 3)
+    pkq = _dev(k_q, "k_q", torch.int8, 4)
+    pvq = _dev(v_q, "v_q", torch.int8, 4)
+    pks = _dev(k_s, "k_s", torch.float32, 3)
+    pvs = _dev(v_s, "v_s", torch.float32, 3)
+    psl = _dev(seq_lens, "seq_lens", torch.int32, 1)
+    po = _dev(out, "out", torch.bfloat16, 3)
+    B, Hq, d = q.shape
+    Hkv, _, rK = P_K.shape
+    rV = P_V.shape[2]
+    L_max = k_q.shape[2]
+    if tuple(P_V.shape) != (Hkv, d, rV) or tuple(kn.shape) != (B, Hkv, d) \
+            or tuple(vn.shape) != (B, Hkv, d) or tuple(k_q.shape) != (B, Hkv, L_max, rK) \
+            or tuple(v_q.shape) != (B, Hkv, L_max, rV) or tuple(k_s.shape) != (B, Hkv, L_max) \
+            or tuple(v_s.shape) != (B, Hkv, L_max) or seq_lens.shape[0] != B \
+            or tuple(out.shape) != (B, Hq, d):
+        raise ValueError("stief_append_decode_q8: inconsistent shapes")
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _invoke("stief_append_decode_q8", (pq, pkn, pvn, ppk, ppv, pkq, pvq, pks, pvs, psl, po,
+                                       workspace.data_ptr(), ws_bytes, B, Hq, Hkv, d, rK, rV,
+                                       L_max, int(max_seq_len), int(num_splits),
+                                       _opt_status(dev_status), _stream_ptr(stream),))
     return out
 
 

@@ -352,17 +352,22 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int NW, int ns, int rK,
 constexpr int kMaxConsumerWarps = 8;
 
 // Kernel modes: the contiguous bf16 cache, the latent decode, paged caches, int8 caches, and
-// joint value latents (one value row per token shared by the KV heads; full or latent output).
-// Each is its own instantiation, so a mode's branches cost the others nothing.
+// joint value latents (one value row per token shared by the KV heads; full or latent output);
+// the int8 fused step (append + decode) is its own int8 mode.  Each is its own instantiation,
+// so a mode's branches cost the others nothing.
 constexpr int kModePlain = 0, kModeLatent = 1, kModePaged = 2, kModeQ8 = 3, kModeJointV = 4,
-              kModeLatentJointV = 5, kModeQ4 = 6, kModePagedQ8 = 7;
+              kModeLatentJointV = 5, kModeQ4 = 6, kModePagedQ8 = 7, kModeQ8Append = 8;
 
 template <int NB, int NKS, int NMV, int TT, int MODE>
 __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
     stief_decode_kernel(const __grid_constant__ DecodeArgs a) {
   constexpr bool LAT = MODE == kModeLatent || MODE == kModeLatentJointV;
   constexpr bool PG = MODE == kModePaged || MODE == kModePagedQ8;
-  constexpr bool Q8 = MODE == kModeQ8 || MODE == kModePagedQ8, Q4 = MODE == kModeQ4;
+  constexpr bool Q8 = MODE == kModeQ8 || MODE == kModePagedQ8 || MODE == kModeQ8Append;
+  constexpr bool Q4 = MODE == kModeQ4;
+  // the new token's rows enter the tile: every bf16 mode that may append, and the int8 fused
+  // step (the other integer modes never append)
+  constexpr bool INJECT = !(Q8 || Q4) || MODE == kModeQ8Append;
   constexpr bool QI = Q8 || Q4;  // integer codes with row scales
   constexpr bool JV = MODE == kModeJointV || MODE == kModeLatentJointV;
   constexpr int kTile = TT;
@@ -493,8 +498,8 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
   // slower: the flood delays q and some CTAs' data by microseconds).  The calls document that
   // the kernel immediately preceding them must not write the cache rows below the lengths
   // (nor, for page pools, the block-table entries of their pages), except, for bf16
-  // per-head caches, the row just below each length (the one a preceding fused step on the
-  // same caches appends), which is read again after the wait.  Paged caches look the early
+  // per-head caches and contiguous int8 caches, the row just below each length (the one a
+  // preceding fused step on the same caches appends), which is read again after the wait.  Paged caches look the early
   // tiles' pages up around the L1 cache, so that no line read before the wait can hide an
   // entry the preceding kernel writes.  Right after a compress of this library (whose new
   // rows may still be in flight) the host clears `early` and nothing is requested before the
@@ -679,7 +684,8 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
         uint16_t* kl = reinterpret_cast<uint16_t*>(smem + L.newlat);
         kl[j] = f32_to_bf16_rn(c[0]);
         kl[j + 8] = f32_to_bf16_rn(c[2]);
-        if (qs == 0) {  // the cache row itself (every sub-group computes the same values)
+        if (!QI && qs == 0) {  // the cache row itself (every sub-group computes the same
+          // values; int8 caches get the row's codes from the producer)
           uint16_t* dst = a.k_lat_w + new_row * rK;
           dst[j] = kl[j];
           dst[j + 8] = kl[j + 8];
@@ -739,6 +745,38 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
       // the MMA (B column 0) into shared memory (and the cache) for the tile that holds it
       // (one 16-row m-tile per call, so the refills in between are not held up)
       int vrow_next = owns_new && setup_ok ? 0 : nmv;  // next m-tile of the new value row
+      // int8 caches (fused step): the new token's bf16 key and value rows (shared memory)
+      // become one fp32 scale each (max |x| / 127, IEEE division) and RNE codes, as the
+      // compress kernels store them; codes [rK] then [rV] and the two scales go to the
+      // new-row area (its k and v inputs are consumed by now), and to the cache row
+      auto quantize_new_rows = [&]() {
+        const uint16_t* lat = reinterpret_cast<const uint16_t*>(smem + L.newlat);
+        int8_t* codes = reinterpret_cast<int8_t*>(smem + L.newraw);
+        float* nsc = reinterpret_cast<float*>(smem + L.newraw + 256);
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+          const int r = part ? rV : rK, off = part ? rK : 0;
+          float amax = 0.f;
+          for (int j = lane; j < r; j += 32) amax = fmaxf(amax, fabsf(bf16_to_f32(lat[off + j])));
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
+          const float scale = __fdiv_rn(amax, 127.f);
+          for (int j = lane; j < r; j += 32) codes[off + j] = (int8_t)quantize_code(bf16_to_f32(lat[off + j]), scale);
+          if (lane == 0) nsc[part] = scale;
+        }
+        __syncwarp();
+        if (qs == 0) {  // the cache rows (every sub-group computes the same values)
+          int8_t* kq = reinterpret_cast<int8_t*>(a.k_lat_w) + new_row * rK;
+          int8_t* vq = reinterpret_cast<int8_t*>(a.v_lat_w) + new_row * rV;
+          for (int j = lane; j < rK; j += 32) kq[j] = codes[j];
+          for (int j = lane; j < rV; j += 32) vq[j] = codes[rK + j];
+          if (lane == 0) {
+            a.k_scale_w[new_row] = nsc[0];
+            a.v_scale_w[new_row] = nsc[1];
+          }
+        }
+        __syncwarp();
+      };
       auto project_vrow = [&]() {
         const uint32_t* vrow = reinterpret_cast<const uint32_t*>(smem + L.newraw + 2u * d);
         const bool vcol = (lane >> 2) == 0;  // lanes holding B column 0
@@ -760,7 +798,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
             const int j = 16 * mv + (lane >> 2);
             vl[j] = f32_to_bf16_rn(cv[0]);
             vl[j + 8] = f32_to_bf16_rn(cv[2]);
-            if (qs == 0) {
+            if (!QI && qs == 0) {
               a.v_lat_w[new_row * rV + j] = vl[j];
               a.v_lat_w[new_row * rV + j + 8] = vl[j + 8];
             }
@@ -768,6 +806,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
         }
         if (++vrow_next == nmv) {
           __syncwarp();
+          if constexpr (MODE == kModeQ8Append) quantize_new_rows();
           if (lane == 0) mbar_arrive(newrow_bar);  // release: the row is visible to the consumers
         }
       };
@@ -935,23 +974,39 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
       const uint32_t sbase = smem_u32(ring + (size_t)st * L.stage);
       const int tok0 = t0 + (warp + k * NW) * kTile;
       const int n = min(kTile, t1 - tok0);
-      if (!QI && !JV && early_tiles && k < kPreIssue && Lb >= 1 && tok0 <= Lb - 1 && Lb - 1 < tok0 + kTile) {
+      // the modes with a fused step: bf16 per-head caches, and contiguous int8 caches
+      constexpr bool RELOAD_Q8 = MODE == kModeQ8 || MODE == kModeQ8Append;
+      if ((RELOAD_Q8 || (!QI && !JV)) && early_tiles && k < kPreIssue && Lb >= 1 && tok0 <= Lb - 1 &&
+          Lb - 1 < tok0 + kTile) {
         // this tile was requested before the dependency wait: the row just below the length
         // may have been appended by the preceding kernel (a fused step on the same caches),
-        // so it is read again now (L2; the wait made it visible)
+        // so it is read again now (L2; the wait made it visible).  int8 caches: its codes (its
+        // scales are loaded after the wait anyway)
         const int r_prev = Lb - 1 - tok0;
         const long long prow = cache_row(cr, b, kvh, Lb - 1);
-        for (int cch = lane; cch < (rK + rV) / 8; cch += 32) {
-          const bool key = cch < rK / 8;
-          const uint4 v = key ? __ldcg(reinterpret_cast<const uint4*>(a.k_lat_w + prow * rK) + cch)
-                              : __ldcg(reinterpret_cast<const uint4*>(a.v_lat_w + prow * rV) + (cch - rK / 8));
-          const PieceLoc pt = key ? locate(rK, kTile, cch) : locate(rV, kTile, cch - rK / 8);
-          *reinterpret_cast<uint4*>(ring + (size_t)st * L.stage + (key ? 0u : kt_bytes) + swz(pt, r_prev)) = v;
+        if constexpr (RELOAD_Q8) {
+          const int8_t* kq = reinterpret_cast<const int8_t*>(a.k_lat_w) + prow * rK;
+          const int8_t* vq = reinterpret_cast<const int8_t*>(a.v_lat_w) + prow * rV;
+          for (int cch = lane; cch < (rK + rV) / 16; cch += 32) {
+            const bool key = cch < rK / 16;
+            const uint4 v = key ? __ldcg(reinterpret_cast<const uint4*>(kq) + cch)
+                                : __ldcg(reinterpret_cast<const uint4*>(vq) + (cch - rK / 16));
+            const PieceLoc pt = key ? locate_i8(rKc, kTile, cch) : locate_i8(rVc, kTile, cch - rK / 16);
+            *reinterpret_cast<uint4*>(ring + (size_t)st * L.stage + (key ? 0u : kt_bytes) + swz(pt, r_prev)) = v;
+          }
+        } else {
+          for (int cch = lane; cch < (rK + rV) / 8; cch += 32) {
+            const bool key = cch < rK / 8;
+            const uint4 v = key ? __ldcg(reinterpret_cast<const uint4*>(a.k_lat_w + prow * rK) + cch)
+                                : __ldcg(reinterpret_cast<const uint4*>(a.v_lat_w + prow * rV) + (cch - rK / 8));
+            const PieceLoc pt = key ? locate(rK, kTile, cch) : locate(rV, kTile, cch - rK / 8);
+            *reinterpret_cast<uint4*>(ring + (size_t)st * L.stage + (key ? 0u : kt_bytes) + swz(pt, r_prev)) = v;
+          }
         }
         fence_proxy_async_smem();  // generic writes into a stage the TMA engine fills
         __syncwarp();
       }
-      if (owns_new && tok0 <= Lb && Lb < tok0 + kTile) {
+      if (INJECT && owns_new && tok0 <= Lb && Lb < tok0 + kTile) {
         // This tile holds the new token, whose cache rows were not written yet when the tile
         // was fetched: put the projected rows (key row from the prologue, value row from
         // the producer) into the tile.
@@ -960,12 +1015,31 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
           break;
         }
         const int r_new = Lb - tok0;
-        const uint16_t* kl = reinterpret_cast<const uint16_t*>(smem + L.newlat);
-        for (int cch = lane; cch < (rK + rV) / 8; cch += 32) {
-          const bool key = cch < rK / 8;
-          const PieceLoc pt = key ? locate(rK, kTile, cch) : locate(rV, kTile, cch - rK / 8);
-          *reinterpret_cast<uint4*>(ring + (size_t)st * L.stage + (key ? 0u : kt_bytes) +
-                                    swz(pt, r_new)) = *reinterpret_cast<const uint4*>(kl + 8 * cch);
+        if constexpr (MODE == kModeQ8Append) {
+          // the codes (16-byte chunks of the rows, addressed as 16-bit columns) and, in the
+          // lane that holds the token's row scales, the scales
+          const uint8_t* nc = smem + L.newraw;
+          for (int cch = lane; cch < (rK + rV) / 16; cch += 32) {
+            const bool key = cch < rK / 16;
+            const PieceLoc pt = key ? locate_i8(rKc, kTile, cch) : locate_i8(rVc, kTile, cch - rK / 16);
+            *reinterpret_cast<uint4*>(ring + (size_t)st * L.stage + (key ? 0u : kt_bytes) +
+                                      swz(pt, r_new)) = *reinterpret_cast<const uint4*>(nc + 16 * cch);
+          }
+          const float* nsc = reinterpret_cast<const float*>(smem + L.newraw + 256);
+#pragma unroll
+          for (int j = 0; j < SJ; ++j)
+            if (lane == (r_new & 31) && j == (r_new >> 5)) {
+              skc[j] = nsc[0];
+              svc[j] = nsc[1];
+            }
+        } else {
+          const uint16_t* kl = reinterpret_cast<const uint16_t*>(smem + L.newlat);
+          for (int cch = lane; cch < (rK + rV) / 8; cch += 32) {
+            const bool key = cch < rK / 8;
+            const PieceLoc pt = key ? locate(rK, kTile, cch) : locate(rV, kTile, cch - rK / 8);
+            *reinterpret_cast<uint4*>(ring + (size_t)st * L.stage + (key ? 0u : kt_bytes) +
+                                      swz(pt, r_new)) = *reinterpret_cast<const uint4*>(kl + 8 * cch);
+          }
         }
         fence_proxy_async_smem();  // generic writes into a stage the TMA engine fills
         __syncwarp();
@@ -1791,7 +1865,9 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
 template <int NB, int NKS, int NMV, int TT, int MODE>
 static cudaError_t launch_k(const DecodeArgs& a, cudaStream_t stream) {
   const DecodeSmem L = decode_smem_layout(a.nwarps, a.nstage, a.rK, a.rV, TT,
-                                          MODE == kModeQ8 || MODE == kModePagedQ8 ? 1 : MODE == kModeQ4 ? 2 : 0);
+                                          MODE == kModeQ8 || MODE == kModePagedQ8 || MODE == kModeQ8Append
+                                              ? 1
+                                              : MODE == kModeQ4 ? 2 : 0);
   auto kern = stief_decode_kernel<NB, NKS, NMV, TT, MODE>;
   static SmemLimit limit;
   cudaError_t e = limit.ensure(reinterpret_cast<const void*>(kern), a.device, (int)L.total);
@@ -1836,6 +1912,7 @@ cudaError_t launch_decode_plain(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_latent(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_paged(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_q8(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_decode_q8_append(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_q4(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_paged_q8(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_joint_v(const DecodeArgs& a, cudaStream_t stream);

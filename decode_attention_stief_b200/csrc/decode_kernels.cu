@@ -23,13 +23,14 @@ cudaError_t launch_decode(const DecodeArgs& planned, cudaStream_t stream) {
     return launch_decode_paged_q8(a, stream);  // int8 codes in page pools
   if ((a.latent != 0) + (a.block_table != nullptr) + (a.q8 != 0) + (a.q4 != 0) > 1)
     return cudaErrorInvalidValue;  // the other modes do not combine
+  if (a.q4 != 0 && a.append != 0) return cudaErrorInvalidValue;  // no 4-bit fused step
   if (a.joint_v) {
     if (a.block_table != nullptr || a.q8 != 0 || a.q4 != 0 || a.append != 0) return cudaErrorInvalidValue;
     return a.latent ? launch_decode_latent_joint_v(a, stream) : launch_decode_joint_v(a, stream);
   }
   if (a.latent) return launch_decode_latent(a, stream);
   if (a.block_table) return launch_decode_paged(a, stream);
-  if (a.q8) return launch_decode_q8(a, stream);
+  if (a.q8) return a.append ? launch_decode_q8_append(a, stream) : launch_decode_q8(a, stream);
   if (a.q4) return launch_decode_q4(a, stream);
   return launch_decode_plain(a, stream);
 }

@@ -288,6 +288,9 @@ stief_status decode_common(const uint16_t* q, const uint16_t* k_new, const uint1
   a.k_lat_w = k_lat;
   a.v_lat_w = v_lat;
   a.seq_lens_w = seq_lens;
+  // the int8 fused step writes the new token's row scales (the caller's arrays are writable)
+  a.k_scale_w = const_cast<float*>(k_scale);
+  a.v_scale_w = const_cast<float*>(v_scale);
   // counters at the start (split tickets, then sequence tickets), then the partial states
   // laid out for the split count used
   const size_t units = (size_t)B * Hkv * a.qsub;
@@ -425,6 +428,22 @@ stief_status stief_decode_attention_q8(const uint16_t* q, const uint16_t* P_K,
                        const_cast<int32_t*>(seq_lens), out, workspace, workspace_bytes, B, Hq, Hkv,
                        d, rK, rV, L_max, max_seq_len, num_splits, dev_status, stream, false, false,
                        Paging{}, k_s, v_s);
+}
+
+stief_status stief_append_decode_q8(const uint16_t* q, const uint16_t* k_new,
+                                    const uint16_t* v_new, const uint16_t* P_K,
+                                    const uint16_t* P_V, int8_t* k_q, int8_t* v_q, float* k_s,
+                                    float* v_s, int32_t* seq_lens, uint16_t* out, void* workspace,
+                                    size_t workspace_bytes, int B, int Hq, int Hkv, int d, int rK,
+                                    int rV, int L_max, int max_seq_len, int num_splits,
+                                    uint32_t* dev_status, stief_stream_t stream) {
+  if (!k_s || !v_s) return STIEF_ERR_INVALID_ARG;
+  if (L_max % kQ8RowQuantum != 0) return STIEF_ERR_INVALID_ARG;
+  if (!aligned16(k_s) || !aligned16(v_s)) return STIEF_ERR_ALIGNMENT;
+  return decode_common(q, k_new, v_new, P_K, P_V, reinterpret_cast<uint16_t*>(k_q),
+                       reinterpret_cast<uint16_t*>(v_q), seq_lens, out, workspace,
+                       workspace_bytes, B, Hq, Hkv, d, rK, rV, L_max, max_seq_len, num_splits,
+                       dev_status, stream, true, false, Paging{}, k_s, v_s);
 }
 
 stief_status stief_decode_attention_q8_paged(const uint16_t* q, const uint16_t* P_K,

@@ -78,6 +78,9 @@ struct DecodeArgs {
   int early;
   const float* k_scale;
   const float* v_scale;
+  // int8 fused step: the scale arrays the new token's row scales are written to
+  float* k_scale_w;
+  float* v_scale_w;
 #ifdef STIEF_TEST_HOOKS
   // test build only: bytes added to the setup barrier's expected count that no copy delivers,
   // so that its phase never completes and the waits for it run out (0: off)

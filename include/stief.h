@@ -214,9 +214,10 @@ STIEF_API size_t stief_decode_workspace_bytes(int B, int Hq, int Hkv, int rV, in
  * that takes it; the rule on the cache rows for every decode call, with two
  * differences: the _paged calls also read the block-table entries of their first
  * tiles before the wait (the preceding kernel must not write the entries of pages
- * that hold rows below seq_lens[b]), and the int8, 4-bit and joint-value calls
+ * that hold rows below seq_lens[b]), and the 4-bit, paged int8 and joint-value calls
  * read no row again after the wait (the preceding kernel must write no row below
- * seq_lens[b], the row just below it included).
+ * seq_lens[b], the row just below it included); the contiguous int8 calls re-read
+ * that row like the bf16 ones, so stief_append_decode_q8 calls may follow one another.
  * Returns STIEF_OK or an argument error (nothing launched).
  */
 STIEF_API stief_status stief_decode_attention(const uint16_t* q, const uint16_t* P_K,
@@ -364,7 +365,11 @@ STIEF_API stief_status stief_append_decode_paged(const uint16_t* q, const uint16
  * 2^-15 of its largest element) and each tile's softmax weights per head as 16-bit fixed point
  * of the tile's largest weight, each split into two 8-bit parts, so both products are exact
  * in 32-bit integers; the row scales multiply the scores and the weights.  Paged int8 caches
- * are the _q8_paged calls below; the fused step is not provided for int8 caches.
+ * are the _q8_paged calls below.  stief_append_decode_q8 is the fused step on this form: one
+ * kernel appends the new token (its projected rows rounded to bf16, then quantised exactly as
+ * the compress does: codes into k_q / v_q and scales into k_s / v_s at row seq_lens[b]) and
+ * decodes over the grown cache, with stief_append_decode's launch behaviour and rules; it is
+ * not provided for 4-bit or paged int8 caches.
  */
 STIEF_API stief_status stief_compress_append_q8(const uint16_t* k_new, const uint16_t* v_new,
                                       const uint16_t* P_K, const uint16_t* P_V, int8_t* k_q,
@@ -380,6 +385,14 @@ STIEF_API stief_status stief_decode_attention_q8(const uint16_t* q, const uint16
                                        int rK, int rV, int L_max, int max_seq_len,
                                        int num_splits, uint32_t* dev_status,
                                        stief_stream_t stream);
+
+STIEF_API stief_status stief_append_decode_q8(const uint16_t* q, const uint16_t* k_new,
+                                    const uint16_t* v_new, const uint16_t* P_K,
+                                    const uint16_t* P_V, int8_t* k_q, int8_t* v_q, float* k_s,
+                                    float* v_s, int32_t* seq_lens, uint16_t* out, void* workspace,
+                                    size_t workspace_bytes, int B, int Hq, int Hkv, int d, int rK,
+                                    int rV, int L_max, int max_seq_len, int num_splits,
+                                    uint32_t* dev_status, stief_stream_t stream);
 
 /*
  * int8 caches in page pools: the int8 form above with the paged layout of the _paged calls.

@@ -376,3 +376,111 @@ def test_paged_q8_compress_then_decode(T):
     want = oracle.decode(f64(q), f64(P_K), f64(P_V), kc * kcs[..., None], vc * vcs[..., None],
                          np.asarray(lens, np.int32))
     assert_decode_close(got, want)
+
+
+# ------------------------------------------------------------------------ the int8 fused step
+
+def _append_decode_q8(q, k_new, v_new, P_K, P_V, kq, vq, ks, vs, lens, max_seq_len, num_splits=0,
+                      expect_status=0):
+    """One stief_append_decode_q8 call on device copies; returns (out, kq, vq, ks, vs, lens)."""
+    B, Hq, d = q.shape
+    dkq, dvq, dks, dvs = (x.to(DEV).contiguous() for x in (kq, vq, ks, vs))
+    lens_t = torch.as_tensor(np.asarray(lens, np.int32)).to(DEV)
+    out = torch.full((B, Hq, d), float("nan"), dtype=torch.bfloat16, device=DEV)
+    ws = stief.workspace_for(B, Hq, P_K.shape[0], P_V.shape[2], max_seq_len)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    stief.stief_append_decode_q8(q.to(DEV), k_new.to(DEV), v_new.to(DEV), P_K.to(DEV), P_V.to(DEV),
+                                 dkq, dvq, dks, dvs, lens_t, out, ws, max_seq_len,
+                                 num_splits=num_splits, dev_status=status)
+    assert stief.stief_read_device_status(status) == expect_status
+    return out.cpu(), dkq.cpu(), dvq.cpu(), dks.cpu(), dvs.cpu(), lens_t.cpu().numpy()
+
+
+def _check_new_rows(kq0, vq0, ks0, vs0, gkq, gvq, gks, gvs, k_new, v_new, P_K, P_V, lens):
+    """Row seq_lens[b] of every head holds the quantised projection of the new token (codes
+    within one of the oracle's where the bf16 row may differ by an ulp, scales within a bf16
+    ulp); every other row is unchanged."""
+    B, Hkv = k_new.shape[:2]
+    for b, L in enumerate(lens):
+        for h in range(Hkv):
+            for q0, s0, gq, gs, x, P in ((kq0, ks0, gkq, gks, k_new, P_K), (vq0, vs0, gvq, gvs, v_new, P_V)):
+                lat = oracle.project(f64(x[b, h]).reshape(1, -1), f64(P[h]), round_to_bf16=True)
+                wq, ws = oracle.quantize_rows(lat)
+                got = gq[b, h, L].numpy().astype(np.int32)
+                assert np.max(np.abs(got - wq[0].astype(np.int32))) <= 1
+                np.testing.assert_allclose(gs[b, h, L].numpy(), ws[0], rtol=2 ** -7)
+                keep = np.ones(q0.shape[2], bool)
+                keep[L] = False
+                assert torch.equal(gq[b, h][keep], q0[b, h][keep])
+                assert torch.equal(gs[b, h][keep], s0[b, h][keep])
+
+
+@pytest.mark.parametrize("rK,rV", [(64, 64), (32, 48), (96, 128)])
+@pytest.mark.parametrize("num_splits", [0, 1, 3])
+def test_append_decode_q8_matches_oracle(rK, rV, num_splits):
+    """The int8 fused step: the new token's rows quantised into the cache at seq_lens[b]
+    (as the compress stores them), the lengths incremented, and the output the oracle's decode
+    over the grown cache (the stored codes and scales, dequantised)."""
+    B, Hq, Hkv, L_max = 3, 16, 4, 768
+    lens = [700, 33, 0]
+    q, P_K, P_V, kq, vq, ks, vs = _q8_case(6900 + rK + num_splits, B, Hq, Hkv, L_max, rK, rV)
+    k_new, v_new = si.full_kv(6950 + rV, B, Hkv, 1, 128)
+    got, gkq, gvq, gks, gvs, glens = _append_decode_q8(q, k_new, v_new, P_K, P_V, kq, vq, ks, vs,
+                                                       lens, 701, num_splits)
+    assert glens.tolist() == [L + 1 for L in lens]
+    _check_new_rows(kq, vq, ks, vs, gkq, gvq, gks, gvs, k_new[:, :, 0], v_new[:, :, 0], P_K, P_V, lens)
+    want = _oracle_q8(q, P_K, P_V, gkq, gvq, gks, gvs, glens)
+    assert_decode_close(got, want)
+
+
+def test_append_decode_q8_steps_follow_one_another():
+    """Fused int8 steps back to back on one stream: each reads the row the previous one
+    appended (the row just below its length, requested before its dependency wait and read
+    again after it), and the final cache and output match the oracle."""
+    B, Hq, Hkv, rK, rV, L_max = 2, 32, 8, 64, 64, 4096
+    lens0 = [4000, 1500]
+    q, P_K, P_V, kq, vq, ks, vs = _q8_case(7000, B, Hq, Hkv, L_max, rK, rV)
+    dkq, dvq, dks, dvs = (x.to(DEV).contiguous() for x in (kq, vq, ks, vs))
+    lens_t = torch.as_tensor(np.asarray(lens0, np.int32)).to(DEV)
+    ws = stief.workspace_for(B, Hq, Hkv, rV, L_max)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    gP_K, gP_V = P_K.to(DEV), P_V.to(DEV)
+    steps = 5
+    news = [si.full_kv(7001 + i, B, Hkv, 1, 128) for i in range(steps)]
+    qs = [si.queries(7100 + i, B, Hq, 128).to(DEV) for i in range(steps)]
+    outs = [torch.empty((B, Hq, 128), dtype=torch.bfloat16, device=DEV) for _ in range(steps)]
+    for i in range(steps):
+        stief.stief_append_decode_q8(qs[i], news[i][0].to(DEV), news[i][1].to(DEV), gP_K, gP_V,
+                                     dkq, dvq, dks, dvs, lens_t, outs[i], ws, L_max,
+                                     dev_status=status)
+    assert stief.stief_read_device_status(status) == 0
+    assert lens_t.cpu().tolist() == [L + steps for L in lens0]
+    gkq, gvq, gks, gvs = dkq.cpu(), dvq.cpu(), dks.cpu(), dvs.cpu()
+    for i in range(steps):
+        step_lens = [L + i for L in lens0]
+        # each step's rows, then the output over the cache as it stood after that step
+        for b, L in enumerate(step_lens):
+            for h in range(Hkv):
+                for gq, gs, x, P in ((gkq, gks, news[i][0], P_K), (gvq, gvs, news[i][1], P_V)):
+                    lat = oracle.project(f64(x[b, h, 0]).reshape(1, -1), f64(P[h]))
+                    wq, wsc = oracle.quantize_rows(lat)
+                    assert np.max(np.abs(gq[b, h, L].numpy().astype(np.int32) - wq[0])) <= 1
+                    np.testing.assert_allclose(gs[b, h, L].numpy(), wsc[0], rtol=2 ** -7)
+        want = _oracle_q8(qs[i].cpu(), P_K, P_V, gkq, gvq, gks, gvs, np.asarray(step_lens) + 1)
+        assert_decode_close(outs[i].cpu(), want)
+
+
+def test_append_decode_q8_full_cache_is_refused():
+    """A sequence whose cache is full is not appended to (capacity bit; its rows and length
+    unchanged) and its output attends over the cache as it was; the other sequences step."""
+    B, Hq, Hkv, rK, rV, L_max = 2, 16, 4, 64, 48, 256
+    lens = [256, 100]
+    q, P_K, P_V, kq, vq, ks, vs = _q8_case(7200, B, Hq, Hkv, L_max, rK, rV)
+    k_new, v_new = si.full_kv(7201, B, Hkv, 1, 128)
+    got, gkq, gvq, gks, gvs, glens = _append_decode_q8(
+        q, k_new, v_new, P_K, P_V, kq, vq, ks, vs, lens, 256,
+        expect_status=stief.DEV_CAPACITY_OVERFLOW)
+    assert glens.tolist() == [256, 101]
+    assert torch.equal(gkq[0], kq[0]) and torch.equal(gks[0], ks[0])
+    want = _oracle_q8(q, P_K, P_V, gkq, gvq, gks, gvs, glens)
+    assert_decode_close(got, want)
