@@ -214,6 +214,28 @@ def test_q8_decode_argument_errors(lib, kw, code):
     assert _q8(lib, **kw) == code
 
 
+def _q8_step(lib, **kw):
+    a = dict(q=FAKE, kn=FAKE, vn=FAKE, P_K=FAKE, P_V=FAKE, kq=FAKE, vq=FAKE, ks=FAKE, vs=FAKE,
+             sl=FAKE, out=FAKE, ws=FAKE, ws_bytes=1 << 40, B=1, Hq=32, Hkv=8, d=128, rK=64, rV=64,
+             L_max=1024, max_seq_len=1024, num_splits=0)
+    a.update(kw)
+    return lib.stief_append_decode_q8(a["q"], a["kn"], a["vn"], a["P_K"], a["P_V"], a["kq"], a["vq"],
+                                      a["ks"], a["vs"], a["sl"], a["out"], a["ws"], a["ws_bytes"],
+                                      a["B"], a["Hq"], a["Hkv"], a["d"], a["rK"], a["rV"], a["L_max"],
+                                      a["max_seq_len"], a["num_splits"], None, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(kn=None), INVALID), (dict(vn=None), INVALID), (dict(ks=None), INVALID),
+    (dict(L_max=1000, max_seq_len=1000), INVALID), (dict(vn=FAKE + 2), ALIGN),
+    (dict(vs=FAKE + 4), ALIGN), (dict(max_seq_len=2048), CAPACITY), (dict(ws=None), WORKSPACE),
+])
+def test_q8_fused_step_argument_errors(lib, kw, code):
+    """The int8 fused step checks its new rows, scales and cache geometry before any CUDA
+    call."""
+    assert _q8_step(lib, **kw) == code
+
+
 @pytest.mark.parametrize("kw,code", [
     (dict(k=None), INVALID), (dict(sl=None), INVALID), (dict(d=96), INVALID),
     (dict(rK=24), INVALID), (dict(T=-1), INVALID), (dict(B=0), INVALID),
