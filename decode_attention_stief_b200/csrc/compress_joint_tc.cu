@@ -28,7 +28,9 @@
 // stage's "empty" barrier, and refills the previous chunk's stage once its MMAs are done, so
 // the next copies are in flight while the MMAs run.  After a tile's last chunk a commit on the
 // accumulator barrier releases the epilogue: warp w reads TMEM lanes 32 (w & 3) .. + 31
-// (rows) and every other group of 16 columns (w >> 2 picks which), rounds and stores.
+// (rows) and every other group of 16 columns (w >> 2 picks which), rounds and stores.  Key
+// CTAs (one chunk per tile, several tiles) keep two accumulator sets instead: tile i + 1's
+// MMAs are issued before tile i's epilogue when its copy is already in.
 //
 // Launched as a programmatic dependent: barrier set-up, the TMEM allocation and the basis
 // staging (weights, which the preceding kernel must not write) overlap the preceding kernel's
