@@ -498,8 +498,9 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
   // slower: the flood delays q and some CTAs' data by microseconds).  The calls document that
   // the kernel immediately preceding them must not write the cache rows below the lengths
   // (nor, for page pools, the block-table entries of their pages), except, for bf16
-  // per-head caches and contiguous int8 caches, the row just below each length (the one a
-  // preceding fused step on the same caches appends), which is read again after the wait.  Paged caches look the early
+  // per-head caches, the row just below each length (the one a preceding fused step on the
+  // same caches appends), which is read again after the wait.  After an int8 fused step the
+  // host clears `early` for the next decode in the stream, as after a compress.  Paged caches look the early
   // tiles' pages up around the L1 cache, so that no line read before the wait can hide an
   // entry the preceding kernel writes.  Right after a compress of this library (whose new
   // rows may still be in flight) the host clears `early` and nothing is requested before the
@@ -974,34 +975,18 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1)
       const uint32_t sbase = smem_u32(ring + (size_t)st * L.stage);
       const int tok0 = t0 + (warp + k * NW) * kTile;
       const int n = min(kTile, t1 - tok0);
-      // the modes with a fused step: bf16 per-head caches, and contiguous int8 caches
-      constexpr bool RELOAD_Q8 = MODE == kModeQ8 || MODE == kModeQ8Append;
-      if ((RELOAD_Q8 || (!QI && !JV)) && early_tiles && k < kPreIssue && Lb >= 1 && tok0 <= Lb - 1 &&
-          Lb - 1 < tok0 + kTile) {
+      if (!QI && !JV && early_tiles && k < kPreIssue && Lb >= 1 && tok0 <= Lb - 1 && Lb - 1 < tok0 + kTile) {
         // this tile was requested before the dependency wait: the row just below the length
         // may have been appended by the preceding kernel (a fused step on the same caches),
-        // so it is read again now (L2; the wait made it visible).  int8 caches: its codes (its
-        // scales are loaded after the wait anyway)
+        // so it is read again now (L2; the wait made it visible)
         const int r_prev = Lb - 1 - tok0;
         const long long prow = cache_row(cr, b, kvh, Lb - 1);
-        if constexpr (RELOAD_Q8) {
-          const int8_t* kq = reinterpret_cast<const int8_t*>(a.k_lat_w) + prow * rK;
-          const int8_t* vq = reinterpret_cast<const int8_t*>(a.v_lat_w) + prow * rV;
-          for (int cch = lane; cch < (rK + rV) / 16; cch += 32) {
-            const bool key = cch < rK / 16;
-            const uint4 v = key ? __ldcg(reinterpret_cast<const uint4*>(kq) + cch)
-                                : __ldcg(reinterpret_cast<const uint4*>(vq) + (cch - rK / 16));
-            const PieceLoc pt = key ? locate_i8(rKc, kTile, cch) : locate_i8(rVc, kTile, cch - rK / 16);
-            *reinterpret_cast<uint4*>(ring + (size_t)st * L.stage + (key ? 0u : kt_bytes) + swz(pt, r_prev)) = v;
-          }
-        } else {
-          for (int cch = lane; cch < (rK + rV) / 8; cch += 32) {
-            const bool key = cch < rK / 8;
-            const uint4 v = key ? __ldcg(reinterpret_cast<const uint4*>(a.k_lat_w + prow * rK) + cch)
-                                : __ldcg(reinterpret_cast<const uint4*>(a.v_lat_w + prow * rV) + (cch - rK / 8));
-            const PieceLoc pt = key ? locate(rK, kTile, cch) : locate(rV, kTile, cch - rK / 8);
-            *reinterpret_cast<uint4*>(ring + (size_t)st * L.stage + (key ? 0u : kt_bytes) + swz(pt, r_prev)) = v;
-          }
+        for (int cch = lane; cch < (rK + rV) / 8; cch += 32) {
+          const bool key = cch < rK / 8;
+          const uint4 v = key ? __ldcg(reinterpret_cast<const uint4*>(a.k_lat_w + prow * rK) + cch)
+                              : __ldcg(reinterpret_cast<const uint4*>(a.v_lat_w + prow * rV) + (cch - rK / 8));
+          const PieceLoc pt = key ? locate(rK, kTile, cch) : locate(rV, kTile, cch - rK / 8);
+          *reinterpret_cast<uint4*>(ring + (size_t)st * L.stage + (key ? 0u : kt_bytes) + swz(pt, r_prev)) = v;
         }
         fence_proxy_async_smem();  // generic writes into a stage the TMA engine fills
         __syncwarp();

@@ -30,7 +30,14 @@ cudaError_t launch_decode(const DecodeArgs& planned, cudaStream_t stream) {
   }
   if (a.latent) return launch_decode_latent(a, stream);
   if (a.block_table) return launch_decode_paged(a, stream);
-  if (a.q8) return a.append ? launch_decode_q8_append(a, stream) : launch_decode_q8(a, stream);
+  if (a.q8 && a.append) {
+    // the int8 fused step writes a cache row that the next decode in the stream would read
+    // before its dependency wait (int8 tiles get no second read of that row): note it
+    const cudaError_t e = launch_decode_q8_append(a, stream);
+    if (e == cudaSuccess) mark_stream_compress(a.device, stream, true);
+    return e;
+  }
+  if (a.q8) return launch_decode_q8(a, stream);
   if (a.q4) return launch_decode_q4(a, stream);
   return launch_decode_plain(a, stream);
 }

@@ -190,10 +190,12 @@ inline size_t decode_tagged_stage_bytes(int G_T, int splits, int rV) {
 }
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
 
-// Per (device, stream): whether the library's last launch there was a compress whose length
-// kernel lets its dependent start early.  A compress marks its stream; a decode reads and
+// Per (device, stream): whether the library's last launch there wrote cache rows that the next
+// decode could request before its dependency wait: a compress (whose length kernel lets its
+// dependent start early) or an int8 fused step.  Those mark their stream; a decode reads and
 // clears the mark (it then requests no cache tile before its dependency wait); the joint
-// compress, whose kernels do not let dependents start early, clears it.  Host only.
+// compress's CUDA-core path, whose kernels do not let dependents start early, clears it.
+// Host only.
 void mark_stream_compress(int device, cudaStream_t s, bool marked);
 bool take_stream_compress_mark(int device, cudaStream_t s);
 

@@ -214,10 +214,12 @@ STIEF_API size_t stief_decode_workspace_bytes(int B, int Hq, int Hkv, int rV, in
  * that takes it; the rule on the cache rows for every decode call, with two
  * differences: the _paged calls also read the block-table entries of their first
  * tiles before the wait (the preceding kernel must not write the entries of pages
- * that hold rows below seq_lens[b]), and the 4-bit, paged int8 and joint-value calls
- * read no row again after the wait (the preceding kernel must write no row below
- * seq_lens[b], the row just below it included); the contiguous int8 calls re-read
- * that row like the bf16 ones, so stief_append_decode_q8 calls may follow one another.
+ * that hold rows below seq_lens[b]), and the int8, 4-bit and joint-value calls read
+ * no row again after the wait (the preceding kernel must write no row below
+ * seq_lens[b], the row just below it included); a decode issued right after one of
+ * this library's int8 fused steps in the same stream requests no cache row before its
+ * wait (the library notes it per stream, as after a compress), so
+ * stief_append_decode_q8 calls may follow one another.
  * Returns STIEF_OK or an argument error (nothing launched).
  */
 STIEF_API stief_status stief_decode_attention(const uint16_t* q, const uint16_t* P_K,

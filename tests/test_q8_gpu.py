@@ -468,6 +468,19 @@ def test_append_decode_q8_steps_follow_one_another():
                     np.testing.assert_allclose(gs[b, h, L].numpy(), wsc[0], rtol=2 ** -7)
         want = _oracle_q8(qs[i].cpu(), P_K, P_V, gkq, gvq, gks, gvs, np.asarray(step_lens) + 1)
         assert_decode_close(outs[i].cpu(), want)
+    # a plain int8 decode right after the last step on the same stream and caches
+    for i in range(steps):
+        stief.stief_append_decode_q8(qs[i], news[i][0].to(DEV), news[i][1].to(DEV), gP_K, gP_V,
+                                     dkq, dvq, dks, dvs, lens_t, outs[i], ws, L_max,
+                                     dev_status=status)
+    out = torch.empty((B, Hq, 128), dtype=torch.bfloat16, device=DEV)
+    stief.stief_decode_attention_q8(qs[0], gP_K, gP_V, dkq, dvq, dks, dvs, lens_t, out, ws, L_max,
+                                    dev_status=status)
+    assert stief.stief_read_device_status(status) == 0
+    assert lens_t.cpu().tolist() == [L + 2 * steps for L in lens0]
+    want = _oracle_q8(qs[0].cpu(), P_K, P_V, dkq.cpu(), dvq.cpu(), dks.cpu(), dvs.cpu(),
+                      lens_t.cpu().numpy())
+    assert_decode_close(out.cpu(), want)
 
 
 def test_append_decode_q8_full_cache_is_refused():
