@@ -433,6 +433,21 @@ def test_append_decode_q8_matches_oracle(rK, rV, num_splits):
     assert_decode_close(got, want)
 
 
+@pytest.mark.parametrize("Hq,Hkv", [(64, 8), (24, 4)])
+def test_append_decode_q8_group_sizes(Hq, Hkv):
+    """The int8 fused step with groups of 8 query heads per KV head (two MMA n-tiles) and of
+    6 (two sub-groups of a KV head, only the first writes the cache row)."""
+    B, L_max, rK, rV = 2, 512, 64, 48
+    lens = [500, 77]
+    q, P_K, P_V, kq, vq, ks, vs = _q8_case(7300 + Hq, B, Hq, Hkv, L_max, rK, rV)
+    k_new, v_new = si.full_kv(7301 + Hq, B, Hkv, 1, 128)
+    got, gkq, gvq, gks, gvs, glens = _append_decode_q8(q, k_new, v_new, P_K, P_V, kq, vq, ks, vs,
+                                                       lens, 501)
+    assert glens.tolist() == [L + 1 for L in lens]
+    _check_new_rows(kq, vq, ks, vs, gkq, gvq, gks, gvs, k_new[:, :, 0], v_new[:, :, 0], P_K, P_V, lens)
+    assert_decode_close(got, _oracle_q8(q, P_K, P_V, gkq, gvq, gks, gvs, glens))
+
+
 def test_append_decode_q8_steps_follow_one_another():
     """Fused int8 steps back to back on one stream: each reads the row the previous one
     appended (the row just below its length, requested before its dependency wait and read
