@@ -250,7 +250,7 @@ __global__ void __launch_bounds__(kJtThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t idesc = idesc_bf16_f32(r);
-  // the exchange area of the pair's rank-0 CTA (partial sums, then rank 1's verdict)
+  // the exchange area of the pair's rank-0 CTA (partial sums, then rank 1's status word)
   const uint32_t exch = smem_u32(smem + L.exch);
   const uint32_t flag_off = (uint32_t)kUmmaRows * (uint32_t)a.rV * 4u;
   bool ok = !(bad || over);
@@ -362,7 +362,7 @@ __global__ void __launch_bounds__(kJtThreads, 1)
     const int m0 = tile_m0(i);
     const int row = (warp & 3) * 32 + lane;
     const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-    if (paired && rank == 1) {  // partial sums into rank 0's exchange area, then the verdict
+    if (paired && rank == 1) {  // partial sums into rank 0's exchange area, then the status word
       const uint32_t rx = cluster_addr(exch, 0u);
       if (ok) {
         for (int c0 = 16 * (warp >> 2); c0 < r; c0 += 32) {
